@@ -1,0 +1,106 @@
+"""Seeded synthetic inputs for exact attention, shared by the oracle tests,
+the GPU parity tests and the benchmark.
+
+This module holds workload shapes and random-number generation only: no
+attention arithmetic lives here.  Every tensor is drawn on the CPU from a
+``torch.Generator`` seeded with ``manual_seed(seed)``, in the order Q, K, V,
+dO, as float32 ``randn`` times ``sigma``, then rounded to the storage dtype
+(bf16 or fp16).  The oracle widens exactly these rounded values to float64,
+and the GPU receives a bit-identical copy, so both sides see the same inputs.
+
+Layouts follow the ``(batch, seqlen, nheads, headdim)`` convention of the
+integration example on "FlashAttention-2：下一代高效注意力机制的突破与实战解析"
+(section "实操落地"); K and V carry ``nheads_kv`` heads (grouped-query
+attention, named on "FlashAttention 四代演进", section "硬件边界与数据类型限制").
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Dict, Optional
+
+import torch
+
+DTYPES = {"bf16": torch.bfloat16, "fp16": torch.float16}
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    """One attention problem: shapes, mask and input distribution."""
+
+    name: str
+    batch: int
+    nheads: int
+    nheads_kv: int
+    seqlen_q: int
+    seqlen_k: int
+    headdim: int
+    causal: bool
+    window_left: int = -1
+    window_right: int = -1
+    dtype: str = "bf16"
+    sigma: float = 1.0
+    seed: int = 0
+    passes: str = "fwd+bwd"
+    softmax_scale: Optional[float] = None
+
+    @property
+    def scale(self) -> float:
+        return self.softmax_scale if self.softmax_scale is not None else 1.0 / math.sqrt(self.headdim)
+
+    def replace(self, **kw) -> "Workload":
+        return dataclasses.replace(self, **kw)
+
+
+# The five workloads attention is measured and checked on.  The seed of each
+# is its index in this list.
+WORKLOADS: Dict[str, Workload] = {
+    "tiny_b1_h2_n128_d64": Workload(
+        "tiny_b1_h2_n128_d64", 1, 2, 2, 128, 128, 64, False, seed=0, passes="fwd+bwd"),
+    "causal_b2_h32_n8192_d128": Workload(
+        "causal_b2_h32_n8192_d128", 2, 32, 32, 8192, 8192, 128, True, seed=1, passes="fwd+bwd"),
+    "full_b1_h16_n16384_d128": Workload(
+        "full_b1_h16_n16384_d128", 1, 16, 16, 16384, 16384, 128, False, seed=2, passes="fwd+bwd"),
+    "gqa_window_b4_h32_kv8_n4096_d128": Workload(
+        "gqa_window_b4_h32_kv8_n4096_d128", 4, 32, 8, 4096, 4096, 128, True,
+        window_left=1024, window_right=0, seed=3, passes="fwd+bwd"),
+    "long_fp16_b1_h8_n65536_d256": Workload(
+        "long_fp16_b1_h8_n65536_d256", 1, 8, 8, 65536, 65536, 256, True,
+        dtype="fp16", sigma=0.5, seed=4, passes="fwd"),
+}
+
+
+def make_inputs(w: Workload, with_dout: bool = True, device: str = "cpu"):
+    """Draw (q, k, v, dout) for workload ``w``.
+
+    Shapes: q, dout (B, Nq, H, d); k, v (B, Nk, Hkv, d).  Returns CPU tensors
+    of the storage dtype unless ``device`` says otherwise (the copy is exact).
+    """
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(w.seed))
+    dt = DTYPES[w.dtype]
+
+    def draw(*shape):
+        x = torch.randn(*shape, generator=g, dtype=torch.float32)
+        return (x * w.sigma).to(dt)
+
+    q = draw(w.batch, w.seqlen_q, w.nheads, w.headdim)
+    k = draw(w.batch, w.seqlen_k, w.nheads_kv, w.headdim)
+    v = draw(w.batch, w.seqlen_k, w.nheads_kv, w.headdim)
+    dout = draw(w.batch, w.seqlen_q, w.nheads, w.headdim) if with_dout else None
+    if device != "cpu":
+        q, k, v = q.to(device), k.to(device), v.to(device)
+        dout = dout.to(device) if dout is not None else None
+    return q, k, v, dout
+
+
+def sample_rows(n: int, count: int, seed: int, must=()) -> torch.Tensor:
+    """A sorted, duplicate-free set of row indices in [0, n): the first and
+    last rows, any ``must`` rows, and ``count`` more drawn from ``seed``."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed) + 7919)
+    picks = set(int(i) for i in must if 0 <= int(i) < n)
+    picks.update({0, n - 1} if n > 0 else set())
+    if n > 0 and count > 0:
+        picks.update(torch.randint(0, n, (count,), generator=g).tolist())
+    return torch.tensor(sorted(picks), dtype=torch.int64)

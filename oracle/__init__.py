@@ -1,0 +1,191 @@
+"""Python access to the float64 CPU attention oracle (``attn_oracle.c``).
+
+TEST INFRASTRUCTURE.  Only the tests, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline / reference leg may import this package.  The CUDA
+library and its Python binding never import it, and it never imports them.
+
+Every function takes torch tensors in the storage dtype (bf16/fp16/fp32/fp64,
+any device), widens them exactly to float64 on the CPU and returns float64
+numpy arrays.  See ``attn_oracle.c`` for what is computed and which passages
+of the pages each step follows.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "attn_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+class OracleParams(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int64),
+        ("seqlen_q", ctypes.c_int64),
+        ("seqlen_k", ctypes.c_int64),
+        ("nheads", ctypes.c_int64),
+        ("nheads_kv", ctypes.c_int64),
+        ("headdim", ctypes.c_int64),
+        ("softmax_scale", ctypes.c_double),
+        ("causal", ctypes.c_int64),
+        ("window_left", ctypes.c_int64),
+        ("window_right", ctypes.c_int64),
+    ]
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (float64, no fast-math, OpenMP)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off",
+               "-fno-fast-math", "-Wall", "-o", tmp, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+class Oracle:
+    """Bindings to one compiled copy of the oracle (the default build, or a
+    variant compiled elsewhere, as the mutation tests do)."""
+
+    def __init__(self, lib_path: str):
+        lib = ctypes.CDLL(lib_path)
+        d = ctypes.POINTER(ctypes.c_double)
+        i64 = ctypes.POINTER(ctypes.c_int64)
+        P = ctypes.POINTER(OracleParams)
+        lib.oracle_attn_fwd.argtypes = [P, d, d, d, d, d]
+        lib.oracle_attn_fwd_rows.argtypes = [P, d, d, d, i64, ctypes.c_int64, d, d]
+        lib.oracle_attn_bwd.argtypes = [P, d, d, d, d, d, d, d]
+        lib.oracle_attn_bwd_rows.argtypes = [P, d, d, d, d, i64, ctypes.c_int64, d,
+                                             i64, ctypes.c_int64, d, d]
+        for f in (lib.oracle_attn_fwd, lib.oracle_attn_fwd_rows, lib.oracle_attn_bwd,
+                  lib.oracle_attn_bwd_rows):
+            f.restype = ctypes.c_int
+        lib.oracle_num_threads.restype = ctypes.c_int
+        lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
+        self.lib = lib
+        self.path = lib_path
+
+    def attention_fwd(self, q, k, v, softmax_scale=None, causal=False, window_left=-1,
+                      window_right=-1):
+        """O (B, Nq, H, d) and LSE (B, H, Nq), float64."""
+        return self.attention_fwd_rows(q, k, v, None, softmax_scale, causal, window_left,
+                                       window_right)
+
+    def attention_fwd_rows(self, q, k, v, rows, softmax_scale=None, causal=False,
+                           window_left=-1, window_right=-1):
+        """O and LSE for the query positions ``rows`` only (all rows if None):
+        O (B, len(rows), H, d), LSE (B, H, len(rows))."""
+        qa, ka, va = _f64(q), _f64(k), _f64(v)
+        p = _params(qa, ka, softmax_scale, causal, window_left, window_right)
+        B, Nq, H, d = qa.shape
+        if rows is None:
+            n, rp = Nq, None
+        else:
+            ra = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+            n, rp = ra.shape[0], _ptr(ra, ctypes.c_int64)
+        o = np.zeros((B, n, H, d), dtype=np.float64)
+        lse = np.zeros((B, H, n), dtype=np.float64)
+        rc = self.lib.oracle_attn_fwd_rows(ctypes.byref(p), _ptr(qa), _ptr(ka), _ptr(va), rp,
+                                           ctypes.c_int64(n), _ptr(o), _ptr(lse))
+        if rc != 0:
+            raise ValueError("oracle_attn_fwd_rows rejected its arguments")
+        return o, lse
+
+    def attention_bwd(self, q, k, v, dout, softmax_scale=None, causal=False, window_left=-1,
+                      window_right=-1):
+        """dQ (B, Nq, H, d), dK and dV (B, Nk, Hkv, d), float64."""
+        qa, ka, va, da = _f64(q), _f64(k), _f64(v), _f64(dout)
+        p = _params(qa, ka, softmax_scale, causal, window_left, window_right)
+        dq = np.zeros_like(qa)
+        dk = np.zeros_like(ka)
+        dv = np.zeros_like(va)
+        rc = self.lib.oracle_attn_bwd(ctypes.byref(p), _ptr(qa), _ptr(ka), _ptr(va), _ptr(da),
+                                      _ptr(dq), _ptr(dk), _ptr(dv))
+        if rc != 0:
+            raise ValueError("oracle_attn_bwd rejected its arguments")
+        return dq, dk, dv
+
+    def attention_bwd_rows(self, q, k, v, dout, qrows, krows, softmax_scale=None, causal=False,
+                           window_left=-1, window_right=-1):
+        """dQ at query positions ``qrows`` (B, nq, H, d) and dK, dV at key
+        positions ``krows`` (B, nk, Hkv, d), float64."""
+        qa, ka, va, da = _f64(q), _f64(k), _f64(v), _f64(dout)
+        p = _params(qa, ka, softmax_scale, causal, window_left, window_right)
+        qr = np.ascontiguousarray(np.asarray(qrows, dtype=np.int64))
+        kr = np.ascontiguousarray(np.asarray(krows, dtype=np.int64))
+        B, _, H, d = qa.shape
+        Hkv = ka.shape[2]
+        dq = np.zeros((B, qr.shape[0], H, d))
+        dk = np.zeros((B, kr.shape[0], Hkv, d))
+        dv = np.zeros((B, kr.shape[0], Hkv, d))
+        rc = self.lib.oracle_attn_bwd_rows(ctypes.byref(p), _ptr(qa), _ptr(ka), _ptr(va),
+                                           _ptr(da), _ptr(qr, ctypes.c_int64),
+                                           ctypes.c_int64(qr.shape[0]), _ptr(dq),
+                                           _ptr(kr, ctypes.c_int64), ctypes.c_int64(kr.shape[0]),
+                                           _ptr(dk), _ptr(dv))
+        if rc != 0:
+            raise ValueError("oracle_attn_bwd_rows rejected its arguments")
+        return dq, dk, dv
+
+
+def default() -> Oracle:
+    """The oracle built from ``attn_oracle.c`` beside this file."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            _lib = Oracle(build())
+    return _lib
+
+
+def num_threads() -> int:
+    return int(default().lib.oracle_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    default().lib.oracle_set_num_threads(int(n))
+
+
+def _f64(t) -> np.ndarray:
+    import torch
+    if isinstance(t, np.ndarray):
+        return np.ascontiguousarray(t, dtype=np.float64)
+    return np.ascontiguousarray(t.detach().to("cpu", torch.float64).numpy())
+
+
+def _ptr(a: np.ndarray, ty=ctypes.c_double):
+    return a.ctypes.data_as(ctypes.POINTER(ty))
+
+
+def _params(q, k, softmax_scale, causal, window_left, window_right) -> OracleParams:
+    B, Nq, H, d = q.shape
+    Bk, Nk, Hkv, dk = k.shape
+    if Bk != B or dk != d or H % Hkv != 0:
+        raise ValueError("inconsistent shapes")
+    scale = 1.0 / math.sqrt(d) if softmax_scale is None else float(softmax_scale)
+    return OracleParams(B, Nq, Nk, H, Hkv, d, scale, int(bool(causal)),
+                        int(window_left), int(window_right))
+
+
+def attention_fwd(*a, **kw):
+    return default().attention_fwd(*a, **kw)
+
+
+def attention_fwd_rows(*a, **kw):
+    return default().attention_fwd_rows(*a, **kw)
+
+
+def attention_bwd(*a, **kw):
+    return default().attention_bwd(*a, **kw)
+
+
+def attention_bwd_rows(*a, **kw):
+    return default().attention_bwd_rows(*a, **kw)

@@ -1,0 +1,366 @@
+/*
+ * Exact attention oracle: plain, slow, float64, CPU.
+ *
+ * TEST INFRASTRUCTURE.  Only the tests, the smoke check and the benchmark's
+ * CPU-baseline leg may load or call this file.  It shares no code, header,
+ * table or helper with the CUDA library, and the CUDA library never calls it.
+ *
+ * What it computes is the definition of attention, written out:
+ *
+ *   O = softmax(Q K^T * scale + mask) V
+ *
+ *   - "FlashAttention ... Transformer optimization" (page 2, first paragraph of
+ *     the technical deep dive) gives Softmax(QK^T / sqrt(d)) V; scale defaults
+ *     to 1/sqrt(d) and is otherwise the caller's softmax_scale (the
+ *     integration example on the FlashAttention-2 page passes it explicitly).
+ *   - The tiled method reaches this same result (page 4, definition: "exact
+ *     attention"; page 5: the result is unchanged by tiling), so the oracle is
+ *     the untiled definition: explicit scores, a two-pass softmax (row max,
+ *     then row sum), explicit masks.
+ *   - Masks (FlashAttention-2 page, section 3 "more flexible masks" and the
+ *     sparse-attention extension): causal and sliding-window.  Reading taken:
+ *     key j is visible from query i iff
+ *         j <= i + off                       (causal)
+ *         j >= i + off - window_left         (window_left  >= 0)
+ *         j <= i + off + window_right        (window_right >= 0)
+ *     with off = seqlen_k - seqlen_q (bottom-right alignment), bounds
+ *     inclusive, -1 meaning unbounded.
+ *   - Grouped-query attention (page 5, hardware/dtype section, MQA/GQA):
+ *     query head h reads kv head h / (nheads / nheads_kv).
+ *   - LSE_i = m_i + ln(l_i), natural log, of the scaled scores.  A row with
+ *     no visible key gets O = 0 and LSE = -inf.
+ *   - Backward (page 2, item 2: the backward pass recomputes the score
+ *     matrix; the arithmetic is the analytic gradient of the definition):
+ *         dV = P^T dO,  dP = dO V^T,
+ *         dS = P o (dP - rowsum(P o dP)),
+ *         dQ = scale * dS K,  dK = scale * dS^T Q,
+ *     with dK and dV summed over the query heads that share a kv head.
+ *
+ * Layouts: q, o, dout, dq (B, Nq, H, d); k, v, dk, dv (B, Nk, Hkv, d);
+ * lse (B, H, Nq).  All float64, contiguous.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+typedef struct {
+  int64_t batch, seqlen_q, seqlen_k, nheads, nheads_kv, headdim;
+  double softmax_scale;
+  int64_t causal, window_left, window_right;
+} oracle_params;
+
+/* Visibility of key j from query i (the mask reading stated above). */
+static int visible(const oracle_params *p, int64_t i, int64_t j) {
+  int64_t ii = i + (p->seqlen_k - p->seqlen_q);
+  if (p->causal && j > ii) return 0;
+  if (p->window_left >= 0 && j < ii - p->window_left) return 0;
+  if (p->window_right >= 0 && j > ii + p->window_right) return 0;
+  return 1;
+}
+
+static const double *qrow(const oracle_params *p, const double *q, int64_t b, int64_t i, int64_t h) {
+  return q + ((b * p->seqlen_q + i) * p->nheads + h) * p->headdim;
+}
+static const double *krow(const oracle_params *p, const double *k, int64_t b, int64_t j, int64_t g) {
+  return k + ((b * p->seqlen_k + j) * p->nheads_kv + g) * p->headdim;
+}
+static int64_t kv_head(const oracle_params *p, int64_t h) {
+  return h / (p->nheads / p->nheads_kv);
+}
+
+static double dot(const double *a, const double *b, int64_t n) {
+  double acc = 0.0;
+  for (int64_t c = 0; c < n; ++c) acc += a[c] * b[c];
+  return acc;
+}
+
+/*
+ * Scores of one query row and its softmax statistics (two passes).
+ * s[j] = scale * q_i . k_j for visible j, -inf otherwise.
+ * *m = max_j s[j]; *l = sum_j exp(s[j] - *m).  No visible key: *l = 0.
+ */
+static void row_scores(const oracle_params *p, const double *q, const double *k,
+                       int64_t b, int64_t h, int64_t i, double *s, double *m, double *l) {
+  const int64_t g = kv_head(p, h);
+  const double *qi = qrow(p, q, b, i, h);
+  double mx = -INFINITY;
+  int64_t count = 0;
+  for (int64_t j = 0; j < p->seqlen_k; ++j) {
+    if (!visible(p, i, j)) { s[j] = -INFINITY; continue; }
+    s[j] = p->softmax_scale * dot(qi, krow(p, k, b, j, g), p->headdim);
+    if (s[j] > mx) mx = s[j];
+    ++count;
+  }
+  double sum = 0.0;
+  if (count > 0)
+    for (int64_t j = 0; j < p->seqlen_k; ++j)
+      if (s[j] != -INFINITY) sum += exp(s[j] - mx);
+  *m = mx;
+  *l = sum;
+}
+
+/* Probability P_ij from the row's score and statistics. */
+static double prob(double s, double m, double l) {
+  return (s == -INFINITY || l == 0.0) ? 0.0 : exp(s - m) / l;
+}
+
+/* One forward row: o_out[0..d) and *lse_out. */
+static void fwd_row(const oracle_params *p, const double *q, const double *k, const double *v,
+                    int64_t b, int64_t h, int64_t i, double *s, double *o_out, double *lse_out) {
+  const int64_t d = p->headdim, g = kv_head(p, h);
+  double m, l;
+  row_scores(p, q, k, b, h, i, s, &m, &l);
+  for (int64_t c = 0; c < d; ++c) o_out[c] = 0.0;
+  if (l == 0.0) { *lse_out = -INFINITY; return; }
+  for (int64_t j = 0; j < p->seqlen_k; ++j) {
+    double pij = prob(s[j], m, l);
+    if (pij == 0.0) continue;
+    const double *vj = krow(p, v, b, j, g);
+    for (int64_t c = 0; c < d; ++c) o_out[c] += pij * vj[c];
+  }
+  *lse_out = m + log(l);
+}
+
+static int valid(const oracle_params *p) {
+  return p && p->batch >= 0 && p->seqlen_q >= 0 && p->seqlen_k >= 0 && p->nheads > 0 &&
+         p->nheads_kv > 0 && p->nheads % p->nheads_kv == 0 && p->headdim > 0;
+}
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
+
+void oracle_set_num_threads(int n) {
+#ifdef _OPENMP
+  if (n > 0) omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
+}
+
+/*
+ * Forward for a list of query positions `rows` (nrows of them, each in
+ * [0, Nq)), for every batch and head.  Outputs: o (B, nrows, H, d) and
+ * lse (B, H, nrows).  rows == NULL means all rows in order (nrows = Nq).
+ * Returns 0, or -1 on invalid arguments.
+ */
+int oracle_attn_fwd_rows(const oracle_params *p, const double *q, const double *k, const double *v,
+                         const int64_t *rows, int64_t nrows, double *o, double *lse) {
+  if (!valid(p)) return -1;
+  if (!rows) nrows = p->seqlen_q;
+  const int64_t B = p->batch, H = p->nheads, d = p->headdim;
+  const int64_t total = B * H * nrows;
+  int bad = 0;
+#pragma omp parallel
+  {
+    double *s = (double *)malloc(sizeof(double) * (size_t)(p->seqlen_k > 0 ? p->seqlen_k : 1));
+    if (!s) {
+#pragma omp atomic write
+      bad = 1;
+    }
+#pragma omp for schedule(dynamic, 4)
+    for (int64_t t = 0; t < total; ++t) {
+      if (!s) continue;
+      const int64_t r = t % nrows, h = (t / nrows) % H, b = t / (nrows * H);
+      const int64_t i = rows ? rows[r] : r;
+      if (i < 0 || i >= p->seqlen_q) {
+#pragma omp atomic write
+        bad = 1;
+        continue;
+      }
+      fwd_row(p, q, k, v, b, h, i, s, o + ((b * nrows + r) * H + h) * d, lse + (b * H + h) * nrows + r);
+    }
+    free(s);
+  }
+  return bad ? -1 : 0;
+}
+
+int oracle_attn_fwd(const oracle_params *p, const double *q, const double *k, const double *v,
+                    double *o, double *lse) {
+  return oracle_attn_fwd_rows(p, q, k, v, NULL, 0, o, lse);
+}
+
+/*
+ * Full backward.  dq (B, Nq, H, d); dk, dv (B, Nk, Hkv, d).
+ * Parallel over (batch, kv head) so that the sums into dk/dv over the heads
+ * of a group and over query rows stay within one thread.
+ */
+int oracle_attn_bwd(const oracle_params *p, const double *q, const double *k, const double *v,
+                    const double *dout, double *dq, double *dk, double *dv) {
+  if (!valid(p)) return -1;
+  const int64_t B = p->batch, H = p->nheads, Hkv = p->nheads_kv, d = p->headdim;
+  const int64_t Nq = p->seqlen_q, Nk = p->seqlen_k, group = H / Hkv;
+  memset(dk, 0, sizeof(double) * (size_t)(B * Nk * Hkv * d));
+  memset(dv, 0, sizeof(double) * (size_t)(B * Nk * Hkv * d));
+  int bad = 0;
+#pragma omp parallel
+  {
+    const size_t n = (size_t)(Nk > 0 ? Nk : 1);
+    double *s = (double *)malloc(sizeof(double) * n);
+    double *pr = (double *)malloc(sizeof(double) * n);
+    double *dp = (double *)malloc(sizeof(double) * n);
+    if (!s || !pr || !dp) {
+#pragma omp atomic write
+      bad = 1;
+    }
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t t = 0; t < B * Hkv; ++t) {
+      if (!s || !pr || !dp) continue;
+      const int64_t b = t / Hkv, g = t % Hkv;
+      for (int64_t h = g * group; h < (g + 1) * group; ++h) {
+        for (int64_t i = 0; i < Nq; ++i) {
+          double m, l;
+          const double *qi = qrow(p, q, b, i, h);
+          const double *doi = qrow(p, dout, b, i, h);
+          double *dqi = dq + ((b * Nq + i) * H + h) * d;
+          row_scores(p, q, k, b, h, i, s, &m, &l);
+          double rowsum = 0.0; /* sum_j P_ij dP_ij */
+          for (int64_t j = 0; j < Nk; ++j) {
+            pr[j] = prob(s[j], m, l);
+            dp[j] = (pr[j] != 0.0) ? dot(doi, krow(p, v, b, j, g), d) : 0.0;
+            rowsum += pr[j] * dp[j];
+          }
+          for (int64_t c = 0; c < d; ++c) dqi[c] = 0.0;
+          for (int64_t j = 0; j < Nk; ++j) {
+            if (pr[j] == 0.0) continue;
+            const double ds = pr[j] * (dp[j] - rowsum);
+            const double *kj = krow(p, k, b, j, g);
+            double *dkj = dk + ((b * Nk + j) * Hkv + g) * d;
+            double *dvj = dv + ((b * Nk + j) * Hkv + g) * d;
+            for (int64_t c = 0; c < d; ++c) {
+              dqi[c] += p->softmax_scale * ds * kj[c];
+              dkj[c] += p->softmax_scale * ds * qi[c];
+              dvj[c] += pr[j] * doi[c];
+            }
+          }
+        }
+      }
+    }
+    free(s); free(pr); free(dp);
+  }
+  return bad ? -1 : 0;
+}
+
+/*
+ * Backward on sampled rows.
+ *   dq rows:  query positions qrows[0..nq) -> dq (B, nq, H, d)
+ *   dk/dv rows: key positions krows[0..nk) -> dk, dv (B, nk, Hkv, d)
+ * The dk/dv rows need every query row's softmax statistics and rowsum(P o dP),
+ * which are computed first for all (b, h, i); the sums over i and over the
+ * heads of a group then run for the sampled keys only.
+ */
+int oracle_attn_bwd_rows(const oracle_params *p, const double *q, const double *k, const double *v,
+                         const double *dout, const int64_t *qrows, int64_t nq, double *dq,
+                         const int64_t *krows, int64_t nk, double *dk, double *dv) {
+  if (!valid(p)) return -1;
+  const int64_t B = p->batch, H = p->nheads, Hkv = p->nheads_kv, d = p->headdim;
+  const int64_t Nq = p->seqlen_q, Nk = p->seqlen_k, group = H / Hkv;
+  int bad = 0;
+  for (int64_t r = 0; r < nq; ++r) if (qrows[r] < 0 || qrows[r] >= Nq) return -1;
+  for (int64_t r = 0; r < nk; ++r) if (krows[r] < 0 || krows[r] >= Nk) return -1;
+
+  /* dq rows: each is independent. */
+#pragma omp parallel
+  {
+    const size_t n = (size_t)(Nk > 0 ? Nk : 1);
+    double *s = (double *)malloc(sizeof(double) * n);
+    double *pr = (double *)malloc(sizeof(double) * n);
+    double *dp = (double *)malloc(sizeof(double) * n);
+    if (!s || !pr || !dp) {
+#pragma omp atomic write
+      bad = 1;
+    }
+#pragma omp for schedule(dynamic, 2)
+    for (int64_t t = 0; t < B * H * nq; ++t) {
+      if (!s || !pr || !dp) continue;
+      const int64_t r = t % nq, h = (t / nq) % H, b = t / (nq * H);
+      const int64_t i = qrows[r], g = kv_head(p, h);
+      const double *doi = qrow(p, dout, b, i, h);
+      double *dqi = dq + ((b * nq + r) * H + h) * d;
+      double m, l;
+      row_scores(p, q, k, b, h, i, s, &m, &l);
+      double rowsum = 0.0;
+      for (int64_t j = 0; j < Nk; ++j) {
+        pr[j] = prob(s[j], m, l);
+        dp[j] = (pr[j] != 0.0) ? dot(doi, krow(p, v, b, j, g), d) : 0.0;
+        rowsum += pr[j] * dp[j];
+      }
+      for (int64_t c = 0; c < d; ++c) dqi[c] = 0.0;
+      for (int64_t j = 0; j < Nk; ++j) {
+        if (pr[j] == 0.0) continue;
+        const double ds = pr[j] * (dp[j] - rowsum);
+        const double *kj = krow(p, k, b, j, g);
+        for (int64_t c = 0; c < d; ++c) dqi[c] += p->softmax_scale * ds * kj[c];
+      }
+    }
+    free(s); free(pr); free(dp);
+  }
+  if (bad || nk == 0) return bad ? -1 : 0;
+
+  /* Row statistics of every query row: max, sum and rowsum(P o dP). */
+  const int64_t nrow_all = B * H * Nq;
+  double *M = (double *)malloc(sizeof(double) * (size_t)(nrow_all > 0 ? nrow_all : 1));
+  double *L = (double *)malloc(sizeof(double) * (size_t)(nrow_all > 0 ? nrow_all : 1));
+  double *R = (double *)malloc(sizeof(double) * (size_t)(nrow_all > 0 ? nrow_all : 1));
+  if (!M || !L || !R) { free(M); free(L); free(R); return -1; }
+#pragma omp parallel
+  {
+    const size_t n = (size_t)(Nk > 0 ? Nk : 1);
+    double *s = (double *)malloc(sizeof(double) * n);
+    if (!s) {
+#pragma omp atomic write
+      bad = 1;
+    }
+#pragma omp for schedule(dynamic, 4)
+    for (int64_t t = 0; t < nrow_all; ++t) {
+      if (!s) continue;
+      const int64_t i = t % Nq, h = (t / Nq) % H, b = t / (Nq * H), g = kv_head(p, h);
+      const double *doi = qrow(p, dout, b, i, h);
+      double m, l, rowsum = 0.0;
+      row_scores(p, q, k, b, h, i, s, &m, &l);
+      for (int64_t j = 0; j < Nk; ++j) {
+        const double pij = prob(s[j], m, l);
+        if (pij != 0.0) rowsum += pij * dot(doi, krow(p, v, b, j, g), d);
+      }
+      M[t] = m; L[t] = l; R[t] = rowsum;
+    }
+    free(s);
+  }
+  if (bad) { free(M); free(L); free(R); return -1; }
+
+  /* dk/dv of the sampled keys: sums over the group's heads and all rows. */
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t t = 0; t < B * Hkv * nk; ++t) {
+    const int64_t r = t % nk, g = (t / nk) % Hkv, b = t / (nk * Hkv);
+    const int64_t j = krows[r];
+    const double *kj = krow(p, k, b, j, g), *vj = krow(p, v, b, j, g);
+    double *dkj = dk + ((b * nk + r) * Hkv + g) * d;
+    double *dvj = dv + ((b * nk + r) * Hkv + g) * d;
+    for (int64_t c = 0; c < d; ++c) { dkj[c] = 0.0; dvj[c] = 0.0; }
+    for (int64_t h = g * group; h < (g + 1) * group; ++h) {
+      for (int64_t i = 0; i < Nq; ++i) {
+        if (!visible(p, i, j)) continue;
+        const int64_t row = (b * H + h) * Nq + i;
+        const double *qi = qrow(p, q, b, i, h), *doi = qrow(p, dout, b, i, h);
+        const double sij = p->softmax_scale * dot(qi, kj, d);
+        const double pij = prob(sij, M[row], L[row]);
+        if (pij == 0.0) continue;
+        const double ds = pij * (dot(doi, vj, d) - R[row]);
+        for (int64_t c = 0; c < d; ++c) {
+          dkj[c] += p->softmax_scale * ds * qi[c];
+          dvj[c] += pij * doi[c];
+        }
+      }
+    }
+  }
+  free(M); free(L); free(R);
+  return 0;
+}

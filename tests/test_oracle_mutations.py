@@ -1,0 +1,58 @@
+"""Plant a mistake in a copy of the oracle and check that the pins catch it.
+
+Each mutation is a plausible slip (a dropped term, a wrong sign, a wrong
+index, a transposed operand, an off-by-one in a mask).  The copy is compiled
+in a temporary directory; the oracle itself is never modified.
+"""
+import os
+import shutil
+import subprocess
+
+import pytest
+
+from oracle_pins import ALL_PINS
+
+MUTATIONS = {
+    "score_scale_dropped": ("s[j] = p->softmax_scale * dot(", "s[j] = dot("),
+    "causal_off_by_one": ("if (p->causal && j > ii) return 0;", "if (p->causal && j >= ii) return 0;"),
+    "window_left_sign": ("j < ii - p->window_left", "j < ii + p->window_left"),
+    "window_right_ignored": ("if (p->window_right >= 0 && j > ii + p->window_right) return 0;", ""),
+    "alignment_top_left": ("int64_t ii = i + (p->seqlen_k - p->seqlen_q);", "int64_t ii = i;"),
+    "gqa_mapping_modulo": ("return h / (p->nheads / p->nheads_kv);", "return h % p->nheads_kv;"),
+    "lse_without_max": ("*lse_out = m + log(l);", "*lse_out = log(l);"),
+    "softmax_not_normalised": ("exp(s - m) / l;", "exp(s - m);"),
+    "ds_sign_flipped": ("(dp[j] - rowsum)", "(rowsum - dp[j])"),
+    "ds_rowsum_dropped": ("(dp[j] - rowsum)", "(dp[j])"),
+    "dk_scale_dropped": ("dkj[c] += p->softmax_scale * ds * qi[c];", "dkj[c] += ds * qi[c];"),
+    "dv_operand_swapped": ("dvj[c] += pr[j] * doi[c];", "dvj[c] += pr[j] * qi[c];"),
+    "dq_uses_values": ("dqi[c] += p->softmax_scale * ds * kj[c];",
+                       "dqi[c] += p->softmax_scale * ds * krow(p, v, b, j, g)[c];"),
+    "scores_wrong_head": ("const double *qi = qrow(p, q, b, i, h);\n  double mx",
+                          "const double *qi = qrow(p, q, b, i, 0);\n  double mx"),
+}
+
+
+@pytest.fixture(scope="module")
+def oracle_src(oracle_mod):
+    with open(os.path.join(os.path.dirname(oracle_mod.__file__), "attn_oracle.c")) as f:
+        return f.read()
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_mutation_is_caught(oracle_mod, oracle_src, tmp_path, name):
+    old, new = MUTATIONS[name]
+    assert old in oracle_src, f"mutation {name} no longer matches the oracle source"
+    src = oracle_src.replace(old, new)
+    c = tmp_path / "mutant.c"
+    so = tmp_path / "mutant.so"
+    c.write_text(src)
+    subprocess.run(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off",
+                    "-o", str(so), str(c), "-lm"], check=True)
+    mutant = oracle_mod.Oracle(str(so))
+    caught = []
+    for pin in ALL_PINS:
+        try:
+            pin(mutant)
+        except AssertionError:
+            caught.append(pin.__name__)
+    assert caught, f"no pin caught mutation {name}"
