@@ -1,0 +1,452 @@
+#!/usr/bin/env python
+"""Attention forward + backward throughput on B200.
+
+One step = one pass of the whole path over one batch of synthetic input:
+attn_fwd (O, LSE) followed by the three backward stages (prepare,
+accumulate, finalize -> dQ, dK, dV), on the causal bf16 workload
+B=2, H=32, N=8192, d=128 with Q, K, V, dO ~ N(0, 1) drawn from seed 1.
+
+FLOPs follow the usual convention: forward 4*B*H*N^2*d, halved for causal;
+backward 2.5x the forward.  `value` is whole-job TFLOP/s (all ranks), with
+inputs resident in device memory; `e2e` is the same metric through the
+public API with pinned host buffers, host<->device copies inside the timed
+region.  Inputs (0.54 GB per step) exceed the 126 MB L2, so no flush is done
+between steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Under torchrun each rank runs the same per-GPU workload (weak scaling, no
+data-path collective); the time is the maximum over ranks.  `--impl
+reference` times the float64 CPU oracle on a bounded sample of the same
+workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd/bwd TFLOP/s (bf16, causal, d=128, N=8K) and % of B200 BF16 peak"
+UNIT = "TFLOP/s"
+WORKLOAD = "causal_b2_h32_n8192_d128"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+NOMINAL_BF16_TFLOPS = 2250.0
+KERNEL_SOURCES = ["io_aware_exact_33_b200/csrc/fwd_kernel.cuh",
+                  "io_aware_exact_33_b200/csrc/bwd_kernel.cuh",
+                  "io_aware_exact_33_b200/csrc/sm100.cuh"]
+
+
+# ---------------------------------------------------------------- accounting
+def step_flops(w):
+    """(forward, backward) FLOPs of one pass by the formula convention."""
+    fwd = 4.0 * w.batch * w.nheads * w.seqlen_q * w.seqlen_k * w.headdim
+    if w.causal:
+        fwd /= 2.0
+    return fwd, 2.5 * fwd
+
+
+def visible_pairs(nq, nk, causal, wl, wr, rows=None):
+    """Exact count of visible (query, key) pairs for the given query rows."""
+    off = nk - nq
+    total = 0
+    for i in (range(nq) if rows is None else rows):
+        hi = nk - 1
+        if causal:
+            hi = min(hi, i + off)
+        if wr >= 0:
+            hi = min(hi, i + off + wr)
+        lo = 0 if wl < 0 else max(0, i + off - wl)
+        total += max(0, hi - lo + 1)
+    return total
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"]))}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, or
+    None if absent or taken on different kernel sources."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        ent = d.get(kernel)
+        if not ent or ent.get("source_hash") != kernel_source_hash():
+            return None
+        return float(ent["bytes_per_launch"])
+    except (OSError, ValueError, KeyError):
+        return None
+
+
+# ---------------------------------------------------------------- ranks
+def world_info():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)),
+            int(os.environ.get("WORLD_SIZE", 1)))
+
+
+def init_dist(backend, world):
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return dist if world > 1 else None
+
+
+def barrier(dist, device=None):
+    if dist is not None:
+        if device is not None and dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def max_over_ranks(value, dist, device=None):
+    """Maximum of a float over all ranks (identity on one rank)."""
+    if dist is None:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64,
+                     device=device if dist.get_backend() == "nccl" else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu_id), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+        return False
+
+    def summary(self):
+        sm, smax, reasons = [], [], set()
+        for ln in getattr(self, "lines", []):
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(self.NAMES, parts[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- CPU oracle
+def oracle_sample(w, rows, heads):
+    """A bounded, exact slice of the workload for the float64 oracle: the last
+    `rows` queries of `heads` heads of batch 0 against all keys.  With the
+    bottom-right causal alignment these queries see exactly the keys they
+    see in the full problem.  Returns (inputs, FLOPs by the 4d/10d convention)."""
+    from attn_inputs import make_inputs
+    q, k, v, do = make_inputs(w)
+    hs = slice(0, heads)
+    kv_heads = max(1, heads * w.nheads_kv // w.nheads)
+    q_s = q[:1, -rows:, hs].contiguous()
+    do_s = do[:1, -rows:, hs].contiguous()
+    k_s = k[:1, :, :kv_heads].contiguous()
+    v_s = v[:1, :, :kv_heads].contiguous()
+    first = w.seqlen_q - rows
+    pairs = visible_pairs(w.seqlen_q, w.seqlen_k, w.causal, w.window_left, w.window_right,
+                          rows=range(first, w.seqlen_q))
+    flops = pairs * heads * (4.0 + 10.0) * w.headdim
+    return (q_s, k_s, v_s, do_s), flops
+
+
+def oracle_step(w, inputs):
+    import oracle
+    q, k, v, do = inputs
+    oracle.attention_fwd(q, k, v, w.scale, w.causal, w.window_left, w.window_right)
+    oracle.attention_bwd(q, k, v, do, w.scale, w.causal, w.window_left, w.window_right)
+
+
+def cpu_baseline(w, target_s=12.0):
+    import oracle
+    oracle.build()
+    threads = oracle.num_threads()
+    heads = max(1, min(w.nheads, threads))
+    probe_rows = 32
+    inputs, flops = oracle_sample(w, probe_rows, heads)
+    t0 = time.perf_counter()
+    oracle_step(w, inputs)
+    dt = time.perf_counter() - t0
+    rows = int(min(w.seqlen_q, max(probe_rows, probe_rows * target_s / max(dt, 1e-3))))
+    rows = max(probe_rows, rows // 32 * 32)
+    inputs, flops = oracle_sample(w, rows, heads)
+    t0 = time.perf_counter()
+    oracle_step(w, inputs)
+    dt = time.perf_counter() - t0
+    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": (f"float64 oracle fwd+bwd on the last {rows} queries of {heads} heads "
+                       f"(batch 0) against all {w.seqlen_k} keys of {w.name}; "
+                       f"{flops / 1e9:.1f} GFLOP in {dt:.1f} s"),
+            "seconds": dt}
+
+
+def run_reference(args):
+    """The reference arm: the oracle as it stands, timed on the host cores."""
+    rank, _, world = world_info()
+    if rank != 0:
+        return 0
+    import oracle
+    from attn_inputs import WORKLOADS
+    w = WORKLOADS[WORKLOAD]
+    oracle.build()
+    threads = oracle.num_threads()
+    heads = max(1, min(w.nheads, threads))
+    rows = 64
+    inputs, flops = oracle_sample(w, rows, heads)
+    for _ in range(args.warmup):
+        oracle_step(w, inputs)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(w, inputs)
+    dt = time.perf_counter() - t0
+    value = flops * args.steps / dt / 1e12
+    sample = (f"float64 oracle fwd+bwd on the last {rows} queries of {heads} heads (batch 0) "
+              f"against all {w.seqlen_k} keys of {w.name} per step")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(w),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w):
+    return {"workload": w.name, "batch": w.batch, "nheads": w.nheads, "nheads_kv": w.nheads_kv,
+            "seqlen": w.seqlen_q, "headdim": w.headdim, "causal": w.causal, "pass": "fwd+bwd",
+            "softmax_scale": w.scale, "inputs": "Q,K,V,dO ~ N(0,1), seed 1",
+            "l2": "no flush: inputs 0.54 GB per step exceed the 126 MB L2",
+            "parallelism": "replicas (weak scaling, no collective)"}
+
+
+# ---------------------------------------------------------------- GPU arm
+def run_gpu(args):
+    import torch
+    import io_aware_exact_33_b200 as attn
+    from attn_inputs import WORKLOADS, make_inputs
+
+    rank, local_rank, world = world_info()
+    dist = init_dist("nccl", world)
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = WORKLOADS[WORKLOAD]
+    f_fwd, f_bwd = step_flops(w)
+
+    q, k, v, do = make_inputs(w)
+    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
+    p = attn.params_for(qd, kd, w.scale, w.causal, w.window_left, w.window_right)
+    o = torch.empty_like(qd)
+    lse = torch.empty(w.batch, w.nheads, w.seqlen_q, dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
+    ws = torch.empty(attn.attn_bwd_workspace_size(p), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    nev = 5
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(args.steps)]
+
+    def step(ev=None):
+        if ev: ev[0].record(stream)
+        attn.attn_fwd(qd, kd, vd, w.scale, w.causal, w.window_left, w.window_right, out=o, lse=lse)
+        if ev: ev[1].record(stream)
+        attn.attn_bwd_prepare(p, o, lse, dod, ws)
+        if ev: ev[2].record(stream)
+        attn.attn_bwd_accumulate(p, qd, kd, vd, dod, dk, dv, ws)
+        if ev: ev[3].record(stream)
+        attn.attn_bwd_finalize(p, dq, ws)
+        if ev: ev[4].record(stream)
+
+    launches_per_step = 4
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if attn.attn_get_device_status() != 0:
+        raise RuntimeError("device status word reports an error after warm-up")
+    gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(dist, dev)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(gpu_id) as clk:
+        start.record(stream)
+        for i in range(args.steps):
+            step(events[i])
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(dist, dev)
+    ms_local = start.elapsed_time(end)
+    ms = max_over_ranks(ms_local, dist, dev)
+    t_fwd = [e[0].elapsed_time(e[1]) for e in events]
+    t_prep = [e[1].elapsed_time(e[2]) for e in events]
+    t_main = [e[2].elapsed_time(e[3]) for e in events]
+    t_fin = [e[3].elapsed_time(e[4]) for e in events]
+    value = (f_fwd + f_bwd) * args.steps * world / (ms / 1e3) / 1e12
+
+    # end to end through the public API with pinned host buffers
+    k_e2e = max(1, min(args.steps, args.e2e_steps))
+    hq, hk, hv, hdo = (t.pin_memory() for t in (q, k, v, do))
+    ho, hlse = torch.empty_like(hq).pin_memory(), torch.empty(lse.shape, dtype=torch.float32).pin_memory()
+    hdq, hdk, hdv = (torch.empty_like(t).pin_memory() for t in (hq, hk, hv))
+
+    def e2e_step():
+        qd.copy_(hq, non_blocking=True)
+        kd.copy_(hk, non_blocking=True)
+        vd.copy_(hv, non_blocking=True)
+        dod.copy_(hdo, non_blocking=True)
+        attn.attn_fwd(qd, kd, vd, w.scale, w.causal, w.window_left, w.window_right, out=o, lse=lse)
+        attn.attn_bwd(qd, kd, vd, o, lse, dod, w.scale, w.causal, w.window_left, w.window_right,
+                      dq=dq, dk=dk, dv=dv, workspace=ws)
+        for dst, src in ((ho, o), (hlse, lse), (hdq, dq), (hdk, dk), (hdv, dv)):
+            dst.copy_(src, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier(dist, dev)
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record(stream)
+    for _ in range(k_e2e):
+        e2e_step()
+    e2.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(dist, dev)
+    ms_e2e = max_over_ranks(s2.elapsed_time(e2), dist, dev)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
+    d2h = sum(t.numel() * t.element_size() for t in (ho, hlse, hdq, hdk, hdv))
+    status = attn.attn_get_device_status()
+
+    if rank != 0:
+        if dist is not None:
+            dist.destroy_process_group()
+        return 0
+
+    peaks, peak_kind = load_peaks()
+    mean = lambda xs: sum(xs) / len(xs)
+    kernels = {
+        "attn_fwd_kernel": {"ms": mean(t_fwd), "flops": f_fwd},
+        "attn_bwd_kernel": {"ms": mean(t_main), "flops": f_bwd},
+    }
+    dominant = max(kernels, key=lambda n: kernels[n]["ms"])
+    rl = {}
+    for name, kk in kernels.items():
+        achieved = kk["flops"] / (kk["ms"] / 1e3) / 1e12
+        traffic = recorded_traffic(name)
+        rl[name] = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                    "unit": UNIT, "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
+                    "peak_source": f"bf16_tflops (burst) of {peak_kind}",
+                    "ms_per_launch": kk["ms"], "flops_per_launch": kk["flops"]}
+    cpu = cpu_baseline(w) if (world == 1 and not args.no_cpu_baseline) else None
+    if cpu is not None:
+        cpu.pop("seconds", None)
+    clocks = clk.summary()
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (Q,K,V,dO ~ N(0,1), seed 1)",
+        "config": workload_config(w),
+        "pct_of_peak": {"measured_bf16": value / world / peaks["bf16_tflops"],
+                        "nominal_2250": value / world / NOMINAL_BF16_TFLOPS,
+                        "peak_source": peak_kind},
+        "fwd_tflops": f_fwd / (mean(t_fwd) / 1e3) / 1e12,
+        "bwd_tflops": f_bwd / ((mean(t_prep) + mean(t_main) + mean(t_fin)) / 1e3) / 1e12,
+        "ms": {"fwd": mean(t_fwd), "bwd_prepare": mean(t_prep), "bwd_accumulate": mean(t_main),
+               "bwd_finalize": mean(t_fin)},
+        "roofline": dict(rl[dominant], kernel=dominant),
+        "kernels": rl,
+        "cpu_baseline": cpu,
+        "e2e": {"value": (f_fwd + f_bwd) * k_e2e * world / (ms_e2e / 1e3) / 1e12, "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": k_e2e},
+        "clocks": clocks,
+        "gpu_launches": launches_per_step * args.steps,
+        "device_status": status,
+    }
+    print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

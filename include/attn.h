@@ -1,0 +1,173 @@
+/*
+ * attn.h - C ABI of the B200 (sm_100a) exact-attention library, libattn.so.
+ *
+ * The library computes exact scaled-dot-product attention,
+ *
+ *     O = softmax(Q K^T * softmax_scale + mask) V,
+ *
+ * tile by tile with an online (running max, running sum) softmax, so the
+ * Nq x Nk score matrix never reaches device memory, and the backward pass
+ * that recomputes the score tiles from Q, K, V and the saved per-row
+ * log-sum-exp instead of storing them.
+ *
+ *   - Definition Softmax(QK^T/sqrt(d))V: "FlashAttention ... transformer
+ *     optimization", technical deep dive, first paragraph.
+ *   - Tiling into on-chip blocks, online softmax with a running maximum and
+ *     normalisation factor, recomputation in the backward pass: same page,
+ *     items 1 and 2 and the paragraph after them; "FlashAttention-2 ...
+ *     windows builds analysis", technical deep dive.
+ *   - (batch, seqlen, nheads, headdim) layout, fp16/bf16 only, causal flag,
+ *     explicit softmax_scale: "FlashAttention-2：下一代高效注意力机制的突破与实战
+ *     解析", section "实操落地" (integration example) and its notes.
+ *   - Causal and sliding-window masks with work skipped outside the mask:
+ *     same page, sections "3 支持更灵活的掩码与因果注意力" and "3 稀疏注意力扩展",
+ *     FAQ Q1.
+ *   - MQA/GQA (nheads_kv < nheads) and head dimensions up to 256:
+ *     "FlashAttention 四代演进", sections on architecture and hardware/dtype
+ *     limits.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Pointers named q, k, v, o, dout, dq, dk, dv, lse and workspace are DEVICE
+ * pointers on the current CUDA device; the caller allocates and owns all of
+ * them.  The library never allocates, frees or synchronises on the normal
+ * path; every call is asynchronous on `stream` (a cudaStream_t passed as
+ * void*, NULL = the legacy default stream).  Outputs are valid once the
+ * stream reaches the end of the call.
+ *
+ * Layouts (row-major, contiguous, headdim innermost):
+ *   q, o, dout, dq : (batch, seqlen_q, nheads,    headdim)
+ *   k, v, dk, dv   : (batch, seqlen_k, nheads_kv, headdim)
+ *   lse            : (batch, nheads, seqlen_q) float32, natural log of the
+ *                    row's sum of exp(scaled scores); -inf for a query that
+ *                    sees no key (its O row is then 0).
+ * Element type of q, k, v, o, dout, dq, dk, dv: `dtype` (bf16 or fp16).
+ *
+ * Masks.  Key j is visible from query i iff, with off = seqlen_k - seqlen_q
+ * (bottom-right alignment),
+ *     causal:            j <= i + off
+ *     window_left  >= 0: j >= i + off - window_left
+ *     window_right >= 0: j <= i + off + window_right
+ * Bounds are inclusive; -1 means unbounded.
+ *
+ * Grouped-query attention: query head h reads kv head h / (nheads/nheads_kv).
+ *
+ * Errors are returned, never raised: no exception or abort crosses the ABI.
+ * Argument errors are detected on the host before anything is launched.
+ * A launch failure returns ATTN_ERR_CUDA (the CUDA error is then available
+ * from cudaGetLastError's successor calls in the caller's runtime).  Kernels
+ * that wait on on-chip barriers give up after a bounded time, record a code
+ * in a device status word and exit; attn_get_device_status() reads it.
+ */
+#ifndef ATTN_H
+#define ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ATTN_API __attribute__((visibility("default")))
+#else
+#define ATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { ATTN_BF16 = 0, ATTN_FP16 = 1 } attn_dtype;
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = 1,          /* null pointer, negative size, H % Hkv != 0, bad window */
+  ATTN_ERR_UNSUPPORTED_HEADDIM = 2,  /* headdim outside the compiled set */
+  ATTN_ERR_UNSUPPORTED_DTYPE = 3,    /* dtype not bf16/fp16 */
+  ATTN_ERR_MISALIGNED = 4,           /* a tensor pointer not 16-byte aligned */
+  ATTN_ERR_WORKSPACE_TOO_SMALL = 5,  /* workspace_bytes below the *_workspace_size() query */
+  ATTN_ERR_CUDA = 6,                 /* a CUDA runtime/driver call failed */
+  ATTN_ERR_TIMEOUT = 7,              /* a device-side bounded wait expired */
+  ATTN_ERR_DEVICE_STATUS = 8         /* the device status word holds another error */
+} attn_status;
+
+typedef struct {
+  int32_t batch;
+  int32_t seqlen_q;
+  int32_t seqlen_k;
+  int32_t nheads;
+  int32_t nheads_kv;
+  int32_t headdim;
+  int32_t dtype;          /* attn_dtype */
+  float softmax_scale;    /* multiplies Q K^T; the usual value is 1/sqrt(headdim) */
+  int32_t causal;         /* 0 or 1 */
+  int32_t window_left;    /* -1 = unbounded */
+  int32_t window_right;   /* -1 = unbounded */
+} attn_params;
+
+/*
+ * Forward pass.  Reads q, k, v; writes o and lse.
+ * Supported: headdim in {64, 128, 256}; dtype bf16 or fp16.
+ * workspace may be NULL when attn_fwd_workspace_size() returns 0.
+ * Sizes may be zero (batch, seqlen_q, seqlen_k): an empty call is a no-op,
+ * and seqlen_k == 0 yields O = 0 and LSE = -inf.
+ */
+ATTN_API attn_status attn_fwd(const attn_params* p, const void* q, const void* k, const void* v, void* o,
+                     float* lse, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Backward pass: given dout = dL/dO and the forward's o and lse, writes
+ * dq = dL/dQ, dk = dL/dK, dv = dL/dV (dk, dv summed over the query heads of
+ * each kv group).  The score tiles are recomputed from q, k and lse.
+ * Supported: headdim in {64, 128}; dtype bf16 or fp16.
+ * workspace: at least attn_bwd_workspace_size(p) bytes, 256-byte aligned;
+ * it holds float32 rowsum(dO o O), lse in base 2 and the float32 dQ
+ * accumulator.  Its contents on entry do not matter.
+ */
+ATTN_API attn_status attn_bwd(const attn_params* p, const void* q, const void* k, const void* v,
+                     const void* o, const float* lse, const void* dout, void* dq, void* dk,
+                     void* dv, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * The three stages attn_bwd runs, in this order, on one stream and one
+ * workspace; exposed so a caller can time or schedule them separately.
+ * Same arguments, layouts and errors as attn_bwd.
+ *   attn_bwd_prepare:    float32 rowsum(dout o o) and lse*log2(e) per query
+ *                        into the workspace; zeroes the dQ accumulator.
+ *   attn_bwd_accumulate: recomputes the score tiles and writes dk and dv;
+ *                        adds every key tile's dQ share into the accumulator.
+ *   attn_bwd_finalize:   dq = softmax_scale * accumulator, in `dtype`.
+ */
+ATTN_API attn_status attn_bwd_prepare(const attn_params* p, const void* o, const float* lse,
+                                      const void* dout, void* workspace, size_t workspace_bytes,
+                                      void* stream);
+ATTN_API attn_status attn_bwd_accumulate(const attn_params* p, const void* q, const void* k,
+                                         const void* v, const void* dout, void* dk, void* dv,
+                                         void* workspace, size_t workspace_bytes, void* stream);
+ATTN_API attn_status attn_bwd_finalize(const attn_params* p, void* dq, void* workspace,
+                                       size_t workspace_bytes, void* stream);
+
+/* Bytes of device workspace attn_fwd / attn_bwd need for these parameters
+ * (0 when none).  Pure host functions; never touch the GPU. */
+ATTN_API size_t attn_fwd_workspace_size(const attn_params* p);
+ATTN_API size_t attn_bwd_workspace_size(const attn_params* p);
+
+/* Host-side argument check that attn_fwd / attn_bwd perform first; exposed so
+ * callers (and the CPU-only tests) can validate without a GPU.  `pass` is 0
+ * for forward, 1 for backward.  Pointers are not inspected. */
+ATTN_API attn_status attn_check_params(const attn_params* p, int pass);
+
+/* A static, human-readable description of a status code. */
+ATTN_API const char* attn_status_string(int status);
+
+/* Reads and clears the device status word (0 = no device-side error).
+ * Synchronises `stream`.  Returns ATTN_OK, or ATTN_ERR_CUDA if the read
+ * failed.  *code receives an ATTN_ERR_* value or 0. */
+ATTN_API attn_status attn_get_device_status(void* stream, int* code);
+
+/* Library version, "major.minor.patch". */
+ATTN_API const char* attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_H */

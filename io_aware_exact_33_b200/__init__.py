@@ -1,0 +1,263 @@
+"""Python binding of libattn.so, the sm_100a exact-attention library.
+
+Argument marshalling only: torch supplies device memory and the current CUDA
+stream, and every step of the attention computation runs in the library's
+kernels.  The entry points carry the C ABI's names (``include/attn.h``):
+``attn_fwd``, ``attn_bwd``, ``attn_fwd_workspace_size``,
+``attn_bwd_workspace_size``, ``attn_check_params``, ``attn_status_string``,
+``attn_get_device_status`` and ``attn_version``.
+
+There is no fallback: if the compiled library is missing, the first call
+raises an ImportError that says how to build it.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Tuple
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libattn.so")
+
+ATTN_BF16, ATTN_FP16 = 0, 1
+STATUS = {
+    0: "ATTN_OK", 1: "ATTN_ERR_INVALID_ARG", 2: "ATTN_ERR_UNSUPPORTED_HEADDIM",
+    3: "ATTN_ERR_UNSUPPORTED_DTYPE", 4: "ATTN_ERR_MISALIGNED", 5: "ATTN_ERR_WORKSPACE_TOO_SMALL",
+    6: "ATTN_ERR_CUDA", 7: "ATTN_ERR_TIMEOUT", 8: "ATTN_ERR_DEVICE_STATUS",
+}
+EXPORTED = ("attn_fwd", "attn_bwd", "attn_bwd_prepare", "attn_bwd_accumulate", "attn_bwd_finalize",
+            "attn_fwd_workspace_size", "attn_bwd_workspace_size", "attn_check_params",
+            "attn_status_string", "attn_get_device_status", "attn_version")
+
+
+class AttnParams(ctypes.Structure):
+    """Mirror of ``attn_params`` in include/attn.h."""
+    _fields_ = [
+        ("batch", ctypes.c_int32),
+        ("seqlen_q", ctypes.c_int32),
+        ("seqlen_k", ctypes.c_int32),
+        ("nheads", ctypes.c_int32),
+        ("nheads_kv", ctypes.c_int32),
+        ("headdim", ctypes.c_int32),
+        ("dtype", ctypes.c_int32),
+        ("softmax_scale", ctypes.c_float),
+        ("causal", ctypes.c_int32),
+        ("window_left", ctypes.c_int32),
+        ("window_right", ctypes.c_int32),
+    ]
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)} ({attn_status_string(status)})")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m io_aware_exact_33_b200.build` "
+            "(nvcc, sm_100a). There is no fallback implementation.")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, sz, P = ctypes.c_void_p, ctypes.c_size_t, ctypes.POINTER(AttnParams)
+    lib.attn_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.attn_fwd.restype = ctypes.c_int
+    lib.attn_bwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.attn_bwd.restype = ctypes.c_int
+    lib.attn_bwd_prepare.argtypes = [P, vp, vp, vp, vp, sz, vp]
+    lib.attn_bwd_prepare.restype = ctypes.c_int
+    lib.attn_bwd_accumulate.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.attn_bwd_accumulate.restype = ctypes.c_int
+    lib.attn_bwd_finalize.argtypes = [P, vp, vp, sz, vp]
+    lib.attn_bwd_finalize.restype = ctypes.c_int
+    lib.attn_fwd_workspace_size.argtypes = [P]
+    lib.attn_fwd_workspace_size.restype = sz
+    lib.attn_bwd_workspace_size.argtypes = [P]
+    lib.attn_bwd_workspace_size.restype = sz
+    lib.attn_check_params.argtypes = [P, ctypes.c_int]
+    lib.attn_check_params.restype = ctypes.c_int
+    lib.attn_status_string.argtypes = [ctypes.c_int]
+    lib.attn_status_string.restype = ctypes.c_char_p
+    lib.attn_get_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
+    lib.attn_get_device_status.restype = ctypes.c_int
+    lib.attn_version.argtypes = []
+    lib.attn_version.restype = ctypes.c_char_p
+    return lib
+
+
+_handle = None
+
+
+class _Lazy:
+    """Loads libattn.so on first use; raises ImportError if it was not built."""
+
+    def __getattr__(self, name):
+        global _handle
+        if _handle is None:
+            _handle = _load()
+        return getattr(_handle, name)
+
+
+_lib = _Lazy()
+
+
+def make_params(batch, seqlen_q, seqlen_k, nheads, nheads_kv, headdim, dtype=ATTN_BF16,
+                softmax_scale=None, causal=False, window_left=-1, window_right=-1) -> AttnParams:
+    scale = 1.0 / math.sqrt(headdim) if softmax_scale is None else float(softmax_scale)
+    return AttnParams(int(batch), int(seqlen_q), int(seqlen_k), int(nheads), int(nheads_kv),
+                      int(headdim), int(dtype), scale, int(bool(causal)), int(window_left),
+                      int(window_right))
+
+
+def attn_status_string(status: int) -> str:
+    return _lib.attn_status_string(int(status)).decode()
+
+
+def attn_version() -> str:
+    return _lib.attn_version().decode()
+
+
+def attn_check_params(p: AttnParams, pass_: int = 0) -> int:
+    return int(_lib.attn_check_params(ctypes.byref(p), int(pass_)))
+
+
+def attn_fwd_workspace_size(p: AttnParams) -> int:
+    return int(_lib.attn_fwd_workspace_size(ctypes.byref(p)))
+
+
+def attn_bwd_workspace_size(p: AttnParams) -> int:
+    return int(_lib.attn_bwd_workspace_size(ctypes.byref(p)))
+
+
+def attn_get_device_status(stream=None) -> int:
+    import torch
+    s = torch.cuda.current_stream().cuda_stream if stream is None else int(stream)
+    code = ctypes.c_int(0)
+    st = _lib.attn_get_device_status(ctypes.c_void_p(s), ctypes.byref(code))
+    if st != 0:
+        raise AttnError(st, "attn_get_device_status")
+    return int(code.value)
+
+
+# ----------------------------------------------------------------- torch side
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.bfloat16:
+        return ATTN_BF16
+    if t.dtype == torch.float16:
+        return ATTN_FP16
+    raise TypeError(f"attention inputs must be bf16 or fp16, got {t.dtype}")
+
+
+def _check(t, name, shape=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr() if t is not None else 0)
+
+
+def _stream(stream):
+    import torch
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream if stream is None else int(stream))
+
+
+def params_for(q, k, softmax_scale=None, causal=False, window_left=-1, window_right=-1):
+    B, Nq, H, d = q.shape
+    Bk, Nk, Hkv, dk = k.shape
+    if Bk != B or dk != d:
+        raise ValueError("q and k disagree on batch or head dim")
+    return make_params(B, Nq, Nk, H, Hkv, d, _dtype_code(q), softmax_scale, causal, window_left,
+                       window_right)
+
+
+def attn_fwd(q, k, v, softmax_scale: Optional[float] = None, causal: bool = False,
+             window_left: int = -1, window_right: int = -1, out=None, lse=None,
+             stream=None) -> Tuple["torch.Tensor", "torch.Tensor"]:
+    """O = softmax(q k^T * scale + mask) v and the per-row natural-log LSE.
+
+    q (B, Nq, H, d), k and v (B, Nk, Hkv, d), bf16 or fp16, contiguous CUDA
+    tensors.  Returns (out (B, Nq, H, d), lse (B, H, Nq) float32)."""
+    import torch
+    p = params_for(q, k, softmax_scale, causal, window_left, window_right)
+    B, Nq, H, d = q.shape
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, n)
+        if t.dtype != q.dtype:
+            raise TypeError("q, k, v must share a dtype")
+    _check(v, "v", k.shape)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    _check(out, "out", q.shape)
+    _check(lse, "lse", (B, H, Nq))
+    ws_bytes = attn_fwd_workspace_size(p)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device) if ws_bytes else None
+    st = _lib.attn_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                       _ptr(ws), ctypes.c_size_t(ws_bytes), _stream(stream))
+    if st != 0:
+        raise AttnError(st, "attn_fwd")
+    return out, lse
+
+
+def attn_bwd(q, k, v, out, lse, dout, softmax_scale: Optional[float] = None, causal: bool = False,
+             window_left: int = -1, window_right: int = -1, dq=None, dk=None, dv=None,
+             workspace=None, stream=None):
+    """Gradients (dq, dk, dv) of sum(out * dout) for attention with the same
+    arguments as ``attn_fwd``; ``out`` and ``lse`` are its results."""
+    import torch
+    p = params_for(q, k, softmax_scale, causal, window_left, window_right)
+    B, Nq, H, d = q.shape
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
+        _check(t, n)
+        if t.dtype != q.dtype:
+            raise TypeError("q, k, v, out, dout must share a dtype")
+    _check(v, "v", k.shape)
+    _check(out, "out", q.shape)
+    _check(dout, "dout", q.shape)
+    _check(lse, "lse", (B, H, Nq))
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    ws_bytes = attn_bwd_workspace_size(p)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
+    st = _lib.attn_bwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                       _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
+                       ctypes.c_size_t(workspace.numel()), _stream(stream))
+    if st != 0:
+        raise AttnError(st, "attn_bwd")
+    return dq, dk, dv
+
+
+def attn_bwd_prepare(p: AttnParams, out, lse, dout, workspace, stream=None) -> None:
+    """First backward stage (rowsum(dout*out), lse in base 2, zeroed dQ
+    accumulator) on already-validated torch tensors and a params struct."""
+    st = _lib.attn_bwd_prepare(ctypes.byref(p), _ptr(out), _ptr(lse), _ptr(dout), _ptr(workspace),
+                               ctypes.c_size_t(workspace.numel()), _stream(stream))
+    if st != 0:
+        raise AttnError(st, "attn_bwd_prepare")
+
+
+def attn_bwd_accumulate(p: AttnParams, q, k, v, dout, dk, dv, workspace, stream=None) -> None:
+    """Second backward stage: dk, dv and the fp32 dQ accumulator."""
+    st = _lib.attn_bwd_accumulate(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dk),
+                                  _ptr(dv), _ptr(workspace), ctypes.c_size_t(workspace.numel()),
+                                  _stream(stream))
+    if st != 0:
+        raise AttnError(st, "attn_bwd_accumulate")
+
+
+def attn_bwd_finalize(p: AttnParams, dq, workspace, stream=None) -> None:
+    """Third backward stage: dq = scale * accumulator in the input dtype."""
+    st = _lib.attn_bwd_finalize(ctypes.byref(p), _ptr(dq), _ptr(workspace),
+                                ctypes.c_size_t(workspace.numel()), _stream(stream))
+    if st != 0:
+        raise AttnError(st, "attn_bwd_finalize")

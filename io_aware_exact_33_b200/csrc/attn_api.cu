@@ -1,0 +1,424 @@
+// attn_api.cu - the C ABI of libattn.so (declared in include/attn.h): host
+// argument checks, TMA tensor-map construction, kernel selection and launch.
+// Every computation of the attention path runs in the kernels; this file
+// only marshals arguments.
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <set>
+#include <utility>
+
+#include "attn.h"
+#include "bwd_kernel.cuh"
+#include "fwd_kernel.cuh"
+#include "sm100.cuh"
+
+namespace {
+
+using namespace attn;
+
+// ------------------------------------------------------------ driver entry
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// (batch, seqlen, heads, headdim) 16-bit tensor as a 4-D TMA map over
+// (headdim, heads, seqlen, batch); box = 64 columns x 1 head x `rows` rows,
+// 128-byte swizzle.  Rows past seqlen read as zero and are never written.
+bool map_bshd(CUtensorMap* m, const void* ptr, bool fp16, int batch, int seqlen, int heads, int d,
+              int rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)seqlen, (cuuint64_t)batch};
+  cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)heads * d * 2,
+                           (cuuint64_t)seqlen * heads * d * 2};
+  cuuint32_t box[4] = {64, 1, (cuuint32_t)rows, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(m, fp16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+                   const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// 2-D fp32 map over (cols, rows_total) with box (box_cols, 1), no swizzle.
+bool map_f32_rows(CUtensorMap* m, const void* ptr, long long cols, long long rows, int box_cols) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * 4};
+  cuuint32_t box[2] = {(cuuint32_t)box_cols, 1};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(ptr), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Opt a kernel into its dynamic shared memory once per (kernel, device).
+bool ensure_smem(const void* kernel, int bytes) {
+  static std::mutex mu;
+  static std::set<std::pair<const void*, int>> done;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  std::lock_guard<std::mutex> g(mu);
+  if (done.count({kernel, dev})) return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+      cudaSuccess)
+    return false;
+  done.insert({kernel, dev});
+  return true;
+}
+
+bool debug_status_enabled() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = std::getenv("ATTN_DEBUG_STATUS");
+    v = (e && e[0] == '1') ? 1 : 0;
+  }
+  return v == 1;
+}
+
+attn_status finish(cudaStream_t stream) {
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  if (debug_status_enabled()) {
+    int code = 0;
+    attn_status s = attn_get_device_status(stream, &code);
+    if (s != ATTN_OK) return s;
+    if (code == ATTN_ERR_TIMEOUT) return ATTN_ERR_TIMEOUT;
+    if (code != 0) return ATTN_ERR_DEVICE_STATUS;
+  }
+  return ATTN_OK;
+}
+
+// O = 0 and LSE = -inf for every query when no key exists.
+__global__ void fill_empty_fwd(uint16_t* o, long long n_o, float* lse, long long n_lse) {
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n_o; i += stride) o[i] = 0;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n_lse; i += stride)
+    lse[i] = -INFINITY;
+}
+
+// Zero a 16-bit tensor (gradients of an empty side).
+__global__ void fill_zero_u16(uint16_t* x, long long n) {
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += stride) x[i] = 0;
+}
+
+int fill_blocks(long long n) {
+  long long b = (n + 255) / 256;
+  return (int)(b < 1 ? 1 : (b > 4096 ? 4096 : b));
+}
+
+template <class C>
+attn_status launch_fwd(const attn_params* p, const void* q, const void* k, const void* v, void* o,
+                       float* lse, cudaStream_t stream) {
+  CUtensorMap mq, mk, mv, mo;
+  const bool fp16 = C::FP16;
+  if (!map_bshd(&mq, q, fp16, p->batch, p->seqlen_q, p->nheads, C::D, C::BM) ||
+      !map_bshd(&mk, k, fp16, p->batch, p->seqlen_k, p->nheads_kv, C::D, C::BN) ||
+      !map_bshd(&mv, v, fp16, p->batch, p->seqlen_k, p->nheads_kv, C::D, C::BN) ||
+      !map_bshd(&mo, o, fp16, p->batch, p->seqlen_q, p->nheads, C::D, C::BM))
+    return ATTN_ERR_CUDA;
+  FwdParams fp;
+  fp.lse = lse;
+  fp.batch = p->batch;
+  fp.nheads = p->nheads;
+  fp.nheads_kv = p->nheads_kv;
+  fp.seqlen_q = p->seqlen_q;
+  fp.seqlen_k = p->seqlen_k;
+  fp.causal = p->causal;
+  fp.window_left = p->window_left;
+  fp.window_right = p->window_right;
+  fp.scale_log2 = p->softmax_scale * 1.4426950408889634f;
+  fp.num_qblocks = (p->seqlen_q + C::BM - 1) / C::BM;
+  auto kern = attn_fwd_kernel<C>;
+  if (!ensure_smem(reinterpret_cast<const void*>(kern), C::SMEM_BYTES)) return ATTN_ERR_CUDA;
+  dim3 grid(fp.num_qblocks, p->nheads, p->batch);
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mo, fp);
+  return finish(stream);
+}
+
+BwdParams bwd_params(const attn_params* p, const float* lse, void* workspace) {
+  const BwdWorkspace ws = bwd_workspace_layout(p->batch, p->nheads, p->seqlen_q, p->headdim);
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  BwdParams bp;
+  bp.lse = lse;
+  bp.dvec = reinterpret_cast<float*>(w + ws.dvec_off);
+  bp.lse2 = reinterpret_cast<float*>(w + ws.lse2_off);
+  bp.dq_acc = reinterpret_cast<float*>(w + ws.dq_off);
+  bp.batch = p->batch;
+  bp.nheads = p->nheads;
+  bp.nheads_kv = p->nheads_kv;
+  bp.seqlen_q = p->seqlen_q;
+  bp.seqlen_k = p->seqlen_k;
+  bp.headdim = p->headdim;
+  bp.causal = p->causal;
+  bp.window_left = p->window_left;
+  bp.window_right = p->window_right;
+  bp.scale_log2 = p->softmax_scale * 1.4426950408889634f;
+  bp.softmax_scale = p->softmax_scale;
+  bp.nq_pad = ws.nq_pad;
+  return bp;
+}
+
+attn_status launch_bwd_prepare(const attn_params* p, const void* o, const float* lse,
+                               const void* dout, void* workspace, cudaStream_t stream) {
+  const BwdParams bp = bwd_params(p, lse, workspace);
+  const long long n_rows = (long long)p->batch * p->nheads * bp.nq_pad;
+  const long long n_elems = (long long)p->batch * p->seqlen_q * p->nheads * p->headdim;
+  if (p->dtype == ATTN_FP16)
+    bwd_preprocess<true><<<2368, 256, 0, stream>>>(static_cast<const uint16_t*>(o),
+                                                    static_cast<const uint16_t*>(dout), bp, n_rows,
+                                                    n_elems / 4);
+  else
+    bwd_preprocess<false><<<2368, 256, 0, stream>>>(static_cast<const uint16_t*>(o),
+                                                     static_cast<const uint16_t*>(dout), bp,
+                                                     n_rows, n_elems / 4);
+  return finish(stream);
+}
+
+template <class C>
+attn_status launch_bwd_main(const attn_params* p, const void* q, const void* k, const void* v,
+                            const void* dout, void* dk, void* dv, void* workspace,
+                            cudaStream_t stream) {
+  const BwdParams bp = bwd_params(p, nullptr, workspace);
+  const bool fp16 = C::FP16;
+  CUtensorMap mq, mk, mv, mdo, ml, md, mdk, mdv;
+  if (!map_bshd(&mq, q, fp16, p->batch, p->seqlen_q, p->nheads, C::D, C::BM) ||
+      !map_bshd(&mk, k, fp16, p->batch, p->seqlen_k, p->nheads_kv, C::D, C::BN) ||
+      !map_bshd(&mv, v, fp16, p->batch, p->seqlen_k, p->nheads_kv, C::D, C::BN) ||
+      !map_bshd(&mdo, dout, fp16, p->batch, p->seqlen_q, p->nheads, C::D, C::BM) ||
+      !map_f32_rows(&ml, bp.lse2, bp.nq_pad, (long long)p->batch * p->nheads, C::BM) ||
+      !map_f32_rows(&md, bp.dvec, bp.nq_pad, (long long)p->batch * p->nheads, C::BM) ||
+      !map_bshd(&mdk, dk, fp16, p->batch, p->seqlen_k, p->nheads_kv, C::D, C::BN) ||
+      !map_bshd(&mdv, dv, fp16, p->batch, p->seqlen_k, p->nheads_kv, C::D, C::BN))
+    return ATTN_ERR_CUDA;
+  auto kern = attn_bwd_kernel<C>;
+  if (!ensure_smem(reinterpret_cast<const void*>(kern), C::SMEM_BYTES)) return ATTN_ERR_CUDA;
+  dim3 grid((p->seqlen_k + C::BN - 1) / C::BN, p->nheads_kv, p->batch);
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, ml, md, mdk, mdv, bp);
+  return finish(stream);
+}
+
+attn_status launch_bwd_finalize(const attn_params* p, void* dq, void* workspace,
+                                cudaStream_t stream) {
+  const BwdParams bp = bwd_params(p, nullptr, workspace);
+  const long long n_elems = (long long)p->batch * p->seqlen_q * p->nheads * p->headdim;
+  if (p->dtype == ATTN_FP16)
+    bwd_convert<true><<<2368, 256, 0, stream>>>(bp.dq_acc, static_cast<uint16_t*>(dq),
+                                                 n_elems / 4, p->softmax_scale);
+  else
+    bwd_convert<false><<<2368, 256, 0, stream>>>(bp.dq_acc, static_cast<uint16_t*>(dq),
+                                                  n_elems / 4, p->softmax_scale);
+  return finish(stream);
+}
+
+// Shared argument checks of the backward entry points.  Returns ATTN_OK when
+// the call has work to do, or sets *done when it is complete without any.
+attn_status bwd_common_checks(const attn_params* p, const void* workspace, size_t workspace_bytes,
+                              bool* empty) {
+  attn_status st = attn_check_params(p, 1);
+  if (st != ATTN_OK) return st;
+  *empty = p->batch == 0 || p->seqlen_q == 0 || p->seqlen_k == 0;
+  if (*empty) return ATTN_OK;
+  const BwdWorkspace ws = bwd_workspace_layout(p->batch, p->nheads, p->seqlen_q, p->headdim);
+  if (!workspace || workspace_bytes < ws.total) return ATTN_ERR_WORKSPACE_TOO_SMALL;
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u) return ATTN_ERR_MISALIGNED;
+  return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* attn_version(void) { return "0.1.0"; }
+
+const char* attn_status_string(int s) {
+  switch (s) {
+    case ATTN_OK: return "ok";
+    case ATTN_ERR_INVALID_ARG: return "invalid argument";
+    case ATTN_ERR_UNSUPPORTED_HEADDIM: return "unsupported head dimension";
+    case ATTN_ERR_UNSUPPORTED_DTYPE: return "unsupported dtype (bf16 or fp16 only)";
+    case ATTN_ERR_MISALIGNED: return "tensor pointer not 16-byte aligned";
+    case ATTN_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case ATTN_ERR_CUDA: return "CUDA call failed";
+    case ATTN_ERR_TIMEOUT: return "device-side wait timed out";
+    case ATTN_ERR_DEVICE_STATUS: return "device status word holds an error";
+    default: return "unknown status";
+  }
+}
+
+attn_status attn_check_params(const attn_params* p, int pass) {
+  if (!p || (pass != 0 && pass != 1)) return ATTN_ERR_INVALID_ARG;
+  if (p->batch < 0 || p->seqlen_q < 0 || p->seqlen_k < 0) return ATTN_ERR_INVALID_ARG;
+  if (p->nheads <= 0 || p->nheads_kv <= 0 || p->nheads % p->nheads_kv != 0)
+    return ATTN_ERR_INVALID_ARG;
+  if (p->nheads > 65535 || p->batch > 65535) return ATTN_ERR_INVALID_ARG;
+  if (p->dtype != ATTN_BF16 && p->dtype != ATTN_FP16) return ATTN_ERR_UNSUPPORTED_DTYPE;
+  const int d = p->headdim;
+  if (pass == 0 && d != 64 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED_HEADDIM;
+  if (pass == 1 && d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED_HEADDIM;
+  if (!(p->softmax_scale > 0.f) || !std::isfinite(p->softmax_scale)) return ATTN_ERR_INVALID_ARG;
+  if (p->causal != 0 && p->causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (p->window_left < -1 || p->window_right < -1) return ATTN_ERR_INVALID_ARG;
+  return ATTN_OK;
+}
+
+size_t attn_fwd_workspace_size(const attn_params* p) {
+  (void)p;
+  return 0;
+}
+
+attn_status attn_fwd(const attn_params* p, const void* q, const void* k, const void* v, void* o,
+                     float* lse, void* workspace, size_t workspace_bytes, void* stream_) {
+  (void)workspace;
+  (void)workspace_bytes;
+  attn_status st = attn_check_params(p, 0);
+  if (st != ATTN_OK) return st;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (p->batch == 0 || p->seqlen_q == 0) return ATTN_OK;
+  if (!o || !lse) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(o) || (reinterpret_cast<uintptr_t>(lse) & 3u)) return ATTN_ERR_MISALIGNED;
+  if (p->seqlen_k == 0) {
+    const long long n_o = (long long)p->batch * p->seqlen_q * p->nheads * p->headdim;
+    const long long n_l = (long long)p->batch * p->nheads * p->seqlen_q;
+    fill_empty_fwd<<<fill_blocks(n_o), 256, 0, stream>>>(static_cast<uint16_t*>(o), n_o, lse, n_l);
+    return finish(stream);
+  }
+  if (!q || !k || !v) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return ATTN_ERR_MISALIGNED;
+  const bool fp16 = p->dtype == ATTN_FP16;
+  switch (p->headdim) {
+    case 64:
+      return fp16 ? launch_fwd<FwdCfg<64, 128, 3, true>>(p, q, k, v, o, lse, stream)
+                  : launch_fwd<FwdCfg<64, 128, 3, false>>(p, q, k, v, o, lse, stream);
+    case 128:
+      return fp16 ? launch_fwd<FwdCfg<128, 128, 2, true>>(p, q, k, v, o, lse, stream)
+                  : launch_fwd<FwdCfg<128, 128, 2, false>>(p, q, k, v, o, lse, stream);
+    case 256:
+      return fp16 ? launch_fwd<FwdCfg<256, 64, 2, true>>(p, q, k, v, o, lse, stream)
+                  : launch_fwd<FwdCfg<256, 64, 2, false>>(p, q, k, v, o, lse, stream);
+    default:
+      return ATTN_ERR_UNSUPPORTED_HEADDIM;
+  }
+}
+
+size_t attn_bwd_workspace_size(const attn_params* p) {
+  if (attn_check_params(p, 1) != ATTN_OK) return 0;
+  return bwd_workspace_layout(p->batch, p->nheads, p->seqlen_q, p->headdim).total;
+}
+
+attn_status attn_bwd_prepare(const attn_params* p, const void* o, const float* lse,
+                             const void* dout, void* workspace, size_t workspace_bytes,
+                             void* stream_) {
+  bool empty = false;
+  attn_status st = bwd_common_checks(p, workspace, workspace_bytes, &empty);
+  if (st != ATTN_OK || empty) return st;
+  if (!o || !lse || !dout) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(o) || !aligned16(dout) || (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return ATTN_ERR_MISALIGNED;
+  return launch_bwd_prepare(p, o, lse, dout, workspace, reinterpret_cast<cudaStream_t>(stream_));
+}
+
+attn_status attn_bwd_accumulate(const attn_params* p, const void* q, const void* k, const void* v,
+                                const void* dout, void* dk, void* dv, void* workspace,
+                                size_t workspace_bytes, void* stream_) {
+  bool empty = false;
+  attn_status st = bwd_common_checks(p, workspace, workspace_bytes, &empty);
+  if (st != ATTN_OK || empty) return st;
+  if (!q || !k || !v || !dout || !dk || !dv) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dk) ||
+      !aligned16(dv))
+    return ATTN_ERR_MISALIGNED;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  const bool fp16 = p->dtype == ATTN_FP16;
+  switch (p->headdim) {
+    case 64:
+      return fp16 ? launch_bwd_main<BwdCfg<64, true>>(p, q, k, v, dout, dk, dv, workspace, stream)
+                  : launch_bwd_main<BwdCfg<64, false>>(p, q, k, v, dout, dk, dv, workspace, stream);
+    case 128:
+      return fp16 ? launch_bwd_main<BwdCfg<128, true>>(p, q, k, v, dout, dk, dv, workspace, stream)
+                  : launch_bwd_main<BwdCfg<128, false>>(p, q, k, v, dout, dk, dv, workspace, stream);
+    default:
+      return ATTN_ERR_UNSUPPORTED_HEADDIM;
+  }
+}
+
+attn_status attn_bwd_finalize(const attn_params* p, void* dq, void* workspace,
+                              size_t workspace_bytes, void* stream_) {
+  bool empty = false;
+  attn_status st = bwd_common_checks(p, workspace, workspace_bytes, &empty);
+  if (st != ATTN_OK || empty) return st;
+  if (!dq) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(dq)) return ATTN_ERR_MISALIGNED;
+  return launch_bwd_finalize(p, dq, workspace, reinterpret_cast<cudaStream_t>(stream_));
+}
+
+attn_status attn_bwd(const attn_params* p, const void* q, const void* k, const void* v,
+                     const void* o, const float* lse, const void* dout, void* dq, void* dk,
+                     void* dv, void* workspace, size_t workspace_bytes, void* stream_) {
+  attn_status st = attn_check_params(p, 1);
+  if (st != ATTN_OK) return st;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (p->batch == 0) return ATTN_OK;
+  const long long n_q = (long long)p->batch * p->seqlen_q * p->nheads * p->headdim;
+  const long long n_k = (long long)p->batch * p->seqlen_k * p->nheads_kv * p->headdim;
+  if (p->seqlen_q == 0 || p->seqlen_k == 0) {
+    // Nothing to attend: every gradient is zero.
+    if ((n_q && !dq) || (n_k && (!dk || !dv))) return ATTN_ERR_INVALID_ARG;
+    if ((n_q && !aligned16(dq)) || (n_k && (!aligned16(dk) || !aligned16(dv))))
+      return ATTN_ERR_MISALIGNED;
+    if (n_q) fill_zero_u16<<<fill_blocks(n_q), 256, 0, stream>>>(static_cast<uint16_t*>(dq), n_q);
+    if (n_k) {
+      fill_zero_u16<<<fill_blocks(n_k), 256, 0, stream>>>(static_cast<uint16_t*>(dk), n_k);
+      fill_zero_u16<<<fill_blocks(n_k), 256, 0, stream>>>(static_cast<uint16_t*>(dv), n_k);
+    }
+    return finish(stream);
+  }
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return ATTN_ERR_MISALIGNED;
+  st = attn_bwd_prepare(p, o, lse, dout, workspace, workspace_bytes, stream_);
+  if (st != ATTN_OK) return st;
+  st = attn_bwd_accumulate(p, q, k, v, dout, dk, dv, workspace, workspace_bytes, stream_);
+  if (st != ATTN_OK) return st;
+  return attn_bwd_finalize(p, dq, workspace, workspace_bytes, stream_);
+}
+
+attn_status attn_get_device_status(void* stream_, int* code) {
+  if (!code) return ATTN_ERR_INVALID_ARG;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  unsigned int host = 0, zero = 0;
+  if (cudaMemcpyFromSymbolAsync(&host, g_attn_status, sizeof(host), 0, cudaMemcpyDeviceToHost,
+                                stream) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  if (cudaMemcpyToSymbolAsync(g_attn_status, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice,
+                              stream) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return ATTN_ERR_CUDA;
+  *code = static_cast<int>(host);
+  return ATTN_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,348 @@
+// fwd_kernel.cuh - exact attention forward pass for sm_100a.
+//
+// One CTA computes one 128-row query tile of one (batch, head):
+//   O = softmax(Q K^T * scale + mask) V,  LSE = log sum exp(scaled scores)
+// streaming the visible K/V tiles through shared memory.  The method is the
+// tiled, online-softmax attention described on the pages ("FlashAttention ...
+// transformer optimization", items 1-2; FlashAttention-2 page, "Tile-level
+// parallelism" and "shared memory"); the mapping onto B200 is this file's:
+//
+//   warp 4      TMA producer: Q once, then K_j and V_j into a STAGES-deep
+//               ring of shared-memory slots, each guarded by mbarriers.
+//   warp 5      allocates tensor memory; lane 0 issues every tcgen05.mma:
+//               S_j = Q K_j^T into one of two TMEM score buffers, and
+//               O += P_j V_j with P_j read straight from TMEM.
+//   warps 0-3   softmax, one thread per query row (TMEM lane = row): load
+//               S_j, mask, running max in log2 units, exp2, running sum,
+//               P_j as 16-bit values back into the score buffer; rescale O
+//               in TMEM only when the running max grew by more than 8
+//               (log2 units), so P stays below 2^8 and the result is the
+//               same; at the end O/l, LSE, and a TMA store of O.
+//
+// Tensor memory (fp32 columns): S0 [0, BN), S1 [BN, 2BN), O [2BN, 2BN + D).
+// P_j overwrites the first BN/2 columns of its score buffer as packed
+// 16-bit pairs.  MMAs issued by one thread execute in issue order, so S_{j+2}
+// (same buffer) is written only after O += P_j V_j has read P_j.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace attn {
+
+struct FwdParams {
+  float* lse;
+  int batch, nheads, nheads_kv, seqlen_q, seqlen_k;
+  int causal, window_left, window_right;
+  float scale_log2;  // softmax_scale * log2(e)
+  int num_qblocks;
+};
+
+// Range of visible key positions for query rows [q0, q1): keys [jmin, jmax].
+struct KeyRange {
+  long long jmin, jmax;
+};
+
+__device__ __forceinline__ KeyRange visible_keys(int q0, int q1, const FwdParams& p) {
+  const long long off = (long long)p.seqlen_k - p.seqlen_q;
+  const long long kInf = 1ll << 40;
+  const long long rb = p.causal ? 0 : (p.window_right >= 0 ? p.window_right : kInf);
+  const long long lb = p.window_left >= 0 ? p.window_left : kInf;
+  long long jmin = (long long)q0 + off - lb;
+  long long jmax = (long long)(q1 - 1) + off + rb;
+  if (jmin < 0) jmin = 0;
+  if (jmax > (long long)p.seqlen_k - 1) jmax = (long long)p.seqlen_k - 1;
+  return {jmin, jmax};
+}
+
+template <int D_, int BN_, int STAGES_, bool FP16_>
+struct FwdCfg {
+  static constexpr int D = D_, BN = BN_, STAGES = STAGES_;
+  static constexpr bool FP16 = FP16_;
+  static constexpr int BM = 128;
+  static constexpr int NBOX = D / 64;              // 64-column (128-byte) boxes per row
+  static constexpr int Q_BYTES = BM * D * 2;
+  static constexpr int KV_BYTES = BN * D * 2;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + Q_BYTES;
+  static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
+  static constexpr int OFF_BAR = OFF_V + STAGES * KV_BYTES;
+  // barriers
+  static constexpr int B_Q = 0;
+  static constexpr int B_KFULL = 1;
+  static constexpr int B_VFULL = B_KFULL + STAGES;
+  static constexpr int B_EMPTY = B_VFULL + STAGES;
+  static constexpr int B_SFULL = B_EMPTY + STAGES;  // 2
+  static constexpr int B_PREADY = B_SFULL + 2;      // 2
+  static constexpr int B_OREADY = B_PREADY + 2;     // 1
+  static constexpr int NBAR = B_OREADY + 1;
+  static constexpr int OFF_TMEMPTR = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM_BYTES = OFF_TMEMPTR + 16 + 1024;  // + alignment slack
+  static constexpr int TM_S0 = 0, TM_S1 = BN, TM_O = 2 * BN;
+  static constexpr int TMEM_COLS = (2 * BN + D) <= 256 ? 256 : 512;
+  static constexpr int THREADS = 192;
+  static_assert(D % 64 == 0 && D <= 256, "head dim");
+  static_assert(BN % 32 == 0 && BN <= 256, "kv tile");
+  static_assert(2 * BN + D <= 512, "tensor memory");
+  static_assert(SMEM_BYTES <= 232448, "shared memory");
+};
+
+template <class C>
+__global__ void __launch_bounds__(C::THREADS, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                    const FwdParams p) {
+  constexpr int D = C::D, BN = C::BN, BM = C::BM, STAGES = C::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t smem0 = (smem_addr(smem_raw) + 1023u) & ~1023u;
+  uint8_t* smem_gen = smem_raw + (smem0 - smem_addr(smem_raw));
+  auto bar = [&](int i) -> uint32_t { return smem0 + C::OFF_BAR + 8u * i; };
+  volatile uint32_t* tmem_ptr_slot = reinterpret_cast<volatile uint32_t*>(smem_gen + C::OFF_TMEMPTR);
+
+  const uint32_t warp = warp_id(), lane = lane_id();
+  const int qblock = p.num_qblocks - 1 - (int)blockIdx.x;  // heaviest causal tiles first
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int kvh = h / (p.nheads / p.nheads_kv);
+  const int q0 = qblock * BM;
+  const int q1 = min(q0 + BM, p.seqlen_q);
+
+  const KeyRange kr = visible_keys(q0, q1, p);
+  const int t_lo = kr.jmax >= kr.jmin ? (int)(kr.jmin / BN) : 0;
+  const int nt = kr.jmax >= kr.jmin ? (int)(kr.jmax / BN) - t_lo + 1 : 0;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::NBAR; ++i) mbar_init(bar(i), 1);
+    mbar_init(bar(C::B_PREADY + 0), 128);
+    mbar_init(bar(C::B_PREADY + 1), 128);
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(smem0 + C::OFF_TMEMPTR, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 4 && lane == 0) {
+    prefetch_tensormap(&tm_q);
+    prefetch_tensormap(&tm_k);
+    prefetch_tensormap(&tm_v);
+    prefetch_tensormap(&tm_o);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_ptr_slot;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && nt > 0) {
+      mbar_arrive_expect_tx(bar(C::B_Q), C::Q_BYTES);
+      for (int bx = 0; bx < C::NBOX; ++bx)
+        tma_load_4d(smem0 + C::OFF_Q + bx * (BM * 128), &tm_q, bar(C::B_Q), bx * 64, h, q0, b);
+      for (int t = 0; t < nt; ++t) {
+        const int st = t % STAGES, n = t / STAGES;
+        if (n > 0 && !mbar_wait(bar(C::B_EMPTY + st), (n - 1) & 1)) break;
+        const int k0 = (t_lo + t) * BN;
+        mbar_arrive_expect_tx(bar(C::B_KFULL + st), C::KV_BYTES);
+        for (int bx = 0; bx < C::NBOX; ++bx)
+          tma_load_4d(smem0 + C::OFF_K + st * C::KV_BYTES + bx * (BN * 128), &tm_k,
+                      bar(C::B_KFULL + st), bx * 64, kvh, k0, b);
+        mbar_arrive_expect_tx(bar(C::B_VFULL + st), C::KV_BYTES);
+        for (int bx = 0; bx < C::NBOX; ++bx)
+          tma_load_4d(smem0 + C::OFF_V + st * C::KV_BYTES + bx * (BN * 128), &tm_v,
+                      bar(C::B_VFULL + st), bx * 64, kvh, k0, b);
+      }
+      // Loads still in flight must land before the CTA can exit: wait (bounded)
+      // for the last fill of every slot used.
+      for (int t = nt - STAGES < 0 ? 0 : nt - STAGES; t < nt; ++t) {
+        const int st = t % STAGES, n = t / STAGES;
+        if (!mbar_wait(bar(C::B_KFULL + st), n & 1)) break;
+        if (!mbar_wait(bar(C::B_VFULL + st), n & 1)) break;
+      }
+      mbar_wait(bar(C::B_Q), 0);
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && nt > 0) {
+      constexpr uint32_t idesc_qk = idesc_f16(BM, BN, C::FP16, false, false);
+      constexpr uint32_t idesc_pv = idesc_f16(BM, D, C::FP16, false, true);
+      bool ok = mbar_wait(bar(C::B_Q), 0);
+      auto issue_pv = [&](int u) -> bool {
+        const int st = u % STAGES, buf = u & 1;
+        if (!mbar_wait(bar(C::B_PREADY + buf), (u >> 1) & 1)) return false;
+        if (!mbar_wait(bar(C::B_VFULL + st), (u / STAGES) & 1)) return false;
+        tc_fence_after();
+        const uint32_t v_base = smem0 + C::OFF_V + st * C::KV_BYTES;
+        const uint32_t p_tmem = tmem + (buf ? C::TM_S1 : C::TM_S0);
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          // V tile as the MN-major B operand: 16 key rows (2048 B) per step;
+          // 64-column boxes BN*128 bytes apart; 8-row groups 1024 B apart.
+          const uint64_t bdesc = sdesc_sw128(v_base + kk * 2048, BN * 128, 1024);
+          mma_ts(tmem + C::TM_O, p_tmem + kk * 8, bdesc, idesc_pv, (u > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(bar(C::B_OREADY));
+        mma_commit(bar(C::B_EMPTY + st));
+        return true;
+      };
+      for (int t = 0; ok && t < nt; ++t) {
+        const int st = t % STAGES, buf = t & 1;
+        if (!mbar_wait(bar(C::B_KFULL + st), (t / STAGES) & 1)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t q_base = smem0 + C::OFF_Q;
+        const uint32_t k_base = smem0 + C::OFF_K + st * C::KV_BYTES;
+        const uint32_t s_tmem = tmem + (buf ? C::TM_S1 : C::TM_S0);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          // K-major operands: 16 columns = 32 bytes per step inside a
+          // 128-byte swizzled row; next 64-column box at +rows*128 bytes.
+          const int bx = kk / 4, w = kk % 4;
+          const uint64_t adesc = sdesc_sw128(q_base + bx * (BM * 128) + w * 32, 16, 1024);
+          const uint64_t bdesc = sdesc_sw128(k_base + bx * (BN * 128) + w * 32, 16, 1024);
+          mma_ss(s_tmem, adesc, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(bar(C::B_SFULL + buf));
+        if (t >= 1 && !issue_pv(t - 1)) { ok = false; break; }
+      }
+      if (ok) issue_pv(nt - 1);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int r = (int)threadIdx.x;  // row within the tile == TMEM lane
+    const int i = q0 + r;            // query position
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const long long off = (long long)p.seqlen_k - p.seqlen_q;
+    const long long kInf = 1ll << 40;
+    const long long rb = p.causal ? 0 : (p.window_right >= 0 ? p.window_right : kInf);
+    const long long lb = p.window_left >= 0 ? p.window_left : kInf;
+    const long long jhi = (long long)i + off + rb;  // visible keys: [jlo, jhi]
+    const long long jlo = (long long)i + off - lb;
+    const long long blk_hi = (long long)q0 + off + rb;            // every row sees up to here
+    const long long blk_lo = (long long)(q0 + BM - 1) + off - lb;  // every row sees from here
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int t = 0; t < nt; ++t) {
+      const int buf = t & 1;
+      if (!mbar_wait_warp(bar(C::B_SFULL + buf), (t >> 1) & 1)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t s_tmem = tmem + lane_base + (buf ? C::TM_S1 : C::TM_S0);
+      float s[BN];
+#pragma unroll
+      for (int c = 0; c < BN; c += 32) {
+        uint32_t raw[32];
+        tmem_ld32(s_tmem + c, raw);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) s[c + e] = __uint_as_float(raw[e]);
+      }
+      tmem_ld_wait();
+      const long long k0 = (long long)(t_lo + t) * BN;
+      const bool full = (k0 + BN <= p.seqlen_k) && (k0 + BN - 1 <= blk_hi) && (k0 >= blk_lo);
+      if (!full) {
+#pragma unroll
+        for (int c = 0; c < BN; ++c) {
+          const long long j = k0 + c;
+          if (j >= p.seqlen_k || j > jhi || j < jlo) s[c] = -INFINITY;
+        }
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int c = 1; c < BN; ++c) mx = fmaxf(mx, s[c]);
+      const float m_tile = mx * p.scale_log2;  // scale > 0
+      // Keep the old reference max unless the row max grew by more than 8
+      // (log2 units); the first tile always sets it.
+      float m_use = m, alpha = 1.f;
+      if (m_tile > m + 8.f) {
+        m_use = m_tile;
+        alpha = (m == -INFINITY) ? 0.f : ex2(m - m_tile);
+      }
+      const float m_sub = (m_use == -INFINITY) ? 0.f : m_use;
+      float rowsum = 0.f;
+      uint32_t packed[BN / 2];
+#pragma unroll
+      for (int c = 0; c < BN; c += 2) {
+        const float p0 = ex2(fmaf(s[c], p.scale_log2, -m_sub));
+        const float p1 = ex2(fmaf(s[c + 1], p.scale_log2, -m_sub));
+        rowsum += p0 + p1;
+        packed[c / 2] = pack2<C::FP16>(p0, p1);
+      }
+      l = l * alpha + rowsum;
+      m = m_use;
+      // Rescale O (after O += P_{t-1} V_{t-1} has landed) if any row of this
+      // warp changed its reference max.
+      if (t > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        if (!mbar_wait_warp(bar(C::B_OREADY), (t - 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t o_tmem = tmem + lane_base + C::TM_O;
+#pragma unroll 1
+        for (int c = 0; c < D; c += 32) {
+          uint32_t raw[32];
+          tmem_ld32(o_tmem + c, raw);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) raw[e] = __float_as_uint(__uint_as_float(raw[e]) * alpha);
+          tmem_st32(o_tmem + c, raw);
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < BN / 2; c += 16) {
+        uint32_t chunk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) chunk[e] = packed[c + e];
+        tmem_st16(s_tmem + c, chunk);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar(C::B_PREADY + buf));
+    }
+    // ------------------------------------------------------------ epilogue
+    if (ok && nt > 0) ok = mbar_wait_warp(bar(C::B_OREADY), (nt - 1) & 1);
+    if (ok) {
+      tc_fence_after();
+      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      const uint32_t o_tmem = tmem + lane_base + C::TM_O;
+      const uint32_t row_addr = smem0 + C::OFF_Q + r * 128;
+#pragma unroll 1
+      for (int c = 0; c < D; c += 32) {
+        uint32_t raw[32];
+        if (nt > 0) {
+          tmem_ld32(o_tmem + c, raw);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) raw[e] = 0u;
+        }
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          w[e] = pack2<C::FP16>(__uint_as_float(raw[2 * e]) * inv_l,
+                                __uint_as_float(raw[2 * e + 1]) * inv_l);
+        // 32 columns = 64 bytes = four 16-byte chunks of a 128-byte swizzled row.
+        const int bx = c / 64, chunk0 = (c % 64) / 8;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const int chunk = (chunk0 + q4) ^ (r & 7);
+          st_shared_v4(row_addr + bx * (BM * 128) + chunk * 16, w[4 * q4], w[4 * q4 + 1],
+                       w[4 * q4 + 2], w[4 * q4 + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      if (i < p.seqlen_q) {
+        const float lse = l > 0.f ? (m + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
+        p.lse[((size_t)b * p.nheads + h) * p.seqlen_q + i] = lse;
+      }
+    }
+    tc_fence_before();
+    named_bar_sync(1, 128);
+    if (ok && threadIdx.x == 0) {
+      for (int bx = 0; bx < C::NBOX; ++bx)
+        tma_store_4d(&tm_o, smem0 + C::OFF_Q + bx * (BM * 128), bx * 64, h, q0, b);
+      bulk_commit_group();
+      bulk_wait_group_all();
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace attn

@@ -1,0 +1,103 @@
+"""The C ABI without a GPU: the library loads, exports every declared entry
+point, and its pure host functions (argument checks, workspace sizes, status
+strings) behave as include/attn.h states."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "attn.h")
+
+
+@pytest.fixture(scope="module")
+def attn():
+    from io_aware_exact_33_b200 import build
+    build.build()
+    import io_aware_exact_33_b200 as m
+    return m
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"ATTN_API\s+[\w\s\*]+?\b(attn_\w+)\s*\(", text)))
+
+
+def test_header_declares_entry_points():
+    syms = declared_symbols()
+    assert "attn_fwd" in syms and "attn_bwd" in syms
+    assert len(syms) >= 8
+
+
+def test_library_exports_every_declared_symbol(attn):
+    lib = ctypes.CDLL(attn.LIB_PATH)
+    for name in declared_symbols():
+        assert hasattr(lib, name), f"libattn.so does not export {name}"
+    assert set(attn.EXPORTED) <= set(declared_symbols())
+
+
+def test_version_and_status_strings(attn):
+    assert re.match(r"^\d+\.\d+\.\d+$", attn.attn_version())
+    for code in range(0, 9):
+        s = attn.attn_status_string(code)
+        assert s and s != "unknown status"
+    assert attn.attn_status_string(99) == "unknown status"
+
+
+def P(attn, **kw):
+    base = dict(batch=2, seqlen_q=100, seqlen_k=90, nheads=8, nheads_kv=2, headdim=128,
+                dtype=attn.ATTN_BF16, softmax_scale=None, causal=False, window_left=-1,
+                window_right=-1)
+    base.update(kw)
+    return attn.make_params(**base)
+
+
+def test_check_params_accepts_valid(attn):
+    for d in (64, 128, 256):
+        assert attn.attn_check_params(P(attn, headdim=d), 0) == 0
+    for d in (64, 128):
+        assert attn.attn_check_params(P(attn, headdim=d), 1) == 0
+    assert attn.attn_check_params(P(attn, dtype=attn.ATTN_FP16, causal=True, window_left=5,
+                                    window_right=0), 0) == 0
+    assert attn.attn_check_params(P(attn, seqlen_q=0, seqlen_k=0, batch=0), 0) == 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(nheads=6, nheads_kv=4), 1),
+    (dict(nheads_kv=0), 1),
+    (dict(batch=-1), 1),
+    (dict(seqlen_q=-5), 1),
+    (dict(softmax_scale=0.0), 1),
+    (dict(softmax_scale=-1.0), 1),
+    (dict(softmax_scale=float("inf")), 1),
+    (dict(window_left=-2), 1),
+    (dict(window_right=-3), 1),
+    (dict(headdim=96), 2),
+    (dict(headdim=32), 2),
+    (dict(dtype=7), 3),
+])
+def test_check_params_rejects(attn, kw, code):
+    assert attn.attn_check_params(P(attn, **kw), 0) == code
+
+
+def test_bwd_headdim_256_unsupported(attn):
+    assert attn.attn_check_params(P(attn, headdim=256), 1) == 2
+
+
+def test_causal_flag_must_be_boolean(attn):
+    p = P(attn)
+    p.causal = 2
+    assert attn.attn_check_params(p, 0) == 1
+
+
+def test_workspace_sizes(attn):
+    p = P(attn, batch=2, seqlen_q=100, nheads=8, headdim=128)
+    assert attn.attn_fwd_workspace_size(p) == 0
+    ws = attn.attn_bwd_workspace_size(p)
+    nq_pad = 128
+    rows = 2 * 8 * nq_pad * 4
+    acc = 2 * 100 * 8 * 128 * 4
+    assert ws >= 2 * rows + acc
+    assert ws % 256 == 0
+    assert attn.attn_bwd_workspace_size(P(attn, headdim=96)) == 0
