@@ -145,6 +145,36 @@ ATTN_API attn_status attn_bwd_accumulate(const attn_params* p, const void* q, co
 ATTN_API attn_status attn_bwd_finalize(const attn_params* p, void* dq, void* workspace,
                                        size_t workspace_bytes, void* stream);
 
+/*
+ * Backward pass for callers that cannot allocate device memory.
+ *
+ * attn_bwd needs a caller-provided workspace.  Some callers cannot make one
+ * at call time: a host framework that has already claimed the GPU's memory
+ * for its own pool and forbids allocations behind its back, or code on a
+ * latency-critical path where cudaMalloc (which synchronises the device and
+ * can fail) is not acceptable.  This entry point takes the same inputs and
+ * outputs as attn_bwd and allocates nothing: its scratch is a fixed array of
+ * ATTN_NOALLOC_SCRATCH_BYTES in the library's own device memory, which every
+ * GPU that loads libattn.so holds until the process exits.  The paper has no
+ * counterpart to this entry point.
+ *
+ *   - Limit: the call is rejected with ATTN_ERR_WORKSPACE_TOO_SMALL when
+ *     attn_bwd_workspace_size(p) exceeds ATTN_NOALLOC_SCRATCH_BYTES, before
+ *     anything is launched.
+ *   - Set-up: the first call on a device looks up that device's copy of the
+ *     array (cudaGetSymbolAddress, with the device current); make that first
+ *     call before any stream capture.  Later calls reuse the address.
+ *   - Sharing: all calls on a device use the same array, which keeps the last
+ *     call's contents; each call clears what must start at zero.  Calls that
+ *     overlap on the GPU (other streams, other threads) race on the array and
+ *     must be serialised by the caller.
+ */
+#define ATTN_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+ATTN_API attn_status attn_bwd_noalloc(const attn_params* p, const void* q, const void* k,
+                                      const void* v, const void* o, const float* lse,
+                                      const void* dout, void* dq, void* dk, void* dv,
+                                      void* stream);
+
 /* Bytes of device workspace attn_fwd / attn_bwd need for these parameters
  * (0 when none).  Pure host functions; never touch the GPU. */
 ATTN_API size_t attn_fwd_workspace_size(const attn_params* p);

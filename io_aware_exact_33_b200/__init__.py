@@ -261,3 +261,27 @@ def attn_bwd_finalize(p: AttnParams, dq, workspace, stream=None) -> None:
                                 ctypes.c_size_t(workspace.numel()), _stream(stream))
     if st != 0:
         raise AttnError(st, "attn_bwd_finalize")
+
+
+def attn_bwd_noalloc(q, k, v, out, lse, dout, softmax_scale: Optional[float] = None,
+                     causal: bool = False, window_left: int = -1, window_right: int = -1,
+                     dq=None, dk=None, dv=None, stream=None):
+    """Like ``attn_bwd`` but the library uses its own fixed device scratch
+    (ATTN_NOALLOC_SCRATCH_BYTES) instead of a caller workspace, for callers
+    that cannot allocate device memory at call time.  The output tensors are
+    the caller's (allocated here only when not given).  Calls that overlap on
+    the GPU share that scratch and must be serialised by the caller."""
+    import torch
+    fn = _lib.attn_bwd_noalloc
+    vp = ctypes.c_void_p
+    fn.argtypes = [ctypes.POINTER(AttnParams), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    fn.restype = ctypes.c_int
+    p = params_for(q, k, softmax_scale, causal, window_left, window_right)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    st = fn(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq),
+            _ptr(dk), _ptr(dv), _stream(stream))
+    if st != 0:
+        raise AttnError(st, "attn_bwd_noalloc")
+    return dq, dk, dv

@@ -5,6 +5,7 @@
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
+#include <map>
 #include <mutex>
 #include <set>
 #include <utility>
@@ -248,6 +249,33 @@ attn_status bwd_common_checks(const attn_params* p, const void* workspace, size_
 
 }  // namespace
 
+// Scratch of attn_bwd_noalloc: a file-scope device array, so the entry point
+// needs no allocation.  Host code must not pass the symbol itself to a kernel
+// (on the host it names a stand-in, not device memory); each device's address
+// comes from cudaGetSymbolAddress with that device current.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[ATTN_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device; nullptr if the lookup fails.
+void* noalloc_scratch_address() {
+  static std::mutex mu;
+  static std::map<int, void*> addr;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+  std::lock_guard<std::mutex> g(mu);
+  auto it = addr.find(dev);
+  if (it != addr.end()) return it->second;
+  void* ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr)
+    return nullptr;
+  addr[dev] = ptr;
+  return ptr;
+}
+
+}  // namespace
+
 extern "C" {
 
 const char* attn_version(void) { return "0.1.0"; }
@@ -404,6 +432,23 @@ attn_status attn_bwd(const attn_params* p, const void* q, const void* k, const v
   st = attn_bwd_accumulate(p, q, k, v, dout, dk, dv, workspace, workspace_bytes, stream_);
   if (st != ATTN_OK) return st;
   return attn_bwd_finalize(p, dq, workspace, workspace_bytes, stream_);
+}
+
+attn_status attn_bwd_noalloc(const attn_params* p, const void* q, const void* k, const void* v,
+                             const void* o, const float* lse, const void* dout, void* dq, void* dk,
+                             void* dv, void* stream_) {
+  attn_status st = attn_check_params(p, 1);
+  if (st != ATTN_OK) return st;
+  if (p->batch == 0 || p->seqlen_q == 0 || p->seqlen_k == 0)  // no scratch needed
+    return attn_bwd(p, q, k, v, o, lse, dout, dq, dk, dv, nullptr, 0, stream_);
+  if (attn_bwd_workspace_size(p) > (size_t)ATTN_NOALLOC_SCRATCH_BYTES)
+    return ATTN_ERR_WORKSPACE_TOO_SMALL;
+  void* scratch = noalloc_scratch_address();
+  if (!scratch) return ATTN_ERR_CUDA;
+  // attn_bwd's first stage rewrites the row statistics and zeroes the dQ
+  // accumulator, so the previous call's contents never leak into this one.
+  return attn_bwd(p, q, k, v, o, lse, dout, dq, dk, dv, scratch, ATTN_NOALLOC_SCRATCH_BYTES,
+                  stream_);
 }
 
 attn_status attn_get_device_status(void* stream_, int* code) {
