@@ -1,0 +1,100 @@
+"""bench.py host logic on the CPU: FLOP accounting, the exact visible-pair
+count, clock-sample parsing, and the multi-rank path (world size 2, gloo):
+barrier and the maximum over ranks that the timing uses."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+import bench
+from attn_inputs import WORKLOADS
+from oracle_pins import mask_matrix
+
+
+def test_step_flops_formula():
+    w = WORKLOADS["causal_b2_h32_n8192_d128"]
+    fwd, bwd = bench.step_flops(w)
+    assert fwd == 4 * 2 * 32 * 8192 * 8192 * 128 / 2
+    assert bwd == 2.5 * fwd
+    w2 = WORKLOADS["full_b1_h16_n16384_d128"]
+    assert bench.step_flops(w2)[0] == 4 * 16 * 16384 ** 2 * 128
+
+
+@pytest.mark.parametrize("nq,nk,causal,wl,wr", [
+    (7, 7, True, -1, -1), (9, 5, True, 2, -1), (5, 9, False, 1, 3), (8, 8, False, -1, 0),
+    (6, 6, False, 0, 0), (10, 4, True, -1, -1),
+])
+def test_visible_pairs_matches_brute_force(nq, nk, causal, wl, wr):
+    vis = mask_matrix(nq, nk, causal=causal, window_left=wl, window_right=wr)
+    assert bench.visible_pairs(nq, nk, causal, wl, wr) == int(vis.sum())
+    rows = [0, nq - 1]
+    assert bench.visible_pairs(nq, nk, causal, wl, wr, rows=rows) == int(vis[rows].sum())
+
+
+def test_window_workload_pair_count():
+    w = WORKLOADS["gqa_window_b4_h32_kv8_n4096_d128"]
+    # min(i, 1024) + 1 keys per query
+    assert bench.visible_pairs(w.seqlen_q, w.seqlen_k, w.causal, w.window_left, w.window_right) == \
+        sum(min(i, 1024) + 1 for i in range(4096)) == 3673600
+
+
+def test_clock_summary_parsing():
+    c = bench.ClockSampler(0)
+    c.lines = [
+        "1965, 1965, 700.1, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "1800, 1965, 990.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "1320, 1965, 1001.2, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+    ]
+    s = c.summary()
+    assert s["sm_mhz"] == 1800 and s["sm_max_mhz"] == 1965
+    assert s["reasons"] == ["sw_power_cap"] and s["samples"] == 3
+
+
+def test_peaks_loaded_or_fallback():
+    peaks, kind = bench.load_peaks()
+    assert kind in ("measured", "fallback")
+    assert peaks["bf16_tflops"] > 1000 and peaks["hbm_gbs"] > 1000
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _rank_main(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      LOCAL_RANK=str(rank), WORLD_SIZE=str(world))
+    r, lr, ws = bench.world_info()
+    dist = bench.init_dist("gloo", ws)
+    bench.barrier(dist)
+    # each rank "measured" a different time; the job time is the slowest rank's
+    got = bench.max_over_ranks(10.0 + 5.0 * r, dist)
+    bench.barrier(dist)
+    q.put((r, lr, ws, got))
+    dist.destroy_process_group()
+
+
+def test_two_ranks_gloo_max_over_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(2))
+    assert [r[0] for r in res] == [0, 1]
+    assert all(r[2] == 2 for r in res)
+    assert all(r[3] == 15.0 for r in res)
+
+
+def test_single_rank_is_identity():
+    assert bench.max_over_ranks(3.5, None) == 3.5
