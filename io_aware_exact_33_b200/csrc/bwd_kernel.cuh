@@ -18,16 +18,22 @@
 //
 // Main kernel roles (320 threads):
 //   warp 8      TMA producer: K_j, V_j once; Q_i, dO_i, LSE2_i, Dvec_i per
-//               query tile through a two-slot ring.
+//               query tile through a three-slot ring.
 //   warp 9      TMEM allocation; lane 0 issues the five MMAs per tile:
 //               S^T = K Q^T, dP^T = V dO^T, dV += P^T dO, dK += dS^T Q, and
-//               dQ^T = K^T dS^T (d = 128) or dQ = dS K (d = 64).
-//   warps 0-3   one thread per key row (TMEM lane): P^T = exp2(S^T*scale*log2e
-//               - LSE2), dS^T = P^T o (dP^T - Dvec); P^T and dS^T go back to
-//               TMEM as 16-bit operands, dS also to shared memory (the dQ MMA
-//               needs it with the other operand order); finally dK, dV out.
-//   warps 4-7   read the dQ tile out of TMEM and add it into the fp32
-//               accumulator with global atomics (other key tiles add too).
+//               dQ^T = K^T dS^T (d = 128) or dQ = dS K (d = 64).  With two
+//               buffers it issues tile t+1's S^T and dP^T before tile t's
+//               gradient MMAs, so the tensor pipe works on one tile while
+//               warps 0-3 exponentiate the other.
+//   warps 0-7   two warps per tensor-memory lane quadrant (one thread per key
+//               row), each owning half of the tile's query columns:
+//               P^T = exp2(S^T*scale*log2e - LSE2) back into tensor memory as
+//               the 16-bit A operand of dV; dS = P o (dP - Dvec) into shared
+//               memory, where it is the K-major A operand of dK and an
+//               MN-major operand of dQ; then the previous tile's dQ block
+//               (which reuses that tile's dP block) out of tensor memory into
+//               the fp32 accumulator with global atomics (other key tiles add
+//               to the same rows); finally dK, dV out through TMA.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -141,46 +147,58 @@ __global__ void __launch_bounds__(256) bwd_convert(const float* __restrict__ acc
 }
 
 // ------------------------------------------------------------ main kernel
+// Tile sizes: BN = 128 key rows per CTA (the tensor-memory lane count);
+// BM query rows per step.  d = 128: BM = 64 with two tensor-memory buffers
+// for S/P and dP/dQ, so the MMAs of one query tile overlap the exponentials
+// of the next.  d = 64: BM = 128 and one buffer (the dQ MMA would otherwise
+// need M = 64).
 template <int D_, bool FP16_>
 struct BwdCfg {
   static constexpr int D = D_;
   static constexpr bool FP16 = FP16_;
-  static constexpr int BN = 128;                 // key rows per CTA (TMEM lanes)
-  static constexpr int BM = (D == 128) ? 64 : 128;  // query rows per step
-  static constexpr bool DQT = (D == 128);        // dQ^T = K^T dS^T, else dQ = dS K
+  static constexpr int BN = 128;
+  static constexpr int BM = (D == 128) ? 64 : 128;
+  static constexpr int NBUF = (D == 128) ? 2 : 1;
+  static constexpr bool DQT = (D == 128);  // dQ^T = K^T dS^T (M = d), else dQ = dS K (M = BM)
+  static constexpr int QSTAGES = 3;
   static constexpr int NBOX = D / 64;
   static constexpr int NQB = BM / 64;
+  static constexpr int HW = BM / 2;  // query columns per compute warp
+  static constexpr int DQW = DQT ? BM : D;  // columns of a dQ block in tensor memory
   static constexpr int KV_BYTES = BN * D * 2;
   static constexpr int Q_BYTES = BM * D * 2;
   static constexpr int DS_BYTES = BN * BM * 2;
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + KV_BYTES;
-  static constexpr int OFF_Q = OFF_V + KV_BYTES;      // 2 slots
-  static constexpr int OFF_DO = OFF_Q + 2 * Q_BYTES;  // 2 slots
-  static constexpr int OFF_DS = OFF_DO + 2 * Q_BYTES;
-  static constexpr int OFF_LSE = OFF_DS + DS_BYTES;   // 2 slots x BM fp32
-  static constexpr int OFF_DVEC = OFF_LSE + 2 * BM * 4;
-  static constexpr int OFF_BAR = OFF_DVEC + 2 * BM * 4;
+  static constexpr int OFF_Q = OFF_V + KV_BYTES;
+  static constexpr int OFF_DO = OFF_Q + QSTAGES * Q_BYTES;
+  static constexpr int OFF_DS = OFF_DO + QSTAGES * Q_BYTES;
+  static constexpr int OFF_LSE = OFF_DS + NBUF * DS_BYTES;
+  static constexpr int OFF_DVEC = OFF_LSE + QSTAGES * BM * 4;
+  static constexpr int OFF_BAR = OFF_DVEC + QSTAGES * BM * 4;
+  // barriers
   static constexpr int B_KV = 0;
-  static constexpr int B_QFULL = 1;     // 2
-  static constexpr int B_DOFULL = 3;    // 2
-  static constexpr int B_EMPTY = 5;     // 2
-  static constexpr int B_SFULL = 7;
-  static constexpr int B_DPFULL = 8;
-  static constexpr int B_PREADY = 9;    // 128 arrivals
-  static constexpr int B_DSREADY = 10;  // 128 arrivals
-  static constexpr int B_DSFREE = 11;
-  static constexpr int B_DQFULL = 12;
-  static constexpr int B_DQFREE = 13;   // 128 arrivals
-  static constexpr int B_DONE = 14;
-  static constexpr int NBAR = 15;
+  static constexpr int B_QFULL = 1;
+  static constexpr int B_DOFULL = B_QFULL + QSTAGES;
+  static constexpr int B_EMPTY = B_DOFULL + QSTAGES;
+  static constexpr int B_SFULL = B_EMPTY + QSTAGES;   // per buffer
+  static constexpr int B_DPFULL = B_SFULL + NBUF;
+  static constexpr int B_PREADY = B_DPFULL + NBUF;    // 256 arrivals
+  static constexpr int B_DSREADY = B_PREADY + NBUF;   // 256 arrivals
+  static constexpr int B_DSFREE = B_DSREADY + NBUF;
+  static constexpr int B_DQFULL = B_DSFREE + NBUF;
+  static constexpr int B_DQFREE = B_DQFULL + NBUF;    // 256 arrivals
+  static constexpr int B_DONE = B_DQFREE + NBUF;
+  static constexpr int NBAR = B_DONE + 1;
   static constexpr int OFF_TMEMPTR = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_TMEMPTR + 16 + 1024;
-  static constexpr int TM_DV = 0, TM_DK = D, TM_S = 2 * D, TM_DP = 2 * D + BM, TM_DQ = 2 * D + 2 * BM;
+  // tensor memory: dV, dK accumulators; per buffer an S/P block and a dP/dQ block
+  static constexpr int TM_DV = 0, TM_DK = D, TM_S = 2 * D, TM_DP = 2 * D + NBUF * BM;
   static constexpr int TMEM_COLS = 512;
   static constexpr int THREADS = 320;
-  static_assert(TM_DQ + (DQT ? BM : D) <= TMEM_COLS, "tensor memory");
-  static_assert(2 * Q_BYTES >= BN * D * 2, "epilogue staging");
+  static_assert(TM_DP + NBUF * BM <= TMEM_COLS, "tensor memory");
+  static_assert(DQT || D <= BM, "dQ block fits its dP block");
+  static_assert(QSTAGES * Q_BYTES >= BN * D * 2, "epilogue staging");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
 
@@ -191,14 +209,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     const __grid_constant__ CUtensorMap tm_lse2, const __grid_constant__ CUtensorMap tm_dvec,
                     const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
                     const BwdParams p) {
-  constexpr int D = C::D, BN = C::BN, BM = C::BM;
+  constexpr int D = C::D, BN = C::BN, BM = C::BM, NBUF = C::NBUF, QS = C::QSTAGES;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t smem0 = (smem_addr(smem_raw) + 1023u) & ~1023u;
   uint8_t* smem_gen = smem_raw + (smem0 - smem_addr(smem_raw));
   auto bar = [&](int i) -> uint32_t { return smem0 + C::OFF_BAR + 8u * i; };
   volatile uint32_t* tmem_ptr_slot = reinterpret_cast<volatile uint32_t*>(smem_gen + C::OFF_TMEMPTR);
-  const float* lse_s = reinterpret_cast<const float*>(smem_gen + C::OFF_LSE);
-  const float* dvec_s = reinterpret_cast<const float*>(smem_gen + C::OFF_DVEC);
 
   const uint32_t warp = warp_id(), lane = lane_id();
   const int kblock = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
@@ -221,8 +237,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NBAR; ++i) {
-      const bool many = i == C::B_PREADY || i == C::B_DSREADY || i == C::B_DQFREE;
-      mbar_init(bar(i), many ? 128 : 1);
+      const bool many = (i >= C::B_PREADY && i < C::B_DSREADY + NBUF) ||
+                        (i >= C::B_DQFREE && i < C::B_DQFREE + NBUF);
+      mbar_init(bar(i), many ? 256 : 1);
     }
     fence_barrier_init();
   }
@@ -244,26 +261,26 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         tma_load_4d(smem0 + C::OFF_V + bx * (BN * 128), &tm_v, bar(C::B_KV), bx * 64, kvh, k0, b);
       }
       for (int t = 0; t < nt; ++t) {
-        const int st = t & 1, n = t >> 1;
-        if (n > 0 && !mbar_wait(bar(C::B_EMPTY + st), (n - 1) & 1)) break;
+        const int slot = t % QS, n = t / QS;
+        if (n > 0 && !mbar_wait(bar(C::B_EMPTY + slot), (n - 1) & 1)) break;
         const int h = kvh * group + t / nqb;
         const int q0 = (qb_lo + t % nqb) * BM;
-        const int row = (b * p.nheads + h);
-        mbar_arrive_expect_tx(bar(C::B_QFULL + st), C::Q_BYTES + BM * 4);
+        const int row = b * p.nheads + h;
+        mbar_arrive_expect_tx(bar(C::B_QFULL + slot), C::Q_BYTES + BM * 4);
         for (int bx = 0; bx < C::NBOX; ++bx)
-          tma_load_4d(smem0 + C::OFF_Q + st * C::Q_BYTES + bx * (BM * 128), &tm_q,
-                      bar(C::B_QFULL + st), bx * 64, h, q0, b);
-        tma_load_2d(smem0 + C::OFF_LSE + st * BM * 4, &tm_lse2, bar(C::B_QFULL + st), q0, row);
-        mbar_arrive_expect_tx(bar(C::B_DOFULL + st), C::Q_BYTES + BM * 4);
+          tma_load_4d(smem0 + C::OFF_Q + slot * C::Q_BYTES + bx * (BM * 128), &tm_q,
+                      bar(C::B_QFULL + slot), bx * 64, h, q0, b);
+        tma_load_2d(smem0 + C::OFF_LSE + slot * BM * 4, &tm_lse2, bar(C::B_QFULL + slot), q0, row);
+        mbar_arrive_expect_tx(bar(C::B_DOFULL + slot), C::Q_BYTES + BM * 4);
         for (int bx = 0; bx < C::NBOX; ++bx)
-          tma_load_4d(smem0 + C::OFF_DO + st * C::Q_BYTES + bx * (BM * 128), &tm_do,
-                      bar(C::B_DOFULL + st), bx * 64, h, q0, b);
-        tma_load_2d(smem0 + C::OFF_DVEC + st * BM * 4, &tm_dvec, bar(C::B_DOFULL + st), q0, row);
+          tma_load_4d(smem0 + C::OFF_DO + slot * C::Q_BYTES + bx * (BM * 128), &tm_do,
+                      bar(C::B_DOFULL + slot), bx * 64, h, q0, b);
+        tma_load_2d(smem0 + C::OFF_DVEC + slot * BM * 4, &tm_dvec, bar(C::B_DOFULL + slot), q0, row);
       }
-      for (int t = nt - 2 < 0 ? 0 : nt - 2; t < nt; ++t) {
-        const int st = t & 1, n = t >> 1;
-        if (!mbar_wait(bar(C::B_QFULL + st), n & 1)) break;
-        if (!mbar_wait(bar(C::B_DOFULL + st), n & 1)) break;
+      for (int t = nt - QS < 0 ? 0 : nt - QS; t < nt; ++t) {
+        const int slot = t % QS, n = t / QS;
+        if (!mbar_wait(bar(C::B_QFULL + slot), n & 1)) break;
+        if (!mbar_wait(bar(C::B_DOFULL + slot), n & 1)) break;
       }
       mbar_wait(bar(C::B_KV), 0);
     }
@@ -275,160 +292,239 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       constexpr uint32_t idesc_dq =
           C::DQT ? idesc_f16(D, BM, C::FP16, true, true) : idesc_f16(BM, D, C::FP16, true, true);
       const uint32_t k_base = smem0 + C::OFF_K, v_base = smem0 + C::OFF_V;
-      const uint32_t ds_base = smem0 + C::OFF_DS;
-      bool ok = mbar_wait(bar(C::B_KV), 0);
-      for (int t = 0; ok && t < nt; ++t) {
-        const int st = t & 1, ph = (t >> 1) & 1;
-        const uint32_t q_base = smem0 + C::OFF_Q + st * C::Q_BYTES;
-        const uint32_t do_base = smem0 + C::OFF_DO + st * C::Q_BYTES;
-        if (!mbar_wait(bar(C::B_QFULL + st), ph)) { ok = false; break; }
+      // S^T_u = K Q_u^T into the S block of buffer u % NBUF.
+      auto issue_s = [&](int u) -> bool {
+        const int slot = u % QS, bf = u % NBUF;
+        const uint32_t q_base = smem0 + C::OFF_Q + slot * C::Q_BYTES;
+        if (!mbar_wait(bar(C::B_QFULL + slot), (u / QS) & 1)) return false;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {  // S^T = K Q^T
+        for (int kk = 0; kk < D / 16; ++kk) {
           const int bx = kk / 4, w = kk % 4;
-          mma_ss(tmem + C::TM_S, sdesc_sw128(k_base + bx * (BN * 128) + w * 32, 16, 1024),
+          mma_ss(tmem + C::TM_S + bf * BM, sdesc_sw128(k_base + bx * (BN * 128) + w * 32, 16, 1024),
                  sdesc_sw128(q_base + bx * (BM * 128) + w * 32, 16, 1024), idesc_s, kk > 0);
         }
-        mma_commit(bar(C::B_SFULL));
-        if (!mbar_wait(bar(C::B_DOFULL + st), ph)) { ok = false; break; }
+        mma_commit(bar(C::B_SFULL + bf));
+        return true;
+      };
+      // dP^T_u = V dO_u^T into the dP block, once tile u - NBUF's dQ left it.
+      auto issue_dp = [&](int u) -> bool {
+        const int slot = u % QS, bf = u % NBUF, use = u / NBUF;
+        const uint32_t do_base = smem0 + C::OFF_DO + slot * C::Q_BYTES;
+        if (use > 0 && !mbar_wait(bar(C::B_DQFREE + bf), (use - 1) & 1)) return false;
+        if (!mbar_wait(bar(C::B_DOFULL + slot), (u / QS) & 1)) return false;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {  // dP^T = V dO^T
+        for (int kk = 0; kk < D / 16; ++kk) {
           const int bx = kk / 4, w = kk % 4;
-          mma_ss(tmem + C::TM_DP, sdesc_sw128(v_base + bx * (BN * 128) + w * 32, 16, 1024),
+          mma_ss(tmem + C::TM_DP + bf * BM, sdesc_sw128(v_base + bx * (BN * 128) + w * 32, 16, 1024),
                  sdesc_sw128(do_base + bx * (BM * 128) + w * 32, 16, 1024), idesc_s, kk > 0);
         }
-        mma_commit(bar(C::B_DPFULL));
-        if (!mbar_wait(bar(C::B_PREADY), t & 1)) { ok = false; break; }
+        mma_commit(bar(C::B_DPFULL + bf));
+        return true;
+      };
+      // dV += P^T dO, dK += dS^T Q and tile t's dQ share.
+      auto issue_grads = [&](int t) -> bool {
+        const int slot = t % QS, bf = t % NBUF, use = t / NBUF;
+        const uint32_t q_base = smem0 + C::OFF_Q + slot * C::Q_BYTES;
+        const uint32_t do_base = smem0 + C::OFF_DO + slot * C::Q_BYTES;
+        const uint32_t ds_base = smem0 + C::OFF_DS + bf * C::DS_BYTES;
+        if (!mbar_wait(bar(C::B_PREADY + bf), use & 1)) return false;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < BM / 16; ++kk)  // dV += P^T dO
-          mma_ts(tmem + C::TM_DV, tmem + C::TM_S + kk * 8,
+        for (int kk = 0; kk < BM / 16; ++kk) {
+          // P^T from tensor memory: each half of the query columns keeps its
+          // packed values at the start of its own score columns.
+          const int half = kk / (C::HW / 16), part = kk % (C::HW / 16);
+          mma_ts(tmem + C::TM_DV, tmem + C::TM_S + bf * BM + half * C::HW + part * 8,
                  sdesc_sw128(do_base + kk * 2048, BM * 128, 1024), idesc_acc, (t > 0 || kk > 0));
-        if (!mbar_wait(bar(C::B_DSREADY), t & 1)) { ok = false; break; }
+        }
+        if (!mbar_wait(bar(C::B_DSREADY + bf), use & 1)) return false;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < BM / 16; ++kk)  // dK += dS^T Q
-          mma_ts(tmem + C::TM_DK, tmem + C::TM_DP + kk * 8,
+        for (int kk = 0; kk < BM / 16; ++kk) {  // dS^T as a K-major smem operand; Q MN-major
+          const int bx = kk / 4, w = kk % 4;
+          mma_ss(tmem + C::TM_DK, sdesc_sw128(ds_base + bx * (BN * 128) + w * 32, 16, 1024),
                  sdesc_sw128(q_base + kk * 2048, BM * 128, 1024), idesc_acc, (t > 0 || kk > 0));
-        if (t > 0 && !mbar_wait(bar(C::B_DQFREE), (t - 1) & 1)) { ok = false; break; }
-        tc_fence_after();
+        }
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
           if constexpr (C::DQT)  // dQ^T = K^T dS^T: both operands MN-major
-            mma_ss(tmem + C::TM_DQ, sdesc_sw128(k_base + kk * 2048, BN * 128, 1024),
+            mma_ss(tmem + C::TM_DP + bf * BM, sdesc_sw128(k_base + kk * 2048, BN * 128, 1024),
                    sdesc_sw128(ds_base + kk * 2048, BN * 128, 1024), idesc_dq, kk > 0);
           else  // dQ = dS K
-            mma_ss(tmem + C::TM_DQ, sdesc_sw128(ds_base + kk * 2048, BN * 128, 1024),
+            mma_ss(tmem + C::TM_DP + bf * BM, sdesc_sw128(ds_base + kk * 2048, BN * 128, 1024),
                    sdesc_sw128(k_base + kk * 2048, BN * 128, 1024), idesc_dq, kk > 0);
         }
-        mma_commit(bar(C::B_DQFULL));
-        mma_commit(bar(C::B_DSFREE));
-        mma_commit(bar(C::B_EMPTY + st));
+        mma_commit(bar(C::B_DQFULL + bf));
+        mma_commit(bar(C::B_DSFREE + bf));
+        mma_commit(bar(C::B_EMPTY + slot));
+        return true;
+      };
+      // Two buffers: S^T_{t+1} goes in before tile t's gradient MMAs, dP^T_{t+1}
+      // after them (its block holds tile t-1's dQ until that is read out).
+      // One buffer: everything of tile t first.
+      bool ok = mbar_wait(bar(C::B_KV), 0) && issue_s(0) && issue_dp(0);
+      for (int t = 0; ok && t < nt; ++t) {
+        const bool more = t + 1 < nt;
+        if (NBUF == 2 && more && !issue_s(t + 1)) { ok = false; break; }
+        if (!issue_grads(t)) { ok = false; break; }
+        if (NBUF == 1 && more && !issue_s(t + 1)) { ok = false; break; }
+        if (more && !issue_dp(t + 1)) { ok = false; break; }
       }
       if (ok) mma_commit(bar(C::B_DONE));
     }
-  } else if (warp < 4) {
-    // ------------------------------------------------------------ P / dS
-    const int r = (int)threadIdx.x;  // key row within the tile == TMEM lane
+  } else if (warp < 8) {
+    // ------------------------------------------------------------ P, dS, dQ out
+    // Warp w: tensor-memory lane quadrant w % 4 (key rows), query-column half
+    // w / 4 (HW columns).
+    const int quad = (int)(warp & 3), half = (int)(warp >> 2);
+    const int r = quad * 32 + (int)lane;  // key row within the tile == TMEM lane
+    const int c0 = half * C::HW;          // first query column of this warp
     const long long j = (long long)k0 + r;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+    // dQ of tile u: read this warp's part out of tensor memory, release the
+    // block, and add it into the fp32 accumulator.
+    auto drain_dq = [&](int u) -> bool {
+      const int bf = u % NBUF;
+      if (!mbar_wait_warp(bar(C::B_DQFULL + bf), (u / NBUF) & 1)) return false;
+      tc_fence_after();
+      const int h = kvh * group + u / nqb;
+      const int q0 = (qb_lo + u % nqb) * BM;
+      constexpr int W = C::DQW / 2;  // this warp's columns of the dQ block
+      const int d0 = half * W;
+      uint32_t raw[W];
+#pragma unroll
+      for (int c = 0; c < W; c += 32) {
+        uint32_t part[32];
+        tmem_ld32(tmem + lane_base + C::TM_DP + bf * BM + d0 + c, part);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) raw[c + e] = part[e];
+      }
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(bar(C::B_DQFREE + bf));
+      if constexpr (C::DQT) {
+        // lane = head-dim column r; columns = query rows q0 + d0 + c
+        const size_t row_stride = (size_t)p.nheads * D;
+        float* dst = p.dq_acc + (((size_t)b * p.seqlen_q + q0 + d0) * p.nheads + h) * D + r;
+        const int nvalid = min(W, p.seqlen_q - q0 - d0);
+#pragma unroll
+        for (int c = 0; c < W; ++c)
+          if (c < nvalid) atomicAdd(dst + c * row_stride, __uint_as_float(raw[c]));
+      } else {
+        // lane = query row q0 + r; columns = head-dim d0 + c
+        if (q0 + r < p.seqlen_q) {
+          float4* dst = reinterpret_cast<float4*>(
+              p.dq_acc + (((size_t)b * p.seqlen_q + q0 + r) * p.nheads + h) * D + d0);
+#pragma unroll
+          for (int c = 0; c < W / 4; ++c)
+            atomicAdd(dst + c, make_float4(__uint_as_float(raw[4 * c]), __uint_as_float(raw[4 * c + 1]),
+                                           __uint_as_float(raw[4 * c + 2]), __uint_as_float(raw[4 * c + 3])));
+        }
+      }
+      return true;
+    };
     bool ok = true;
     for (int t = 0; t < nt; ++t) {
-      const int st = t & 1, ph = (t >> 1) & 1;
+      const int slot = t % QS, ph = (t / QS) & 1, bf = t % NBUF, use = t / NBUF;
       const int q0 = (qb_lo + t % nqb) * BM;
-      if (!mbar_wait_warp(bar(C::B_SFULL), t & 1)) { ok = false; break; }
-      if (!mbar_wait_warp(bar(C::B_QFULL + st), ph)) { ok = false; break; }
+      if (!mbar_wait_warp(bar(C::B_SFULL + bf), use & 1)) { ok = false; break; }
+      if (!mbar_wait_warp(bar(C::B_QFULL + slot), ph)) { ok = false; break; }
       tc_fence_after();
-      float pr[BM];
+      const uint32_t s_tmem = tmem + lane_base + C::TM_S + bf * BM + c0;
+      float pr[C::HW];
 #pragma unroll
-      for (int c = 0; c < BM; c += 32) {
+      for (int c = 0; c < C::HW; c += 32) {
         uint32_t raw[32];
-        tmem_ld32(tmem + lane_base + C::TM_S + c, raw);
+        tmem_ld32(s_tmem + c, raw);
 #pragma unroll
         for (int e = 0; e < 32; ++e) pr[c + e] = __uint_as_float(raw[e]);
       }
       tmem_ld_wait();
-      const float* lse_t = lse_s + st * BM;
-      // Whole tile visible (query rows past seqlen_q have LSE2 = +inf, so P = 0).
+      // Whole half visible (query rows past seqlen_q have LSE2 = +inf: P = 0).
+      const int qa = q0 + c0;
       const bool full = ((long long)k0 + BN <= p.seqlen_k) &&
-                        ((long long)k0 + BN - 1 <= (long long)q0 + off + rb) &&
-                        ((long long)k0 >= (long long)(q0 + BM - 1) + off - lb);
+                        ((long long)k0 + BN - 1 <= (long long)qa + off + rb) &&
+                        ((long long)k0 >= (long long)(qa + C::HW - 1) + off - lb);
+      const uint32_t lse_addr = smem0 + C::OFF_LSE + (slot * BM + c0) * 4;
 #pragma unroll
-      for (int c = 0; c < BM; ++c) {
-        float v = ex2(fmaf(pr[c], p.scale_log2, -lse_t[c]));
-        if (!full) {
-          const long long i = (long long)q0 + c;
-          if (j >= p.seqlen_k || j > i + off + rb || j < i + off - lb) v = 0.f;
-        }
-        pr[c] = v;
+      for (int c = 0; c < C::HW; c += 4) {
+        float l4[4];
+        ld_shared_v4f(lse_addr + c * 4, l4);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) pr[c + e] = ex2(fmaf(pr[c + e], p.scale_log2, -l4[e]));
       }
-      {
-        uint32_t w[BM / 2];
+      if (!full) {
 #pragma unroll
-        for (int c = 0; c < BM; c += 2) w[c / 2] = pack2<C::FP16>(pr[c], pr[c + 1]);
-#pragma unroll
-        for (int c = 0; c < BM / 2; c += 16) {
-          uint32_t chunk[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) chunk[e] = w[c + e];
-          tmem_st16(tmem + lane_base + C::TM_S + c, chunk);
+        for (int c = 0; c < C::HW; ++c) {
+          const long long i = (long long)qa + c;
+          if (j >= p.seqlen_k || j > i + off + rb || j < i + off - lb) pr[c] = 0.f;
         }
+      }
+#pragma unroll
+      for (int c = 0; c < C::HW; c += 32) {
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) w[e] = pack2<C::FP16>(pr[c + 2 * e], pr[c + 2 * e + 1]);
+        tmem_st16(s_tmem + c / 2, w);
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(bar(C::B_PREADY));
-      if (!mbar_wait_warp(bar(C::B_DPFULL), t & 1)) { ok = false; break; }
-      if (!mbar_wait_warp(bar(C::B_DOFULL + st), ph)) { ok = false; break; }
+      mbar_arrive(bar(C::B_PREADY + bf));
+      if (!mbar_wait_warp(bar(C::B_DPFULL + bf), use & 1)) { ok = false; break; }
+      if (!mbar_wait_warp(bar(C::B_DOFULL + slot), ph)) { ok = false; break; }
       tc_fence_after();
-      const float* dvec_t = dvec_s + st * BM;
+      const uint32_t dvec_addr = smem0 + C::OFF_DVEC + (slot * BM + c0) * 4;
 #pragma unroll
-      for (int c = 0; c < BM; c += 32) {
+      for (int c = 0; c < C::HW; c += 32) {
         uint32_t raw[32];
-        tmem_ld32(tmem + lane_base + C::TM_DP + c, raw);
+        tmem_ld32(tmem + lane_base + C::TM_DP + bf * BM + c0 + c, raw);
         tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) pr[c + e] = pr[c + e] * (__uint_as_float(raw[e]) - dvec_t[c + e]);
+        for (int e = 0; e < 32; e += 4) {
+          float d4[4];
+          ld_shared_v4f(dvec_addr + (c + e) * 4, d4);
+#pragma unroll
+          for (int f = 0; f < 4; ++f)
+            pr[c + e + f] = pr[c + e + f] * (__uint_as_float(raw[e + f]) - d4[f]);
+        }
       }
-      // dS smem tile is free once the previous tile's dQ MMA has read it.
-      if (t > 0 && !mbar_wait_warp(bar(C::B_DSFREE), (t - 1) & 1)) { ok = false; break; }
+      // dS smem buffer is free once tile t - NBUF's dK and dQ MMAs have read it.
+      if (use > 0 && !mbar_wait_warp(bar(C::B_DSFREE + bf), (use - 1) & 1)) { ok = false; break; }
       {
-        uint32_t w[BM / 2];
-#pragma unroll
-        for (int c = 0; c < BM; c += 2) w[c / 2] = pack2<C::FP16>(pr[c], pr[c + 1]);
-#pragma unroll
-        for (int c = 0; c < BM / 2; c += 16) {
-          uint32_t chunk[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) chunk[e] = w[c + e];
-          tmem_st16(tmem + lane_base + C::TM_DP + c, chunk);
-        }
         // dS as [key row][query] with 128-byte swizzle, 64 queries per box.
-        const uint32_t row_addr = smem0 + C::OFF_DS + r * 128;
+        const uint32_t row_addr = smem0 + C::OFF_DS + bf * C::DS_BYTES + r * 128;
 #pragma unroll
-        for (int c8 = 0; c8 < BM / 8; ++c8) {
-          const int bx = c8 / 8, chunk = (c8 % 8) ^ (r & 7);
-          st_shared_v4(row_addr + bx * (BN * 128) + chunk * 16, w[4 * c8], w[4 * c8 + 1],
-                       w[4 * c8 + 2], w[4 * c8 + 3]);
+        for (int c8 = 0; c8 < C::HW / 8; ++c8) {
+          const int col = c0 + c8 * 8;
+          const int bx = col / 64, chunk = ((col % 64) / 8) ^ (r & 7);
+          st_shared_v4(row_addr + bx * (BN * 128) + chunk * 16,
+                       pack2<C::FP16>(pr[8 * c8], pr[8 * c8 + 1]), pack2<C::FP16>(pr[8 * c8 + 2], pr[8 * c8 + 3]),
+                       pack2<C::FP16>(pr[8 * c8 + 4], pr[8 * c8 + 5]), pack2<C::FP16>(pr[8 * c8 + 6], pr[8 * c8 + 7]));
         }
       }
-      tmem_st_wait();
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(bar(C::B_DSREADY));
+      mbar_arrive(bar(C::B_DSREADY + bf));
+      // The dQ of tile t - NBUF + 1 is ready by now (it was issued right after
+      // that tile's dS); reading it out frees the block for a later dP.
+      if (t - NBUF + 1 >= 0 && !drain_dq(t - NBUF + 1)) { ok = false; break; }
     }
+    for (int u = nt - NBUF + 1 < 0 ? 0 : nt - NBUF + 1; ok && u < nt; ++u) ok = drain_dq(u);
     // ------------------------------------------------------------ epilogue
     if (ok && nt > 0) ok = mbar_wait_warp(bar(C::B_DONE), 0);
     if (ok) {
       tc_fence_after();
-      // dK (x scale) staged in the Q slots, dV in the dO slots.
+      // dK (x scale) staged in the Q slots, dV in the dO slots; this warp
+      // writes head-dim columns [half * D/2, (half + 1) * D/2) of its rows.
 #pragma unroll 1
       for (int which = 0; which < 2; ++which) {
         const uint32_t src = tmem + lane_base + (which == 0 ? C::TM_DK : C::TM_DV);
         const uint32_t row_addr = smem0 + (which == 0 ? C::OFF_Q : C::OFF_DO) + r * 128;
         const float mul = which == 0 ? p.softmax_scale : 1.f;
 #pragma unroll 1
-        for (int c = 0; c < D; c += 32) {
+        for (int c = half * (D / 2); c < (half + 1) * (D / 2); c += 32) {
           uint32_t raw[32];
           if (nt > 0) {
             tmem_ld32(src + c, raw);
@@ -453,7 +549,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       fence_proxy_async_smem();
     }
     tc_fence_before();
-    named_bar_sync(1, 128);
+    named_bar_sync(1, 256);
     if (ok && threadIdx.x == 0) {
       for (int bx = 0; bx < C::NBOX; ++bx) {
         tma_store_4d(&tm_dk, smem0 + C::OFF_Q + bx * (BN * 128), bx * 64, kvh, k0, b);
@@ -461,55 +557,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       }
       bulk_commit_group();
       bulk_wait_group_all();
-    }
-  } else {
-    // ------------------------------------------------------------ dQ readout (warps 4-7)
-    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    const int r = (int)((warp & 3) * 32 + lane);  // TMEM lane
-    for (int t = 0; t < nt; ++t) {
-      const int h = kvh * group + t / nqb;
-      const int q0 = (qb_lo + t % nqb) * BM;
-      if (!mbar_wait_warp(bar(C::B_DQFULL), t & 1)) break;
-      tc_fence_after();
-      if constexpr (C::DQT) {
-        // lane = head-dim column r, columns = query rows q0..q0+BM
-        float vals[BM];
-#pragma unroll
-        for (int c = 0; c < BM; c += 32) {
-          uint32_t raw[32];
-          tmem_ld32(tmem + lane_base + C::TM_DQ + c, raw);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) vals[c + e] = __uint_as_float(raw[e]);
-        }
-        tmem_ld_wait();
-        tc_fence_before();
-        mbar_arrive(bar(C::B_DQFREE));
-        float* dst = p.dq_acc + (((size_t)b * p.seqlen_q + q0) * p.nheads + h) * D + r;
-        const size_t row_stride = (size_t)p.nheads * D;
-#pragma unroll 8
-        for (int c = 0; c < BM; ++c)
-          if (q0 + c < p.seqlen_q) atomicAdd(dst + c * row_stride, vals[c]);
-      } else {
-        // lane = query row q0 + r, columns = head-dim
-        float vals[D];
-#pragma unroll
-        for (int c = 0; c < D; c += 32) {
-          uint32_t raw[32];
-          tmem_ld32(tmem + lane_base + C::TM_DQ + c, raw);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) vals[c + e] = __uint_as_float(raw[e]);
-        }
-        tmem_ld_wait();
-        tc_fence_before();
-        mbar_arrive(bar(C::B_DQFREE));
-        if (q0 + r < p.seqlen_q) {
-          float4* dst = reinterpret_cast<float4*>(
-              p.dq_acc + (((size_t)b * p.seqlen_q + q0 + r) * p.nheads + h) * D);
-#pragma unroll
-          for (int c = 0; c < D / 4; ++c)
-            atomicAdd(dst + c, make_float4(vals[4 * c], vals[4 * c + 1], vals[4 * c + 2], vals[4 * c + 3]));
-        }
-      }
     }
   }
   tc_fence_before();
