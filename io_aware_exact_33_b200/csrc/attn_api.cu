@@ -129,6 +129,19 @@ int fill_blocks(long long n) {
   return (int)(b < 1 ? 1 : (b > 4096 ? 4096 : b));
 }
 
+// Kernel and grid width of a forward configuration: two query tiles per CTA
+// where both O tiles fit tensor memory (d <= 128), one otherwise.
+template <class C>
+struct FwdLaunch {
+  static constexpr auto kernel() { return attn_fwd_kernel<C>; }
+  static constexpr int rows_per_cta = C::BM;
+};
+template <int D, int S, bool F>
+struct FwdLaunch<FwdPPCfg<D, S, F>> {
+  static constexpr auto kernel() { return attn_fwd_pp_kernel<FwdPPCfg<D, S, F>>; }
+  static constexpr int rows_per_cta = 2 * FwdPPCfg<D, S, F>::BM;
+};
+
 template <class C>
 attn_status launch_fwd(const attn_params* p, const void* q, const void* k, const void* v, void* o,
                        float* lse, cudaStream_t stream) {
@@ -150,8 +163,8 @@ attn_status launch_fwd(const attn_params* p, const void* q, const void* k, const
   fp.window_left = p->window_left;
   fp.window_right = p->window_right;
   fp.scale_log2 = p->softmax_scale * 1.4426950408889634f;
-  fp.num_qblocks = (p->seqlen_q + C::BM - 1) / C::BM;
-  auto kern = attn_fwd_kernel<C>;
+  fp.num_qblocks = (p->seqlen_q + FwdLaunch<C>::rows_per_cta - 1) / FwdLaunch<C>::rows_per_cta;
+  auto kern = FwdLaunch<C>::kernel();
   if (!ensure_smem(reinterpret_cast<const void*>(kern), C::SMEM_BYTES)) return ATTN_ERR_CUDA;
   dim3 grid(fp.num_qblocks, p->nheads, p->batch);
   kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mo, fp);
@@ -337,11 +350,11 @@ attn_status attn_fwd(const attn_params* p, const void* q, const void* k, const v
   const bool fp16 = p->dtype == ATTN_FP16;
   switch (p->headdim) {
     case 64:
-      return fp16 ? launch_fwd<FwdCfg<64, 128, 3, true>>(p, q, k, v, o, lse, stream)
-                  : launch_fwd<FwdCfg<64, 128, 3, false>>(p, q, k, v, o, lse, stream);
+      return fp16 ? launch_fwd<FwdPPCfg<64, 3, true>>(p, q, k, v, o, lse, stream)
+                  : launch_fwd<FwdPPCfg<64, 3, false>>(p, q, k, v, o, lse, stream);
     case 128:
-      return fp16 ? launch_fwd<FwdCfg<128, 128, 2, true>>(p, q, k, v, o, lse, stream)
-                  : launch_fwd<FwdCfg<128, 128, 2, false>>(p, q, k, v, o, lse, stream);
+      return fp16 ? launch_fwd<FwdPPCfg<128, 2, true>>(p, q, k, v, o, lse, stream)
+                  : launch_fwd<FwdPPCfg<128, 2, false>>(p, q, k, v, o, lse, stream);
     case 256:
       return fp16 ? launch_fwd<FwdCfg<256, 64, 2, true>>(p, q, k, v, o, lse, stream)
                   : launch_fwd<FwdCfg<256, 64, 2, false>>(p, q, k, v, o, lse, stream);

@@ -110,9 +110,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   const int nt = kr.jmax >= kr.jmin ? (int)(kr.jmax / BN) - t_lo + 1 : 0;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < C::NBAR; ++i) mbar_init(bar(i), 1);
-    mbar_init(bar(C::B_PREADY + 0), 128);
-    mbar_init(bar(C::B_PREADY + 1), 128);
+    for (int i = 0; i < C::NBAR; ++i)
+      mbar_init(bar(i), (i == C::B_PREADY || i == C::B_PREADY + 1) ? 128 : 1);
     fence_barrier_init();
   }
   if (warp == 5) {
@@ -340,6 +339,365 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   tc_fence_before();
   __syncthreads();
   if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace attn
+
+namespace attn {
+
+// ---------------------------------------------------------------------------
+// Two query tiles per CTA (d <= 128).
+//
+// Same computation as attn_fwd_kernel, with two 128-row query tiles of one
+// (batch, head) sharing each K/V tile, so that the tensor pipe always has
+// one tile's MMAs to run while the other tile's softmax warps exponentiate:
+//
+//   warps 0-3   softmax of query tile 0     warps 4-7   softmax of tile 1
+//   warp 8      TMA producer                warp 9      MMA issuer
+//
+// MMA order per key tile j:  S0_j, PV1_{j-1}, S1_j, PV0_j  (each only where
+// tile 0 / tile 1 sees key tile j).  S_i of one key tile is issued after
+// PV_i of the previous one, so whenever tile i's softmax runs, its O_i is
+// settled in tensor memory and the (conditional) rescale needs no wait.
+// Softmax reads its scores twice from tensor memory in 32-column chunks:
+// once for the row max, once for exp2 / sum / 16-bit P, which keeps the
+// per-thread register footprint small.
+//
+// Tensor memory: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D).
+// ---------------------------------------------------------------------------
+template <int D_, int STAGES_, bool FP16_>
+struct FwdPPCfg {
+  static constexpr int D = D_, BN = 128, STAGES = STAGES_;
+  static constexpr bool FP16 = FP16_;
+  static constexpr int BM = 128;   // rows per query tile; two tiles per CTA
+  static constexpr int NBOX = D / 64;
+  static constexpr int Q_BYTES = BM * D * 2;
+  static constexpr int KV_BYTES = BN * D * 2;
+  static constexpr int OFF_Q = 0;  // two tiles
+  static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
+  static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
+  static constexpr int OFF_BAR = OFF_V + STAGES * KV_BYTES;
+  static constexpr int B_Q = 0;
+  static constexpr int B_KFULL = 1;
+  static constexpr int B_VFULL = B_KFULL + STAGES;
+  static constexpr int B_EMPTY = B_VFULL + STAGES;
+  static constexpr int B_SFULL = B_EMPTY + STAGES;  // per query tile
+  static constexpr int B_PREADY = B_SFULL + 2;      // per query tile, 128 arrivals
+  static constexpr int B_OREADY = B_PREADY + 2;     // per query tile
+  static constexpr int NBAR = B_OREADY + 2;
+  static constexpr int OFF_TMEMPTR = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM_BYTES = OFF_TMEMPTR + 16 + 1024;
+  static constexpr int TM_S = 0, TM_O = 2 * BN;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int THREADS = 320;
+  static_assert(D == 64 || D == 128, "two O tiles must fit tensor memory");
+  static_assert(TM_O + 2 * D <= TMEM_COLS, "tensor memory");
+  static_assert(SMEM_BYTES <= 232448, "shared memory");
+};
+
+// One row's softmax of one key tile, run by each softmax thread (row =
+// TMEM lane).  Scores are read from tensor memory 32 columns at a time with
+// the next chunk's load in flight.  Pass 1: row max (columns outside
+// [vlo, vhi) count as -inf when MASK).  Then the reference max (kept unless
+// the row max grew by more than 8 in log2 units) and, if any row of the warp
+// moved it, O_i *= alpha in tensor memory.  Pass 2: P = exp2(s*scale*log2e -
+// m), the row sum, and 16-bit P written over score columns already read
+// (chunk c's P lands in columns [16c, 16c + 16), below the chunk in flight).
+template <bool MASK, class C>
+__device__ __forceinline__ void softmax_tile(uint32_t s_tmem, uint32_t o_tmem, int n, int vlo,
+                                             int vhi, float scale_log2, float m, float& mx,
+                                             float& rowsum, float& alpha, float& m_use) {
+  constexpr int BN = C::BN, D = C::D;
+  auto val = [&](uint32_t bits, int col) -> float {
+    return (MASK && (col < vlo || col >= vhi)) ? -INFINITY : __uint_as_float(bits);
+  };
+  mx = -INFINITY;
+  {
+    uint32_t buf[2][32];
+    tmem_ld32(s_tmem, buf[0]);
+    tmem_ld_wait();
+#pragma unroll
+    for (int c = 0; c < BN / 32; ++c) {
+      if (c + 1 < BN / 32) tmem_ld32(s_tmem + (c + 1) * 32, buf[(c + 1) & 1]);
+#pragma unroll
+      for (int e = 0; e < 32; ++e) mx = fmaxf(mx, val(buf[c & 1][e], c * 32 + e));
+      if (c + 1 < BN / 32) tmem_ld_wait();
+    }
+  }
+  const float m_tile = mx * scale_log2;  // scale > 0
+  m_use = m;
+  alpha = 1.f;
+  if (m_tile > m + 8.f) {
+    m_use = m_tile;
+    alpha = (m == -INFINITY) ? 0.f : ex2(m - m_tile);
+  }
+  const float m_sub = (m_use == -INFINITY) ? 0.f : m_use;
+  if (n > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+    for (int c = 0; c < D; c += 32) {
+      uint32_t raw[32];
+      tmem_ld32(o_tmem + c, raw);
+      tmem_ld_wait();
+#pragma unroll
+      for (int e = 0; e < 32; ++e) raw[e] = __float_as_uint(__uint_as_float(raw[e]) * alpha);
+      tmem_st32(o_tmem + c, raw);
+    }
+    tmem_st_wait();
+  }
+  rowsum = 0.f;
+  {
+    uint32_t buf[2][32];
+    tmem_ld32(s_tmem, buf[0]);
+    tmem_ld_wait();
+#pragma unroll
+    for (int c = 0; c < BN / 32; ++c) {
+      if (c + 1 < BN / 32) tmem_ld32(s_tmem + (c + 1) * 32, buf[(c + 1) & 1]);
+      uint32_t w[16];
+#pragma unroll
+      for (int e = 0; e < 32; e += 2) {
+        const float p0 = ex2(fmaf(val(buf[c & 1][e], c * 32 + e), scale_log2, -m_sub));
+        const float p1 = ex2(fmaf(val(buf[c & 1][e + 1], c * 32 + e + 1), scale_log2, -m_sub));
+        rowsum += p0 + p1;
+        w[e / 2] = pack2<C::FP16>(p0, p1);
+      }
+      if (c + 1 < BN / 32) tmem_ld_wait();
+      tmem_st16(s_tmem + c * 16, w);
+    }
+  }
+}
+
+template <class C>
+__global__ void __launch_bounds__(C::THREADS, 1)
+    attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                       const FwdParams p) {
+  constexpr int D = C::D, BN = C::BN, BM = C::BM, STAGES = C::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t smem0 = (smem_addr(smem_raw) + 1023u) & ~1023u;
+  uint8_t* smem_gen = smem_raw + (smem0 - smem_addr(smem_raw));
+  auto bar = [&](int i) -> uint32_t { return smem0 + C::OFF_BAR + 8u * i; };
+  volatile uint32_t* tmem_ptr_slot = reinterpret_cast<volatile uint32_t*>(smem_gen + C::OFF_TMEMPTR);
+
+  const uint32_t warp = warp_id(), lane = lane_id();
+  const int pair = p.num_qblocks - 1 - (int)blockIdx.x;  // heaviest causal pairs first
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int kvh = h / (p.nheads / p.nheads_kv);
+
+  // Key-tile range [lo_i, hi_i) of each query tile; union [ulo, uhi).
+  int lo[2], hi[2], qs[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    qs[i] = (2 * pair + i) * BM;
+    const int q1 = min(qs[i] + BM, p.seqlen_q);
+    lo[i] = hi[i] = 0;
+    if (qs[i] < q1) {
+      const KeyRange kr = visible_keys(qs[i], q1, p);
+      if (kr.jmax >= kr.jmin) {
+        lo[i] = (int)(kr.jmin / BN);
+        hi[i] = (int)(kr.jmax / BN) + 1;
+      }
+    }
+  }
+  const bool has0 = hi[0] > lo[0], has1 = hi[1] > lo[1];
+  const int ulo = has0 && has1 ? min(lo[0], lo[1]) : (has0 ? lo[0] : lo[1]);
+  const int uhi = has0 && has1 ? max(hi[0], hi[1]) : (has0 ? hi[0] : hi[1]);
+  const int nt = (has0 || has1) ? uhi - ulo : 0;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::NBAR; ++i)
+      mbar_init(bar(i), (i == C::B_PREADY || i == C::B_PREADY + 1) ? 128 : 1);
+    fence_barrier_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem0 + C::OFF_TMEMPTR, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 8 && lane == 0) {
+    prefetch_tensormap(&tm_q);
+    prefetch_tensormap(&tm_k);
+    prefetch_tensormap(&tm_v);
+    prefetch_tensormap(&tm_o);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_ptr_slot;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && nt > 0) {
+      mbar_arrive_expect_tx(bar(C::B_Q), 2 * C::Q_BYTES);
+      for (int i = 0; i < 2; ++i)
+        for (int bx = 0; bx < C::NBOX; ++bx)
+          tma_load_4d(smem0 + C::OFF_Q + i * C::Q_BYTES + bx * (BM * 128), &tm_q, bar(C::B_Q),
+                      bx * 64, h, qs[i], b);
+      for (int t = 0; t < nt; ++t) {
+        const int st = t % STAGES, n = t / STAGES;
+        if (n > 0 && !mbar_wait(bar(C::B_EMPTY + st), (n - 1) & 1)) break;
+        const int k0 = (ulo + t) * BN;
+        mbar_arrive_expect_tx(bar(C::B_KFULL + st), C::KV_BYTES);
+        for (int bx = 0; bx < C::NBOX; ++bx)
+          tma_load_4d(smem0 + C::OFF_K + st * C::KV_BYTES + bx * (BN * 128), &tm_k,
+                      bar(C::B_KFULL + st), bx * 64, kvh, k0, b);
+        mbar_arrive_expect_tx(bar(C::B_VFULL + st), C::KV_BYTES);
+        for (int bx = 0; bx < C::NBOX; ++bx)
+          tma_load_4d(smem0 + C::OFF_V + st * C::KV_BYTES + bx * (BN * 128), &tm_v,
+                      bar(C::B_VFULL + st), bx * 64, kvh, k0, b);
+      }
+      for (int t = nt - STAGES < 0 ? 0 : nt - STAGES; t < nt; ++t) {
+        const int st = t % STAGES, n = t / STAGES;
+        if (!mbar_wait(bar(C::B_KFULL + st), n & 1)) break;
+        if (!mbar_wait(bar(C::B_VFULL + st), n & 1)) break;
+      }
+      mbar_wait(bar(C::B_Q), 0);
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && nt > 0) {
+      constexpr uint32_t idesc_qk = idesc_f16(BM, BN, C::FP16, false, false);
+      constexpr uint32_t idesc_pv = idesc_f16(BM, D, C::FP16, false, true);
+      int ns[2] = {0, 0};  // S MMAs issued per query tile
+      int np[2] = {0, 0};  // PV MMAs issued per query tile
+      auto in = [&](int i, int j) { return j >= lo[i] && j < hi[i]; };
+      auto issue_s = [&](int i, int j) {
+        const int st = (j - ulo) % STAGES;
+        const uint32_t q_base = smem0 + C::OFF_Q + i * C::Q_BYTES;
+        const uint32_t k_base = smem0 + C::OFF_K + st * C::KV_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int bx = kk / 4, w = kk % 4;
+          mma_ss(tmem + C::TM_S + i * BN, sdesc_sw128(q_base + bx * (BM * 128) + w * 32, 16, 1024),
+                 sdesc_sw128(k_base + bx * (BN * 128) + w * 32, 16, 1024), idesc_qk, kk > 0);
+        }
+        mma_commit(bar(C::B_SFULL + i));
+        ++ns[i];
+      };
+      auto issue_pv = [&](int i, int j, bool last_use) -> bool {
+        const int u = j - ulo, st = u % STAGES;
+        if (!mbar_wait(bar(C::B_PREADY + i), np[i] & 1)) return false;
+        if (!mbar_wait(bar(C::B_VFULL + st), (u / STAGES) & 1)) return false;
+        tc_fence_after();
+        const uint32_t v_base = smem0 + C::OFF_V + st * C::KV_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          mma_ts(tmem + C::TM_O + i * D, tmem + C::TM_S + i * BN + kk * 8,
+                 sdesc_sw128(v_base + kk * 2048, BN * 128, 1024), idesc_pv,
+                 (np[i] > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(bar(C::B_OREADY + i));
+        if (last_use) mma_commit(bar(C::B_EMPTY + st));
+        ++np[i];
+        return true;
+      };
+      bool ok = mbar_wait(bar(C::B_Q), 0);
+      for (int j = ulo; ok && j < uhi; ++j) {
+        const int u = j - ulo, st = u % STAGES;
+        if (!mbar_wait(bar(C::B_KFULL + st), (u / STAGES) & 1)) { ok = false; break; }
+        tc_fence_after();
+        if (in(0, j)) issue_s(0, j);
+        if (j > ulo && in(1, j - 1) && !issue_pv(1, j - 1, true)) { ok = false; break; }
+        if (in(1, j)) issue_s(1, j);
+        if (in(0, j) && !issue_pv(0, j, !in(1, j))) { ok = false; break; }
+      }
+      if (ok && in(1, uhi - 1)) issue_pv(1, uhi - 1, true);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax (tile i)
+    const int i = (int)(warp >> 2);
+    const int quad = (int)(warp & 3);
+    const int q_i = i ? qs[1] : qs[0], lo_i = i ? lo[1] : lo[0], hi_i = i ? hi[1] : hi[0];
+    const int r = quad * 32 + (int)lane;  // row within the tile == TMEM lane
+    const int row = q_i + r;             // query position
+    const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+    const uint32_t s_tmem = tmem + lane_base + C::TM_S + i * BN;
+    const uint32_t o_tmem = tmem + lane_base + C::TM_O + i * D;
+    const long long off = (long long)p.seqlen_k - p.seqlen_q;
+    const long long kInf = 1ll << 40;
+    const long long rb = p.causal ? 0 : (p.window_right >= 0 ? p.window_right : kInf);
+    const long long lb = p.window_left >= 0 ? p.window_left : kInf;
+    const long long jhi = (long long)row + off + rb;  // visible keys: [jlo, jhi]
+    const long long jlo = (long long)row + off - lb;
+    const long long blk_hi = (long long)q_i + off + rb;
+    const long long blk_lo = (long long)(q_i + BM - 1) + off - lb;
+    const int n_i = hi_i - lo_i;
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int n = 0; n < n_i; ++n) {
+      if (!mbar_wait_warp(bar(C::B_SFULL + i), n & 1)) { ok = false; break; }
+      tc_fence_after();
+      const long long k0 = (long long)(lo_i + n) * BN;
+      const bool full = (k0 + BN <= p.seqlen_k) && (k0 + BN - 1 <= blk_hi) && (k0 >= blk_lo);
+      // Visible columns of this row within the key tile: [vlo, vhi).
+      int vlo = 0, vhi = BN;
+      if (!full) {
+        const long long a = jlo - k0, z = min(jhi, (long long)p.seqlen_k - 1) - k0 + 1;
+        vlo = (int)max(0ll, min((long long)BN, a));
+        vhi = (int)max(0ll, min((long long)BN, z));
+      }
+      float mx, rowsum, alpha, m_use;
+      if (full)
+        softmax_tile<false, C>(s_tmem, o_tmem, n, vlo, vhi, p.scale_log2, m, mx, rowsum, alpha, m_use);
+      else
+        softmax_tile<true, C>(s_tmem, o_tmem, n, vlo, vhi, p.scale_log2, m, mx, rowsum, alpha, m_use);
+      l = l * alpha + rowsum;
+      m = m_use;
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar(C::B_PREADY + i));
+    }
+    // ------------------------------------------------------------ epilogue
+    if (ok && n_i > 0) ok = mbar_wait_warp(bar(C::B_OREADY + i), (n_i - 1) & 1);
+    // A tile with no visible key still had its Q loaded (when the CTA has
+    // work): that load must land before the staging area is overwritten.
+    if (ok && n_i == 0 && nt > 0) ok = mbar_wait_warp(bar(C::B_Q), 0);
+    const uint32_t stage = smem0 + C::OFF_Q + i * C::Q_BYTES;  // Q_i is no longer read
+    if (ok) {
+      tc_fence_after();
+      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      const uint32_t row_addr = stage + r * 128;
+#pragma unroll 1
+      for (int c = 0; c < D; c += 32) {
+        uint32_t raw[32];
+        if (n_i > 0) {
+          tmem_ld32(o_tmem + c, raw);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) raw[e] = 0u;
+        }
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          w[e] = pack2<C::FP16>(__uint_as_float(raw[2 * e]) * inv_l,
+                                __uint_as_float(raw[2 * e + 1]) * inv_l);
+        const int bx = c / 64, chunk0 = (c % 64) / 8;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const int chunk = (chunk0 + q4) ^ (r & 7);
+          st_shared_v4(row_addr + bx * (BM * 128) + chunk * 16, w[4 * q4], w[4 * q4 + 1],
+                       w[4 * q4 + 2], w[4 * q4 + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      if (row < p.seqlen_q) {
+        const float lse = l > 0.f ? (m + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
+        p.lse[((size_t)b * p.nheads + h) * p.seqlen_q + row] = lse;
+      }
+    }
+    tc_fence_before();
+    named_bar_sync(1 + i, 128);
+    if (ok && quad == 0 && lane == 0 && q_i < p.seqlen_q) {
+      for (int bx = 0; bx < C::NBOX; ++bx)
+        tma_store_4d(&tm_o, stage + bx * (BM * 128), bx * 64, h, q_i, b);
+      bulk_commit_group();
+      bulk_wait_group_all();
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
