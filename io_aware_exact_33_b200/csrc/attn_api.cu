@@ -136,10 +136,10 @@ struct FwdLaunch {
   static constexpr auto kernel() { return attn_fwd_kernel<C>; }
   static constexpr int rows_per_cta = C::BM;
 };
-template <int D, int S, bool F>
-struct FwdLaunch<FwdPPCfg<D, S, F>> {
-  static constexpr auto kernel() { return attn_fwd_pp_kernel<FwdPPCfg<D, S, F>>; }
-  static constexpr int rows_per_cta = 2 * FwdPPCfg<D, S, F>::BM;
+template <int D, int KS, int VS, bool F>
+struct FwdLaunch<FwdPPCfg<D, KS, VS, F>> {
+  static constexpr auto kernel() { return attn_fwd_pp_kernel<FwdPPCfg<D, KS, VS, F>>; }
+  static constexpr int rows_per_cta = 2 * FwdPPCfg<D, KS, VS, F>::BM;
 };
 
 template <class C>
@@ -350,11 +350,11 @@ attn_status attn_fwd(const attn_params* p, const void* q, const void* k, const v
   const bool fp16 = p->dtype == ATTN_FP16;
   switch (p->headdim) {
     case 64:
-      return fp16 ? launch_fwd<FwdPPCfg<64, 3, true>>(p, q, k, v, o, lse, stream)
-                  : launch_fwd<FwdPPCfg<64, 3, false>>(p, q, k, v, o, lse, stream);
+      return fp16 ? launch_fwd<FwdPPCfg<64, 3, 3, true>>(p, q, k, v, o, lse, stream)
+                  : launch_fwd<FwdPPCfg<64, 3, 3, false>>(p, q, k, v, o, lse, stream);
     case 128:
-      return fp16 ? launch_fwd<FwdPPCfg<128, 2, true>>(p, q, k, v, o, lse, stream)
-                  : launch_fwd<FwdPPCfg<128, 2, false>>(p, q, k, v, o, lse, stream);
+      return fp16 ? launch_fwd<FwdPPCfg<128, 3, 2, true>>(p, q, k, v, o, lse, stream)
+                  : launch_fwd<FwdPPCfg<128, 3, 2, false>>(p, q, k, v, o, lse, stream);
     case 256:
       return fp16 ? launch_fwd<FwdCfg<256, 64, 2, true>>(p, q, k, v, o, lse, stream)
                   : launch_fwd<FwdCfg<256, 64, 2, false>>(p, q, k, v, o, lse, stream);

@@ -368,9 +368,9 @@ namespace attn {
 //
 // Tensor memory: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D).
 // ---------------------------------------------------------------------------
-template <int D_, int STAGES_, bool FP16_>
+template <int D_, int KSTAGES_, int VSTAGES_, bool FP16_>
 struct FwdPPCfg {
-  static constexpr int D = D_, BN = 128, STAGES = STAGES_;
+  static constexpr int D = D_, BN = 128, KSTAGES = KSTAGES_, VSTAGES = VSTAGES_;
   static constexpr bool FP16 = FP16_;
   static constexpr int BM = 128;   // rows per query tile; two tiles per CTA
   static constexpr int NBOX = D / 64;
@@ -378,15 +378,16 @@ struct FwdPPCfg {
   static constexpr int KV_BYTES = BN * D * 2;
   static constexpr int OFF_Q = 0;  // two tiles
   static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
-  static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
-  static constexpr int OFF_BAR = OFF_V + STAGES * KV_BYTES;
+  static constexpr int OFF_V = OFF_K + KSTAGES * KV_BYTES;
+  static constexpr int OFF_BAR = OFF_V + VSTAGES * KV_BYTES;
   static constexpr int B_Q = 0;
   static constexpr int B_KFULL = 1;
-  static constexpr int B_VFULL = B_KFULL + STAGES;
-  static constexpr int B_EMPTY = B_VFULL + STAGES;
-  static constexpr int B_SFULL = B_EMPTY + STAGES;  // per query tile
-  static constexpr int B_PREADY = B_SFULL + 2;      // per query tile, 128 arrivals
-  static constexpr int B_OREADY = B_PREADY + 2;     // per query tile
+  static constexpr int B_VFULL = B_KFULL + KSTAGES;
+  static constexpr int B_KEMPTY = B_VFULL + VSTAGES;   // K slot read by its last S MMA
+  static constexpr int B_VEMPTY = B_KEMPTY + KSTAGES;  // V slot read by its last PV MMA
+  static constexpr int B_SFULL = B_VEMPTY + VSTAGES;   // per query tile
+  static constexpr int B_PREADY = B_SFULL + 2;  // per (query tile, half of the key tile), 128 arrivals
+  static constexpr int B_OREADY = B_PREADY + 4;  // per query tile
   static constexpr int NBAR = B_OREADY + 2;
   static constexpr int OFF_TMEMPTR = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_TMEMPTR + 16 + 1024;
@@ -409,7 +410,8 @@ struct FwdPPCfg {
 template <bool MASK, class C>
 __device__ __forceinline__ void softmax_tile(uint32_t s_tmem, uint32_t o_tmem, int n, int vlo,
                                              int vhi, float scale_log2, float m, float& mx,
-                                             float& rowsum, float& alpha, float& m_use) {
+                                             float& rowsum, float& alpha, float& m_use,
+                                             uint32_t pready_half0, uint32_t pready_half1) {
   constexpr int BN = C::BN, D = C::D;
   auto val = [&](uint32_t bits, int col) -> float {
     return (MASK && (col < vlo || col >= vhi)) ? -INFINITY : __uint_as_float(bits);
@@ -423,7 +425,8 @@ __device__ __forceinline__ void softmax_tile(uint32_t s_tmem, uint32_t o_tmem, i
     for (int c = 0; c < BN / 32; ++c) {
       if (c + 1 < BN / 32) tmem_ld32(s_tmem + (c + 1) * 32, buf[(c + 1) & 1]);
 #pragma unroll
-      for (int e = 0; e < 32; ++e) mx = fmaxf(mx, val(buf[c & 1][e], c * 32 + e));
+      for (int e = 0; e < 32; e += 2)
+        mx = max3f(mx, val(buf[c & 1][e], c * 32 + e), val(buf[c & 1][e + 1], c * 32 + e + 1));
       if (c + 1 < BN / 32) tmem_ld_wait();
     }
   }
@@ -441,13 +444,24 @@ __device__ __forceinline__ void softmax_tile(uint32_t s_tmem, uint32_t o_tmem, i
       uint32_t raw[32];
       tmem_ld32(o_tmem + c, raw);
       tmem_ld_wait();
+      const uint64_t alpha2 = f2_pack(alpha, alpha);
 #pragma unroll
-      for (int e = 0; e < 32; ++e) raw[e] = __float_as_uint(__uint_as_float(raw[e]) * alpha);
+      for (int e = 0; e < 32; e += 2) {
+        float lo, hi;
+        f2_unpack(f2_mul(f2_pack(__uint_as_float(raw[e]), __uint_as_float(raw[e + 1])), alpha2), lo, hi);
+        raw[e] = __float_as_uint(lo);
+        raw[e + 1] = __float_as_uint(hi);
+      }
       tmem_st32(o_tmem + c, raw);
     }
     tmem_st_wait();
   }
-  rowsum = 0.f;
+  // Column pairs go through packed f32x2 FMA / ADD: one instruction computes
+  // s*scale*log2e - m for two columns, one adds two P values to two running
+  // sums (combined at the end).
+  const uint64_t scale2 = f2_pack(scale_log2, scale_log2);
+  const uint64_t neg_m2 = f2_pack(-m_sub, -m_sub);
+  uint64_t sum2 = f2_pack(0.f, 0.f);
   {
     uint32_t buf[2][32];
     tmem_ld32(s_tmem, buf[0]);
@@ -458,14 +472,27 @@ __device__ __forceinline__ void softmax_tile(uint32_t s_tmem, uint32_t o_tmem, i
       uint32_t w[16];
 #pragma unroll
       for (int e = 0; e < 32; e += 2) {
-        const float p0 = ex2(fmaf(val(buf[c & 1][e], c * 32 + e), scale_log2, -m_sub));
-        const float p1 = ex2(fmaf(val(buf[c & 1][e + 1], c * 32 + e + 1), scale_log2, -m_sub));
-        rowsum += p0 + p1;
+        const uint64_t x2 = f2_pack(val(buf[c & 1][e], c * 32 + e), val(buf[c & 1][e + 1], c * 32 + e + 1));
+        float a0, a1;
+        f2_unpack(f2_fma(x2, scale2, neg_m2), a0, a1);
+        const float p0 = ex2(a0), p1 = ex2(a1);
+        sum2 = f2_add(sum2, f2_pack(p0, p1));
         w[e / 2] = pack2<C::FP16>(p0, p1);
       }
       if (c + 1 < BN / 32) tmem_ld_wait();
       tmem_st16(s_tmem + c * 16, w);
+      if (c == BN / 64 - 1 || c == BN / 32 - 1) {
+        // this half of P is in tensor memory: let its PV MMAs start
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(c == BN / 32 - 1 ? pready_half1 : pready_half0);
+      }
     }
+  }
+  {
+    float s0, s1;
+    f2_unpack(sum2, s0, s1);
+    rowsum = s0 + s1;
   }
 }
 
@@ -474,7 +501,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                        const FwdParams p) {
-  constexpr int D = C::D, BN = C::BN, BM = C::BM, STAGES = C::STAGES;
+  constexpr int D = C::D, BN = C::BN, BM = C::BM, KS = C::KSTAGES, VS = C::VSTAGES;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t smem0 = (smem_addr(smem_raw) + 1023u) & ~1023u;
   uint8_t* smem_gen = smem_raw + (smem0 - smem_addr(smem_raw));
@@ -508,7 +535,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NBAR; ++i)
-      mbar_init(bar(i), (i == C::B_PREADY || i == C::B_PREADY + 1) ? 128 : 1);
+      mbar_init(bar(i), (i >= C::B_PREADY && i < C::B_PREADY + 4) ? 128 : 1);
     fence_barrier_init();
   }
   if (warp == 9) {
@@ -534,24 +561,37 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         for (int bx = 0; bx < C::NBOX; ++bx)
           tma_load_4d(smem0 + C::OFF_Q + i * C::Q_BYTES + bx * (BM * 128), &tm_q, bar(C::B_Q),
                       bx * 64, h, qs[i], b);
-      for (int t = 0; t < nt; ++t) {
-        const int st = t % STAGES, n = t / STAGES;
-        if (n > 0 && !mbar_wait(bar(C::B_EMPTY + st), (n - 1) & 1)) break;
-        const int k0 = (ulo + t) * BN;
+      // K and V slots are released separately: K_j after key tile j's last S
+      // MMA (same iteration), V_j after its last PV MMA (up to one later).
+      // K runs one tile ahead of V in the issue order, so a V slot that is
+      // still in use never holds back the next K load.
+      auto load_k = [&](int t) -> bool {
+        const int st = t % KS, n = t / KS;
+        if (n > 0 && !mbar_wait(bar(C::B_KEMPTY + st), (n - 1) & 1)) return false;
         mbar_arrive_expect_tx(bar(C::B_KFULL + st), C::KV_BYTES);
         for (int bx = 0; bx < C::NBOX; ++bx)
           tma_load_4d(smem0 + C::OFF_K + st * C::KV_BYTES + bx * (BN * 128), &tm_k,
-                      bar(C::B_KFULL + st), bx * 64, kvh, k0, b);
+                      bar(C::B_KFULL + st), bx * 64, kvh, (ulo + t) * BN, b);
+        return true;
+      };
+      auto load_v = [&](int t) -> bool {
+        const int st = t % VS, n = t / VS;
+        if (n > 0 && !mbar_wait(bar(C::B_VEMPTY + st), (n - 1) & 1)) return false;
         mbar_arrive_expect_tx(bar(C::B_VFULL + st), C::KV_BYTES);
         for (int bx = 0; bx < C::NBOX; ++bx)
           tma_load_4d(smem0 + C::OFF_V + st * C::KV_BYTES + bx * (BN * 128), &tm_v,
-                      bar(C::B_VFULL + st), bx * 64, kvh, k0, b);
+                      bar(C::B_VFULL + st), bx * 64, kvh, (ulo + t) * BN, b);
+        return true;
+      };
+      bool go = load_k(0);
+      for (int t = 0; go && t < nt; ++t) {
+        if (t + 1 < nt) go = load_k(t + 1);
+        go = go && load_v(t);
       }
-      for (int t = nt - STAGES < 0 ? 0 : nt - STAGES; t < nt; ++t) {
-        const int st = t % STAGES, n = t / STAGES;
-        if (!mbar_wait(bar(C::B_KFULL + st), n & 1)) break;
-        if (!mbar_wait(bar(C::B_VFULL + st), n & 1)) break;
-      }
+      for (int t = nt - KS < 0 ? 0 : nt - KS; t < nt; ++t)
+        if (!mbar_wait(bar(C::B_KFULL + t % KS), (t / KS) & 1)) break;
+      for (int t = nt - VS < 0 ? 0 : nt - VS; t < nt; ++t)
+        if (!mbar_wait(bar(C::B_VFULL + t % VS), (t / VS) & 1)) break;
       mbar_wait(bar(C::B_Q), 0);
     }
   } else if (warp == 9) {
@@ -562,8 +602,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       int ns[2] = {0, 0};  // S MMAs issued per query tile
       int np[2] = {0, 0};  // PV MMAs issued per query tile
       auto in = [&](int i, int j) { return j >= lo[i] && j < hi[i]; };
-      auto issue_s = [&](int i, int j) {
-        const int st = (j - ulo) % STAGES;
+      auto issue_s = [&](int i, int j, bool last_use) {
+        const int st = (j - ulo) % KS;
         const uint32_t q_base = smem0 + C::OFF_Q + i * C::Q_BYTES;
         const uint32_t k_base = smem0 + C::OFF_K + st * C::KV_BYTES;
 #pragma unroll
@@ -573,32 +613,38 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                  sdesc_sw128(k_base + bx * (BN * 128) + w * 32, 16, 1024), idesc_qk, kk > 0);
         }
         mma_commit(bar(C::B_SFULL + i));
+        if (last_use) mma_commit(bar(C::B_KEMPTY + st));
         ++ns[i];
       };
+      // O_i += P_i V_j in two halves of the key tile, each issued as soon as
+      // the softmax warps have stored that half of P.
       auto issue_pv = [&](int i, int j, bool last_use) -> bool {
-        const int u = j - ulo, st = u % STAGES;
-        if (!mbar_wait(bar(C::B_PREADY + i), np[i] & 1)) return false;
-        if (!mbar_wait(bar(C::B_VFULL + st), (u / STAGES) & 1)) return false;
-        tc_fence_after();
+        const int u = j - ulo, st = u % VS;
+        if (!mbar_wait(bar(C::B_VFULL + st), (u / VS) & 1)) return false;
         const uint32_t v_base = smem0 + C::OFF_V + st * C::KV_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          mma_ts(tmem + C::TM_O + i * D, tmem + C::TM_S + i * BN + kk * 8,
-                 sdesc_sw128(v_base + kk * 2048, BN * 128, 1024), idesc_pv,
-                 (np[i] > 0 || kk > 0) ? 1u : 0u);
+        for (int hf = 0; hf < 2; ++hf) {
+          if (!mbar_wait(bar(C::B_PREADY + 2 * i + hf), np[i] & 1)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = hf * (BN / 32); kk < (hf + 1) * (BN / 32); ++kk)
+            mma_ts(tmem + C::TM_O + i * D, tmem + C::TM_S + i * BN + kk * 8,
+                   sdesc_sw128(v_base + kk * 2048, BN * 128, 1024), idesc_pv,
+                   (np[i] > 0 || kk > 0) ? 1u : 0u);
+        }
         mma_commit(bar(C::B_OREADY + i));
-        if (last_use) mma_commit(bar(C::B_EMPTY + st));
+        if (last_use) mma_commit(bar(C::B_VEMPTY + st));
         ++np[i];
         return true;
       };
       bool ok = mbar_wait(bar(C::B_Q), 0);
       for (int j = ulo; ok && j < uhi; ++j) {
-        const int u = j - ulo, st = u % STAGES;
-        if (!mbar_wait(bar(C::B_KFULL + st), (u / STAGES) & 1)) { ok = false; break; }
+        const int u = j - ulo, st = u % KS;
+        if (!mbar_wait(bar(C::B_KFULL + st), (u / KS) & 1)) { ok = false; break; }
         tc_fence_after();
-        if (in(0, j)) issue_s(0, j);
+        if (in(0, j)) issue_s(0, j, !in(1, j));
         if (j > ulo && in(1, j - 1) && !issue_pv(1, j - 1, true)) { ok = false; break; }
-        if (in(1, j)) issue_s(1, j);
+        if (in(1, j)) issue_s(1, j, true);
         if (in(0, j) && !issue_pv(0, j, !in(1, j))) { ok = false; break; }
       }
       if (ok && in(1, uhi - 1)) issue_pv(1, uhi - 1, true);
@@ -637,15 +683,15 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         vhi = (int)max(0ll, min((long long)BN, z));
       }
       float mx, rowsum, alpha, m_use;
+      const uint32_t ph0 = bar(C::B_PREADY + 2 * i), ph1 = bar(C::B_PREADY + 2 * i + 1);
       if (full)
-        softmax_tile<false, C>(s_tmem, o_tmem, n, vlo, vhi, p.scale_log2, m, mx, rowsum, alpha, m_use);
+        softmax_tile<false, C>(s_tmem, o_tmem, n, vlo, vhi, p.scale_log2, m, mx, rowsum, alpha,
+                               m_use, ph0, ph1);
       else
-        softmax_tile<true, C>(s_tmem, o_tmem, n, vlo, vhi, p.scale_log2, m, mx, rowsum, alpha, m_use);
+        softmax_tile<true, C>(s_tmem, o_tmem, n, vlo, vhi, p.scale_log2, m, mx, rowsum, alpha,
+                              m_use, ph0, ph1);
       l = l * alpha + rowsum;
       m = m_use;
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(bar(C::B_PREADY + i));
     }
     // ------------------------------------------------------------ epilogue
     if (ok && n_i > 0) ok = mbar_wait_warp(bar(C::B_OREADY + i), (n_i - 1) & 1);

@@ -258,6 +258,55 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// Packed pairs of fp32 (sm_100 f32x2 arithmetic): one instruction does the
+// same IEEE operation on both halves.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t r, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(r));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// max of three floats in one instruction (sm_100)
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x on the FMA pipe, to take part of the exponentials off the MUFU unit.
+// Range reduction x = n + f (n = floor(x), f in [0, 1)), a degree-3 minimax
+// polynomial for 2^f fitted by the Remez exchange algorithm
+// (csrc/fit_exp2.py; max relative error 7.5e-5), and 2^n applied by adding n
+// to the exponent field.  Valid for x <= 127; returns 0 below -126 (and for
+// -inf), so masked scores give exactly 0.
+__device__ __forceinline__ float exp2_poly(float x) {
+  const float xc = fmaxf(x, -127.f);
+  const float nf = floorf(xc);
+  const float f = xc - nf;
+  float p = fmaf(7.802452147e-02f, f, 2.260671556e-01f);
+  p = fmaf(p, f, 6.958335638e-01f);
+  p = fmaf(p, f, 9.999251962e-01f);
+  const int bits = __float_as_int(p) + (static_cast<int>(nf) << 23);
+  return x < -126.f ? 0.f : __int_as_float(bits);
+}
+
 // Pack two floats into one 32-bit word of two 16-bit values, `lo` in the
 // low half (the lower column/k index), round to nearest even.
 template <bool FP16>
