@@ -58,6 +58,22 @@ bool map_bshd(CUtensorMap* m, const void* ptr, bool fp16, int batch, int seqlen,
   return r == CUDA_SUCCESS;
 }
 
+// fp32 (batch, seqlen, heads, headdim) tensor as a 4-D map with a box of
+// 32 columns x 1 head x 32 rows and 128-byte swizzle (the dQ accumulator).
+bool map_bshd_f32_32x32(CUtensorMap* m, const void* ptr, int batch, int seqlen, int heads, int d) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)seqlen, (cuuint64_t)batch};
+  cuuint64_t strides[3] = {(cuuint64_t)d * 4, (cuuint64_t)heads * d * 4,
+                           (cuuint64_t)seqlen * heads * d * 4};
+  cuuint32_t box[4] = {32, 1, 32, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void*>(ptr), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // 2-D fp32 map over (cols, rows_total) with box (box_cols, 1), no swizzle.
 bool map_f32_rows(CUtensorMap* m, const void* ptr, long long cols, long long rows, int box_cols) {
   EncodeTiledFn enc = encode_fn();
@@ -216,7 +232,7 @@ attn_status launch_bwd_main(const attn_params* p, const void* q, const void* k, 
                             cudaStream_t stream) {
   const BwdParams bp = bwd_params(p, nullptr, workspace);
   const bool fp16 = C::FP16;
-  CUtensorMap mq, mk, mv, mdo, ml, md, mdk, mdv;
+  CUtensorMap mq, mk, mv, mdo, ml, md, mdk, mdv, mdq;
   if (!map_bshd(&mq, q, fp16, p->batch, p->seqlen_q, p->nheads, C::D, C::BM) ||
       !map_bshd(&mk, k, fp16, p->batch, p->seqlen_k, p->nheads_kv, C::D, C::BN) ||
       !map_bshd(&mv, v, fp16, p->batch, p->seqlen_k, p->nheads_kv, C::D, C::BN) ||
@@ -224,12 +240,13 @@ attn_status launch_bwd_main(const attn_params* p, const void* q, const void* k, 
       !map_f32_rows(&ml, bp.lse2, bp.nq_pad, (long long)p->batch * p->nheads, C::BM) ||
       !map_f32_rows(&md, bp.dvec, bp.nq_pad, (long long)p->batch * p->nheads, C::BM) ||
       !map_bshd(&mdk, dk, fp16, p->batch, p->seqlen_k, p->nheads_kv, C::D, C::BN) ||
-      !map_bshd(&mdv, dv, fp16, p->batch, p->seqlen_k, p->nheads_kv, C::D, C::BN))
+      !map_bshd(&mdv, dv, fp16, p->batch, p->seqlen_k, p->nheads_kv, C::D, C::BN) ||
+      !map_bshd_f32_32x32(&mdq, bp.dq_acc, p->batch, p->seqlen_q, p->nheads, C::D))
     return ATTN_ERR_CUDA;
   auto kern = attn_bwd_kernel<C>;
   if (!ensure_smem(reinterpret_cast<const void*>(kern), C::SMEM_BYTES)) return ATTN_ERR_CUDA;
   dim3 grid((p->seqlen_k + C::BN - 1) / C::BN, p->nheads_kv, p->batch);
-  kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, ml, md, mdk, mdv, bp);
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, ml, md, mdk, mdv, mdq, bp);
   return finish(stream);
 }
 

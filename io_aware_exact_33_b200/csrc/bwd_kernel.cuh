@@ -32,8 +32,9 @@
 //               memory, where it is the K-major A operand of dK and an
 //               MN-major operand of dQ; then the previous tile's dQ block
 //               (which reuses that tile's dP block) out of tensor memory into
-//               the fp32 accumulator with global atomics (other key tiles add
-//               to the same rows); finally dK, dV out through TMA.
+//               the fp32 accumulator with a TMA reduce-add per warp (other
+//               key tiles add to the same rows); finally dK, dV out through
+//               TMA.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -165,6 +166,7 @@ struct BwdCfg {
   static constexpr int NQB = BM / 64;
   static constexpr int HW = BM / 2;  // query columns per compute warp
   static constexpr int DQW = DQT ? BM : D;  // columns of a dQ block in tensor memory
+  static_assert(DQW == 64, "each compute warp drains a 32 x 32 part of the dQ block");
   static constexpr int KV_BYTES = BN * D * 2;
   static constexpr int Q_BYTES = BM * D * 2;
   static constexpr int DS_BYTES = BN * BM * 2;
@@ -173,7 +175,10 @@ struct BwdCfg {
   static constexpr int OFF_Q = OFF_V + KV_BYTES;
   static constexpr int OFF_DO = OFF_Q + QSTAGES * Q_BYTES;
   static constexpr int OFF_DS = OFF_DO + QSTAGES * Q_BYTES;
-  static constexpr int OFF_LSE = OFF_DS + NBUF * DS_BYTES;
+  // dQ staging: one 4 KB box (32 x 32 fp32, 128-byte swizzle) per compute warp
+  static constexpr int DQS_BYTES = 32 * 32 * 4;
+  static constexpr int OFF_DQS = OFF_DS + NBUF * DS_BYTES;
+  static constexpr int OFF_LSE = OFF_DQS + 8 * DQS_BYTES;
   static constexpr int OFF_DVEC = OFF_LSE + QSTAGES * BM * 4;
   static constexpr int OFF_BAR = OFF_DVEC + QSTAGES * BM * 4;
   // barriers
@@ -208,7 +213,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const __grid_constant__ CUtensorMap tm_lse2, const __grid_constant__ CUtensorMap tm_dvec,
                     const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
-                    const BwdParams p) {
+                    const __grid_constant__ CUtensorMap tm_dqacc, const BwdParams p) {
   constexpr int D = C::D, BN = C::BN, BM = C::BM, NBUF = C::NBUF, QS = C::QSTAGES;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t smem0 = (smem_addr(smem_raw) + 1023u) & ~1023u;
@@ -383,46 +388,53 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const int c0 = half * C::HW;          // first query column of this warp
     const long long j = (long long)k0 + r;
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
-    // dQ of tile u: read this warp's part out of tensor memory, release the
-    // block, and add it into the fp32 accumulator.
+    // dQ of tile u: read this warp's 32 x 32 part out of tensor memory,
+    // release the block, stage it in shared memory as a [query][head-dim]
+    // fp32 box, and add it into the accumulator with one TMA reduce-add
+    // (rows past seqlen_q are clipped by the tensor map).
+    const uint32_t dqs = smem0 + C::OFF_DQS + warp * C::DQS_BYTES;
+    bool staged = false;  // a reduce from this warp's box may still be reading it
     auto drain_dq = [&](int u) -> bool {
       const int bf = u % NBUF;
       if (!mbar_wait_warp(bar(C::B_DQFULL + bf), (u / NBUF) & 1)) return false;
       tc_fence_after();
       const int h = kvh * group + u / nqb;
       const int q0 = (qb_lo + u % nqb) * BM;
-      constexpr int W = C::DQW / 2;  // this warp's columns of the dQ block
-      const int d0 = half * W;
-      uint32_t raw[W];
-#pragma unroll
-      for (int c = 0; c < W; c += 32) {
-        uint32_t part[32];
-        tmem_ld32(tmem + lane_base + C::TM_DP + bf * BM + d0 + c, part);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) raw[c + e] = part[e];
-      }
+      uint32_t raw[32];
+      tmem_ld32(tmem + lane_base + C::TM_DP + bf * BM + half * 32, raw);
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(bar(C::B_DQFREE + bf));
-      if constexpr (C::DQT) {
-        // lane = head-dim column r; columns = query rows q0 + d0 + c
-        const size_t row_stride = (size_t)p.nheads * D;
-        float* dst = p.dq_acc + (((size_t)b * p.seqlen_q + q0 + d0) * p.nheads + h) * D + r;
-        const int nvalid = min(W, p.seqlen_q - q0 - d0);
-#pragma unroll
-        for (int c = 0; c < W; ++c)
-          if (c < nvalid) atomicAdd(dst + c * row_stride, __uint_as_float(raw[c]));
-      } else {
-        // lane = query row q0 + r; columns = head-dim d0 + c
-        if (q0 + r < p.seqlen_q) {
-          float4* dst = reinterpret_cast<float4*>(
-              p.dq_acc + (((size_t)b * p.seqlen_q + q0 + r) * p.nheads + h) * D + d0);
-#pragma unroll
-          for (int c = 0; c < W / 4; ++c)
-            atomicAdd(dst + c, make_float4(__uint_as_float(raw[4 * c]), __uint_as_float(raw[4 * c + 1]),
-                                           __uint_as_float(raw[4 * c + 2]), __uint_as_float(raw[4 * c + 3])));
-        }
+      if (staged) {
+        if (lane == 0) bulk_wait_group_read_all();
+        __syncwarp();
       }
+      // Box element (row, col) sits at row * 128 + ((col / 4) ^ (row % 8)) * 16 + (col % 4) * 4.
+      int qrow, dcol;  // this warp's box origin in (query, head-dim)
+      if constexpr (C::DQT) {
+        // lane = head-dim column quad*32 + lane; columns = queries q0 + half*32 + c
+#pragma unroll
+        for (int c = 0; c < 32; ++c)
+          st_shared_f32(dqs + c * 128 + (((lane >> 2) ^ (c & 7)) << 4) + ((lane & 3) << 2),
+                        __uint_as_float(raw[c]));
+        qrow = q0 + half * 32;
+        dcol = quad * 32;
+      } else {
+        // lane = query q0 + quad*32 + lane; columns = head-dim half*32 + c
+#pragma unroll
+        for (int c4 = 0; c4 < 8; ++c4)
+          st_shared_v4(dqs + lane * 128 + ((c4 ^ (lane & 7)) << 4), raw[4 * c4], raw[4 * c4 + 1],
+                       raw[4 * c4 + 2], raw[4 * c4 + 3]);
+        qrow = q0 + quad * 32;
+        dcol = half * 32;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0 && qrow < p.seqlen_q) {
+        tma_reduce_add_4d(&tm_dqacc, dqs, dcol, h, qrow, b);
+        bulk_commit_group();
+      }
+      staged = true;
       return true;
     };
     bool ok = true;
@@ -556,8 +568,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         tma_store_4d(&tm_dv, smem0 + C::OFF_DO + bx * (BN * 128), bx * 64, kvh, k0, b);
       }
       bulk_commit_group();
-      bulk_wait_group_all();
     }
+    // every warp's dQ reduces (and the dK/dV stores) complete before exit
+    if (lane == 0) bulk_wait_group_all();
   }
   tc_fence_before();
   __syncthreads();
