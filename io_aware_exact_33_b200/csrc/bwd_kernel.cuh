@@ -296,18 +296,22 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       constexpr uint32_t idesc_acc = idesc_f16(BN, D, C::FP16, false, true);
       constexpr uint32_t idesc_dq =
           C::DQT ? idesc_f16(D, BM, C::FP16, true, true) : idesc_f16(BM, D, C::FP16, true, true);
-      const uint32_t k_base = smem0 + C::OFF_K, v_base = smem0 + C::OFF_V;
+      // K and V stay put: their descriptors (K-major for S^T / dP^T, MN-major
+      // K for the dQ MMA) are built once.
+      const uint64_t k_kdesc = sdesc_sw128(smem0 + C::OFF_K, 16, 1024);
+      const uint64_t v_kdesc = sdesc_sw128(smem0 + C::OFF_V, 16, 1024);
+      const uint64_t k_mndesc = sdesc_sw128(smem0 + C::OFF_K, BN * 128, 1024);
       // S^T_u = K Q_u^T into the S block of buffer u % NBUF.
       auto issue_s = [&](int u) -> bool {
         const int slot = u % QS, bf = u % NBUF;
-        const uint32_t q_base = smem0 + C::OFF_Q + slot * C::Q_BYTES;
+        const uint64_t q_desc = sdesc_sw128(smem0 + C::OFF_Q + slot * C::Q_BYTES, 16, 1024);
         if (!mbar_wait(bar(C::B_QFULL + slot), (u / QS) & 1)) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int bx = kk / 4, w = kk % 4;
-          mma_ss(tmem + C::TM_S + bf * BM, sdesc_sw128(k_base + bx * (BN * 128) + w * 32, 16, 1024),
-                 sdesc_sw128(q_base + bx * (BM * 128) + w * 32, 16, 1024), idesc_s, kk > 0);
+          mma_ss(tmem + C::TM_S + bf * BM, desc_at(k_kdesc, bx * (BN * 128) + w * 32),
+                 desc_at(q_desc, bx * (BM * 128) + w * 32), idesc_s, kk > 0);
         }
         mma_commit(bar(C::B_SFULL + bf));
         return true;
@@ -315,15 +319,15 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       // dP^T_u = V dO_u^T into the dP block, once tile u - NBUF's dQ left it.
       auto issue_dp = [&](int u) -> bool {
         const int slot = u % QS, bf = u % NBUF, use = u / NBUF;
-        const uint32_t do_base = smem0 + C::OFF_DO + slot * C::Q_BYTES;
+        const uint64_t do_desc = sdesc_sw128(smem0 + C::OFF_DO + slot * C::Q_BYTES, 16, 1024);
         if (use > 0 && !mbar_wait(bar(C::B_DQFREE + bf), (use - 1) & 1)) return false;
         if (!mbar_wait(bar(C::B_DOFULL + slot), (u / QS) & 1)) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int bx = kk / 4, w = kk % 4;
-          mma_ss(tmem + C::TM_DP + bf * BM, sdesc_sw128(v_base + bx * (BN * 128) + w * 32, 16, 1024),
-                 sdesc_sw128(do_base + bx * (BM * 128) + w * 32, 16, 1024), idesc_s, kk > 0);
+          mma_ss(tmem + C::TM_DP + bf * BM, desc_at(v_kdesc, bx * (BN * 128) + w * 32),
+                 desc_at(do_desc, bx * (BM * 128) + w * 32), idesc_s, kk > 0);
         }
         mma_commit(bar(C::B_DPFULL + bf));
         return true;
@@ -331,9 +335,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       // dV += P^T dO, dK += dS^T Q and tile t's dQ share.
       auto issue_grads = [&](int t) -> bool {
         const int slot = t % QS, bf = t % NBUF, use = t / NBUF;
-        const uint32_t q_base = smem0 + C::OFF_Q + slot * C::Q_BYTES;
-        const uint32_t do_base = smem0 + C::OFF_DO + slot * C::Q_BYTES;
+        const uint64_t q_mn = sdesc_sw128(smem0 + C::OFF_Q + slot * C::Q_BYTES, BM * 128, 1024);
+        const uint64_t do_mn = sdesc_sw128(smem0 + C::OFF_DO + slot * C::Q_BYTES, BM * 128, 1024);
         const uint32_t ds_base = smem0 + C::OFF_DS + bf * C::DS_BYTES;
+        const uint64_t ds_k = sdesc_sw128(ds_base, 16, 1024);
+        const uint64_t ds_mn = sdesc_sw128(ds_base, BN * 128, 1024);
         if (!mbar_wait(bar(C::B_PREADY + bf), use & 1)) return false;
         tc_fence_after();
 #pragma unroll
@@ -342,24 +348,24 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           // packed values at the start of its own score columns.
           const int half = kk / (C::HW / 16), part = kk % (C::HW / 16);
           mma_ts(tmem + C::TM_DV, tmem + C::TM_S + bf * BM + half * C::HW + part * 8,
-                 sdesc_sw128(do_base + kk * 2048, BM * 128, 1024), idesc_acc, (t > 0 || kk > 0));
+                 desc_at(do_mn, kk * 2048), idesc_acc, (t > 0 || kk > 0));
         }
         if (!mbar_wait(bar(C::B_DSREADY + bf), use & 1)) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk) {  // dS^T as a K-major smem operand; Q MN-major
           const int bx = kk / 4, w = kk % 4;
-          mma_ss(tmem + C::TM_DK, sdesc_sw128(ds_base + bx * (BN * 128) + w * 32, 16, 1024),
-                 sdesc_sw128(q_base + kk * 2048, BM * 128, 1024), idesc_acc, (t > 0 || kk > 0));
+          mma_ss(tmem + C::TM_DK, desc_at(ds_k, bx * (BN * 128) + w * 32),
+                 desc_at(q_mn, kk * 2048), idesc_acc, (t > 0 || kk > 0));
         }
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
           if constexpr (C::DQT)  // dQ^T = K^T dS^T: both operands MN-major
-            mma_ss(tmem + C::TM_DP + bf * BM, sdesc_sw128(k_base + kk * 2048, BN * 128, 1024),
-                   sdesc_sw128(ds_base + kk * 2048, BN * 128, 1024), idesc_dq, kk > 0);
+            mma_ss(tmem + C::TM_DP + bf * BM, desc_at(k_mndesc, kk * 2048),
+                   desc_at(ds_mn, kk * 2048), idesc_dq, kk > 0);
           else  // dQ = dS K
-            mma_ss(tmem + C::TM_DP + bf * BM, sdesc_sw128(ds_base + kk * 2048, BN * 128, 1024),
-                   sdesc_sw128(k_base + kk * 2048, BN * 128, 1024), idesc_dq, kk > 0);
+            mma_ss(tmem + C::TM_DP + bf * BM, desc_at(ds_mn, kk * 2048),
+                   desc_at(k_mndesc, kk * 2048), idesc_dq, kk > 0);
         }
         mma_commit(bar(C::B_DQFULL + bf));
         mma_commit(bar(C::B_DSFREE + bf));
@@ -369,13 +375,15 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       // Two buffers: S^T_{t+1} goes in before tile t's gradient MMAs, dP^T_{t+1}
       // after them (its block holds tile t-1's dQ until that is read out).
       // One buffer: everything of tile t first.
+      // Two buffers: tile t+1's S^T and dP^T go in before tile t's gradient
+      // MMAs (the dP block of t+1 is released when the compute warps drain
+      // tile t-1's dQ, midway through tile t).  One buffer: tile t first.
       bool ok = mbar_wait(bar(C::B_KV), 0) && issue_s(0) && issue_dp(0);
       for (int t = 0; ok && t < nt; ++t) {
         const bool more = t + 1 < nt;
-        if (NBUF == 2 && more && !issue_s(t + 1)) { ok = false; break; }
+        if (NBUF == 2 && more && !(issue_s(t + 1) && issue_dp(t + 1))) { ok = false; break; }
         if (!issue_grads(t)) { ok = false; break; }
-        if (NBUF == 1 && more && !issue_s(t + 1)) { ok = false; break; }
-        if (more && !issue_dp(t + 1)) { ok = false; break; }
+        if (NBUF == 1 && more && !(issue_s(t + 1) && issue_dp(t + 1))) { ok = false; break; }
       }
       if (ok) mma_commit(bar(C::B_DONE));
     }
@@ -460,12 +468,19 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         ((long long)k0 + BN - 1 <= (long long)qa + off + rb) &&
                         ((long long)k0 >= (long long)(qa + C::HW - 1) + off - lb);
       const uint32_t lse_addr = smem0 + C::OFF_LSE + (slot * BM + c0) * 4;
+      const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
 #pragma unroll
       for (int c = 0; c < C::HW; c += 4) {
         float l4[4];
         ld_shared_v4f(lse_addr + c * 4, l4);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) pr[c + e] = ex2(fmaf(pr[c + e], p.scale_log2, -l4[e]));
+        for (int e = 0; e < 4; e += 2) {
+          float a0, a1;
+          f2_unpack(f2_fma(f2_pack(pr[c + e], pr[c + e + 1]), scale2, f2_pack(-l4[e], -l4[e + 1])),
+                    a0, a1);
+          pr[c + e] = ex2(a0);
+          pr[c + e + 1] = ex2(a1);
+        }
       }
       if (!full) {
 #pragma unroll
@@ -484,6 +499,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar(C::B_PREADY + bf));
+      // Two buffers: tile t-1's dQ finished while P_t was computed; reading
+      // it out now frees its block for dP_{t+1} (issued next by the MMA warp).
+      if (NBUF == 2 && t >= 1 && !drain_dq(t - 1)) { ok = false; break; }
       if (!mbar_wait_warp(bar(C::B_DPFULL + bf), use & 1)) { ok = false; break; }
       if (!mbar_wait_warp(bar(C::B_DOFULL + slot), ph)) { ok = false; break; }
       tc_fence_after();
@@ -498,8 +516,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           float d4[4];
           ld_shared_v4f(dvec_addr + (c + e) * 4, d4);
 #pragma unroll
-          for (int f = 0; f < 4; ++f)
-            pr[c + e + f] = pr[c + e + f] * (__uint_as_float(raw[e + f]) - d4[f]);
+          for (int f = 0; f < 4; f += 2) {
+            // dS = P * (dP - Dvec), two columns per packed instruction pair
+            const uint64_t diff = f2_add(f2_pack(__uint_as_float(raw[e + f]), __uint_as_float(raw[e + f + 1])),
+                                         f2_pack(-d4[f], -d4[f + 1]));
+            f2_unpack(f2_mul(f2_pack(pr[c + e + f], pr[c + e + f + 1]), diff), pr[c + e + f],
+                      pr[c + e + f + 1]);
+          }
         }
       }
       // dS smem buffer is free once tile t - NBUF's dK and dQ MMAs have read it.
@@ -519,9 +542,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bar(C::B_DSREADY + bf));
-      // The dQ of tile t - NBUF + 1 is ready by now (it was issued right after
-      // that tile's dS); reading it out frees the block for a later dP.
-      if (t - NBUF + 1 >= 0 && !drain_dq(t - NBUF + 1)) { ok = false; break; }
+      // One buffer: this tile's dQ (issued right after its dS) is read out
+      // before the next dP can use the block.
+      if (NBUF == 1 && !drain_dq(t)) { ok = false; break; }
     }
     for (int u = nt - NBUF + 1 < 0 ? 0 : nt - NBUF + 1; ok && u < nt; ++u) ok = drain_dq(u);
     // ------------------------------------------------------------ epilogue

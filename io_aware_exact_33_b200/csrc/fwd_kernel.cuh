@@ -170,11 +170,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         tc_fence_after();
         const uint32_t v_base = smem0 + C::OFF_V + st * C::KV_BYTES;
         const uint32_t p_tmem = tmem + (buf ? C::TM_S1 : C::TM_S0);
+        // V tile as the MN-major B operand: 16 key rows (2048 B) per step;
+        // 64-column boxes BN*128 bytes apart; 8-row groups 1024 B apart.
+        const uint64_t v_desc = sdesc_sw128(v_base, BN * 128, 1024);
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
-          // V tile as the MN-major B operand: 16 key rows (2048 B) per step;
-          // 64-column boxes BN*128 bytes apart; 8-row groups 1024 B apart.
-          const uint64_t bdesc = sdesc_sw128(v_base + kk * 2048, BN * 128, 1024);
+          const uint64_t bdesc = desc_at(v_desc, kk * 2048);
           mma_ts(tmem + C::TM_O, p_tmem + kk * 8, bdesc, idesc_pv, (u > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(bar(C::B_OREADY));
@@ -185,16 +186,16 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         const int st = t % STAGES, buf = t & 1;
         if (!mbar_wait(bar(C::B_KFULL + st), (t / STAGES) & 1)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t q_base = smem0 + C::OFF_Q;
-        const uint32_t k_base = smem0 + C::OFF_K + st * C::KV_BYTES;
         const uint32_t s_tmem = tmem + (buf ? C::TM_S1 : C::TM_S0);
+        const uint64_t q_desc = sdesc_sw128(smem0 + C::OFF_Q, 16, 1024);
+        const uint64_t k_desc = sdesc_sw128(smem0 + C::OFF_K + st * C::KV_BYTES, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           // K-major operands: 16 columns = 32 bytes per step inside a
           // 128-byte swizzled row; next 64-column box at +rows*128 bytes.
           const int bx = kk / 4, w = kk % 4;
-          const uint64_t adesc = sdesc_sw128(q_base + bx * (BM * 128) + w * 32, 16, 1024);
-          const uint64_t bdesc = sdesc_sw128(k_base + bx * (BN * 128) + w * 32, 16, 1024);
+          const uint64_t adesc = desc_at(q_desc, bx * (BM * 128) + w * 32);
+          const uint64_t bdesc = desc_at(k_desc, bx * (BN * 128) + w * 32);
           mma_ss(s_tmem, adesc, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
         }
         mma_commit(bar(C::B_SFULL + buf));
@@ -604,13 +605,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       auto in = [&](int i, int j) { return j >= lo[i] && j < hi[i]; };
       auto issue_s = [&](int i, int j, bool last_use) {
         const int st = (j - ulo) % KS;
-        const uint32_t q_base = smem0 + C::OFF_Q + i * C::Q_BYTES;
-        const uint32_t k_base = smem0 + C::OFF_K + st * C::KV_BYTES;
+        const uint64_t q_desc = sdesc_sw128(smem0 + C::OFF_Q + i * C::Q_BYTES, 16, 1024);
+        const uint64_t k_desc = sdesc_sw128(smem0 + C::OFF_K + st * C::KV_BYTES, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int bx = kk / 4, w = kk % 4;
-          mma_ss(tmem + C::TM_S + i * BN, sdesc_sw128(q_base + bx * (BM * 128) + w * 32, 16, 1024),
-                 sdesc_sw128(k_base + bx * (BN * 128) + w * 32, 16, 1024), idesc_qk, kk > 0);
+          mma_ss(tmem + C::TM_S + i * BN, desc_at(q_desc, bx * (BM * 128) + w * 32),
+                 desc_at(k_desc, bx * (BN * 128) + w * 32), idesc_qk, kk > 0);
         }
         mma_commit(bar(C::B_SFULL + i));
         if (last_use) mma_commit(bar(C::B_KEMPTY + st));
@@ -621,7 +622,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       auto issue_pv = [&](int i, int j, bool last_use) -> bool {
         const int u = j - ulo, st = u % VS;
         if (!mbar_wait(bar(C::B_VFULL + st), (u / VS) & 1)) return false;
-        const uint32_t v_base = smem0 + C::OFF_V + st * C::KV_BYTES;
+        const uint64_t v_desc = sdesc_sw128(smem0 + C::OFF_V + st * C::KV_BYTES, BN * 128, 1024);
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
           if (!mbar_wait(bar(C::B_PREADY + 2 * i + hf), np[i] & 1)) return false;
@@ -629,7 +630,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
           for (int kk = hf * (BN / 32); kk < (hf + 1) * (BN / 32); ++kk)
             mma_ts(tmem + C::TM_O + i * D, tmem + C::TM_S + i * BN + kk * 8,
-                   sdesc_sw128(v_base + kk * 2048, BN * 128, 1024), idesc_pv,
+                   desc_at(v_desc, kk * 2048), idesc_pv,
                    (np[i] > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(bar(C::B_OREADY + i));

@@ -190,6 +190,14 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
   return d;
 }
 
+// The descriptor of the same layout `bytes` further on: the start address
+// sits in the low 14 bits (in 16-byte units) and shared-memory addresses stay
+// below 256 KB, so the add never carries out of the field.  Lets the MMA
+// issuer build each operand's descriptor once and step through K with adds.
+__device__ __forceinline__ uint64_t desc_at(uint64_t desc, uint32_t bytes) {
+  return desc + static_cast<uint64_t>(bytes >> 4);
+}
+
 // Instruction descriptor of tcgen05.mma kind::f16 with an f32 accumulator.
 // a_mn / b_mn: operand is MN-major (else K-major).
 __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool fp16, bool a_mn, bool b_mn) {
