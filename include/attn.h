@@ -193,6 +193,20 @@ ATTN_API const char* attn_status_string(int status);
  * failed.  *code receives an ATTN_ERR_* value or 0. */
 ATTN_API attn_status attn_get_device_status(void* stream, int* code);
 
+/* Diagnostic with no counterpart on the pages: checks the failure-detection
+ * path on the device without faulting it.  Launches one small kernel on
+ * `stream` whose two waiters (one warp-wide, one single-thread) wait on an
+ * on-chip barrier that nothing ever arrives at; each gives up after
+ * `wait_limit_us` microseconds (1 .. 1,000,000, else ATTN_ERR_INVALID_ARG,
+ * nothing launched), ORs ATTN_ERR_TIMEOUT into the device status word and
+ * returns.  `result`, if not NULL, is caller-owned device memory of two ints
+ * that receive 1 for each waiter that gave up (0 if its wait had
+ * succeeded).  Asynchronous; ATTN_ERR_CUDA if the launch fails.  Afterwards
+ * attn_get_device_status() reports ATTN_ERR_TIMEOUT and clears it, and the
+ * CUDA context stays usable. */
+ATTN_API attn_status attn_selftest_bounded_wait(unsigned int wait_limit_us, int* result,
+                                                void* stream);
+
 /* Library version, "major.minor.patch". */
 ATTN_API const char* attn_version(void);
 

@@ -28,7 +28,8 @@ STATUS = {
 }
 EXPORTED = ("attn_fwd", "attn_bwd", "attn_bwd_prepare", "attn_bwd_accumulate", "attn_bwd_finalize",
             "attn_fwd_workspace_size", "attn_bwd_workspace_size", "attn_check_params",
-            "attn_status_string", "attn_get_device_status", "attn_version")
+            "attn_status_string", "attn_get_device_status", "attn_version", "attn_bwd_noalloc",
+            "attn_selftest_bounded_wait")
 
 
 class AttnParams(ctypes.Structure):
@@ -81,6 +82,8 @@ def _load() -> ctypes.CDLL:
     lib.attn_status_string.restype = ctypes.c_char_p
     lib.attn_get_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
     lib.attn_get_device_status.restype = ctypes.c_int
+    lib.attn_selftest_bounded_wait.argtypes = [ctypes.c_uint, vp, vp]
+    lib.attn_selftest_bounded_wait.restype = ctypes.c_int
     lib.attn_version.argtypes = []
     lib.attn_version.restype = ctypes.c_char_p
     return lib
@@ -138,6 +141,23 @@ def attn_get_device_status(stream=None) -> int:
     if st != 0:
         raise AttnError(st, "attn_get_device_status")
     return int(code.value)
+
+
+def attn_selftest_bounded_wait(wait_limit_us: int, result=None, stream=None) -> None:
+    """Launch the bounded-wait self-test: a kernel whose two waiters give up
+    after ``wait_limit_us`` microseconds on a barrier nothing arrives at.
+    ``result`` (optional) is a CUDA int32 tensor of 2 elements receiving 1 per
+    waiter that gave up.  Afterwards ``attn_get_device_status()`` returns
+    ATTN_ERR_TIMEOUT.  Raises AttnError on a bad limit or a launch failure."""
+    rp = None
+    if result is not None:
+        if result.numel() < 2 or not result.is_cuda or result.dtype.itemsize != 4:
+            raise ValueError("result must be a CUDA int32 tensor with 2 elements")
+        rp = ctypes.c_void_p(result.data_ptr())
+    st = _lib.attn_selftest_bounded_wait(ctypes.c_uint(int(wait_limit_us) & 0xffffffff), rp,
+                                         _stream(stream))
+    if st != 0:
+        raise AttnError(st, "attn_selftest_bounded_wait")
 
 
 # ----------------------------------------------------------------- torch side

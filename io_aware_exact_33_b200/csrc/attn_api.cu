@@ -304,6 +304,27 @@ void* noalloc_scratch_address() {
   return ptr;
 }
 
+
+// Self-test of the bounded wait: two waiters (one warp-uniform, one single
+// thread) on an mbarrier that nothing ever arrives at.  Both must give up
+// after `limit_ns`, record the timeout in the status word, and return.
+__global__ void selftest_bounded_wait_kernel(unsigned long long limit_ns, int* result) {
+  __shared__ __align__(8) unsigned long long bar_word;
+  const uint32_t bar = smem_addr(&bar_word);
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    const bool ok = mbar_wait_warp(bar, 0, limit_ns);
+    if (threadIdx.x == 0 && result) result[0] = ok ? 0 : 1;
+  } else if (threadIdx.x == 32) {
+    const bool ok = mbar_wait(bar, 0, limit_ns);
+    if (result) result[1] = ok ? 0 : 1;
+  }
+}
+
 }  // namespace
 
 extern "C" {
@@ -494,6 +515,13 @@ attn_status attn_get_device_status(void* stream_, int* code) {
   if (cudaStreamSynchronize(stream) != cudaSuccess) return ATTN_ERR_CUDA;
   *code = static_cast<int>(host);
   return ATTN_OK;
+}
+
+attn_status attn_selftest_bounded_wait(unsigned int wait_limit_us, int* result, void* stream_) {
+  if (wait_limit_us == 0 || wait_limit_us > 1000000u) return ATTN_ERR_INVALID_ARG;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  selftest_bounded_wait_kernel<<<1, 64, 0, stream>>>(1000ull * wait_limit_us, result);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 }  // extern "C"

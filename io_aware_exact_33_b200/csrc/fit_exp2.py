@@ -1,15 +1,15 @@
-"""Fit the polynomial the kernels use for 2^f on [0, 1).
+"""Fit the polynomial the kernels use for 2^f on [-1/2, 1/2].
 
-Method: Cody-Waite style range reduction (x = n + f with n = floor(x),
+Method: Cody-Waite style range reduction (x = n + f with n = round(x),
 2^x = 2^n * 2^f, 2^n applied by adding n to the float's exponent field) and a
-minimax polynomial for 2^f on [0, 1), found with the Remez exchange algorithm
-(relative error, equioscillation on degree + 2 points).  Everything here is
-computed from the mathematics; no library's constants are used.
+minimax polynomial for 2^f on [-1/2, 1/2], found with the Remez exchange
+algorithm (relative error, equioscillation on degree + 2 points).  Everything
+here is computed from the mathematics; no library's constants are used.
 
 Run:  python io_aware_exact_33_b200/csrc/fit_exp2.py [degree]
 It prints the coefficients (float32-rounded) and the achieved maximum
 relative error of the float32 Horner evaluation; the values are pasted into
-sm100.cuh (exp2_poly).
+sm100.cuh (exp2_poly2).
 """
 from __future__ import annotations
 
@@ -19,12 +19,12 @@ import numpy as np
 
 
 def remez_relative(degree: int, iters: int = 60):
-    """Minimax (relative error) polynomial for 2^f on [0, 1]."""
+    """Minimax (relative error) polynomial for 2^f on [-1/2, 1/2]."""
     n = degree + 2
     # Chebyshev extrema as the initial reference
     k = np.arange(n)
-    xs = 0.5 - 0.5 * np.cos(np.pi * k / (n - 1))
-    grid = np.linspace(0.0, 1.0, 200001)
+    xs = -0.5 * np.cos(np.pi * k / (n - 1))
+    grid = np.linspace(-0.5, 0.5, 200001)
     target = np.exp2(grid)
     coef = None
     for _ in range(iters):
@@ -66,7 +66,7 @@ def main():
     degree = int(sys.argv[1]) if len(sys.argv) > 1 else 3
     coef = remez_relative(degree)
     coef32 = [np.float32(c) for c in coef]
-    f = np.linspace(0.0, 1.0, 100001, dtype=np.float32)
+    f = np.linspace(-0.5, 0.5, 100001, dtype=np.float32)
     approx = np.array([horner_f32(coef32, x) for x in f[::10]], dtype=np.float64)
     exact = np.exp2(f[::10].astype(np.float64))
     rel = np.max(np.abs(approx - exact) / exact)

@@ -408,6 +408,11 @@ struct FwdPPCfg {
 // moved it, O_i *= alpha in tensor memory.  Pass 2: P = exp2(s*scale*log2e -
 // m), the row sum, and 16-bit P written over score columns already read
 // (chunk c's P lands in columns [16c, 16c + 16), below the chunk in flight).
+// Column pairs of each 32-column chunk whose exponentials go through the
+// FMA-pipe polynomial instead of MUFU ex2 (bit i = pair i), on tiles with no
+// masked column; the two units then work in parallel.
+constexpr uint32_t kPolyPairs = 0x2222u;
+
 template <bool MASK, class C>
 __device__ __forceinline__ void softmax_tile(uint32_t s_tmem, uint32_t o_tmem, int n, int vlo,
                                              int vhi, float scale_log2, float m, float& mx,
@@ -474,9 +479,14 @@ __device__ __forceinline__ void softmax_tile(uint32_t s_tmem, uint32_t o_tmem, i
 #pragma unroll
       for (int e = 0; e < 32; e += 2) {
         const uint64_t x2 = f2_pack(val(buf[c & 1][e], c * 32 + e), val(buf[c & 1][e + 1], c * 32 + e + 1));
-        float a0, a1;
+        float a0, a1, p0, p1;
         f2_unpack(f2_fma(x2, scale2, neg_m2), a0, a1);
-        const float p0 = ex2(a0), p1 = ex2(a1);
+        if (!MASK && ((kPolyPairs >> (e / 2)) & 1)) {
+          exp2_poly2(a0, a1, p0, p1);
+        } else {
+          p0 = ex2(a0);
+          p1 = ex2(a1);
+        }
         sum2 = f2_add(sum2, f2_pack(p0, p1));
         w[e / 2] = pack2<C::FP16>(p0, p1);
       }

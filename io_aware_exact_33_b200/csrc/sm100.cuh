@@ -65,15 +65,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Wait for the phase with parity `parity` of barrier `bar` to complete, for
-// at most kWaitLimitNs.  On expiry the status word gets kStatusTimeout and
+// at most `limit_ns`.  On expiry the status word gets kStatusTimeout and
 // false is returned; the caller must then wind down without further waits
 // on this barrier.  Single-thread version.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
+    if ((it & 63u) == 0 && globaltimer_ns() - t0 > limit_ns) {
       atomicOr(&g_attn_status, kStatusTimeout);
       return false;
     }
@@ -82,12 +83,13 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
 
 // Warp-uniform version: every lane of a converged warp calls it and all get
 // the same answer, so warp-collective instructions after it stay uniform.
-__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity,
+                                               unsigned long long limit_ns = kWaitLimitNs) {
   if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
   const unsigned long long t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
-    bool late = (it & 63u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs;
+    bool late = (it & 63u) == 0 && globaltimer_ns() - t0 > limit_ns;
     if (__any_sync(0xffffffffu, late)) {
       if (lane_id() == 0) atomicOr(&g_attn_status, kStatusTimeout);
       return false;
@@ -315,21 +317,31 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   return d;
 }
 
-// 2^x on the FMA pipe, to take part of the exponentials off the MUFU unit.
-// Range reduction x = n + f (n = floor(x), f in [0, 1)), a degree-3 minimax
-// polynomial for 2^f fitted by the Remez exchange algorithm
-// (csrc/fit_exp2.py; max relative error 7.5e-5), and 2^n applied by adding n
-// to the exponent field.  Valid for x <= 127; returns 0 below -126 (and for
-// -inf), so masked scores give exactly 0.
-__device__ __forceinline__ float exp2_poly(float x) {
-  const float xc = fmaxf(x, -127.f);
-  const float nf = floorf(xc);
-  const float f = xc - nf;
-  float p = fmaf(7.802452147e-02f, f, 2.260671556e-01f);
-  p = fmaf(p, f, 6.958335638e-01f);
-  p = fmaf(p, f, 9.999251962e-01f);
-  const int bits = __float_as_int(p) + (static_cast<int>(nf) << 23);
-  return x < -126.f ? 0.f : __int_as_float(bits);
+// 2^x for two floats on the FMA and integer pipes, to take part of the
+// exponentials off the MUFU unit.  Range reduction x = n + f with n = round(x)
+// taken by the 1.5 * 2^23 shifter (adding it leaves n in the low mantissa
+// bits, subtracting it again gives n exactly, all in packed f32x2 adds), f in
+// [-1/2, 1/2]; a degree-3 minimax polynomial for 2^f fitted by the Remez
+// exchange algorithm (csrc/fit_exp2.py; max relative error 7.5e-5); 2^n
+// applied by adding the shifted low bits of the shifter sum to the exponent
+// field.  Arguments are clamped to >= -125 (the result stays a normal float),
+// so a tiny argument gives about 2^-125 instead of 0: use it only where every
+// argument is finite and the row sum it feeds is >= 1.  Valid for x <= 126.
+__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& r0, float& r1) {
+  constexpr float kShifter = 12582912.f;  // 1.5 * 2^23
+  const uint64_t x = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t t = f2_add(x, f2_pack(kShifter, kShifter));
+  const uint64_t n = f2_add(t, f2_pack(-kShifter, -kShifter));
+  const uint64_t f = f2_fma(n, f2_pack(-1.f, -1.f), x);
+  uint64_t p = f2_fma(f2_pack(5.517166853e-02f, 5.517166853e-02f), f,
+                      f2_pack(2.426111251e-01f, 2.426111251e-01f));
+  p = f2_fma(p, f, f2_pack(6.932609677e-01f, 6.932609677e-01f));
+  p = f2_fma(p, f, f2_pack(9.999280572e-01f, 9.999280572e-01f));
+  float p0, p1, t0, t1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(t, t0, t1);
+  r0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+  r1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
 }
 
 // Pack two floats into one 32-bit word of two 16-bit values, `lo` in the
