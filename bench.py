@@ -49,11 +49,29 @@ KERNEL_SOURCES = ["io_aware_exact_33_b200/csrc/fwd_kernel.cuh",
 
 # ---------------------------------------------------------------- accounting
 def step_flops(w):
-    """(forward, backward) FLOPs of one pass by the formula convention."""
-    fwd = 4.0 * w.batch * w.nheads * w.seqlen_q * w.seqlen_k * w.headdim
-    if w.causal:
-        fwd /= 2.0
-    return fwd, 2.5 * fwd
+    """(forward, backward) FLOPs of one pass.  Without a window: the formula
+    convention (4*B*H*Nq*Nk*d, halved for causal).  With a sliding window the
+    halved-causal formula overstates the work, so the exact count of visible
+    (query, key) pairs times 4*d is used instead.  Backward = 2.5 x forward;
+    0 for forward-only workloads."""
+    if w.window_left >= 0 or w.window_right >= 0:
+        pairs = visible_pairs(w.seqlen_q, w.seqlen_k, w.causal, w.window_left, w.window_right)
+        fwd = 4.0 * w.batch * w.nheads * pairs * w.headdim
+    else:
+        fwd = 4.0 * w.batch * w.nheads * w.seqlen_q * w.seqlen_k * w.headdim
+        if w.causal:
+            fwd /= 2.0
+    return fwd, (2.5 * fwd if has_bwd(w) else 0.0)
+
+
+def has_bwd(w):
+    return "bwd" in w.passes
+
+
+def flops_convention(w):
+    if w.window_left >= 0 or w.window_right >= 0:
+        return "exact visible pairs x 4d (fwd), x 10d (bwd)"
+    return "4*B*H*N^2*d, halved for causal (fwd); bwd = 2.5 x fwd"
 
 
 def visible_pairs(nq, nk, causal, wl, wr, rows=None):
@@ -210,7 +228,7 @@ def oracle_sample(w, rows, heads):
     first = w.seqlen_q - rows
     pairs = visible_pairs(w.seqlen_q, w.seqlen_k, w.causal, w.window_left, w.window_right,
                           rows=range(first, w.seqlen_q))
-    flops = pairs * heads * (4.0 + 10.0) * w.headdim
+    flops = pairs * heads * (4.0 + (10.0 if has_bwd(w) else 0.0)) * w.headdim
     return (q_s, k_s, v_s, do_s), flops
 
 
@@ -218,7 +236,8 @@ def oracle_step(w, inputs):
     import oracle
     q, k, v, do = inputs
     oracle.attention_fwd(q, k, v, w.scale, w.causal, w.window_left, w.window_right)
-    oracle.attention_bwd(q, k, v, do, w.scale, w.causal, w.window_left, w.window_right)
+    if has_bwd(w):
+        oracle.attention_bwd(q, k, v, do, w.scale, w.causal, w.window_left, w.window_right)
 
 
 def cpu_baseline(w, target_s=12.0):
@@ -238,7 +257,7 @@ def cpu_baseline(w, target_s=12.0):
     oracle_step(w, inputs)
     dt = time.perf_counter() - t0
     return {"value": flops / dt / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
-            "sample": (f"float64 oracle fwd+bwd on the last {rows} queries of {heads} heads "
+            "sample": (f"float64 oracle {w.passes} on the last {rows} queries of {heads} heads "
                        f"(batch 0) against all {w.seqlen_k} keys of {w.name}; "
                        f"{flops / 1e9:.1f} GFLOP in {dt:.1f} s"),
             "seconds": dt}
@@ -251,7 +270,7 @@ def run_reference(args):
         return 0
     import oracle
     from attn_inputs import WORKLOADS
-    w = WORKLOADS[WORKLOAD]
+    w = WORKLOADS[args.workload]
     oracle.build()
     threads = oracle.num_threads()
     heads = max(1, min(w.nheads, threads))
@@ -264,7 +283,7 @@ def run_reference(args):
         oracle_step(w, inputs)
     dt = time.perf_counter() - t0
     value = flops * args.steps / dt / 1e12
-    sample = (f"float64 oracle fwd+bwd on the last {rows} queries of {heads} heads (batch 0) "
+    sample = (f"float64 oracle {w.passes} on the last {rows} queries of {heads} heads (batch 0) "
               f"against all {w.seqlen_k} keys of {w.name} per step")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
@@ -279,12 +298,27 @@ def run_reference(args):
     return 0
 
 
+def input_bytes(w):
+    """Bytes of the inputs one step reads (Q, K, V and, with a backward, dO)."""
+    es = 2
+    q = w.batch * w.seqlen_q * w.nheads * w.headdim * es
+    kv = 2 * w.batch * w.seqlen_k * w.nheads_kv * w.headdim * es
+    return q + kv + (q if has_bwd(w) else 0)
+
+
 def workload_config(w):
-    return {"workload": w.name, "batch": w.batch, "nheads": w.nheads, "nheads_kv": w.nheads_kv,
-            "seqlen": w.seqlen_q, "headdim": w.headdim, "causal": w.causal, "pass": "fwd+bwd",
-            "softmax_scale": w.scale, "inputs": "Q,K,V,dO ~ N(0,1), seed 1",
-            "l2": "no flush: inputs 0.54 GB per step exceed the 126 MB L2",
-            "parallelism": "replicas (weak scaling, no collective)"}
+    names = "Q,K,V,dO" if has_bwd(w) else "Q,K,V"
+    cfg = {"workload": w.name, "batch": w.batch, "nheads": w.nheads, "nheads_kv": w.nheads_kv,
+           "seqlen": w.seqlen_q, "headdim": w.headdim, "causal": w.causal, "pass": w.passes,
+           "dtype": w.dtype, "softmax_scale": w.scale,
+           "inputs": f"{names} ~ N(0,{w.sigma:g}^2), seed {w.seed}",
+           "l2": (f"no flush: inputs {input_bytes(w) / 1e9:.2f} GB per step exceed the "
+                  "126 MB L2"),
+           "flops": flops_convention(w),
+           "parallelism": "replicas (weak scaling, no collective)"}
+    if w.window_left >= 0 or w.window_right >= 0:
+        cfg["window"] = [w.window_left, w.window_right]
+    return cfg
 
 
 # ---------------------------------------------------------------- GPU arm
@@ -297,16 +331,19 @@ def run_gpu(args):
     dist = init_dist("nccl", world)
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    w = WORKLOADS[WORKLOAD]
+    w = WORKLOADS[args.workload]
     f_fwd, f_bwd = step_flops(w)
+    bwd = has_bwd(w)
 
-    q, k, v, do = make_inputs(w)
+    q, k, v, do = make_inputs(w, with_dout=bwd)
+    if do is None:
+        do = torch.empty(0, dtype=q.dtype)
     qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
     p = attn.params_for(qd, kd, w.scale, w.causal, w.window_left, w.window_right)
     o = torch.empty_like(qd)
     lse = torch.empty(w.batch, w.nheads, w.seqlen_q, dtype=torch.float32, device=dev)
-    dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
-    ws = torch.empty(attn.attn_bwd_workspace_size(p), dtype=torch.uint8, device=dev)
+    dq, dk, dv = (torch.empty_like(t) if bwd else None for t in (qd, kd, vd))
+    ws = torch.empty(attn.attn_bwd_workspace_size(p) if bwd else 0, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     nev = 5
@@ -316,6 +353,8 @@ def run_gpu(args):
         if ev: ev[0].record(stream)
         attn.attn_fwd(qd, kd, vd, w.scale, w.causal, w.window_left, w.window_right, out=o, lse=lse)
         if ev: ev[1].record(stream)
+        if not bwd:
+            return
         attn.attn_bwd_prepare(p, o, lse, dod, ws)
         if ev: ev[2].record(stream)
         attn.attn_bwd_accumulate(p, qd, kd, vd, dod, dk, dv, ws)
@@ -323,7 +362,7 @@ def run_gpu(args):
         attn.attn_bwd_finalize(p, dq, ws)
         if ev: ev[4].record(stream)
 
-    launches_per_step = 4
+    launches_per_step = 4 if bwd else 1
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
@@ -343,26 +382,28 @@ def run_gpu(args):
     ms_local = start.elapsed_time(end)
     ms = max_over_ranks(ms_local, dist, dev)
     t_fwd = [e[0].elapsed_time(e[1]) for e in events]
-    t_prep = [e[1].elapsed_time(e[2]) for e in events]
-    t_main = [e[2].elapsed_time(e[3]) for e in events]
-    t_fin = [e[3].elapsed_time(e[4]) for e in events]
+    t_prep = [e[1].elapsed_time(e[2]) for e in events] if bwd else [0.0]
+    t_main = [e[2].elapsed_time(e[3]) for e in events] if bwd else [0.0]
+    t_fin = [e[3].elapsed_time(e[4]) for e in events] if bwd else [0.0]
     value = (f_fwd + f_bwd) * args.steps * world / (ms / 1e3) / 1e12
 
     # end to end through the public API with pinned host buffers
     k_e2e = max(1, min(args.steps, args.e2e_steps))
     hq, hk, hv, hdo = (t.pin_memory() for t in (q, k, v, do))
     ho, hlse = torch.empty_like(hq).pin_memory(), torch.empty(lse.shape, dtype=torch.float32).pin_memory()
-    hdq, hdk, hdv = (torch.empty_like(t).pin_memory() for t in (hq, hk, hv))
+    hdq, hdk, hdv = ((torch.empty_like(t).pin_memory() for t in (hq, hk, hv)) if bwd
+                     else (None, None, None))
+    h2d_pairs = [(qd, hq), (kd, hk), (vd, hv)] + ([(dod, hdo)] if bwd else [])
+    d2h_pairs = [(ho, o), (hlse, lse)] + ([(hdq, dq), (hdk, dk), (hdv, dv)] if bwd else [])
 
     def e2e_step():
-        qd.copy_(hq, non_blocking=True)
-        kd.copy_(hk, non_blocking=True)
-        vd.copy_(hv, non_blocking=True)
-        dod.copy_(hdo, non_blocking=True)
+        for dst, src in h2d_pairs:
+            dst.copy_(src, non_blocking=True)
         attn.attn_fwd(qd, kd, vd, w.scale, w.causal, w.window_left, w.window_right, out=o, lse=lse)
-        attn.attn_bwd(qd, kd, vd, o, lse, dod, w.scale, w.causal, w.window_left, w.window_right,
-                      dq=dq, dk=dk, dv=dv, workspace=ws)
-        for dst, src in ((ho, o), (hlse, lse), (hdq, dq), (hdk, dk), (hdv, dv)):
+        if bwd:
+            attn.attn_bwd(qd, kd, vd, o, lse, dod, w.scale, w.causal, w.window_left,
+                          w.window_right, dq=dq, dk=dk, dv=dv, workspace=ws)
+        for dst, src in d2h_pairs:
             dst.copy_(src, non_blocking=True)
 
     e2e_step()
@@ -376,8 +417,8 @@ def run_gpu(args):
     torch.cuda.synchronize(dev)
     barrier(dist, dev)
     ms_e2e = max_over_ranks(s2.elapsed_time(e2), dist, dev)
-    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
-    d2h = sum(t.numel() * t.element_size() for t in (ho, hlse, hdq, hdk, hdv))
+    h2d = sum(t.numel() * t.element_size() for _, t in h2d_pairs)
+    d2h = sum(t.numel() * t.element_size() for t, _ in d2h_pairs)
     status = attn.attn_get_device_status()
 
     if rank != 0:
@@ -387,10 +428,9 @@ def run_gpu(args):
 
     peaks, peak_kind = load_peaks()
     mean = lambda xs: sum(xs) / len(xs)
-    kernels = {
-        "attn_fwd_kernel": {"ms": mean(t_fwd), "flops": f_fwd},
-        "attn_bwd_kernel": {"ms": mean(t_main), "flops": f_bwd},
-    }
+    kernels = {"attn_fwd_kernel": {"ms": mean(t_fwd), "flops": f_fwd}}
+    if bwd:
+        kernels["attn_bwd_kernel"] = {"ms": mean(t_main), "flops": f_bwd}
     dominant = max(kernels, key=lambda n: kernels[n]["ms"])
     rl = {}
     for name, kk in kernels.items():
@@ -407,14 +447,15 @@ def run_gpu(args):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (Q,K,V,dO ~ N(0,1), seed 1)",
+        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": f"synthetic ({workload_config(w)['inputs']})",
         "config": workload_config(w),
         "pct_of_peak": {"measured_bf16": value / world / peaks["bf16_tflops"],
                         "nominal_2250": value / world / NOMINAL_BF16_TFLOPS,
                         "peak_source": peak_kind},
         "fwd_tflops": f_fwd / (mean(t_fwd) / 1e3) / 1e12,
-        "bwd_tflops": f_bwd / ((mean(t_prep) + mean(t_main) + mean(t_fin)) / 1e3) / 1e12,
+        "bwd_tflops": (f_bwd / ((mean(t_prep) + mean(t_main) + mean(t_fin)) / 1e3) / 1e12
+                       if bwd else None),
         "ms": {"fwd": mean(t_fwd), "bwd_prepare": mean(t_prep), "bwd_accumulate": mean(t_main),
                "bwd_finalize": mean(t_fin)},
         "roofline": dict(rl[dominant], kernel=dominant),
@@ -483,6 +524,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--workload", default=WORKLOAD,
+                    help=f"attn_inputs workload to time (default {WORKLOAD}, the headline)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--probe-mma", action="store_true",
                     help="measure tcgen05.mma throughput by shape instead of the attention step")
@@ -492,6 +535,11 @@ def main(argv=None):
         return 0
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    from attn_inputs import WORKLOADS
+    if args.workload not in WORKLOADS:
+        ap.error(f"unknown workload {args.workload}; choose from {sorted(WORKLOADS)}")
+    if input_bytes(WORKLOADS[args.workload]) < 2 * 126e6:
+        ap.error(f"{args.workload} fits in L2; it is a parity case, not a bench workload")
     if args.impl == "reference":
         return run_reference(args)
     return run_gpu(args)
