@@ -2,6 +2,7 @@
 // argument checks, TMA tensor-map construction, kernel selection and launch.
 // Every computation of the attention path runs in the kernels; this file
 // only marshals arguments.
+#include <climits>
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
@@ -105,6 +106,16 @@ bool ensure_smem(const void* kernel, int bytes) {
   return true;
 }
 
+// Heads per scheduling group (grouped_lpt): as many as keep the tiles they
+// share within this share of the 126 MB L2.
+constexpr double kL2GroupBudget = 64.0 * 1024 * 1024;
+int l2_group(double bytes_per_head, int heads) {
+  double g = bytes_per_head > 0 ? kL2GroupBudget / bytes_per_head : heads;
+  if (g < 1) g = 1;
+  if (g > heads) g = heads;
+  return heads > 0 ? (int)g : 1;
+}
+
 bool debug_status_enabled() {
   static int v = -1;
   if (v < 0) {
@@ -180,10 +191,14 @@ attn_status launch_fwd(const attn_params* p, const void* q, const void* k, const
   fp.window_right = p->window_right;
   fp.scale_log2 = p->softmax_scale * 1.4426950408889634f;
   fp.num_qblocks = (p->seqlen_q + FwdLaunch<C>::rows_per_cta - 1) / FwdLaunch<C>::rows_per_cta;
+  const int heads = p->batch * p->nheads;
+  // K and V bytes each query head streams (its kv head's, shared by the group)
+  fp.sched_group = l2_group(4.0 * p->seqlen_k * C::D / (p->nheads / p->nheads_kv), heads);
+  const long long blocks = (long long)fp.num_qblocks * heads;
+  if (blocks > INT_MAX) return ATTN_ERR_INVALID_ARG;
   auto kern = FwdLaunch<C>::kernel();
   if (!ensure_smem(reinterpret_cast<const void*>(kern), C::SMEM_BYTES)) return ATTN_ERR_CUDA;
-  dim3 grid(fp.num_qblocks, p->nheads, p->batch);
-  kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mo, fp);
+  kern<<<(unsigned)blocks, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mo, fp);
   return finish(stream);
 }
 
@@ -243,10 +258,18 @@ attn_status launch_bwd_main(const attn_params* p, const void* q, const void* k, 
       !map_bshd(&mdv, dv, fp16, p->batch, p->seqlen_k, p->nheads_kv, C::D, C::BN) ||
       !map_bshd_f32_32x32(&mdq, bp.dq_acc, p->batch, p->seqlen_q, p->nheads, C::D))
     return ATTN_ERR_CUDA;
+  BwdParams bpl = bp;
+  bpl.num_kblocks = (p->seqlen_k + C::BN - 1) / C::BN;
+  const int heads = p->batch * p->nheads_kv;
+  // bytes of Q, dO (16-bit) and the fp32 dQ accumulator each kv head's
+  // key tiles share: all query heads of its group
+  bpl.sched_group = l2_group(8.0 * p->seqlen_q * C::D * (p->nheads / p->nheads_kv), heads);
+  const long long blocks = (long long)bpl.num_kblocks * heads;
+  if (blocks > INT_MAX) return ATTN_ERR_INVALID_ARG;
   auto kern = attn_bwd_kernel<C>;
   if (!ensure_smem(reinterpret_cast<const void*>(kern), C::SMEM_BYTES)) return ATTN_ERR_CUDA;
-  dim3 grid((p->seqlen_k + C::BN - 1) / C::BN, p->nheads_kv, p->batch);
-  kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, ml, md, mdk, mdv, mdq, bp);
+  kern<<<(unsigned)blocks, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, ml, md, mdk,
+                                                                 mdv, mdq, bpl);
   return finish(stream);
 }
 

@@ -75,6 +75,8 @@ struct BwdParams {
   float scale_log2;
   float softmax_scale;
   long long nq_pad;
+  int num_kblocks;   // key tiles per (batch, kv head): the work units
+  int sched_group;   // kv heads per scheduling group (grouped_lpt)
 };
 
 // ------------------------------------------------------------ preprocess
@@ -222,7 +224,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   volatile uint32_t* tmem_ptr_slot = reinterpret_cast<volatile uint32_t*>(smem_gen + C::OFF_TMEMPTR);
 
   const uint32_t warp = warp_id(), lane = lane_id();
-  const int kblock = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  // earlier key tiles are seen by more queries under a causal mask: heaviest
+  // first
+  const UnitOrder uo = grouped_lpt((int)blockIdx.x, p.num_kblocks, p.batch * p.nheads_kv,
+                                   p.sched_group);
+  const int kblock = uo.rank, kvh = uo.head % p.nheads_kv, b = uo.head / p.nheads_kv;
   const int group = p.nheads / p.nheads_kv;
   const int k0 = kblock * BN;
   const int k1 = min(k0 + BN, p.seqlen_k);
@@ -291,7 +297,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && nt > 0) {
+    // The whole warp runs the issue loop (its values stay warp-uniform); one
+    // elected lane issues each MMA and commit.
+    if (nt > 0) {
       constexpr uint32_t idesc_s = idesc_f16(BN, BM, C::FP16, false, false);
       constexpr uint32_t idesc_acc = idesc_f16(BN, D, C::FP16, false, true);
       constexpr uint32_t idesc_dq =
@@ -305,31 +313,31 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       auto issue_s = [&](int u) -> bool {
         const int slot = u % QS, bf = u % NBUF;
         const uint64_t q_desc = sdesc_sw128(smem0 + C::OFF_Q + slot * C::Q_BYTES, 16, 1024);
-        if (!mbar_wait(bar(C::B_QFULL + slot), (u / QS) & 1)) return false;
+        if (!mbar_wait_warp(bar(C::B_QFULL + slot), (u / QS) & 1)) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int bx = kk / 4, w = kk % 4;
-          mma_ss(tmem + C::TM_S + bf * BM, desc_at(k_kdesc, bx * (BN * 128) + w * 32),
+          mma_ss_warp(tmem + C::TM_S + bf * BM, desc_at(k_kdesc, bx * (BN * 128) + w * 32),
                  desc_at(q_desc, bx * (BM * 128) + w * 32), idesc_s, kk > 0);
         }
-        mma_commit(bar(C::B_SFULL + bf));
+        mma_commit_warp(bar(C::B_SFULL + bf));
         return true;
       };
       // dP^T_u = V dO_u^T into the dP block, once tile u - NBUF's dQ left it.
       auto issue_dp = [&](int u) -> bool {
         const int slot = u % QS, bf = u % NBUF, use = u / NBUF;
         const uint64_t do_desc = sdesc_sw128(smem0 + C::OFF_DO + slot * C::Q_BYTES, 16, 1024);
-        if (use > 0 && !mbar_wait(bar(C::B_DQFREE + bf), (use - 1) & 1)) return false;
-        if (!mbar_wait(bar(C::B_DOFULL + slot), (u / QS) & 1)) return false;
+        if (use > 0 && !mbar_wait_warp(bar(C::B_DQFREE + bf), (use - 1) & 1)) return false;
+        if (!mbar_wait_warp(bar(C::B_DOFULL + slot), (u / QS) & 1)) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int bx = kk / 4, w = kk % 4;
-          mma_ss(tmem + C::TM_DP + bf * BM, desc_at(v_kdesc, bx * (BN * 128) + w * 32),
+          mma_ss_warp(tmem + C::TM_DP + bf * BM, desc_at(v_kdesc, bx * (BN * 128) + w * 32),
                  desc_at(do_desc, bx * (BM * 128) + w * 32), idesc_s, kk > 0);
         }
-        mma_commit(bar(C::B_DPFULL + bf));
+        mma_commit_warp(bar(C::B_DPFULL + bf));
         return true;
       };
       // dV += P^T dO, dK += dS^T Q and tile t's dQ share.
@@ -340,52 +348,49 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         const uint32_t ds_base = smem0 + C::OFF_DS + bf * C::DS_BYTES;
         const uint64_t ds_k = sdesc_sw128(ds_base, 16, 1024);
         const uint64_t ds_mn = sdesc_sw128(ds_base, BN * 128, 1024);
-        if (!mbar_wait(bar(C::B_PREADY + bf), use & 1)) return false;
+        if (!mbar_wait_warp(bar(C::B_PREADY + bf), use & 1)) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk) {
           // P^T from tensor memory: each half of the query columns keeps its
           // packed values at the start of its own score columns.
           const int half = kk / (C::HW / 16), part = kk % (C::HW / 16);
-          mma_ts(tmem + C::TM_DV, tmem + C::TM_S + bf * BM + half * C::HW + part * 8,
+          mma_ts_warp(tmem + C::TM_DV, tmem + C::TM_S + bf * BM + half * C::HW + part * 8,
                  desc_at(do_mn, kk * 2048), idesc_acc, (t > 0 || kk > 0));
         }
-        if (!mbar_wait(bar(C::B_DSREADY + bf), use & 1)) return false;
+        if (!mbar_wait_warp(bar(C::B_DSREADY + bf), use & 1)) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk) {  // dS^T as a K-major smem operand; Q MN-major
           const int bx = kk / 4, w = kk % 4;
-          mma_ss(tmem + C::TM_DK, desc_at(ds_k, bx * (BN * 128) + w * 32),
+          mma_ss_warp(tmem + C::TM_DK, desc_at(ds_k, bx * (BN * 128) + w * 32),
                  desc_at(q_mn, kk * 2048), idesc_acc, (t > 0 || kk > 0));
         }
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
           if constexpr (C::DQT)  // dQ^T = K^T dS^T: both operands MN-major
-            mma_ss(tmem + C::TM_DP + bf * BM, desc_at(k_mndesc, kk * 2048),
+            mma_ss_warp(tmem + C::TM_DP + bf * BM, desc_at(k_mndesc, kk * 2048),
                    desc_at(ds_mn, kk * 2048), idesc_dq, kk > 0);
           else  // dQ = dS K
-            mma_ss(tmem + C::TM_DP + bf * BM, desc_at(ds_mn, kk * 2048),
+            mma_ss_warp(tmem + C::TM_DP + bf * BM, desc_at(ds_mn, kk * 2048),
                    desc_at(k_mndesc, kk * 2048), idesc_dq, kk > 0);
         }
-        mma_commit(bar(C::B_DQFULL + bf));
-        mma_commit(bar(C::B_DSFREE + bf));
-        mma_commit(bar(C::B_EMPTY + slot));
+        mma_commit_warp(bar(C::B_DQFULL + bf));
+        mma_commit_warp(bar(C::B_DSFREE + bf));
+        mma_commit_warp(bar(C::B_EMPTY + slot));
         return true;
       };
-      // Two buffers: S^T_{t+1} goes in before tile t's gradient MMAs, dP^T_{t+1}
-      // after them (its block holds tile t-1's dQ until that is read out).
-      // One buffer: everything of tile t first.
       // Two buffers: tile t+1's S^T and dP^T go in before tile t's gradient
       // MMAs (the dP block of t+1 is released when the compute warps drain
       // tile t-1's dQ, midway through tile t).  One buffer: tile t first.
-      bool ok = mbar_wait(bar(C::B_KV), 0) && issue_s(0) && issue_dp(0);
+      bool ok = mbar_wait_warp(bar(C::B_KV), 0) && issue_s(0) && issue_dp(0);
       for (int t = 0; ok && t < nt; ++t) {
         const bool more = t + 1 < nt;
         if (NBUF == 2 && more && !(issue_s(t + 1) && issue_dp(t + 1))) { ok = false; break; }
         if (!issue_grads(t)) { ok = false; break; }
         if (NBUF == 1 && more && !(issue_s(t + 1) && issue_dp(t + 1))) { ok = false; break; }
       }
-      if (ok) mma_commit(bar(C::B_DONE));
+      if (ok) mma_commit_warp(bar(C::B_DONE));
     }
   } else if (warp < 8) {
     // ------------------------------------------------------------ P, dS, dQ out
@@ -592,8 +597,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       }
       bulk_commit_group();
     }
-    // every warp's dQ reduces (and the dK/dV stores) complete before exit
-    if (lane == 0) bulk_wait_group_all();
+    // every warp's dQ reduces (and the dK/dV stores) have read their shared
+    // memory before exit
+    if (lane == 0) bulk_wait_group_read_all();
   }
   tc_fence_before();
   __syncthreads();

@@ -34,7 +34,8 @@ struct FwdParams {
   int batch, nheads, nheads_kv, seqlen_q, seqlen_k;
   int causal, window_left, window_right;
   float scale_log2;  // softmax_scale * log2(e)
-  int num_qblocks;
+  int num_qblocks;   // work units per (batch, head): query tiles or tile pairs
+  int sched_group;   // heads per scheduling group (grouped_lpt)
 };
 
 // Range of visible key positions for query rows [q0, q1): keys [jmin, jmax].
@@ -99,8 +100,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   volatile uint32_t* tmem_ptr_slot = reinterpret_cast<volatile uint32_t*>(smem_gen + C::OFF_TMEMPTR);
 
   const uint32_t warp = warp_id(), lane = lane_id();
-  const int qblock = p.num_qblocks - 1 - (int)blockIdx.x;  // heaviest causal tiles first
-  const int h = blockIdx.y, b = blockIdx.z;
+  // later query tiles see more keys under a causal mask: heaviest first
+  const UnitOrder uo = grouped_lpt((int)blockIdx.x, p.num_qblocks, p.batch * p.nheads,
+                                   p.sched_group);
+  const int qblock = p.num_qblocks - 1 - uo.rank;
+  const int h = uo.head % p.nheads, b = uo.head / p.nheads;
   const int kvh = h / (p.nheads / p.nheads_kv);
   const int q0 = qblock * BM;
   const int q1 = min(q0 + BM, p.seqlen_q);
@@ -159,14 +163,15 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     }
   } else if (warp == 5) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && nt > 0) {
+    // The whole warp runs the issue loop; one elected lane issues.
+    if (nt > 0) {
       constexpr uint32_t idesc_qk = idesc_f16(BM, BN, C::FP16, false, false);
       constexpr uint32_t idesc_pv = idesc_f16(BM, D, C::FP16, false, true);
-      bool ok = mbar_wait(bar(C::B_Q), 0);
+      bool ok = mbar_wait_warp(bar(C::B_Q), 0);
       auto issue_pv = [&](int u) -> bool {
         const int st = u % STAGES, buf = u & 1;
-        if (!mbar_wait(bar(C::B_PREADY + buf), (u >> 1) & 1)) return false;
-        if (!mbar_wait(bar(C::B_VFULL + st), (u / STAGES) & 1)) return false;
+        if (!mbar_wait_warp(bar(C::B_PREADY + buf), (u >> 1) & 1)) return false;
+        if (!mbar_wait_warp(bar(C::B_VFULL + st), (u / STAGES) & 1)) return false;
         tc_fence_after();
         const uint32_t v_base = smem0 + C::OFF_V + st * C::KV_BYTES;
         const uint32_t p_tmem = tmem + (buf ? C::TM_S1 : C::TM_S0);
@@ -176,15 +181,15 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
           const uint64_t bdesc = desc_at(v_desc, kk * 2048);
-          mma_ts(tmem + C::TM_O, p_tmem + kk * 8, bdesc, idesc_pv, (u > 0 || kk > 0) ? 1u : 0u);
+          mma_ts_warp(tmem + C::TM_O, p_tmem + kk * 8, bdesc, idesc_pv, (u > 0 || kk > 0) ? 1u : 0u);
         }
-        mma_commit(bar(C::B_OREADY));
-        mma_commit(bar(C::B_EMPTY + st));
+        mma_commit_warp(bar(C::B_OREADY));
+        mma_commit_warp(bar(C::B_EMPTY + st));
         return true;
       };
       for (int t = 0; ok && t < nt; ++t) {
         const int st = t % STAGES, buf = t & 1;
-        if (!mbar_wait(bar(C::B_KFULL + st), (t / STAGES) & 1)) { ok = false; break; }
+        if (!mbar_wait_warp(bar(C::B_KFULL + st), (t / STAGES) & 1)) { ok = false; break; }
         tc_fence_after();
         const uint32_t s_tmem = tmem + (buf ? C::TM_S1 : C::TM_S0);
         const uint64_t q_desc = sdesc_sw128(smem0 + C::OFF_Q, 16, 1024);
@@ -196,9 +201,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           const int bx = kk / 4, w = kk % 4;
           const uint64_t adesc = desc_at(q_desc, bx * (BM * 128) + w * 32);
           const uint64_t bdesc = desc_at(k_desc, bx * (BN * 128) + w * 32);
-          mma_ss(s_tmem, adesc, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
+          mma_ss_warp(s_tmem, adesc, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
         }
-        mma_commit(bar(C::B_SFULL + buf));
+        mma_commit_warp(bar(C::B_SFULL + buf));
         if (t >= 1 && !issue_pv(t - 1)) { ok = false; break; }
       }
       if (ok) issue_pv(nt - 1);
@@ -334,7 +339,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       for (int bx = 0; bx < C::NBOX; ++bx)
         tma_store_4d(&tm_o, smem0 + C::OFF_Q + bx * (BM * 128), bx * 64, h, q0, b);
       bulk_commit_group();
-      bulk_wait_group_all();
+      bulk_wait_group_read_all();
     }
   }
   tc_fence_before();
@@ -520,8 +525,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   volatile uint32_t* tmem_ptr_slot = reinterpret_cast<volatile uint32_t*>(smem_gen + C::OFF_TMEMPTR);
 
   const uint32_t warp = warp_id(), lane = lane_id();
-  const int pair = p.num_qblocks - 1 - (int)blockIdx.x;  // heaviest causal pairs first
-  const int h = blockIdx.y, b = blockIdx.z;
+  // later query tiles see more keys under a causal mask: heaviest first
+  const UnitOrder uo = grouped_lpt((int)blockIdx.x, p.num_qblocks, p.batch * p.nheads,
+                                   p.sched_group);
+  const int pair = p.num_qblocks - 1 - uo.rank;
+  const int h = uo.head % p.nheads, b = uo.head / p.nheads;
   const int kvh = h / (p.nheads / p.nheads_kv);
 
   // Key-tile range [lo_i, hi_i) of each query tile; union [ulo, uhi).
@@ -607,7 +615,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && nt > 0) {
+    // The whole warp runs the issue loop (its values stay warp-uniform); one
+    // elected lane issues each MMA and commit.
+    if (nt > 0) {
       constexpr uint32_t idesc_qk = idesc_f16(BM, BN, C::FP16, false, false);
       constexpr uint32_t idesc_pv = idesc_f16(BM, D, C::FP16, false, true);
       int ns[2] = {0, 0};  // S MMAs issued per query tile
@@ -620,38 +630,38 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int bx = kk / 4, w = kk % 4;
-          mma_ss(tmem + C::TM_S + i * BN, desc_at(q_desc, bx * (BM * 128) + w * 32),
+          mma_ss_warp(tmem + C::TM_S + i * BN, desc_at(q_desc, bx * (BM * 128) + w * 32),
                  desc_at(k_desc, bx * (BN * 128) + w * 32), idesc_qk, kk > 0);
         }
-        mma_commit(bar(C::B_SFULL + i));
-        if (last_use) mma_commit(bar(C::B_KEMPTY + st));
+        mma_commit_warp(bar(C::B_SFULL + i));
+        if (last_use) mma_commit_warp(bar(C::B_KEMPTY + st));
         ++ns[i];
       };
       // O_i += P_i V_j in two halves of the key tile, each issued as soon as
       // the softmax warps have stored that half of P.
       auto issue_pv = [&](int i, int j, bool last_use) -> bool {
         const int u = j - ulo, st = u % VS;
-        if (!mbar_wait(bar(C::B_VFULL + st), (u / VS) & 1)) return false;
+        if (!mbar_wait_warp(bar(C::B_VFULL + st), (u / VS) & 1)) return false;
         const uint64_t v_desc = sdesc_sw128(smem0 + C::OFF_V + st * C::KV_BYTES, BN * 128, 1024);
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
-          if (!mbar_wait(bar(C::B_PREADY + 2 * i + hf), np[i] & 1)) return false;
+          if (!mbar_wait_warp(bar(C::B_PREADY + 2 * i + hf), np[i] & 1)) return false;
           tc_fence_after();
 #pragma unroll
           for (int kk = hf * (BN / 32); kk < (hf + 1) * (BN / 32); ++kk)
-            mma_ts(tmem + C::TM_O + i * D, tmem + C::TM_S + i * BN + kk * 8,
+            mma_ts_warp(tmem + C::TM_O + i * D, tmem + C::TM_S + i * BN + kk * 8,
                    desc_at(v_desc, kk * 2048), idesc_pv,
                    (np[i] > 0 || kk > 0) ? 1u : 0u);
         }
-        mma_commit(bar(C::B_OREADY + i));
-        if (last_use) mma_commit(bar(C::B_VEMPTY + st));
+        mma_commit_warp(bar(C::B_OREADY + i));
+        if (last_use) mma_commit_warp(bar(C::B_VEMPTY + st));
         ++np[i];
         return true;
       };
-      bool ok = mbar_wait(bar(C::B_Q), 0);
+      bool ok = mbar_wait_warp(bar(C::B_Q), 0);
       for (int j = ulo; ok && j < uhi; ++j) {
         const int u = j - ulo, st = u % KS;
-        if (!mbar_wait(bar(C::B_KFULL + st), (u / KS) & 1)) { ok = false; break; }
+        if (!mbar_wait_warp(bar(C::B_KFULL + st), (u / KS) & 1)) { ok = false; break; }
         tc_fence_after();
         if (in(0, j)) issue_s(0, j, !in(1, j));
         if (j > ulo && in(1, j - 1) && !issue_pv(1, j - 1, true)) { ok = false; break; }
@@ -749,7 +759,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       for (int bx = 0; bx < C::NBOX; ++bx)
         tma_store_4d(&tm_o, stage + bx * (BM * 128), bx * 64, h, q_i, b);
       bulk_commit_group();
-      bulk_wait_group_all();
+      bulk_wait_group_read_all();
     }
   }
   tc_fence_before();

@@ -37,6 +37,26 @@ __device__ __forceinline__ uint32_t warp_id() {
   return __shfl_sync(0xffffffffu, threadIdx.x >> 5, 0);
 }
 
+// ---------------------------------------------------------------- work order
+// Order of a grid's work units: `units` per head (rank 0 = the heaviest) for
+// `heads` heads, in groups of `group` heads.  Within a group, all heads' rank-0
+// units come first, then all rank-1 units, and so on (longest processing time
+// first, so the lightest units fill the tail); groups follow one another, so
+// only about one group's heads are in flight at a time and the tiles those
+// heads share stay in L2.  Returns the unit's rank and head for linear block
+// index `L` in [0, units * heads).
+struct UnitOrder {
+  int rank, head;
+};
+__device__ __forceinline__ UnitOrder grouped_lpt(int L, int units, int heads, int group) {
+  const int per_group = group * units;
+  const int g = L / per_group;
+  const int g0 = g * group;
+  const int gsize = min(group, heads - g0);
+  const int idx = L - g * per_group;
+  return {idx / gsize, g0 + idx % gsize};
+}
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
@@ -229,6 +249,35 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// Warp-wide forms: every lane of a converged warp executes them (so the
+// operands can stay in the warp's uniform registers) and one lane, chosen by
+// elect.sync, issues the instruction.  With the full mask the same lane is
+// elected each time, so its commits track its own MMAs.
+__device__ __forceinline__ void mma_ss_warp(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_ts_warp(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit_warp(uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(bar)
+      : "memory");
+}
+
 // Arrive once on `bar` when every tcgen05 operation issued so far by this
 // thread has completed.
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
