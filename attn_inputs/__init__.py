@@ -94,6 +94,39 @@ def make_inputs(w: Workload, with_dout: bool = True, device: str = "cpu"):
     return q, k, v, dout
 
 
+def make_varlen_inputs(lens_q, lens_k, nheads: int, nheads_kv: int, headdim: int,
+                       dtype: str = "bf16", sigma: float = 1.0, seed: int = 0,
+                       with_dout: bool = True, extra_q: int = 0, extra_k: int = 0):
+    """Packed variable-length inputs: sequence b has ``lens_q[b]`` query and
+    ``lens_k[b]`` key rows, stored back to back.  Returns (q (Tq, H, d),
+    k, v (Tk, Hkv, d), dout (Tq, H, d) or None, cu_q, cu_k) with int32 offsets
+    of len(lens) + 1 entries; ``extra_q`` / ``extra_k`` rows past the last
+    sequence belong to none.  Drawn like ``make_inputs``: one generator seeded
+    with ``seed``, in the order Q, K, V, dO, float32 randn * sigma rounded to
+    the storage dtype."""
+    if len(lens_q) != len(lens_k):
+        raise ValueError("lens_q and lens_k must have one entry per sequence")
+    cu_q = [0]
+    cu_k = [0]
+    for a, b in zip(lens_q, lens_k):
+        cu_q.append(cu_q[-1] + int(a))
+        cu_k.append(cu_k[-1] + int(b))
+    tq, tk = cu_q[-1] + int(extra_q), cu_k[-1] + int(extra_k)
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    dt = DTYPES[dtype]
+
+    def draw(*shape):
+        return (torch.randn(*shape, generator=g, dtype=torch.float32) * sigma).to(dt)
+
+    q = draw(tq, nheads, headdim)
+    k = draw(tk, nheads_kv, headdim)
+    v = draw(tk, nheads_kv, headdim)
+    dout = draw(tq, nheads, headdim) if with_dout else None
+    return (q, k, v, dout, torch.tensor(cu_q, dtype=torch.int32),
+            torch.tensor(cu_k, dtype=torch.int32))
+
+
 def sample_rows(n: int, count: int, seed: int, must=()) -> torch.Tensor:
     """A sorted, duplicate-free set of row indices in [0, n): the first and
     last rows, any ``must`` rows, and ``count`` more drawn from ``seed``."""

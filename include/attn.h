@@ -175,6 +175,72 @@ ATTN_API attn_status attn_bwd_noalloc(const attn_params* p, const void* q, const
                                       const void* dout, void* dq, void* dk, void* dv,
                                       void* stream);
 
+/* ------------------------------------------------------------------ packed
+ * Variable-length sequences packed back to back (the varlen interface named
+ * on "FlashAttention-2：下一代高效注意力机制的突破与实战解析", section
+ * "实操落地", and the inference-with-cache use of "FlashAttention 四代演进",
+ * interface section).  Each sequence is an independent attention problem
+ * with the masks of attn_params applied with its own lengths (bottom-right
+ * alignment when its query and key lengths differ).
+ *
+ * Layout: sequence b owns rows [cu_seqlens_q[b], cu_seqlens_q[b+1]) of q, o,
+ * dout, dq, each a (total_q, nheads, headdim) 16-bit tensor, and rows
+ * [cu_seqlens_k[b], cu_seqlens_k[b+1]) of k, v, dk, dv, each
+ * (total_k, nheads_kv, headdim).  lse is fp32 (nheads, total_q), natural log.
+ * cu_seqlens_q / cu_seqlens_k are DEVICE arrays of batch + 1 int32 offsets,
+ * non-decreasing from 0 to total_q / total_k; every sequence must be at most
+ * max_seqlen_q / max_seqlen_k long.  The offsets are read only by the
+ * kernels (no host synchronisation): values outside [0, total] are clamped,
+ * so a malformed array gives unspecified results but no access outside the
+ * tensors.  Tiles of one sequence may read rows of its neighbours (masked to
+ * zero weight), so inputs must be finite.
+ */
+typedef struct {
+  int32_t batch;          /* number of sequences */
+  int32_t total_q;        /* rows of q, o, dout, dq */
+  int32_t total_k;        /* rows of k, v, dk, dv */
+  int32_t max_seqlen_q;   /* >= every query sequence length */
+  int32_t max_seqlen_k;   /* >= every key sequence length */
+  int32_t nheads;
+  int32_t nheads_kv;
+  int32_t headdim;
+  int32_t dtype;          /* attn_dtype */
+  float softmax_scale;
+  int32_t causal;
+  int32_t window_left;
+  int32_t window_right;
+} attn_varlen_params;
+
+/* Host-side checks of a packed call (pass 0 forward, 1 backward): the
+ * attn_params rules with batch, max_seqlen_q/k as the sizes, and
+ * non-negative totals.  Pointers and offsets are not inspected. */
+ATTN_API attn_status attn_check_varlen_params(const attn_varlen_params* p, int pass);
+
+/* Forward over packed sequences; needs no workspace (the arguments are
+ * accepted for symmetry).  Asynchronous on `stream`.  A sequence with no
+ * keys gets O = 0 and LSE = -inf; rows of q not covered by any sequence are
+ * left untouched.  Errors as attn_fwd, plus ATTN_ERR_MISALIGNED for offset
+ * arrays that are not 4-byte aligned. */
+ATTN_API attn_status attn_fwd_varlen(const attn_varlen_params* p, const int32_t* cu_seqlens_q,
+                                     const int32_t* cu_seqlens_k, const void* q, const void* k,
+                                     const void* v, void* o, float* lse, void* workspace,
+                                     size_t workspace_bytes, void* stream);
+
+/* Bytes of the caller-owned device workspace attn_bwd_varlen needs:
+ * per-query statistics and an fp32 dQ accumulator over total_q rows plus
+ * 136 rows of padding per sequence.  0 for invalid parameters. */
+ATTN_API size_t attn_bwd_varlen_workspace_size(const attn_varlen_params* p);
+
+/* Backward over packed sequences: dq, dk, dv (layouts as above) from the
+ * forward's o and lse and the output gradient dout.  headdim 64 or 128.
+ * The workspace (256-byte aligned, at least attn_bwd_varlen_workspace_size
+ * bytes) is overwritten.  Asynchronous on `stream`; errors as attn_bwd. */
+ATTN_API attn_status attn_bwd_varlen(const attn_varlen_params* p, const int32_t* cu_seqlens_q,
+                                     const int32_t* cu_seqlens_k, const void* q, const void* k,
+                                     const void* v, const void* o, const float* lse,
+                                     const void* dout, void* dq, void* dk, void* dv,
+                                     void* workspace, size_t workspace_bytes, void* stream);
+
 /* Bytes of device workspace attn_fwd / attn_bwd need for these parameters
  * (0 when none).  Pure host functions; never touch the GPU. */
 ATTN_API size_t attn_fwd_workspace_size(const attn_params* p);

@@ -29,7 +29,8 @@ STATUS = {
 EXPORTED = ("attn_fwd", "attn_bwd", "attn_bwd_prepare", "attn_bwd_accumulate", "attn_bwd_finalize",
             "attn_fwd_workspace_size", "attn_bwd_workspace_size", "attn_check_params",
             "attn_status_string", "attn_get_device_status", "attn_version", "attn_bwd_noalloc",
-            "attn_selftest_bounded_wait")
+            "attn_selftest_bounded_wait", "attn_check_varlen_params", "attn_fwd_varlen",
+            "attn_bwd_varlen_workspace_size", "attn_bwd_varlen")
 
 
 class AttnParams(ctypes.Structure):
@@ -38,6 +39,25 @@ class AttnParams(ctypes.Structure):
         ("batch", ctypes.c_int32),
         ("seqlen_q", ctypes.c_int32),
         ("seqlen_k", ctypes.c_int32),
+        ("nheads", ctypes.c_int32),
+        ("nheads_kv", ctypes.c_int32),
+        ("headdim", ctypes.c_int32),
+        ("dtype", ctypes.c_int32),
+        ("softmax_scale", ctypes.c_float),
+        ("causal", ctypes.c_int32),
+        ("window_left", ctypes.c_int32),
+        ("window_right", ctypes.c_int32),
+    ]
+
+
+class AttnVarlenParams(ctypes.Structure):
+    """Mirror of ``attn_varlen_params`` in include/attn.h."""
+    _fields_ = [
+        ("batch", ctypes.c_int32),
+        ("total_q", ctypes.c_int32),
+        ("total_k", ctypes.c_int32),
+        ("max_seqlen_q", ctypes.c_int32),
+        ("max_seqlen_k", ctypes.c_int32),
         ("nheads", ctypes.c_int32),
         ("nheads_kv", ctypes.c_int32),
         ("headdim", ctypes.c_int32),
@@ -82,6 +102,15 @@ def _load() -> ctypes.CDLL:
     lib.attn_status_string.restype = ctypes.c_char_p
     lib.attn_get_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
     lib.attn_get_device_status.restype = ctypes.c_int
+    VP = ctypes.POINTER(AttnVarlenParams)
+    lib.attn_check_varlen_params.argtypes = [VP, ctypes.c_int]
+    lib.attn_check_varlen_params.restype = ctypes.c_int
+    lib.attn_bwd_varlen_workspace_size.argtypes = [VP]
+    lib.attn_bwd_varlen_workspace_size.restype = sz
+    lib.attn_fwd_varlen.argtypes = [VP, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.attn_fwd_varlen.restype = ctypes.c_int
+    lib.attn_bwd_varlen.argtypes = [VP, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.attn_bwd_varlen.restype = ctypes.c_int
     lib.attn_selftest_bounded_wait.argtypes = [ctypes.c_uint, vp, vp]
     lib.attn_selftest_bounded_wait.restype = ctypes.c_int
     lib.attn_version.argtypes = []
@@ -304,4 +333,106 @@ def attn_bwd_noalloc(q, k, v, out, lse, dout, softmax_scale: Optional[float] = N
             _ptr(dk), _ptr(dv), _stream(stream))
     if st != 0:
         raise AttnError(st, "attn_bwd_noalloc")
+    return dq, dk, dv
+
+
+# ----------------------------------------------------------------- packed sequences
+def make_varlen_params(batch, total_q, total_k, max_seqlen_q, max_seqlen_k, nheads, nheads_kv,
+                       headdim, dtype=ATTN_BF16, softmax_scale=None, causal=False,
+                       window_left=-1, window_right=-1) -> AttnVarlenParams:
+    scale = 1.0 / math.sqrt(headdim) if softmax_scale is None else float(softmax_scale)
+    return AttnVarlenParams(int(batch), int(total_q), int(total_k), int(max_seqlen_q),
+                            int(max_seqlen_k), int(nheads), int(nheads_kv), int(headdim),
+                            int(dtype), scale, int(bool(causal)), int(window_left),
+                            int(window_right))
+
+
+def attn_check_varlen_params(p: AttnVarlenParams, pass_: int = 0) -> int:
+    return int(_lib.attn_check_varlen_params(ctypes.byref(p), int(pass_)))
+
+
+def attn_bwd_varlen_workspace_size(p: AttnVarlenParams) -> int:
+    return int(_lib.attn_bwd_varlen_workspace_size(ctypes.byref(p)))
+
+
+def _varlen_params(q, k, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, softmax_scale,
+                   causal, window_left, window_right):
+    import torch
+    if q.dim() != 3 or k.dim() != 3:
+        raise ValueError("packed q must be (total_q, nheads, d) and k (total_k, nheads_kv, d)")
+    Tq, H, d = q.shape
+    Tk, Hkv, dk = k.shape
+    if dk != d:
+        raise ValueError("q and k disagree on head dim")
+    for t, n in ((cu_seqlens_q, "cu_seqlens_q"), (cu_seqlens_k, "cu_seqlens_k")):
+        _check(t, n)
+        if t.dtype != torch.int32 or t.dim() != 1:
+            raise TypeError(f"{n} must be a 1-D int32 CUDA tensor")
+    if cu_seqlens_q.numel() != cu_seqlens_k.numel() or cu_seqlens_q.numel() < 1:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must both have batch + 1 entries")
+    return make_varlen_params(cu_seqlens_q.numel() - 1, Tq, Tk, max_seqlen_q, max_seqlen_k, H, Hkv,
+                              d, _dtype_code(q), softmax_scale, causal, window_left, window_right)
+
+
+def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int,
+                    softmax_scale: Optional[float] = None, causal: bool = False,
+                    window_left: int = -1, window_right: int = -1, out=None, lse=None,
+                    stream=None):
+    """Attention over packed variable-length sequences.
+
+    q (total_q, H, d), k and v (total_k, Hkv, d); sequence b owns rows
+    cu_seqlens_q[b]:cu_seqlens_q[b+1] of q and cu_seqlens_k[b]:cu_seqlens_k[b+1]
+    of k, v (int32 CUDA tensors of batch + 1 offsets).  Returns (out
+    (total_q, H, d), lse (H, total_q) float32)."""
+    import torch
+    p = _varlen_params(q, k, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
+                       softmax_scale, causal, window_left, window_right)
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, n)
+        if t.dtype != q.dtype:
+            raise TypeError("q, k, v must share a dtype")
+    _check(v, "v", k.shape)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((q.shape[1], q.shape[0]), dtype=torch.float32, device=q.device)
+    _check(out, "out", q.shape)
+    _check(lse, "lse", (q.shape[1], q.shape[0]))
+    st = _lib.attn_fwd_varlen(ctypes.byref(p), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), _ptr(q),
+                              _ptr(k), _ptr(v), _ptr(out), _ptr(lse), None, ctypes.c_size_t(0),
+                              _stream(stream))
+    if st != 0:
+        raise AttnError(st, "attn_fwd_varlen")
+    return out, lse
+
+
+def attn_bwd_varlen(q, k, v, out, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int,
+                    max_seqlen_k: int, softmax_scale: Optional[float] = None,
+                    causal: bool = False, window_left: int = -1, window_right: int = -1,
+                    dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """Gradients (dq, dk, dv) of sum(out * dout) for ``attn_fwd_varlen`` with
+    the same arguments; ``out`` and ``lse`` are its results."""
+    import torch
+    p = _varlen_params(q, k, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
+                       softmax_scale, causal, window_left, window_right)
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
+        _check(t, n)
+        if t.dtype != q.dtype:
+            raise TypeError("q, k, v, out, dout must share a dtype")
+    _check(v, "v", k.shape)
+    _check(out, "out", q.shape)
+    _check(dout, "dout", q.shape)
+    _check(lse, "lse", (q.shape[1], q.shape[0]))
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    ws_bytes = attn_bwd_varlen_workspace_size(p)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
+    st = _lib.attn_bwd_varlen(ctypes.byref(p), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), _ptr(q),
+                              _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq),
+                              _ptr(dk), _ptr(dv), _ptr(workspace),
+                              ctypes.c_size_t(workspace.numel()), _stream(stream))
+    if st != 0:
+        raise AttnError(st, "attn_bwd_varlen")
     return dq, dk, dv

@@ -156,6 +156,16 @@ int fill_blocks(long long n) {
   return (int)(b < 1 ? 1 : (b > 4096 ? 4096 : b));
 }
 
+// Packed (variable-length) layout of a call: device offsets of the
+// sequences and the row counts of the packed tensors.  cu_q == nullptr means
+// the dense (batch, seqlen, heads, d) layout.
+struct Packed {
+  const int* cu_q = nullptr;
+  const int* cu_k = nullptr;
+  int total_q = 0, total_k = 0;
+  bool on() const { return cu_q != nullptr; }
+};
+
 // Kernel and grid width of a forward configuration: two query tiles per CTA
 // where both O tiles fit tensor memory (d <= 128), one otherwise.
 template <class C>
@@ -169,17 +179,26 @@ struct FwdLaunch<FwdPPCfg<D, KS, VS, F>> {
   static constexpr int rows_per_cta = 2 * FwdPPCfg<D, KS, VS, F>::BM;
 };
 
+// Forward launch.  Dense: p->seqlen_q/k are the lengths.  Packed: p->batch
+// sequences of at most p->seqlen_q / p->seqlen_k rows each.
 template <class C>
 attn_status launch_fwd(const attn_params* p, const void* q, const void* k, const void* v, void* o,
-                       float* lse, cudaStream_t stream) {
+                       float* lse, cudaStream_t stream, const Packed& pk = Packed()) {
   CUtensorMap mq, mk, mv, mo;
   const bool fp16 = C::FP16;
-  if (!map_bshd(&mq, q, fp16, p->batch, p->seqlen_q, p->nheads, C::D, C::BM) ||
-      !map_bshd(&mk, k, fp16, p->batch, p->seqlen_k, p->nheads_kv, C::D, C::BN) ||
-      !map_bshd(&mv, v, fp16, p->batch, p->seqlen_k, p->nheads_kv, C::D, C::BN) ||
-      !map_bshd(&mo, o, fp16, p->batch, p->seqlen_q, p->nheads, C::D, C::BM))
+  const int mb = pk.on() ? 1 : p->batch;
+  const int nq = pk.on() ? pk.total_q : p->seqlen_q, nk = pk.on() ? pk.total_k : p->seqlen_k;
+  if (!map_bshd(&mq, q, fp16, mb, nq, p->nheads, C::D, C::BM) ||
+      !map_bshd(&mk, k, fp16, mb, nk, p->nheads_kv, C::D, C::BN) ||
+      !map_bshd(&mv, v, fp16, mb, nk, p->nheads_kv, C::D, C::BN) ||
+      !map_bshd(&mo, o, fp16, mb, nq, p->nheads, C::D, C::BM))
     return ATTN_ERR_CUDA;
   FwdParams fp;
+  fp.cu_q = pk.cu_q;
+  fp.cu_k = pk.cu_k;
+  fp.total_q = pk.total_q;
+  fp.total_k = pk.total_k;
+  fp.o = static_cast<uint16_t*>(o);
   fp.lse = lse;
   fp.batch = p->batch;
   fp.nheads = p->nheads;
@@ -202,10 +221,21 @@ attn_status launch_fwd(const attn_params* p, const void* q, const void* k, const
   return finish(stream);
 }
 
-BwdParams bwd_params(const attn_params* p, const float* lse, void* workspace) {
-  const BwdWorkspace ws = bwd_workspace_layout(p->batch, p->nheads, p->seqlen_q, p->headdim);
+BwdWorkspace bwd_layout(const attn_params* p, const Packed& pk) {
+  return pk.on() ? bwd_workspace_layout_packed(pk.total_q, p->batch, p->nheads, p->headdim)
+                 : bwd_workspace_layout(p->batch, p->nheads, p->seqlen_q, p->headdim);
+}
+
+BwdParams bwd_params(const attn_params* p, const float* lse, void* workspace, const Packed& pk) {
+  const BwdWorkspace ws = bwd_layout(p, pk);
   uint8_t* w = static_cast<uint8_t*>(workspace);
   BwdParams bp;
+  bp.cu_q = pk.cu_q;
+  bp.cu_k = pk.cu_k;
+  bp.total_q = pk.total_q;
+  bp.total_k = pk.total_k;
+  bp.dk = bp.dv = nullptr;
+  bp.num_kblocks = bp.sched_group = 0;
   bp.lse = lse;
   bp.dvec = reinterpret_cast<float*>(w + ws.dvec_off);
   bp.lse2 = reinterpret_cast<float*>(w + ws.lse2_off);
@@ -226,10 +256,13 @@ BwdParams bwd_params(const attn_params* p, const float* lse, void* workspace) {
 }
 
 attn_status launch_bwd_prepare(const attn_params* p, const void* o, const float* lse,
-                               const void* dout, void* workspace, cudaStream_t stream) {
-  const BwdParams bp = bwd_params(p, lse, workspace);
-  const long long n_rows = (long long)p->batch * p->nheads * bp.nq_pad;
-  const long long n_elems = (long long)p->batch * p->seqlen_q * p->nheads * p->headdim;
+                               const void* dout, void* workspace, cudaStream_t stream,
+                               const Packed& pk = Packed()) {
+  const BwdParams bp = bwd_params(p, lse, workspace, pk);
+  const long long n_rows = (long long)(pk.on() ? 1 : p->batch) * p->nheads * bp.nq_pad;
+  // elements of the dQ accumulator
+  const long long n_elems = (pk.on() ? bp.nq_pad : (long long)p->batch * p->seqlen_q) *
+                            p->nheads * p->headdim;
   if (p->dtype == ATTN_FP16)
     bwd_preprocess<true><<<2368, 256, 0, stream>>>(static_cast<const uint16_t*>(o),
                                                     static_cast<const uint16_t*>(dout), bp, n_rows,
@@ -244,21 +277,27 @@ attn_status launch_bwd_prepare(const attn_params* p, const void* o, const float*
 template <class C>
 attn_status launch_bwd_main(const attn_params* p, const void* q, const void* k, const void* v,
                             const void* dout, void* dk, void* dv, void* workspace,
-                            cudaStream_t stream) {
-  const BwdParams bp = bwd_params(p, nullptr, workspace);
+                            cudaStream_t stream, const Packed& pk = Packed()) {
+  const BwdParams bp = bwd_params(p, nullptr, workspace, pk);
   const bool fp16 = C::FP16;
+  const int mb = pk.on() ? 1 : p->batch;
+  const int nq = pk.on() ? pk.total_q : p->seqlen_q, nk = pk.on() ? pk.total_k : p->seqlen_k;
+  const long long stat_rows = (long long)mb * p->nheads;  // rows of the Dvec / LSE2 arrays
   CUtensorMap mq, mk, mv, mdo, ml, md, mdk, mdv, mdq;
-  if (!map_bshd(&mq, q, fp16, p->batch, p->seqlen_q, p->nheads, C::D, C::BM) ||
-      !map_bshd(&mk, k, fp16, p->batch, p->seqlen_k, p->nheads_kv, C::D, C::BN) ||
-      !map_bshd(&mv, v, fp16, p->batch, p->seqlen_k, p->nheads_kv, C::D, C::BN) ||
-      !map_bshd(&mdo, dout, fp16, p->batch, p->seqlen_q, p->nheads, C::D, C::BM) ||
-      !map_f32_rows(&ml, bp.lse2, bp.nq_pad, (long long)p->batch * p->nheads, C::BM) ||
-      !map_f32_rows(&md, bp.dvec, bp.nq_pad, (long long)p->batch * p->nheads, C::BM) ||
-      !map_bshd(&mdk, dk, fp16, p->batch, p->seqlen_k, p->nheads_kv, C::D, C::BN) ||
-      !map_bshd(&mdv, dv, fp16, p->batch, p->seqlen_k, p->nheads_kv, C::D, C::BN) ||
-      !map_bshd_f32_32x32(&mdq, bp.dq_acc, p->batch, p->seqlen_q, p->nheads, C::D))
+  if (!map_bshd(&mq, q, fp16, mb, nq, p->nheads, C::D, C::BM) ||
+      !map_bshd(&mk, k, fp16, mb, nk, p->nheads_kv, C::D, C::BN) ||
+      !map_bshd(&mv, v, fp16, mb, nk, p->nheads_kv, C::D, C::BN) ||
+      !map_bshd(&mdo, dout, fp16, mb, nq, p->nheads, C::D, C::BM) ||
+      !map_f32_rows(&ml, bp.lse2, bp.nq_pad, stat_rows, C::BM) ||
+      !map_f32_rows(&md, bp.dvec, bp.nq_pad, stat_rows, C::BM) ||
+      !map_bshd(&mdk, dk, fp16, mb, nk, p->nheads_kv, C::D, C::BN) ||
+      !map_bshd(&mdv, dv, fp16, mb, nk, p->nheads_kv, C::D, C::BN) ||
+      !map_bshd_f32_32x32(&mdq, bp.dq_acc, mb, pk.on() ? (int)bp.nq_pad : p->seqlen_q,
+                          p->nheads, C::D))
     return ATTN_ERR_CUDA;
   BwdParams bpl = bp;
+  bpl.dk = static_cast<uint16_t*>(dk);
+  bpl.dv = static_cast<uint16_t*>(dv);
   bpl.num_kblocks = (p->seqlen_k + C::BN - 1) / C::BN;
   const int heads = p->batch * p->nheads_kv;
   // bytes of Q, dO (16-bit) and the fp32 dQ accumulator each kv head's
@@ -274,15 +313,16 @@ attn_status launch_bwd_main(const attn_params* p, const void* q, const void* k, 
 }
 
 attn_status launch_bwd_finalize(const attn_params* p, void* dq, void* workspace,
-                                cudaStream_t stream) {
-  const BwdParams bp = bwd_params(p, nullptr, workspace);
-  const long long n_elems = (long long)p->batch * p->seqlen_q * p->nheads * p->headdim;
+                                cudaStream_t stream, const Packed& pk = Packed()) {
+  const BwdParams bp = bwd_params(p, nullptr, workspace, pk);
+  const long long n_elems = (pk.on() ? (long long)pk.total_q : (long long)p->batch * p->seqlen_q) *
+                            p->nheads * p->headdim;
   if (p->dtype == ATTN_FP16)
     bwd_convert<true><<<2368, 256, 0, stream>>>(bp.dq_acc, static_cast<uint16_t*>(dq),
-                                                 n_elems / 4, p->softmax_scale);
+                                                 n_elems / 4, p->softmax_scale, bp);
   else
     bwd_convert<false><<<2368, 256, 0, stream>>>(bp.dq_acc, static_cast<uint16_t*>(dq),
-                                                  n_elems / 4, p->softmax_scale);
+                                                  n_elems / 4, p->softmax_scale, bp);
   return finish(stream);
 }
 
@@ -327,6 +367,59 @@ void* noalloc_scratch_address() {
   return ptr;
 }
 
+
+// Kernel choice by head dimension and dtype.
+attn_status dispatch_fwd(const attn_params* p, const void* q, const void* k, const void* v,
+                         void* o, float* lse, cudaStream_t stream, const Packed& pk) {
+  const bool fp16 = p->dtype == ATTN_FP16;
+  switch (p->headdim) {
+    case 64:
+      return fp16 ? launch_fwd<FwdPPCfg<64, 3, 3, true>>(p, q, k, v, o, lse, stream, pk)
+                  : launch_fwd<FwdPPCfg<64, 3, 3, false>>(p, q, k, v, o, lse, stream, pk);
+    case 128:
+      return fp16 ? launch_fwd<FwdPPCfg<128, 3, 2, true>>(p, q, k, v, o, lse, stream, pk)
+                  : launch_fwd<FwdPPCfg<128, 3, 2, false>>(p, q, k, v, o, lse, stream, pk);
+    case 256:
+      return fp16 ? launch_fwd<FwdCfg<256, 64, 2, true>>(p, q, k, v, o, lse, stream, pk)
+                  : launch_fwd<FwdCfg<256, 64, 2, false>>(p, q, k, v, o, lse, stream, pk);
+    default:
+      return ATTN_ERR_UNSUPPORTED_HEADDIM;
+  }
+}
+
+attn_status dispatch_bwd_main(const attn_params* p, const void* q, const void* k, const void* v,
+                              const void* dout, void* dk, void* dv, void* workspace,
+                              cudaStream_t stream, const Packed& pk) {
+  const bool fp16 = p->dtype == ATTN_FP16;
+  switch (p->headdim) {
+    case 64:
+      return fp16 ? launch_bwd_main<BwdCfg<64, true>>(p, q, k, v, dout, dk, dv, workspace, stream, pk)
+                  : launch_bwd_main<BwdCfg<64, false>>(p, q, k, v, dout, dk, dv, workspace, stream, pk);
+    case 128:
+      return fp16 ? launch_bwd_main<BwdCfg<128, true>>(p, q, k, v, dout, dk, dv, workspace, stream, pk)
+                  : launch_bwd_main<BwdCfg<128, false>>(p, q, k, v, dout, dk, dv, workspace, stream, pk);
+    default:
+      return ATTN_ERR_UNSUPPORTED_HEADDIM;
+  }
+}
+
+// The dense-layout view of a packed call: `batch` sequences of at most
+// max_seqlen rows (the kernels read each one's own length from the offsets).
+attn_params packed_view(const attn_varlen_params* v) {
+  attn_params p;
+  p.batch = v->batch;
+  p.seqlen_q = v->max_seqlen_q;
+  p.seqlen_k = v->max_seqlen_k;
+  p.nheads = v->nheads;
+  p.nheads_kv = v->nheads_kv;
+  p.headdim = v->headdim;
+  p.dtype = v->dtype;
+  p.softmax_scale = v->softmax_scale;
+  p.causal = v->causal;
+  p.window_left = v->window_left;
+  p.window_right = v->window_right;
+  return p;
+}
 
 // Self-test of the bounded wait: two waiters (one warp-uniform, one single
 // thread) on an mbarrier that nothing ever arrives at.  Both must give up
@@ -408,20 +501,7 @@ attn_status attn_fwd(const attn_params* p, const void* q, const void* k, const v
   }
   if (!q || !k || !v) return ATTN_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return ATTN_ERR_MISALIGNED;
-  const bool fp16 = p->dtype == ATTN_FP16;
-  switch (p->headdim) {
-    case 64:
-      return fp16 ? launch_fwd<FwdPPCfg<64, 3, 3, true>>(p, q, k, v, o, lse, stream)
-                  : launch_fwd<FwdPPCfg<64, 3, 3, false>>(p, q, k, v, o, lse, stream);
-    case 128:
-      return fp16 ? launch_fwd<FwdPPCfg<128, 3, 2, true>>(p, q, k, v, o, lse, stream)
-                  : launch_fwd<FwdPPCfg<128, 3, 2, false>>(p, q, k, v, o, lse, stream);
-    case 256:
-      return fp16 ? launch_fwd<FwdCfg<256, 64, 2, true>>(p, q, k, v, o, lse, stream)
-                  : launch_fwd<FwdCfg<256, 64, 2, false>>(p, q, k, v, o, lse, stream);
-    default:
-      return ATTN_ERR_UNSUPPORTED_HEADDIM;
-  }
+  return dispatch_fwd(p, q, k, v, o, lse, stream, Packed());
 }
 
 size_t attn_bwd_workspace_size(const attn_params* p) {
@@ -451,18 +531,8 @@ attn_status attn_bwd_accumulate(const attn_params* p, const void* q, const void*
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dk) ||
       !aligned16(dv))
     return ATTN_ERR_MISALIGNED;
-  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-  const bool fp16 = p->dtype == ATTN_FP16;
-  switch (p->headdim) {
-    case 64:
-      return fp16 ? launch_bwd_main<BwdCfg<64, true>>(p, q, k, v, dout, dk, dv, workspace, stream)
-                  : launch_bwd_main<BwdCfg<64, false>>(p, q, k, v, dout, dk, dv, workspace, stream);
-    case 128:
-      return fp16 ? launch_bwd_main<BwdCfg<128, true>>(p, q, k, v, dout, dk, dv, workspace, stream)
-                  : launch_bwd_main<BwdCfg<128, false>>(p, q, k, v, dout, dk, dv, workspace, stream);
-    default:
-      return ATTN_ERR_UNSUPPORTED_HEADDIM;
-  }
+  return dispatch_bwd_main(p, q, k, v, dout, dk, dv, workspace,
+                           reinterpret_cast<cudaStream_t>(stream_), Packed());
 }
 
 attn_status attn_bwd_finalize(const attn_params* p, void* dq, void* workspace,
@@ -538,6 +608,97 @@ attn_status attn_get_device_status(void* stream_, int* code) {
   if (cudaStreamSynchronize(stream) != cudaSuccess) return ATTN_ERR_CUDA;
   *code = static_cast<int>(host);
   return ATTN_OK;
+}
+
+attn_status attn_check_varlen_params(const attn_varlen_params* v, int pass) {
+  if (!v) return ATTN_ERR_INVALID_ARG;
+  if (v->total_q < 0 || v->total_k < 0 || v->max_seqlen_q < 0 || v->max_seqlen_k < 0)
+    return ATTN_ERR_INVALID_ARG;
+  const attn_params p = packed_view(v);
+  return attn_check_params(&p, pass);
+}
+
+size_t attn_bwd_varlen_workspace_size(const attn_varlen_params* v) {
+  if (attn_check_varlen_params(v, 1) != ATTN_OK) return 0;
+  return bwd_workspace_layout_packed(v->total_q, v->batch, v->nheads, v->headdim).total;
+}
+
+attn_status attn_fwd_varlen(const attn_varlen_params* v, const int32_t* cu_seqlens_q,
+                            const int32_t* cu_seqlens_k, const void* q, const void* k,
+                            const void* vv, void* o, float* lse, void* workspace,
+                            size_t workspace_bytes, void* stream_) {
+  (void)workspace;
+  (void)workspace_bytes;
+  attn_status st = attn_check_varlen_params(v, 0);
+  if (st != ATTN_OK) return st;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (v->batch == 0 || v->total_q == 0 || v->max_seqlen_q == 0) return ATTN_OK;
+  if (!o || !lse || !cu_seqlens_q || !cu_seqlens_k) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(o) || (reinterpret_cast<uintptr_t>(lse) & 3u) ||
+      (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) ||
+      (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u))
+    return ATTN_ERR_MISALIGNED;
+  if (v->total_k == 0 || v->max_seqlen_k == 0) {
+    const long long n_o = (long long)v->total_q * v->nheads * v->headdim;
+    const long long n_l = (long long)v->nheads * v->total_q;
+    fill_empty_fwd<<<fill_blocks(n_o), 256, 0, stream>>>(static_cast<uint16_t*>(o), n_o, lse, n_l);
+    return finish(stream);
+  }
+  if (!q || !k || !vv) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(vv)) return ATTN_ERR_MISALIGNED;
+  const attn_params p = packed_view(v);
+  Packed pk;
+  pk.cu_q = cu_seqlens_q;
+  pk.cu_k = cu_seqlens_k;
+  pk.total_q = v->total_q;
+  pk.total_k = v->total_k;
+  return dispatch_fwd(&p, q, k, vv, o, lse, stream, pk);
+}
+
+attn_status attn_bwd_varlen(const attn_varlen_params* v, const int32_t* cu_seqlens_q,
+                            const int32_t* cu_seqlens_k, const void* q, const void* k,
+                            const void* vv, const void* o, const float* lse, const void* dout,
+                            void* dq, void* dk, void* dv, void* workspace,
+                            size_t workspace_bytes, void* stream_) {
+  attn_status st = attn_check_varlen_params(v, 1);
+  if (st != ATTN_OK) return st;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (v->batch == 0) return ATTN_OK;
+  const long long n_q = (long long)v->total_q * v->nheads * v->headdim;
+  const long long n_k = (long long)v->total_k * v->nheads_kv * v->headdim;
+  if ((n_q && !dq) || (n_k && (!dk || !dv))) return ATTN_ERR_INVALID_ARG;
+  if ((n_q && !aligned16(dq)) || (n_k && (!aligned16(dk) || !aligned16(dv))))
+    return ATTN_ERR_MISALIGNED;
+  if (n_q == 0 || n_k == 0 || v->max_seqlen_q == 0 || v->max_seqlen_k == 0) {
+    // Nothing to attend: every gradient is zero.
+    if (n_q) fill_zero_u16<<<fill_blocks(n_q), 256, 0, stream>>>(static_cast<uint16_t*>(dq), n_q);
+    if (n_k) {
+      fill_zero_u16<<<fill_blocks(n_k), 256, 0, stream>>>(static_cast<uint16_t*>(dk), n_k);
+      fill_zero_u16<<<fill_blocks(n_k), 256, 0, stream>>>(static_cast<uint16_t*>(dv), n_k);
+    }
+    return finish(stream);
+  }
+  if (!q || !k || !vv || !o || !lse || !dout || !cu_seqlens_q || !cu_seqlens_k)
+    return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(vv) || !aligned16(o) || !aligned16(dout) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u) ||
+      (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) ||
+      (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u))
+    return ATTN_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < attn_bwd_varlen_workspace_size(v))
+    return ATTN_ERR_WORKSPACE_TOO_SMALL;
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u) return ATTN_ERR_MISALIGNED;
+  const attn_params p = packed_view(v);
+  Packed pk;
+  pk.cu_q = cu_seqlens_q;
+  pk.cu_k = cu_seqlens_k;
+  pk.total_q = v->total_q;
+  pk.total_k = v->total_k;
+  st = launch_bwd_prepare(&p, o, lse, dout, workspace, stream, pk);
+  if (st != ATTN_OK) return st;
+  st = dispatch_bwd_main(&p, q, k, vv, dout, dk, dv, workspace, stream, pk);
+  if (st != ATTN_OK) return st;
+  return launch_bwd_finalize(&p, dq, workspace, stream, pk);
 }
 
 attn_status attn_selftest_bounded_wait(unsigned int wait_limit_us, int* result, void* stream_) {

@@ -52,7 +52,8 @@ __host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a -
 
 // Workspace: Dvec and LSE2 as (batch*nheads, nq_pad) fp32 with nq_pad a
 // multiple of 128 (TMA-aligned rows), then the fp32 dQ accumulator
-// (batch, seqlen_q, nheads, headdim).
+// (batch, seqlen_q, nheads, headdim).  Packed sequences: see
+// bwd_workspace_layout_packed.
 __host__ __device__ inline BwdWorkspace bwd_workspace_layout(int batch, int nheads, int seqlen_q,
                                                             int headdim) {
   BwdWorkspace w;
@@ -62,6 +63,30 @@ __host__ __device__ inline BwdWorkspace bwd_workspace_layout(int batch, int nhea
   w.lse2_off = align_up(rows, 256);
   w.dq_off = w.lse2_off + align_up(rows, 256);
   w.total = w.dq_off + align_up((size_t)batch * seqlen_q * nheads * headdim * 4, 256);
+  return w;
+}
+
+// Packed sequences: sequence b's rows start at padded row
+// packed_row0(cu_q[b], b) = align4(cu_q[b]) + 136 b, a multiple of 4 (TMA
+// alignment of the fp32 rows) with >= 128 rows of slack after every sequence,
+// so a query tile that ends past its sequence reads and adds only slack rows.
+// Dvec and LSE2 are (nheads, nq_pad) and the dQ accumulator is
+// (nq_pad, nheads, headdim), nq_pad = packed_rows(total_q, batch).
+__host__ __device__ inline long long packed_row0(int cu_b, int b) {
+  return (((long long)cu_b + 3) & ~3ll) + 136ll * b;
+}
+__host__ __device__ inline long long packed_rows(int total_q, int batch) {
+  return (((long long)total_q + 3) & ~3ll) + 136ll * batch + 128;
+}
+__host__ __device__ inline BwdWorkspace bwd_workspace_layout_packed(int total_q, int batch,
+                                                                   int nheads, int headdim) {
+  BwdWorkspace w;
+  w.nq_pad = packed_rows(total_q, batch);
+  const size_t rows = (size_t)nheads * (size_t)w.nq_pad * 4;
+  w.dvec_off = 0;
+  w.lse2_off = align_up(rows, 256);
+  w.dq_off = w.lse2_off + align_up(rows, 256);
+  w.total = w.dq_off + align_up((size_t)w.nq_pad * nheads * headdim * 4, 256);
   return w;
 }
 
@@ -77,11 +102,44 @@ struct BwdParams {
   long long nq_pad;
   int num_kblocks;   // key tiles per (batch, kv head): the work units
   int sched_group;   // kv heads per scheduling group (grouped_lpt)
+  // Packed variable-length sequences when cu_q != nullptr (see seq_span and
+  // packed_row0): seqlen_q / seqlen_k then hold the longest sequence,
+  // total_q / total_k the rows of the packed tensors, lse is (nheads,
+  // total_q), and a key tile that ends past its sequence writes dk / dv row
+  // by row.
+  const int* cu_q;
+  const int* cu_k;
+  int total_q, total_k;
+  uint16_t* dk;
+  uint16_t* dv;
 };
+
+// Packed layout: the sequence owning padded row `pr` (the last b with
+// packed_row0 <= pr) and the sequence owning token row `t` (the last b with
+// cu_q[b] <= t), by binary search over the clamped offsets.
+__device__ inline int packed_seq_of_row(const BwdParams& p, long long pr) {
+  int lo = 0, hi = p.batch - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    const int c = min(max(__ldg(p.cu_q + mid), 0), p.total_q);
+    if (packed_row0(c, mid) <= pr) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+__device__ inline int packed_seq_of_token(const BwdParams& p, long long t) {
+  int lo = 0, hi = p.batch - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    const int c = min(max(__ldg(p.cu_q + mid), 0), p.total_q);
+    if (c <= t) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
 
 // ------------------------------------------------------------ preprocess
 // One warp per (b, h, i) row of the padded range: Dvec_i = sum_c dO_ic O_ic,
-// LSE2_i = LSE_i * log2(e).  Blocks past the rows zero the dQ accumulator.
+// LSE2_i = LSE_i * log2(e); padding rows get 0 and +inf (P = 0 there).  All
+// threads then zero the dQ accumulator.
 template <bool FP16>
 __global__ void __launch_bounds__(256) bwd_preprocess(const uint16_t* __restrict__ o,
                                                       const uint16_t* __restrict__ dout,
@@ -91,12 +149,28 @@ __global__ void __launch_bounds__(256) bwd_preprocess(const uint16_t* __restrict
   const int lane = threadIdx.x & 31;
   const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
   for (long long row = warp_global; row < n_rows; row += nwarps) {
-    const long long i = row % p.nq_pad;
+    const long long ip = row % p.nq_pad;
     const long long bh = row / p.nq_pad;
-    const int h = (int)(bh % p.nheads), b = (int)(bh / p.nheads);
+    int h, b;
+    long long i, tok;  // row within the sequence; row of the o / dout / lse tensors
+    bool valid;
+    if (p.cu_q) {
+      h = (int)bh;
+      b = packed_seq_of_row(p, ip);
+      const SeqSpan sq = seq_span(p.cu_q, p.cu_k, p.total_q, p.total_k, b, 0, 0);
+      i = ip - packed_row0(sq.q_row0, b);
+      valid = i >= 0 && i < sq.len_q;
+      tok = sq.q_row0 + i;
+    } else {
+      h = (int)(bh % p.nheads);
+      b = (int)(bh / p.nheads);
+      i = ip;
+      valid = i < p.seqlen_q;
+      tok = (long long)b * p.seqlen_q + i;
+    }
     float dv = 0.f, l2 = INFINITY;
-    if (i < p.seqlen_q) {
-      const size_t base = (((size_t)b * p.seqlen_q + i) * p.nheads + h) * p.headdim;
+    if (valid) {
+      const size_t base = ((size_t)tok * p.nheads + h) * p.headdim;
       float acc = 0.f;
       for (int c = lane * 2; c < p.headdim; c += 64) {
         const uint32_t ov = *reinterpret_cast<const uint32_t*>(o + base + c);
@@ -119,7 +193,8 @@ __global__ void __launch_bounds__(256) bwd_preprocess(const uint16_t* __restrict
 #pragma unroll
       for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
       dv = acc;
-      const float l = p.lse[((size_t)b * p.nheads + h) * p.seqlen_q + i];
+      const float l = p.cu_q ? p.lse[(size_t)h * p.total_q + tok]
+                             : p.lse[((size_t)b * p.nheads + h) * p.seqlen_q + i];
       l2 = (l == -INFINITY) ? INFINITY : l * 1.4426950408889634f;
     }
     if (lane == 0) {
@@ -134,14 +209,24 @@ __global__ void __launch_bounds__(256) bwd_preprocess(const uint16_t* __restrict
 }
 
 // ------------------------------------------------------------ convert
+// dQ = scale * accumulator, four elements per step.  Packed sequences: token
+// row t of sequence b reads padded row packed_row0(cu_q[b], b) + t - cu_q[b].
 template <bool FP16>
 __global__ void __launch_bounds__(256) bwd_convert(const float* __restrict__ acc,
                                                    uint16_t* __restrict__ dq, long long n4,
-                                                   float scale) {
+                                                   float scale, BwdParams p) {
   const long long tid = blockIdx.x * (long long)blockDim.x + threadIdx.x;
   const long long nthreads = (long long)gridDim.x * blockDim.x;
+  const long long row_len = (long long)p.nheads * p.headdim;
   for (long long k = tid; k < n4; k += nthreads) {
-    const float4 a = reinterpret_cast<const float4*>(acc)[k];
+    long long src = k;
+    if (p.cu_q) {
+      const long long e = 4 * k, t = e / row_len;
+      const int b = packed_seq_of_token(p, t);
+      const long long c = min(max(__ldg(p.cu_q + b), 0), p.total_q);
+      src = ((packed_row0((int)c, b) + (t - c)) * row_len + e % row_len) / 4;
+    }
+    const float4 a = reinterpret_cast<const float4*>(acc)[src];
     uint2 w;
     w.x = pack2<FP16>(a.x * scale, a.y * scale);
     w.y = pack2<FP16>(a.z * scale, a.w * scale);
@@ -215,7 +300,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const __grid_constant__ CUtensorMap tm_lse2, const __grid_constant__ CUtensorMap tm_dvec,
                     const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
-                    const __grid_constant__ CUtensorMap tm_dqacc, const BwdParams p) {
+                    const __grid_constant__ CUtensorMap tm_dqacc, const BwdParams pin) {
   constexpr int D = C::D, BN = C::BN, BM = C::BM, NBUF = C::NBUF, QS = C::QSTAGES;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t smem0 = (smem_addr(smem_raw) + 1023u) & ~1023u;
@@ -226,12 +311,22 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   const uint32_t warp = warp_id(), lane = lane_id();
   // earlier key tiles are seen by more queries under a causal mask: heaviest
   // first
-  const UnitOrder uo = grouped_lpt((int)blockIdx.x, p.num_kblocks, p.batch * p.nheads_kv,
-                                   p.sched_group);
-  const int kblock = uo.rank, kvh = uo.head % p.nheads_kv, b = uo.head / p.nheads_kv;
+  const UnitOrder uo = grouped_lpt((int)blockIdx.x, pin.num_kblocks, pin.batch * pin.nheads_kv,
+                                   pin.sched_group);
+  const int kblock = uo.rank, kvh = uo.head % pin.nheads_kv, b = uo.head / pin.nheads_kv;
+  const SeqSpan sq = seq_span(pin.cu_q, pin.cu_k, pin.total_q, pin.total_k, b, pin.seqlen_q,
+                              pin.seqlen_k);
+  BwdParams p = pin;  // lengths of this block's sequence
+  p.seqlen_q = sq.len_q;
+  p.seqlen_k = sq.len_k;
   const int group = p.nheads / p.nheads_kv;
   const int k0 = kblock * BN;
+  if (k0 >= p.seqlen_k) return;  // past a packed sequence: nothing to do
   const int k1 = min(k0 + BN, p.seqlen_k);
+  // Padded row of this sequence's first query in the Dvec / LSE2 rows and
+  // the dQ accumulator (packed layout; the dense layout indexes by batch).
+  const long long prow0 = p.cu_q ? packed_row0(sq.q_row0, b) : 0;
+  const bool row_store = p.cu_q != nullptr && k0 + BN > p.seqlen_k;
 
   // Query rows that see any key of [k0, k1).
   const long long off = (long long)p.seqlen_k - p.seqlen_q;
@@ -268,25 +363,29 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     if (lane == 0 && nt > 0) {
       mbar_arrive_expect_tx(bar(C::B_KV), 2 * C::KV_BYTES);
       for (int bx = 0; bx < C::NBOX; ++bx) {
-        tma_load_4d(smem0 + C::OFF_K + bx * (BN * 128), &tm_k, bar(C::B_KV), bx * 64, kvh, k0, b);
-        tma_load_4d(smem0 + C::OFF_V + bx * (BN * 128), &tm_v, bar(C::B_KV), bx * 64, kvh, k0, b);
+        tma_load_4d(smem0 + C::OFF_K + bx * (BN * 128), &tm_k, bar(C::B_KV), bx * 64, kvh,
+                    sq.k_row0 + k0, sq.tma_b);
+        tma_load_4d(smem0 + C::OFF_V + bx * (BN * 128), &tm_v, bar(C::B_KV), bx * 64, kvh,
+                    sq.k_row0 + k0, sq.tma_b);
       }
       for (int t = 0; t < nt; ++t) {
         const int slot = t % QS, n = t / QS;
         if (n > 0 && !mbar_wait(bar(C::B_EMPTY + slot), (n - 1) & 1)) break;
         const int h = kvh * group + t / nqb;
         const int q0 = (qb_lo + t % nqb) * BM;
-        const int row = b * p.nheads + h;
+        // Dvec / LSE2 coordinates: (padded row, head) packed, (row, batch*head) dense
+        const int row = p.cu_q ? h : b * p.nheads + h;
+        const int xs = (int)prow0 + q0;
         mbar_arrive_expect_tx(bar(C::B_QFULL + slot), C::Q_BYTES + BM * 4);
         for (int bx = 0; bx < C::NBOX; ++bx)
           tma_load_4d(smem0 + C::OFF_Q + slot * C::Q_BYTES + bx * (BM * 128), &tm_q,
-                      bar(C::B_QFULL + slot), bx * 64, h, q0, b);
-        tma_load_2d(smem0 + C::OFF_LSE + slot * BM * 4, &tm_lse2, bar(C::B_QFULL + slot), q0, row);
+                      bar(C::B_QFULL + slot), bx * 64, h, sq.q_row0 + q0, sq.tma_b);
+        tma_load_2d(smem0 + C::OFF_LSE + slot * BM * 4, &tm_lse2, bar(C::B_QFULL + slot), xs, row);
         mbar_arrive_expect_tx(bar(C::B_DOFULL + slot), C::Q_BYTES + BM * 4);
         for (int bx = 0; bx < C::NBOX; ++bx)
           tma_load_4d(smem0 + C::OFF_DO + slot * C::Q_BYTES + bx * (BM * 128), &tm_do,
-                      bar(C::B_DOFULL + slot), bx * 64, h, q0, b);
-        tma_load_2d(smem0 + C::OFF_DVEC + slot * BM * 4, &tm_dvec, bar(C::B_DOFULL + slot), q0, row);
+                      bar(C::B_DOFULL + slot), bx * 64, h, sq.q_row0 + q0, sq.tma_b);
+        tma_load_2d(smem0 + C::OFF_DVEC + slot * BM * 4, &tm_dvec, bar(C::B_DOFULL + slot), xs, row);
       }
       for (int t = nt - QS < 0 ? 0 : nt - QS; t < nt; ++t) {
         const int slot = t % QS, n = t / QS;
@@ -444,7 +543,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0 && qrow < p.seqlen_q) {
-        tma_reduce_add_4d(&tm_dqacc, dqs, dcol, h, qrow, b);
+        tma_reduce_add_4d(&tm_dqacc, dqs, dcol, h, (int)prow0 + qrow, sq.tma_b);
         bulk_commit_group();
       }
       staged = true;
@@ -577,6 +676,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
           for (int e = 0; e < 16; ++e)
             w[e] = pack2<C::FP16>(__uint_as_float(raw[2 * e]) * mul, __uint_as_float(raw[2 * e + 1]) * mul);
+          if (row_store) {
+            if (k0 + r < p.seqlen_k) {
+              uint16_t* dst = which == 0 ? p.dk : p.dv;
+              store_row32(dst + ((size_t)(sq.k_row0 + k0 + r) * p.nheads_kv + kvh) * D + c, w);
+            }
+            continue;
+          }
           const int bx = c / 64, chunk0 = (c % 64) / 8;
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4) {
@@ -590,10 +696,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     }
     tc_fence_before();
     named_bar_sync(1, 256);
-    if (ok && threadIdx.x == 0) {
+    if (ok && threadIdx.x == 0 && !row_store) {
       for (int bx = 0; bx < C::NBOX; ++bx) {
-        tma_store_4d(&tm_dk, smem0 + C::OFF_Q + bx * (BN * 128), bx * 64, kvh, k0, b);
-        tma_store_4d(&tm_dv, smem0 + C::OFF_DO + bx * (BN * 128), bx * 64, kvh, k0, b);
+        tma_store_4d(&tm_dk, smem0 + C::OFF_Q + bx * (BN * 128), bx * 64, kvh, sq.k_row0 + k0,
+                     sq.tma_b);
+        tma_store_4d(&tm_dv, smem0 + C::OFF_DO + bx * (BN * 128), bx * 64, kvh, sq.k_row0 + k0,
+                     sq.tma_b);
       }
       bulk_commit_group();
     }

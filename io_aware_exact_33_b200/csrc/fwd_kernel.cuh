@@ -36,7 +36,24 @@ struct FwdParams {
   float scale_log2;  // softmax_scale * log2(e)
   int num_qblocks;   // work units per (batch, head): query tiles or tile pairs
   int sched_group;   // heads per scheduling group (grouped_lpt)
+  // Packed variable-length sequences when cu_q != nullptr (see seq_span):
+  // seqlen_q / seqlen_k then hold the longest sequence, total_q / total_k
+  // the rows of the packed tensors, lse is (nheads, total_q), and a query
+  // tile that ends past its sequence is written through `o` row by row.
+  const int* cu_q;
+  const int* cu_k;
+  int total_q, total_k;
+  uint16_t* o;
 };
+
+// Row `row` of query head h of sequence (b, sq) in the LSE output.
+__device__ __forceinline__ size_t lse_index(const FwdParams& p, const SeqSpan& sq, int b, int h,
+                                            int row) {
+  return p.cu_q ? (size_t)h * p.total_q + sq.q_row0 + row
+                : ((size_t)b * p.nheads + h) * p.seqlen_q + row;
+}
+
+
 
 // Range of visible key positions for query rows [q0, q1): keys [jmin, jmax].
 struct KeyRange {
@@ -91,7 +108,7 @@ template <class C>
 __global__ void __launch_bounds__(C::THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-                    const FwdParams p) {
+                    const FwdParams pin) {
   constexpr int D = C::D, BN = C::BN, BM = C::BM, STAGES = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t smem0 = (smem_addr(smem_raw) + 1023u) & ~1023u;
@@ -101,13 +118,20 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 
   const uint32_t warp = warp_id(), lane = lane_id();
   // later query tiles see more keys under a causal mask: heaviest first
-  const UnitOrder uo = grouped_lpt((int)blockIdx.x, p.num_qblocks, p.batch * p.nheads,
-                                   p.sched_group);
-  const int qblock = p.num_qblocks - 1 - uo.rank;
-  const int h = uo.head % p.nheads, b = uo.head / p.nheads;
+  const UnitOrder uo = grouped_lpt((int)blockIdx.x, pin.num_qblocks, pin.batch * pin.nheads,
+                                   pin.sched_group);
+  const int qblock = pin.num_qblocks - 1 - uo.rank;
+  const int h = uo.head % pin.nheads, b = uo.head / pin.nheads;
+  const SeqSpan sq = seq_span(pin.cu_q, pin.cu_k, pin.total_q, pin.total_k, b, pin.seqlen_q,
+                              pin.seqlen_k);
+  FwdParams p = pin;  // lengths of this block's sequence
+  p.seqlen_q = sq.len_q;
+  p.seqlen_k = sq.len_k;
   const int kvh = h / (p.nheads / p.nheads_kv);
   const int q0 = qblock * BM;
+  if (q0 >= p.seqlen_q) return;  // past a packed sequence: nothing to do
   const int q1 = min(q0 + BM, p.seqlen_q);
+  const bool row_store = p.cu_q != nullptr && q0 + BM > p.seqlen_q;
 
   const KeyRange kr = visible_keys(q0, q1, p);
   const int t_lo = kr.jmax >= kr.jmin ? (int)(kr.jmin / BN) : 0;
@@ -138,7 +162,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     if (lane == 0 && nt > 0) {
       mbar_arrive_expect_tx(bar(C::B_Q), C::Q_BYTES);
       for (int bx = 0; bx < C::NBOX; ++bx)
-        tma_load_4d(smem0 + C::OFF_Q + bx * (BM * 128), &tm_q, bar(C::B_Q), bx * 64, h, q0, b);
+        tma_load_4d(smem0 + C::OFF_Q + bx * (BM * 128), &tm_q, bar(C::B_Q), bx * 64, h,
+                    sq.q_row0 + q0, sq.tma_b);
       for (int t = 0; t < nt; ++t) {
         const int st = t % STAGES, n = t / STAGES;
         if (n > 0 && !mbar_wait(bar(C::B_EMPTY + st), (n - 1) & 1)) break;
@@ -146,11 +171,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         mbar_arrive_expect_tx(bar(C::B_KFULL + st), C::KV_BYTES);
         for (int bx = 0; bx < C::NBOX; ++bx)
           tma_load_4d(smem0 + C::OFF_K + st * C::KV_BYTES + bx * (BN * 128), &tm_k,
-                      bar(C::B_KFULL + st), bx * 64, kvh, k0, b);
+                      bar(C::B_KFULL + st), bx * 64, kvh, sq.k_row0 + k0, sq.tma_b);
         mbar_arrive_expect_tx(bar(C::B_VFULL + st), C::KV_BYTES);
         for (int bx = 0; bx < C::NBOX; ++bx)
           tma_load_4d(smem0 + C::OFF_V + st * C::KV_BYTES + bx * (BN * 128), &tm_v,
-                      bar(C::B_VFULL + st), bx * 64, kvh, k0, b);
+                      bar(C::B_VFULL + st), bx * 64, kvh, sq.k_row0 + k0, sq.tma_b);
       }
       // Loads still in flight must land before the CTA can exit: wait (bounded)
       // for the last fill of every slot used.
@@ -318,6 +343,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         for (int e = 0; e < 16; ++e)
           w[e] = pack2<C::FP16>(__uint_as_float(raw[2 * e]) * inv_l,
                                 __uint_as_float(raw[2 * e + 1]) * inv_l);
+        if (row_store) {
+          if (i < p.seqlen_q)
+            store_row32(p.o + ((size_t)(sq.q_row0 + i) * p.nheads + h) * D + c, w);
+          continue;
+        }
         // 32 columns = 64 bytes = four 16-byte chunks of a 128-byte swizzled row.
         const int bx = c / 64, chunk0 = (c % 64) / 8;
 #pragma unroll
@@ -330,14 +360,15 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       fence_proxy_async_smem();
       if (i < p.seqlen_q) {
         const float lse = l > 0.f ? (m + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
-        p.lse[((size_t)b * p.nheads + h) * p.seqlen_q + i] = lse;
+        p.lse[lse_index(p, sq, b, h, i)] = lse;
       }
     }
     tc_fence_before();
     named_bar_sync(1, 128);
-    if (ok && threadIdx.x == 0) {
+    if (ok && threadIdx.x == 0 && !row_store) {
       for (int bx = 0; bx < C::NBOX; ++bx)
-        tma_store_4d(&tm_o, smem0 + C::OFF_Q + bx * (BM * 128), bx * 64, h, q0, b);
+        tma_store_4d(&tm_o, smem0 + C::OFF_Q + bx * (BM * 128), bx * 64, h, sq.q_row0 + q0,
+                     sq.tma_b);
       bulk_commit_group();
       bulk_wait_group_read_all();
     }
@@ -516,7 +547,7 @@ template <class C>
 __global__ void __launch_bounds__(C::THREADS, 1)
     attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-                       const FwdParams p) {
+                       const FwdParams pin) {
   constexpr int D = C::D, BN = C::BN, BM = C::BM, KS = C::KSTAGES, VS = C::VSTAGES;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t smem0 = (smem_addr(smem_raw) + 1023u) & ~1023u;
@@ -526,10 +557,16 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 
   const uint32_t warp = warp_id(), lane = lane_id();
   // later query tiles see more keys under a causal mask: heaviest first
-  const UnitOrder uo = grouped_lpt((int)blockIdx.x, p.num_qblocks, p.batch * p.nheads,
-                                   p.sched_group);
-  const int pair = p.num_qblocks - 1 - uo.rank;
-  const int h = uo.head % p.nheads, b = uo.head / p.nheads;
+  const UnitOrder uo = grouped_lpt((int)blockIdx.x, pin.num_qblocks, pin.batch * pin.nheads,
+                                   pin.sched_group);
+  const int pair = pin.num_qblocks - 1 - uo.rank;
+  const int h = uo.head % pin.nheads, b = uo.head / pin.nheads;
+  const SeqSpan sq = seq_span(pin.cu_q, pin.cu_k, pin.total_q, pin.total_k, b, pin.seqlen_q,
+                              pin.seqlen_k);
+  FwdParams p = pin;  // lengths of this block's sequence
+  p.seqlen_q = sq.len_q;
+  p.seqlen_k = sq.len_k;
+  if (2 * pair * BM >= p.seqlen_q) return;  // past a packed sequence: nothing to do
   const int kvh = h / (p.nheads / p.nheads_kv);
 
   // Key-tile range [lo_i, hi_i) of each query tile; union [ulo, uhi).
@@ -579,7 +616,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       for (int i = 0; i < 2; ++i)
         for (int bx = 0; bx < C::NBOX; ++bx)
           tma_load_4d(smem0 + C::OFF_Q + i * C::Q_BYTES + bx * (BM * 128), &tm_q, bar(C::B_Q),
-                      bx * 64, h, qs[i], b);
+                      bx * 64, h, sq.q_row0 + qs[i], sq.tma_b);
       // K and V slots are released separately: K_j after key tile j's last S
       // MMA (same iteration), V_j after its last PV MMA (up to one later).
       // K runs one tile ahead of V in the issue order, so a V slot that is
@@ -590,7 +627,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         mbar_arrive_expect_tx(bar(C::B_KFULL + st), C::KV_BYTES);
         for (int bx = 0; bx < C::NBOX; ++bx)
           tma_load_4d(smem0 + C::OFF_K + st * C::KV_BYTES + bx * (BN * 128), &tm_k,
-                      bar(C::B_KFULL + st), bx * 64, kvh, (ulo + t) * BN, b);
+                      bar(C::B_KFULL + st), bx * 64, kvh, sq.k_row0 + (ulo + t) * BN, sq.tma_b);
         return true;
       };
       auto load_v = [&](int t) -> bool {
@@ -599,7 +636,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         mbar_arrive_expect_tx(bar(C::B_VFULL + st), C::KV_BYTES);
         for (int bx = 0; bx < C::NBOX; ++bx)
           tma_load_4d(smem0 + C::OFF_V + st * C::KV_BYTES + bx * (BN * 128), &tm_v,
-                      bar(C::B_VFULL + st), bx * 64, kvh, (ulo + t) * BN, b);
+                      bar(C::B_VFULL + st), bx * 64, kvh, sq.k_row0 + (ulo + t) * BN, sq.tma_b);
         return true;
       };
       bool go = load_k(0);
@@ -720,6 +757,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     // work): that load must land before the staging area is overwritten.
     if (ok && n_i == 0 && nt > 0) ok = mbar_wait_warp(bar(C::B_Q), 0);
     const uint32_t stage = smem0 + C::OFF_Q + i * C::Q_BYTES;  // Q_i is no longer read
+    const bool row_store = p.cu_q != nullptr && q_i + BM > p.seqlen_q;
     if (ok) {
       tc_fence_after();
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
@@ -739,6 +777,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         for (int e = 0; e < 16; ++e)
           w[e] = pack2<C::FP16>(__uint_as_float(raw[2 * e]) * inv_l,
                                 __uint_as_float(raw[2 * e + 1]) * inv_l);
+        if (row_store) {
+          if (row < p.seqlen_q)
+            store_row32(p.o + ((size_t)(sq.q_row0 + row) * p.nheads + h) * D + c, w);
+          continue;
+        }
         const int bx = c / 64, chunk0 = (c % 64) / 8;
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
@@ -750,14 +793,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       fence_proxy_async_smem();
       if (row < p.seqlen_q) {
         const float lse = l > 0.f ? (m + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
-        p.lse[((size_t)b * p.nheads + h) * p.seqlen_q + row] = lse;
+        p.lse[lse_index(p, sq, b, h, row)] = lse;
       }
     }
     tc_fence_before();
     named_bar_sync(1 + i, 128);
-    if (ok && quad == 0 && lane == 0 && q_i < p.seqlen_q) {
+    if (ok && quad == 0 && lane == 0 && q_i < p.seqlen_q && !row_store) {
       for (int bx = 0; bx < C::NBOX; ++bx)
-        tma_store_4d(&tm_o, stage + bx * (BM * 128), bx * 64, h, q_i, b);
+        tma_store_4d(&tm_o, stage + bx * (BM * 128), bx * 64, h, sq.q_row0 + q_i, sq.tma_b);
       bulk_commit_group();
       bulk_wait_group_read_all();
     }

@@ -57,6 +57,36 @@ __device__ __forceinline__ UnitOrder grouped_lpt(int L, int units, int heads, in
   return {idx / gsize, g0 + idx % gsize};
 }
 
+// ---------------------------------------------------------------- sequences
+// Rows of sequence b.  Dense layout (cu_q == nullptr): batch entry b of the
+// (batch, seqlen, heads, d) tensors, TMA batch coordinate b, rows from 0.
+// Packed layout: rows [cu_q[b], cu_q[b+1]) of the (total_q, heads, d) query
+// tensors and [cu_k[b], cu_k[b+1]) of the key tensors, TMA batch coordinate
+// 0.  Offsets are clamped to the tensors, so malformed offsets can give wrong
+// results but never an access outside them.
+struct SeqSpan {
+  int q_row0, k_row0, len_q, len_k, tma_b;
+};
+__device__ __forceinline__ SeqSpan seq_span(const int* cu_q, const int* cu_k, int total_q,
+                                            int total_k, int b, int seqlen_q, int seqlen_k) {
+  if (cu_q == nullptr) return {0, 0, seqlen_q, seqlen_k, b};
+  const int q0 = min(max(__ldg(cu_q + b), 0), total_q);
+  const int q1 = min(max(__ldg(cu_q + b + 1), q0), total_q);
+  const int k0 = min(max(__ldg(cu_k + b), 0), total_k);
+  const int k1 = min(max(__ldg(cu_k + b + 1), k0), total_k);
+  return {q0, k0, q1 - q0, k1 - k0, 0};
+}
+
+// 32 16-bit values (packed in pairs) from registers to global memory, for
+// tiles that end past their packed sequence, where a TMA store would write
+// into the next sequence.  `dst` is 16-byte aligned.
+__device__ __forceinline__ void store_row32(uint16_t* dst, const uint32_t (&w)[16]) {
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int q4 = 0; q4 < 4; ++q4)
+    d4[q4] = make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
+}
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");

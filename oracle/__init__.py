@@ -137,6 +137,46 @@ class Oracle:
         return dq, dk, dv
 
 
+    # Packed variable-length sequences: each sequence is its own attention
+    # problem (the varlen interface of "FlashAttention-2：下一代高效注意力机制
+    # 的突破与实战解析", section "实操落地"), so the oracle runs the dense
+    # definition on every sequence's rows.
+    def attention_fwd_varlen(self, q, k, v, cu_q, cu_k, softmax_scale=None, causal=False,
+                             window_left=-1, window_right=-1):
+        """q (Tq, H, d), k, v (Tk, Hkv, d), offsets cu_q, cu_k (batch + 1):
+        O (Tq, H, d) and LSE (H, Tq), float64."""
+        qa, ka, va = _f64(q), _f64(k), _f64(v)
+        cq, ck = _offsets(cu_q), _offsets(cu_k)
+        Tq, H, d = qa.shape
+        o = np.zeros((Tq, H, d))
+        lse = np.zeros((H, Tq))
+        for b in range(len(cq) - 1):
+            q0, q1, k0, k1 = cq[b], cq[b + 1], ck[b], ck[b + 1]
+            if q1 == q0:
+                continue
+            ob, lb = self.attention_fwd(qa[None, q0:q1], ka[None, k0:k1], va[None, k0:k1],
+                                        softmax_scale, causal, window_left, window_right)
+            o[q0:q1] = ob[0]
+            lse[:, q0:q1] = lb[0]
+        return o, lse
+
+    def attention_bwd_varlen(self, q, k, v, dout, cu_q, cu_k, softmax_scale=None, causal=False,
+                             window_left=-1, window_right=-1):
+        """dQ (Tq, H, d), dK and dV (Tk, Hkv, d), float64, per sequence."""
+        qa, ka, va, da = _f64(q), _f64(k), _f64(v), _f64(dout)
+        cq, ck = _offsets(cu_q), _offsets(cu_k)
+        dq, dk, dv = np.zeros_like(qa), np.zeros_like(ka), np.zeros_like(va)
+        for b in range(len(cq) - 1):
+            q0, q1, k0, k1 = cq[b], cq[b + 1], ck[b], ck[b + 1]
+            if q1 == q0 or k1 == k0:
+                continue
+            g = self.attention_bwd(qa[None, q0:q1], ka[None, k0:k1], va[None, k0:k1],
+                                   da[None, q0:q1], softmax_scale, causal, window_left,
+                                   window_right)
+            dq[q0:q1], dk[k0:k1], dv[k0:k1] = g[0][0], g[1][0], g[2][0]
+        return dq, dk, dv
+
+
 def default() -> Oracle:
     """The oracle built from ``attn_oracle.c`` beside this file."""
     global _lib
@@ -159,6 +199,16 @@ def _f64(t) -> np.ndarray:
     if isinstance(t, np.ndarray):
         return np.ascontiguousarray(t, dtype=np.float64)
     return np.ascontiguousarray(t.detach().to("cpu", torch.float64).numpy())
+
+
+def _offsets(cu) -> list:
+    import torch
+    if isinstance(cu, torch.Tensor):
+        cu = cu.detach().cpu().tolist()
+    cu = [int(x) for x in cu]
+    if not cu or cu[0] != 0 or any(b < a for a, b in zip(cu, cu[1:])):
+        raise ValueError("sequence offsets must start at 0 and not decrease")
+    return cu
 
 
 def _ptr(a: np.ndarray, ty=ctypes.c_double):
@@ -189,3 +239,11 @@ def attention_bwd(*a, **kw):
 
 def attention_bwd_rows(*a, **kw):
     return default().attention_bwd_rows(*a, **kw)
+
+
+def attention_fwd_varlen(*a, **kw):
+    return default().attention_fwd_varlen(*a, **kw)
+
+
+def attention_bwd_varlen(*a, **kw):
+    return default().attention_bwd_varlen(*a, **kw)

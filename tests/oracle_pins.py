@@ -363,6 +363,53 @@ def pin_rows_match_full(orc):
         _close(dv_r, dv[:, krows], 1e-13, f"rows dV {m}")
 
 
+def pin_varlen_per_sequence(orc):
+    """Packed sequences: every sequence's rows equal torch's scaled dot
+    product attention (float64, explicit bottom-right mask, autograd
+    gradients) run on that sequence alone, with query and key lengths that
+    differ per sequence, an empty query sequence and an empty key sequence;
+    rows of a sequence with no keys get O = 0, LSE = -inf and zero
+    gradients."""
+    import torch.nn.functional as F
+    H, Hkv, d, scale = 4, 2, 8, 0.35
+    lq = [5, 0, 9, 3, 7]
+    lk = [7, 4, 9, 0, 2]
+    cq = np.concatenate([[0], np.cumsum(lq)]).tolist()
+    ck = np.concatenate([[0], np.cumsum(lk)]).tolist()
+    q, k, v = rand((cq[-1], H, d), 70), rand((ck[-1], Hkv, d), 71), rand((ck[-1], Hkv, d), 72)
+    do = rand((cq[-1], H, d), 73)
+    for m in MASKS:
+        o, lse = orc.attention_fwd_varlen(q, k, v, cq, ck, scale, **m)
+        dq, dk, dv = orc.attention_bwd_varlen(q, k, v, do, cq, ck, scale, **m)
+        assert o.shape == (cq[-1], H, d) and lse.shape == (H, cq[-1])
+        for b in range(len(lq)):
+            q0, q1, k0, k1 = cq[b], cq[b + 1], ck[b], ck[b + 1]
+            if q1 == q0:
+                continue
+            if k1 == k0:
+                assert np.all(o[q0:q1] == 0.0) and np.all(lse[:, q0:q1] == -np.inf)
+                assert np.all(dq[q0:q1] == 0.0)
+                continue
+            vis = mask_matrix(q1 - q0, k1 - k0, **m)
+            seen = vis.any(axis=1)
+            qt = q[q0:q1].permute(1, 0, 2)[None].clone().requires_grad_(True)
+            kt = k[k0:k1].permute(1, 0, 2)[None].clone().requires_grad_(True)
+            vt = v[k0:k1].permute(1, 0, 2)[None].clone().requires_grad_(True)
+            rep = H // Hkv
+            # rows with no visible key are left out of the library call
+            out = F.scaled_dot_product_attention(
+                qt[:, :, seen], kt.repeat_interleave(rep, dim=1),
+                vt.repeat_interleave(rep, dim=1), attn_mask=torch.from_numpy(vis[seen]),
+                scale=scale)
+            (out * do[q0:q1][seen].permute(1, 0, 2)[None]).sum().backward()
+            _close(o[q0:q1][seen], out.detach()[0].permute(1, 0, 2).numpy(), 1e-10,
+                   f"varlen O seq {b} {m}")
+            assert np.all(o[q0:q1][~seen] == 0.0)
+            _close(dq[q0:q1], qt.grad[0].permute(1, 0, 2).numpy(), 1e-10, f"varlen dQ {b} {m}")
+            _close(dk[k0:k1], kt.grad[0].permute(1, 0, 2).numpy(), 1e-10, f"varlen dK {b} {m}")
+            _close(dv[k0:k1], vt.grad[0].permute(1, 0, 2).numpy(), 1e-10, f"varlen dV {b} {m}")
+
+
 ALL_PINS = [
     pin_golden_handworked,
     pin_identical_keys,
@@ -376,4 +423,5 @@ ALL_PINS = [
     pin_gqa_equals_repeated_mha,
     pin_empty_rows,
     pin_rows_match_full,
+    pin_varlen_per_sequence,
 ]
