@@ -70,6 +70,45 @@ WORKLOADS: Dict[str, Workload] = {
 }
 
 
+@dataclasses.dataclass(frozen=True)
+class VarlenWorkload:
+    """Packed variable-length sequences: per-sequence query and key lengths
+    (equal here), shared head counts, mask and input distribution."""
+
+    name: str
+    lens: tuple
+    nheads: int
+    nheads_kv: int
+    headdim: int
+    causal: bool
+    window_left: int = -1
+    window_right: int = -1
+    dtype: str = "bf16"
+    sigma: float = 1.0
+    seed: int = 0
+    passes: str = "fwd+bwd"
+    softmax_scale: Optional[float] = None
+
+    @property
+    def scale(self) -> float:
+        return self.softmax_scale if self.softmax_scale is not None else 1.0 / math.sqrt(self.headdim)
+
+
+def _uniform_lengths(n: int, lo: int, hi: int, seed: int) -> tuple:
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    return tuple(int(x) for x in torch.randint(lo, hi + 1, (n,), generator=g))
+
+
+# A length mix for the packed entry points: 16 causal sequences of 256-1792
+# tokens (uniform, seeded), about the token count of the causal N=8192 batch.
+VARLEN_WORKLOADS: Dict[str, VarlenWorkload] = {
+    "varlen_causal_16seq_h32_d128": VarlenWorkload(
+        "varlen_causal_16seq_h32_d128", _uniform_lengths(16, 256, 1792, 11), 32, 32, 128, True,
+        seed=11),
+}
+
+
 def make_inputs(w: Workload, with_dout: bool = True, device: str = "cpu"):
     """Draw (q, k, v, dout) for workload ``w``.
 

@@ -473,6 +473,182 @@ def run_gpu(args):
     return 0
 
 
+# ---------------------------------------------------------------- packed arm
+def varlen_flops(w):
+    """(forward, backward) FLOPs of a packed workload: exact visible pairs of
+    every sequence x 4d (forward), x 2.5 of that (backward)."""
+    pairs = sum(visible_pairs(n, n, w.causal, w.window_left, w.window_right) for n in w.lens)
+    fwd = 4.0 * w.nheads * w.headdim * pairs
+    return fwd, (2.5 * fwd if "bwd" in w.passes else 0.0)
+
+
+def varlen_config(w):
+    return {"workload": w.name, "sequences": len(w.lens), "tokens": sum(w.lens),
+            "lengths": list(w.lens), "nheads": w.nheads, "nheads_kv": w.nheads_kv,
+            "headdim": w.headdim, "causal": w.causal, "pass": w.passes, "dtype": w.dtype,
+            "softmax_scale": w.scale, "layout": "packed (cu_seqlens)",
+            "inputs": f"Q,K,V,dO ~ N(0,{w.sigma:g}^2), seed {w.seed}",
+            "l2": "no flush: inputs exceed the 126 MB L2",
+            "flops": "exact visible pairs x 4d (fwd), x 10d (bwd)",
+            "parallelism": "replicas (weak scaling, no collective)"}
+
+
+def varlen_cpu_baseline(w, inputs, target_s=12.0):
+    """The float64 oracle on the last rows of the longest sequence (its keys
+    in full), sized to about ``target_s`` seconds."""
+    import oracle
+    oracle.build()
+    q, k, v, do, cu_q, cu_k = inputs
+    threads = oracle.num_threads()
+    heads = max(1, min(w.nheads, threads))
+    kvh = max(1, heads * w.nheads_kv // w.nheads)
+    b = max(range(len(w.lens)), key=lambda i: w.lens[i])
+    q0, n = int(cu_q[b]), w.lens[b]
+
+    def run(rows):
+        sl = slice(q0 + n - rows, q0 + n)
+        qs = q[sl, :heads][None].contiguous()
+        dos = do[sl, :heads][None].contiguous()
+        ks = k[q0:q0 + n, :kvh][None].contiguous()
+        vs = v[q0:q0 + n, :kvh][None].contiguous()
+        t0 = time.perf_counter()
+        oracle.attention_fwd(qs, ks, vs, w.scale, w.causal, w.window_left, w.window_right)
+        oracle.attention_bwd(qs, ks, vs, dos, w.scale, w.causal, w.window_left, w.window_right)
+        dt = time.perf_counter() - t0
+        pairs = visible_pairs(n, n, w.causal, w.window_left, w.window_right,
+                              rows=range(n - rows, n))
+        return dt, pairs * heads * 14.0 * w.headdim
+
+    dt, _ = run(16)
+    rows = int(min(n, max(16, 16 * target_s / max(dt, 1e-3))))
+    dt, flops = run(rows)
+    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": (f"float64 oracle fwd+bwd on the last {rows} queries of {heads} heads of "
+                       f"the longest sequence ({n} tokens) of {w.name}; "
+                       f"{flops / 1e9:.1f} GFLOP in {dt:.1f} s")}
+
+
+def run_gpu_varlen(args, w):
+    """The packed entry points on a length mix: attn_fwd_varlen then
+    attn_bwd_varlen (its three kernels) per step."""
+    import torch
+    import io_aware_exact_33_b200 as attn
+    from attn_inputs import make_varlen_inputs
+
+    rank, local_rank, world = world_info()
+    dist = init_dist("nccl", world)
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    f_fwd, f_bwd = varlen_flops(w)
+    inputs = make_varlen_inputs(w.lens, w.lens, w.nheads, w.nheads_kv, w.headdim, w.dtype,
+                                w.sigma, w.seed)
+    q, k, v, do, cu_q, cu_k = inputs
+    qd, kd, vd, dod, cqd, ckd = (t.to(dev) for t in inputs)
+    mx = max(w.lens)
+    args_m = (w.scale, w.causal, w.window_left, w.window_right)
+    o = torch.empty_like(qd)
+    lse = torch.empty((w.nheads, qd.shape[0]), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
+    p = attn.make_varlen_params(len(w.lens), qd.shape[0], kd.shape[0], mx, mx, w.nheads,
+                                w.nheads_kv, w.headdim, attn._dtype_code(qd), w.scale, w.causal,
+                                w.window_left, w.window_right)
+    ws = torch.empty(attn.attn_bwd_varlen_workspace_size(p), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+
+    def step(ev=None):
+        if ev: ev[0].record(stream)
+        attn.attn_fwd_varlen(qd, kd, vd, cqd, ckd, mx, mx, *args_m, out=o, lse=lse)
+        if ev: ev[1].record(stream)
+        attn.attn_bwd_varlen(qd, kd, vd, o, lse, dod, cqd, ckd, mx, mx, *args_m, dq=dq, dk=dk,
+                             dv=dv, workspace=ws)
+        if ev: ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if attn.attn_get_device_status() != 0:
+        raise RuntimeError("device status word reports an error after warm-up")
+    gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(dist, dev)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(gpu_id) as clk:
+        start.record(stream)
+        for i in range(args.steps):
+            step(events[i])
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(dist, dev)
+    ms = max_over_ranks(start.elapsed_time(end), dist, dev)
+    t_fwd = [e[0].elapsed_time(e[1]) for e in events]
+    t_bwd = [e[1].elapsed_time(e[2]) for e in events]
+    value = (f_fwd + f_bwd) * args.steps * world / (ms / 1e3) / 1e12
+
+    k_e2e = max(1, min(args.steps, args.e2e_steps))
+    host = [t.pin_memory() for t in (q, k, v, do, cu_q, cu_k)]
+    ho, hlse = torch.empty_like(host[0]).pin_memory(), torch.empty(lse.shape).pin_memory()
+    hg = [torch.empty_like(t).pin_memory() for t in host[:3]]
+
+    def e2e_step():
+        for dst, src in zip((qd, kd, vd, dod, cqd, ckd), host):
+            dst.copy_(src, non_blocking=True)
+        attn.attn_fwd_varlen(qd, kd, vd, cqd, ckd, mx, mx, *args_m, out=o, lse=lse)
+        attn.attn_bwd_varlen(qd, kd, vd, o, lse, dod, cqd, ckd, mx, mx, *args_m, dq=dq, dk=dk,
+                             dv=dv, workspace=ws)
+        for dst, src in zip([ho, hlse] + hg, (o, lse, dq, dk, dv)):
+            dst.copy_(src, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier(dist, dev)
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record(stream)
+    for _ in range(k_e2e):
+        e2e_step()
+    e2.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(dist, dev)
+    ms_e2e = max_over_ranks(s2.elapsed_time(e2), dist, dev)
+    h2d = sum(t.numel() * t.element_size() for t in host)
+    d2h = sum(t.numel() * t.element_size() for t in [ho, hlse] + hg)
+    status = attn.attn_get_device_status()
+    if rank != 0:
+        if dist is not None:
+            dist.destroy_process_group()
+        return 0
+    peaks, peak_kind = load_peaks()
+    mean = lambda xs: sum(xs) / len(xs)
+    rl = {}
+    for name, ms_k, fl in (("attn_fwd_varlen", mean(t_fwd), f_fwd),
+                           ("attn_bwd_varlen (3 kernels)", mean(t_bwd), f_bwd)):
+        a = fl / (ms_k / 1e3) / 1e12
+        rl[name] = {"bound": "tensor", "achieved": a, "peak": peaks["bf16_tflops"], "unit": UNIT,
+                    "frac": a / peaks["bf16_tflops"], "traffic": None,
+                    "peak_source": f"bf16_tflops (burst) of {peak_kind}", "ms_per_launch": ms_k,
+                    "flops_per_launch": fl}
+    dominant = max(rl, key=lambda n: rl[n]["ms_per_launch"])
+    cpu = varlen_cpu_baseline(w, inputs) if (world == 1 and not args.no_cpu_baseline) else None
+    line = {
+        "metric": "packed variable-length attention fwd/bwd TFLOP/s", "value": value,
+        "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype, "data": f"synthetic ({varlen_config(w)['inputs']})",
+        "config": varlen_config(w),
+        "fwd_tflops": rl["attn_fwd_varlen"]["achieved"],
+        "bwd_tflops": rl["attn_bwd_varlen (3 kernels)"]["achieved"],
+        "ms": {"fwd": mean(t_fwd), "bwd": mean(t_bwd)},
+        "roofline": dict(rl[dominant], kernel=dominant), "kernels": rl, "cpu_baseline": cpu,
+        "e2e": {"value": (f_fwd + f_bwd) * k_e2e * world / (ms_e2e / 1e3) / 1e12, "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": k_e2e},
+        "clocks": clk.summary(), "gpu_launches": 4 * args.steps, "device_status": status,
+    }
+    print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
 PROBE_CASES = [  # (description, M, N) in the order of probe_mma_case()
     ("A smem K-major, B smem K-major, 1 accumulator", 128, 128),
     ("A smem K-major, B smem K-major, 2 accumulators", 128, 128),
@@ -535,9 +711,16 @@ def main(argv=None):
         return 0
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
-    from attn_inputs import WORKLOADS
+    from attn_inputs import VARLEN_WORKLOADS, WORKLOADS
+    if args.workload in VARLEN_WORKLOADS:
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable":
+                              "the reference arm times the dense headline workload only"}))
+            return 0
+        return run_gpu_varlen(args, VARLEN_WORKLOADS[args.workload])
     if args.workload not in WORKLOADS:
-        ap.error(f"unknown workload {args.workload}; choose from {sorted(WORKLOADS)}")
+        ap.error(f"unknown workload {args.workload}; choose from "
+                 f"{sorted(WORKLOADS) + sorted(VARLEN_WORKLOADS)}")
     if input_bytes(WORKLOADS[args.workload]) < 2 * 126e6:
         ap.error(f"{args.workload} fits in L2; it is a parity case, not a bench workload")
     if args.impl == "reference":
