@@ -137,7 +137,33 @@ __device__ inline int packed_seq_of_token(const BwdParams& p, long long t) {
 }
 
 // ------------------------------------------------------------ preprocess
-// One warp per (b, h, i) row of the padded range: Dvec_i = sum_c dO_ic O_ic,
+// fp32 dot product of eight 16-bit values of `a` and `b` (16 bytes each).
+template <bool FP16>
+__device__ __forceinline__ float dot8(uint4 a, uint4 b) {
+  const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+  float acc = 0.f;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    float a0, a1, b0, b1;
+    if constexpr (FP16) {
+      a0 = __half2float(__ushort_as_half((unsigned short)(av[k] & 0xFFFFu)));
+      a1 = __half2float(__ushort_as_half((unsigned short)(av[k] >> 16)));
+      b0 = __half2float(__ushort_as_half((unsigned short)(bv[k] & 0xFFFFu)));
+      b1 = __half2float(__ushort_as_half((unsigned short)(bv[k] >> 16)));
+    } else {
+      a0 = __uint_as_float(av[k] << 16);
+      a1 = __uint_as_float(av[k] & 0xFFFF0000u);
+      b0 = __uint_as_float(bv[k] << 16);
+      b1 = __uint_as_float(bv[k] & 0xFFFF0000u);
+    }
+    acc = fmaf(a0, b0, acc);
+    acc = fmaf(a1, b1, acc);
+  }
+  return acc;
+}
+
+// Rows of the padded (b, h, i) range, headdim / 8 lanes per row with one
+// 16-byte load of O and of dO each: Dvec_i = sum_c dO_ic O_ic and
 // LSE2_i = LSE_i * log2(e); padding rows get 0 and +inf (P = 0 there).  All
 // threads then zero the dQ accumulator.
 template <bool FP16>
@@ -145,60 +171,51 @@ __global__ void __launch_bounds__(256) bwd_preprocess(const uint16_t* __restrict
                                                       const uint16_t* __restrict__ dout,
                                                       BwdParams p, long long n_rows,
                                                       long long n_zero4) {
-  const long long warp_global = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 5;
+  const int lpr = p.headdim / 8;          // lanes per row: 8 (d = 64) or 16 (d = 128)
+  const int rpw = 32 / lpr;               // rows per warp step
   const int lane = threadIdx.x & 31;
+  const int sub = lane % lpr;
+  const long long warp_global = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 5;
   const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
-  for (long long row = warp_global; row < n_rows; row += nwarps) {
+  for (long long row0 = warp_global * rpw; row0 < n_rows; row0 += nwarps * rpw) {
+    const long long row = row0 + lane / lpr;
+    const bool in_range = row < n_rows;
     const long long ip = row % p.nq_pad;
     const long long bh = row / p.nq_pad;
-    int h, b;
-    long long i, tok;  // row within the sequence; row of the o / dout / lse tensors
-    bool valid;
-    if (p.cu_q) {
-      h = (int)bh;
-      b = packed_seq_of_row(p, ip);
-      const SeqSpan sq = seq_span(p.cu_q, p.cu_k, p.total_q, p.total_k, b, 0, 0);
-      i = ip - packed_row0(sq.q_row0, b);
-      valid = i >= 0 && i < sq.len_q;
-      tok = sq.q_row0 + i;
-    } else {
-      h = (int)(bh % p.nheads);
-      b = (int)(bh / p.nheads);
-      i = ip;
-      valid = i < p.seqlen_q;
-      tok = (long long)b * p.seqlen_q + i;
-    }
-    float dv = 0.f, l2 = INFINITY;
-    if (valid) {
-      const size_t base = ((size_t)tok * p.nheads + h) * p.headdim;
-      float acc = 0.f;
-      for (int c = lane * 2; c < p.headdim; c += 64) {
-        const uint32_t ov = *reinterpret_cast<const uint32_t*>(o + base + c);
-        const uint32_t dov = *reinterpret_cast<const uint32_t*>(dout + base + c);
-        float o0, o1, d0, d1;
-        if constexpr (FP16) {
-          o0 = __half2float(__ushort_as_half((unsigned short)(ov & 0xFFFFu)));
-          o1 = __half2float(__ushort_as_half((unsigned short)(ov >> 16)));
-          d0 = __half2float(__ushort_as_half((unsigned short)(dov & 0xFFFFu)));
-          d1 = __half2float(__ushort_as_half((unsigned short)(dov >> 16)));
-        } else {
-          o0 = __uint_as_float(ov << 16);
-          o1 = __uint_as_float(ov & 0xFFFF0000u);
-          d0 = __uint_as_float(dov << 16);
-          d1 = __uint_as_float(dov & 0xFFFF0000u);
-        }
-        acc = fmaf(o0, d0, acc);
-        acc = fmaf(o1, d1, acc);
+    int h = 0, b = 0;
+    long long i = 0, tok = 0;  // row within the sequence; row of the o / dout / lse tensors
+    bool valid = false;
+    if (in_range) {
+      if (p.cu_q) {
+        h = (int)bh;
+        b = packed_seq_of_row(p, ip);
+        const SeqSpan sq = seq_span(p.cu_q, p.cu_k, p.total_q, p.total_k, b, 0, 0);
+        i = ip - packed_row0(sq.q_row0, b);
+        valid = i >= 0 && i < sq.len_q;
+        tok = sq.q_row0 + i;
+      } else {
+        h = (int)(bh % p.nheads);
+        b = (int)(bh / p.nheads);
+        i = ip;
+        valid = i < p.seqlen_q;
+        tok = (long long)b * p.seqlen_q + i;
       }
-#pragma unroll
-      for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
-      dv = acc;
-      const float l = p.cu_q ? p.lse[(size_t)h * p.total_q + tok]
-                             : p.lse[((size_t)b * p.nheads + h) * p.seqlen_q + i];
-      l2 = (l == -INFINITY) ? INFINITY : l * 1.4426950408889634f;
     }
-    if (lane == 0) {
-      p.dvec[row] = dv;
+    float acc = 0.f;
+    if (valid) {
+      const size_t base = ((size_t)tok * p.nheads + h) * p.headdim + sub * 8;
+      acc = dot8<FP16>(*reinterpret_cast<const uint4*>(o + base),
+                       *reinterpret_cast<const uint4*>(dout + base));
+    }
+    for (int s = lpr / 2; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+    if (in_range && sub == 0) {
+      float l2 = INFINITY;
+      if (valid) {
+        const float l = p.cu_q ? p.lse[(size_t)h * p.total_q + tok]
+                               : p.lse[((size_t)b * p.nheads + h) * p.seqlen_q + i];
+        l2 = (l == -INFINITY) ? INFINITY : l * 1.4426950408889634f;
+      }
+      p.dvec[row] = valid ? acc : 0.f;
       p.lse2[row] = l2;
     }
   }
