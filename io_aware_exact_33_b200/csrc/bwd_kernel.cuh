@@ -358,13 +358,49 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   const int nqb = imax >= imin ? (int)(imax / BM) - qb_lo + 1 : 0;
   const int nt = nqb * group;  // tiles: (head in group) x (query tile)
 
-  if (threadIdx.x == 0) {
+  // Q, LSE2, dO, Dvec of tile t (query head, query tile) into its slot.
+  auto load_q = [&](int t) -> bool {
+    const int slot = t % QS, n = t / QS;
+    if (n > 0 && !mbar_wait(bar(C::B_EMPTY + slot), (n - 1) & 1)) return false;
+    const int h = kvh * group + t / nqb;
+    const int q0 = (qb_lo + t % nqb) * BM;
+    // Dvec / LSE2 coordinates: (padded row, head) packed, (row, batch*head) dense
+    const int row = p.cu_q ? h : b * p.nheads + h;
+    const int xs = (int)prow0 + q0;
+    mbar_arrive_expect_tx(bar(C::B_QFULL + slot), C::Q_BYTES + BM * 4);
+    for (int bx = 0; bx < C::NBOX; ++bx)
+      tma_load_4d(smem0 + C::OFF_Q + slot * C::Q_BYTES + bx * (BM * 128), &tm_q,
+                  bar(C::B_QFULL + slot), bx * 64, h, sq.q_row0 + q0, sq.tma_b);
+    tma_load_2d(smem0 + C::OFF_LSE + slot * BM * 4, &tm_lse2, bar(C::B_QFULL + slot), xs, row);
+    mbar_arrive_expect_tx(bar(C::B_DOFULL + slot), C::Q_BYTES + BM * 4);
+    for (int bx = 0; bx < C::NBOX; ++bx)
+      tma_load_4d(smem0 + C::OFF_DO + slot * C::Q_BYTES + bx * (BM * 128), &tm_do,
+                  bar(C::B_DOFULL + slot), bx * 64, h, sq.q_row0 + q0, sq.tma_b);
+    tma_load_2d(smem0 + C::OFF_DVEC + slot * BM * 4, &tm_dvec, bar(C::B_DOFULL + slot), xs, row);
+    return true;
+  };
+
+  // The producer lane initialises the barriers and starts the K, V and
+  // first query-tile loads before the block-wide barrier, so that their
+  // latency overlaps the tensor-memory allocation and the barrier itself.
+  if (warp == 8 && lane == 0) {
     for (int i = 0; i < C::NBAR; ++i) {
       const bool many = (i >= C::B_PREADY && i < C::B_DSREADY + NBUF) ||
                         (i >= C::B_DQFREE && i < C::B_DQFREE + NBUF);
       mbar_init(bar(i), many ? 256 : 1);
     }
     fence_barrier_init();
+    fence_proxy_async_smem();
+    if (nt > 0) {
+      mbar_arrive_expect_tx(bar(C::B_KV), 2 * C::KV_BYTES);
+      for (int bx = 0; bx < C::NBOX; ++bx) {
+        tma_load_4d(smem0 + C::OFF_K + bx * (BN * 128), &tm_k, bar(C::B_KV), bx * 64, kvh,
+                    sq.k_row0 + k0, sq.tma_b);
+        tma_load_4d(smem0 + C::OFF_V + bx * (BN * 128), &tm_v, bar(C::B_KV), bx * 64, kvh,
+                    sq.k_row0 + k0, sq.tma_b);
+      }
+      load_q(0);  // first use of its slot: no wait
+    }
   }
   if (warp == 9) {
     tmem_alloc(smem0 + C::OFF_TMEMPTR, C::TMEM_COLS);
@@ -378,32 +414,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && nt > 0) {
-      mbar_arrive_expect_tx(bar(C::B_KV), 2 * C::KV_BYTES);
-      for (int bx = 0; bx < C::NBOX; ++bx) {
-        tma_load_4d(smem0 + C::OFF_K + bx * (BN * 128), &tm_k, bar(C::B_KV), bx * 64, kvh,
-                    sq.k_row0 + k0, sq.tma_b);
-        tma_load_4d(smem0 + C::OFF_V + bx * (BN * 128), &tm_v, bar(C::B_KV), bx * 64, kvh,
-                    sq.k_row0 + k0, sq.tma_b);
-      }
-      for (int t = 0; t < nt; ++t) {
-        const int slot = t % QS, n = t / QS;
-        if (n > 0 && !mbar_wait(bar(C::B_EMPTY + slot), (n - 1) & 1)) break;
-        const int h = kvh * group + t / nqb;
-        const int q0 = (qb_lo + t % nqb) * BM;
-        // Dvec / LSE2 coordinates: (padded row, head) packed, (row, batch*head) dense
-        const int row = p.cu_q ? h : b * p.nheads + h;
-        const int xs = (int)prow0 + q0;
-        mbar_arrive_expect_tx(bar(C::B_QFULL + slot), C::Q_BYTES + BM * 4);
-        for (int bx = 0; bx < C::NBOX; ++bx)
-          tma_load_4d(smem0 + C::OFF_Q + slot * C::Q_BYTES + bx * (BM * 128), &tm_q,
-                      bar(C::B_QFULL + slot), bx * 64, h, sq.q_row0 + q0, sq.tma_b);
-        tma_load_2d(smem0 + C::OFF_LSE + slot * BM * 4, &tm_lse2, bar(C::B_QFULL + slot), xs, row);
-        mbar_arrive_expect_tx(bar(C::B_DOFULL + slot), C::Q_BYTES + BM * 4);
-        for (int bx = 0; bx < C::NBOX; ++bx)
-          tma_load_4d(smem0 + C::OFF_DO + slot * C::Q_BYTES + bx * (BM * 128), &tm_do,
-                      bar(C::B_DOFULL + slot), bx * 64, h, sq.q_row0 + q0, sq.tma_b);
-        tma_load_2d(smem0 + C::OFF_DVEC + slot * BM * 4, &tm_dvec, bar(C::B_DOFULL + slot), xs, row);
-      }
+      for (int t = 1; t < nt; ++t)  // K, V and tile 0 are on their way
+        if (!load_q(t)) break;
       for (int t = nt - QS < 0 ? 0 : nt - QS; t < nt; ++t) {
         const int slot = t % QS, n = t / QS;
         if (!mbar_wait(bar(C::B_QFULL + slot), n & 1)) break;

@@ -589,20 +589,53 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   const int uhi = has0 && has1 ? max(hi[0], hi[1]) : (has0 ? hi[0] : hi[1]);
   const int nt = (has0 || has1) ? uhi - ulo : 0;
 
-  if (threadIdx.x == 0) {
+  // K and V slots are released separately: K_j after key tile j's last S
+  // MMA (same iteration), V_j after its last PV MMA (up to one later).  K
+  // runs one tile ahead of V in the issue order, so a V slot that is still
+  // in use never holds back the next K load.
+  auto load_k = [&](int t) -> bool {
+    const int st = t % KS, n = t / KS;
+    if (n > 0 && !mbar_wait(bar(C::B_KEMPTY + st), (n - 1) & 1)) return false;
+    mbar_arrive_expect_tx(bar(C::B_KFULL + st), C::KV_BYTES);
+    for (int bx = 0; bx < C::NBOX; ++bx)
+      tma_load_4d(smem0 + C::OFF_K + st * C::KV_BYTES + bx * (BN * 128), &tm_k,
+                  bar(C::B_KFULL + st), bx * 64, kvh, sq.k_row0 + (ulo + t) * BN, sq.tma_b);
+    return true;
+  };
+  auto load_v = [&](int t) -> bool {
+    const int st = t % VS, n = t / VS;
+    if (n > 0 && !mbar_wait(bar(C::B_VEMPTY + st), (n - 1) & 1)) return false;
+    mbar_arrive_expect_tx(bar(C::B_VFULL + st), C::KV_BYTES);
+    for (int bx = 0; bx < C::NBOX; ++bx)
+      tma_load_4d(smem0 + C::OFF_V + st * C::KV_BYTES + bx * (BN * 128), &tm_v,
+                  bar(C::B_VFULL + st), bx * 64, kvh, sq.k_row0 + (ulo + t) * BN, sq.tma_b);
+    return true;
+  };
+
+  // The producer lane initialises the barriers and starts the Q and first K
+  // loads before the block-wide barrier, so that their latency overlaps the
+  // tensor-memory allocation and the barrier itself.
+  if (warp == 8 && lane == 0) {
     for (int i = 0; i < C::NBAR; ++i)
       mbar_init(bar(i), (i >= C::B_PREADY && i < C::B_PREADY + 4) ? 128 : 1);
     fence_barrier_init();
-  }
-  if (warp == 9) {
-    tmem_alloc(smem0 + C::OFF_TMEMPTR, C::TMEM_COLS);
-    tmem_relinquish();
-  }
-  if (warp == 8 && lane == 0) {
+    fence_proxy_async_smem();
     prefetch_tensormap(&tm_q);
     prefetch_tensormap(&tm_k);
     prefetch_tensormap(&tm_v);
     prefetch_tensormap(&tm_o);
+    if (nt > 0) {
+      mbar_arrive_expect_tx(bar(C::B_Q), 2 * C::Q_BYTES);
+      for (int i = 0; i < 2; ++i)
+        for (int bx = 0; bx < C::NBOX; ++bx)
+          tma_load_4d(smem0 + C::OFF_Q + i * C::Q_BYTES + bx * (BM * 128), &tm_q, bar(C::B_Q),
+                      bx * 64, h, sq.q_row0 + qs[i], sq.tma_b);
+      load_k(0);  // first use of its slot: no wait
+    }
+  }
+  if (warp == 9) {
+    tmem_alloc(smem0 + C::OFF_TMEMPTR, C::TMEM_COLS);
+    tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
@@ -612,34 +645,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && nt > 0) {
-      mbar_arrive_expect_tx(bar(C::B_Q), 2 * C::Q_BYTES);
-      for (int i = 0; i < 2; ++i)
-        for (int bx = 0; bx < C::NBOX; ++bx)
-          tma_load_4d(smem0 + C::OFF_Q + i * C::Q_BYTES + bx * (BM * 128), &tm_q, bar(C::B_Q),
-                      bx * 64, h, sq.q_row0 + qs[i], sq.tma_b);
-      // K and V slots are released separately: K_j after key tile j's last S
-      // MMA (same iteration), V_j after its last PV MMA (up to one later).
-      // K runs one tile ahead of V in the issue order, so a V slot that is
-      // still in use never holds back the next K load.
-      auto load_k = [&](int t) -> bool {
-        const int st = t % KS, n = t / KS;
-        if (n > 0 && !mbar_wait(bar(C::B_KEMPTY + st), (n - 1) & 1)) return false;
-        mbar_arrive_expect_tx(bar(C::B_KFULL + st), C::KV_BYTES);
-        for (int bx = 0; bx < C::NBOX; ++bx)
-          tma_load_4d(smem0 + C::OFF_K + st * C::KV_BYTES + bx * (BN * 128), &tm_k,
-                      bar(C::B_KFULL + st), bx * 64, kvh, sq.k_row0 + (ulo + t) * BN, sq.tma_b);
-        return true;
-      };
-      auto load_v = [&](int t) -> bool {
-        const int st = t % VS, n = t / VS;
-        if (n > 0 && !mbar_wait(bar(C::B_VEMPTY + st), (n - 1) & 1)) return false;
-        mbar_arrive_expect_tx(bar(C::B_VFULL + st), C::KV_BYTES);
-        for (int bx = 0; bx < C::NBOX; ++bx)
-          tma_load_4d(smem0 + C::OFF_V + st * C::KV_BYTES + bx * (BN * 128), &tm_v,
-                      bar(C::B_VFULL + st), bx * 64, kvh, sq.k_row0 + (ulo + t) * BN, sq.tma_b);
-        return true;
-      };
-      bool go = load_k(0);
+      bool go = true;  // Q and K_0 are on their way
       for (int t = 0; go && t < nt; ++t) {
         if (t + 1 < nt) go = load_k(t + 1);
         go = go && load_v(t);
