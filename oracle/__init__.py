@@ -38,6 +38,7 @@ class OracleParams(ctypes.Structure):
         ("causal", ctypes.c_int64),
         ("window_left", ctypes.c_int64),
         ("window_right", ctypes.c_int64),
+        ("alibi_slopes", ctypes.c_void_p),
     ]
 
 
@@ -75,17 +76,18 @@ class Oracle:
         self.path = lib_path
 
     def attention_fwd(self, q, k, v, softmax_scale=None, causal=False, window_left=-1,
-                      window_right=-1):
-        """O (B, Nq, H, d) and LSE (B, H, Nq), float64."""
+                      window_right=-1, alibi_slopes=None):
+        """O (B, Nq, H, d) and LSE (B, H, Nq), float64.  ``alibi_slopes``
+        (H values, optional) adds -slope_h * |i + Nk - Nq - j| to the scores."""
         return self.attention_fwd_rows(q, k, v, None, softmax_scale, causal, window_left,
-                                       window_right)
+                                       window_right, alibi_slopes)
 
     def attention_fwd_rows(self, q, k, v, rows, softmax_scale=None, causal=False,
-                           window_left=-1, window_right=-1):
+                           window_left=-1, window_right=-1, alibi_slopes=None):
         """O and LSE for the query positions ``rows`` only (all rows if None):
         O (B, len(rows), H, d), LSE (B, H, len(rows))."""
         qa, ka, va = _f64(q), _f64(k), _f64(v)
-        p = _params(qa, ka, softmax_scale, causal, window_left, window_right)
+        p, _keep = _params(qa, ka, softmax_scale, causal, window_left, window_right, alibi_slopes)
         B, Nq, H, d = qa.shape
         if rows is None:
             n, rp = Nq, None
@@ -101,10 +103,10 @@ class Oracle:
         return o, lse
 
     def attention_bwd(self, q, k, v, dout, softmax_scale=None, causal=False, window_left=-1,
-                      window_right=-1):
+                      window_right=-1, alibi_slopes=None):
         """dQ (B, Nq, H, d), dK and dV (B, Nk, Hkv, d), float64."""
         qa, ka, va, da = _f64(q), _f64(k), _f64(v), _f64(dout)
-        p = _params(qa, ka, softmax_scale, causal, window_left, window_right)
+        p, _keep = _params(qa, ka, softmax_scale, causal, window_left, window_right, alibi_slopes)
         dq = np.zeros_like(qa)
         dk = np.zeros_like(ka)
         dv = np.zeros_like(va)
@@ -115,11 +117,11 @@ class Oracle:
         return dq, dk, dv
 
     def attention_bwd_rows(self, q, k, v, dout, qrows, krows, softmax_scale=None, causal=False,
-                           window_left=-1, window_right=-1):
+                           window_left=-1, window_right=-1, alibi_slopes=None):
         """dQ at query positions ``qrows`` (B, nq, H, d) and dK, dV at key
         positions ``krows`` (B, nk, Hkv, d), float64."""
         qa, ka, va, da = _f64(q), _f64(k), _f64(v), _f64(dout)
-        p = _params(qa, ka, softmax_scale, causal, window_left, window_right)
+        p, _keep = _params(qa, ka, softmax_scale, causal, window_left, window_right, alibi_slopes)
         qr = np.ascontiguousarray(np.asarray(qrows, dtype=np.int64))
         kr = np.ascontiguousarray(np.asarray(krows, dtype=np.int64))
         B, _, H, d = qa.shape
@@ -142,7 +144,7 @@ class Oracle:
     # 的突破与实战解析", section "实操落地"), so the oracle runs the dense
     # definition on every sequence's rows.
     def attention_fwd_varlen(self, q, k, v, cu_q, cu_k, softmax_scale=None, causal=False,
-                             window_left=-1, window_right=-1):
+                             window_left=-1, window_right=-1, alibi_slopes=None):
         """q (Tq, H, d), k, v (Tk, Hkv, d), offsets cu_q, cu_k (batch + 1):
         O (Tq, H, d) and LSE (H, Tq), float64."""
         qa, ka, va = _f64(q), _f64(k), _f64(v)
@@ -155,13 +157,14 @@ class Oracle:
             if q1 == q0:
                 continue
             ob, lb = self.attention_fwd(qa[None, q0:q1], ka[None, k0:k1], va[None, k0:k1],
-                                        softmax_scale, causal, window_left, window_right)
+                                        softmax_scale, causal, window_left, window_right,
+                                        alibi_slopes)
             o[q0:q1] = ob[0]
             lse[:, q0:q1] = lb[0]
         return o, lse
 
     def attention_bwd_varlen(self, q, k, v, dout, cu_q, cu_k, softmax_scale=None, causal=False,
-                             window_left=-1, window_right=-1):
+                             window_left=-1, window_right=-1, alibi_slopes=None):
         """dQ (Tq, H, d), dK and dV (Tk, Hkv, d), float64, per sequence."""
         qa, ka, va, da = _f64(q), _f64(k), _f64(v), _f64(dout)
         cq, ck = _offsets(cu_q), _offsets(cu_k)
@@ -172,7 +175,7 @@ class Oracle:
                 continue
             g = self.attention_bwd(qa[None, q0:q1], ka[None, k0:k1], va[None, k0:k1],
                                    da[None, q0:q1], softmax_scale, causal, window_left,
-                                   window_right)
+                                   window_right, alibi_slopes)
             dq[q0:q1], dk[k0:k1], dv[k0:k1] = g[0][0], g[1][0], g[2][0]
         return dq, dk, dv
 
@@ -215,14 +218,24 @@ def _ptr(a: np.ndarray, ty=ctypes.c_double):
     return a.ctypes.data_as(ctypes.POINTER(ty))
 
 
-def _params(q, k, softmax_scale, causal, window_left, window_right) -> OracleParams:
+def _params(q, k, softmax_scale, causal, window_left, window_right, alibi_slopes=None):
+    """The C parameter block and the slopes array it points to (keep both
+    alive for the call)."""
     B, Nq, H, d = q.shape
     Bk, Nk, Hkv, dk = k.shape
     if Bk != B or dk != d or H % Hkv != 0:
         raise ValueError("inconsistent shapes")
     scale = 1.0 / math.sqrt(d) if softmax_scale is None else float(softmax_scale)
+    slopes = None
+    if alibi_slopes is not None:
+        slopes = np.ascontiguousarray(
+            _f64(alibi_slopes if hasattr(alibi_slopes, "shape") else np.asarray(alibi_slopes))
+            .reshape(-1))
+        if slopes.shape[0] != H:
+            raise ValueError("alibi_slopes needs one slope per query head")
+    ptr = slopes.ctypes.data if slopes is not None else None
     return OracleParams(B, Nq, Nk, H, Hkv, d, scale, int(bool(causal)),
-                        int(window_left), int(window_right))
+                        int(window_left), int(window_right), ptr), slopes
 
 
 def attention_fwd(*a, **kw):

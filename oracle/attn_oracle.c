@@ -27,6 +27,12 @@
  *     inclusive, -1 meaning unbounded.
  *   - Grouped-query attention (page 5, hardware/dtype section, MQA/GQA):
  *     query head h reads kv head h / (nheads / nheads_kv).
+ *   - Positional bias from per-head slopes (the alibi_slopes argument named
+ *     on the FlashAttention-2 page, FAQ Q2, and on page 5's backend list;
+ *     neither gives the formula).  Reading taken: when slopes are given,
+ *         S_ij += -slope_h * |i + off - j|
+ *     on the scaled scores, with the masks' bottom-right alignment; no
+ *     slopes (NULL) means no bias.
  *   - LSE_i = m_i + ln(l_i), natural log, of the scaled scores.  A row with
  *     no visible key gets O = 0 and LSE = -inf.
  *   - Backward (page 2, item 2: the backward pass recomputes the score
@@ -51,6 +57,7 @@ typedef struct {
   int64_t batch, seqlen_q, seqlen_k, nheads, nheads_kv, headdim;
   double softmax_scale;
   int64_t causal, window_left, window_right;
+  const double *alibi_slopes; /* nheads slopes, or NULL */
 } oracle_params;
 
 /* Visibility of key j from query i (the mask reading stated above). */
@@ -92,6 +99,8 @@ static void row_scores(const oracle_params *p, const double *q, const double *k,
   for (int64_t j = 0; j < p->seqlen_k; ++j) {
     if (!visible(p, i, j)) { s[j] = -INFINITY; continue; }
     s[j] = p->softmax_scale * dot(qi, krow(p, k, b, j, g), p->headdim);
+    if (p->alibi_slopes)
+      s[j] -= p->alibi_slopes[h] * fabs((double)(i + p->seqlen_k - p->seqlen_q - j));
     if (s[j] > mx) mx = s[j];
     ++count;
   }

@@ -410,6 +410,56 @@ def pin_varlen_per_sequence(orc):
             _close(dv[k0:k1], vt.grad[0].permute(1, 0, 2).numpy(), 1e-10, f"varlen dV {b} {m}")
 
 
+def alibi_bias(nq, nk, slopes):
+    """-slope_h * |i + Nk - Nq - j| for every head, query and key (H, Nq, Nk),
+    written out by brute force."""
+    out = np.zeros((len(slopes), nq, nk))
+    for h, sl in enumerate(slopes):
+        for i in range(nq):
+            for j in range(nk):
+                out[h, i, j] = -sl * abs(i + nk - nq - j)
+    return out
+
+
+def pin_alibi_sdpa(orc):
+    """Per-head positional slopes: torch's scaled dot product attention with
+    the bias written into a float mask (-inf where hidden), and its autograd
+    gradients, for every mask, GQA and Nq != Nk; zero slopes give exactly
+    the unbiased result."""
+    import torch.nn.functional as F
+    B, H, Hkv, d, scale = 2, 4, 2, 8, 0.3
+    slopes = [0.5, 0.25, 0.125, 0.0625]
+    for nq, nk in ((10, 10), (6, 11), (9, 7)):
+        q, k, v = rand((B, nq, H, d), 80), rand((B, nk, Hkv, d), 81), rand((B, nk, Hkv, d), 82)
+        do = rand((B, nq, H, d), 83)
+        bias = alibi_bias(nq, nk, slopes)
+        for m in MASKS:
+            vis = mask_matrix(nq, nk, **m)
+            seen = vis.any(axis=1)
+            o, lse = orc.attention_fwd(q, k, v, scale, alibi_slopes=slopes, **m)
+            dq, dk, dv = orc.attention_bwd(q, k, v, do, scale, alibi_slopes=slopes, **m)
+            if not seen.any():
+                continue
+            qt = q.permute(0, 2, 1, 3)[:, :, seen].clone().requires_grad_(True)
+            kt = k.permute(0, 2, 1, 3).clone().requires_grad_(True)
+            vt = v.permute(0, 2, 1, 3).clone().requires_grad_(True)
+            rep = H // Hkv
+            fmask = torch.from_numpy(np.where(vis[seen][None], bias[:, seen], -np.inf))
+            out = F.scaled_dot_product_attention(
+                qt, kt.repeat_interleave(rep, dim=1), vt.repeat_interleave(rep, dim=1),
+                attn_mask=fmask[None], scale=scale)
+            (out * do.permute(0, 2, 1, 3)[:, :, seen]).sum().backward()
+            what = f"alibi {nq}x{nk} {m}"
+            _close(o[:, seen], out.detach().permute(0, 2, 1, 3).numpy(), 1e-10, what + " O")
+            assert np.all(o[:, ~seen] == 0.0)
+            _close(dq[:, seen], qt.grad.permute(0, 2, 1, 3).numpy(), 1e-10, what + " dQ")
+            _close(dk, kt.grad.permute(0, 2, 1, 3).numpy(), 1e-10, what + " dK")
+            _close(dv, vt.grad.permute(0, 2, 1, 3).numpy(), 1e-10, what + " dV")
+            o0, lse0 = orc.attention_fwd(q, k, v, scale, alibi_slopes=[0.0] * H, **m)
+            o1, lse1 = orc.attention_fwd(q, k, v, scale, **m)
+            assert np.array_equal(o0, o1) and np.array_equal(lse0, lse1)
+
+
 ALL_PINS = [
     pin_golden_handworked,
     pin_identical_keys,
@@ -424,4 +474,5 @@ ALL_PINS = [
     pin_empty_rows,
     pin_rows_match_full,
     pin_varlen_per_sequence,
+    pin_alibi_sdpa,
 ]

@@ -21,6 +21,11 @@ MUTATIONS = {
     "gqa_mapping_modulo": ("return h / (p->nheads / p->nheads_kv);", "return h % p->nheads_kv;"),
     "lse_without_max": ("*lse_out = m + log(l);", "*lse_out = log(l);"),
     "softmax_not_normalised": ("exp(s - m) / l;", "exp(s - m);"),
+    "alibi_abs_dropped": ("fabs((double)(i + p->seqlen_k - p->seqlen_q - j))",
+                          "((double)(i + p->seqlen_k - p->seqlen_q - j))"),
+    "alibi_alignment_top_left": ("fabs((double)(i + p->seqlen_k - p->seqlen_q - j))",
+                                 "fabs((double)(i - j))"),
+    "alibi_wrong_head": ("p->alibi_slopes[h]", "p->alibi_slopes[0]"),
     "ds_sign_flipped": ("(dp[j] - rowsum)", "(rowsum - dp[j])"),
     "ds_rowsum_dropped": ("(dp[j] - rowsum)", "(dp[j])"),
     "dk_scale_dropped": ("dkj[c] += p->softmax_scale * ds * qi[c];", "dkj[c] += ds * qi[c];"),
