@@ -101,6 +101,12 @@ typedef struct {
   int32_t causal;         /* 0 or 1 */
   int32_t window_left;    /* -1 = unbounded */
   int32_t window_right;   /* -1 = unbounded */
+  /* Per-head positional slopes: NULL, or a DEVICE array of nheads floats
+   * (4-byte aligned); score (i, j) of head h then gains
+   * -alibi_slopes[h] * |i + seqlen_k - seqlen_q - j| (the alibi_slopes
+   * argument of the FlashAttention-2 interface; see the mask rules below for
+   * the alignment).  Read by the kernels only. */
+  const float* alibi_slopes;
 } attn_params;
 
 /*
@@ -209,6 +215,7 @@ typedef struct {
   int32_t causal;
   int32_t window_left;
   int32_t window_right;
+  const float* alibi_slopes;  /* as in attn_params; lengths per sequence */
 } attn_varlen_params;
 
 /* Host-side checks of a packed call (pass 0 forward, 1 backward): the

@@ -47,6 +47,7 @@ class AttnParams(ctypes.Structure):
         ("causal", ctypes.c_int32),
         ("window_left", ctypes.c_int32),
         ("window_right", ctypes.c_int32),
+        ("alibi_slopes", ctypes.c_void_p),
     ]
 
 
@@ -66,6 +67,7 @@ class AttnVarlenParams(ctypes.Structure):
         ("causal", ctypes.c_int32),
         ("window_left", ctypes.c_int32),
         ("window_right", ctypes.c_int32),
+        ("alibi_slopes", ctypes.c_void_p),
     ]
 
 
@@ -135,11 +137,27 @@ _lib = _Lazy()
 
 
 def make_params(batch, seqlen_q, seqlen_k, nheads, nheads_kv, headdim, dtype=ATTN_BF16,
-                softmax_scale=None, causal=False, window_left=-1, window_right=-1) -> AttnParams:
+                softmax_scale=None, causal=False, window_left=-1, window_right=-1,
+                alibi_slopes=None) -> AttnParams:
+    """``alibi_slopes``: None, or the device address (int) of nheads float32
+    slopes."""
     scale = 1.0 / math.sqrt(headdim) if softmax_scale is None else float(softmax_scale)
     return AttnParams(int(batch), int(seqlen_q), int(seqlen_k), int(nheads), int(nheads_kv),
                       int(headdim), int(dtype), scale, int(bool(causal)), int(window_left),
-                      int(window_right))
+                      int(window_right), alibi_slopes)
+
+
+def _slopes_ptr(alibi_slopes, nheads, device):
+    """Device address of a (nheads,) float32 CUDA tensor of slopes, or None."""
+    if alibi_slopes is None:
+        return None
+    import torch
+    if (not isinstance(alibi_slopes, torch.Tensor) or not alibi_slopes.is_cuda or
+            alibi_slopes.dtype != torch.float32 or not alibi_slopes.is_contiguous() or
+            alibi_slopes.numel() != nheads or alibi_slopes.device != device):
+        raise ValueError("alibi_slopes must be a contiguous float32 tensor of nheads values "
+                         "on the inputs' device")
+    return alibi_slopes.data_ptr()
 
 
 def attn_status_string(status: int) -> str:
@@ -217,24 +235,27 @@ def _stream(stream):
     return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream if stream is None else int(stream))
 
 
-def params_for(q, k, softmax_scale=None, causal=False, window_left=-1, window_right=-1):
+def params_for(q, k, softmax_scale=None, causal=False, window_left=-1, window_right=-1,
+               alibi_slopes=None):
     B, Nq, H, d = q.shape
     Bk, Nk, Hkv, dk = k.shape
     if Bk != B or dk != d:
         raise ValueError("q and k disagree on batch or head dim")
     return make_params(B, Nq, Nk, H, Hkv, d, _dtype_code(q), softmax_scale, causal, window_left,
-                       window_right)
+                       window_right, _slopes_ptr(alibi_slopes, H, q.device))
 
 
 def attn_fwd(q, k, v, softmax_scale: Optional[float] = None, causal: bool = False,
              window_left: int = -1, window_right: int = -1, out=None, lse=None,
-             stream=None) -> Tuple["torch.Tensor", "torch.Tensor"]:
-    """O = softmax(q k^T * scale + mask) v and the per-row natural-log LSE.
+             stream=None, alibi_slopes=None) -> Tuple["torch.Tensor", "torch.Tensor"]:
+    """O = softmax(q k^T * scale + bias + mask) v and the per-row natural-log LSE.
 
     q (B, Nq, H, d), k and v (B, Nk, Hkv, d), bf16 or fp16, contiguous CUDA
-    tensors.  Returns (out (B, Nq, H, d), lse (B, H, Nq) float32)."""
+    tensors; ``alibi_slopes`` (optional, (H,) float32) adds
+    -slope_h * |i + Nk - Nq - j|.  Returns (out (B, Nq, H, d), lse (B, H, Nq)
+    float32)."""
     import torch
-    p = params_for(q, k, softmax_scale, causal, window_left, window_right)
+    p = params_for(q, k, softmax_scale, causal, window_left, window_right, alibi_slopes)
     B, Nq, H, d = q.shape
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _check(t, n)
@@ -258,11 +279,11 @@ def attn_fwd(q, k, v, softmax_scale: Optional[float] = None, causal: bool = Fals
 
 def attn_bwd(q, k, v, out, lse, dout, softmax_scale: Optional[float] = None, causal: bool = False,
              window_left: int = -1, window_right: int = -1, dq=None, dk=None, dv=None,
-             workspace=None, stream=None):
+             workspace=None, stream=None, alibi_slopes=None):
     """Gradients (dq, dk, dv) of sum(out * dout) for attention with the same
     arguments as ``attn_fwd``; ``out`` and ``lse`` are its results."""
     import torch
-    p = params_for(q, k, softmax_scale, causal, window_left, window_right)
+    p = params_for(q, k, softmax_scale, causal, window_left, window_right, alibi_slopes)
     B, Nq, H, d = q.shape
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
         _check(t, n)
@@ -314,7 +335,7 @@ def attn_bwd_finalize(p: AttnParams, dq, workspace, stream=None) -> None:
 
 def attn_bwd_noalloc(q, k, v, out, lse, dout, softmax_scale: Optional[float] = None,
                      causal: bool = False, window_left: int = -1, window_right: int = -1,
-                     dq=None, dk=None, dv=None, stream=None):
+                     dq=None, dk=None, dv=None, stream=None, alibi_slopes=None):
     """Like ``attn_bwd`` but the library uses its own fixed device scratch
     (ATTN_NOALLOC_SCRATCH_BYTES) instead of a caller workspace, for callers
     that cannot allocate device memory at call time.  The output tensors are
@@ -325,7 +346,7 @@ def attn_bwd_noalloc(q, k, v, out, lse, dout, softmax_scale: Optional[float] = N
     vp = ctypes.c_void_p
     fn.argtypes = [ctypes.POINTER(AttnParams), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     fn.restype = ctypes.c_int
-    p = params_for(q, k, softmax_scale, causal, window_left, window_right)
+    p = params_for(q, k, softmax_scale, causal, window_left, window_right, alibi_slopes)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
@@ -339,12 +360,12 @@ def attn_bwd_noalloc(q, k, v, out, lse, dout, softmax_scale: Optional[float] = N
 # ----------------------------------------------------------------- packed sequences
 def make_varlen_params(batch, total_q, total_k, max_seqlen_q, max_seqlen_k, nheads, nheads_kv,
                        headdim, dtype=ATTN_BF16, softmax_scale=None, causal=False,
-                       window_left=-1, window_right=-1) -> AttnVarlenParams:
+                       window_left=-1, window_right=-1, alibi_slopes=None) -> AttnVarlenParams:
     scale = 1.0 / math.sqrt(headdim) if softmax_scale is None else float(softmax_scale)
     return AttnVarlenParams(int(batch), int(total_q), int(total_k), int(max_seqlen_q),
                             int(max_seqlen_k), int(nheads), int(nheads_kv), int(headdim),
                             int(dtype), scale, int(bool(causal)), int(window_left),
-                            int(window_right))
+                            int(window_right), alibi_slopes)
 
 
 def attn_check_varlen_params(p: AttnVarlenParams, pass_: int = 0) -> int:
@@ -356,7 +377,7 @@ def attn_bwd_varlen_workspace_size(p: AttnVarlenParams) -> int:
 
 
 def _varlen_params(q, k, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, softmax_scale,
-                   causal, window_left, window_right):
+                   causal, window_left, window_right, alibi_slopes=None):
     import torch
     if q.dim() != 3 or k.dim() != 3:
         raise ValueError("packed q must be (total_q, nheads, d) and k (total_k, nheads_kv, d)")
@@ -371,13 +392,14 @@ def _varlen_params(q, k, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
     if cu_seqlens_q.numel() != cu_seqlens_k.numel() or cu_seqlens_q.numel() < 1:
         raise ValueError("cu_seqlens_q and cu_seqlens_k must both have batch + 1 entries")
     return make_varlen_params(cu_seqlens_q.numel() - 1, Tq, Tk, max_seqlen_q, max_seqlen_k, H, Hkv,
-                              d, _dtype_code(q), softmax_scale, causal, window_left, window_right)
+                              d, _dtype_code(q), softmax_scale, causal, window_left, window_right,
+                              _slopes_ptr(alibi_slopes, H, q.device))
 
 
 def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int,
                     softmax_scale: Optional[float] = None, causal: bool = False,
                     window_left: int = -1, window_right: int = -1, out=None, lse=None,
-                    stream=None):
+                    stream=None, alibi_slopes=None):
     """Attention over packed variable-length sequences.
 
     q (total_q, H, d), k and v (total_k, Hkv, d); sequence b owns rows
@@ -386,7 +408,7 @@ def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_
     (total_q, H, d), lse (H, total_q) float32)."""
     import torch
     p = _varlen_params(q, k, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
-                       softmax_scale, causal, window_left, window_right)
+                       softmax_scale, causal, window_left, window_right, alibi_slopes)
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _check(t, n)
         if t.dtype != q.dtype:
@@ -409,12 +431,12 @@ def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_
 def attn_bwd_varlen(q, k, v, out, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int,
                     max_seqlen_k: int, softmax_scale: Optional[float] = None,
                     causal: bool = False, window_left: int = -1, window_right: int = -1,
-                    dq=None, dk=None, dv=None, workspace=None, stream=None):
+                    dq=None, dk=None, dv=None, workspace=None, stream=None, alibi_slopes=None):
     """Gradients (dq, dk, dv) of sum(out * dout) for ``attn_fwd_varlen`` with
     the same arguments; ``out`` and ``lse`` are its results."""
     import torch
     p = _varlen_params(q, k, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
-                       softmax_scale, causal, window_left, window_right)
+                       softmax_scale, causal, window_left, window_right, alibi_slopes)
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
         _check(t, n)
         if t.dtype != q.dtype:

@@ -170,12 +170,14 @@ struct Packed {
 // where both O tiles fit tensor memory (d <= 128), one otherwise.
 template <class C>
 struct FwdLaunch {
-  static constexpr auto kernel() { return attn_fwd_kernel<C>; }
+  template <bool ALIBI>
+  static constexpr auto kernel() { return attn_fwd_kernel<C, ALIBI>; }
   static constexpr int rows_per_cta = C::BM;
 };
 template <int D, int KS, int VS, bool F>
 struct FwdLaunch<FwdPPCfg<D, KS, VS, F>> {
-  static constexpr auto kernel() { return attn_fwd_pp_kernel<FwdPPCfg<D, KS, VS, F>>; }
+  template <bool ALIBI>
+  static constexpr auto kernel() { return attn_fwd_pp_kernel<FwdPPCfg<D, KS, VS, F>, ALIBI>; }
   static constexpr int rows_per_cta = 2 * FwdPPCfg<D, KS, VS, F>::BM;
 };
 
@@ -199,6 +201,7 @@ attn_status launch_fwd(const attn_params* p, const void* q, const void* k, const
   fp.total_q = pk.total_q;
   fp.total_k = pk.total_k;
   fp.o = static_cast<uint16_t*>(o);
+  fp.alibi = p->alibi_slopes;
   fp.lse = lse;
   fp.batch = p->batch;
   fp.nheads = p->nheads;
@@ -215,7 +218,8 @@ attn_status launch_fwd(const attn_params* p, const void* q, const void* k, const
   fp.sched_group = l2_group(4.0 * p->seqlen_k * C::D / (p->nheads / p->nheads_kv), heads);
   const long long blocks = (long long)fp.num_qblocks * heads;
   if (blocks > INT_MAX) return ATTN_ERR_INVALID_ARG;
-  auto kern = FwdLaunch<C>::kernel();
+  auto kern = p->alibi_slopes ? FwdLaunch<C>::template kernel<true>()
+                              : FwdLaunch<C>::template kernel<false>();
   if (!ensure_smem(reinterpret_cast<const void*>(kern), C::SMEM_BYTES)) return ATTN_ERR_CUDA;
   kern<<<(unsigned)blocks, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mo, fp);
   return finish(stream);
@@ -235,6 +239,7 @@ BwdParams bwd_params(const attn_params* p, const float* lse, void* workspace, co
   bp.total_q = pk.total_q;
   bp.total_k = pk.total_k;
   bp.dk = bp.dv = nullptr;
+  bp.alibi = p->alibi_slopes;
   bp.num_kblocks = bp.sched_group = 0;
   bp.lse = lse;
   bp.dvec = reinterpret_cast<float*>(w + ws.dvec_off);
@@ -305,7 +310,7 @@ attn_status launch_bwd_main(const attn_params* p, const void* q, const void* k, 
   bpl.sched_group = l2_group(8.0 * p->seqlen_q * C::D * (p->nheads / p->nheads_kv), heads);
   const long long blocks = (long long)bpl.num_kblocks * heads;
   if (blocks > INT_MAX) return ATTN_ERR_INVALID_ARG;
-  auto kern = attn_bwd_kernel<C>;
+  auto kern = p->alibi_slopes ? attn_bwd_kernel<C, true> : attn_bwd_kernel<C, false>;
   if (!ensure_smem(reinterpret_cast<const void*>(kern), C::SMEM_BYTES)) return ATTN_ERR_CUDA;
   kern<<<(unsigned)blocks, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, ml, md, mdk,
                                                                  mdv, mdq, bpl);
@@ -418,6 +423,7 @@ attn_params packed_view(const attn_varlen_params* v) {
   p.causal = v->causal;
   p.window_left = v->window_left;
   p.window_right = v->window_right;
+  p.alibi_slopes = v->alibi_slopes;
   return p;
 }
 
@@ -475,6 +481,7 @@ attn_status attn_check_params(const attn_params* p, int pass) {
   if (!(p->softmax_scale > 0.f) || !std::isfinite(p->softmax_scale)) return ATTN_ERR_INVALID_ARG;
   if (p->causal != 0 && p->causal != 1) return ATTN_ERR_INVALID_ARG;
   if (p->window_left < -1 || p->window_right < -1) return ATTN_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(p->alibi_slopes) & 3u) return ATTN_ERR_MISALIGNED;
   return ATTN_OK;
 }
 

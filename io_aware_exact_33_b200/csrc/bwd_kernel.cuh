@@ -112,6 +112,9 @@ struct BwdParams {
   int total_q, total_k;
   uint16_t* dk;
   uint16_t* dv;
+  // Per-head positional slopes (nheads floats), or nullptr: scores gain
+  // -slope_h * |i + seqlen_k - seqlen_q - j| (kernel instantiated with ALIBI).
+  const float* alibi;
 };
 
 // Packed layout: the sequence owning padded row `pr` (the last b with
@@ -311,7 +314,7 @@ struct BwdCfg {
   static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
 
-template <class C>
+template <class C, bool ALIBI>
 __global__ void __launch_bounds__(C::THREADS, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -602,6 +605,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         ((long long)k0 >= (long long)(qa + C::HW - 1) + off - lb);
       const uint32_t lse_addr = smem0 + C::OFF_LSE + (slot * BM + c0) * 4;
       const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
+      // positional bias of query column c (ALIBI): bk * |c - bd|, log2 units
+      const int hq = kvh * group + t / nqb;  // this tile's query head
+      const float bk = ALIBI ? -p.alibi[hq] * 1.4426950408889634f : 0.f;
+      const float bd = ALIBI ? (float)(j - off - qa) : 0.f;
 #pragma unroll
       for (int c = 0; c < C::HW; c += 4) {
         float l4[4];
@@ -611,6 +618,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           float a0, a1;
           f2_unpack(f2_fma(f2_pack(pr[c + e], pr[c + e + 1]), scale2, f2_pack(-l4[e], -l4[e + 1])),
                     a0, a1);
+          if constexpr (ALIBI) {
+            a0 = fmaf(fabsf((float)(c + e) - bd), bk, a0);
+            a1 = fmaf(fabsf((float)(c + e + 1) - bd), bk, a1);
+          }
           pr[c + e] = ex2(a0);
           pr[c + e + 1] = ex2(a1);
         }

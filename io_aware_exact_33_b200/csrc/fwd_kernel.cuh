@@ -44,6 +44,9 @@ struct FwdParams {
   const int* cu_k;
   int total_q, total_k;
   uint16_t* o;
+  // Per-head positional slopes (nheads floats), or nullptr: scores gain
+  // -slope_h * |i + seqlen_k - seqlen_q - j| (kernels instantiated with ALIBI).
+  const float* alibi;
 };
 
 // Row `row` of query head h of sequence (b, sq) in the LSE output.
@@ -104,7 +107,7 @@ struct FwdCfg {
   static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
 
-template <class C>
+template <class C, bool ALIBI>
 __global__ void __launch_bounds__(C::THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -246,6 +249,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const long long jlo = (long long)i + off - lb;
     const long long blk_hi = (long long)q0 + off + rb;            // every row sees up to here
     const long long blk_lo = (long long)(q0 + BM - 1) + off - lb;  // every row sees from here
+    // positional slope in log2 units (negated): bias_c = bk * |bd - c|
+    const float bk = ALIBI ? -p.alibi[h] * 1.4426950408889634f : 0.f;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int t = 0; t < nt; ++t) {
@@ -271,10 +276,18 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           if (j >= p.seqlen_k || j > jhi || j < jlo) s[c] = -INFINITY;
         }
       }
+      // sl: the factor still to apply to s (the bias case scales up front)
+      float sl = p.scale_log2;
+      if constexpr (ALIBI) {
+        const float bd = (float)((long long)i + off - k0);
+#pragma unroll
+        for (int c = 0; c < BN; ++c) s[c] = fmaf(s[c], p.scale_log2, bk * fabsf(bd - (float)c));
+        sl = 1.f;
+      }
       float mx = s[0];
 #pragma unroll
       for (int c = 1; c < BN; ++c) mx = fmaxf(mx, s[c]);
-      const float m_tile = mx * p.scale_log2;  // scale > 0
+      const float m_tile = mx * sl;  // scale > 0
       // Keep the old reference max unless the row max grew by more than 8
       // (log2 units); the first tile always sets it.
       float m_use = m, alpha = 1.f;
@@ -287,8 +300,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       uint32_t packed[BN / 2];
 #pragma unroll
       for (int c = 0; c < BN; c += 2) {
-        const float p0 = ex2(fmaf(s[c], p.scale_log2, -m_sub));
-        const float p1 = ex2(fmaf(s[c + 1], p.scale_log2, -m_sub));
+        const float p0 = ex2(fmaf(s[c], sl, -m_sub));
+        const float p1 = ex2(fmaf(s[c + 1], sl, -m_sub));
         rowsum += p0 + p1;
         packed[c / 2] = pack2<C::FP16>(p0, p1);
       }
@@ -449,14 +462,25 @@ struct FwdPPCfg {
 // masked column; the two units then work in parallel.
 constexpr uint32_t kPolyPairs = 0x2222u;
 
-template <bool MASK, class C>
+// With ALIBI, column c of the tile gains bk * |bd - c| (log2 units): bd is
+// the row's position (plus the alignment offset) minus the tile's first key,
+// bk the negated slope times log2(e); the row max is then taken on the
+// biased, scaled scores.
+template <bool MASK, bool ALIBI, class C>
 __device__ __forceinline__ void softmax_tile(uint32_t s_tmem, uint32_t o_tmem, int n, int vlo,
                                              int vhi, float scale_log2, float m, float& mx,
                                              float& rowsum, float& alpha, float& m_use,
-                                             uint32_t pready_half0, uint32_t pready_half1) {
+                                             uint32_t pready_half0, uint32_t pready_half1,
+                                             float bd, float bk) {
   constexpr int BN = C::BN, D = C::D;
   auto val = [&](uint32_t bits, int col) -> float {
     return (MASK && (col < vlo || col >= vhi)) ? -INFINITY : __uint_as_float(bits);
+  };
+  // the value the row max is taken over: raw scores, or scaled + biased
+  auto score = [&](uint32_t bits, int col) -> float {
+    const float v = val(bits, col);
+    if constexpr (ALIBI) return fmaf(v, scale_log2, bk * fabsf(bd - (float)col));
+    return v;
   };
   mx = -INFINITY;
   {
@@ -468,11 +492,11 @@ __device__ __forceinline__ void softmax_tile(uint32_t s_tmem, uint32_t o_tmem, i
       if (c + 1 < BN / 32) tmem_ld32(s_tmem + (c + 1) * 32, buf[(c + 1) & 1]);
 #pragma unroll
       for (int e = 0; e < 32; e += 2)
-        mx = max3f(mx, val(buf[c & 1][e], c * 32 + e), val(buf[c & 1][e + 1], c * 32 + e + 1));
+        mx = max3f(mx, score(buf[c & 1][e], c * 32 + e), score(buf[c & 1][e + 1], c * 32 + e + 1));
       if (c + 1 < BN / 32) tmem_ld_wait();
     }
   }
-  const float m_tile = mx * scale_log2;  // scale > 0
+  const float m_tile = ALIBI ? mx : mx * scale_log2;  // scale > 0
   m_use = m;
   alpha = 1.f;
   if (m_tile > m + 8.f) {
@@ -517,6 +541,10 @@ __device__ __forceinline__ void softmax_tile(uint32_t s_tmem, uint32_t o_tmem, i
         const uint64_t x2 = f2_pack(val(buf[c & 1][e], c * 32 + e), val(buf[c & 1][e + 1], c * 32 + e + 1));
         float a0, a1, p0, p1;
         f2_unpack(f2_fma(x2, scale2, neg_m2), a0, a1);
+        if constexpr (ALIBI) {
+          a0 = fmaf(fabsf(bd - (float)(c * 32 + e)), bk, a0);
+          a1 = fmaf(fabsf(bd - (float)(c * 32 + e + 1)), bk, a1);
+        }
         if (!MASK && ((kPolyPairs >> (e / 2)) & 1)) {
           exp2_poly2(a0, a1, p0, p1);
         } else {
@@ -543,7 +571,7 @@ __device__ __forceinline__ void softmax_tile(uint32_t s_tmem, uint32_t o_tmem, i
   }
 }
 
-template <class C>
+template <class C, bool ALIBI>
 __global__ void __launch_bounds__(C::THREADS, 1)
     attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -732,6 +760,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const long long blk_hi = (long long)q_i + off + rb;
     const long long blk_lo = (long long)(q_i + BM - 1) + off - lb;
     const int n_i = hi_i - lo_i;
+    // positional slope in log2 units (negated): bias of column c = bk * |bd - c|
+    const float bk = ALIBI ? -p.alibi[h] * 1.4426950408889634f : 0.f;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int n = 0; n < n_i; ++n) {
@@ -748,12 +778,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       }
       float mx, rowsum, alpha, m_use;
       const uint32_t ph0 = bar(C::B_PREADY + 2 * i), ph1 = bar(C::B_PREADY + 2 * i + 1);
+      const float bd = ALIBI ? (float)((long long)row + off - k0) : 0.f;
       if (full)
-        softmax_tile<false, C>(s_tmem, o_tmem, n, vlo, vhi, p.scale_log2, m, mx, rowsum, alpha,
-                               m_use, ph0, ph1);
+        softmax_tile<false, ALIBI, C>(s_tmem, o_tmem, n, vlo, vhi, p.scale_log2, m, mx, rowsum,
+                                      alpha, m_use, ph0, ph1, bd, bk);
       else
-        softmax_tile<true, C>(s_tmem, o_tmem, n, vlo, vhi, p.scale_log2, m, mx, rowsum, alpha,
-                              m_use, ph0, ph1);
+        softmax_tile<true, ALIBI, C>(s_tmem, o_tmem, n, vlo, vhi, p.scale_log2, m, mx, rowsum,
+                                     alpha, m_use, ph0, ph1, bd, bk);
       l = l * alpha + rowsum;
       m = m_use;
     }

@@ -101,3 +101,11 @@ def test_workspace_sizes(attn):
     assert ws >= 2 * rows + acc
     assert ws % 256 == 0
     assert attn.attn_bwd_workspace_size(P(attn, headdim=96)) == 0
+
+
+def test_alibi_pointer_alignment(attn):
+    p = P(attn)
+    p.alibi_slopes = 2  # not 4-byte aligned; never dereferenced on the host
+    assert attn.attn_check_params(p, 0) == 4  # ATTN_ERR_MISALIGNED
+    p.alibi_slopes = 256
+    assert attn.attn_check_params(p, 0) == 0
