@@ -25,6 +25,8 @@
 // (same buffer) is written only after O += P_j V_j has read P_j.
 #pragma once
 
+#include <type_traits>
+
 #include "sm100.cuh"
 
 namespace attn {
@@ -464,24 +466,28 @@ constexpr uint32_t kPolyPairs = 0x2222u;
 
 // With ALIBI, column c of the tile gains bk * |bd - c| (log2 units): bd is
 // the row's position (plus the alignment offset) minus the tile's first key,
-// bk the negated slope times log2(e); the row max is then taken on the
-// biased, scaled scores.
+// bk the negated slope times log2(e), and `left` says every visible column
+// lies left of (or on) the row's diagonal (causal masks).
+//  * Row max: when the bias varies by at most 64 across the tile, an upper
+//    bound — the raw maximum, scaled, plus the tile's largest bias
+//    (bk * distance of bd from [0, BN)); a reference max above the true one
+//    only scales P (and l) by a common power of two, so O and LSE are
+//    unchanged.  Otherwise the exact maximum of the biased scores.
+//  * Exponentials: when, for every row of the warp, all visible columns lie
+//    on one side of its diagonal, the bias is linear in the column, b0 +
+//    dl * c, and rides in the FMA's addend (one extra packed FMA per column
+//    pair); tiles the diagonal crosses add it column by column.
 template <bool MASK, bool ALIBI, class C>
 __device__ __forceinline__ void softmax_tile(uint32_t s_tmem, uint32_t o_tmem, int n, int vlo,
                                              int vhi, float scale_log2, float m, float& mx,
                                              float& rowsum, float& alpha, float& m_use,
                                              uint32_t pready_half0, uint32_t pready_half1,
-                                             float bd, float bk) {
+                                             float bd, float bk, bool left) {
   constexpr int BN = C::BN, D = C::D;
   auto val = [&](uint32_t bits, int col) -> float {
     return (MASK && (col < vlo || col >= vhi)) ? -INFINITY : __uint_as_float(bits);
   };
-  // the value the row max is taken over: raw scores, or scaled + biased
-  auto score = [&](uint32_t bits, int col) -> float {
-    const float v = val(bits, col);
-    if constexpr (ALIBI) return fmaf(v, scale_log2, bk * fabsf(bd - (float)col));
-    return v;
-  };
+  const bool bounded = !ALIBI || (-bk * (float)(BN - 1) <= 64.f);  // uniform: one slope per CTA
   mx = -INFINITY;
   {
     uint32_t buf[2][32];
@@ -490,13 +496,22 @@ __device__ __forceinline__ void softmax_tile(uint32_t s_tmem, uint32_t o_tmem, i
 #pragma unroll
     for (int c = 0; c < BN / 32; ++c) {
       if (c + 1 < BN / 32) tmem_ld32(s_tmem + (c + 1) * 32, buf[(c + 1) & 1]);
+      if (bounded) {
 #pragma unroll
-      for (int e = 0; e < 32; e += 2)
-        mx = max3f(mx, score(buf[c & 1][e], c * 32 + e), score(buf[c & 1][e + 1], c * 32 + e + 1));
+        for (int e = 0; e < 32; e += 2)
+          mx = max3f(mx, val(buf[c & 1][e], c * 32 + e), val(buf[c & 1][e + 1], c * 32 + e + 1));
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int col = c * 32 + e;
+          mx = fmaxf(mx, fmaf(val(buf[c & 1][e], col), scale_log2, bk * fabsf(bd - (float)col)));
+        }
+      }
       if (c + 1 < BN / 32) tmem_ld_wait();
     }
   }
-  const float m_tile = ALIBI ? mx : mx * scale_log2;  // scale > 0
+  float m_tile = bounded ? mx * scale_log2 : mx;  // scale > 0
+  if (ALIBI && bounded) m_tile += bk * fmaxf(fmaxf(-bd, bd - (float)(BN - 1)), 0.f);
   m_use = m;
   alpha = 1.f;
   if (m_tile > m + 8.f) {
@@ -528,7 +543,23 @@ __device__ __forceinline__ void softmax_tile(uint32_t s_tmem, uint32_t o_tmem, i
   const uint64_t scale2 = f2_pack(scale_log2, scale_log2);
   const uint64_t neg_m2 = f2_pack(-m_sub, -m_sub);
   uint64_t sum2 = f2_pack(0.f, 0.f);
-  {
+  // linear bias for the whole warp? (b0 = bias at column 0, dl per column)
+  bool lin = false;
+  uint64_t base2 = neg_m2, step2 = f2_pack(0.f, 0.f);
+  if constexpr (ALIBI) {
+    const bool right = bd <= 0.f;
+    const bool row_left = left || bd >= (float)(BN - 1);
+    lin = __all_sync(0xffffffffu, row_left || right);
+    const float b0 = row_left ? bk * bd : -bk * bd;
+    const float dl = row_left ? -bk : bk;
+    base2 = f2_pack(b0 - m_sub, b0 - m_sub);
+    step2 = f2_pack(dl, dl);
+  }
+  auto exp_pass = [&](auto lin_tag) {
+    constexpr bool LIN = decltype(lin_tag)::value;
+    // linear bias: addend of columns (col, col + 1), advanced by 2 dl a pair
+    uint64_t add2 = f2_fma(f2_pack(0.f, 1.f), step2, base2);
+    const uint64_t step2x2 = f2_add(step2, step2);
     uint32_t buf[2][32];
     tmem_ld32(s_tmem, buf[0]);
     tmem_ld_wait();
@@ -538,12 +569,18 @@ __device__ __forceinline__ void softmax_tile(uint32_t s_tmem, uint32_t o_tmem, i
       uint32_t w[16];
 #pragma unroll
       for (int e = 0; e < 32; e += 2) {
-        const uint64_t x2 = f2_pack(val(buf[c & 1][e], c * 32 + e), val(buf[c & 1][e + 1], c * 32 + e + 1));
+        const int col = c * 32 + e;
+        const uint64_t x2 = f2_pack(val(buf[c & 1][e], col), val(buf[c & 1][e + 1], col + 1));
         float a0, a1, p0, p1;
-        f2_unpack(f2_fma(x2, scale2, neg_m2), a0, a1);
-        if constexpr (ALIBI) {
-          a0 = fmaf(fabsf(bd - (float)(c * 32 + e)), bk, a0);
-          a1 = fmaf(fabsf(bd - (float)(c * 32 + e + 1)), bk, a1);
+        if constexpr (LIN) {
+          f2_unpack(f2_fma(x2, scale2, add2), a0, a1);
+          add2 = f2_add(add2, step2x2);
+        } else {
+          f2_unpack(f2_fma(x2, scale2, neg_m2), a0, a1);
+          if constexpr (ALIBI) {
+            a0 = fmaf(fabsf(bd - (float)col), bk, a0);
+            a1 = fmaf(fabsf(bd - (float)(col + 1)), bk, a1);
+          }
         }
         if (!MASK && ((kPolyPairs >> (e / 2)) & 1)) {
           exp2_poly2(a0, a1, p0, p1);
@@ -563,7 +600,11 @@ __device__ __forceinline__ void softmax_tile(uint32_t s_tmem, uint32_t o_tmem, i
         mbar_arrive(c == BN / 32 - 1 ? pready_half1 : pready_half0);
       }
     }
-  }
+  };
+  if (ALIBI && lin)
+    exp_pass(std::true_type{});
+  else
+    exp_pass(std::false_type{});
   {
     float s0, s1;
     f2_unpack(sum2, s0, s1);
@@ -781,10 +822,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       const float bd = ALIBI ? (float)((long long)row + off - k0) : 0.f;
       if (full)
         softmax_tile<false, ALIBI, C>(s_tmem, o_tmem, n, vlo, vhi, p.scale_log2, m, mx, rowsum,
-                                      alpha, m_use, ph0, ph1, bd, bk);
+                                      alpha, m_use, ph0, ph1, bd, bk, p.causal != 0);
       else
         softmax_tile<true, ALIBI, C>(s_tmem, o_tmem, n, vlo, vhi, p.scale_log2, m, mx, rowsum,
-                                     alpha, m_use, ph0, ph1, bd, bk);
+                                     alpha, m_use, ph0, ph1, bd, bk, p.causal != 0);
       l = l * alpha + rowsum;
       m = m_use;
     }

@@ -97,3 +97,25 @@ def test_alibi_packed_sequences(attn):
     refs = oracle.attention_bwd_varlen(q, k, v, do, cu_q, cu_k, *args, alibi_slopes=sl.double())
     for g, r, n in zip(grads, refs, ("dQ", "dK", "dV")):
         check_grad(g.cpu(), r, f"packed alibi {n}")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_alibi_steep_slopes(attn, causal):
+    """Slopes above ~0.35 make the bias vary by more than 64 (log2 units)
+    across a key tile; the forward then takes the exact biased row max
+    instead of its upper bound.  Mixed heads exercise both."""
+    w = W("steep", 1, 4, 4, 300, 300, 128, causal=causal, seed=513)
+    q, k, v, do = make_inputs(w)
+    sl = torch.tensor([2.0, 0.5, 0.02, 1.0], dtype=torch.float32)
+    args = (w.scale, w.causal, -1, -1)
+    qc, kc, vc, doc = q.cuda(), k.cuda(), v.cuda(), do.cuda()
+    o, lse = attn.attn_fwd(qc, kc, vc, *args, alibi_slopes=sl.cuda())
+    grads = attn.attn_bwd(qc, kc, vc, o, lse, doc, *args, alibi_slopes=sl.cuda())
+    torch.cuda.synchronize()
+    assert attn.attn_get_device_status() == 0
+    o_ref, lse_ref = oracle.attention_fwd(q, k, v, *args, alibi_slopes=sl.double())
+    check_o(o.cpu(), o_ref, "steep")
+    check_lse(lse.cpu(), lse_ref, "steep")
+    refs = oracle.attention_bwd(q, k, v, do, *args, alibi_slopes=sl.double())
+    for g, r, n in zip(grads, refs, ("dQ", "dK", "dV")):
+        check_grad(g.cpu(), r, f"steep {n}")
