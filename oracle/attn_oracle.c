@@ -90,6 +90,16 @@ static double dot(const double *a, const double *b, int64_t n) {
  * s[j] = scale * q_i . k_j for visible j, -inf otherwise.
  * *m = max_j s[j]; *l = sum_j exp(s[j] - *m).  No visible key: *l = 0.
  */
+/* Score of query i (head h, row qi) against key j (row kj): the scaled dot
+ * product plus the positional bias when slopes are given. */
+static double score(const oracle_params *p, const double *qi, const double *kj, int64_t h,
+                    int64_t i, int64_t j) {
+  double sij = p->softmax_scale * dot(qi, kj, p->headdim);
+  if (p->alibi_slopes)
+    sij -= p->alibi_slopes[h] * fabs((double)(i + p->seqlen_k - p->seqlen_q - j));
+  return sij;
+}
+
 static void row_scores(const oracle_params *p, const double *q, const double *k,
                        int64_t b, int64_t h, int64_t i, double *s, double *m, double *l) {
   const int64_t g = kv_head(p, h);
@@ -98,9 +108,7 @@ static void row_scores(const oracle_params *p, const double *q, const double *k,
   int64_t count = 0;
   for (int64_t j = 0; j < p->seqlen_k; ++j) {
     if (!visible(p, i, j)) { s[j] = -INFINITY; continue; }
-    s[j] = p->softmax_scale * dot(qi, krow(p, k, b, j, g), p->headdim);
-    if (p->alibi_slopes)
-      s[j] -= p->alibi_slopes[h] * fabs((double)(i + p->seqlen_k - p->seqlen_q - j));
+    s[j] = score(p, qi, krow(p, k, b, j, g), h, i, j);
     if (s[j] > mx) mx = s[j];
     ++count;
   }
@@ -359,7 +367,7 @@ int oracle_attn_bwd_rows(const oracle_params *p, const double *q, const double *
         if (!visible(p, i, j)) continue;
         const int64_t row = (b * H + h) * Nq + i;
         const double *qi = qrow(p, q, b, i, h), *doi = qrow(p, dout, b, i, h);
-        const double sij = p->softmax_scale * dot(qi, kj, d);
+        const double sij = score(p, qi, kj, h, i, j);
         const double pij = prob(sij, M[row], L[row]);
         if (pij == 0.0) continue;
         const double ds = pij * (dot(doi, vj, d) - R[row]);

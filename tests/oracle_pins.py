@@ -347,20 +347,22 @@ def pin_empty_rows(orc):
 
 def pin_rows_match_full(orc):
     """The sampled-row entry points return exactly the full entry points'
-    rows."""
+    rows, with and without positional slopes."""
     B, H, Hkv, Nq, Nk, d = 2, 4, 2, 9, 11, 3
     q, k, v = rand((B, Nq, H, d), 60), rand((B, Nk, Hkv, d), 61), rand((B, Nk, Hkv, d), 62)
     do = rand((B, Nq, H, d), 63)
     qrows, krows = [0, 3, 8], [1, 10, 5]
-    for m in MASKS:
-        o, lse = orc.attention_fwd(q, k, v, 0.4, **m)
-        o_r, lse_r = orc.attention_fwd_rows(q, k, v, qrows, 0.4, **m)
-        assert np.array_equal(o[:, qrows], o_r) and np.array_equal(lse[:, :, qrows], lse_r)
-        dq, dk, dv = orc.attention_bwd(q, k, v, do, 0.4, **m)
-        dq_r, dk_r, dv_r = orc.attention_bwd_rows(q, k, v, do, qrows, krows, 0.4, **m)
-        _close(dq_r, dq[:, qrows], 1e-13, f"rows dQ {m}")
-        _close(dk_r, dk[:, krows], 1e-13, f"rows dK {m}")
-        _close(dv_r, dv[:, krows], 1e-13, f"rows dV {m}")
+    for slopes in (None, [0.5, 0.1, 0.02, 1.5]):
+        for m in MASKS:
+            kw = dict(m, alibi_slopes=slopes)
+            o, lse = orc.attention_fwd(q, k, v, 0.4, **kw)
+            o_r, lse_r = orc.attention_fwd_rows(q, k, v, qrows, 0.4, **kw)
+            assert np.array_equal(o[:, qrows], o_r) and np.array_equal(lse[:, :, qrows], lse_r)
+            dq, dk, dv = orc.attention_bwd(q, k, v, do, 0.4, **kw)
+            dq_r, dk_r, dv_r = orc.attention_bwd_rows(q, k, v, do, qrows, krows, 0.4, **kw)
+            _close(dq_r, dq[:, qrows], 1e-13, f"rows dQ {m} {slopes}")
+            _close(dk_r, dk[:, krows], 1e-13, f"rows dK {m} {slopes}")
+            _close(dv_r, dv[:, krows], 1e-13, f"rows dV {m} {slopes}")
 
 
 def pin_varlen_per_sequence(orc):

@@ -13,7 +13,10 @@ import pytest
 from oracle_pins import ALL_PINS
 
 MUTATIONS = {
-    "score_scale_dropped": ("s[j] = p->softmax_scale * dot(", "s[j] = dot("),
+    "score_scale_dropped": ("double sij = p->softmax_scale * dot(qi, kj, p->headdim);",
+                            "double sij = dot(qi, kj, p->headdim);"),
+    "rows_bias_dropped": ("const double sij = score(p, qi, kj, h, i, j);",
+                          "const double sij = p->softmax_scale * dot(qi, kj, d);"),
     "causal_off_by_one": ("if (p->causal && j > ii) return 0;", "if (p->causal && j >= ii) return 0;"),
     "window_left_sign": ("j < ii - p->window_left", "j < ii + p->window_left"),
     "window_right_ignored": ("if (p->window_right >= 0 && j > ii + p->window_right) return 0;", ""),
