@@ -70,6 +70,8 @@ class Oracle:
         for f in (lib.oracle_attn_fwd, lib.oracle_attn_fwd_rows, lib.oracle_attn_bwd,
                   lib.oracle_attn_bwd_rows):
             f.restype = ctypes.c_int
+        lib.oracle_attn_merge.argtypes = [ctypes.c_int64] * 5 + [d, d, d, d]
+        lib.oracle_attn_merge.restype = ctypes.c_int
         lib.oracle_num_threads.restype = ctypes.c_int
         lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
         self.lib = lib
@@ -180,6 +182,22 @@ class Oracle:
         return dq, dk, dv
 
 
+    def attention_merge(self, o_parts, lse_parts):
+        """Merge partial results over disjoint key sets: o_parts (S, B, Nq,
+        H, d), lse_parts (S, B, H, Nq) -> O (B, Nq, H, d), LSE (B, H, Nq),
+        float64."""
+        op, lp = _f64(o_parts), _f64(lse_parts)
+        S, B, Nq, H, d = op.shape
+        if lp.shape != (S, B, H, Nq):
+            raise ValueError("lse_parts must be (splits, batch, nheads, seqlen_q)")
+        o = np.zeros((B, Nq, H, d))
+        lse = np.zeros((B, H, Nq))
+        rc = self.lib.oracle_attn_merge(S, B, Nq, H, d, _ptr(op), _ptr(lp), _ptr(o), _ptr(lse))
+        if rc != 0:
+            raise ValueError("oracle_attn_merge rejected its arguments")
+        return o, lse
+
+
 def default() -> Oracle:
     """The oracle built from ``attn_oracle.c`` beside this file."""
     global _lib
@@ -260,3 +278,7 @@ def attention_fwd_varlen(*a, **kw):
 
 def attention_bwd_varlen(*a, **kw):
     return default().attention_bwd_varlen(*a, **kw)
+
+
+def attention_merge(*a, **kw):
+    return default().attention_merge(*a, **kw)

@@ -381,3 +381,45 @@ int oracle_attn_bwd_rows(const oracle_params *p, const double *q, const double *
   free(M); free(L); free(R);
   return 0;
 }
+
+/*
+ * Merge of partial results over disjoint key sets (split-KV decoding,
+ * sequence-parallel partials).  The exact identity behind the online softmax
+ * (the tiled, exact computation described on "FlashAttention ... Transformer
+ * optimization", items 1-2, and the FlashAttention-2 page's online softmax):
+ * for query row r with parts s computed over disjoint key sets,
+ *     LSE_r = log sum_s exp(LSE_s,r)
+ *     O_r   = sum_s exp(LSE_s,r - LSE_r) O_s,r
+ * and a row whose parts all have LSE = -inf (no key) gets O = 0, LSE = -inf.
+ * Layouts: o_parts (splits, B, Nq, H, d), lse_parts (splits, B, H, Nq); o
+ * (B, Nq, H, d), lse (B, H, Nq).
+ */
+int oracle_attn_merge(int64_t splits, int64_t B, int64_t Nq, int64_t H, int64_t d,
+                      const double *o_parts, const double *lse_parts, double *o, double *lse) {
+  if (splits < 1 || B < 0 || Nq < 0 || H < 1 || d < 1) return -1;
+  const int64_t rows = B * Nq * H, lrows = B * H * Nq;
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < rows; ++r) {
+    const int64_t h = r % H, i = (r / H) % Nq, b = r / (H * Nq);
+    const int64_t lr = (b * H + h) * Nq + i;
+    double m = -INFINITY;
+    for (int64_t s = 0; s < splits; ++s)
+      if (lse_parts[s * lrows + lr] > m) m = lse_parts[s * lrows + lr];
+    double *orow = o + r * d;
+    for (int64_t c = 0; c < d; ++c) orow[c] = 0.0;
+    if (m == -INFINITY) {
+      lse[lr] = -INFINITY;
+      continue;
+    }
+    double z = 0.0;
+    for (int64_t s = 0; s < splits; ++s) z += exp(lse_parts[s * lrows + lr] - m);
+    const double total = m + log(z);
+    for (int64_t s = 0; s < splits; ++s) {
+      const double w = exp(lse_parts[s * lrows + lr] - total);
+      const double *op = o_parts + s * rows * d + r * d;
+      for (int64_t c = 0; c < d; ++c) orow[c] += w * op[c];
+    }
+    lse[lr] = total;
+  }
+  return 0;
+}

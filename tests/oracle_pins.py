@@ -462,6 +462,30 @@ def pin_alibi_sdpa(orc):
             assert np.array_equal(o0, o1) and np.array_equal(lse0, lse1)
 
 
+def pin_merge_of_key_chunks(orc):
+    """Merging the oracle's results over disjoint key chunks (one of them
+    empty) equals the oracle over all keys: non-causal with GQA, and the
+    causal split-KV decoding shape (queries at the end of the keys, causal
+    only in the last chunk, which holds them)."""
+    B, H, Hkv, d = 2, 4, 2, 8
+    for nq, nk, causal, cuts in ((7, 23, False, (0, 5, 5, 16, 23)),
+                                 (3, 29, True, (0, 11, 20, 29))):
+        q, k, v = rand((B, nq, H, d), 90), rand((B, nk, Hkv, d), 91), rand((B, nk, Hkv, d), 92)
+        o_full, lse_full = orc.attention_fwd(q, k, v, 0.37, causal=causal)
+        parts_o, parts_l = [], []
+        for a, z in zip(cuts, cuts[1:]):
+            last = z == nk
+            o_p, l_p = orc.attention_fwd(q, k[:, a:z], v[:, a:z], 0.37, causal=causal and last)
+            parts_o.append(o_p)
+            parts_l.append(l_p)
+        o_m, lse_m = orc.attention_merge(np.stack(parts_o), np.stack(parts_l))
+        _close(o_m, o_full, 1e-12, f"merge O causal={causal}")
+        _close(lse_m, lse_full, 1e-12, f"merge LSE causal={causal}")
+    # a row no part sees: O = 0, LSE = -inf
+    o_m, lse_m = orc.attention_merge(np.zeros((2, 1, 1, 1, 4)), np.full((2, 1, 1, 1), -np.inf))
+    assert np.all(o_m == 0.0) and np.all(lse_m == -np.inf)
+
+
 ALL_PINS = [
     pin_golden_handworked,
     pin_identical_keys,
@@ -477,4 +501,5 @@ ALL_PINS = [
     pin_rows_match_full,
     pin_varlen_per_sequence,
     pin_alibi_sdpa,
+    pin_merge_of_key_chunks,
 ]

@@ -29,6 +29,9 @@ MUTATIONS = {
     "alibi_alignment_top_left": ("fabs((double)(i + p->seqlen_k - p->seqlen_q - j))",
                                  "fabs((double)(i - j))"),
     "alibi_wrong_head": ("p->alibi_slopes[h]", "p->alibi_slopes[0]"),
+    "merge_weight_not_normalised": ("const double w = exp(lse_parts[s * lrows + lr] - total);",
+                                    "const double w = exp(lse_parts[s * lrows + lr] - m);"),
+    "merge_lse_without_max": ("const double total = m + log(z);", "const double total = log(z);"),
     "ds_sign_flipped": ("(dp[j] - rowsum)", "(rowsum - dp[j])"),
     "ds_rowsum_dropped": ("(dp[j] - rowsum)", "(dp[j])"),
     "dk_scale_dropped": ("dkj[c] += p->softmax_scale * ds * qi[c];", "dkj[c] += ds * qi[c];"),
