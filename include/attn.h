@@ -266,6 +266,33 @@ ATTN_API const char* attn_status_string(int status);
  * failed.  *code receives an ATTN_ERR_* value or 0. */
 ATTN_API attn_status attn_get_device_status(void* stream, int* code);
 
+/* ------------------------------------------------------------------ merge
+ * Merge of partial results computed over disjoint key sets (split-KV
+ * decoding, sequence-parallel partials): for every query row,
+ *     LSE = log sum_s exp(LSE_s),   O = sum_s exp(LSE_s - LSE) O_s,
+ * the identity the tiled online softmax itself rests on ("FlashAttention ...
+ * transformer optimization", items 1-2).  A row whose parts all have
+ * LSE = -inf gets O = 0, LSE = -inf.  The parts are typically attn_fwd
+ * results over key ranges of one sequence (for causal decoding, the queries'
+ * own range causal and the earlier ranges not).
+ *
+ * Layouts (device, contiguous): o_parts (splits, batch, seqlen_q, nheads,
+ * headdim) 16-bit, 16-byte aligned; lse_parts (splits, batch, nheads,
+ * seqlen_q) fp32; o (batch, seqlen_q, nheads, headdim); lse (batch, nheads,
+ * seqlen_q).  Packed sequences: batch = 1, seqlen_q = total rows.  headdim
+ * 64, 128 or 256; splits 1 .. 65535.  Asynchronous on `stream`. */
+typedef struct {
+  int32_t splits;
+  int32_t batch;
+  int32_t seqlen_q;
+  int32_t nheads;
+  int32_t headdim;
+  int32_t dtype;  /* attn_dtype */
+} attn_merge_params;
+
+ATTN_API attn_status attn_merge(const attn_merge_params* p, const void* o_parts,
+                                const float* lse_parts, void* o, float* lse, void* stream);
+
 /* Diagnostic with no counterpart on the pages: checks the failure-detection
  * path on the device without faulting it.  Launches one small kernel on
  * `stream` whose two waiters (one warp-wide, one single-thread) wait on an

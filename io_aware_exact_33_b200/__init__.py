@@ -30,7 +30,7 @@ EXPORTED = ("attn_fwd", "attn_bwd", "attn_bwd_prepare", "attn_bwd_accumulate", "
             "attn_fwd_workspace_size", "attn_bwd_workspace_size", "attn_check_params",
             "attn_status_string", "attn_get_device_status", "attn_version", "attn_bwd_noalloc",
             "attn_selftest_bounded_wait", "attn_check_varlen_params", "attn_fwd_varlen",
-            "attn_bwd_varlen_workspace_size", "attn_bwd_varlen")
+            "attn_bwd_varlen_workspace_size", "attn_bwd_varlen", "attn_merge")
 
 
 class AttnParams(ctypes.Structure):
@@ -69,6 +69,12 @@ class AttnVarlenParams(ctypes.Structure):
         ("window_right", ctypes.c_int32),
         ("alibi_slopes", ctypes.c_void_p),
     ]
+
+
+class AttnMergeParams(ctypes.Structure):
+    """Mirror of ``attn_merge_params`` in include/attn.h."""
+    _fields_ = [(n, ctypes.c_int32) for n in
+                ("splits", "batch", "seqlen_q", "nheads", "headdim", "dtype")]
 
 
 class AttnError(RuntimeError):
@@ -113,6 +119,8 @@ def _load() -> ctypes.CDLL:
     lib.attn_fwd_varlen.restype = ctypes.c_int
     lib.attn_bwd_varlen.argtypes = [VP, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.attn_bwd_varlen.restype = ctypes.c_int
+    lib.attn_merge.argtypes = [ctypes.POINTER(AttnMergeParams), vp, vp, vp, vp, vp]
+    lib.attn_merge.restype = ctypes.c_int
     lib.attn_selftest_bounded_wait.argtypes = [ctypes.c_uint, vp, vp]
     lib.attn_selftest_bounded_wait.restype = ctypes.c_int
     lib.attn_version.argtypes = []
@@ -458,3 +466,28 @@ def attn_bwd_varlen(q, k, v, out, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seq
     if st != 0:
         raise AttnError(st, "attn_bwd_varlen")
     return dq, dk, dv
+
+
+# ----------------------------------------------------------------- merge of partial results
+def attn_merge(o_parts, lse_parts, out=None, lse=None, stream=None):
+    """Merge partial results over disjoint key sets (split-KV): o_parts
+    (S, B, Nq, H, d) 16-bit, lse_parts (S, B, H, Nq) float32, both CUDA and
+    contiguous.  Returns (out (B, Nq, H, d), lse (B, H, Nq))."""
+    import torch
+    _check(o_parts, "o_parts")
+    _check(lse_parts, "lse_parts")
+    if o_parts.dim() != 5 or lse_parts.dtype != torch.float32:
+        raise ValueError("o_parts must be (splits, B, Nq, H, d); lse_parts float32 (splits, B, H, Nq)")
+    S, B, Nq, H, d = o_parts.shape
+    if tuple(lse_parts.shape) != (S, B, H, Nq):
+        raise ValueError(f"lse_parts has shape {tuple(lse_parts.shape)}, expected {(S, B, H, Nq)}")
+    out = torch.empty(o_parts.shape[1:], dtype=o_parts.dtype, device=o_parts.device) if out is None else out
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=o_parts.device) if lse is None else lse
+    _check(out, "out", o_parts.shape[1:])
+    _check(lse, "lse", (B, H, Nq))
+    p = AttnMergeParams(S, B, Nq, H, d, _dtype_code(o_parts))
+    st = _lib.attn_merge(ctypes.byref(p), _ptr(o_parts), _ptr(lse_parts), _ptr(out), _ptr(lse),
+                         _stream(stream))
+    if st != 0:
+        raise AttnError(st, "attn_merge")
+    return out, lse

@@ -14,6 +14,7 @@
 #include "attn.h"
 #include "bwd_kernel.cuh"
 #include "fwd_kernel.cuh"
+#include "merge_kernel.cuh"
 #include "sm100.cuh"
 
 namespace {
@@ -706,6 +707,41 @@ attn_status attn_bwd_varlen(const attn_varlen_params* v, const int32_t* cu_seqle
   st = dispatch_bwd_main(&p, q, k, vv, dout, dk, dv, workspace, stream, pk);
   if (st != ATTN_OK) return st;
   return launch_bwd_finalize(&p, dq, workspace, stream, pk);
+}
+
+attn_status attn_merge(const attn_merge_params* p, const void* o_parts, const float* lse_parts,
+                       void* o, float* lse, void* stream_) {
+  if (!p || p->splits < 1 || p->splits > 65535 || p->batch < 0 || p->seqlen_q < 0 ||
+      p->nheads < 1)
+    return ATTN_ERR_INVALID_ARG;
+  if (p->headdim != 64 && p->headdim != 128 && p->headdim != 256)
+    return ATTN_ERR_UNSUPPORTED_HEADDIM;
+  if (p->dtype != ATTN_BF16 && p->dtype != ATTN_FP16) return ATTN_ERR_UNSUPPORTED_DTYPE;
+  const long long rows = (long long)p->batch * p->seqlen_q * p->nheads;
+  if (rows == 0) return ATTN_OK;
+  if (!o_parts || !lse_parts || !o || !lse) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(o_parts) || !aligned16(o) || (reinterpret_cast<uintptr_t>(lse_parts) & 3u) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return ATTN_ERR_MISALIGNED;
+  MergeParams mp;
+  mp.o_parts = static_cast<const uint16_t*>(o_parts);
+  mp.lse_parts = lse_parts;
+  mp.o = static_cast<uint16_t*>(o);
+  mp.lse = lse;
+  mp.splits = p->splits;
+  mp.nq = p->seqlen_q;
+  mp.nheads = p->nheads;
+  mp.headdim = p->headdim;
+  mp.rows = rows;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  const long long rows_per_block = 8LL * (32 / (p->headdim / 8));
+  long long blocks = (rows + rows_per_block - 1) / rows_per_block;
+  if (blocks > 4736) blocks = 4736;  // 32 x 148 SMs, grid-stride beyond
+  if (p->dtype == ATTN_FP16)
+    attn_merge_kernel<true><<<(unsigned)blocks, 256, 0, stream>>>(mp);
+  else
+    attn_merge_kernel<false><<<(unsigned)blocks, 256, 0, stream>>>(mp);
+  return finish(stream);
 }
 
 attn_status attn_selftest_bounded_wait(unsigned int wait_limit_us, int* result, void* stream_) {

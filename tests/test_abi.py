@@ -109,3 +109,19 @@ def test_alibi_pointer_alignment(attn):
     assert attn.attn_check_params(p, 0) == 4  # ATTN_ERR_MISALIGNED
     p.alibi_slopes = 256
     assert attn.attn_check_params(p, 0) == 0
+
+
+def test_merge_host_checks(attn):
+    """attn_merge rejects bad sizes before touching the GPU; an empty merge
+    is a no-op."""
+    def call(**kw):
+        base = dict(splits=2, batch=1, seqlen_q=4, nheads=2, headdim=128, dtype=0)
+        base.update(kw)
+        p = attn.AttnMergeParams(*[base[n] for n, _ in attn.AttnMergeParams._fields_])
+        return attn._lib.attn_merge(ctypes.byref(p), None, None, None, None, None)
+    assert call(splits=0) == 1
+    assert call(nheads=0) == 1
+    assert call(headdim=96) == 2
+    assert call(dtype=5) == 3
+    assert call(batch=0) == 0
+    assert call() == 1  # null pointers with work to do
