@@ -71,15 +71,26 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const MergeParams p) {
       float z = 0.f;
       for (int s = 0; s < p.splits; ++s) z += __expf(p.lse_parts[s * lrows + lr] - m);
       total = m + __logf(z);
-      for (int s = 0; s < p.splits; ++s) {
-        const float w = __expf(p.lse_parts[s * lrows + lr] - total);
-        if (w == 0.f) continue;  // a part with no key (its O is zero anyway)
-        float f[8];
-        unpack8<FP16>(*reinterpret_cast<const uint4*>(p.o_parts + (s * p.rows + r) * p.headdim +
-                                                       sub * 8),
-                      f);
+      // parts in groups of four, their loads issued before any is used
+      const uint16_t* base = p.o_parts + r * p.headdim + sub * 8;
+      const long long part_stride = p.rows * p.headdim;
+      for (int s0 = 0; s0 < p.splits; s0 += 4) {
+        uint4 v[4];
+        float w[4];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] = fmaf(w, f[e], acc[e]);
+        for (int u = 0; u < 4; ++u) {
+          const int s = s0 + u;
+          w[u] = s < p.splits ? __expf(p.lse_parts[s * lrows + lr] - total) : 0.f;
+          v[u] = s < p.splits ? *reinterpret_cast<const uint4*>(base + s * part_stride)
+                              : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          float f[8];
+          unpack8<FP16>(v[u], f);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[e] = fmaf(w[u], f[e], acc[e]);
+        }
       }
     }
     uint4 out;
