@@ -387,38 +387,61 @@ def run_gpu(args):
     t_fin = [e[3].elapsed_time(e[4]) for e in events] if bwd else [0.0]
     value = (f_fwd + f_bwd) * args.steps * world / (ms / 1e3) / 1e12
 
-    # end to end through the public API with pinned host buffers
+    # end to end through the public API with pinned host buffers: every step
+    # uploads its inputs, runs forward and backward, and downloads its
+    # results.  Two device buffer sets let step i+1's upload and step i-1's
+    # download run on their own streams while step i computes; the timed
+    # region spans the first upload to the last download.
     k_e2e = max(1, min(args.steps, args.e2e_steps))
-    hq, hk, hv, hdo = (t.pin_memory() for t in (q, k, v, do))
-    ho, hlse = torch.empty_like(hq).pin_memory(), torch.empty(lse.shape, dtype=torch.float32).pin_memory()
-    hdq, hdk, hdv = ((torch.empty_like(t).pin_memory() for t in (hq, hk, hv)) if bwd
-                     else (None, None, None))
-    h2d_pairs = [(qd, hq), (kd, hk), (vd, hv)] + ([(dod, hdo)] if bwd else [])
-    d2h_pairs = [(ho, o), (hlse, lse)] + ([(hdq, dq), (hdk, dk), (hdv, dv)] if bwd else [])
+    host_in = [t.pin_memory() for t in ((q, k, v, do) if bwd else (q, k, v))]
+    dev_out0 = [o, lse] + ([dq, dk, dv] if bwd else [])
+    host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in dev_out0]
+    sets = [([qd, kd, vd] + ([dod] if bwd else []), dev_out0)]
+    sets.append(([torch.empty_like(t) for t in sets[0][0]], [torch.empty_like(t) for t in dev_out0]))
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
 
-    def e2e_step():
-        for dst, src in h2d_pairs:
-            dst.copy_(src, non_blocking=True)
-        attn.attn_fwd(qd, kd, vd, w.scale, w.causal, w.window_left, w.window_right, out=o, lse=lse)
-        if bwd:
-            attn.attn_bwd(qd, kd, vd, o, lse, dod, w.scale, w.causal, w.window_left,
-                          w.window_right, dq=dq, dk=dk, dv=dv, workspace=ws)
-        for dst, src in d2h_pairs:
-            dst.copy_(src, non_blocking=True)
+    def e2e_run(n):
+        ev = [[torch.cuda.Event() for _ in range(3)] for _ in range(n)]  # uploaded, computed, downloaded
+        for i in range(n):
+            d_in, d_out = sets[i % 2]
+            with torch.cuda.stream(up):
+                if i >= 2:
+                    up.wait_event(ev[i - 2][1])  # this set's inputs are no longer read
+                for dst, src in zip(d_in, host_in):
+                    dst.copy_(src, non_blocking=True)
+                ev[i][0].record(up)
+            stream.wait_event(ev[i][0])
+            if i >= 2:
+                stream.wait_event(ev[i - 2][2])  # this set's outputs have been downloaded
+            qx, kx, vx = d_in[:3]
+            attn.attn_fwd(qx, kx, vx, w.scale, w.causal, w.window_left, w.window_right,
+                          out=d_out[0], lse=d_out[1])
+            if bwd:
+                attn.attn_bwd(qx, kx, vx, d_out[0], d_out[1], d_in[3], w.scale, w.causal,
+                              w.window_left, w.window_right, dq=d_out[2], dk=d_out[3],
+                              dv=d_out[4], workspace=ws)
+            ev[i][1].record(stream)
+            with torch.cuda.stream(down):
+                down.wait_event(ev[i][1])
+                for dst, src in zip(host_out, d_out):
+                    dst.copy_(src, non_blocking=True)
+                ev[i][2].record(down)
 
-    e2e_step()
+    e2e_run(2)
     torch.cuda.synchronize(dev)
     barrier(dist, dev)
     s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s2.record(stream)
-    for _ in range(k_e2e):
-        e2e_step()
-    e2.record(stream)
+    s2.record(up)
+    with torch.cuda.stream(down):
+        down.wait_event(s2)
+    stream.wait_event(s2)
+    e2e_run(k_e2e)
+    e2.record(down)
     torch.cuda.synchronize(dev)
     barrier(dist, dev)
     ms_e2e = max_over_ranks(s2.elapsed_time(e2), dist, dev)
-    h2d = sum(t.numel() * t.element_size() for _, t in h2d_pairs)
-    d2h = sum(t.numel() * t.element_size() for t, _ in d2h_pairs)
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
     status = attn.attn_get_device_status()
 
     if rank != 0:
@@ -462,7 +485,10 @@ def run_gpu(args):
         "kernels": rl,
         "cpu_baseline": cpu,
         "e2e": {"value": (f_fwd + f_bwd) * k_e2e * world / (ms_e2e / 1e3) / 1e12, "unit": UNIT,
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": k_e2e},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": k_e2e,
+                "ms_per_step": ms_e2e / k_e2e,
+                "copies": "pinned host buffers; uploads and downloads on their own streams, "
+                          "two device buffer sets, overlapping the neighbouring steps' compute"},
         "clocks": clocks,
         "gpu_launches": launches_per_step * args.steps,
         "device_status": status,
