@@ -125,3 +125,39 @@ def test_merge_host_checks(attn):
     assert call(dtype=5) == 3
     assert call(batch=0) == 0
     assert call() == 1  # null pointers with work to do
+
+
+def test_header_is_plain_c(attn, tmp_path):
+    """include/attn.h compiles as strict C99 and a C program links against
+    libattn.so and calls its host-only entry points (no GPU needed)."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_attn.c"
+    src.write_text(r"""
+#include <stdio.h>
+#include "attn.h"
+int main(void) {
+  attn_params p = {0};
+  p.batch = 2; p.seqlen_q = 100; p.seqlen_k = 100; p.nheads = 8; p.nheads_kv = 2;
+  p.headdim = 128; p.dtype = ATTN_BF16; p.softmax_scale = 0.088f;
+  attn_varlen_params v = {0};
+  v.batch = 3; v.total_q = 50; v.total_k = 60; v.max_seqlen_q = 20; v.max_seqlen_k = 30;
+  v.nheads = 8; v.nheads_kv = 2; v.headdim = 64; v.dtype = ATTN_FP16; v.softmax_scale = 0.125f;
+  printf("%d %d %d %zu %zu %s\n", (int)attn_check_params(&p, 0), (int)attn_check_params(&p, 1),
+         (int)attn_check_varlen_params(&v, 1), attn_bwd_workspace_size(&p),
+         attn_bwd_varlen_workspace_size(&v), attn_version());
+  return 0;
+}
+""")
+    libdir = os.path.dirname(attn.LIB_PATH)
+    exe = tmp_path / "use_attn"
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I",
+                    os.path.join(ROOT, "include"), str(src), "-o", str(exe), "-L", libdir, "-lattn",
+                    f"-Wl,-rpath,{libdir}"], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()
+    assert out[:3] == ["0", "0", "0"]
+    p = P(attn, batch=2, seqlen_q=100, seqlen_k=100, nheads=8, nheads_kv=2, headdim=128)
+    assert int(out[3]) == attn.attn_bwd_workspace_size(p)
+    assert int(out[4]) > 0 and out[5] == attn.attn_version()
