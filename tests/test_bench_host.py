@@ -1,6 +1,7 @@
 """bench.py host logic on the CPU: FLOP accounting, the exact visible-pair
 count, clock-sample parsing, and the multi-rank path (world size 2, gloo):
 barrier and the maximum over ranks that the timing uses."""
+import json
 import os
 import socket
 
@@ -98,3 +99,25 @@ def test_two_ranks_gloo_max_over_ranks():
 
 def test_single_rank_is_identity():
     assert bench.max_over_ranks(3.5, None) == 3.5
+
+
+def test_varlen_flops_match_closed_form():
+    """The packed workload's FLOPs: every causal sequence of L tokens has
+    L (L + 1) / 2 visible pairs (4 d FLOPs each forward, 2.5x backward)."""
+    import bench
+    from attn_inputs import VARLEN_WORKLOADS
+    w = VARLEN_WORKLOADS["varlen_causal_16seq_h32_d128"]
+    pairs = sum(n * (n + 1) // 2 for n in w.lens)
+    f, b = bench.varlen_flops(w)
+    assert f == 4.0 * w.nheads * w.headdim * pairs and b == 2.5 * f
+    assert len(w.lens) == 16 and all(256 <= n <= 1792 for n in w.lens)
+    cfg = bench.varlen_config(w)
+    assert cfg["tokens"] == sum(w.lens) and cfg["workload"] == w.name
+
+
+def test_reference_arm_declines_packed_workload(capsys):
+    import bench
+    assert bench.main(["--impl", "reference", "--workload", "varlen_causal_16seq_h32_d128",
+                       "--steps", "1", "--warmup", "3"]) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and "unavailable" in line
