@@ -68,6 +68,36 @@ def has_bwd(w):
     return "bwd" in w.passes
 
 
+def exact_pair_flops(w):
+    """(forward, backward) FLOPs counted on the exact visible (query, key)
+    pairs (for a causal N x N problem N (N + 1) / 2 pairs, where the formula
+    convention counts N^2 / 2)."""
+    pairs = visible_pairs(w.seqlen_q, w.seqlen_k, w.causal, w.window_left, w.window_right)
+    fwd = 4.0 * w.batch * w.nheads * pairs * w.headdim
+    return fwd, (2.5 * fwd if has_bwd(w) else 0.0)
+
+
+def environment(torch, dev):
+    """GPU, driver and library versions for the result line (best effort)."""
+    env = {}
+    try:
+        prop = torch.cuda.get_device_properties(dev)
+        env.update(gpu=prop.name, sm_count=prop.multi_processor_count,
+                   memory_gb=round(prop.total_memory / 1e9, 1))
+    except Exception:
+        pass
+    env.update(torch=torch.__version__, cuda_runtime=torch.version.cuda)
+    try:
+        out = subprocess.run(["nvidia-smi", "--query-gpu=driver_version", "--format=csv,noheader",
+                              "-i", str(dev.index or 0)], capture_output=True, text=True,
+                             timeout=10).stdout.strip()
+        if out:
+            env["driver"] = out.splitlines()[0]
+    except Exception:
+        pass
+    return env
+
+
 def flops_convention(w):
     if w.window_left >= 0 or w.window_right >= 0:
         return "exact visible pairs x 4d (fwd), x 10d (bwd)"
@@ -477,6 +507,7 @@ def run_gpu(args):
                         "nominal_2250": value / world / NOMINAL_BF16_TFLOPS,
                         "peak_source": peak_kind},
         "fwd_tflops": f_fwd / (mean(t_fwd) / 1e3) / 1e12,
+        "value_exact_pairs": (sum(exact_pair_flops(w)) * args.steps * world / (ms / 1e3) / 1e12),
         "bwd_tflops": (f_bwd / ((mean(t_prep) + mean(t_main) + mean(t_fin)) / 1e3) / 1e12
                        if bwd else None),
         "ms": {"fwd": mean(t_fwd), "bwd_prepare": mean(t_prep), "bwd_accumulate": mean(t_main),
@@ -492,6 +523,7 @@ def run_gpu(args):
         "clocks": clocks,
         "gpu_launches": launches_per_step * args.steps,
         "device_status": status,
+        "env": environment(torch, dev),
     }
     print(json.dumps(line), flush=True)
     if dist is not None:

@@ -121,3 +121,33 @@ def test_reference_arm_declines_packed_workload(capsys):
                        "--steps", "1", "--warmup", "3"]) == 0
     line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
     assert line["impl"] == "reference" and "unavailable" in line
+
+
+def test_exact_pair_flops():
+    import bench
+    w = WORKLOADS["causal_b2_h32_n8192_d128"]
+    f, b = bench.exact_pair_flops(w)
+    n = w.seqlen_q
+    assert f == 4.0 * w.batch * w.nheads * (n * (n + 1) // 2) * w.headdim and b == 2.5 * f
+    fc, _ = bench.step_flops(w)
+    assert 1.0 < f / fc < 1.0 + 2.0 / n
+    w4 = WORKLOADS["gqa_window_b4_h32_kv8_n4096_d128"]
+    assert bench.exact_pair_flops(w4) == bench.step_flops(w4)  # windows already count exactly
+
+
+def test_environment_is_best_effort():
+    import bench
+
+    class NoGpu:
+        __version__ = "x"
+
+        class version:
+            cuda = None
+
+        class cuda:
+            @staticmethod
+            def get_device_properties(dev):
+                raise RuntimeError("no device")
+
+    env = bench.environment(NoGpu, torch.device("cpu"))
+    assert env["torch"] == "x" and "gpu" not in env
