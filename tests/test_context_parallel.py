@@ -1,0 +1,261 @@
+"""Context-parallel attention (context_parallel.py).
+
+CPU: the chunk layouts and the ring schedule checked by brute force (every
+visible pair of chunks computed exactly once, zigzag balanced), and the ring
+itself run as gloo ranks (world sizes 1-3) with the library's kernels
+replaced by fakes: the forward by the float64 oracle on each chunk pair, the
+merge by the oracle's merge, the staged backward by the textbook gradient
+formulas against the given O and LSE.  The whole-sequence result is then
+compared with the oracle over the whole sequence.  GPU: one process (the
+ring of one rank, two zigzag chunks) on the real kernels."""
+import math
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+import oracle
+from attn_inputs import Workload, make_inputs
+from parity import check_grad, check_lse, check_o
+
+
+# ------------------------------------------------------------------ layouts and schedule
+@pytest.mark.parametrize("layout", ["contiguous", "zigzag"])
+@pytest.mark.parametrize("world", [1, 2, 3, 4, 5])
+@pytest.mark.parametrize("causal", [False, True])
+def test_schedule_covers_every_visible_pair_once(layout, world, causal):
+    from io_aware_exact_33_b200 import context_parallel as cp
+    nc = cp.num_chunks(world, layout)
+    owned = sorted(g for r in range(world) for g in cp.chunk_ids(r, world, layout))
+    assert owned == list(range(nc))
+    seen = {}
+    for r in range(world):
+        mine = cp.chunk_ids(r, world, layout)
+        for s, step in enumerate(cp.schedule(r, world, layout, causal)):
+            theirs = cp.chunk_ids((r - s) % world, world, layout)
+            for c, kc, cz in step:
+                key = (mine[c], theirs[kc])
+                assert key not in seen
+                seen[key] = cz
+    want = {(a, b): (causal and a == b) for a in range(nc) for b in range(nc)
+            if not causal or b <= a}
+    assert seen == want
+
+
+@pytest.mark.parametrize("world", [1, 2, 3, 4, 8])
+def test_zigzag_causal_steps_are_balanced(world):
+    """Work per rank and step in units of one full n x n pair (a causal
+    diagonal pair is half of one): two units everywhere."""
+    from io_aware_exact_33_b200 import context_parallel as cp
+    for r in range(world):
+        for step in cp.schedule(r, world, "zigzag", True):
+            assert sum(0.5 if cz else 1.0 for _, _, cz in step) == 2.0
+
+
+def test_shard_unshard_roundtrip():
+    from io_aware_exact_33_b200 import context_parallel as cp
+    x = torch.arange(2 * 24 * 3).reshape(2, 24, 3)
+    for layout in ("contiguous", "zigzag"):
+        for world in (1, 2, 3):
+            shards = [cp.shard(x, r, world, layout) for r in range(world)]
+            assert all(s.is_contiguous() for s in shards)
+            assert torch.equal(cp.unshard(shards, layout), x)
+    z = cp.shard(x, 0, 3, "zigzag")  # chunks 0 and 5 of 6
+    assert torch.equal(z[0], x[:, 0:4]) and torch.equal(z[1], x[:, 20:24])
+    with pytest.raises(ValueError):
+        cp.shard(torch.zeros(1, 10, 1), 0, 3, "zigzag")
+
+
+# ------------------------------------------------------------------ fakes of the kernels
+_STATE = {}
+
+
+def _fake_fwd(q, k, v, softmax_scale=None, causal=False, window_left=-1, window_right=-1,
+              out=None, lse=None, stream=None, alibi_slopes=None):
+    for t in (q, k, v, out, lse):
+        assert t.is_contiguous()
+    assert q.shape[1] == k.shape[1] and alibi_slopes is None
+    o, l = oracle.attention_fwd(q, k, v, softmax_scale, causal, window_left, window_right)
+    out.copy_(torch.from_numpy(o))
+    lse.copy_(torch.from_numpy(l))
+    return out, lse
+
+
+def _fake_merge(o_parts, lse_parts, out=None, lse=None, stream=None):
+    for t in (o_parts, lse_parts, out, lse):
+        assert t.is_contiguous()
+    o, l = oracle.attention_merge(o_parts, lse_parts)
+    out.copy_(torch.from_numpy(o))
+    lse.copy_(torch.from_numpy(l))
+    return out, lse
+
+
+def _fake_ws_size(p):
+    return 64
+
+
+def _fake_prepare(p, out, lse, dout, workspace, stream=None):
+    _STATE[workspace.data_ptr()] = dict(o=out.double(), lse=lse.double(), do=dout.double(),
+                                        dq=torch.zeros(out.shape, dtype=torch.float64))
+
+
+def _fake_accumulate(p, q, k, v, dout, dk, dv, workspace, stream=None):
+    """Gradient shares of one key block, probabilities taken against the
+    given (global) LSE and D = rowsum(dO o O) from the given (global) O."""
+    st = _STATE[workspace.data_ptr()]
+    assert p.seqlen_q == q.shape[1] and p.seqlen_k == k.shape[1] and p.window_left == -1
+    g = p.nheads // p.nheads_kv
+    qd = q.double()
+    kd = k.double().repeat_interleave(g, dim=2)
+    vd = v.double().repeat_interleave(g, dim=2)
+    s = torch.einsum("bihd,bjhd->bhij", qd, kd) * p.softmax_scale
+    if p.causal:
+        n, m = s.shape[-2:]
+        vis = torch.arange(m)[None, :] <= torch.arange(n)[:, None] + (m - n)
+        s = s.masked_fill(~vis, -math.inf)
+    prob = torch.exp(s - st["lse"][..., None])
+    dvec = (st["do"] * st["o"]).sum(-1).transpose(1, 2)  # (B, H, n)
+    dp = torch.einsum("bihd,bjhd->bhij", st["do"], vd)
+    ds = prob * (dp - dvec[..., None])
+    st["dq"] += torch.einsum("bhij,bjhd->bihd", ds, kd) * p.softmax_scale
+    dkh = torch.einsum("bhij,bihd->bjhd", ds, qd) * p.softmax_scale
+    dvh = torch.einsum("bhij,bihd->bjhd", prob, st["do"])
+    B, m, hkv, d = k.shape
+    dk.copy_(dkh.reshape(B, m, hkv, g, d).sum(3))
+    dv.copy_(dvh.reshape(B, m, hkv, g, d).sum(3))
+
+
+def _fake_finalize(p, dq, workspace, stream=None):
+    dq.copy_(_STATE.pop(workspace.data_ptr())["dq"])
+
+
+def _install_fakes():
+    import io_aware_exact_33_b200 as attn
+    attn.attn_fwd = _fake_fwd
+    attn.attn_merge = _fake_merge
+    attn.attn_bwd_workspace_size = _fake_ws_size
+    attn.attn_bwd_prepare = _fake_prepare
+    attn.attn_bwd_accumulate = _fake_accumulate
+    attn.attn_bwd_finalize = _fake_finalize
+
+
+@pytest.fixture
+def fakes(monkeypatch):
+    import io_aware_exact_33_b200 as attn
+    for name, f in (("attn_fwd", _fake_fwd), ("attn_merge", _fake_merge),
+                    ("attn_bwd_workspace_size", _fake_ws_size),
+                    ("attn_bwd_prepare", _fake_prepare),
+                    ("attn_bwd_accumulate", _fake_accumulate),
+                    ("attn_bwd_finalize", _fake_finalize)):
+        monkeypatch.setattr(attn, name, f)
+
+
+# ------------------------------------------------------------------ the ring on gloo ranks
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _ring_rank(rank, world, port, w, layout, queue):
+    import torch.distributed as dist
+    from io_aware_exact_33_b200 import context_parallel as cp
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        _install_fakes()
+        q, k, v, do = (cp.shard(t, rank, world, layout) for t in make_inputs(w))
+        o, lse = cp.ring_attn_fwd(q, k, v, w.softmax_scale, w.causal, layout)
+        dq, dk, dv = cp.ring_attn_bwd(q, k, v, o, lse, do, w.softmax_scale, w.causal, layout)
+        # the autograd wrapper runs the same two passes
+        ql, kl, vl = (t.clone().requires_grad_(True) for t in (q, k, v))
+        out = cp.ring_flash_attn_func(ql, kl, vl, w.softmax_scale, w.causal, layout)
+        out.backward(do)
+        same = (torch.equal(out.detach(), o) and torch.equal(ql.grad, dq) and
+                torch.equal(kl.grad, dk) and torch.equal(vl.grad, dv))
+        queue.put((rank, o, lse, dq, dk, dv, same))
+    finally:
+        dist.destroy_process_group()
+
+
+def _run_ring(world, w, layout):
+    oracle.build()
+    ctx = mp.get_context("spawn")
+    queue = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_ring_rank, args=(r, world, port, w, layout, queue))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted((queue.get(timeout=300) for _ in range(world)), key=lambda x: x[0])
+    for p in procs:
+        p.join(60)
+        assert p.exitcode == 0
+    return res
+
+
+def _compare_whole(res, w, layout, what):
+    from io_aware_exact_33_b200 import context_parallel as cp
+    q, k, v, do = make_inputs(w)
+    o_ref, lse_ref = oracle.attention_fwd(q, k, v, w.softmax_scale, w.causal)
+    g_ref = oracle.attention_bwd(q, k, v, do, w.softmax_scale, w.causal)
+    o = cp.unshard([r[1] for r in res], layout)
+    lse = cp.unshard([r[2] for r in res], layout, dim=2)
+    check_o(o, o_ref, what + " O")
+    check_lse(lse, lse_ref, what + " LSE")
+    for i, name in enumerate(("dQ", "dK", "dV")):
+        check_grad(cp.unshard([r[3 + i] for r in res], layout), g_ref[i], f"{what} {name}")
+    assert all(r[6] for r in res), f"{what}: autograd wrapper differs from the direct calls"
+
+
+@pytest.mark.parametrize("world,layout,causal", [
+    (2, "zigzag", True), (3, "zigzag", True), (2, "contiguous", True), (3, "contiguous", False),
+    (2, "zigzag", False),
+])
+def test_ring_on_gloo_ranks(world, layout, causal):
+    from io_aware_exact_33_b200 import context_parallel as cp
+    n = 6  # rows per chunk
+    N = n * cp.num_chunks(world, layout)
+    w = Workload("cp", 2, 4, 2, N, N, 8, causal, -1, -1, "bf16", 1.0, 800 + world,
+                 softmax_scale=0.4)
+    res = _run_ring(world, w, layout)
+    _compare_whole(res, w, layout, f"ring W={world} {layout} causal={causal}")
+
+
+def test_ring_of_one_process(fakes):
+    """Without a process group the ring is this process alone; zigzag then
+    holds chunks 0 and 1, and key chunk 0 collects dK / dV from both query
+    chunks."""
+    from io_aware_exact_33_b200 import context_parallel as cp
+    w = Workload("cp1", 1, 2, 1, 10, 10, 8, True, -1, -1, "bf16", 1.0, 810)
+    q, k, v, do = (cp.shard(t, 0, 1) for t in make_inputs(w))
+    o, lse = cp.ring_attn_fwd(q, k, v, None, True)
+    dq, dk, dv = cp.ring_attn_bwd(q, k, v, o, lse, do, None, True)
+    _compare_whole([(0, o, lse, dq, dk, dv, True)], w, "zigzag", "ring W=1")
+
+
+def test_ring_rejects_bad_layouts(fakes):
+    from io_aware_exact_33_b200 import context_parallel as cp
+    q = torch.zeros(1, 1, 4, 2, 8, dtype=torch.bfloat16)  # one chunk, zigzag wants two
+    with pytest.raises(ValueError):
+        cp.ring_attn_fwd(q, q, q, causal=True)
+    with pytest.raises(ValueError):
+        cp.chunk_ids(0, 2, "striped")
+
+
+# ------------------------------------------------------------------ GPU
+@pytest.mark.gpu
+def test_ring_of_one_process_on_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from io_aware_exact_33_b200 import context_parallel as cp
+    w = Workload("cpg", 2, 4, 2, 400, 400, 128, True, -1, -1, "bf16", 1.0, 811)
+    q, k, v, do = (cp.shard(t, 0, 1).cuda() for t in make_inputs(w))
+    o, lse = cp.ring_attn_fwd(q, k, v, None, True)
+    dq, dk, dv = cp.ring_attn_bwd(q, k, v, o, lse, do, None, True)
+    torch.cuda.synchronize()
+    res = [(0, o.cpu(), lse.cpu(), dq.cpu(), dk.cpu(), dv.cpu(), True)]
+    _compare_whole(res, w, "zigzag", "ring W=1 on GPU")
