@@ -161,8 +161,8 @@ ATTN_API attn_status attn_bwd_finalize(const attn_params* p, void* dq, void* wor
  * can fail) is not acceptable.  This entry point takes the same inputs and
  * outputs as attn_bwd and allocates nothing: its scratch is a fixed array of
  * ATTN_NOALLOC_SCRATCH_BYTES in the library's own device memory, which every
- * GPU that loads libattn.so holds until the process exits.  The paper has no
- * counterpart to this entry point.
+ * GPU that loads libattn.so holds until the process exits.  The method as the
+ * pages describe it has no counterpart to this entry point.
  *
  *   - Limit: the call is rejected with ATTN_ERR_WORKSPACE_TOO_SMALL when
  *     attn_bwd_workspace_size(p) exceeds ATTN_NOALLOC_SCRATCH_BYTES, before

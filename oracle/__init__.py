@@ -39,6 +39,10 @@ class OracleParams(ctypes.Structure):
         ("window_left", ctypes.c_int64),
         ("window_right", ctypes.c_int64),
         ("alibi_slopes", ctypes.c_void_p),
+        ("dropout_threshold", ctypes.c_int64),
+        ("dropout_seed", ctypes.c_uint64),
+        ("dropout_offset", ctypes.c_int64),
+        ("batch_base", ctypes.c_int64),
     ]
 
 
@@ -72,24 +76,33 @@ class Oracle:
             f.restype = ctypes.c_int
         lib.oracle_attn_merge.argtypes = [ctypes.c_int64] * 5 + [d, d, d, d]
         lib.oracle_attn_merge.restype = ctypes.c_int
+        u32p = ctypes.POINTER(ctypes.c_uint32)
+        lib.oracle_philox4x32_10.argtypes = [u32p, u32p, u32p]
+        lib.oracle_philox4x32_10.restype = None
+        lib.oracle_dropout_keep.argtypes = [P, ctypes.POINTER(ctypes.c_uint8)]
+        lib.oracle_dropout_keep.restype = ctypes.c_int
         lib.oracle_num_threads.restype = ctypes.c_int
         lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
         self.lib = lib
         self.path = lib_path
 
     def attention_fwd(self, q, k, v, softmax_scale=None, causal=False, window_left=-1,
-                      window_right=-1, alibi_slopes=None):
+                      window_right=-1, alibi_slopes=None, dropout_p=0.0, dropout_seed=0,
+                      dropout_offset=0):
         """O (B, Nq, H, d) and LSE (B, H, Nq), float64.  ``alibi_slopes``
         (H values, optional) adds -slope_h * |i + Nk - Nq - j| to the scores."""
         return self.attention_fwd_rows(q, k, v, None, softmax_scale, causal, window_left,
-                                       window_right, alibi_slopes)
+                                       window_right, alibi_slopes, dropout_p, dropout_seed,
+                                       dropout_offset)
 
     def attention_fwd_rows(self, q, k, v, rows, softmax_scale=None, causal=False,
-                           window_left=-1, window_right=-1, alibi_slopes=None):
+                           window_left=-1, window_right=-1, alibi_slopes=None, dropout_p=0.0,
+                           dropout_seed=0, dropout_offset=0, batch_base=0):
         """O and LSE for the query positions ``rows`` only (all rows if None):
         O (B, len(rows), H, d), LSE (B, H, len(rows))."""
         qa, ka, va = _f64(q), _f64(k), _f64(v)
-        p, _keep = _params(qa, ka, softmax_scale, causal, window_left, window_right, alibi_slopes)
+        p, _keep = _params(qa, ka, softmax_scale, causal, window_left, window_right, alibi_slopes,
+                           dropout_p, dropout_seed, dropout_offset, batch_base)
         B, Nq, H, d = qa.shape
         if rows is None:
             n, rp = Nq, None
@@ -105,10 +118,12 @@ class Oracle:
         return o, lse
 
     def attention_bwd(self, q, k, v, dout, softmax_scale=None, causal=False, window_left=-1,
-                      window_right=-1, alibi_slopes=None):
+                      window_right=-1, alibi_slopes=None, dropout_p=0.0, dropout_seed=0,
+                      dropout_offset=0, batch_base=0):
         """dQ (B, Nq, H, d), dK and dV (B, Nk, Hkv, d), float64."""
         qa, ka, va, da = _f64(q), _f64(k), _f64(v), _f64(dout)
-        p, _keep = _params(qa, ka, softmax_scale, causal, window_left, window_right, alibi_slopes)
+        p, _keep = _params(qa, ka, softmax_scale, causal, window_left, window_right, alibi_slopes,
+                           dropout_p, dropout_seed, dropout_offset, batch_base)
         dq = np.zeros_like(qa)
         dk = np.zeros_like(ka)
         dv = np.zeros_like(va)
@@ -119,11 +134,13 @@ class Oracle:
         return dq, dk, dv
 
     def attention_bwd_rows(self, q, k, v, dout, qrows, krows, softmax_scale=None, causal=False,
-                           window_left=-1, window_right=-1, alibi_slopes=None):
+                           window_left=-1, window_right=-1, alibi_slopes=None, dropout_p=0.0,
+                           dropout_seed=0, dropout_offset=0):
         """dQ at query positions ``qrows`` (B, nq, H, d) and dK, dV at key
         positions ``krows`` (B, nk, Hkv, d), float64."""
         qa, ka, va, da = _f64(q), _f64(k), _f64(v), _f64(dout)
-        p, _keep = _params(qa, ka, softmax_scale, causal, window_left, window_right, alibi_slopes)
+        p, _keep = _params(qa, ka, softmax_scale, causal, window_left, window_right, alibi_slopes,
+                           dropout_p, dropout_seed, dropout_offset)
         qr = np.ascontiguousarray(np.asarray(qrows, dtype=np.int64))
         kr = np.ascontiguousarray(np.asarray(krows, dtype=np.int64))
         B, _, H, d = qa.shape
@@ -146,7 +163,8 @@ class Oracle:
     # 的突破与实战解析", section "实操落地"), so the oracle runs the dense
     # definition on every sequence's rows.
     def attention_fwd_varlen(self, q, k, v, cu_q, cu_k, softmax_scale=None, causal=False,
-                             window_left=-1, window_right=-1, alibi_slopes=None):
+                             window_left=-1, window_right=-1, alibi_slopes=None, dropout_p=0.0,
+                             dropout_seed=0, dropout_offset=0):
         """q (Tq, H, d), k, v (Tk, Hkv, d), offsets cu_q, cu_k (batch + 1):
         O (Tq, H, d) and LSE (H, Tq), float64."""
         qa, ka, va = _f64(q), _f64(k), _f64(v)
@@ -158,15 +176,17 @@ class Oracle:
             q0, q1, k0, k1 = cq[b], cq[b + 1], ck[b], ck[b + 1]
             if q1 == q0:
                 continue
-            ob, lb = self.attention_fwd(qa[None, q0:q1], ka[None, k0:k1], va[None, k0:k1],
-                                        softmax_scale, causal, window_left, window_right,
-                                        alibi_slopes)
+            ob, lb = self.attention_fwd_rows(qa[None, q0:q1], ka[None, k0:k1], va[None, k0:k1],
+                                             None, softmax_scale, causal, window_left,
+                                             window_right, alibi_slopes, dropout_p, dropout_seed,
+                                             dropout_offset, batch_base=b)
             o[q0:q1] = ob[0]
             lse[:, q0:q1] = lb[0]
         return o, lse
 
     def attention_bwd_varlen(self, q, k, v, dout, cu_q, cu_k, softmax_scale=None, causal=False,
-                             window_left=-1, window_right=-1, alibi_slopes=None):
+                             window_left=-1, window_right=-1, alibi_slopes=None, dropout_p=0.0,
+                             dropout_seed=0, dropout_offset=0):
         """dQ (Tq, H, d), dK and dV (Tk, Hkv, d), float64, per sequence."""
         qa, ka, va, da = _f64(q), _f64(k), _f64(v), _f64(dout)
         cq, ck = _offsets(cu_q), _offsets(cu_k)
@@ -177,10 +197,34 @@ class Oracle:
                 continue
             g = self.attention_bwd(qa[None, q0:q1], ka[None, k0:k1], va[None, k0:k1],
                                    da[None, q0:q1], softmax_scale, causal, window_left,
-                                   window_right, alibi_slopes)
+                                   window_right, alibi_slopes, dropout_p, dropout_seed,
+                                   dropout_offset, batch_base=b)
             dq[q0:q1], dk[k0:k1], dv[k0:k1] = g[0][0], g[1][0], g[2][0]
         return dq, dk, dv
 
+
+    def philox4x32_10(self, counter, key):
+        """The generator's four output words for a counter of four 32-bit
+        words and a key of two."""
+        c = (ctypes.c_uint32 * 4)(*[int(x) & 0xFFFFFFFF for x in counter])
+        k = (ctypes.c_uint32 * 2)(*[int(x) & 0xFFFFFFFF for x in key])
+        out = (ctypes.c_uint32 * 4)()
+        self.lib.oracle_philox4x32_10(c, k, out)
+        return list(out)
+
+    def dropout_keep(self, batch, nheads, seqlen_q, seqlen_k, dropout_p, dropout_seed=0,
+                     dropout_offset=0, batch_base=0):
+        """The keep mask (B, H, Nq, Nk) uint8 of the dropout contract: 1 kept,
+        0 dropped (independent of the attention mask)."""
+        p = OracleParams(batch, seqlen_q, seqlen_k, nheads, 1, 1, 1.0, 0, -1, -1, None,
+                         dropout_threshold(dropout_p), int(dropout_seed) & (2 ** 64 - 1),
+                         int(dropout_offset) & 0xFFFFFFFF, int(batch_base))
+        keep = np.zeros((batch, nheads, seqlen_q, seqlen_k), dtype=np.uint8)
+        rc = self.lib.oracle_dropout_keep(ctypes.byref(p),
+                                          keep.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)))
+        if rc != 0:
+            raise ValueError("oracle_dropout_keep rejected its arguments")
+        return keep
 
     def attention_merge(self, o_parts, lse_parts):
         """Merge partial results over disjoint key sets: o_parts (S, B, Nq,
@@ -236,7 +280,19 @@ def _ptr(a: np.ndarray, ty=ctypes.c_double):
     return a.ctypes.data_as(ctypes.POINTER(ty))
 
 
-def _params(q, k, softmax_scale, causal, window_left, window_right, alibi_slopes=None):
+def dropout_threshold(dropout_p: float) -> int:
+    """The drop threshold t = round(256 p) of the dropout contract (an
+    element is dropped iff its random byte is below t); p' = t / 256 is the
+    rate actually applied.  p must lie in [0, 1) with t <= 255."""
+    p = float(dropout_p)
+    t = int(math.floor(256.0 * p + 0.5))
+    if not (0.0 <= p < 1.0) or t > 255:
+        raise ValueError(f"dropout_p must be in [0, 255.5/256), got {dropout_p}")
+    return t
+
+
+def _params(q, k, softmax_scale, causal, window_left, window_right, alibi_slopes=None,
+            dropout_p=0.0, dropout_seed=0, dropout_offset=0, batch_base=0):
     """The C parameter block and the slopes array it points to (keep both
     alive for the call)."""
     B, Nq, H, d = q.shape
@@ -253,7 +309,9 @@ def _params(q, k, softmax_scale, causal, window_left, window_right, alibi_slopes
             raise ValueError("alibi_slopes needs one slope per query head")
     ptr = slopes.ctypes.data if slopes is not None else None
     return OracleParams(B, Nq, Nk, H, Hkv, d, scale, int(bool(causal)),
-                        int(window_left), int(window_right), ptr), slopes
+                        int(window_left), int(window_right), ptr, dropout_threshold(dropout_p),
+                        int(dropout_seed) & (2 ** 64 - 1), int(dropout_offset) & 0xFFFFFFFF,
+                        int(batch_base)), slopes
 
 
 def attention_fwd(*a, **kw):
@@ -282,3 +340,11 @@ def attention_bwd_varlen(*a, **kw):
 
 def attention_merge(*a, **kw):
     return default().attention_merge(*a, **kw)
+
+
+def philox4x32_10(*a, **kw):
+    return default().philox4x32_10(*a, **kw)
+
+
+def dropout_keep(*a, **kw):
+    return default().dropout_keep(*a, **kw)

@@ -35,6 +35,22 @@
  *     slopes (NULL) means no bias.
  *   - LSE_i = m_i + ln(l_i), natural log, of the scaled scores.  A row with
  *     no visible key gets O = 0 and LSE = -inf.
+ *   - Dropout on the attention probabilities (named as a supported feature
+ *     on page 5, hardware/dtype section: the backward's head-dim limit
+ *     "without dropout" and the backends that offer dropout; no formula is
+ *     given).  Reading taken: inverted dropout,
+ *         O_i = sum_j P_ij z_ij V_j,   z_ij = 0 (dropped) or 1 / (1 - p'),
+ *     with P, m, l and LSE those of the undropped scores.  The drop
+ *     decisions come from a counter-based generator so that any program can
+ *     reproduce them: Philox4x32-10 (Salmon, Moraes, Dror and Shaw,
+ *     "Parallel random numbers: as easy as 1, 2, 3", SC 2011) with key
+ *     (seed low word, seed high word) and, for element (b, h, i, j) of the
+ *     score matrix, counter (j / 4, i / 4, b * H + h, offset); its output
+ *     word i mod 4, byte j mod 4 (bits 8 (j mod 4) and up) is the element's
+ *     random byte u, and the element is dropped iff u < t for the threshold
+ *     t = round(256 p) in [0, 255]; p' = t / 256.  t = 0 is no dropout.
+ *     Backward through the same mask: dP_ij = z_ij dO_i . V_j and
+ *     dV_j = sum_i P_ij z_ij dO_i; the dS formula below is unchanged.
  *   - Backward (page 2, item 2: the backward pass recomputes the score
  *     matrix; the arithmetic is the analytic gradient of the definition):
  *         dV = P^T dO,  dP = dO V^T,
@@ -58,7 +74,48 @@ typedef struct {
   double softmax_scale;
   int64_t causal, window_left, window_right;
   const double *alibi_slopes; /* nheads slopes, or NULL */
+  int64_t dropout_threshold;  /* t in [0, 255]; 0 = no dropout */
+  uint64_t dropout_seed;
+  int64_t dropout_offset;     /* the counter's last word (32 bits) */
+  int64_t batch_base;         /* counter batch index of this call's batch 0 */
 } oracle_params;
+
+/* Philox4x32-10 (the SC 2011 paper above).  One round: the 64-bit products
+ * of counter words 0 and 2 with the two multipliers; the new words are
+ * (high half of product 2) ^ word 1 ^ key 0, low half of product 2,
+ * (high half of product 0) ^ word 3 ^ key 1, low half of product 0.  The key
+ * advances by the two Weyl constants after every round; ten rounds. */
+void oracle_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4]) {
+  const uint32_t m0 = 0xD2511F53u, m1 = 0xCD9E8D57u, w0 = 0x9E3779B9u, w1 = 0xBB67AE85u;
+  uint32_t x0 = ctr[0], x1 = ctr[1], x2 = ctr[2], x3 = ctr[3], k0 = key[0], k1 = key[1];
+  for (int r = 0; r < 10; ++r) {
+    const uint64_t p0 = (uint64_t)m0 * x0, p1 = (uint64_t)m1 * x2;
+    const uint32_t y0 = (uint32_t)(p1 >> 32) ^ x1 ^ k0;
+    const uint32_t y2 = (uint32_t)(p0 >> 32) ^ x3 ^ k1;
+    x1 = (uint32_t)p1;
+    x3 = (uint32_t)p0;
+    x0 = y0;
+    x2 = y2;
+    k0 += w0;
+    k1 += w1;
+  }
+  out[0] = x0; out[1] = x1; out[2] = x2; out[3] = x3;
+}
+
+/* Dropout factor z of score element (b, h, i, j): 1 without dropout, else 0
+ * (dropped) or 256 / (256 - t) (the counter layout stated above). */
+static double keep_scale(const oracle_params *p, int64_t b, int64_t h, int64_t i, int64_t j) {
+  if (p->dropout_threshold <= 0) return 1.0;
+  const uint32_t ctr[4] = {(uint32_t)(j >> 2), (uint32_t)(i >> 2),
+                           (uint32_t)((p->batch_base + b) * p->nheads + h),
+                           (uint32_t)p->dropout_offset};
+  const uint32_t key[2] = {(uint32_t)p->dropout_seed, (uint32_t)(p->dropout_seed >> 32)};
+  uint32_t out[4];
+  oracle_philox4x32_10(ctr, key, out);
+  const uint32_t u = (out[i & 3] >> (8 * (j & 3))) & 0xFFu;
+  if (u < (uint32_t)p->dropout_threshold) return 0.0;
+  return 256.0 / (256.0 - (double)p->dropout_threshold);
+}
 
 /* Visibility of key j from query i (the mask reading stated above). */
 static int visible(const oracle_params *p, int64_t i, int64_t j) {
@@ -136,15 +193,17 @@ static void fwd_row(const oracle_params *p, const double *q, const double *k, co
   for (int64_t j = 0; j < p->seqlen_k; ++j) {
     double pij = prob(s[j], m, l);
     if (pij == 0.0) continue;
+    const double zij = keep_scale(p, b, h, i, j);
     const double *vj = krow(p, v, b, j, g);
-    for (int64_t c = 0; c < d; ++c) o_out[c] += pij * vj[c];
+    for (int64_t c = 0; c < d; ++c) o_out[c] += pij * zij * vj[c];
   }
   *lse_out = m + log(l);
 }
 
 static int valid(const oracle_params *p) {
   return p && p->batch >= 0 && p->seqlen_q >= 0 && p->seqlen_k >= 0 && p->nheads > 0 &&
-         p->nheads_kv > 0 && p->nheads % p->nheads_kv == 0 && p->headdim > 0;
+         p->nheads_kv > 0 && p->nheads % p->nheads_kv == 0 && p->headdim > 0 &&
+         p->dropout_threshold >= 0 && p->dropout_threshold <= 255 && p->batch_base >= 0;
 }
 
 int oracle_num_threads(void) {
@@ -224,13 +283,14 @@ int oracle_attn_bwd(const oracle_params *p, const double *q, const double *k, co
     double *s = (double *)malloc(sizeof(double) * n);
     double *pr = (double *)malloc(sizeof(double) * n);
     double *dp = (double *)malloc(sizeof(double) * n);
-    if (!s || !pr || !dp) {
+    double *zr = (double *)malloc(sizeof(double) * n);
+    if (!s || !pr || !dp || !zr) {
 #pragma omp atomic write
       bad = 1;
     }
 #pragma omp for schedule(dynamic, 1)
     for (int64_t t = 0; t < B * Hkv; ++t) {
-      if (!s || !pr || !dp) continue;
+      if (!s || !pr || !dp || !zr) continue;
       const int64_t b = t / Hkv, g = t % Hkv;
       for (int64_t h = g * group; h < (g + 1) * group; ++h) {
         for (int64_t i = 0; i < Nq; ++i) {
@@ -242,7 +302,8 @@ int oracle_attn_bwd(const oracle_params *p, const double *q, const double *k, co
           double rowsum = 0.0; /* sum_j P_ij dP_ij */
           for (int64_t j = 0; j < Nk; ++j) {
             pr[j] = prob(s[j], m, l);
-            dp[j] = (pr[j] != 0.0) ? dot(doi, krow(p, v, b, j, g), d) : 0.0;
+            zr[j] = (pr[j] != 0.0) ? keep_scale(p, b, h, i, j) : 0.0;
+            dp[j] = (pr[j] != 0.0) ? zr[j] * dot(doi, krow(p, v, b, j, g), d) : 0.0;
             rowsum += pr[j] * dp[j];
           }
           for (int64_t c = 0; c < d; ++c) dqi[c] = 0.0;
@@ -255,13 +316,13 @@ int oracle_attn_bwd(const oracle_params *p, const double *q, const double *k, co
             for (int64_t c = 0; c < d; ++c) {
               dqi[c] += p->softmax_scale * ds * kj[c];
               dkj[c] += p->softmax_scale * ds * qi[c];
-              dvj[c] += pr[j] * doi[c];
+              dvj[c] += pr[j] * zr[j] * doi[c];
             }
           }
         }
       }
     }
-    free(s); free(pr); free(dp);
+    free(s); free(pr); free(dp); free(zr);
   }
   return bad ? -1 : 0;
 }
@@ -307,7 +368,8 @@ int oracle_attn_bwd_rows(const oracle_params *p, const double *q, const double *
       double rowsum = 0.0;
       for (int64_t j = 0; j < Nk; ++j) {
         pr[j] = prob(s[j], m, l);
-        dp[j] = (pr[j] != 0.0) ? dot(doi, krow(p, v, b, j, g), d) : 0.0;
+        dp[j] = (pr[j] != 0.0) ? keep_scale(p, b, h, i, j) * dot(doi, krow(p, v, b, j, g), d)
+                               : 0.0;
         rowsum += pr[j] * dp[j];
       }
       for (int64_t c = 0; c < d; ++c) dqi[c] = 0.0;
@@ -345,7 +407,8 @@ int oracle_attn_bwd_rows(const oracle_params *p, const double *q, const double *
       row_scores(p, q, k, b, h, i, s, &m, &l);
       for (int64_t j = 0; j < Nk; ++j) {
         const double pij = prob(s[j], m, l);
-        if (pij != 0.0) rowsum += pij * dot(doi, krow(p, v, b, j, g), d);
+        if (pij != 0.0)
+          rowsum += pij * keep_scale(p, b, h, i, j) * dot(doi, krow(p, v, b, j, g), d);
       }
       M[t] = m; L[t] = l; R[t] = rowsum;
     }
@@ -370,15 +433,33 @@ int oracle_attn_bwd_rows(const oracle_params *p, const double *q, const double *
         const double sij = score(p, qi, kj, h, i, j);
         const double pij = prob(sij, M[row], L[row]);
         if (pij == 0.0) continue;
-        const double ds = pij * (dot(doi, vj, d) - R[row]);
+        const double zij = keep_scale(p, b, h, i, j);
+        const double ds = pij * (zij * dot(doi, vj, d) - R[row]);
         for (int64_t c = 0; c < d; ++c) {
           dkj[c] += p->softmax_scale * ds * qi[c];
-          dvj[c] += pij * doi[c];
+          dvj[c] += pij * zij * doi[c];
         }
       }
     }
   }
   free(M); free(L); free(R);
+  return 0;
+}
+
+/*
+ * The dropout keep mask: keep (B, H, Nq, Nk), 1 where element (b, h, i, j)
+ * is kept, 0 where dropped, for every element whether masked or not (the
+ * decision does not depend on the mask).  Returns 0, or -1 on invalid
+ * arguments.
+ */
+int oracle_dropout_keep(const oracle_params *p, uint8_t *keep) {
+  if (!valid(p)) return -1;
+  const int64_t B = p->batch, H = p->nheads, Nq = p->seqlen_q, Nk = p->seqlen_k;
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < B * H * Nq; ++t) {
+    const int64_t i = t % Nq, h = (t / Nq) % H, b = t / (Nq * H);
+    for (int64_t j = 0; j < Nk; ++j) keep[t * Nk + j] = keep_scale(p, b, h, i, j) != 0.0;
+  }
   return 0;
 }
 

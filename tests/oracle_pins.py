@@ -486,6 +486,186 @@ def pin_merge_of_key_chunks(orc):
     assert np.all(o_m == 0.0) and np.all(lse_m == -np.inf)
 
 
+# --- dropout -----------------------------------------------------------------
+# Dropout on the attention probabilities is named on page 5 (hardware/dtype
+# section) without a formula; the oracle's reading is inverted dropout with
+# the drop decisions of a Philox4x32-10 counter-based generator (see
+# attn_oracle.c).  The generator is pinned to cuRAND's host-side Philox
+# generator (run, not read); the arithmetic to unbiasedness, finite
+# differences and the no-dropout special case.
+
+def _curand_philox_groups(seed, ngroups):
+    """cuRAND's host generator (PHILOX4_32_10, default ordering) for a 64-bit
+    seed: its first ngroups blocks of four 32-bit outputs."""
+    import ctypes
+    lib = ctypes.CDLL("libcurand.so")
+    gen = ctypes.c_void_p()
+    assert lib.curandCreateGeneratorHost(ctypes.byref(gen), 161) == 0  # PHILOX4_32_10
+    try:
+        assert lib.curandSetPseudoRandomGeneratorSeed(gen, ctypes.c_ulonglong(seed)) == 0
+        buf = (ctypes.c_uint32 * (4 * ngroups))()
+        assert lib.curandGenerate(gen, buf, ctypes.c_size_t(4 * ngroups)) == 0
+        out = list(buf)
+    finally:
+        lib.curandDestroyGenerator(gen)
+    return [out[4 * g:4 * g + 4] for g in range(ngroups)]
+
+
+def pin_philox_against_curand(orc):
+    """The oracle's Philox4x32-10 equals cuRAND's host generator, whose g-th
+    block of four outputs is the generator at counter (0, 0, g, 0) under key
+    (seed low word, seed high word)."""
+    for seed in (0x123456789ABCDEF0, 0, 42, 2 ** 64 - 1, 0x0F1E2D3C4B5A6978):
+        key = (seed & 0xFFFFFFFF, seed >> 32)
+        for g, want in enumerate(_curand_philox_groups(seed, 48)):
+            got = orc.philox4x32_10((0, 0, g, 0), key)
+            assert got == want, f"philox seed={seed:#x} counter word2={g}: {got} != {want}"
+
+
+def _contract_keep(orc, B, H, Nq, Nk, t, seed, offset):
+    """The keep mask evaluated from the generator by the counter layout."""
+    key = (seed & 0xFFFFFFFF, seed >> 32)
+    keep = np.zeros((B, H, Nq, Nk), dtype=np.uint8)
+    for b in range(B):
+        for h in range(H):
+            for i0 in range(0, Nq, 4):
+                for j0 in range(0, Nk, 4):
+                    words = orc.philox4x32_10((j0 // 4, i0 // 4, b * H + h, offset), key)
+                    for i in range(i0, min(i0 + 4, Nq)):
+                        for j in range(j0, min(j0 + 4, Nk)):
+                            u = (words[i % 4] >> (8 * (j % 4))) & 0xFF
+                            keep[b, h, i, j] = u >= t
+    return keep
+
+
+def pin_dropout_mask(orc):
+    """The keep mask: it follows the counter layout from the generator; the
+    drop rate is t / 256 at several thresholds (a uniform byte); neighbours
+    along rows, columns and diagonals, other offsets and other heads are
+    uncorrelated (|corr| within 5 / sqrt(n))."""
+    B, H, N = 2, 3, 256
+    seed = 0xDEADBEEF12345
+    keep = orc.dropout_keep(B, H, 9, 13, 0.3, seed, 7)
+    assert np.array_equal(keep, _contract_keep(orc, B, H, 9, 13, orc_threshold(0.3), seed, 7))
+    n = B * H * N * N
+    for p in (1 / 256, 0.1, 0.5, 255 / 256):
+        t = orc_threshold(p)
+        drop = 1.0 - orc.dropout_keep(B, H, N, N, p, seed, 3).astype(np.float64)
+        rate = t / 256
+        sd = math.sqrt(rate * (1 - rate) / n)
+        assert abs(drop.mean() - rate) <= 5 * sd + 1e-12, f"drop rate {drop.mean()} vs {rate}"
+    k = orc.dropout_keep(B, H, N, N, 0.5, seed, 3).astype(np.float64) - 0.5
+    k2 = orc.dropout_keep(B, H, N, N, 0.5, seed, 4).astype(np.float64) - 0.5
+
+    def corr(a, b):
+        return float((a * b).mean() / math.sqrt((a * a).mean() * (b * b).mean()))
+
+    pairs = {"row": (k[..., :, 1:], k[..., :, :-1]), "col": (k[..., 1:, :], k[..., :-1, :]),
+             "diag": (k[..., 1:, 1:], k[..., :-1, :-1]), "offset": (k, k2),
+             "head": (k[:, 1:], k[:, :-1]), "batch": (k[1:], k[:-1])}
+    for what, (a, b) in pairs.items():
+        assert abs(corr(a, b)) <= 5 / math.sqrt(a.size), f"keep bits correlated along {what}"
+
+
+def orc_threshold(p):
+    import oracle
+    return oracle.dropout_threshold(p)
+
+
+def pin_dropout_special_cases(orc):
+    """p = 0 and any p below 1/512 (threshold 0) are exactly no dropout; a
+    threshold of 1 changes the output; the mask ignores the attention mask."""
+    B, H, Hkv, Nq, Nk, d = 1, 2, 1, 6, 9, 3
+    q, k, v = rand((B, Nq, H, d), 90), rand((B, Nk, Hkv, d), 91), rand((B, Nk, Hkv, d), 92)
+    do = rand((B, Nq, H, d), 93)
+    o0, l0 = orc.attention_fwd(q, k, v, 0.5, True)
+    g0 = orc.attention_bwd(q, k, v, do, 0.5, True)
+    for p in (0.0, 1.0 / 1024):
+        o, l = orc.attention_fwd(q, k, v, 0.5, True, dropout_p=p, dropout_seed=5)
+        g = orc.attention_bwd(q, k, v, do, 0.5, True, dropout_p=p, dropout_seed=5)
+        assert np.array_equal(o, o0) and np.array_equal(l, l0)
+        assert all(np.array_equal(a, b) for a, b in zip(g, g0))
+    o, l = orc.attention_fwd(q, k, v, 0.5, True, dropout_p=0.5, dropout_seed=5)
+    assert np.array_equal(l, l0), "dropout must not change the LSE"
+    assert not np.allclose(o, o0)
+
+
+def pin_dropout_unbiased(orc):
+    """Inverted dropout keeps the expectation: the mean of O over many
+    offsets converges to O without dropout (within 5 standard errors per
+    element), for p = 0.25 and p = 0.6, causal and full."""
+    B, H, Hkv, Nq, Nk, d = 1, 2, 1, 5, 11, 3
+    q, k, v = rand((B, Nq, H, d), 94), rand((B, Nk, Hkv, d), 95), rand((B, Nk, Hkv, d), 96)
+    K = 1500
+    for p, causal in ((0.25, True), (0.6, False)):
+        o_ref, _ = orc.attention_fwd(q, k, v, 0.8, causal)
+        samples = np.stack([orc.attention_fwd(q, k, v, 0.8, causal, dropout_p=p,
+                                              dropout_seed=77, dropout_offset=off)[0]
+                            for off in range(K)])
+        mean, se = samples.mean(0), samples.std(0) / math.sqrt(K)
+        assert np.all(np.abs(mean - o_ref) <= 5 * se + 1e-12), \
+            f"dropout mean off by {np.max(np.abs(mean - o_ref) / (se + 1e-300)):.1f} s.e."
+
+
+def pin_dropout_finite_differences(orc):
+    """With the drop decisions fixed (seed and offset), O is a smooth
+    function of Q, K and V: central differences of sum(O o dO) agree with
+    the backward, and the sampled-row backward equals the full one."""
+    h = 1e-6
+    B, H, Hkv, Nq, Nk, d = 1, 2, 1, 6, 8, 3
+    q, k, v = rand((B, Nq, H, d), 97), rand((B, Nk, Hkv, d), 98), rand((B, Nk, Hkv, d), 99)
+    do = rand((B, Nq, H, d), 100)
+    for m in (dict(causal=False), dict(causal=True)):
+        kw = dict(m, dropout_p=0.35, dropout_seed=1234, dropout_offset=9)
+        dq, dk, dv = orc.attention_bwd(q, k, v, do, 0.6, **kw)
+
+        def loss(qq, kk, vv):
+            return float((orc.attention_fwd(qq, kk, vv, 0.6, **kw)[0] * do.numpy()).sum())
+
+        for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+            fd = np.zeros(x.shape)
+            flat = x.reshape(-1)
+            for idx in range(flat.numel()):
+                args = {"q": q, "k": k, "v": v}
+                xp, xm = flat.clone(), flat.clone()
+                xp[idx] += h
+                xm[idx] -= h
+                args[name] = xp.reshape(x.shape)
+                lp = loss(args["q"], args["k"], args["v"])
+                args[name] = xm.reshape(x.shape)
+                lm = loss(args["q"], args["k"], args["v"])
+                fd.reshape(-1)[idx] = (lp - lm) / (2 * h)
+            err = np.abs(fd - g).max() / max(1.0, np.abs(fd).max())
+            assert err <= 1e-6, f"dropout finite differences d{name} {m}: {err:.2e}"
+        qrows, krows = [0, 5, 2], [7, 0, 3]
+        dq_r, dk_r, dv_r = orc.attention_bwd_rows(q, k, v, do, qrows, krows, 0.6, **kw)
+        _close(dq_r, dq[:, qrows], 1e-13, "dropout rows dQ")
+        _close(dk_r, dk[:, krows], 1e-13, "dropout rows dK")
+        _close(dv_r, dv[:, krows], 1e-13, "dropout rows dV")
+        o_r, _ = orc.attention_fwd_rows(q, k, v, qrows, 0.6, **kw)
+        assert np.array_equal(o_r, orc.attention_fwd(q, k, v, 0.6, **kw)[0][:, qrows])
+
+
+def pin_dropout_varlen_numbering(orc):
+    """Packed sequences number their drop decisions by sequence index: equal
+    lengths packed give the dense batched result."""
+    B, H, N, d = 3, 2, 7, 3
+    q, k, v = rand((B, N, H, d), 101), rand((B, N, H, d), 102), rand((B, N, H, d), 103)
+    do = rand((B, N, H, d), 104)
+    kw = dict(dropout_p=0.4, dropout_seed=99, dropout_offset=1)
+    cu = [0, N, 2 * N, 3 * N]
+    o, lse = orc.attention_fwd(q, k, v, 0.5, True, **kw)
+    ov, lv = orc.attention_fwd_varlen(q.reshape(B * N, H, d), k.reshape(B * N, H, d),
+                                      v.reshape(B * N, H, d), cu, cu, 0.5, True, **kw)
+    _close(ov, o.reshape(B * N, H, d), 1e-14, "varlen dropout O")
+    g = orc.attention_bwd(q, k, v, do, 0.5, True, **kw)
+    gv = orc.attention_bwd_varlen(q.reshape(B * N, H, d), k.reshape(B * N, H, d),
+                                  v.reshape(B * N, H, d), do.reshape(B * N, H, d), cu, cu, 0.5,
+                                  True, **kw)
+    for a, b_, n in zip(gv, g, ("dQ", "dK", "dV")):
+        _close(a, b_.reshape(B * N, H, d), 1e-14, "varlen dropout " + n)
+
+
 ALL_PINS = [
     pin_golden_handworked,
     pin_identical_keys,
@@ -502,4 +682,10 @@ ALL_PINS = [
     pin_varlen_per_sequence,
     pin_alibi_sdpa,
     pin_merge_of_key_chunks,
+    pin_philox_against_curand,
+    pin_dropout_mask,
+    pin_dropout_special_cases,
+    pin_dropout_unbiased,
+    pin_dropout_finite_differences,
+    pin_dropout_varlen_numbering,
 ]

@@ -35,7 +35,21 @@ MUTATIONS = {
     "ds_sign_flipped": ("(dp[j] - rowsum)", "(rowsum - dp[j])"),
     "ds_rowsum_dropped": ("(dp[j] - rowsum)", "(dp[j])"),
     "dk_scale_dropped": ("dkj[c] += p->softmax_scale * ds * qi[c];", "dkj[c] += ds * qi[c];"),
-    "dv_operand_swapped": ("dvj[c] += pr[j] * doi[c];", "dvj[c] += pr[j] * qi[c];"),
+    "dv_operand_swapped": ("dvj[c] += pr[j] * zr[j] * doi[c];", "dvj[c] += pr[j] * zr[j] * qi[c];"),
+    "dropout_scale_dropped": ("return 256.0 / (256.0 - (double)p->dropout_threshold);",
+                              "return 1.0;"),
+    "dropout_dv_unmasked": ("dvj[c] += pr[j] * zr[j] * doi[c];", "dvj[c] += pr[j] * doi[c];"),
+    "dropout_dp_unmasked": ("? zr[j] * dot(doi, krow(p, v, b, j, g), d)",
+                            "? dot(doi, krow(p, v, b, j, g), d)"),
+    "dropout_threshold_inclusive": ("if (u < (uint32_t)p->dropout_threshold) return 0.0;",
+                                    "if (u <= (uint32_t)p->dropout_threshold) return 0.0;"),
+    "dropout_byte_from_row": ("(out[i & 3] >> (8 * (j & 3)))", "(out[j & 3] >> (8 * (i & 3)))"),
+    "dropout_head_ignored": ("(uint32_t)((p->batch_base + b) * p->nheads + h)",
+                             "(uint32_t)(p->batch_base + b)"),
+    "philox_key_not_advanced": ("    k0 += w0;\n", ""),
+    "philox_words_swapped": ("    x1 = (uint32_t)p1;\n    x3 = (uint32_t)p0;",
+                             "    x1 = (uint32_t)p0;\n    x3 = (uint32_t)p1;"),
+    "philox_nine_rounds": ("for (int r = 0; r < 10; ++r)", "for (int r = 0; r < 9; ++r)"),
     "dq_uses_values": ("dqi[c] += p->softmax_scale * ds * kj[c];",
                        "dqi[c] += p->softmax_scale * ds * krow(p, v, b, j, g)[c];"),
     "scores_wrong_head": ("const double *qi = qrow(p, q, b, i, h);\n  double mx",
