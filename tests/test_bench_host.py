@@ -151,3 +151,23 @@ def test_environment_is_best_effort():
 
     env = bench.environment(NoGpu, torch.device("cpu"))
     assert env["torch"] == "x" and "gpu" not in env
+
+
+def test_reference_arm_line(capsys):
+    """The reference arm runs the float64 oracle on the host and prints one
+    JSON line with the contract's keys (rank 0 of a single process)."""
+    for key in ("RANK", "WORLD_SIZE", "LOCAL_RANK"):
+        os.environ.pop(key, None)
+    assert bench.main(["--impl", "reference", "--steps", "1", "--warmup", "3"]) == 0
+    out = [ln for ln in capsys.readouterr().out.splitlines() if ln.startswith("{")]
+    assert len(out) == 1
+    line = json.loads(out[0])
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC
+    assert line["unit"] == bench.UNIT and line["value"] > 0 and line["steps"] == 1
+    assert line["higher_is_better"] is True and line["dtype"] == "f64"
+    assert line["config"]["workload"] == bench.WORKLOAD
+    cpu = line["cpu_baseline"]
+    assert cpu["kind"] == "oracle" and cpu["cores"] >= 1 and cpu["value"] == line["value"]
+    assert "queries" in cpu["sample"]
+    assert line["e2e"] == {"value": line["value"], "unit": bench.UNIT, "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
