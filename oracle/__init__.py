@@ -81,6 +81,11 @@ class Oracle:
         lib.oracle_philox4x32_10.restype = None
         lib.oracle_dropout_keep.argtypes = [P, ctypes.POINTER(ctypes.c_uint8)]
         lib.oracle_dropout_keep.restype = ctypes.c_int
+        lib.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
+        lib.oracle_e4m3_value.restype = ctypes.c_double
+        lib.oracle_e4m3_quantize.argtypes = [d, ctypes.c_int64, ctypes.c_double,
+                                             ctypes.POINTER(ctypes.c_uint8)]
+        lib.oracle_e4m3_quantize.restype = None
         lib.oracle_num_threads.restype = ctypes.c_int
         lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
         self.lib = lib
@@ -226,6 +231,20 @@ class Oracle:
             raise ValueError("oracle_dropout_keep rejected its arguments")
         return keep
 
+    def e4m3_quantize(self, x, scale=1.0):
+        """E4M3 codes (uint8, x's shape) of x / scale: round to nearest even,
+        saturating at +-448."""
+        xa = _f64(x)
+        codes = np.zeros(xa.shape, dtype=np.uint8)
+        self.lib.oracle_e4m3_quantize(_ptr(xa), ctypes.c_int64(xa.size), ctypes.c_double(scale),
+                                      codes.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)))
+        return codes
+
+    def e4m3_dequantize(self, codes, scale=1.0):
+        """float64 values scale * e4m3(code) of uint8 codes."""
+        table = np.array([self.lib.oracle_e4m3_value(c) for c in range(256)])
+        return table[np.asarray(codes, dtype=np.uint8)] * scale
+
     def attention_merge(self, o_parts, lse_parts):
         """Merge partial results over disjoint key sets: o_parts (S, B, Nq,
         H, d), lse_parts (S, B, H, Nq) -> O (B, Nq, H, d), LSE (B, H, Nq),
@@ -348,3 +367,11 @@ def philox4x32_10(*a, **kw):
 
 def dropout_keep(*a, **kw):
     return default().dropout_keep(*a, **kw)
+
+
+def e4m3_quantize(*a, **kw):
+    return default().e4m3_quantize(*a, **kw)
+
+
+def e4m3_dequantize(*a, **kw):
+    return default().e4m3_dequantize(*a, **kw)

@@ -504,3 +504,43 @@ int oracle_attn_merge(int64_t splits, int64_t B, int64_t Nq, int64_t H, int64_t 
   }
   return 0;
 }
+
+/*
+ * E4M3, the 8-bit float of FP8 attention (FlashAttention-3's FP8 forward,
+ * named on page 5's hardware/dtype section): sign bit, 4 exponent bits with
+ * bias 7, 3 mantissa bits.  Exponent field 0 holds subnormals m/8 * 2^-6;
+ * there are no infinities; S.1111.111 is NaN, so the largest finite value
+ * is 1.75 * 2^8 = 448.
+ */
+double oracle_e4m3_value(uint8_t c) {
+  const int s = c >> 7, e = (c >> 3) & 15, m = c & 7;
+  if (e == 15 && m == 7) return NAN;
+  const double mag = e == 0 ? ldexp(m / 8.0, -6) : ldexp(1.0 + m / 8.0, e - 7);
+  return s ? -mag : mag;
+}
+
+/* The code nearest to x among all finite codes of x's sign (a search over
+ * the table above); a tie goes to the code with an even mantissa (round to
+ * nearest even); magnitudes beyond 448 give +-448 (saturation), NaN gives
+ * 0x7F. */
+uint8_t oracle_e4m3_code(double x) {
+  if (isnan(x)) return 0x7F;
+  const uint8_t sign = signbit(x) ? 0x80 : 0x00;
+  const double a = fabs(x);
+  int best = 0;
+  double best_err = INFINITY;
+  for (int c = 0; c < 0x7F; ++c) {
+    const double err = fabs(oracle_e4m3_value((uint8_t)c) - a);
+    if (err < best_err || (err == best_err && (c & 1) == 0)) {
+      best = c;
+      best_err = err;
+    }
+  }
+  return (uint8_t)(sign | best);
+}
+
+/* codes[i] = e4m3 code of x[i] / scale (per-tensor scale: x ~ scale * code). */
+void oracle_e4m3_quantize(const double *x, int64_t n, double scale, uint8_t *codes) {
+#pragma omp parallel for schedule(static)
+  for (int64_t i = 0; i < n; ++i) codes[i] = oracle_e4m3_code(x[i] / scale);
+}

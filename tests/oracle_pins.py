@@ -666,6 +666,40 @@ def pin_dropout_varlen_numbering(orc):
         _close(a, b_.reshape(B * N, H, d), 1e-14, "varlen dropout " + n)
 
 
+# --- FP8 (E4M3) --------------------------------------------------------------
+
+def pin_e4m3_codec(orc):
+    """The oracle's E4M3 codec against torch's float8_e4m3fn (run, not read):
+    the value of every one of the 256 codes; the code of every finite bf16
+    number within +-448 and of every midpoint between neighbouring codes
+    (ties to the even mantissa); every finite code round-trips; beyond 448
+    the oracle saturates where torch gives NaN."""
+    codes = np.arange(256, dtype=np.uint8)
+    mine = orc.e4m3_dequantize(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).double().numpy()
+    assert np.array_equal(np.isnan(mine), np.isnan(ref))
+    fin = ~np.isnan(ref)
+    assert np.array_equal(mine[fin], ref[fin]), "E4M3 values"
+    assert np.array_equal(np.signbit(mine[fin]), np.signbit(ref[fin]))
+
+    def torch_codes(x32):
+        return x32.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+    bf = torch.arange(-32768, 32768, dtype=torch.int32).to(torch.int16).view(torch.bfloat16)
+    x = bf.float()
+    x = x[torch.isfinite(x) & (x.abs() <= 448)]
+    assert np.array_equal(orc.e4m3_quantize(x), torch_codes(x)), "E4M3 codes of bf16 values"
+    pos = mine[:0x7F]
+    mids = torch.tensor((pos[:-1] + pos[1:]) / 2, dtype=torch.float32)
+    for m in (mids, -mids):
+        assert np.array_equal(orc.e4m3_quantize(m), torch_codes(m)), "E4M3 ties"
+    assert np.array_equal(orc.e4m3_quantize(mine[fin]), codes[fin]), "E4M3 round trip"
+    sat = orc.e4m3_quantize(np.array([449.0, 464.0, 1e6, -500.0, np.inf]))
+    assert sat.tolist() == [0x7E, 0x7E, 0x7E, 0xFE, 0x7E], sat
+    scaled = orc.e4m3_quantize(np.array([3.0, -1.5]), scale=0.5)
+    assert scaled.tolist() == torch_codes(torch.tensor([6.0, -3.0])).tolist()
+
+
 ALL_PINS = [
     pin_golden_handworked,
     pin_identical_keys,
@@ -688,4 +722,5 @@ ALL_PINS = [
     pin_dropout_unbiased,
     pin_dropout_finite_differences,
     pin_dropout_varlen_numbering,
+    pin_e4m3_codec,
 ]

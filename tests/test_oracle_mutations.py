@@ -50,6 +50,9 @@ MUTATIONS = {
     "philox_words_swapped": ("    x1 = (uint32_t)p1;\n    x3 = (uint32_t)p0;",
                              "    x1 = (uint32_t)p0;\n    x3 = (uint32_t)p1;"),
     "philox_nine_rounds": ("for (int r = 0; r < 10; ++r)", "for (int r = 0; r < 9; ++r)"),
+    "e4m3_bias_off_by_one": ("ldexp(1.0 + m / 8.0, e - 7)", "ldexp(1.0 + m / 8.0, e - 8)"),
+    "e4m3_subnormal_scale": ("ldexp(m / 8.0, -6)", "ldexp(m / 8.0, -7)"),
+    "e4m3_ties_to_odd": ("(err == best_err && (c & 1) == 0)", "(err == best_err && (c & 1) == 1)"),
     "dq_uses_values": ("dqi[c] += p->softmax_scale * ds * kj[c];",
                        "dqi[c] += p->softmax_scale * ds * krow(p, v, b, j, g)[c];"),
     "scores_wrong_head": ("const double *qi = qrow(p, q, b, i, h);\n  double mx",
