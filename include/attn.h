@@ -107,6 +107,21 @@ typedef struct {
    * argument of the FlashAttention-2 interface; see the mask rules below for
    * the alignment).  Read by the kernels only. */
   const float* alibi_slopes;
+  /* Dropout on the attention probabilities (inverted dropout; 0 = none,
+   * the value a zero-initialised struct holds).  dropout_p in [0, 1): the
+   * applied rate is t / 256 with t = round(256 * dropout_p) <= 255, kept
+   * values are scaled by 256 / (256 - t), and P, the LSE and the row sums are
+   * those of the undropped scores.  The drop decision of score element
+   * (b, h, i, j) (batch or sequence b, query head h of H, query row i, key j)
+   * is fixed by the generator contract: Philox4x32-10 with key
+   * (dropout_seed low word, high word) at counter (j / 4, i / 4, b * H + h,
+   * dropout_offset); byte (j % 4) of output word (i % 4) is the element's
+   * random byte, dropped iff below t.  The backward pass must get the same
+   * seed and offset as the forward.  Forward with headdim 256 does not
+   * support dropout (ATTN_ERR_UNSUPPORTED_HEADDIM). */
+  float dropout_p;
+  uint32_t dropout_offset;
+  uint64_t dropout_seed;
 } attn_params;
 
 /*
@@ -216,6 +231,9 @@ typedef struct {
   int32_t window_left;
   int32_t window_right;
   const float* alibi_slopes;  /* as in attn_params; lengths per sequence */
+  float dropout_p;            /* as in attn_params; b = sequence index and */
+  uint32_t dropout_offset;    /* i, j positions within the sequence */
+  uint64_t dropout_seed;
 } attn_varlen_params;
 
 /* Host-side checks of a packed call (pass 0 forward, 1 backward): the

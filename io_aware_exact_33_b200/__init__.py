@@ -48,6 +48,9 @@ class AttnParams(ctypes.Structure):
         ("window_left", ctypes.c_int32),
         ("window_right", ctypes.c_int32),
         ("alibi_slopes", ctypes.c_void_p),
+        ("dropout_p", ctypes.c_float),
+        ("dropout_offset", ctypes.c_uint32),
+        ("dropout_seed", ctypes.c_uint64),
     ]
 
 
@@ -68,6 +71,9 @@ class AttnVarlenParams(ctypes.Structure):
         ("window_left", ctypes.c_int32),
         ("window_right", ctypes.c_int32),
         ("alibi_slopes", ctypes.c_void_p),
+        ("dropout_p", ctypes.c_float),
+        ("dropout_offset", ctypes.c_uint32),
+        ("dropout_seed", ctypes.c_uint64),
     ]
 
 
@@ -146,13 +152,15 @@ _lib = _Lazy()
 
 def make_params(batch, seqlen_q, seqlen_k, nheads, nheads_kv, headdim, dtype=ATTN_BF16,
                 softmax_scale=None, causal=False, window_left=-1, window_right=-1,
-                alibi_slopes=None) -> AttnParams:
+                alibi_slopes=None, dropout_p=0.0, dropout_seed=0, dropout_offset=0) -> AttnParams:
     """``alibi_slopes``: None, or the device address (int) of nheads float32
-    slopes."""
+    slopes.  Dropout: rate ``dropout_p`` (applied as round(256 p) / 256), the
+    generator's 64-bit seed and 32-bit offset (see include/attn.h)."""
     scale = 1.0 / math.sqrt(headdim) if softmax_scale is None else float(softmax_scale)
     return AttnParams(int(batch), int(seqlen_q), int(seqlen_k), int(nheads), int(nheads_kv),
                       int(headdim), int(dtype), scale, int(bool(causal)), int(window_left),
-                      int(window_right), alibi_slopes)
+                      int(window_right), alibi_slopes, float(dropout_p),
+                      int(dropout_offset) & 0xFFFFFFFF, int(dropout_seed) & (2 ** 64 - 1))
 
 
 def _slopes_ptr(alibi_slopes, nheads, device):
@@ -244,26 +252,31 @@ def _stream(stream):
 
 
 def params_for(q, k, softmax_scale=None, causal=False, window_left=-1, window_right=-1,
-               alibi_slopes=None):
+               alibi_slopes=None, dropout_p=0.0, dropout_seed=0, dropout_offset=0):
     B, Nq, H, d = q.shape
     Bk, Nk, Hkv, dk = k.shape
     if Bk != B or dk != d:
         raise ValueError("q and k disagree on batch or head dim")
     return make_params(B, Nq, Nk, H, Hkv, d, _dtype_code(q), softmax_scale, causal, window_left,
-                       window_right, _slopes_ptr(alibi_slopes, H, q.device))
+                       window_right, _slopes_ptr(alibi_slopes, H, q.device), dropout_p,
+                       dropout_seed, dropout_offset)
 
 
 def attn_fwd(q, k, v, softmax_scale: Optional[float] = None, causal: bool = False,
              window_left: int = -1, window_right: int = -1, out=None, lse=None,
-             stream=None, alibi_slopes=None) -> Tuple["torch.Tensor", "torch.Tensor"]:
+             stream=None, alibi_slopes=None, dropout_p: float = 0.0, dropout_seed: int = 0,
+             dropout_offset: int = 0) -> Tuple["torch.Tensor", "torch.Tensor"]:
     """O = softmax(q k^T * scale + bias + mask) v and the per-row natural-log LSE.
 
     q (B, Nq, H, d), k and v (B, Nk, Hkv, d), bf16 or fp16, contiguous CUDA
     tensors; ``alibi_slopes`` (optional, (H,) float32) adds
-    -slope_h * |i + Nk - Nq - j|.  Returns (out (B, Nq, H, d), lse (B, H, Nq)
-    float32)."""
+    -slope_h * |i + Nk - Nq - j|.  ``dropout_p`` > 0 drops attention
+    probabilities by the generator contract of include/attn.h (seed, offset);
+    the backward needs the same three values.  Returns (out (B, Nq, H, d),
+    lse (B, H, Nq) float32)."""
     import torch
-    p = params_for(q, k, softmax_scale, causal, window_left, window_right, alibi_slopes)
+    p = params_for(q, k, softmax_scale, causal, window_left, window_right, alibi_slopes,
+                   dropout_p, dropout_seed, dropout_offset)
     B, Nq, H, d = q.shape
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _check(t, n)
@@ -287,11 +300,13 @@ def attn_fwd(q, k, v, softmax_scale: Optional[float] = None, causal: bool = Fals
 
 def attn_bwd(q, k, v, out, lse, dout, softmax_scale: Optional[float] = None, causal: bool = False,
              window_left: int = -1, window_right: int = -1, dq=None, dk=None, dv=None,
-             workspace=None, stream=None, alibi_slopes=None):
+             workspace=None, stream=None, alibi_slopes=None, dropout_p: float = 0.0,
+             dropout_seed: int = 0, dropout_offset: int = 0):
     """Gradients (dq, dk, dv) of sum(out * dout) for attention with the same
     arguments as ``attn_fwd``; ``out`` and ``lse`` are its results."""
     import torch
-    p = params_for(q, k, softmax_scale, causal, window_left, window_right, alibi_slopes)
+    p = params_for(q, k, softmax_scale, causal, window_left, window_right, alibi_slopes,
+                   dropout_p, dropout_seed, dropout_offset)
     B, Nq, H, d = q.shape
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
         _check(t, n)
@@ -343,7 +358,8 @@ def attn_bwd_finalize(p: AttnParams, dq, workspace, stream=None) -> None:
 
 def attn_bwd_noalloc(q, k, v, out, lse, dout, softmax_scale: Optional[float] = None,
                      causal: bool = False, window_left: int = -1, window_right: int = -1,
-                     dq=None, dk=None, dv=None, stream=None, alibi_slopes=None):
+                     dq=None, dk=None, dv=None, stream=None, alibi_slopes=None,
+                     dropout_p: float = 0.0, dropout_seed: int = 0, dropout_offset: int = 0):
     """Like ``attn_bwd`` but the library uses its own fixed device scratch
     (ATTN_NOALLOC_SCRATCH_BYTES) instead of a caller workspace, for callers
     that cannot allocate device memory at call time.  The output tensors are
@@ -354,7 +370,8 @@ def attn_bwd_noalloc(q, k, v, out, lse, dout, softmax_scale: Optional[float] = N
     vp = ctypes.c_void_p
     fn.argtypes = [ctypes.POINTER(AttnParams), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     fn.restype = ctypes.c_int
-    p = params_for(q, k, softmax_scale, causal, window_left, window_right, alibi_slopes)
+    p = params_for(q, k, softmax_scale, causal, window_left, window_right, alibi_slopes,
+                   dropout_p, dropout_seed, dropout_offset)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
@@ -368,12 +385,14 @@ def attn_bwd_noalloc(q, k, v, out, lse, dout, softmax_scale: Optional[float] = N
 # ----------------------------------------------------------------- packed sequences
 def make_varlen_params(batch, total_q, total_k, max_seqlen_q, max_seqlen_k, nheads, nheads_kv,
                        headdim, dtype=ATTN_BF16, softmax_scale=None, causal=False,
-                       window_left=-1, window_right=-1, alibi_slopes=None) -> AttnVarlenParams:
+                       window_left=-1, window_right=-1, alibi_slopes=None, dropout_p=0.0,
+                       dropout_seed=0, dropout_offset=0) -> AttnVarlenParams:
     scale = 1.0 / math.sqrt(headdim) if softmax_scale is None else float(softmax_scale)
     return AttnVarlenParams(int(batch), int(total_q), int(total_k), int(max_seqlen_q),
                             int(max_seqlen_k), int(nheads), int(nheads_kv), int(headdim),
                             int(dtype), scale, int(bool(causal)), int(window_left),
-                            int(window_right), alibi_slopes)
+                            int(window_right), alibi_slopes, float(dropout_p),
+                            int(dropout_offset) & 0xFFFFFFFF, int(dropout_seed) & (2 ** 64 - 1))
 
 
 def attn_check_varlen_params(p: AttnVarlenParams, pass_: int = 0) -> int:
@@ -385,7 +404,8 @@ def attn_bwd_varlen_workspace_size(p: AttnVarlenParams) -> int:
 
 
 def _varlen_params(q, k, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, softmax_scale,
-                   causal, window_left, window_right, alibi_slopes=None):
+                   causal, window_left, window_right, alibi_slopes=None, dropout_p=0.0,
+                   dropout_seed=0, dropout_offset=0):
     import torch
     if q.dim() != 3 or k.dim() != 3:
         raise ValueError("packed q must be (total_q, nheads, d) and k (total_k, nheads_kv, d)")
@@ -401,13 +421,15 @@ def _varlen_params(q, k, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
         raise ValueError("cu_seqlens_q and cu_seqlens_k must both have batch + 1 entries")
     return make_varlen_params(cu_seqlens_q.numel() - 1, Tq, Tk, max_seqlen_q, max_seqlen_k, H, Hkv,
                               d, _dtype_code(q), softmax_scale, causal, window_left, window_right,
-                              _slopes_ptr(alibi_slopes, H, q.device))
+                              _slopes_ptr(alibi_slopes, H, q.device), dropout_p, dropout_seed,
+                              dropout_offset)
 
 
 def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int,
                     softmax_scale: Optional[float] = None, causal: bool = False,
                     window_left: int = -1, window_right: int = -1, out=None, lse=None,
-                    stream=None, alibi_slopes=None):
+                    stream=None, alibi_slopes=None, dropout_p: float = 0.0, dropout_seed: int = 0,
+                    dropout_offset: int = 0):
     """Attention over packed variable-length sequences.
 
     q (total_q, H, d), k and v (total_k, Hkv, d); sequence b owns rows
@@ -416,7 +438,8 @@ def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_
     (total_q, H, d), lse (H, total_q) float32)."""
     import torch
     p = _varlen_params(q, k, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
-                       softmax_scale, causal, window_left, window_right, alibi_slopes)
+                       softmax_scale, causal, window_left, window_right, alibi_slopes,
+                       dropout_p, dropout_seed, dropout_offset)
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _check(t, n)
         if t.dtype != q.dtype:
@@ -439,12 +462,14 @@ def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_
 def attn_bwd_varlen(q, k, v, out, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int,
                     max_seqlen_k: int, softmax_scale: Optional[float] = None,
                     causal: bool = False, window_left: int = -1, window_right: int = -1,
-                    dq=None, dk=None, dv=None, workspace=None, stream=None, alibi_slopes=None):
+                    dq=None, dk=None, dv=None, workspace=None, stream=None, alibi_slopes=None,
+                    dropout_p: float = 0.0, dropout_seed: int = 0, dropout_offset: int = 0):
     """Gradients (dq, dk, dv) of sum(out * dout) for ``attn_fwd_varlen`` with
     the same arguments; ``out`` and ``lse`` are its results."""
     import torch
     p = _varlen_params(q, k, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
-                       softmax_scale, causal, window_left, window_right, alibi_slopes)
+                       softmax_scale, causal, window_left, window_right, alibi_slopes,
+                       dropout_p, dropout_seed, dropout_offset)
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
         _check(t, n)
         if t.dtype != q.dtype:

@@ -169,18 +169,26 @@ struct Packed {
 
 // Kernel and grid width of a forward configuration: two query tiles per CTA
 // where both O tiles fit tensor memory (d <= 128), one otherwise.
+// The one-tile kernel (d = 256) has no dropout variant: attn_check_params
+// rejects dropout there before any launch.
 template <class C>
 struct FwdLaunch {
-  template <bool ALIBI>
+  template <bool ALIBI, bool DROP>
   static constexpr auto kernel() { return attn_fwd_kernel<C, ALIBI>; }
   static constexpr int rows_per_cta = C::BM;
 };
 template <int D, int KS, int VS, bool F>
 struct FwdLaunch<FwdPPCfg<D, KS, VS, F>> {
-  template <bool ALIBI>
-  static constexpr auto kernel() { return attn_fwd_pp_kernel<FwdPPCfg<D, KS, VS, F>, ALIBI>; }
+  template <bool ALIBI, bool DROP>
+  static constexpr auto kernel() {
+    return attn_fwd_pp_kernel<FwdPPCfg<D, KS, VS, F>, ALIBI, DROP>;
+  }
   static constexpr int rows_per_cta = 2 * FwdPPCfg<D, KS, VS, F>::BM;
 };
+
+// Dropout threshold t = round(256 p) of the contract in philox.cuh (0 = no
+// dropout); p has been checked to lie in [0, 255.5 / 256).
+uint32_t drop_threshold(float p) { return (uint32_t)std::floor(256.0 * (double)p + 0.5); }
 
 // Forward launch.  Dense: p->seqlen_q/k are the lengths.  Packed: p->batch
 // sequences of at most p->seqlen_q / p->seqlen_k rows each.
@@ -203,6 +211,11 @@ attn_status launch_fwd(const attn_params* p, const void* q, const void* k, const
   fp.total_k = pk.total_k;
   fp.o = static_cast<uint16_t*>(o);
   fp.alibi = p->alibi_slopes;
+  const uint32_t t = drop_threshold(p->dropout_p);
+  fp.drop_seed = p->dropout_seed;
+  fp.drop_offset = p->dropout_offset;
+  fp.drop_kadd = dropout_kadd(t);
+  fp.drop_scale = 256.f / (float)(256u - t);
   fp.lse = lse;
   fp.batch = p->batch;
   fp.nheads = p->nheads;
@@ -219,8 +232,10 @@ attn_status launch_fwd(const attn_params* p, const void* q, const void* k, const
   fp.sched_group = l2_group(4.0 * p->seqlen_k * C::D / (p->nheads / p->nheads_kv), heads);
   const long long blocks = (long long)fp.num_qblocks * heads;
   if (blocks > INT_MAX) return ATTN_ERR_INVALID_ARG;
-  auto kern = p->alibi_slopes ? FwdLaunch<C>::template kernel<true>()
-                              : FwdLaunch<C>::template kernel<false>();
+  auto kern = p->alibi_slopes ? (t ? FwdLaunch<C>::template kernel<true, true>()
+                                    : FwdLaunch<C>::template kernel<true, false>())
+                              : (t ? FwdLaunch<C>::template kernel<false, true>()
+                                   : FwdLaunch<C>::template kernel<false, false>());
   if (!ensure_smem(reinterpret_cast<const void*>(kern), C::SMEM_BYTES)) return ATTN_ERR_CUDA;
   kern<<<(unsigned)blocks, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mo, fp);
   return finish(stream);
@@ -241,6 +256,11 @@ BwdParams bwd_params(const attn_params* p, const float* lse, void* workspace, co
   bp.total_k = pk.total_k;
   bp.dk = bp.dv = nullptr;
   bp.alibi = p->alibi_slopes;
+  const uint32_t t = drop_threshold(p->dropout_p);
+  bp.drop_seed = p->dropout_seed;
+  bp.drop_offset = p->dropout_offset;
+  bp.drop_kadd = dropout_kadd(t);
+  bp.drop_scale = 256.f / (float)(256u - t);
   bp.num_kblocks = bp.sched_group = 0;
   bp.lse = lse;
   bp.dvec = reinterpret_cast<float*>(w + ws.dvec_off);
@@ -311,7 +331,9 @@ attn_status launch_bwd_main(const attn_params* p, const void* q, const void* k, 
   bpl.sched_group = l2_group(8.0 * p->seqlen_q * C::D * (p->nheads / p->nheads_kv), heads);
   const long long blocks = (long long)bpl.num_kblocks * heads;
   if (blocks > INT_MAX) return ATTN_ERR_INVALID_ARG;
-  auto kern = p->alibi_slopes ? attn_bwd_kernel<C, true> : attn_bwd_kernel<C, false>;
+  const bool drop = drop_threshold(p->dropout_p) != 0;
+  auto kern = p->alibi_slopes ? (drop ? attn_bwd_kernel<C, true, true> : attn_bwd_kernel<C, true, false>)
+                              : (drop ? attn_bwd_kernel<C, false, true> : attn_bwd_kernel<C, false, false>);
   if (!ensure_smem(reinterpret_cast<const void*>(kern), C::SMEM_BYTES)) return ATTN_ERR_CUDA;
   kern<<<(unsigned)blocks, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, ml, md, mdk,
                                                                  mdv, mdq, bpl);
@@ -425,6 +447,9 @@ attn_params packed_view(const attn_varlen_params* v) {
   p.window_left = v->window_left;
   p.window_right = v->window_right;
   p.alibi_slopes = v->alibi_slopes;
+  p.dropout_p = v->dropout_p;
+  p.dropout_offset = v->dropout_offset;
+  p.dropout_seed = v->dropout_seed;
   return p;
 }
 
@@ -483,6 +508,9 @@ attn_status attn_check_params(const attn_params* p, int pass) {
   if (p->causal != 0 && p->causal != 1) return ATTN_ERR_INVALID_ARG;
   if (p->window_left < -1 || p->window_right < -1) return ATTN_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(p->alibi_slopes) & 3u) return ATTN_ERR_MISALIGNED;
+  if (!(p->dropout_p >= 0.f) || !(p->dropout_p < 1.f) || drop_threshold(p->dropout_p) > 255u)
+    return ATTN_ERR_INVALID_ARG;
+  if (d == 256 && drop_threshold(p->dropout_p) != 0) return ATTN_ERR_UNSUPPORTED_HEADDIM;
   return ATTN_OK;
 }
 

@@ -111,6 +111,20 @@ def test_alibi_pointer_alignment(attn):
     assert attn.attn_check_params(p, 0) == 0
 
 
+def test_dropout_checks(attn):
+    """dropout_p must be in [0, 255.5 / 256) (its threshold round(256 p) at
+    most 255); the headdim-256 forward has no dropout variant, but a rate
+    that rounds to threshold 0 is no dropout and passes."""
+    assert attn.attn_check_params(P(attn, dropout_p=0.1, dropout_seed=7), 0) == 0
+    assert attn.attn_check_params(P(attn, dropout_p=0.1), 1) == 0
+    for bad in (-0.1, 1.0, 0.999, float("nan"), float("inf")):
+        assert attn.attn_check_params(P(attn, dropout_p=bad), 0) == 1, bad
+    assert attn.attn_check_params(P(attn, headdim=256, dropout_p=0.1), 0) == 2
+    assert attn.attn_check_params(P(attn, headdim=256, dropout_p=0.001), 0) == 0
+    v = attn.make_varlen_params(2, 10, 10, 5, 5, 4, 2, 64, dropout_p=1.5)
+    assert attn.attn_check_varlen_params(v, 0) == 1
+
+
 def test_merge_host_checks(attn):
     """attn_merge rejects bad sizes before touching the GPU; an empty merge
     is a no-op."""
@@ -136,6 +150,7 @@ def test_header_is_plain_c(attn, tmp_path):
         pytest.skip("no C compiler")
     src = tmp_path / "use_attn.c"
     src.write_text(r"""
+#include <stddef.h>
 #include <stdio.h>
 #include "attn.h"
 int main(void) {
@@ -148,6 +163,11 @@ int main(void) {
   printf("%d %d %d %zu %zu %s\n", (int)attn_check_params(&p, 0), (int)attn_check_params(&p, 1),
          (int)attn_check_varlen_params(&v, 1), attn_bwd_workspace_size(&p),
          attn_bwd_varlen_workspace_size(&v), attn_version());
+  printf("%zu %zu %zu %zu %zu %zu %zu %zu\n", sizeof(attn_params),
+         offsetof(attn_params, dropout_p), offsetof(attn_params, dropout_offset),
+         offsetof(attn_params, dropout_seed), sizeof(attn_varlen_params),
+         offsetof(attn_varlen_params, dropout_p), offsetof(attn_varlen_params, dropout_offset),
+         offsetof(attn_varlen_params, dropout_seed));
   return 0;
 }
 """)
@@ -158,6 +178,12 @@ int main(void) {
                     f"-Wl,-rpath,{libdir}"], check=True)
     out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()
     assert out[:3] == ["0", "0", "0"]
+    # the Python mirrors of the parameter structs have the C layout
+    layout = [int(x) for x in out[6:14]]
+    A, V = attn.AttnParams, attn.AttnVarlenParams
+    assert layout == [ctypes.sizeof(A), A.dropout_p.offset, A.dropout_offset.offset,
+                      A.dropout_seed.offset, ctypes.sizeof(V), V.dropout_p.offset,
+                      V.dropout_offset.offset, V.dropout_seed.offset]
     p = P(attn, batch=2, seqlen_q=100, seqlen_k=100, nheads=8, nheads_kv=2, headdim=128)
     assert int(out[3]) == attn.attn_bwd_workspace_size(p)
     assert int(out[4]) > 0 and out[5] == attn.attn_version()
