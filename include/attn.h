@@ -135,6 +135,22 @@ ATTN_API attn_status attn_fwd(const attn_params* p, const void* q, const void* k
                      float* lse, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Forward pass with E4M3 (FP8) inputs, the FP8 forward the pages name for
+ * FlashAttention-3.  q, k, v hold E4M3 codes, one byte per element, in the
+ * attn_fwd layouts; each tensor has one scale (element ~ scale *
+ * e4m3(code)), and the result is attention over those values:
+ * S = (q k^T) * q_scale * k_scale * softmax_scale, O = softmax(S) v * v_scale.
+ * o is written in p->dtype (bf16 or fp16), lse as attn_fwd's.  The kernel
+ * rounds P to E4M3 before the P V product (relative 2^-4).  Supported:
+ * headdim 128, causal and window masks, GQA; alibi_slopes must be NULL.
+ * Scales must be positive and finite (ATTN_ERR_INVALID_ARG).  Needs no
+ * workspace; asynchronous on `stream`.
+ */
+ATTN_API attn_status attn_fwd_e4m3(const attn_params* p, const void* q, const void* k,
+                                   const void* v, float q_scale, float k_scale, float v_scale,
+                                   void* o, float* lse, void* stream);
+
+/*
  * Backward pass: given dout = dL/dO and the forward's o and lse, writes
  * dq = dL/dQ, dk = dL/dK, dv = dL/dV (dk, dv summed over the query heads of
  * each kv group).  The score tiles are recomputed from q, k and lse.

@@ -30,6 +30,7 @@ EXPORTED = ("attn_fwd", "attn_bwd", "attn_bwd_prepare", "attn_bwd_accumulate", "
             "attn_fwd_workspace_size", "attn_bwd_workspace_size", "attn_check_params",
             "attn_status_string", "attn_get_device_status", "attn_version", "attn_bwd_noalloc",
             "attn_selftest_bounded_wait", "attn_check_varlen_params", "attn_fwd_varlen",
+            "attn_fwd_e4m3",
             "attn_bwd_varlen_workspace_size", "attn_bwd_varlen", "attn_merge")
 
 
@@ -295,6 +296,48 @@ def attn_fwd(q, k, v, softmax_scale: Optional[float] = None, causal: bool = Fals
                        _ptr(ws), ctypes.c_size_t(ws_bytes), _stream(stream))
     if st != 0:
         raise AttnError(st, "attn_fwd")
+    return out, lse
+
+
+def attn_fwd_e4m3(q, k, v, q_scale: float, k_scale: float, v_scale: float,
+                  softmax_scale: Optional[float] = None, causal: bool = False,
+                  window_left: int = -1, window_right: int = -1, out_dtype=None, out=None,
+                  lse=None, stream=None) -> Tuple["torch.Tensor", "torch.Tensor"]:
+    """Attention over E4M3 inputs: q (B, Nq, H, 128), k and v (B, Nk, Hkv,
+    128) hold E4M3 codes (uint8 or float8_e4m3fn CUDA tensors), element ~
+    scale * e4m3(code) with one scale per tensor.  Returns (out (B, Nq, H,
+    128) in ``out_dtype`` (bf16 by default, or fp16), lse (B, H, Nq)
+    float32)."""
+    import torch
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, n)
+        if t.element_size() != 1:
+            raise TypeError(f"{n} must hold one-byte E4M3 codes")
+    _check(v, "v", k.shape)
+    B, Nq, H, d = q.shape
+    Bk, Nk, Hkv, dk = k.shape
+    if Bk != B or dk != d:
+        raise ValueError("q and k disagree on batch or head dim")
+    out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
+    code = {torch.bfloat16: ATTN_BF16, torch.float16: ATTN_FP16}.get(out_dtype)
+    if code is None:
+        raise TypeError("out_dtype must be bfloat16 or float16")
+    p = make_params(B, Nq, Nk, H, Hkv, d, code, softmax_scale, causal, window_left, window_right)
+    if out is None:
+        out = torch.empty((B, Nq, H, d), dtype=out_dtype, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    _check(out, "out", (B, Nq, H, d))
+    _check(lse, "lse", (B, H, Nq))
+    fn = _lib.attn_fwd_e4m3
+    vp = ctypes.c_void_p
+    fn.argtypes = [ctypes.POINTER(AttnParams), vp, vp, vp, ctypes.c_float, ctypes.c_float,
+                   ctypes.c_float, vp, vp, vp]
+    fn.restype = ctypes.c_int
+    st = fn(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), float(q_scale), float(k_scale),
+            float(v_scale), _ptr(out), _ptr(lse), _stream(stream))
+    if st != 0:
+        raise AttnError(st, "attn_fwd_e4m3")
     return out, lse
 
 

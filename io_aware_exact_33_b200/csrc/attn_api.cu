@@ -13,6 +13,7 @@
 
 #include "attn.h"
 #include "bwd_kernel.cuh"
+#include "fwd_fp8_kernel.cuh"
 #include "fwd_kernel.cuh"
 #include "merge_kernel.cuh"
 #include "sm100.cuh"
@@ -57,6 +58,22 @@ bool map_bshd(CUtensorMap* m, const void* ptr, bool fp16, int batch, int seqlen,
                    const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// 8-bit (batch, seqlen, heads, 128) tensor of E4M3 codes as a 4-D map with a
+// box of 128 columns (one 128-byte swizzled row) x 1 head x `rows` rows.
+bool map_bshd_u8(CUtensorMap* m, const void* ptr, int batch, int seqlen, int heads, int d,
+                 int rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)seqlen, (cuuint64_t)batch};
+  cuuint64_t strides[3] = {(cuuint64_t)d, (cuuint64_t)heads * d, (cuuint64_t)seqlen * heads * d};
+  cuuint32_t box[4] = {128, 1, (cuuint32_t)rows, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(ptr), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -238,6 +255,42 @@ attn_status launch_fwd(const attn_params* p, const void* q, const void* k, const
                                    : FwdLaunch<C>::template kernel<false, false>());
   if (!ensure_smem(reinterpret_cast<const void*>(kern), C::SMEM_BYTES)) return ATTN_ERR_CUDA;
   kern<<<(unsigned)blocks, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mo, fp);
+  return finish(stream);
+}
+
+// Forward with E4M3 inputs (dense batches, d = 128).
+template <class C>
+attn_status launch_fwd_e4m3(const attn_params* p, const void* q, const void* k, const void* v,
+                            float q_scale, float k_scale, float v_scale, void* o, float* lse,
+                            cudaStream_t stream) {
+  CUtensorMap mq, mk, mv, mo;
+  if (!map_bshd_u8(&mq, q, p->batch, p->seqlen_q, p->nheads, C::D, C::BM) ||
+      !map_bshd_u8(&mk, k, p->batch, p->seqlen_k, p->nheads_kv, C::D, C::BN) ||
+      !map_bshd_u8(&mv, v, p->batch, p->seqlen_k, p->nheads_kv, C::D, C::BN) ||
+      !map_bshd(&mo, o, C::FP16, p->batch, p->seqlen_q, p->nheads, C::D, C::BM))
+    return ATTN_ERR_CUDA;
+  FwdParams fp;
+  std::memset(&fp, 0, sizeof(fp));
+  fp.o = static_cast<uint16_t*>(o);
+  fp.lse = lse;
+  fp.batch = p->batch;
+  fp.nheads = p->nheads;
+  fp.nheads_kv = p->nheads_kv;
+  fp.seqlen_q = p->seqlen_q;
+  fp.seqlen_k = p->seqlen_k;
+  fp.causal = p->causal;
+  fp.window_left = p->window_left;
+  fp.window_right = p->window_right;
+  fp.scale_log2 = p->softmax_scale * q_scale * k_scale * 1.4426950408889634f;
+  fp.num_qblocks = (p->seqlen_q + 2 * C::BM - 1) / (2 * C::BM);
+  const int heads = p->batch * p->nheads;
+  // K and V bytes (one per element) each query head streams
+  fp.sched_group = l2_group(2.0 * p->seqlen_k * C::D / (p->nheads / p->nheads_kv), heads);
+  const long long blocks = (long long)fp.num_qblocks * heads;
+  if (blocks > INT_MAX) return ATTN_ERR_INVALID_ARG;
+  auto kern = attn_fwd_e4m3_kernel<C>;
+  if (!ensure_smem(reinterpret_cast<const void*>(kern), C::SMEM_BYTES)) return ATTN_ERR_CUDA;
+  kern<<<(unsigned)blocks, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mo, fp, v_scale);
   return finish(stream);
 }
 
@@ -512,6 +565,34 @@ attn_status attn_check_params(const attn_params* p, int pass) {
     return ATTN_ERR_INVALID_ARG;
   if (d == 256 && drop_threshold(p->dropout_p) != 0) return ATTN_ERR_UNSUPPORTED_HEADDIM;
   return ATTN_OK;
+}
+
+attn_status attn_fwd_e4m3(const attn_params* p, const void* q, const void* k, const void* v,
+                          float q_scale, float k_scale, float v_scale, void* o, float* lse,
+                          void* stream_) {
+  attn_status st = attn_check_params(p, 0);
+  if (st != ATTN_OK) return st;
+  if (p->headdim != 128) return ATTN_ERR_UNSUPPORTED_HEADDIM;
+  if (p->alibi_slopes) return ATTN_ERR_INVALID_ARG;
+  for (float sc : {q_scale, k_scale, v_scale})
+    if (!(sc > 0.f) || !std::isfinite(sc)) return ATTN_ERR_INVALID_ARG;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (p->batch == 0 || p->seqlen_q == 0) return ATTN_OK;
+  if (!o || !lse) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(o) || (reinterpret_cast<uintptr_t>(lse) & 3u)) return ATTN_ERR_MISALIGNED;
+  if (p->seqlen_k == 0) {
+    const long long n_o = (long long)p->batch * p->seqlen_q * p->nheads * p->headdim;
+    const long long n_l = (long long)p->batch * p->nheads * p->seqlen_q;
+    fill_empty_fwd<<<fill_blocks(n_o), 256, 0, stream>>>(static_cast<uint16_t*>(o), n_o, lse, n_l);
+    return finish(stream);
+  }
+  if (!q || !k || !v) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return ATTN_ERR_MISALIGNED;
+  return p->dtype == ATTN_FP16
+             ? launch_fwd_e4m3<FwdF8Cfg<3, 2, true>>(p, q, k, v, q_scale, k_scale, v_scale, o, lse,
+                                                     stream)
+             : launch_fwd_e4m3<FwdF8Cfg<3, 2, false>>(p, q, k, v, q_scale, k_scale, v_scale, o,
+                                                      lse, stream);
 }
 
 size_t attn_fwd_workspace_size(const attn_params* p) {
