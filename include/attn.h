@@ -142,13 +142,31 @@ ATTN_API attn_status attn_fwd(const attn_params* p, const void* q, const void* k
  * S = (q k^T) * q_scale * k_scale * softmax_scale, O = softmax(S) v * v_scale.
  * o is written in p->dtype (bf16 or fp16), lse as attn_fwd's.  The kernel
  * rounds P to E4M3 before the P V product (relative 2^-4).  Supported:
- * headdim 128, causal and window masks, GQA; alibi_slopes must be NULL.
+ * headdim 128, causal and window masks, GQA; alibi_slopes must be NULL
+ * and dropout_p 0.
  * Scales must be positive and finite (ATTN_ERR_INVALID_ARG).  Needs no
  * workspace; asynchronous on `stream`.
  */
 ATTN_API attn_status attn_fwd_e4m3(const attn_params* p, const void* q, const void* k,
                                    const void* v, float q_scale, float k_scale, float v_scale,
                                    void* o, float* lse, void* stream);
+
+/*
+ * Forward pass for decoding: a few query rows per sequence against a long
+ * key / value sequence (a cache), with the same arguments, layouts, masks
+ * (bottom-right aligned) and results as attn_fwd.  The keys are split over
+ * blocks of the CUDA cores (the work is bound by reading K and V; every kv
+ * head's K and V rows are read once for all the query heads of its group)
+ * and the splits' partial results are merged as attn_merge does.
+ * Supported: headdim 64 or 128, (nheads / nheads_kv) * seqlen_q <= 16,
+ * no positional slopes and no dropout (ATTN_ERR_INVALID_ARG otherwise).  workspace: at
+ * least attn_fwd_decode_workspace_size(p) bytes, 256-byte aligned, caller-
+ * owned, overwritten.  Asynchronous on `stream`.
+ */
+ATTN_API size_t attn_fwd_decode_workspace_size(const attn_params* p);
+ATTN_API attn_status attn_fwd_decode(const attn_params* p, const void* q, const void* k,
+                                     const void* v, void* o, float* lse, void* workspace,
+                                     size_t workspace_bytes, void* stream);
 
 /*
  * Backward pass: given dout = dL/dO and the forward's o and lse, writes

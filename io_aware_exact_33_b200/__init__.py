@@ -30,7 +30,7 @@ EXPORTED = ("attn_fwd", "attn_bwd", "attn_bwd_prepare", "attn_bwd_accumulate", "
             "attn_fwd_workspace_size", "attn_bwd_workspace_size", "attn_check_params",
             "attn_status_string", "attn_get_device_status", "attn_version", "attn_bwd_noalloc",
             "attn_selftest_bounded_wait", "attn_check_varlen_params", "attn_fwd_varlen",
-            "attn_fwd_e4m3",
+            "attn_fwd_e4m3", "attn_fwd_decode", "attn_fwd_decode_workspace_size",
             "attn_bwd_varlen_workspace_size", "attn_bwd_varlen", "attn_merge")
 
 
@@ -338,6 +338,42 @@ def attn_fwd_e4m3(q, k, v, q_scale: float, k_scale: float, v_scale: float,
             float(v_scale), _ptr(out), _ptr(lse), _stream(stream))
     if st != 0:
         raise AttnError(st, "attn_fwd_e4m3")
+    return out, lse
+
+
+def attn_fwd_decode(q, k, v, softmax_scale: Optional[float] = None, causal: bool = False,
+                    window_left: int = -1, window_right: int = -1, out=None, lse=None,
+                    workspace=None, stream=None) -> Tuple["torch.Tensor", "torch.Tensor"]:
+    """``attn_fwd`` for decoding: a few query rows ((H / Hkv) * Nq <= 16)
+    against a long key / value sequence, on the CUDA cores with the keys
+    split over blocks.  Same arguments, layouts and results as ``attn_fwd``
+    (no positional slopes)."""
+    import torch
+    p = params_for(q, k, softmax_scale, causal, window_left, window_right)
+    B, Nq, H, d = q.shape
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, n)
+        if t.dtype != q.dtype:
+            raise TypeError("q, k, v must share a dtype")
+    _check(v, "v", k.shape)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device) if lse is None else lse
+    _check(out, "out", q.shape)
+    _check(lse, "lse", (B, H, Nq))
+    fn = _lib.attn_fwd_decode_workspace_size
+    fn.argtypes = [ctypes.POINTER(AttnParams)]
+    fn.restype = ctypes.c_size_t
+    ws_bytes = int(fn(ctypes.byref(p)))
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
+    vp = ctypes.c_void_p
+    call = _lib.attn_fwd_decode
+    call.argtypes = [ctypes.POINTER(AttnParams), vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
+    call.restype = ctypes.c_int
+    st = call(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(workspace),
+              ctypes.c_size_t(workspace.numel()), _stream(stream))
+    if st != 0:
+        raise AttnError(st, "attn_fwd_decode")
     return out, lse
 
 

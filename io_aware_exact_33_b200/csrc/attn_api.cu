@@ -13,6 +13,7 @@
 
 #include "attn.h"
 #include "bwd_kernel.cuh"
+#include "decode_kernel.cuh"
 #include "fwd_fp8_kernel.cuh"
 #include "fwd_kernel.cuh"
 #include "merge_kernel.cuh"
@@ -294,6 +295,62 @@ attn_status launch_fwd_e4m3(const attn_params* p, const void* q, const void* k, 
   return finish(stream);
 }
 
+// Key splits of a decode call: about two blocks per SM over the
+// (batch, kv head) pairs, at least 256 keys per split.
+int decode_splits(const attn_params* p) {
+  const long long groups = (long long)p->batch * p->nheads_kv;
+  long long want = (2 * 148 + groups - 1) / groups;
+  const long long by_len = ((long long)p->seqlen_k + 255) / 256;
+  if (want > by_len) want = by_len;
+  if (want > 65535) want = 65535;
+  return (int)(want < 1 ? 1 : want);
+}
+
+// Workspace of a decode call: the splits' 16-bit partial outputs, then
+// their LSE values.
+struct DecodeWorkspace {
+  size_t o_bytes, total;
+};
+DecodeWorkspace decode_layout(const attn_params* p) {
+  const size_t rows = (size_t)decode_splits(p) * p->batch * p->seqlen_q * p->nheads;
+  DecodeWorkspace w;
+  w.o_bytes = (rows * p->headdim * 2 + 255) / 256 * 256;
+  w.total = w.o_bytes + (rows * 4 + 255) / 256 * 256;
+  return w;
+}
+
+template <int D, bool FP16>
+attn_status launch_decode(const attn_params* p, const void* q, const void* k, const void* v,
+                          void* o, float* lse, void* workspace, cudaStream_t stream) {
+  const int splits = decode_splits(p);
+  const DecodeWorkspace ws = decode_layout(p);
+  DecodeParams dp;
+  dp.q = static_cast<const uint16_t*>(q);
+  dp.k = static_cast<const uint16_t*>(k);
+  dp.v = static_cast<const uint16_t*>(v);
+  dp.o_parts = static_cast<uint16_t*>(workspace);
+  dp.lse_parts = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + ws.o_bytes);
+  dp.batch = p->batch;
+  dp.nheads = p->nheads;
+  dp.nheads_kv = p->nheads_kv;
+  dp.seqlen_q = p->seqlen_q;
+  dp.seqlen_k = p->seqlen_k;
+  dp.causal = p->causal;
+  dp.window_left = p->window_left;
+  dp.window_right = p->window_right;
+  dp.scale_log2 = p->softmax_scale * 1.4426950408889634f;
+  dp.splits = splits;
+  dp.chunk = (int)((((long long)p->seqlen_k + splits - 1) / splits + 31) / 32 * 32);
+  auto kern = attn_decode_kernel<D, FP16>;
+  if (!ensure_smem(reinterpret_cast<const void*>(kern), DecodeSmem<D>::BYTES)) return ATTN_ERR_CUDA;
+  const dim3 grid((unsigned)splits, (unsigned)(p->batch * p->nheads_kv));
+  kern<<<grid, kDecodeWarps * 32, DecodeSmem<D>::BYTES, stream>>>(dp);
+  const attn_status st = finish(stream);
+  if (st != ATTN_OK) return st;
+  const attn_merge_params mp = {splits, p->batch, p->seqlen_q, p->nheads, p->headdim, p->dtype};
+  return attn_merge(&mp, dp.o_parts, dp.lse_parts, o, lse, stream);
+}
+
 BwdWorkspace bwd_layout(const attn_params* p, const Packed& pk) {
   return pk.on() ? bwd_workspace_layout_packed(pk.total_q, p->batch, p->nheads, p->headdim)
                  : bwd_workspace_layout(p->batch, p->nheads, p->seqlen_q, p->headdim);
@@ -573,7 +630,7 @@ attn_status attn_fwd_e4m3(const attn_params* p, const void* q, const void* k, co
   attn_status st = attn_check_params(p, 0);
   if (st != ATTN_OK) return st;
   if (p->headdim != 128) return ATTN_ERR_UNSUPPORTED_HEADDIM;
-  if (p->alibi_slopes) return ATTN_ERR_INVALID_ARG;
+  if (p->alibi_slopes || drop_threshold(p->dropout_p) != 0) return ATTN_ERR_INVALID_ARG;
   for (float sc : {q_scale, k_scale, v_scale})
     if (!(sc > 0.f) || !std::isfinite(sc)) return ATTN_ERR_INVALID_ARG;
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
@@ -593,6 +650,41 @@ attn_status attn_fwd_e4m3(const attn_params* p, const void* q, const void* k, co
                                                      stream)
              : launch_fwd_e4m3<FwdF8Cfg<3, 2, false>>(p, q, k, v, q_scale, k_scale, v_scale, o,
                                                       lse, stream);
+}
+
+size_t attn_fwd_decode_workspace_size(const attn_params* p) {
+  if (attn_check_params(p, 0) != ATTN_OK) return 0;
+  return decode_layout(p).total;
+}
+
+attn_status attn_fwd_decode(const attn_params* p, const void* q, const void* k, const void* v,
+                            void* o, float* lse, void* workspace, size_t workspace_bytes,
+                            void* stream_) {
+  attn_status st = attn_check_params(p, 0);
+  if (st != ATTN_OK) return st;
+  if (p->headdim != 64 && p->headdim != 128) return ATTN_ERR_UNSUPPORTED_HEADDIM;
+  if (p->alibi_slopes || drop_threshold(p->dropout_p) != 0) return ATTN_ERR_INVALID_ARG;
+  if ((long long)(p->nheads / p->nheads_kv) * p->seqlen_q > kDecodeRows) return ATTN_ERR_INVALID_ARG;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (p->batch == 0 || p->seqlen_q == 0) return ATTN_OK;
+  if (!o || !lse) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(o) || (reinterpret_cast<uintptr_t>(lse) & 3u)) return ATTN_ERR_MISALIGNED;
+  if (p->seqlen_k == 0) {
+    const long long n_o = (long long)p->batch * p->seqlen_q * p->nheads * p->headdim;
+    const long long n_l = (long long)p->batch * p->nheads * p->seqlen_q;
+    fill_empty_fwd<<<fill_blocks(n_o), 256, 0, stream>>>(static_cast<uint16_t*>(o), n_o, lse, n_l);
+    return finish(stream);
+  }
+  if (!q || !k || !v || !workspace) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return ATTN_ERR_MISALIGNED;
+  if (workspace_bytes < decode_layout(p).total) return ATTN_ERR_WORKSPACE_TOO_SMALL;
+  const bool fp16 = p->dtype == ATTN_FP16;
+  if (p->headdim == 64)
+    return fp16 ? launch_decode<64, true>(p, q, k, v, o, lse, workspace, stream)
+                : launch_decode<64, false>(p, q, k, v, o, lse, workspace, stream);
+  return fp16 ? launch_decode<128, true>(p, q, k, v, o, lse, workspace, stream)
+              : launch_decode<128, false>(p, q, k, v, o, lse, workspace, stream);
 }
 
 size_t attn_fwd_workspace_size(const attn_params* p) {

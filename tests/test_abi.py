@@ -187,3 +187,28 @@ int main(void) {
     p = P(attn, batch=2, seqlen_q=100, seqlen_k=100, nheads=8, nheads_kv=2, headdim=128)
     assert int(out[3]) == attn.attn_bwd_workspace_size(p)
     assert int(out[4]) > 0 and out[5] == attn.attn_version()
+
+
+def test_decode_host_checks(attn):
+    """attn_fwd_decode's workspace follows its split rule (about two blocks
+    per SM over the (batch, kv head) pairs, at least 256 keys per split) and
+    it refuses, before touching any pointer, more than 16 query rows per kv
+    head, head dim 256 and positional slopes."""
+    fn = attn._lib.attn_fwd_decode_workspace_size
+    fn.argtypes = [ctypes.POINTER(attn.AttnParams)]
+    fn.restype = ctypes.c_size_t
+    p = P(attn, batch=2, seqlen_q=1, seqlen_k=5000, nheads=32, nheads_kv=4)
+    splits = min(-(-296 // 8), -(-5000 // 256))  # 20
+    rows = splits * 2 * 1 * 32
+    assert fn(ctypes.byref(p)) == -(-rows * 128 * 2 // 256) * 256 + -(-rows * 4 // 256) * 256
+    call = attn._lib.attn_fwd_decode
+    vp = ctypes.c_void_p
+    call.argtypes = [ctypes.POINTER(attn.AttnParams), vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
+    call.restype = ctypes.c_int
+    too_many = P(attn, seqlen_q=5, nheads=8, nheads_kv=2)  # 4 heads x 5 tokens = 20 rows
+    assert call(ctypes.byref(too_many), None, None, None, None, None, None, 0, None) == 1
+    assert call(ctypes.byref(P(attn, headdim=256)), None, None, None, None, None, None, 0,
+                None) == 2
+    slopes = P(attn, seqlen_q=1)
+    slopes.alibi_slopes = 256
+    assert call(ctypes.byref(slopes), None, None, None, None, None, None, 0, None) == 1
