@@ -173,7 +173,9 @@ def _ring_rank(rank, world, store_path, w, layout, queue):
         near = lambda a, b: torch.allclose(a.float(), b.float(), rtol=2 ** -7, atol=2 ** -12)
         same = (torch.equal(out.detach(), o) and near(ql.grad, dq) and near(kl.grad, dk) and
                 near(vl.grad, dv))
-        queue.put((rank, o, lse, dq, dk, dv, same))
+        # plain arrays, pickled by value: a tensor would travel through shared
+        # memory that needs this process alive until the parent has it
+        queue.put((rank, *(t.float().numpy() for t in (o, lse, dq, dk, dv)), same))
     finally:
         dist.destroy_process_group()
 
@@ -191,7 +193,9 @@ def _run_ring(world, w, layout, tmp_path):
     for p in procs:
         p.join(60)
         assert p.exitcode == 0, f"rank exit code {p.exitcode}"
-    return res
+    bf = lambda a: torch.from_numpy(a).to(torch.bfloat16)
+    return [(r, bf(o), torch.from_numpy(lse), bf(dq), bf(dk), bf(dv), same)
+            for r, o, lse, dq, dk, dv, same in res]
 
 
 def _compare_whole(res, w, layout, what):
