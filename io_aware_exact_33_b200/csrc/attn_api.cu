@@ -343,7 +343,7 @@ attn_status launch_decode(const attn_params* p, const void* q, const void* k, co
   dp.chunk = (int)((((long long)p->seqlen_k + splits - 1) / splits + 31) / 32 * 32);
   auto kern = attn_decode_kernel<D, FP16>;
   if (!ensure_smem(reinterpret_cast<const void*>(kern), DecodeSmem<D>::BYTES)) return ATTN_ERR_CUDA;
-  const dim3 grid((unsigned)splits, (unsigned)(p->batch * p->nheads_kv));
+  const dim3 grid((unsigned)(p->batch * p->nheads_kv), (unsigned)splits);  // splits <= 65535
   kern<<<grid, kDecodeWarps * 32, DecodeSmem<D>::BYTES, stream>>>(dp);
   const attn_status st = finish(stream);
   if (st != ATTN_OK) return st;

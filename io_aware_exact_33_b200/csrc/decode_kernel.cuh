@@ -70,7 +70,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) attn_decode_kernel(const De
   float* os = ps + S::P;
   float* mls = os + S::O;
 
-  const int split = blockIdx.x, bk = blockIdx.y;
+  const int split = blockIdx.y, bk = blockIdx.x;  // x: (batch, kv head), up to 2^31 - 1
   const int b = bk / p.nheads_kv, kvh = bk % p.nheads_kv;
   const int G = p.nheads / p.nheads_kv, Nq = p.seqlen_q, R = G * Nq;  // row r = g * Nq + i
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
