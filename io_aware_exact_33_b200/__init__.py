@@ -107,6 +107,8 @@ def _load() -> ctypes.CDLL:
     lib.attn_bwd_accumulate.restype = ctypes.c_int
     lib.attn_bwd_finalize.argtypes = [P, vp, vp, sz, vp]
     lib.attn_bwd_finalize.restype = ctypes.c_int
+    lib.attn_bwd_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.attn_bwd_noalloc.restype = ctypes.c_int
     lib.attn_fwd_workspace_size.argtypes = [P]
     lib.attn_fwd_workspace_size.restype = sz
     lib.attn_bwd_workspace_size.argtypes = [P]
@@ -445,17 +447,13 @@ def attn_bwd_noalloc(q, k, v, out, lse, dout, softmax_scale: Optional[float] = N
     the caller's (allocated here only when not given).  Calls that overlap on
     the GPU share that scratch and must be serialised by the caller."""
     import torch
-    fn = _lib.attn_bwd_noalloc
-    vp = ctypes.c_void_p
-    fn.argtypes = [ctypes.POINTER(AttnParams), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
-    fn.restype = ctypes.c_int
     p = params_for(q, k, softmax_scale, causal, window_left, window_right, alibi_slopes,
                    dropout_p, dropout_seed, dropout_offset)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
-    st = fn(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq),
-            _ptr(dk), _ptr(dv), _stream(stream))
+    st = _lib.attn_bwd_noalloc(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                               _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _stream(stream))
     if st != 0:
         raise AttnError(st, "attn_bwd_noalloc")
     return dq, dk, dv
