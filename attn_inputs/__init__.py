@@ -70,6 +70,19 @@ WORKLOADS: Dict[str, Workload] = {
 }
 
 
+# Workloads of the extra entry points (decode on the CUDA cores, FP8 forward):
+# the decode case is 8 sequences each with one new query token against a
+# 32,768-token key/value cache (GQA 32/8); the FP8 case is the headline
+# causal shape, forward only, its inputs rounded to E4M3 with one scale per
+# tensor.
+EXTRA_WORKLOADS: Dict[str, Workload] = {
+    "decode_b8_h32_kv8_n32768_d128": Workload(
+        "decode_b8_h32_kv8_n32768_d128", 8, 32, 8, 1, 32768, 128, True, seed=12, passes="fwd"),
+    "fp8_causal_b2_h32_n8192_d128": Workload(
+        "fp8_causal_b2_h32_n8192_d128", 2, 32, 32, 8192, 8192, 128, True, seed=13, passes="fwd"),
+}
+
+
 @dataclasses.dataclass(frozen=True)
 class VarlenWorkload:
     """Packed variable-length sequences: per-sequence query and key lengths

@@ -23,6 +23,7 @@ workload (rank 0 only).
 from __future__ import annotations
 
 import argparse
+import ctypes
 import datetime
 import hashlib
 import json
@@ -707,6 +708,128 @@ def run_gpu_varlen(args, w):
     return 0
 
 
+# ---------------------------------------------------------------- extra entry points
+def run_gpu_extra(args, w):
+    """The decode path (CUDA cores, HBM-bound: GB/s of K, V, Q read and O, LSE
+    written, against the measured copy bandwidth) or the FP8 forward (TFLOP/s
+    of the exact visible pairs against the measured bf16 peak times the
+    nominal FP8 / BF16 ratio of 2).  Inputs resident in HBM; every step
+    reads more than the L2 holds."""
+    import torch
+    import io_aware_exact_33_b200 as attn
+    from attn_inputs import make_inputs
+
+    rank, local_rank, world = world_info()
+    dist = init_dist("nccl", world)
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    decode = w.name.startswith("decode")
+    q, k, v, _ = make_inputs(w, with_dout=False)
+    pairs = visible_pairs(w.seqlen_q, w.seqlen_k, w.causal, w.window_left, w.window_right)
+    flops = 4.0 * w.batch * w.nheads * w.headdim * pairs
+    o = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.batch, w.nheads, w.seqlen_q), dtype=torch.float32, device=dev)
+    mask = (w.scale, w.causal, w.window_left, w.window_right)
+    if decode:
+        qd, kd, vd = (t.to(dev) for t in (q, k, v))
+        p = attn.params_for(qd, kd, w.scale, w.causal, w.window_left, w.window_right)
+        fn = attn._lib.attn_fwd_decode_workspace_size
+        fn.argtypes = [ctypes.POINTER(attn.AttnParams)]
+        fn.restype = ctypes.c_size_t
+        ws = torch.empty(max(int(fn(ctypes.byref(p))), 1), dtype=torch.uint8, device=dev)
+
+        def call(qx):
+            attn.attn_fwd_decode(qx, kd, vd, *mask, out=o, lse=lse, workspace=ws)
+        launches, qdev, host_q = 2, qd, q.pin_memory()
+        alg_bytes = sum(t.numel() * t.element_size() for t in (q, k, v)) + 2 * o.numel() + 4 * lse.numel()
+    else:
+        scales = [float(t.double().abs().max()) / 448.0 for t in (q, k, v)]
+        q8, k8, v8 = ((t.float() / sc).to(torch.float8_e4m3fn) for t, sc in zip((q, k, v), scales))
+        qd8, kd8, vd8 = (t.to(dev) for t in (q8, k8, v8))
+
+        def call(qx):
+            attn.attn_fwd_e4m3(qx, kd8, vd8, *scales, *mask, out=o, lse=lse)
+        launches, qdev, host_q = 1, qd8, q8.pin_memory()
+        alg_bytes = sum(t.numel() for t in (q8, k8, v8)) + 2 * o.numel() + 4 * lse.numel()
+    stream = torch.cuda.current_stream(dev)
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    for _ in range(args.warmup):
+        call(qdev)
+    torch.cuda.synchronize(dev)
+    if attn.attn_get_device_status() != 0:
+        raise RuntimeError("device status word reports an error after warm-up")
+    gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(dist, dev)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(gpu_id) as clk:
+        start.record(stream)
+        for i in range(args.steps):
+            events[i][0].record(stream)
+            call(qdev)
+            events[i][1].record(stream)
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(dist, dev)
+    ms = max_over_ranks(start.elapsed_time(end), dist, dev)
+    ms_call = sum(e[0].elapsed_time(e[1]) for e in events) / args.steps
+    # end to end: the step's queries up from pinned host memory (the K / V
+    # operands stay resident, as a cache or weights-like inputs would), the
+    # output down
+    host_o = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    k_e2e = max(1, min(args.steps, args.e2e_steps))
+    barrier(dist, dev)
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record(stream)
+    for _ in range(k_e2e):
+        qdev.copy_(host_q, non_blocking=True)
+        call(qdev)
+        host_o.copy_(o, non_blocking=True)
+    e2.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(dist, dev)
+    ms_e2e = max_over_ranks(s2.elapsed_time(e2), dist, dev)
+    status = attn.attn_get_device_status()
+    if rank != 0:
+        if dist is not None:
+            dist.destroy_process_group()
+        return 0
+    peaks, peak_kind = load_peaks()
+    if decode:
+        unit, value = "GB/s", alg_bytes * args.steps * world / (ms / 1e3) / 1e9
+        achieved = alg_bytes / (ms_call / 1e3) / 1e9
+        rl = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": unit,
+              "frac": achieved / peaks["hbm_gbs"], "traffic": None, "kernel": "attn_fwd_decode",
+              "peak_source": f"hbm_gbs of {peak_kind}", "bytes_per_launch": alg_bytes}
+        metric, e2e_value = "decode attention HBM GB/s", alg_bytes * k_e2e * world / (ms_e2e / 1e3) / 1e9
+    else:
+        unit, value = UNIT, flops * args.steps * world / (ms / 1e3) / 1e12
+        achieved = flops / (ms_call / 1e3) / 1e12
+        peak = 2.0 * peaks["bf16_tflops"]
+        rl = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": unit,
+              "frac": achieved / peak, "traffic": None, "kernel": "attn_fwd_e4m3_kernel",
+              "peak_source": f"2 x bf16_tflops (burst) of {peak_kind}: the nominal FP8/BF16 ratio",
+              "flops_per_launch": flops}
+        metric, e2e_value = "FP8 (E4M3) attention forward TFLOP/s", flops * k_e2e * world / (ms_e2e / 1e3) / 1e12
+    cfg = workload_config(w)
+    cfg["l2"] = f"no flush: {alg_bytes / 1e9:.2f} GB read and written per step exceed the 126 MB L2"
+    line = {
+        "metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3" if not decode else w.dtype,
+        "data": f"synthetic ({cfg['inputs']})", "config": cfg, "roofline": rl,
+        "cpu_baseline": None,
+        "e2e": {"value": e2e_value, "unit": unit, "steps": k_e2e,
+                "h2d_bytes_per_step": host_q.numel() * host_q.element_size(),
+                "d2h_bytes_per_step": host_o.numel() * host_o.element_size()},
+        "clocks": clk.summary(), "gpu_launches": launches * args.steps, "device_status": status,
+    }
+    print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
 PROBE_CASES = [  # (description, M, N) in the order of probe_mma_case()
     ("A smem K-major, B smem K-major, 1 accumulator", 128, 128),
     ("A smem K-major, B smem K-major, 2 accumulators", 128, 128),
@@ -769,7 +892,13 @@ def main(argv=None):
         return 0
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
-    from attn_inputs import VARLEN_WORKLOADS, WORKLOADS
+    from attn_inputs import EXTRA_WORKLOADS, VARLEN_WORKLOADS, WORKLOADS
+    if args.workload in EXTRA_WORKLOADS:
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable":
+                              "the reference arm times the dense headline workload only"}))
+            return 0
+        return run_gpu_extra(args, EXTRA_WORKLOADS[args.workload])
     if args.workload in VARLEN_WORKLOADS:
         if args.impl == "reference":
             print(json.dumps({"impl": "reference", "unavailable":
@@ -778,7 +907,7 @@ def main(argv=None):
         return run_gpu_varlen(args, VARLEN_WORKLOADS[args.workload])
     if args.workload not in WORKLOADS:
         ap.error(f"unknown workload {args.workload}; choose from "
-                 f"{sorted(WORKLOADS) + sorted(VARLEN_WORKLOADS)}")
+                 f"{sorted(WORKLOADS) + sorted(VARLEN_WORKLOADS) + sorted(EXTRA_WORKLOADS)}")
     if input_bytes(WORKLOADS[args.workload]) < 2 * 126e6:
         ap.error(f"{args.workload} fits in L2; it is a parity case, not a bench workload")
     if args.impl == "reference":

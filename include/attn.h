@@ -107,6 +107,21 @@ typedef struct {
    * argument of the FlashAttention-2 interface; see the mask rules below for
    * the alignment).  Read by the kernels only. */
   const float* alibi_slopes;
+  /* Dropout on the attention probabilities (inverted dropout; 0 = none,
+   * the value a zero-initialised struct holds).  dropout_p in [0, 1): the
+   * applied rate is t / 256 with t = round(256 * dropout_p) <= 255, kept
+   * values are scaled by 256 / (256 - t), and P, the LSE and the row sums are
+   * those of the undropped scores.  The drop decision of score element
+   * (b, h, i, j) (batch or sequence b, query head h of H, query row i, key j)
+   * is fixed by the generator contract: Philox4x32-10 with key
+   * (dropout_seed low word, high word) at counter (j / 4, i / 4, b * H + h,
+   * dropout_offset); byte (j % 4) of output word (i % 4) is the element's
+   * random byte, dropped iff below t.  The backward pass must get the same
+   * seed and offset as the forward.  Forward with headdim 256 does not
+   * support dropout (ATTN_ERR_UNSUPPORTED_HEADDIM). */
+  float dropout_p;
+  uint32_t dropout_offset;
+  uint64_t dropout_seed;
 } attn_params;
 
 /*
@@ -118,6 +133,40 @@ typedef struct {
  */
 ATTN_API attn_status attn_fwd(const attn_params* p, const void* q, const void* k, const void* v, void* o,
                      float* lse, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Forward pass with E4M3 (FP8) inputs, the FP8 forward the pages name for
+ * FlashAttention-3.  q, k, v hold E4M3 codes, one byte per element, in the
+ * attn_fwd layouts; each tensor has one scale (element ~ scale *
+ * e4m3(code)), and the result is attention over those values:
+ * S = (q k^T) * q_scale * k_scale * softmax_scale, O = softmax(S) v * v_scale.
+ * o is written in p->dtype (bf16 or fp16), lse as attn_fwd's.  The kernel
+ * rounds P to E4M3 before the P V product (relative 2^-4).  Supported:
+ * headdim 128, causal and window masks, GQA; alibi_slopes must be NULL
+ * and dropout_p 0.
+ * Scales must be positive and finite (ATTN_ERR_INVALID_ARG).  Needs no
+ * workspace; asynchronous on `stream`.
+ */
+ATTN_API attn_status attn_fwd_e4m3(const attn_params* p, const void* q, const void* k,
+                                   const void* v, float q_scale, float k_scale, float v_scale,
+                                   void* o, float* lse, void* stream);
+
+/*
+ * Forward pass for decoding: a few query rows per sequence against a long
+ * key / value sequence (a cache), with the same arguments, layouts, masks
+ * (bottom-right aligned) and results as attn_fwd.  The keys are split over
+ * blocks of the CUDA cores (the work is bound by reading K and V; every kv
+ * head's K and V rows are read once for all the query heads of its group)
+ * and the splits' partial results are merged as attn_merge does.
+ * Supported: headdim 64 or 128, (nheads / nheads_kv) * seqlen_q <= 16,
+ * no positional slopes and no dropout (ATTN_ERR_INVALID_ARG otherwise).  workspace: at
+ * least attn_fwd_decode_workspace_size(p) bytes, 256-byte aligned, caller-
+ * owned, overwritten.  Asynchronous on `stream`.
+ */
+ATTN_API size_t attn_fwd_decode_workspace_size(const attn_params* p);
+ATTN_API attn_status attn_fwd_decode(const attn_params* p, const void* q, const void* k,
+                                     const void* v, void* o, float* lse, void* workspace,
+                                     size_t workspace_bytes, void* stream);
 
 /*
  * Backward pass: given dout = dL/dO and the forward's o and lse, writes
@@ -216,6 +265,9 @@ typedef struct {
   int32_t window_left;
   int32_t window_right;
   const float* alibi_slopes;  /* as in attn_params; lengths per sequence */
+  float dropout_p;            /* as in attn_params; b = sequence index and */
+  uint32_t dropout_offset;    /* i, j positions within the sequence */
+  uint64_t dropout_seed;
 } attn_varlen_params;
 
 /* Host-side checks of a packed call (pass 0 forward, 1 backward): the

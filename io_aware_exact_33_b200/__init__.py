@@ -30,6 +30,7 @@ EXPORTED = ("attn_fwd", "attn_bwd", "attn_bwd_prepare", "attn_bwd_accumulate", "
             "attn_fwd_workspace_size", "attn_bwd_workspace_size", "attn_check_params",
             "attn_status_string", "attn_get_device_status", "attn_version", "attn_bwd_noalloc",
             "attn_selftest_bounded_wait", "attn_check_varlen_params", "attn_fwd_varlen",
+            "attn_fwd_e4m3", "attn_fwd_decode", "attn_fwd_decode_workspace_size",
             "attn_bwd_varlen_workspace_size", "attn_bwd_varlen", "attn_merge")
 
 
@@ -48,6 +49,9 @@ class AttnParams(ctypes.Structure):
         ("window_left", ctypes.c_int32),
         ("window_right", ctypes.c_int32),
         ("alibi_slopes", ctypes.c_void_p),
+        ("dropout_p", ctypes.c_float),
+        ("dropout_offset", ctypes.c_uint32),
+        ("dropout_seed", ctypes.c_uint64),
     ]
 
 
@@ -68,6 +72,9 @@ class AttnVarlenParams(ctypes.Structure):
         ("window_left", ctypes.c_int32),
         ("window_right", ctypes.c_int32),
         ("alibi_slopes", ctypes.c_void_p),
+        ("dropout_p", ctypes.c_float),
+        ("dropout_offset", ctypes.c_uint32),
+        ("dropout_seed", ctypes.c_uint64),
     ]
 
 
@@ -148,13 +155,15 @@ _lib = _Lazy()
 
 def make_params(batch, seqlen_q, seqlen_k, nheads, nheads_kv, headdim, dtype=ATTN_BF16,
                 softmax_scale=None, causal=False, window_left=-1, window_right=-1,
-                alibi_slopes=None) -> AttnParams:
+                alibi_slopes=None, dropout_p=0.0, dropout_seed=0, dropout_offset=0) -> AttnParams:
     """``alibi_slopes``: None, or the device address (int) of nheads float32
-    slopes."""
+    slopes.  Dropout: rate ``dropout_p`` (applied as round(256 p) / 256), the
+    generator's 64-bit seed and 32-bit offset (see include/attn.h)."""
     scale = 1.0 / math.sqrt(headdim) if softmax_scale is None else float(softmax_scale)
     return AttnParams(int(batch), int(seqlen_q), int(seqlen_k), int(nheads), int(nheads_kv),
                       int(headdim), int(dtype), scale, int(bool(causal)), int(window_left),
-                      int(window_right), alibi_slopes)
+                      int(window_right), alibi_slopes, float(dropout_p),
+                      int(dropout_offset) & 0xFFFFFFFF, int(dropout_seed) & (2 ** 64 - 1))
 
 
 def _slopes_ptr(alibi_slopes, nheads, device):
@@ -246,26 +255,31 @@ def _stream(stream):
 
 
 def params_for(q, k, softmax_scale=None, causal=False, window_left=-1, window_right=-1,
-               alibi_slopes=None):
+               alibi_slopes=None, dropout_p=0.0, dropout_seed=0, dropout_offset=0):
     B, Nq, H, d = q.shape
     Bk, Nk, Hkv, dk = k.shape
     if Bk != B or dk != d:
         raise ValueError("q and k disagree on batch or head dim")
     return make_params(B, Nq, Nk, H, Hkv, d, _dtype_code(q), softmax_scale, causal, window_left,
-                       window_right, _slopes_ptr(alibi_slopes, H, q.device))
+                       window_right, _slopes_ptr(alibi_slopes, H, q.device), dropout_p,
+                       dropout_seed, dropout_offset)
 
 
 def attn_fwd(q, k, v, softmax_scale: Optional[float] = None, causal: bool = False,
              window_left: int = -1, window_right: int = -1, out=None, lse=None,
-             stream=None, alibi_slopes=None) -> Tuple["torch.Tensor", "torch.Tensor"]:
+             stream=None, alibi_slopes=None, dropout_p: float = 0.0, dropout_seed: int = 0,
+             dropout_offset: int = 0) -> Tuple["torch.Tensor", "torch.Tensor"]:
     """O = softmax(q k^T * scale + bias + mask) v and the per-row natural-log LSE.
 
     q (B, Nq, H, d), k and v (B, Nk, Hkv, d), bf16 or fp16, contiguous CUDA
     tensors; ``alibi_slopes`` (optional, (H,) float32) adds
-    -slope_h * |i + Nk - Nq - j|.  Returns (out (B, Nq, H, d), lse (B, H, Nq)
-    float32)."""
+    -slope_h * |i + Nk - Nq - j|.  ``dropout_p`` > 0 drops attention
+    probabilities by the generator contract of include/attn.h (seed, offset);
+    the backward needs the same three values.  Returns (out (B, Nq, H, d),
+    lse (B, H, Nq) float32)."""
     import torch
-    p = params_for(q, k, softmax_scale, causal, window_left, window_right, alibi_slopes)
+    p = params_for(q, k, softmax_scale, causal, window_left, window_right, alibi_slopes,
+                   dropout_p, dropout_seed, dropout_offset)
     B, Nq, H, d = q.shape
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _check(t, n)
@@ -287,13 +301,93 @@ def attn_fwd(q, k, v, softmax_scale: Optional[float] = None, causal: bool = Fals
     return out, lse
 
 
+def attn_fwd_e4m3(q, k, v, q_scale: float, k_scale: float, v_scale: float,
+                  softmax_scale: Optional[float] = None, causal: bool = False,
+                  window_left: int = -1, window_right: int = -1, out_dtype=None, out=None,
+                  lse=None, stream=None) -> Tuple["torch.Tensor", "torch.Tensor"]:
+    """Attention over E4M3 inputs: q (B, Nq, H, 128), k and v (B, Nk, Hkv,
+    128) hold E4M3 codes (uint8 or float8_e4m3fn CUDA tensors), element ~
+    scale * e4m3(code) with one scale per tensor.  Returns (out (B, Nq, H,
+    128) in ``out_dtype`` (bf16 by default, or fp16), lse (B, H, Nq)
+    float32)."""
+    import torch
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, n)
+        if t.element_size() != 1:
+            raise TypeError(f"{n} must hold one-byte E4M3 codes")
+    _check(v, "v", k.shape)
+    B, Nq, H, d = q.shape
+    Bk, Nk, Hkv, dk = k.shape
+    if Bk != B or dk != d:
+        raise ValueError("q and k disagree on batch or head dim")
+    out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
+    code = {torch.bfloat16: ATTN_BF16, torch.float16: ATTN_FP16}.get(out_dtype)
+    if code is None:
+        raise TypeError("out_dtype must be bfloat16 or float16")
+    p = make_params(B, Nq, Nk, H, Hkv, d, code, softmax_scale, causal, window_left, window_right)
+    if out is None:
+        out = torch.empty((B, Nq, H, d), dtype=out_dtype, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    _check(out, "out", (B, Nq, H, d))
+    _check(lse, "lse", (B, H, Nq))
+    fn = _lib.attn_fwd_e4m3
+    vp = ctypes.c_void_p
+    fn.argtypes = [ctypes.POINTER(AttnParams), vp, vp, vp, ctypes.c_float, ctypes.c_float,
+                   ctypes.c_float, vp, vp, vp]
+    fn.restype = ctypes.c_int
+    st = fn(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), float(q_scale), float(k_scale),
+            float(v_scale), _ptr(out), _ptr(lse), _stream(stream))
+    if st != 0:
+        raise AttnError(st, "attn_fwd_e4m3")
+    return out, lse
+
+
+def attn_fwd_decode(q, k, v, softmax_scale: Optional[float] = None, causal: bool = False,
+                    window_left: int = -1, window_right: int = -1, out=None, lse=None,
+                    workspace=None, stream=None) -> Tuple["torch.Tensor", "torch.Tensor"]:
+    """``attn_fwd`` for decoding: a few query rows ((H / Hkv) * Nq <= 16)
+    against a long key / value sequence, on the CUDA cores with the keys
+    split over blocks.  Same arguments, layouts and results as ``attn_fwd``
+    (no positional slopes)."""
+    import torch
+    p = params_for(q, k, softmax_scale, causal, window_left, window_right)
+    B, Nq, H, d = q.shape
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, n)
+        if t.dtype != q.dtype:
+            raise TypeError("q, k, v must share a dtype")
+    _check(v, "v", k.shape)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device) if lse is None else lse
+    _check(out, "out", q.shape)
+    _check(lse, "lse", (B, H, Nq))
+    fn = _lib.attn_fwd_decode_workspace_size
+    fn.argtypes = [ctypes.POINTER(AttnParams)]
+    fn.restype = ctypes.c_size_t
+    ws_bytes = int(fn(ctypes.byref(p)))
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
+    vp = ctypes.c_void_p
+    call = _lib.attn_fwd_decode
+    call.argtypes = [ctypes.POINTER(AttnParams), vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
+    call.restype = ctypes.c_int
+    st = call(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(workspace),
+              ctypes.c_size_t(workspace.numel()), _stream(stream))
+    if st != 0:
+        raise AttnError(st, "attn_fwd_decode")
+    return out, lse
+
+
 def attn_bwd(q, k, v, out, lse, dout, softmax_scale: Optional[float] = None, causal: bool = False,
              window_left: int = -1, window_right: int = -1, dq=None, dk=None, dv=None,
-             workspace=None, stream=None, alibi_slopes=None):
+             workspace=None, stream=None, alibi_slopes=None, dropout_p: float = 0.0,
+             dropout_seed: int = 0, dropout_offset: int = 0):
     """Gradients (dq, dk, dv) of sum(out * dout) for attention with the same
     arguments as ``attn_fwd``; ``out`` and ``lse`` are its results."""
     import torch
-    p = params_for(q, k, softmax_scale, causal, window_left, window_right, alibi_slopes)
+    p = params_for(q, k, softmax_scale, causal, window_left, window_right, alibi_slopes,
+                   dropout_p, dropout_seed, dropout_offset)
     B, Nq, H, d = q.shape
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
         _check(t, n)
@@ -345,14 +439,16 @@ def attn_bwd_finalize(p: AttnParams, dq, workspace, stream=None) -> None:
 
 def attn_bwd_noalloc(q, k, v, out, lse, dout, softmax_scale: Optional[float] = None,
                      causal: bool = False, window_left: int = -1, window_right: int = -1,
-                     dq=None, dk=None, dv=None, stream=None, alibi_slopes=None):
+                     dq=None, dk=None, dv=None, stream=None, alibi_slopes=None,
+                     dropout_p: float = 0.0, dropout_seed: int = 0, dropout_offset: int = 0):
     """Like ``attn_bwd`` but the library uses its own fixed device scratch
     (ATTN_NOALLOC_SCRATCH_BYTES) instead of a caller workspace, for callers
     that cannot allocate device memory at call time.  The output tensors are
     the caller's (allocated here only when not given).  Calls that overlap on
     the GPU share that scratch and must be serialised by the caller."""
     import torch
-    p = params_for(q, k, softmax_scale, causal, window_left, window_right, alibi_slopes)
+    p = params_for(q, k, softmax_scale, causal, window_left, window_right, alibi_slopes,
+                   dropout_p, dropout_seed, dropout_offset)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
@@ -366,12 +462,14 @@ def attn_bwd_noalloc(q, k, v, out, lse, dout, softmax_scale: Optional[float] = N
 # ----------------------------------------------------------------- packed sequences
 def make_varlen_params(batch, total_q, total_k, max_seqlen_q, max_seqlen_k, nheads, nheads_kv,
                        headdim, dtype=ATTN_BF16, softmax_scale=None, causal=False,
-                       window_left=-1, window_right=-1, alibi_slopes=None) -> AttnVarlenParams:
+                       window_left=-1, window_right=-1, alibi_slopes=None, dropout_p=0.0,
+                       dropout_seed=0, dropout_offset=0) -> AttnVarlenParams:
     scale = 1.0 / math.sqrt(headdim) if softmax_scale is None else float(softmax_scale)
     return AttnVarlenParams(int(batch), int(total_q), int(total_k), int(max_seqlen_q),
                             int(max_seqlen_k), int(nheads), int(nheads_kv), int(headdim),
                             int(dtype), scale, int(bool(causal)), int(window_left),
-                            int(window_right), alibi_slopes)
+                            int(window_right), alibi_slopes, float(dropout_p),
+                            int(dropout_offset) & 0xFFFFFFFF, int(dropout_seed) & (2 ** 64 - 1))
 
 
 def attn_check_varlen_params(p: AttnVarlenParams, pass_: int = 0) -> int:
@@ -383,7 +481,8 @@ def attn_bwd_varlen_workspace_size(p: AttnVarlenParams) -> int:
 
 
 def _varlen_params(q, k, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, softmax_scale,
-                   causal, window_left, window_right, alibi_slopes=None):
+                   causal, window_left, window_right, alibi_slopes=None, dropout_p=0.0,
+                   dropout_seed=0, dropout_offset=0):
     import torch
     if q.dim() != 3 or k.dim() != 3:
         raise ValueError("packed q must be (total_q, nheads, d) and k (total_k, nheads_kv, d)")
@@ -399,13 +498,15 @@ def _varlen_params(q, k, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
         raise ValueError("cu_seqlens_q and cu_seqlens_k must both have batch + 1 entries")
     return make_varlen_params(cu_seqlens_q.numel() - 1, Tq, Tk, max_seqlen_q, max_seqlen_k, H, Hkv,
                               d, _dtype_code(q), softmax_scale, causal, window_left, window_right,
-                              _slopes_ptr(alibi_slopes, H, q.device))
+                              _slopes_ptr(alibi_slopes, H, q.device), dropout_p, dropout_seed,
+                              dropout_offset)
 
 
 def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int,
                     softmax_scale: Optional[float] = None, causal: bool = False,
                     window_left: int = -1, window_right: int = -1, out=None, lse=None,
-                    stream=None, alibi_slopes=None):
+                    stream=None, alibi_slopes=None, dropout_p: float = 0.0, dropout_seed: int = 0,
+                    dropout_offset: int = 0):
     """Attention over packed variable-length sequences.
 
     q (total_q, H, d), k and v (total_k, Hkv, d); sequence b owns rows
@@ -414,7 +515,8 @@ def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_
     (total_q, H, d), lse (H, total_q) float32)."""
     import torch
     p = _varlen_params(q, k, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
-                       softmax_scale, causal, window_left, window_right, alibi_slopes)
+                       softmax_scale, causal, window_left, window_right, alibi_slopes,
+                       dropout_p, dropout_seed, dropout_offset)
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _check(t, n)
         if t.dtype != q.dtype:
@@ -437,12 +539,14 @@ def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_
 def attn_bwd_varlen(q, k, v, out, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int,
                     max_seqlen_k: int, softmax_scale: Optional[float] = None,
                     causal: bool = False, window_left: int = -1, window_right: int = -1,
-                    dq=None, dk=None, dv=None, workspace=None, stream=None, alibi_slopes=None):
+                    dq=None, dk=None, dv=None, workspace=None, stream=None, alibi_slopes=None,
+                    dropout_p: float = 0.0, dropout_seed: int = 0, dropout_offset: int = 0):
     """Gradients (dq, dk, dv) of sum(out * dout) for ``attn_fwd_varlen`` with
     the same arguments; ``out`` and ``lse`` are its results."""
     import torch
     p = _varlen_params(q, k, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
-                       softmax_scale, causal, window_left, window_right, alibi_slopes)
+                       softmax_scale, causal, window_left, window_right, alibi_slopes,
+                       dropout_p, dropout_seed, dropout_offset)
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
         _check(t, n)
         if t.dtype != q.dtype:

@@ -13,6 +13,8 @@
 
 #include "attn.h"
 #include "bwd_kernel.cuh"
+#include "decode_kernel.cuh"
+#include "fwd_fp8_kernel.cuh"
 #include "fwd_kernel.cuh"
 #include "merge_kernel.cuh"
 #include "sm100.cuh"
@@ -57,6 +59,22 @@ bool map_bshd(CUtensorMap* m, const void* ptr, bool fp16, int batch, int seqlen,
                    const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// 8-bit (batch, seqlen, heads, 128) tensor of E4M3 codes as a 4-D map with a
+// box of 128 columns (one 128-byte swizzled row) x 1 head x `rows` rows.
+bool map_bshd_u8(CUtensorMap* m, const void* ptr, int batch, int seqlen, int heads, int d,
+                 int rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)seqlen, (cuuint64_t)batch};
+  cuuint64_t strides[3] = {(cuuint64_t)d, (cuuint64_t)heads * d, (cuuint64_t)seqlen * heads * d};
+  cuuint32_t box[4] = {128, 1, (cuuint32_t)rows, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(ptr), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -169,18 +187,26 @@ struct Packed {
 
 // Kernel and grid width of a forward configuration: two query tiles per CTA
 // where both O tiles fit tensor memory (d <= 128), one otherwise.
+// The one-tile kernel (d = 256) has no dropout variant: attn_check_params
+// rejects dropout there before any launch.
 template <class C>
 struct FwdLaunch {
-  template <bool ALIBI>
+  template <bool ALIBI, bool DROP>
   static constexpr auto kernel() { return attn_fwd_kernel<C, ALIBI>; }
   static constexpr int rows_per_cta = C::BM;
 };
 template <int D, int KS, int VS, bool F>
 struct FwdLaunch<FwdPPCfg<D, KS, VS, F>> {
-  template <bool ALIBI>
-  static constexpr auto kernel() { return attn_fwd_pp_kernel<FwdPPCfg<D, KS, VS, F>, ALIBI>; }
+  template <bool ALIBI, bool DROP>
+  static constexpr auto kernel() {
+    return attn_fwd_pp_kernel<FwdPPCfg<D, KS, VS, F>, ALIBI, DROP>;
+  }
   static constexpr int rows_per_cta = 2 * FwdPPCfg<D, KS, VS, F>::BM;
 };
+
+// Dropout threshold t = round(256 p) of the contract in philox.cuh (0 = no
+// dropout); p has been checked to lie in [0, 255.5 / 256).
+uint32_t drop_threshold(float p) { return (uint32_t)std::floor(256.0 * (double)p + 0.5); }
 
 // Forward launch.  Dense: p->seqlen_q/k are the lengths.  Packed: p->batch
 // sequences of at most p->seqlen_q / p->seqlen_k rows each.
@@ -203,6 +229,11 @@ attn_status launch_fwd(const attn_params* p, const void* q, const void* k, const
   fp.total_k = pk.total_k;
   fp.o = static_cast<uint16_t*>(o);
   fp.alibi = p->alibi_slopes;
+  const uint32_t t = drop_threshold(p->dropout_p);
+  fp.drop_seed = p->dropout_seed;
+  fp.drop_offset = p->dropout_offset;
+  fp.drop_kadd = dropout_kadd(t);
+  fp.drop_scale = 256.f / (float)(256u - t);
   fp.lse = lse;
   fp.batch = p->batch;
   fp.nheads = p->nheads;
@@ -219,11 +250,105 @@ attn_status launch_fwd(const attn_params* p, const void* q, const void* k, const
   fp.sched_group = l2_group(4.0 * p->seqlen_k * C::D / (p->nheads / p->nheads_kv), heads);
   const long long blocks = (long long)fp.num_qblocks * heads;
   if (blocks > INT_MAX) return ATTN_ERR_INVALID_ARG;
-  auto kern = p->alibi_slopes ? FwdLaunch<C>::template kernel<true>()
-                              : FwdLaunch<C>::template kernel<false>();
+  auto kern = p->alibi_slopes ? (t ? FwdLaunch<C>::template kernel<true, true>()
+                                    : FwdLaunch<C>::template kernel<true, false>())
+                              : (t ? FwdLaunch<C>::template kernel<false, true>()
+                                   : FwdLaunch<C>::template kernel<false, false>());
   if (!ensure_smem(reinterpret_cast<const void*>(kern), C::SMEM_BYTES)) return ATTN_ERR_CUDA;
   kern<<<(unsigned)blocks, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mo, fp);
   return finish(stream);
+}
+
+// Forward with E4M3 inputs (dense batches, d = 128).
+template <class C>
+attn_status launch_fwd_e4m3(const attn_params* p, const void* q, const void* k, const void* v,
+                            float q_scale, float k_scale, float v_scale, void* o, float* lse,
+                            cudaStream_t stream) {
+  CUtensorMap mq, mk, mv, mo;
+  if (!map_bshd_u8(&mq, q, p->batch, p->seqlen_q, p->nheads, C::D, C::BM) ||
+      !map_bshd_u8(&mk, k, p->batch, p->seqlen_k, p->nheads_kv, C::D, C::BN) ||
+      !map_bshd_u8(&mv, v, p->batch, p->seqlen_k, p->nheads_kv, C::D, C::BN) ||
+      !map_bshd(&mo, o, C::FP16, p->batch, p->seqlen_q, p->nheads, C::D, C::BM))
+    return ATTN_ERR_CUDA;
+  FwdParams fp;
+  std::memset(&fp, 0, sizeof(fp));
+  fp.o = static_cast<uint16_t*>(o);
+  fp.lse = lse;
+  fp.batch = p->batch;
+  fp.nheads = p->nheads;
+  fp.nheads_kv = p->nheads_kv;
+  fp.seqlen_q = p->seqlen_q;
+  fp.seqlen_k = p->seqlen_k;
+  fp.causal = p->causal;
+  fp.window_left = p->window_left;
+  fp.window_right = p->window_right;
+  fp.scale_log2 = p->softmax_scale * q_scale * k_scale * 1.4426950408889634f;
+  fp.num_qblocks = (p->seqlen_q + 2 * C::BM - 1) / (2 * C::BM);
+  const int heads = p->batch * p->nheads;
+  // K and V bytes (one per element) each query head streams
+  fp.sched_group = l2_group(2.0 * p->seqlen_k * C::D / (p->nheads / p->nheads_kv), heads);
+  const long long blocks = (long long)fp.num_qblocks * heads;
+  if (blocks > INT_MAX) return ATTN_ERR_INVALID_ARG;
+  auto kern = attn_fwd_e4m3_kernel<C>;
+  if (!ensure_smem(reinterpret_cast<const void*>(kern), C::SMEM_BYTES)) return ATTN_ERR_CUDA;
+  kern<<<(unsigned)blocks, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mo, fp, v_scale);
+  return finish(stream);
+}
+
+// Key splits of a decode call: about two blocks per SM over the
+// (batch, kv head) pairs, at least 256 keys per split.
+int decode_splits(const attn_params* p) {
+  const long long groups = (long long)p->batch * p->nheads_kv;
+  long long want = (2 * 148 + groups - 1) / groups;
+  const long long by_len = ((long long)p->seqlen_k + 255) / 256;
+  if (want > by_len) want = by_len;
+  if (want > 65535) want = 65535;
+  return (int)(want < 1 ? 1 : want);
+}
+
+// Workspace of a decode call: the splits' 16-bit partial outputs, then
+// their LSE values.
+struct DecodeWorkspace {
+  size_t o_bytes, total;
+};
+DecodeWorkspace decode_layout(const attn_params* p) {
+  const size_t rows = (size_t)decode_splits(p) * p->batch * p->seqlen_q * p->nheads;
+  DecodeWorkspace w;
+  w.o_bytes = (rows * p->headdim * 2 + 255) / 256 * 256;
+  w.total = w.o_bytes + (rows * 4 + 255) / 256 * 256;
+  return w;
+}
+
+template <int D, bool FP16>
+attn_status launch_decode(const attn_params* p, const void* q, const void* k, const void* v,
+                          void* o, float* lse, void* workspace, cudaStream_t stream) {
+  const int splits = decode_splits(p);
+  const DecodeWorkspace ws = decode_layout(p);
+  DecodeParams dp;
+  dp.q = static_cast<const uint16_t*>(q);
+  dp.k = static_cast<const uint16_t*>(k);
+  dp.v = static_cast<const uint16_t*>(v);
+  dp.o_parts = static_cast<uint16_t*>(workspace);
+  dp.lse_parts = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + ws.o_bytes);
+  dp.batch = p->batch;
+  dp.nheads = p->nheads;
+  dp.nheads_kv = p->nheads_kv;
+  dp.seqlen_q = p->seqlen_q;
+  dp.seqlen_k = p->seqlen_k;
+  dp.causal = p->causal;
+  dp.window_left = p->window_left;
+  dp.window_right = p->window_right;
+  dp.scale_log2 = p->softmax_scale * 1.4426950408889634f;
+  dp.splits = splits;
+  dp.chunk = (int)((((long long)p->seqlen_k + splits - 1) / splits + 31) / 32 * 32);
+  auto kern = attn_decode_kernel<D, FP16>;
+  if (!ensure_smem(reinterpret_cast<const void*>(kern), DecodeSmem<D>::BYTES)) return ATTN_ERR_CUDA;
+  const dim3 grid((unsigned)(p->batch * p->nheads_kv), (unsigned)splits);  // splits <= 65535
+  kern<<<grid, kDecodeWarps * 32, DecodeSmem<D>::BYTES, stream>>>(dp);
+  const attn_status st = finish(stream);
+  if (st != ATTN_OK) return st;
+  const attn_merge_params mp = {splits, p->batch, p->seqlen_q, p->nheads, p->headdim, p->dtype};
+  return attn_merge(&mp, dp.o_parts, dp.lse_parts, o, lse, stream);
 }
 
 BwdWorkspace bwd_layout(const attn_params* p, const Packed& pk) {
@@ -241,6 +366,11 @@ BwdParams bwd_params(const attn_params* p, const float* lse, void* workspace, co
   bp.total_k = pk.total_k;
   bp.dk = bp.dv = nullptr;
   bp.alibi = p->alibi_slopes;
+  const uint32_t t = drop_threshold(p->dropout_p);
+  bp.drop_seed = p->dropout_seed;
+  bp.drop_offset = p->dropout_offset;
+  bp.drop_kadd = dropout_kadd(t);
+  bp.drop_scale = 256.f / (float)(256u - t);
   bp.num_kblocks = bp.sched_group = 0;
   bp.lse = lse;
   bp.dvec = reinterpret_cast<float*>(w + ws.dvec_off);
@@ -311,7 +441,9 @@ attn_status launch_bwd_main(const attn_params* p, const void* q, const void* k, 
   bpl.sched_group = l2_group(8.0 * p->seqlen_q * C::D * (p->nheads / p->nheads_kv), heads);
   const long long blocks = (long long)bpl.num_kblocks * heads;
   if (blocks > INT_MAX) return ATTN_ERR_INVALID_ARG;
-  auto kern = p->alibi_slopes ? attn_bwd_kernel<C, true> : attn_bwd_kernel<C, false>;
+  const bool drop = drop_threshold(p->dropout_p) != 0;
+  auto kern = p->alibi_slopes ? (drop ? attn_bwd_kernel<C, true, true> : attn_bwd_kernel<C, true, false>)
+                              : (drop ? attn_bwd_kernel<C, false, true> : attn_bwd_kernel<C, false, false>);
   if (!ensure_smem(reinterpret_cast<const void*>(kern), C::SMEM_BYTES)) return ATTN_ERR_CUDA;
   kern<<<(unsigned)blocks, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, ml, md, mdk,
                                                                  mdv, mdq, bpl);
@@ -425,6 +557,9 @@ attn_params packed_view(const attn_varlen_params* v) {
   p.window_left = v->window_left;
   p.window_right = v->window_right;
   p.alibi_slopes = v->alibi_slopes;
+  p.dropout_p = v->dropout_p;
+  p.dropout_offset = v->dropout_offset;
+  p.dropout_seed = v->dropout_seed;
   return p;
 }
 
@@ -483,7 +618,73 @@ attn_status attn_check_params(const attn_params* p, int pass) {
   if (p->causal != 0 && p->causal != 1) return ATTN_ERR_INVALID_ARG;
   if (p->window_left < -1 || p->window_right < -1) return ATTN_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(p->alibi_slopes) & 3u) return ATTN_ERR_MISALIGNED;
+  if (!(p->dropout_p >= 0.f) || !(p->dropout_p < 1.f) || drop_threshold(p->dropout_p) > 255u)
+    return ATTN_ERR_INVALID_ARG;
+  if (d == 256 && drop_threshold(p->dropout_p) != 0) return ATTN_ERR_UNSUPPORTED_HEADDIM;
   return ATTN_OK;
+}
+
+attn_status attn_fwd_e4m3(const attn_params* p, const void* q, const void* k, const void* v,
+                          float q_scale, float k_scale, float v_scale, void* o, float* lse,
+                          void* stream_) {
+  attn_status st = attn_check_params(p, 0);
+  if (st != ATTN_OK) return st;
+  if (p->headdim != 128) return ATTN_ERR_UNSUPPORTED_HEADDIM;
+  if (p->alibi_slopes || drop_threshold(p->dropout_p) != 0) return ATTN_ERR_INVALID_ARG;
+  for (float sc : {q_scale, k_scale, v_scale})
+    if (!(sc > 0.f) || !std::isfinite(sc)) return ATTN_ERR_INVALID_ARG;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (p->batch == 0 || p->seqlen_q == 0) return ATTN_OK;
+  if (!o || !lse) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(o) || (reinterpret_cast<uintptr_t>(lse) & 3u)) return ATTN_ERR_MISALIGNED;
+  if (p->seqlen_k == 0) {
+    const long long n_o = (long long)p->batch * p->seqlen_q * p->nheads * p->headdim;
+    const long long n_l = (long long)p->batch * p->nheads * p->seqlen_q;
+    fill_empty_fwd<<<fill_blocks(n_o), 256, 0, stream>>>(static_cast<uint16_t*>(o), n_o, lse, n_l);
+    return finish(stream);
+  }
+  if (!q || !k || !v) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return ATTN_ERR_MISALIGNED;
+  return p->dtype == ATTN_FP16
+             ? launch_fwd_e4m3<FwdF8Cfg<3, 2, true>>(p, q, k, v, q_scale, k_scale, v_scale, o, lse,
+                                                     stream)
+             : launch_fwd_e4m3<FwdF8Cfg<3, 2, false>>(p, q, k, v, q_scale, k_scale, v_scale, o,
+                                                      lse, stream);
+}
+
+size_t attn_fwd_decode_workspace_size(const attn_params* p) {
+  if (attn_check_params(p, 0) != ATTN_OK) return 0;
+  return decode_layout(p).total;
+}
+
+attn_status attn_fwd_decode(const attn_params* p, const void* q, const void* k, const void* v,
+                            void* o, float* lse, void* workspace, size_t workspace_bytes,
+                            void* stream_) {
+  attn_status st = attn_check_params(p, 0);
+  if (st != ATTN_OK) return st;
+  if (p->headdim != 64 && p->headdim != 128) return ATTN_ERR_UNSUPPORTED_HEADDIM;
+  if (p->alibi_slopes || drop_threshold(p->dropout_p) != 0) return ATTN_ERR_INVALID_ARG;
+  if ((long long)(p->nheads / p->nheads_kv) * p->seqlen_q > kDecodeRows) return ATTN_ERR_INVALID_ARG;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (p->batch == 0 || p->seqlen_q == 0) return ATTN_OK;
+  if (!o || !lse) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(o) || (reinterpret_cast<uintptr_t>(lse) & 3u)) return ATTN_ERR_MISALIGNED;
+  if (p->seqlen_k == 0) {
+    const long long n_o = (long long)p->batch * p->seqlen_q * p->nheads * p->headdim;
+    const long long n_l = (long long)p->batch * p->nheads * p->seqlen_q;
+    fill_empty_fwd<<<fill_blocks(n_o), 256, 0, stream>>>(static_cast<uint16_t*>(o), n_o, lse, n_l);
+    return finish(stream);
+  }
+  if (!q || !k || !v || !workspace) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return ATTN_ERR_MISALIGNED;
+  if (workspace_bytes < decode_layout(p).total) return ATTN_ERR_WORKSPACE_TOO_SMALL;
+  const bool fp16 = p->dtype == ATTN_FP16;
+  if (p->headdim == 64)
+    return fp16 ? launch_decode<64, true>(p, q, k, v, o, lse, workspace, stream)
+                : launch_decode<64, false>(p, q, k, v, o, lse, workspace, stream);
+  return fp16 ? launch_decode<128, true>(p, q, k, v, o, lse, workspace, stream)
+              : launch_decode<128, false>(p, q, k, v, o, lse, workspace, stream);
 }
 
 size_t attn_fwd_workspace_size(const attn_params* p) {

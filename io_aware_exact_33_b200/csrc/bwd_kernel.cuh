@@ -39,6 +39,7 @@
 
 #include <cuda_fp16.h>
 
+#include "philox.cuh"
 #include "sm100.cuh"
 
 namespace attn {
@@ -115,6 +116,11 @@ struct BwdParams {
   // Per-head positional slopes (nheads floats), or nullptr: scores gain
   // -slope_h * |i + seqlen_k - seqlen_q - j| (kernel instantiated with ALIBI).
   const float* alibi;
+  // Dropout (kernel instantiated with DROP; the contract in philox.cuh):
+  // drop_kadd = dropout_kadd(t), drop_scale = 256 / (256 - t).
+  unsigned long long drop_seed;
+  uint32_t drop_offset, drop_kadd;
+  float drop_scale;
 };
 
 // Packed layout: the sequence owning padded row `pr` (the last b with
@@ -314,7 +320,7 @@ struct BwdCfg {
   static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
 
-template <class C, bool ALIBI>
+template <class C, bool ALIBI, bool DROP>
 __global__ void __launch_bounds__(C::THREADS, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -633,11 +639,30 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           if (j >= p.seqlen_k || j > i + off + rb || j < i + off - lb) pr[c] = 0.f;
         }
       }
+      // Dropout: this key's random bytes for the warp's query columns, kw[k]
+      // for columns 4k .. 4k + 3.  P^T goes to the dV MMA with dropped
+      // elements zeroed (dV's 1 / (1 - p) is applied in the epilogue); pr
+      // keeps the undropped P for dS.
+      [[maybe_unused]] uint32_t kw[C::HW / 4];
+      if constexpr (DROP) {
+        const uint32_t bh = (uint32_t)(b * p.nheads + hq);
+#pragma unroll
+        for (int c = 0; c < C::HW; c += 32) {
+          uint32_t part[8];
+          dropout_col32(p.drop_seed, p.drop_offset, bh, (uint32_t)j, (uint32_t)(qa + c), part);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) kw[c / 4 + k] = part[k];
+        }
+      }
 #pragma unroll
       for (int c = 0; c < C::HW; c += 32) {
         uint32_t w[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) w[e] = pack2<C::FP16>(pr[c + 2 * e], pr[c + 2 * e + 1]);
+        for (int e = 0; e < 16; ++e) {
+          w[e] = pack2<C::FP16>(pr[c + 2 * e], pr[c + 2 * e + 1]);
+          if constexpr (DROP)
+            w[e] &= dropout_pair_mask(dropout_keep_bits(kw[(c + 2 * e) / 4], e & 1, p.drop_kadd));
+        }
         tmem_st16(s_tmem + c / 2, w);
       }
       tmem_st_wait();
@@ -661,9 +686,20 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           ld_shared_v4f(dvec_addr + (c + e) * 4, d4);
 #pragma unroll
           for (int f = 0; f < 4; f += 2) {
-            // dS = P * (dP - Dvec), two columns per packed instruction pair
-            const uint64_t diff = f2_add(f2_pack(__uint_as_float(raw[e + f]), __uint_as_float(raw[e + f + 1])),
-                                         f2_pack(-d4[f], -d4[f + 1]));
+            // dS = P * (dP - Dvec), two columns per packed instruction pair;
+            // with dropout dP of a kept element is scaled by 1 / (1 - p) and
+            // that of a dropped one is 0.
+            uint64_t diff;
+            if constexpr (DROP) {
+              const uint32_t kb = dropout_keep_bits(kw[(c + e) / 4], f / 2, p.drop_kadd);
+              const float g0 = __uint_as_float(raw[e + f] & dropout_lo_mask(kb));
+              const float g1 = __uint_as_float(raw[e + f + 1] & dropout_hi_mask(kb));
+              diff = f2_fma(f2_pack(g0, g1), f2_pack(p.drop_scale, p.drop_scale),
+                            f2_pack(-d4[f], -d4[f + 1]));
+            } else {
+              diff = f2_add(f2_pack(__uint_as_float(raw[e + f]), __uint_as_float(raw[e + f + 1])),
+                            f2_pack(-d4[f], -d4[f + 1]));
+            }
             f2_unpack(f2_mul(f2_pack(pr[c + e + f], pr[c + e + f + 1]), diff), pr[c + e + f],
                       pr[c + e + f + 1]);
           }
@@ -701,7 +737,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       for (int which = 0; which < 2; ++which) {
         const uint32_t src = tmem + lane_base + (which == 0 ? C::TM_DK : C::TM_DV);
         const uint32_t row_addr = smem0 + (which == 0 ? C::OFF_Q : C::OFF_DO) + r * 128;
-        const float mul = which == 0 ? p.softmax_scale : 1.f;
+        const float mul = which == 0 ? p.softmax_scale : (DROP ? p.drop_scale : 1.f);
 #pragma unroll 1
         for (int c = half * (D / 2); c < (half + 1) * (D / 2); c += 32) {
           uint32_t raw[32];

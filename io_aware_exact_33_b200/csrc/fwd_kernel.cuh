@@ -27,6 +27,7 @@
 
 #include <type_traits>
 
+#include "philox.cuh"
 #include "sm100.cuh"
 
 namespace attn {
@@ -49,6 +50,18 @@ struct FwdParams {
   // Per-head positional slopes (nheads floats), or nullptr: scores gain
   // -slope_h * |i + seqlen_k - seqlen_q - j| (kernels instantiated with ALIBI).
   const float* alibi;
+  // Dropout (kernels instantiated with DROP; the contract in philox.cuh):
+  // drop_kadd = dropout_kadd(t), drop_scale = 256 / (256 - t).
+  unsigned long long drop_seed;
+  uint32_t drop_offset, drop_kadd;
+  float drop_scale;
+};
+
+// Where one softmax thread's dropout bytes come from: generator key and
+// offset, head index b * H + h, the thread's query row.
+struct DropRow {
+  unsigned long long seed;
+  uint32_t offset, bh, row, kadd;
 };
 
 // Row `row` of query head h of sequence (b, sq) in the LSE output.
@@ -477,12 +490,19 @@ constexpr uint32_t kPolyPairs = 0x2222u;
 //    on one side of its diagonal, the bias is linear in the column, b0 +
 //    dl * c, and rides in the FMA's addend (one extra packed FMA per column
 //    pair); tiles the diagonal crosses add it column by column.
-template <bool MASK, bool ALIBI, class C>
+//
+// With DROP, P is written to tensor memory with dropped elements zeroed
+// (the row sum keeps them: l and the LSE are those of the undropped scores);
+// the 1 / (1 - p) factor is applied to O in the epilogue.  The generator's
+// integer work then shares the FMA pipe, so no exponential is offloaded to
+// the polynomial.
+template <bool MASK, bool ALIBI, bool DROP, class C>
 __device__ __forceinline__ void softmax_tile(uint32_t s_tmem, uint32_t o_tmem, int n, int vlo,
                                              int vhi, float scale_log2, float m, float& mx,
                                              float& rowsum, float& alpha, float& m_use,
                                              uint32_t pready_half0, uint32_t pready_half1,
-                                             float bd, float bk, bool left) {
+                                             float bd, float bk, bool left, const DropRow& dr,
+                                             uint32_t k0) {
   constexpr int BN = C::BN, D = C::D;
   auto val = [&](uint32_t bits, int col) -> float {
     return (MASK && (col < vlo || col >= vhi)) ? -INFINITY : __uint_as_float(bits);
@@ -565,6 +585,19 @@ __device__ __forceinline__ void softmax_tile(uint32_t s_tmem, uint32_t o_tmem, i
     tmem_ld_wait();
 #pragma unroll
     for (int c = 0; c < BN / 32; ++c) {
+      // this row's random bytes for the chunk's 32 columns (DROP), made
+      // before the next chunk's load is in flight
+      [[maybe_unused]] uint32_t kw[8];
+      if constexpr (DROP) {
+        uint32_t a[4], z[4];
+        dropout_row16(dr.seed, dr.offset, dr.bh, dr.row, k0 + 32u * c, a);
+        dropout_row16(dr.seed, dr.offset, dr.bh, dr.row, k0 + 32u * c + 16u, z);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          kw[k] = a[k];
+          kw[4 + k] = z[k];
+        }
+      }
       if (c + 1 < BN / 32) tmem_ld32(s_tmem + (c + 1) * 32, buf[(c + 1) & 1]);
       uint32_t w[16];
 #pragma unroll
@@ -582,7 +615,7 @@ __device__ __forceinline__ void softmax_tile(uint32_t s_tmem, uint32_t o_tmem, i
             a1 = fmaf(fabsf(bd - (float)(col + 1)), bk, a1);
           }
         }
-        if (!MASK && ((kPolyPairs >> (e / 2)) & 1)) {
+        if (!MASK && !DROP && ((kPolyPairs >> (e / 2)) & 1)) {
           exp2_poly2(a0, a1, p0, p1);
         } else {
           p0 = ex2(a0);
@@ -590,6 +623,8 @@ __device__ __forceinline__ void softmax_tile(uint32_t s_tmem, uint32_t o_tmem, i
         }
         sum2 = f2_add(sum2, f2_pack(p0, p1));
         w[e / 2] = pack2<C::FP16>(p0, p1);
+        if constexpr (DROP)
+          w[e / 2] &= dropout_pair_mask(dropout_keep_bits(kw[e / 4], (e / 2) & 1, dr.kadd));
       }
       if (c + 1 < BN / 32) tmem_ld_wait();
       tmem_st16(s_tmem + c * 16, w);
@@ -612,7 +647,7 @@ __device__ __forceinline__ void softmax_tile(uint32_t s_tmem, uint32_t o_tmem, i
   }
 }
 
-template <class C, bool ALIBI>
+template <class C, bool ALIBI, bool DROP>
 __global__ void __launch_bounds__(C::THREADS, 1)
     attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -803,6 +838,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const int n_i = hi_i - lo_i;
     // positional slope in log2 units (negated): bias of column c = bk * |bd - c|
     const float bk = ALIBI ? -p.alibi[h] * 1.4426950408889634f : 0.f;
+    // seed, offset and kadd straight from the kernel parameters (constant
+    // bank), so they hold no registers across the key loop
+    const DropRow dr{pin.drop_seed, pin.drop_offset, (uint32_t)(b * pin.nheads + h),
+                     (uint32_t)row, pin.drop_kadd};
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int n = 0; n < n_i; ++n) {
@@ -821,11 +860,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       const uint32_t ph0 = bar(C::B_PREADY + 2 * i), ph1 = bar(C::B_PREADY + 2 * i + 1);
       const float bd = ALIBI ? (float)((long long)row + off - k0) : 0.f;
       if (full)
-        softmax_tile<false, ALIBI, C>(s_tmem, o_tmem, n, vlo, vhi, p.scale_log2, m, mx, rowsum,
-                                      alpha, m_use, ph0, ph1, bd, bk, p.causal != 0);
+        softmax_tile<false, ALIBI, DROP, C>(s_tmem, o_tmem, n, vlo, vhi, p.scale_log2, m, mx,
+                                            rowsum, alpha, m_use, ph0, ph1, bd, bk, p.causal != 0,
+                                            dr, (uint32_t)k0);
       else
-        softmax_tile<true, ALIBI, C>(s_tmem, o_tmem, n, vlo, vhi, p.scale_log2, m, mx, rowsum,
-                                     alpha, m_use, ph0, ph1, bd, bk, p.causal != 0);
+        softmax_tile<true, ALIBI, DROP, C>(s_tmem, o_tmem, n, vlo, vhi, p.scale_log2, m, mx,
+                                           rowsum, alpha, m_use, ph0, ph1, bd, bk, p.causal != 0,
+                                           dr, (uint32_t)k0);
       l = l * alpha + rowsum;
       m = m_use;
     }
@@ -838,7 +879,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const bool row_store = p.cu_q != nullptr && q_i + BM > p.seqlen_q;
     if (ok) {
       tc_fence_after();
-      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      const float inv_l = l > 0.f ? (DROP ? p.drop_scale : 1.f) / l : 0.f;
       const uint32_t row_addr = stage + r * 128;
 #pragma unroll 1
       for (int c = 0; c < D; c += 32) {

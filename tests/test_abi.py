@@ -111,6 +111,20 @@ def test_alibi_pointer_alignment(attn):
     assert attn.attn_check_params(p, 0) == 0
 
 
+def test_dropout_checks(attn):
+    """dropout_p must be in [0, 255.5 / 256) (its threshold round(256 p) at
+    most 255); the headdim-256 forward has no dropout variant, but a rate
+    that rounds to threshold 0 is no dropout and passes."""
+    assert attn.attn_check_params(P(attn, dropout_p=0.1, dropout_seed=7), 0) == 0
+    assert attn.attn_check_params(P(attn, dropout_p=0.1), 1) == 0
+    for bad in (-0.1, 1.0, 0.999, float("nan"), float("inf")):
+        assert attn.attn_check_params(P(attn, dropout_p=bad), 0) == 1, bad
+    assert attn.attn_check_params(P(attn, headdim=256, dropout_p=0.1), 0) == 2
+    assert attn.attn_check_params(P(attn, headdim=256, dropout_p=0.001), 0) == 0
+    v = attn.make_varlen_params(2, 10, 10, 5, 5, 4, 2, 64, dropout_p=1.5)
+    assert attn.attn_check_varlen_params(v, 0) == 1
+
+
 def test_merge_host_checks(attn):
     """attn_merge rejects bad sizes before touching the GPU; an empty merge
     is a no-op."""
@@ -136,6 +150,7 @@ def test_header_is_plain_c(attn, tmp_path):
         pytest.skip("no C compiler")
     src = tmp_path / "use_attn.c"
     src.write_text(r"""
+#include <stddef.h>
 #include <stdio.h>
 #include "attn.h"
 int main(void) {
@@ -148,6 +163,11 @@ int main(void) {
   printf("%d %d %d %zu %zu %s\n", (int)attn_check_params(&p, 0), (int)attn_check_params(&p, 1),
          (int)attn_check_varlen_params(&v, 1), attn_bwd_workspace_size(&p),
          attn_bwd_varlen_workspace_size(&v), attn_version());
+  printf("%zu %zu %zu %zu %zu %zu %zu %zu\n", sizeof(attn_params),
+         offsetof(attn_params, dropout_p), offsetof(attn_params, dropout_offset),
+         offsetof(attn_params, dropout_seed), sizeof(attn_varlen_params),
+         offsetof(attn_varlen_params, dropout_p), offsetof(attn_varlen_params, dropout_offset),
+         offsetof(attn_varlen_params, dropout_seed));
   return 0;
 }
 """)
@@ -158,6 +178,37 @@ int main(void) {
                     f"-Wl,-rpath,{libdir}"], check=True)
     out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()
     assert out[:3] == ["0", "0", "0"]
+    # the Python mirrors of the parameter structs have the C layout
+    layout = [int(x) for x in out[6:14]]
+    A, V = attn.AttnParams, attn.AttnVarlenParams
+    assert layout == [ctypes.sizeof(A), A.dropout_p.offset, A.dropout_offset.offset,
+                      A.dropout_seed.offset, ctypes.sizeof(V), V.dropout_p.offset,
+                      V.dropout_offset.offset, V.dropout_seed.offset]
     p = P(attn, batch=2, seqlen_q=100, seqlen_k=100, nheads=8, nheads_kv=2, headdim=128)
     assert int(out[3]) == attn.attn_bwd_workspace_size(p)
     assert int(out[4]) > 0 and out[5] == attn.attn_version()
+
+
+def test_decode_host_checks(attn):
+    """attn_fwd_decode's workspace follows its split rule (about two blocks
+    per SM over the (batch, kv head) pairs, at least 256 keys per split) and
+    it refuses, before touching any pointer, more than 16 query rows per kv
+    head, head dim 256 and positional slopes."""
+    fn = attn._lib.attn_fwd_decode_workspace_size
+    fn.argtypes = [ctypes.POINTER(attn.AttnParams)]
+    fn.restype = ctypes.c_size_t
+    p = P(attn, batch=2, seqlen_q=1, seqlen_k=5000, nheads=32, nheads_kv=4)
+    splits = min(-(-296 // 8), -(-5000 // 256))  # 20
+    rows = splits * 2 * 1 * 32
+    assert fn(ctypes.byref(p)) == -(-rows * 128 * 2 // 256) * 256 + -(-rows * 4 // 256) * 256
+    call = attn._lib.attn_fwd_decode
+    vp = ctypes.c_void_p
+    call.argtypes = [ctypes.POINTER(attn.AttnParams), vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
+    call.restype = ctypes.c_int
+    too_many = P(attn, seqlen_q=5, nheads=8, nheads_kv=2)  # 4 heads x 5 tokens = 20 rows
+    assert call(ctypes.byref(too_many), None, None, None, None, None, None, 0, None) == 1
+    assert call(ctypes.byref(P(attn, headdim=256)), None, None, None, None, None, None, 0,
+                None) == 2
+    slopes = P(attn, seqlen_q=1)
+    slopes.alibi_slopes = 256
+    assert call(ctypes.byref(slopes), None, None, None, None, None, None, 0, None) == 1

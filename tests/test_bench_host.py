@@ -171,3 +171,18 @@ def test_reference_arm_line(capsys):
     assert "queries" in cpu["sample"]
     assert line["e2e"] == {"value": line["value"], "unit": bench.UNIT, "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
+
+
+def test_extra_workloads(capsys):
+    """The decode and FP8 workloads exist, read more than the L2 per step,
+    and the reference arm declines them (it times the headline only)."""
+    from attn_inputs import EXTRA_WORKLOADS
+    dec = EXTRA_WORKLOADS["decode_b8_h32_kv8_n32768_d128"]
+    assert dec.seqlen_q == 1 and dec.nheads // dec.nheads_kv * dec.seqlen_q <= 16
+    assert bench.input_bytes(dec) > 8 * 126e6
+    fp8 = EXTRA_WORKLOADS["fp8_causal_b2_h32_n8192_d128"]
+    assert (fp8.batch, fp8.nheads, fp8.seqlen_q, fp8.headdim, fp8.causal) == (2, 32, 8192, 128, True)
+    for name in EXTRA_WORKLOADS:
+        assert bench.main(["--impl", "reference", "--workload", name]) == 0
+        line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+        assert line["impl"] == "reference" and "unavailable" in line

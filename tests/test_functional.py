@@ -1,7 +1,8 @@
 """The differentiable wrappers (functional.py): their autograd plumbing on
 the CPU, with the library calls replaced by the float64 oracle (argument
 pass-through, gradient routing, the upstream gradient reaching the backward,
-LSE not differentiable, dropout refused); and the real library on the GPU."""
+LSE not differentiable, the dropout seed shared by both passes); and the real
+library on the GPU."""
 import numpy as np
 import pytest
 import torch
@@ -15,27 +16,29 @@ def fake_lib(monkeypatch):
     import io_aware_exact_33_b200 as attn
     calls = []
 
-    def fwd(q, k, v, scale, causal, wl, wr, alibi_slopes=None):
-        calls.append(("fwd", scale, causal, wl, wr, alibi_slopes))
-        o, lse = oracle.attention_fwd(q, k, v, scale, causal, wl, wr, alibi_slopes=alibi_slopes)
+    def fwd(q, k, v, scale, causal, wl, wr, alibi_slopes=None, **drop):
+        calls.append(("fwd", scale, causal, wl, wr, alibi_slopes, drop))
+        o, lse = oracle.attention_fwd(q, k, v, scale, causal, wl, wr, alibi_slopes=alibi_slopes,
+                                      **drop)
         return torch.from_numpy(o).to(q.dtype), torch.from_numpy(lse).float()
 
-    def bwd(q, k, v, o, lse, do, scale, causal, wl, wr, alibi_slopes=None):
-        calls.append(("bwd", scale, causal, wl, wr, alibi_slopes))
-        g = oracle.attention_bwd(q, k, v, do, scale, causal, wl, wr, alibi_slopes=alibi_slopes)
+    def bwd(q, k, v, o, lse, do, scale, causal, wl, wr, alibi_slopes=None, **drop):
+        calls.append(("bwd", scale, causal, wl, wr, alibi_slopes, drop))
+        g = oracle.attention_bwd(q, k, v, do, scale, causal, wl, wr, alibi_slopes=alibi_slopes,
+                                 **drop)
         return tuple(torch.from_numpy(x).to(q.dtype) for x in g)
 
-    def fwd_varlen(q, k, v, cu_q, cu_k, mq, mk, scale, causal, wl, wr, alibi_slopes=None):
-        calls.append(("fwd_varlen", mq, mk, scale, causal, wl, wr))
+    def fwd_varlen(q, k, v, cu_q, cu_k, mq, mk, scale, causal, wl, wr, alibi_slopes=None, **drop):
+        calls.append(("fwd_varlen", mq, mk, scale, causal, wl, wr, drop))
         o, lse = oracle.attention_fwd_varlen(q, k, v, cu_q, cu_k, scale, causal, wl, wr,
-                                             alibi_slopes=alibi_slopes)
+                                             alibi_slopes=alibi_slopes, **drop)
         return torch.from_numpy(o).to(q.dtype), torch.from_numpy(lse).float()
 
     def bwd_varlen(q, k, v, o, lse, do, cu_q, cu_k, mq, mk, scale, causal, wl, wr,
-                   alibi_slopes=None):
-        calls.append(("bwd_varlen", mq, mk, scale, causal, wl, wr))
+                   alibi_slopes=None, **drop):
+        calls.append(("bwd_varlen", mq, mk, scale, causal, wl, wr, drop))
         g = oracle.attention_bwd_varlen(q, k, v, do, cu_q, cu_k, scale, causal, wl, wr,
-                                        alibi_slopes=alibi_slopes)
+                                        alibi_slopes=alibi_slopes, **drop)
         return tuple(torch.from_numpy(x).to(q.dtype) for x in g)
 
     monkeypatch.setattr(attn, "attn_fwd", fwd)
@@ -84,10 +87,33 @@ def test_varlen_autograd_plumbing(fake_lib):
 def test_dropout_and_window_arguments():
     from io_aware_exact_33_b200.functional import flash_attn_func
     q = torch.zeros(1, 4, 1, 64)
-    with pytest.raises(NotImplementedError):
-        flash_attn_func(q, q, q, dropout_p=0.1)
+    with pytest.raises(ValueError):
+        flash_attn_func(q, q, q, dropout_p=1.0)
     with pytest.raises(ValueError):
         flash_attn_func(q, q, q, window_size=(-2, 0))
+
+
+def test_dropout_seed_shared_by_both_passes(fake_lib):
+    """The forward draws one seed (repeatable under torch.manual_seed) and
+    the backward gets the same seed and offset; the gradients are those of
+    the oracle with that mask."""
+    from io_aware_exact_33_b200.functional import flash_attn_func
+    w = Workload("fd", 1, 2, 1, 8, 8, 8, True, -1, -1, "bf16", 1.0, 703)
+    q, k, v, do = (_leaf(t) for t in make_inputs(w))
+    torch.manual_seed(5)
+    out = flash_attn_func(q, k, v, dropout_p=0.3, softmax_scale=0.5, causal=True)
+    (out * do.detach()).sum().backward()
+    (f, b) = fake_lib
+    assert f[0] == "fwd" and b[0] == "bwd" and f[6] == b[6]
+    drop = f[6]
+    assert drop["dropout_p"] == 0.3 and drop["dropout_offset"] == 0
+    torch.manual_seed(5)
+    out2 = flash_attn_func(q.detach(), k.detach(), v.detach(), dropout_p=0.3, softmax_scale=0.5,
+                           causal=True)
+    assert torch.equal(out.detach(), out2) and fake_lib[2][6] == drop
+    g = oracle.attention_bwd(q.detach(), k.detach(), v.detach(), do.detach(), 0.5, True, **drop)
+    for t, r in zip((q, k, v), g):
+        assert np.array_equal(t.grad.numpy(), r)
 
 
 @pytest.mark.gpu
