@@ -830,50 +830,6 @@ def run_gpu_extra(args, w):
     return 0
 
 
-PROBE_CASES = [  # (description, M, N) in the order of probe_mma_case()
-    ("A smem K-major, B smem K-major, 1 accumulator", 128, 128),
-    ("A smem K-major, B smem K-major, 2 accumulators", 128, 128),
-    ("A smem K-major, B smem K-major, 1 accumulator", 128, 64),
-    ("A smem K-major, B smem K-major, 2 accumulators", 128, 64),
-    ("A smem K-major, B smem K-major, 1 accumulator", 128, 256),
-    ("A smem MN-major, B smem MN-major, 1 accumulator", 128, 64),
-    ("A smem K-major, B smem MN-major, 1 accumulator", 128, 128),
-    ("A tmem, B smem MN-major, 1 accumulator", 128, 128),
-    ("A tmem, B smem K-major, 1 accumulator", 128, 64),
-    ("A tmem, B smem MN-major, 1 accumulator", 128, 256),
-]
-
-
-def run_probe_mma():
-    """tcgen05.mma cycles per instruction by shape / operand source (builds
-    csrc/probe_mma.cu into io_aware_exact_33_b200/libprobe_mma.so)."""
-    import ctypes
-    import torch
-    from io_aware_exact_33_b200 import build as b
-    so = os.path.join(os.path.dirname(b.LIB), "libprobe_mma.so")
-    src = os.path.join(b.CSRC, "probe_mma.cu")
-    if not os.path.exists(so) or os.path.getmtime(so) < os.path.getmtime(src):
-        subprocess.run([b.nvcc(), *b.NVCC_FLAGS, "-I", b.CSRC, "-shared", "-o", so, src], check=True)
-    lib = ctypes.CDLL(so)
-    lib.probe_mma_case.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_void_p]
-    out = torch.zeros(148, dtype=torch.int64, device="cuda")
-    iters = 4096 * 3
-    rows = []
-    for i, (desc, m, n) in enumerate(PROBE_CASES):
-        for _ in range(2):
-            rc = lib.probe_mma_case(i, iters, ctypes.c_void_p(out.data_ptr()))
-            torch.cuda.synchronize()
-        if rc != 0:
-            raise RuntimeError(f"probe case {i} failed: {rc}")
-        cyc = out.double().median().item() / iters
-        ideal = m * n * 16 / 4096.0
-        rows.append({"M": m, "N": n, "K": 16, "operands": desc, "cycles_per_mma": cyc,
-                     "ideal_cycles": ideal, "efficiency": ideal / cyc})
-        print(f"M{m} N{n} K16 {desc:48s}: {cyc:6.1f} cycles (ideal {ideal:5.1f}) "
-              f"-> {100 * ideal / cyc:5.1f}%", flush=True)
-    return rows
-
-
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -884,12 +840,7 @@ def main(argv=None):
     ap.add_argument("--workload", default=WORKLOAD,
                     help=f"attn_inputs workload to time (default {WORKLOAD}, the headline)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--probe-mma", action="store_true",
-                    help="measure tcgen05.mma throughput by shape instead of the attention step")
     args = ap.parse_args(argv)
-    if args.probe_mma:
-        run_probe_mma()
-        return 0
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     from attn_inputs import EXTRA_WORKLOADS, VARLEN_WORKLOADS, WORKLOADS

@@ -218,7 +218,9 @@ ATTN_API attn_status attn_bwd_finalize(const attn_params* p, void* dq, void* wor
  *     anything is launched.
  *   - Set-up: the first call on a device looks up that device's copy of the
  *     array (cudaGetSymbolAddress, with the device current); make that first
- *     call before any stream capture.  Later calls reuse the address.
+ *     call before any stream capture.  Later calls reuse the address, which
+ *     is kept for the life of the process: after cudaDeviceReset on a device,
+ *     this entry point must not be called on that device again.
  *   - Sharing: all calls on a device use the same array, which keeps the last
  *     call's contents; each call clears what must start at zero.  Calls that
  *     overlap on the GPU (other streams, other threads) race on the array and

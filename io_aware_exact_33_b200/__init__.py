@@ -379,15 +379,12 @@ def attn_fwd_decode(q, k, v, softmax_scale: Optional[float] = None, causal: bool
     return out, lse
 
 
-def attn_bwd(q, k, v, out, lse, dout, softmax_scale: Optional[float] = None, causal: bool = False,
-             window_left: int = -1, window_right: int = -1, dq=None, dk=None, dv=None,
-             workspace=None, stream=None, alibi_slopes=None, dropout_p: float = 0.0,
-             dropout_seed: int = 0, dropout_offset: int = 0):
-    """Gradients (dq, dk, dv) of sum(out * dout) for attention with the same
-    arguments as ``attn_fwd``; ``out`` and ``lse`` are its results."""
+def _bwd_tensors(q, k, v, out, lse, dout, dq, dk, dv):
+    """Checks every tensor of a backward call before any pointer reaches the
+    library (CUDA, contiguous, shapes, one 16-bit dtype; lse float32) and
+    allocates the gradients the caller did not pass.  Raises ValueError or
+    TypeError, so a wrong tensor never becomes an out-of-bounds access."""
     import torch
-    p = params_for(q, k, softmax_scale, causal, window_left, window_right, alibi_slopes,
-                   dropout_p, dropout_seed, dropout_offset)
     B, Nq, H, d = q.shape
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
         _check(t, n)
@@ -397,9 +394,28 @@ def attn_bwd(q, k, v, out, lse, dout, softmax_scale: Optional[float] = None, cau
     _check(out, "out", q.shape)
     _check(dout, "dout", q.shape)
     _check(lse, "lse", (B, H, Nq))
+    if lse.dtype != torch.float32:
+        raise TypeError("lse must be float32")
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
+    for t, n, shape in ((dq, "dq", q.shape), (dk, "dk", k.shape), (dv, "dv", k.shape)):
+        _check(t, n, shape)
+        if t.dtype != q.dtype:
+            raise TypeError(f"{n} must have the inputs' dtype")
+    return dq, dk, dv
+
+
+def attn_bwd(q, k, v, out, lse, dout, softmax_scale: Optional[float] = None, causal: bool = False,
+             window_left: int = -1, window_right: int = -1, dq=None, dk=None, dv=None,
+             workspace=None, stream=None, alibi_slopes=None, dropout_p: float = 0.0,
+             dropout_seed: int = 0, dropout_offset: int = 0):
+    """Gradients (dq, dk, dv) of sum(out * dout) for attention with the same
+    arguments as ``attn_fwd``; ``out`` and ``lse`` are its results."""
+    import torch
+    p = params_for(q, k, softmax_scale, causal, window_left, window_right, alibi_slopes,
+                   dropout_p, dropout_seed, dropout_offset)
+    dq, dk, dv = _bwd_tensors(q, k, v, out, lse, dout, dq, dk, dv)
     ws_bytes = attn_bwd_workspace_size(p)
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
@@ -446,12 +462,9 @@ def attn_bwd_noalloc(q, k, v, out, lse, dout, softmax_scale: Optional[float] = N
     that cannot allocate device memory at call time.  The output tensors are
     the caller's (allocated here only when not given).  Calls that overlap on
     the GPU share that scratch and must be serialised by the caller."""
-    import torch
     p = params_for(q, k, softmax_scale, causal, window_left, window_right, alibi_slopes,
                    dropout_p, dropout_seed, dropout_offset)
-    dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty_like(k) if dk is None else dk
-    dv = torch.empty_like(v) if dv is None else dv
+    dq, dk, dv = _bwd_tensors(q, k, v, out, lse, dout, dq, dk, dv)
     st = _lib.attn_bwd_noalloc(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
                                _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _stream(stream))
     if st != 0:

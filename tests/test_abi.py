@@ -212,3 +212,15 @@ def test_decode_host_checks(attn):
     slopes = P(attn, seqlen_q=1)
     slopes.alibi_slopes = 256
     assert call(ctypes.byref(slopes), None, None, None, None, None, None, 0, None) == 1
+
+
+def test_backward_wrappers_refuse_host_tensors(attn):
+    """attn_bwd and attn_bwd_noalloc check their tensors before any pointer
+    reaches the library: host tensors are refused with ValueError."""
+    import torch
+    q = torch.zeros(1, 16, 2, 64, dtype=torch.bfloat16)
+    k = torch.zeros(1, 16, 2, 64, dtype=torch.bfloat16)
+    lse = torch.zeros(1, 2, 16)
+    for fn in (attn.attn_bwd, attn.attn_bwd_noalloc):
+        with pytest.raises(ValueError, match="CUDA"):
+            fn(q, k, k, q, lse, q, 0.125)

@@ -7,15 +7,19 @@ instead of a caller workspace.
 Called here straight through the C ABI (ctypes on libattn.so) and compared
 with attn_bwd, the entry point that takes a caller workspace, on two calls in
 a row: the second call must not see the first call's leftovers in the shared
-scratch.  This file is collected last so that a run stopping at its first
-failure has already run every other test; it passes alone in a fresh process
-as well as after the others.
+scratch.  Both calls are also checked against the float64 oracle directly,
+and the Python wrapper of the same name is run once (its results against the
+oracle, its argument checks against tensors of the wrong shape or layout).
+This file is collected last so that a run stopping at its first failure has
+already run every other test; it passes alone in a fresh process as well as
+after the others.
 """
 import ctypes
 
 import pytest
 import torch
 
+import oracle
 from attn_inputs import Workload, make_inputs
 from parity import check_grad, rel_fro
 
@@ -67,6 +71,8 @@ def test_noalloc_matches_workspace_entry_point_twice(abi, w):
                       *(_ptr(t) for t in ref), _ptr(ws), ctypes.c_size_t(ws_bytes), stream)
     assert st == 0
 
+    dq_r, dk_r, dv_r = oracle.attention_bwd(*(t.cpu() for t in (q, k, v, do)), w.scale, w.causal,
+                                            w.window_left, w.window_right)
     for call in range(2):
         out = [torch.full_like(q, float("nan")), torch.full_like(k, float("nan")),
                torch.full_like(v, float("nan"))]
@@ -75,9 +81,34 @@ def test_noalloc_matches_workspace_entry_point_twice(abi, w):
         assert st == 0, f"call {call}: status {st}"
         torch.cuda.synchronize()
         assert m.attn_get_device_status() == 0
-        for name, got, want in zip(("dq", "dk", "dv"), out, ref):
+        for name, got, want, exact in zip(("dq", "dk", "dv"), out, ref, (dq_r, dk_r, dv_r)):
             check_grad(got.cpu(), want.double().cpu().numpy(), f"{w.name} call {call} {name}")
             assert rel_fro(got.cpu(), want.double().cpu().numpy()) <= 1e-2
+            check_grad(got.cpu(), exact, f"{w.name} call {call} {name} vs the oracle")
+
+
+def test_noalloc_python_wrapper(abi):
+    m, _ = abi
+    w = CASES[0]
+    q, k, v, do = (t.cuda() for t in make_inputs(w))
+    args = (w.scale, w.causal, w.window_left, w.window_right)
+    o, lse = m.attn_fwd(q, k, v, *args)
+    dq, dk, dv = m.attn_bwd_noalloc(q, k, v, o, lse, do, *args)
+    torch.cuda.synchronize()
+    assert m.attn_get_device_status() == 0
+    exact = oracle.attention_bwd(*(t.cpu() for t in (q, k, v, do)), *args)
+    for name, got, want in zip(("dq", "dk", "dv"), (dq, dk, dv), exact):
+        check_grad(got.cpu(), want, f"wrapper {name} vs the oracle")
+    # tensors of the wrong shape or layout are refused before the library sees them
+    with pytest.raises(ValueError):
+        m.attn_bwd_noalloc(q, k, v, o, lse, do, *args, dq=torch.empty_like(q)[:, :-1])
+    with pytest.raises(ValueError):
+        m.attn_bwd_noalloc(q, k, v, o, lse, do.transpose(1, 2).contiguous().transpose(1, 2),
+                           *args)
+    with pytest.raises(ValueError):
+        m.attn_bwd_noalloc(q, k, v[:, :-1].contiguous(), o, lse, do, *args)
+    with pytest.raises(ValueError):
+        m.attn_bwd_noalloc(q, k, v, o, lse[..., :-1].contiguous(), do, *args)
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch(abi):
