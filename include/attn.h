@@ -201,6 +201,31 @@ ATTN_API attn_status attn_bwd_finalize(const attn_params* p, void* dq, void* wor
                                        size_t workspace_bytes, void* stream);
 
 /*
+ * attn_bwd_accumulate with float32 key gradients added instead of written:
+ * dk_acc += softmax_scale * dS^T Q and dv_acc += P^T dout, both float32
+ * (batch, seqlen_k, nheads_kv, headdim), 16-byte aligned, caller-owned.
+ * For callers that sum the key gradients of several calls over the same
+ * keys, such as one sequence split across devices: each (query block, key
+ * block) pair is one call, and a key block's gradients are the sum over the
+ * query blocks, accumulated block by block without forming the full matrix
+ * ("What is FlashAttention", five-stage map, stage 4).  Dense batches, no
+ * dropout (ATTN_ERR_INVALID_ARG); otherwise as attn_bwd_accumulate,
+ * including its dQ share.
+ */
+ATTN_API attn_status attn_bwd_accumulate_f32(const attn_params* p, const void* q, const void* k,
+                                             const void* v, const void* dout, float* dk_acc,
+                                             float* dv_acc, void* workspace,
+                                             size_t workspace_bytes, void* stream);
+
+/*
+ * dst = src rounded to `dtype` (ATTN_BF16 or ATTN_FP16, nearest even), n
+ * elements, n a multiple of 4; src 16-byte and dst 8-byte aligned.  The
+ * last step after attn_bwd_accumulate_f32.
+ */
+ATTN_API attn_status attn_f32_to_16(const float* src, void* dst, long long n, int dtype,
+                                    void* stream);
+
+/*
  * Backward pass for callers that cannot allocate device memory.
  *
  * attn_bwd needs a caller-provided workspace.  Some callers cannot make one

@@ -31,7 +31,8 @@ EXPORTED = ("attn_fwd", "attn_bwd", "attn_bwd_prepare", "attn_bwd_accumulate", "
             "attn_status_string", "attn_get_device_status", "attn_version", "attn_bwd_noalloc",
             "attn_selftest_bounded_wait", "attn_check_varlen_params", "attn_fwd_varlen",
             "attn_fwd_e4m3", "attn_fwd_decode", "attn_fwd_decode_workspace_size",
-            "attn_bwd_varlen_workspace_size", "attn_bwd_varlen", "attn_merge")
+            "attn_bwd_varlen_workspace_size", "attn_bwd_varlen", "attn_merge",
+            "attn_bwd_accumulate_f32", "attn_f32_to_16")
 
 
 class AttnParams(ctypes.Structure):
@@ -107,6 +108,10 @@ def _load() -> ctypes.CDLL:
     lib.attn_bwd_accumulate.restype = ctypes.c_int
     lib.attn_bwd_finalize.argtypes = [P, vp, vp, sz, vp]
     lib.attn_bwd_finalize.restype = ctypes.c_int
+    lib.attn_bwd_accumulate_f32.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.attn_bwd_accumulate_f32.restype = ctypes.c_int
+    lib.attn_f32_to_16.argtypes = [vp, vp, ctypes.c_longlong, ctypes.c_int, vp]
+    lib.attn_f32_to_16.restype = ctypes.c_int
     lib.attn_bwd_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.attn_bwd_noalloc.restype = ctypes.c_int
     lib.attn_fwd_workspace_size.argtypes = [P]
@@ -443,6 +448,35 @@ def attn_bwd_accumulate(p: AttnParams, q, k, v, dout, dk, dv, workspace, stream=
                                   _stream(stream))
     if st != 0:
         raise AttnError(st, "attn_bwd_accumulate")
+
+
+def attn_bwd_accumulate_f32(p: AttnParams, q, k, v, dout, dk_acc, dv_acc, workspace,
+                            stream=None) -> None:
+    """Second backward stage with the key gradients added in float32:
+    dk_acc += scale * dS^T Q, dv_acc += P^T dout (float32 tensors of k's
+    shape), plus the dQ share into the workspace accumulator."""
+    for t, n in ((dk_acc, "dk_acc"), (dv_acc, "dv_acc")):
+        _check(t, n, k.shape)
+        if t.element_size() != 4 or not t.is_floating_point():
+            raise TypeError(f"{n} must be float32")
+    st = _lib.attn_bwd_accumulate_f32(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(dout),
+                                      _ptr(dk_acc), _ptr(dv_acc), _ptr(workspace),
+                                      ctypes.c_size_t(workspace.numel()), _stream(stream))
+    if st != 0:
+        raise AttnError(st, "attn_bwd_accumulate_f32")
+
+
+def attn_f32_to_16(src, dst, stream=None) -> None:
+    """dst (bf16 or fp16) = src (float32, same number of elements) rounded
+    to nearest even, on the GPU."""
+    _check(src, "src")
+    _check(dst, "dst")
+    if src.numel() != dst.numel() or src.element_size() != 4:
+        raise ValueError("src must be float32 with dst's number of elements")
+    st = _lib.attn_f32_to_16(_ptr(src), _ptr(dst), ctypes.c_longlong(src.numel()),
+                             _dtype_code(dst), _stream(stream))
+    if st != 0:
+        raise AttnError(st, "attn_f32_to_16")
 
 
 def attn_bwd_finalize(p: AttnParams, dq, workspace, stream=None) -> None:

@@ -201,25 +201,24 @@ def ring_attn_bwd(q, k, v, o, lse, do, softmax_scale: Optional[float] = None,
         _lib.attn_bwd_prepare(p, o[c], lse[c], do[c], w)
         ws.append(w)
         pq.append(p)
-    dk_part, dv_part = torch.empty_like(k[0]), torch.empty_like(v[0])
     kv = torch.stack((k, v))
+    # float32 dK / dV sums of the block held now; they travel round the ring
+    # one step behind their block.  The kernels add into them directly.
+    dkv = torch.zeros(kv.shape, dtype=torch.float32, device=kv.device)
     dkv_in, dkv_works = None, []
     for s in range(ring.world):
         nxt, works = None, []
         if s + 1 < ring.world:
             nxt = torch.empty_like(kv)
             works = ring.exchange(kv, nxt)
-        # dK / dV of the block held now: this rank's share first ...
-        dkv = torch.zeros(kv.shape, dtype=torch.float32, device=kv.device)
+        if s > 0:
+            # the sums of the ranks the block visited before: added onto here
+            _wait(dkv_works)
+            dkv = dkv_in
         for c, kc, cz in steps[s]:
             p = _lib.params_for(q[c], kv[0, kc], softmax_scale, cz)
-            _lib.attn_bwd_accumulate(p, q[c], kv[0, kc], kv[1, kc], do[c], dk_part, dv_part, ws[c])
-            dkv[0, kc] += dk_part
-            dkv[1, kc] += dv_part
-        # ... then the shares of the ranks the block visited before
-        if s > 0:
-            _wait(dkv_works)
-            dkv += dkv_in
+            _lib.attn_bwd_accumulate_f32(p, q[c], kv[0, kc], kv[1, kc], do[c], dkv[0, kc],
+                                         dkv[1, kc], ws[c])
         if ring.world > 1:
             dkv_in = torch.empty_like(dkv)
             dkv_works = ring.exchange(dkv, dkv_in)
@@ -232,7 +231,10 @@ def ring_attn_bwd(q, k, v, o, lse, do, softmax_scale: Optional[float] = None,
     for c in range(C):
         _lib.attn_bwd_finalize(pq[c], dq[c], ws[c])
     _wait(dkv_works)  # the last hop brings this rank's own block home
-    return dq, dkv_in[0].to(k.dtype), dkv_in[1].to(v.dtype)
+    dk, dv = torch.empty_like(k), torch.empty_like(v)
+    _lib.attn_f32_to_16(dkv_in[0], dk)
+    _lib.attn_f32_to_16(dkv_in[1], dv)
+    return dq, dk, dv
 
 
 class _RingAttn(torch.autograd.Function):

@@ -2,6 +2,7 @@
 // argument checks, TMA tensor-map construction, kernel selection and launch.
 // Every computation of the attention path runs in the kernels; this file
 // only marshals arguments.
+#include <algorithm>
 #include <climits>
 #include <cmath>
 #include <cstdlib>
@@ -104,6 +105,22 @@ bool map_f32_rows(CUtensorMap* m, const void* ptr, long long cols, long long row
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(ptr), dims, strides, box,
                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// bf16 statistics slab (rows_total, nq_pad, kSlabCols) as a 3-D map with a
+// box of kSlabCols columns (32 bytes) x `box_rows` rows x 1 and 32-byte
+// swizzle, the layout the main kernel's statistics MMA step reads.
+bool map_slab(CUtensorMap* m, const void* ptr, long long nq_pad, long long rows, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)kSlabCols, (cuuint64_t)nq_pad, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {(cuuint64_t)kSlabRowBytes, (cuuint64_t)nq_pad * kSlabRowBytes};
+  cuuint32_t box[3] = {(cuuint32_t)kSlabCols, (cuuint32_t)box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -295,15 +312,45 @@ attn_status launch_fwd_e4m3(const attn_params* p, const void* q, const void* k, 
   return finish(stream);
 }
 
-// Key splits of a decode call: about two blocks per SM over the
-// (batch, kv head) pairs, at least 256 keys per split.
-int decode_splits(const attn_params* p) {
-  const long long groups = (long long)p->batch * p->nheads_kv;
-  long long want = (2 * 148 + groups - 1) / groups;
-  const long long by_len = ((long long)p->seqlen_k + 255) / 256;
-  if (want > by_len) want = by_len;
-  if (want > 65535) want = 65535;
-  return (int)(want < 1 ? 1 : want);
+// Key tiles and splits of a decode call: the tiles of kDecodeBN keys from
+// the first key any query row sees to the last one, cut into splits so that
+// the (batch x kv head x split) blocks fill whole waves of the SMs; cost
+// model: waves x (tiles per block + 2 tiles of fixed cost).
+struct DecodeSplit {
+  int key_lo, tiles_total, splits, tiles_per_split, rmax;
+};
+DecodeSplit decode_split(const attn_params* p) {
+  DecodeSplit d;
+  const long long off = (long long)p->seqlen_k - p->seqlen_q;
+  const long long kInf = 1ll << 40;
+  const long long rb = p->causal ? 0 : (p->window_right >= 0 ? p->window_right : kInf);
+  const long long lb = p->window_left >= 0 ? p->window_left : kInf;
+  const long long lo = std::max(0ll, off - lb);
+  const long long hi = std::min((long long)p->seqlen_k - 1, (long long)p->seqlen_q - 1 + off + rb);
+  d.key_lo = (int)std::min(lo, (long long)p->seqlen_k);
+  d.tiles_total = hi >= lo ? (int)((hi - lo + kDecodeBN) / kDecodeBN) : 0;
+  const int rows = (p->nheads / p->nheads_kv) * p->seqlen_q;
+  d.rmax = rows <= 4 ? 4 : (rows <= 8 ? 8 : 16);
+  int sms = 148, dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long slots = (long long)sms * (d.rmax <= 8 ? 2 : 1);
+  const long long pairs = (long long)p->batch * p->nheads_kv;
+  d.splits = 1;
+  d.tiles_per_split = std::max(d.tiles_total, 1);
+  long long best = -1;
+  for (int s = 1; s <= std::min(d.tiles_total, 4096); ++s) {
+    const int tps = (d.tiles_total + s - 1) / s;
+    const int s_eff = (d.tiles_total + tps - 1) / tps;  // no empty splits
+    const long long waves = (pairs * s_eff + slots - 1) / slots;
+    const long long cost = waves * (tps + 2);
+    if (best < 0 || cost < best) {
+      best = cost;
+      d.splits = s_eff;
+      d.tiles_per_split = tps;
+    }
+  }
+  return d;
 }
 
 // Workspace of a decode call: the splits' 16-bit partial outputs, then
@@ -312,7 +359,7 @@ struct DecodeWorkspace {
   size_t o_bytes, total;
 };
 DecodeWorkspace decode_layout(const attn_params* p) {
-  const size_t rows = (size_t)decode_splits(p) * p->batch * p->seqlen_q * p->nheads;
+  const size_t rows = (size_t)decode_split(p).splits * p->batch * p->seqlen_q * p->nheads;
   DecodeWorkspace w;
   w.o_bytes = (rows * p->headdim * 2 + 255) / 256 * 256;
   w.total = w.o_bytes + (rows * 4 + 255) / 256 * 256;
@@ -322,12 +369,14 @@ DecodeWorkspace decode_layout(const attn_params* p) {
 template <int D, bool FP16>
 attn_status launch_decode(const attn_params* p, const void* q, const void* k, const void* v,
                           void* o, float* lse, void* workspace, cudaStream_t stream) {
-  const int splits = decode_splits(p);
+  const DecodeSplit ds = decode_split(p);
   const DecodeWorkspace ws = decode_layout(p);
+  CUtensorMap mk, mv;
+  if (!map_bshd(&mk, k, FP16, p->batch, p->seqlen_k, p->nheads_kv, D, kDecodeBN) ||
+      !map_bshd(&mv, v, FP16, p->batch, p->seqlen_k, p->nheads_kv, D, kDecodeBN))
+    return ATTN_ERR_CUDA;
   DecodeParams dp;
   dp.q = static_cast<const uint16_t*>(q);
-  dp.k = static_cast<const uint16_t*>(k);
-  dp.v = static_cast<const uint16_t*>(v);
   dp.o_parts = static_cast<uint16_t*>(workspace);
   dp.lse_parts = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + ws.o_bytes);
   dp.batch = p->batch;
@@ -339,15 +388,20 @@ attn_status launch_decode(const attn_params* p, const void* q, const void* k, co
   dp.window_left = p->window_left;
   dp.window_right = p->window_right;
   dp.scale_log2 = p->softmax_scale * 1.4426950408889634f;
-  dp.splits = splits;
-  dp.chunk = (int)((((long long)p->seqlen_k + splits - 1) / splits + 31) / 32 * 32);
-  auto kern = attn_decode_kernel<D, FP16>;
-  if (!ensure_smem(reinterpret_cast<const void*>(kern), DecodeSmem<D>::BYTES)) return ATTN_ERR_CUDA;
-  const dim3 grid((unsigned)(p->batch * p->nheads_kv), (unsigned)splits);  // splits <= 65535
-  kern<<<grid, kDecodeWarps * 32, DecodeSmem<D>::BYTES, stream>>>(dp);
+  dp.splits = ds.splits;
+  dp.key_lo = ds.key_lo;
+  dp.tiles_per_split = ds.tiles_per_split;
+  dp.tiles_total = ds.tiles_total;
+  auto kern = ds.rmax == 4 ? attn_decode_kernel<D, FP16, 4>
+                           : (ds.rmax == 8 ? attn_decode_kernel<D, FP16, 8>
+                                           : attn_decode_kernel<D, FP16, 16>);
+  if (!ensure_smem(reinterpret_cast<const void*>(kern), DecodeCfg<D>::SMEM_BYTES))
+    return ATTN_ERR_CUDA;
+  const dim3 grid((unsigned)(p->batch * p->nheads_kv), (unsigned)ds.splits);  // splits <= 4096
+  kern<<<grid, kDecodeThreads, DecodeCfg<D>::SMEM_BYTES, stream>>>(mk, mv, dp);
   const attn_status st = finish(stream);
   if (st != ATTN_OK) return st;
-  const attn_merge_params mp = {splits, p->batch, p->seqlen_q, p->nheads, p->headdim, p->dtype};
+  const attn_merge_params mp = {ds.splits, p->batch, p->seqlen_q, p->nheads, p->headdim, p->dtype};
   return attn_merge(&mp, dp.o_parts, dp.lse_parts, o, lse, stream);
 }
 
@@ -365,6 +419,7 @@ BwdParams bwd_params(const attn_params* p, const float* lse, void* workspace, co
   bp.total_q = pk.total_q;
   bp.total_k = pk.total_k;
   bp.dk = bp.dv = nullptr;
+  bp.acc_f32 = 0;
   bp.alibi = p->alibi_slopes;
   const uint32_t t = drop_threshold(p->dropout_p);
   bp.drop_seed = p->dropout_seed;
@@ -375,6 +430,10 @@ BwdParams bwd_params(const attn_params* p, const float* lse, void* workspace, co
   bp.lse = lse;
   bp.dvec = reinterpret_cast<float*>(w + ws.dvec_off);
   bp.lse2 = reinterpret_cast<float*>(w + ws.lse2_off);
+  bp.lse_slab = reinterpret_cast<uint16_t*>(w + ws.lsb_off);
+  bp.dvec_slab = reinterpret_cast<uint16_t*>(w + ws.dvb_off);
+  // bf16 without dropout: the main kernel folds the statistics into its MMAs
+  bp.fold = (p->dtype == ATTN_BF16 && t == 0) ? 1 : 0;
   bp.dq_acc = reinterpret_cast<float*>(w + ws.dq_off);
   bp.batch = p->batch;
   bp.nheads = p->nheads;
@@ -413,7 +472,8 @@ attn_status launch_bwd_prepare(const attn_params* p, const void* o, const float*
 template <class C>
 attn_status launch_bwd_main(const attn_params* p, const void* q, const void* k, const void* v,
                             const void* dout, void* dk, void* dv, void* workspace,
-                            cudaStream_t stream, const Packed& pk = Packed()) {
+                            cudaStream_t stream, const Packed& pk = Packed(),
+                            bool acc_f32 = false) {
   const BwdParams bp = bwd_params(p, nullptr, workspace, pk);
   const bool fp16 = C::FP16;
   const int mb = pk.on() ? 1 : p->batch;
@@ -424,16 +484,21 @@ attn_status launch_bwd_main(const attn_params* p, const void* q, const void* k, 
       !map_bshd(&mk, k, fp16, mb, nk, p->nheads_kv, C::D, C::BN) ||
       !map_bshd(&mv, v, fp16, mb, nk, p->nheads_kv, C::D, C::BN) ||
       !map_bshd(&mdo, dout, fp16, mb, nq, p->nheads, C::D, C::BM) ||
-      !map_f32_rows(&ml, bp.lse2, bp.nq_pad, stat_rows, C::BM) ||
-      !map_f32_rows(&md, bp.dvec, bp.nq_pad, stat_rows, C::BM) ||
-      !map_bshd(&mdk, dk, fp16, mb, nk, p->nheads_kv, C::D, C::BN) ||
-      !map_bshd(&mdv, dv, fp16, mb, nk, p->nheads_kv, C::D, C::BN) ||
+      !(bp.fold ? map_slab(&ml, bp.lse_slab, bp.nq_pad, stat_rows, C::BM)
+                : map_f32_rows(&ml, bp.lse2, bp.nq_pad, stat_rows, C::BM)) ||
+      !(bp.fold ? map_slab(&md, bp.dvec_slab, bp.nq_pad, stat_rows, C::BM)
+                : map_f32_rows(&md, bp.dvec, bp.nq_pad, stat_rows, C::BM)) ||
+      !(acc_f32 ? map_bshd_f32_32x32(&mdk, dk, mb, nk, p->nheads_kv, C::D)
+                : map_bshd(&mdk, dk, fp16, mb, nk, p->nheads_kv, C::D, C::BN)) ||
+      !(acc_f32 ? map_bshd_f32_32x32(&mdv, dv, mb, nk, p->nheads_kv, C::D)
+                : map_bshd(&mdv, dv, fp16, mb, nk, p->nheads_kv, C::D, C::BN)) ||
       !map_bshd_f32_32x32(&mdq, bp.dq_acc, mb, pk.on() ? (int)bp.nq_pad : p->seqlen_q,
                           p->nheads, C::D))
     return ATTN_ERR_CUDA;
   BwdParams bpl = bp;
-  bpl.dk = static_cast<uint16_t*>(dk);
-  bpl.dv = static_cast<uint16_t*>(dv);
+  bpl.dk = acc_f32 ? nullptr : static_cast<uint16_t*>(dk);
+  bpl.dv = acc_f32 ? nullptr : static_cast<uint16_t*>(dv);
+  bpl.acc_f32 = acc_f32 ? 1 : 0;
   bpl.num_kblocks = (p->seqlen_k + C::BN - 1) / C::BN;
   const int heads = p->batch * p->nheads_kv;
   // bytes of Q, dO (16-bit) and the fp32 dQ accumulator each kv head's
@@ -527,15 +592,19 @@ attn_status dispatch_fwd(const attn_params* p, const void* q, const void* k, con
 
 attn_status dispatch_bwd_main(const attn_params* p, const void* q, const void* k, const void* v,
                               const void* dout, void* dk, void* dv, void* workspace,
-                              cudaStream_t stream, const Packed& pk) {
+                              cudaStream_t stream, const Packed& pk, bool acc_f32 = false) {
   const bool fp16 = p->dtype == ATTN_FP16;
   switch (p->headdim) {
     case 64:
-      return fp16 ? launch_bwd_main<BwdCfg<64, true>>(p, q, k, v, dout, dk, dv, workspace, stream, pk)
-                  : launch_bwd_main<BwdCfg<64, false>>(p, q, k, v, dout, dk, dv, workspace, stream, pk);
+      return fp16 ? launch_bwd_main<BwdCfg<64, true>>(p, q, k, v, dout, dk, dv, workspace, stream,
+                                                      pk, acc_f32)
+                  : launch_bwd_main<BwdCfg<64, false>>(p, q, k, v, dout, dk, dv, workspace, stream,
+                                                       pk, acc_f32);
     case 128:
-      return fp16 ? launch_bwd_main<BwdCfg<128, true>>(p, q, k, v, dout, dk, dv, workspace, stream, pk)
-                  : launch_bwd_main<BwdCfg<128, false>>(p, q, k, v, dout, dk, dv, workspace, stream, pk);
+      return fp16 ? launch_bwd_main<BwdCfg<128, true>>(p, q, k, v, dout, dk, dv, workspace, stream,
+                                                       pk, acc_f32)
+                  : launch_bwd_main<BwdCfg<128, false>>(p, q, k, v, dout, dk, dv, workspace, stream,
+                                                        pk, acc_f32);
     default:
       return ATTN_ERR_UNSUPPORTED_HEADDIM;
   }
@@ -742,6 +811,36 @@ attn_status attn_bwd_accumulate(const attn_params* p, const void* q, const void*
     return ATTN_ERR_MISALIGNED;
   return dispatch_bwd_main(p, q, k, v, dout, dk, dv, workspace,
                            reinterpret_cast<cudaStream_t>(stream_), Packed());
+}
+
+attn_status attn_bwd_accumulate_f32(const attn_params* p, const void* q, const void* k,
+                                    const void* v, const void* dout, float* dk_acc, float* dv_acc,
+                                    void* workspace, size_t workspace_bytes, void* stream_) {
+  bool empty = false;
+  attn_status st = bwd_common_checks(p, workspace, workspace_bytes, &empty);
+  if (st != ATTN_OK || empty) return st;
+  if (drop_threshold(p->dropout_p) != 0) return ATTN_ERR_INVALID_ARG;
+  if (!q || !k || !v || !dout || !dk_acc || !dv_acc) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dk_acc) ||
+      !aligned16(dv_acc))
+    return ATTN_ERR_MISALIGNED;
+  return dispatch_bwd_main(p, q, k, v, dout, dk_acc, dv_acc, workspace,
+                           reinterpret_cast<cudaStream_t>(stream_), Packed(), true);
+}
+
+attn_status attn_f32_to_16(const float* src, void* dst, long long n, int dtype, void* stream_) {
+  if (n < 0 || (dtype != ATTN_BF16 && dtype != ATTN_FP16)) return ATTN_ERR_INVALID_ARG;
+  if (n == 0) return ATTN_OK;
+  if (!src || !dst || (n & 3)) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(src) || (reinterpret_cast<uintptr_t>(dst) & 7u)) return ATTN_ERR_MISALIGNED;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  BwdParams bp;
+  std::memset(&bp, 0, sizeof(bp));  // cu_q == nullptr: a plain element-wise conversion
+  if (dtype == ATTN_FP16)
+    bwd_convert<true><<<2368, 256, 0, stream>>>(src, static_cast<uint16_t*>(dst), n / 4, 1.f, bp);
+  else
+    bwd_convert<false><<<2368, 256, 0, stream>>>(src, static_cast<uint16_t*>(dst), n / 4, 1.f, bp);
+  return finish(stream);
 }
 
 attn_status attn_bwd_finalize(const attn_params* p, void* dq, void* workspace,

@@ -17,20 +17,20 @@
 //   bwd_convert     dQ = scale * accumulator, rounded to the input dtype.
 //
 // Main kernel roles (320 threads):
-//   warp 8      TMA producer: K_j, V_j once; Q_i, dO_i, LSE2_i, Dvec_i per
-//               query tile through a three-slot ring.
-//   warp 9      TMEM allocation; lane 0 issues the five MMAs per tile:
-//               S^T = K Q^T, dP^T = V dO^T, dV += P^T dO, dK += dS^T Q, and
-//               dQ^T = K^T dS^T (d = 128) or dQ = dS K (d = 64).  With two
-//               buffers it issues tile t+1's S^T and dP^T before tile t's
-//               gradient MMAs, so the tensor pipe works on one tile while
-//               warps 0-3 exponentiate the other.
+//   warp 8      TMA producer: K_j, V_j once; Q_i (with its LSE2 statistics)
+//               and dO_i (with Dvec) per query tile through rings of their own.
+//   warp 9      TMEM allocation; issues the five MMAs per tile (one elected
+//               lane): S^T = K Q^T, dP^T = V dO^T, dV += P^T dO, dK += dS^T Q,
+//               and dQ^T = K^T dS^T (d = 128) or dQ = dS K (d = 64).  With two
+//               buffers it issues tile t+1's S^T before tile t's gradient
+//               MMAs and its dP^T after them, so the tensor pipe works on one
+//               tile while the compute warps exponentiate the other.
 //   warps 0-7   two warps per tensor-memory lane quadrant (one thread per key
 //               row), each owning half of the tile's query columns:
 //               P^T = exp2(S^T*scale*log2e - LSE2) back into tensor memory as
-//               the 16-bit A operand of dV; dS = P o (dP - Dvec) into shared
-//               memory, where it is the K-major A operand of dK and an
-//               MN-major operand of dQ; then the previous tile's dQ block
+//               the 16-bit A operand of dV; dS = P o (dP - Dvec) into tensor
+//               memory beside it (the A operand of dK) and into shared
+//               memory (an MN-major operand of dQ); then the previous tile's dQ block
 //               (which reuses that tile's dP block) out of tensor memory into
 //               the fp32 accumulator with a TMA reduce-add per warp (other
 //               key tiles add to the same rows); finally dK, dV out through
@@ -45,25 +45,42 @@
 namespace attn {
 
 struct BwdWorkspace {
-  size_t dvec_off, lse2_off, dq_off, total;
+  size_t dvec_off, lse2_off, lsb_off, dvb_off, dq_off, total;
   long long nq_pad;
 };
 
 __host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Per-query statistics of one padded query row in the form the main kernel's
+// MMAs take them (bf16 kernels without dropout): 16 bf16 values, the first
+// three a split v = hi + mid + lo of the value that the extra K = 16 step of
+// the S^T (v = -LSE2 / (scale log2 e)) or dP^T (v = -Dvec) product adds to
+// every key row; the rest zero.
+constexpr int kSlabCols = 16;
+constexpr int kSlabRowBytes = kSlabCols * 2;
+
+// The arrays after the fp32 Dvec / LSE2 rows (rows = statistics rows, each
+// nq_pad long): the two bf16 slabs, then the fp32 dQ accumulator.
+__host__ __device__ inline void bwd_workspace_tail(BwdWorkspace& w, size_t stat_rows,
+                                                   size_t acc_elems) {
+  const size_t rows4 = stat_rows * (size_t)w.nq_pad * 4;
+  w.dvec_off = 0;
+  w.lse2_off = align_up(rows4, 256);
+  w.lsb_off = w.lse2_off + align_up(rows4, 256);
+  w.dvb_off = w.lsb_off + align_up(stat_rows * (size_t)w.nq_pad * kSlabRowBytes, 256);
+  w.dq_off = w.dvb_off + align_up(stat_rows * (size_t)w.nq_pad * kSlabRowBytes, 256);
+  w.total = w.dq_off + align_up(acc_elems * 4, 256);
+}
+
 // Workspace: Dvec and LSE2 as (batch*nheads, nq_pad) fp32 with nq_pad a
-// multiple of 128 (TMA-aligned rows), then the fp32 dQ accumulator
-// (batch, seqlen_q, nheads, headdim).  Packed sequences: see
-// bwd_workspace_layout_packed.
+// multiple of 128 (TMA-aligned rows), their bf16 slabs (batch*nheads,
+// nq_pad, 16), then the fp32 dQ accumulator (batch, seqlen_q, nheads,
+// headdim).  Packed sequences: see bwd_workspace_layout_packed.
 __host__ __device__ inline BwdWorkspace bwd_workspace_layout(int batch, int nheads, int seqlen_q,
                                                             int headdim) {
   BwdWorkspace w;
   w.nq_pad = ((long long)seqlen_q + 127) / 128 * 128;
-  const size_t rows = (size_t)batch * nheads * (size_t)w.nq_pad * 4;
-  w.dvec_off = 0;
-  w.lse2_off = align_up(rows, 256);
-  w.dq_off = w.lse2_off + align_up(rows, 256);
-  w.total = w.dq_off + align_up((size_t)batch * seqlen_q * nheads * headdim * 4, 256);
+  bwd_workspace_tail(w, (size_t)batch * nheads, (size_t)batch * seqlen_q * nheads * headdim);
   return w;
 }
 
@@ -71,8 +88,9 @@ __host__ __device__ inline BwdWorkspace bwd_workspace_layout(int batch, int nhea
 // packed_row0(cu_q[b], b) = align4(cu_q[b]) + 136 b, a multiple of 4 (TMA
 // alignment of the fp32 rows) with >= 128 rows of slack after every sequence,
 // so a query tile that ends past its sequence reads and adds only slack rows.
-// Dvec and LSE2 are (nheads, nq_pad) and the dQ accumulator is
-// (nq_pad, nheads, headdim), nq_pad = packed_rows(total_q, batch).
+// Dvec and LSE2 are (nheads, nq_pad), the slabs (nheads, nq_pad, 16) and the
+// dQ accumulator is (nq_pad, nheads, headdim), nq_pad = packed_rows(total_q,
+// batch).
 __host__ __device__ inline long long packed_row0(int cu_b, int b) {
   return (((long long)cu_b + 3) & ~3ll) + 136ll * b;
 }
@@ -83,11 +101,7 @@ __host__ __device__ inline BwdWorkspace bwd_workspace_layout_packed(int total_q,
                                                                    int nheads, int headdim) {
   BwdWorkspace w;
   w.nq_pad = packed_rows(total_q, batch);
-  const size_t rows = (size_t)nheads * (size_t)w.nq_pad * 4;
-  w.dvec_off = 0;
-  w.lse2_off = align_up(rows, 256);
-  w.dq_off = w.lse2_off + align_up(rows, 256);
-  w.total = w.dq_off + align_up((size_t)w.nq_pad * nheads * headdim * 4, 256);
+  bwd_workspace_tail(w, (size_t)nheads, (size_t)w.nq_pad * nheads * headdim);
   return w;
 }
 
@@ -95,6 +109,11 @@ struct BwdParams {
   const float* lse;
   float* dvec;
   float* lse2;
+  // bf16 slabs of -LSE2 / scale_log2 and -Dvec (kSlabCols per padded row),
+  // written instead of dvec / lse2 when `fold` is set (bf16, no dropout).
+  uint16_t* lse_slab;
+  uint16_t* dvec_slab;
+  int fold;
   float* dq_acc;
   int batch, nheads, nheads_kv, seqlen_q, seqlen_k, headdim;
   int causal, window_left, window_right;
@@ -113,6 +132,10 @@ struct BwdParams {
   int total_q, total_k;
   uint16_t* dk;
   uint16_t* dv;
+  // When set, tm_dk / tm_dv map float32 (batch, seqlen_k, nheads_kv, headdim)
+  // buffers and the epilogue adds dK (x scale) and dV into them (TMA
+  // reduce-add) instead of storing them in the input dtype; dense only.
+  int acc_f32;
   // Per-head positional slopes (nheads floats), or nullptr: scores gain
   // -slope_h * |i + seqlen_k - seqlen_q - j| (kernel instantiated with ALIBI).
   const float* alibi;
@@ -171,9 +194,27 @@ __device__ __forceinline__ float dot8(uint4 a, uint4 b) {
   return acc;
 }
 
+// bf16 bits of x, round to nearest even.
+__device__ __forceinline__ uint32_t bf16_bits(float x) { return pack2<false>(x, 0.f) & 0xFFFFu; }
+
+// One slab row: x split into three bf16 values hi + mid + lo (each the
+// bf16 rounding of what the previous ones leave; the differences are exact
+// in fp32, so the sum carries 24 significant bits), then 13 zeros.
+__device__ __forceinline__ void write_slab_row(uint16_t* dst, float x) {
+  const uint32_t hi = bf16_bits(x);
+  const float r1 = x - __uint_as_float(hi << 16);
+  const uint32_t mid = bf16_bits(r1);
+  const float r2 = r1 - __uint_as_float(mid << 16);
+  const uint32_t lo = bf16_bits(r2);
+  uint4* d = reinterpret_cast<uint4*>(dst);
+  d[0] = make_uint4(hi | (mid << 16), lo, 0u, 0u);
+  d[1] = make_uint4(0u, 0u, 0u, 0u);
+}
+
 // Rows of the padded (b, h, i) range, headdim / 8 lanes per row with one
 // 16-byte load of O and of dO each: Dvec_i = sum_c dO_ic O_ic and
-// LSE2_i = LSE_i * log2(e); padding rows get 0 and +inf (P = 0 there).  All
+// LSE2_i = LSE_i * log2(e); padding rows get 0 and +inf (P = 0 there).  With
+// p.fold the same values go to the bf16 slabs instead (write_slab_row).  All
 // threads then zero the dQ accumulator.
 template <bool FP16>
 __global__ void __launch_bounds__(256) bwd_preprocess(const uint16_t* __restrict__ o,
@@ -224,8 +265,16 @@ __global__ void __launch_bounds__(256) bwd_preprocess(const uint16_t* __restrict
                                : p.lse[((size_t)b * p.nheads + h) * p.seqlen_q + i];
         l2 = (l == -INFINITY) ? INFINITY : l * 1.4426950408889634f;
       }
-      p.dvec[row] = valid ? acc : 0.f;
-      p.lse2[row] = l2;
+      if (p.fold) {
+        // Rows with no visible key or past the sequence get 0: the main
+        // kernel masks every one of their elements.
+        const float x = (valid && l2 != INFINITY) ? -l2 / p.scale_log2 : 0.f;
+        write_slab_row(p.lse_slab + (size_t)row * kSlabCols, x);
+        write_slab_row(p.dvec_slab + (size_t)row * kSlabCols, valid ? -acc : 0.f);
+      } else {
+        p.dvec[row] = valid ? acc : 0.f;
+        p.lse2[row] = l2;
+      }
     }
   }
   float4* z = reinterpret_cast<float4*>(p.dq_acc);
@@ -266,6 +315,25 @@ __global__ void __launch_bounds__(256) bwd_convert(const float* __restrict__ acc
 // for S/P and dP/dQ, so the MMAs of one query tile overlap the exponentials
 // of the next.  d = 64: BM = 128 and one buffer (the dQ MMA would otherwise
 // need M = 64).
+//
+// Q and dO have rings of their own: three Q slots, and for d = 128 two dO
+// slots.  The MMA warp issues tile t+1's S^T before tile t's gradient MMAs
+// and tile t+1's dP^T after them, so a dO slot is refilled one tile after it
+// is released (the dP^T of tile t+1 is needed only once the compute warps
+// have finished P_{t+1} and drained dQ_t).
+//
+// Statistics folded into the MMAs (bf16 kernels without dropout): the
+// per-query values LSE2_i and Dvec_i would otherwise be read by every thread
+// (one key row each) for every query column, 64 KB of shared-memory
+// broadcast per 64-query tile.  Instead each S^T and dP^T product takes one
+// more K = 16 step: A = a ones block (128 key rows x 16, columns {0, 1, 2,
+// 8, 9, 10} one), B = the query tile's slab (its rows hold a three-way bf16
+// split of -LSE2_i / (scale log2 e), resp. -Dvec_i, in columns 0-2, zeros
+// elsewhere).  The accumulators then hold S - LSE2/(scale log2 e) and
+// dP - Dvec, so P = exp2(acc * scale * log2 e) and dS = P o acc.  The ones
+// rows are all equal and each 16-byte half of a row holds the same values,
+// so the 32-byte swizzle (which only exchanges the halves of a row) leaves
+// the block unchanged.
 template <int D_, bool FP16_>
 struct BwdCfg {
   static constexpr int D = D_;
@@ -275,6 +343,7 @@ struct BwdCfg {
   static constexpr int NBUF = (D == 128) ? 2 : 1;
   static constexpr bool DQT = (D == 128);  // dQ^T = K^T dS^T (M = d), else dQ = dS K (M = BM)
   static constexpr int QSTAGES = 3;
+  static constexpr int DOSTAGES = (D == 128) ? 2 : 3;
   static constexpr int NBOX = D / 64;
   static constexpr int NQB = BM / 64;
   static constexpr int HW = BM / 2;  // query columns per compute warp
@@ -283,23 +352,29 @@ struct BwdCfg {
   static constexpr int KV_BYTES = BN * D * 2;
   static constexpr int Q_BYTES = BM * D * 2;
   static constexpr int DS_BYTES = BN * BM * 2;
+  static constexpr int SLAB_BYTES = BM * kSlabRowBytes;  // one tile's statistics slab
+  static constexpr int ONES_BYTES = BN * kSlabRowBytes;
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + KV_BYTES;
   static constexpr int OFF_Q = OFF_V + KV_BYTES;
   static constexpr int OFF_DO = OFF_Q + QSTAGES * Q_BYTES;
-  static constexpr int OFF_DS = OFF_DO + QSTAGES * Q_BYTES;
+  static constexpr int OFF_DS = OFF_DO + DOSTAGES * Q_BYTES;
   // dQ staging: one 4 KB box (32 x 32 fp32, 128-byte swizzle) per compute warp
   static constexpr int DQS_BYTES = 32 * 32 * 4;
   static constexpr int OFF_DQS = OFF_DS + NBUF * DS_BYTES;
-  static constexpr int OFF_LSE = OFF_DQS + 8 * DQS_BYTES;
-  static constexpr int OFF_DVEC = OFF_LSE + QSTAGES * BM * 4;
-  static constexpr int OFF_BAR = OFF_DVEC + QSTAGES * BM * 4;
+  static constexpr int OFF_LSB = OFF_DQS + 8 * DQS_BYTES;  // -LSE2 slabs, one per Q slot
+  static constexpr int OFF_DVB = OFF_LSB + QSTAGES * SLAB_BYTES;  // -Dvec slabs, per dO slot
+  static constexpr int OFF_ONES = OFF_DVB + DOSTAGES * SLAB_BYTES;
+  static constexpr int OFF_LSE = OFF_ONES + ONES_BYTES;  // fp32 LSE2, per Q slot (no fold)
+  static constexpr int OFF_DVEC = OFF_LSE + QSTAGES * BM * 4;  // fp32 Dvec, per dO slot
+  static constexpr int OFF_BAR = OFF_DVEC + DOSTAGES * BM * 4;
   // barriers
   static constexpr int B_KV = 0;
   static constexpr int B_QFULL = 1;
   static constexpr int B_DOFULL = B_QFULL + QSTAGES;
-  static constexpr int B_EMPTY = B_DOFULL + QSTAGES;
-  static constexpr int B_SFULL = B_EMPTY + QSTAGES;   // per buffer
+  static constexpr int B_QEMPTY = B_DOFULL + DOSTAGES;
+  static constexpr int B_DOEMPTY = B_QEMPTY + QSTAGES;
+  static constexpr int B_SFULL = B_DOEMPTY + DOSTAGES;  // per buffer
   static constexpr int B_DPFULL = B_SFULL + NBUF;
   static constexpr int B_PREADY = B_DPFULL + NBUF;    // 256 arrivals
   static constexpr int B_DSREADY = B_PREADY + NBUF;   // 256 arrivals
@@ -316,7 +391,9 @@ struct BwdCfg {
   static constexpr int THREADS = 320;
   static_assert(TM_DP + NBUF * BM <= TMEM_COLS, "tensor memory");
   static_assert(DQT || D <= BM, "dQ block fits its dP block");
-  static_assert(QSTAGES * Q_BYTES >= BN * D * 2, "epilogue staging");
+  static_assert(QSTAGES * Q_BYTES >= BN * D * 2, "dK epilogue staging");
+  static_assert(DOSTAGES * Q_BYTES >= BN * D * 2, "dV epilogue staging");
+  static_assert(OFF_LSB % 1024 == 0 && SLAB_BYTES % 256 == 0, "32-byte swizzle atoms");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
 
@@ -328,6 +405,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
                     const __grid_constant__ CUtensorMap tm_dqacc, const BwdParams pin) {
   constexpr int D = C::D, BN = C::BN, BM = C::BM, NBUF = C::NBUF, QS = C::QSTAGES;
+  constexpr int DS = C::DOSTAGES;
+  // tm_lse2 / tm_dvec are the slab maps when FOLD, the fp32 row maps otherwise
+  constexpr bool FOLD = !C::FP16 && !DROP;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t smem0 = (smem_addr(smem_raw) + 1023u) & ~1023u;
   uint8_t* smem_gen = smem_raw + (smem0 - smem_addr(smem_raw));
@@ -367,25 +447,48 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   const int nqb = imax >= imin ? (int)(imax / BM) - qb_lo + 1 : 0;
   const int nt = nqb * group;  // tiles: (head in group) x (query tile)
 
-  // Q, LSE2, dO, Dvec of tile t (query head, query tile) into its slot.
+  // Statistics coordinates of tile t: query head, first query row, the row
+  // of the statistics arrays ((padded row, head) packed, (row, batch*head)
+  // dense) and its column.
+  auto tile_stat = [&](int t, int& h, int& q0, int& row, int& xs) {
+    h = kvh * group + t / nqb;
+    q0 = (qb_lo + t % nqb) * BM;
+    row = p.cu_q ? h : b * p.nheads + h;
+    xs = (int)prow0 + q0;
+  };
+  // Q_t (and its LSE2 statistics) into Q slot t % QS.
   auto load_q = [&](int t) -> bool {
     const int slot = t % QS, n = t / QS;
-    if (n > 0 && !mbar_wait(bar(C::B_EMPTY + slot), (n - 1) & 1)) return false;
-    const int h = kvh * group + t / nqb;
-    const int q0 = (qb_lo + t % nqb) * BM;
-    // Dvec / LSE2 coordinates: (padded row, head) packed, (row, batch*head) dense
-    const int row = p.cu_q ? h : b * p.nheads + h;
-    const int xs = (int)prow0 + q0;
-    mbar_arrive_expect_tx(bar(C::B_QFULL + slot), C::Q_BYTES + BM * 4);
+    if (n > 0 && !mbar_wait(bar(C::B_QEMPTY + slot), (n - 1) & 1)) return false;
+    int h, q0, row, xs;
+    tile_stat(t, h, q0, row, xs);
+    mbar_arrive_expect_tx(bar(C::B_QFULL + slot), C::Q_BYTES + (FOLD ? C::SLAB_BYTES : BM * 4));
     for (int bx = 0; bx < C::NBOX; ++bx)
       tma_load_4d(smem0 + C::OFF_Q + slot * C::Q_BYTES + bx * (BM * 128), &tm_q,
                   bar(C::B_QFULL + slot), bx * 64, h, sq.q_row0 + q0, sq.tma_b);
-    tma_load_2d(smem0 + C::OFF_LSE + slot * BM * 4, &tm_lse2, bar(C::B_QFULL + slot), xs, row);
-    mbar_arrive_expect_tx(bar(C::B_DOFULL + slot), C::Q_BYTES + BM * 4);
+    if constexpr (FOLD)
+      tma_load_3d(smem0 + C::OFF_LSB + slot * C::SLAB_BYTES, &tm_lse2, bar(C::B_QFULL + slot), 0,
+                  xs, row);
+    else
+      tma_load_2d(smem0 + C::OFF_LSE + slot * BM * 4, &tm_lse2, bar(C::B_QFULL + slot), xs, row);
+    return true;
+  };
+  // dO_t (and its Dvec statistics) into dO slot t % DS.
+  auto load_do = [&](int t) -> bool {
+    const int slot = t % DS, n = t / DS;
+    if (n > 0 && !mbar_wait(bar(C::B_DOEMPTY + slot), (n - 1) & 1)) return false;
+    int h, q0, row, xs;
+    tile_stat(t, h, q0, row, xs);
+    mbar_arrive_expect_tx(bar(C::B_DOFULL + slot), C::Q_BYTES + (FOLD ? C::SLAB_BYTES : BM * 4));
     for (int bx = 0; bx < C::NBOX; ++bx)
       tma_load_4d(smem0 + C::OFF_DO + slot * C::Q_BYTES + bx * (BM * 128), &tm_do,
                   bar(C::B_DOFULL + slot), bx * 64, h, sq.q_row0 + q0, sq.tma_b);
-    tma_load_2d(smem0 + C::OFF_DVEC + slot * BM * 4, &tm_dvec, bar(C::B_DOFULL + slot), xs, row);
+    if constexpr (FOLD)
+      tma_load_3d(smem0 + C::OFF_DVB + slot * C::SLAB_BYTES, &tm_dvec, bar(C::B_DOFULL + slot),
+                  0, xs, row);
+    else
+      tma_load_2d(smem0 + C::OFF_DVEC + slot * BM * 4, &tm_dvec, bar(C::B_DOFULL + slot), xs,
+                  row);
     return true;
   };
 
@@ -408,7 +511,16 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         tma_load_4d(smem0 + C::OFF_V + bx * (BN * 128), &tm_v, bar(C::B_KV), bx * 64, kvh,
                     sq.k_row0 + k0, sq.tma_b);
       }
-      load_q(0);  // first use of its slot: no wait
+      load_q(0);  // first use of its slots: no wait
+      load_do(0);
+    }
+  }
+  if constexpr (FOLD) {
+    // The ones block of the statistics step: 128 rows of 32 bytes, each
+    // 16-byte half = bf16 {1, 1, 1, 0, 0, 0, 0, 0}; one half per thread.
+    if (warp < 8) {
+      st_shared_v4(smem0 + C::OFF_ONES + threadIdx.x * 16, 0x3F803F80u, 0x00003F80u, 0u, 0u);
+      fence_proxy_async_smem();
     }
   }
   if (warp == 9) {
@@ -424,12 +536,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     // ------------------------------------------------------------ producer
     if (lane == 0 && nt > 0) {
       for (int t = 1; t < nt; ++t)  // K, V and tile 0 are on their way
-        if (!load_q(t)) break;
-      for (int t = nt - QS < 0 ? 0 : nt - QS; t < nt; ++t) {
-        const int slot = t % QS, n = t / QS;
-        if (!mbar_wait(bar(C::B_QFULL + slot), n & 1)) break;
-        if (!mbar_wait(bar(C::B_DOFULL + slot), n & 1)) break;
-      }
+        if (!load_q(t) || !load_do(t)) break;
+      for (int t = nt - QS < 0 ? 0 : nt - QS; t < nt; ++t)
+        if (!mbar_wait(bar(C::B_QFULL + t % QS), (t / QS) & 1)) break;
+      for (int t = nt - DS < 0 ? 0 : nt - DS; t < nt; ++t)
+        if (!mbar_wait(bar(C::B_DOFULL + t % DS), (t / DS) & 1)) break;
       mbar_wait(bar(C::B_KV), 0);
     }
   } else if (warp == 9) {
@@ -446,7 +557,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       const uint64_t k_kdesc = sdesc_sw128(smem0 + C::OFF_K, 16, 1024);
       const uint64_t v_kdesc = sdesc_sw128(smem0 + C::OFF_V, 16, 1024);
       const uint64_t k_mndesc = sdesc_sw128(smem0 + C::OFF_K, BN * 128, 1024);
-      // S^T_u = K Q_u^T into the S block of buffer u % NBUF.
+      const uint64_t ones_desc = sdesc_sw32(smem0 + C::OFF_ONES, 256);
+      // S^T_u = K Q_u^T (- LSE2 / (scale log2 e) when FOLD) into the S block
+      // of buffer u % NBUF.
       auto issue_s = [&](int u) -> bool {
         const int slot = u % QS, bf = u % NBUF;
         const uint64_t q_desc = sdesc_sw128(smem0 + C::OFF_Q + slot * C::Q_BYTES, 16, 1024);
@@ -458,15 +571,19 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           mma_ss_warp(tmem + C::TM_S + bf * BM, desc_at(k_kdesc, bx * (BN * 128) + w * 32),
                  desc_at(q_desc, bx * (BM * 128) + w * 32), idesc_s, kk > 0);
         }
+        if constexpr (FOLD)
+          mma_ss_warp(tmem + C::TM_S + bf * BM, ones_desc,
+                      sdesc_sw32(smem0 + C::OFF_LSB + slot * C::SLAB_BYTES, 256), idesc_s, 1u);
         mma_commit_warp(bar(C::B_SFULL + bf));
         return true;
       };
-      // dP^T_u = V dO_u^T into the dP block, once tile u - NBUF's dQ left it.
+      // dP^T_u = V dO_u^T (- Dvec when FOLD) into the dP block, once tile
+      // u - NBUF's dQ left it.
       auto issue_dp = [&](int u) -> bool {
-        const int slot = u % QS, bf = u % NBUF, use = u / NBUF;
+        const int slot = u % DS, bf = u % NBUF, use = u / NBUF;
         const uint64_t do_desc = sdesc_sw128(smem0 + C::OFF_DO + slot * C::Q_BYTES, 16, 1024);
         if (use > 0 && !mbar_wait_warp(bar(C::B_DQFREE + bf), (use - 1) & 1)) return false;
-        if (!mbar_wait_warp(bar(C::B_DOFULL + slot), (u / QS) & 1)) return false;
+        if (!mbar_wait_warp(bar(C::B_DOFULL + slot), (u / DS) & 1)) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -474,16 +591,19 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           mma_ss_warp(tmem + C::TM_DP + bf * BM, desc_at(v_kdesc, bx * (BN * 128) + w * 32),
                  desc_at(do_desc, bx * (BM * 128) + w * 32), idesc_s, kk > 0);
         }
+        if constexpr (FOLD)
+          mma_ss_warp(tmem + C::TM_DP + bf * BM, ones_desc,
+                      sdesc_sw32(smem0 + C::OFF_DVB + slot * C::SLAB_BYTES, 256), idesc_s, 1u);
         mma_commit_warp(bar(C::B_DPFULL + bf));
         return true;
       };
-      // dV += P^T dO, dK += dS^T Q and tile t's dQ share.
+      // dV += P^T dO, dK += dS^T Q and tile t's dQ share; then Q and dO of
+      // tile t are released.
       auto issue_grads = [&](int t) -> bool {
-        const int slot = t % QS, bf = t % NBUF, use = t / NBUF;
-        const uint64_t q_mn = sdesc_sw128(smem0 + C::OFF_Q + slot * C::Q_BYTES, BM * 128, 1024);
-        const uint64_t do_mn = sdesc_sw128(smem0 + C::OFF_DO + slot * C::Q_BYTES, BM * 128, 1024);
+        const int qslot = t % QS, dslot = t % DS, bf = t % NBUF, use = t / NBUF;
+        const uint64_t q_mn = sdesc_sw128(smem0 + C::OFF_Q + qslot * C::Q_BYTES, BM * 128, 1024);
+        const uint64_t do_mn = sdesc_sw128(smem0 + C::OFF_DO + dslot * C::Q_BYTES, BM * 128, 1024);
         const uint32_t ds_base = smem0 + C::OFF_DS + bf * C::DS_BYTES;
-        const uint64_t ds_k = sdesc_sw128(ds_base, 16, 1024);
         const uint64_t ds_mn = sdesc_sw128(ds_base, BN * 128, 1024);
         if (!mbar_wait_warp(bar(C::B_PREADY + bf), use & 1)) return false;
         tc_fence_after();
@@ -498,10 +618,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         if (!mbar_wait_warp(bar(C::B_DSREADY + bf), use & 1)) return false;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < BM / 16; ++kk) {  // dS^T as a K-major smem operand; Q MN-major
-          const int bx = kk / 4, w = kk % 4;
-          mma_ss_warp(tmem + C::TM_DK, desc_at(ds_k, bx * (BN * 128) + w * 32),
-                 desc_at(q_mn, kk * 2048), idesc_acc, (t > 0 || kk > 0));
+        for (int kk = 0; kk < BM / 16; ++kk) {
+          // dS^T from tensor memory, packed after each half's P^T; Q MN-major
+          const int half = kk / (C::HW / 16), part = kk % (C::HW / 16);
+          mma_ts_warp(tmem + C::TM_DK,
+                      tmem + C::TM_S + bf * BM + half * C::HW + C::HW / 2 + part * 8,
+                      desc_at(q_mn, kk * 2048), idesc_acc, (t > 0 || kk > 0));
         }
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
@@ -514,17 +636,20 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         }
         mma_commit_warp(bar(C::B_DQFULL + bf));
         mma_commit_warp(bar(C::B_DSFREE + bf));
-        mma_commit_warp(bar(C::B_EMPTY + slot));
+        mma_commit_warp(bar(C::B_QEMPTY + qslot));
+        mma_commit_warp(bar(C::B_DOEMPTY + dslot));
         return true;
       };
-      // Two buffers: tile t+1's S^T and dP^T go in before tile t's gradient
-      // MMAs (the dP block of t+1 is released when the compute warps drain
-      // tile t-1's dQ, midway through tile t).  One buffer: tile t first.
+      // Two buffers: tile t+1's S^T goes in before tile t's gradient MMAs
+      // and its dP^T after them (the dP block of t+1 is released when the
+      // compute warps drain tile t-1's dQ, midway through tile t).  One
+      // buffer: tile t first.
       bool ok = mbar_wait_warp(bar(C::B_KV), 0) && issue_s(0) && issue_dp(0);
       for (int t = 0; ok && t < nt; ++t) {
         const bool more = t + 1 < nt;
-        if (NBUF == 2 && more && !(issue_s(t + 1) && issue_dp(t + 1))) { ok = false; break; }
+        if (NBUF == 2 && more && !issue_s(t + 1)) { ok = false; break; }
         if (!issue_grads(t)) { ok = false; break; }
+        if (NBUF == 2 && more && !issue_dp(t + 1)) { ok = false; break; }
         if (NBUF == 1 && more && !(issue_s(t + 1) && issue_dp(t + 1))) { ok = false; break; }
       }
       if (ok) mma_commit_warp(bar(C::B_DONE));
@@ -589,10 +714,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     };
     bool ok = true;
     for (int t = 0; t < nt; ++t) {
-      const int slot = t % QS, ph = (t / QS) & 1, bf = t % NBUF, use = t / NBUF;
+      const int qslot = t % QS, dslot = t % DS, bf = t % NBUF, use = t / NBUF;
       const int q0 = (qb_lo + t % nqb) * BM;
       if (!mbar_wait_warp(bar(C::B_SFULL + bf), use & 1)) { ok = false; break; }
-      if (!mbar_wait_warp(bar(C::B_QFULL + slot), ph)) { ok = false; break; }
+      if (!FOLD && !mbar_wait_warp(bar(C::B_QFULL + qslot), (t / QS) & 1)) { ok = false; break; }
       tc_fence_after();
       const uint32_t s_tmem = tmem + lane_base + C::TM_S + bf * BM + c0;
       float pr[C::HW];
@@ -604,39 +729,57 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         for (int e = 0; e < 32; ++e) pr[c + e] = __uint_as_float(raw[e]);
       }
       tmem_ld_wait();
-      // Whole half visible (query rows past seqlen_q have LSE2 = +inf: P = 0).
+      // Whole half visible.  Without the fold, query rows past seqlen_q have
+      // LSE2 = +inf (P = 0); with it they are masked here.
       const int qa = q0 + c0;
       const bool full = ((long long)k0 + BN <= p.seqlen_k) &&
                         ((long long)k0 + BN - 1 <= (long long)qa + off + rb) &&
-                        ((long long)k0 >= (long long)(qa + C::HW - 1) + off - lb);
-      const uint32_t lse_addr = smem0 + C::OFF_LSE + (slot * BM + c0) * 4;
+                        ((long long)k0 >= (long long)(qa + C::HW - 1) + off - lb) &&
+                        (!FOLD || qa + C::HW <= p.seqlen_q);
       const uint64_t scale2 = f2_pack(p.scale_log2, p.scale_log2);
       // positional bias of query column c (ALIBI): bk * |c - bd|, log2 units
       const int hq = kvh * group + t / nqb;  // this tile's query head
       const float bk = ALIBI ? -p.alibi[hq] * 1.4426950408889634f : 0.f;
       const float bd = ALIBI ? (float)(j - off - qa) : 0.f;
+      if constexpr (FOLD) {
 #pragma unroll
-      for (int c = 0; c < C::HW; c += 4) {
-        float l4[4];
-        ld_shared_v4f(lse_addr + c * 4, l4);
-#pragma unroll
-        for (int e = 0; e < 4; e += 2) {
+        for (int c = 0; c < C::HW; c += 2) {
           float a0, a1;
-          f2_unpack(f2_fma(f2_pack(pr[c + e], pr[c + e + 1]), scale2, f2_pack(-l4[e], -l4[e + 1])),
-                    a0, a1);
+          f2_unpack(f2_mul(f2_pack(pr[c], pr[c + 1]), scale2), a0, a1);
           if constexpr (ALIBI) {
-            a0 = fmaf(fabsf((float)(c + e) - bd), bk, a0);
-            a1 = fmaf(fabsf((float)(c + e + 1) - bd), bk, a1);
+            a0 = fmaf(fabsf((float)c - bd), bk, a0);
+            a1 = fmaf(fabsf((float)(c + 1) - bd), bk, a1);
           }
-          pr[c + e] = ex2(a0);
-          pr[c + e + 1] = ex2(a1);
+          pr[c] = ex2(a0);
+          pr[c + 1] = ex2(a1);
+        }
+      } else {
+        const uint32_t lse_addr = smem0 + C::OFF_LSE + (qslot * BM + c0) * 4;
+#pragma unroll
+        for (int c = 0; c < C::HW; c += 4) {
+          float l4[4];
+          ld_shared_v4f(lse_addr + c * 4, l4);
+#pragma unroll
+          for (int e = 0; e < 4; e += 2) {
+            float a0, a1;
+            f2_unpack(f2_fma(f2_pack(pr[c + e], pr[c + e + 1]), scale2, f2_pack(-l4[e], -l4[e + 1])),
+                      a0, a1);
+            if constexpr (ALIBI) {
+              a0 = fmaf(fabsf((float)(c + e) - bd), bk, a0);
+              a1 = fmaf(fabsf((float)(c + e + 1) - bd), bk, a1);
+            }
+            pr[c + e] = ex2(a0);
+            pr[c + e + 1] = ex2(a1);
+          }
         }
       }
       if (!full) {
 #pragma unroll
         for (int c = 0; c < C::HW; ++c) {
           const long long i = (long long)qa + c;
-          if (j >= p.seqlen_k || j > i + off + rb || j < i + off - lb) pr[c] = 0.f;
+          if (j >= p.seqlen_k || j > i + off + rb || j < i + off - lb ||
+              (FOLD && i >= p.seqlen_q))
+            pr[c] = 0.f;
         }
       }
       // Dropout: this key's random bytes for the warp's query columns, kw[k]
@@ -669,56 +812,82 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       tc_fence_before();
       mbar_arrive(bar(C::B_PREADY + bf));
       // Two buffers: tile t-1's dQ finished while P_t was computed; reading
-      // it out now frees its block for dP_{t+1} (issued next by the MMA warp).
+      // it out now frees its block for dP_{t+1} (issued by the MMA warp after
+      // tile t's gradient MMAs).
       if (NBUF == 2 && t >= 1 && !drain_dq(t - 1)) { ok = false; break; }
       if (!mbar_wait_warp(bar(C::B_DPFULL + bf), use & 1)) { ok = false; break; }
-      if (!mbar_wait_warp(bar(C::B_DOFULL + slot), ph)) { ok = false; break; }
+      if (!FOLD && !mbar_wait_warp(bar(C::B_DOFULL + dslot), (t / DS) & 1)) { ok = false; break; }
       tc_fence_after();
-      const uint32_t dvec_addr = smem0 + C::OFF_DVEC + (slot * BM + c0) * 4;
+      if constexpr (FOLD) {
+        // the accumulator holds dP - Dvec: dS = P o acc
 #pragma unroll
-      for (int c = 0; c < C::HW; c += 32) {
-        uint32_t raw[32];
-        tmem_ld32(tmem + lane_base + C::TM_DP + bf * BM + c0 + c, raw);
-        tmem_ld_wait();
+        for (int c = 0; c < C::HW; c += 32) {
+          uint32_t raw[32];
+          tmem_ld32(tmem + lane_base + C::TM_DP + bf * BM + c0 + c, raw);
+          tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          float d4[4];
-          ld_shared_v4f(dvec_addr + (c + e) * 4, d4);
+          for (int e = 0; e < 32; e += 2)
+            f2_unpack(f2_mul(f2_pack(pr[c + e], pr[c + e + 1]),
+                             f2_pack(__uint_as_float(raw[e]), __uint_as_float(raw[e + 1]))),
+                      pr[c + e], pr[c + e + 1]);
+        }
+      } else {
+        const uint32_t dvec_addr = smem0 + C::OFF_DVEC + (dslot * BM + c0) * 4;
 #pragma unroll
-          for (int f = 0; f < 4; f += 2) {
-            // dS = P * (dP - Dvec), two columns per packed instruction pair;
-            // with dropout dP of a kept element is scaled by 1 / (1 - p) and
-            // that of a dropped one is 0.
-            uint64_t diff;
-            if constexpr (DROP) {
-              const uint32_t kb = dropout_keep_bits(kw[(c + e) / 4], f / 2, p.drop_kadd);
-              const float g0 = __uint_as_float(raw[e + f] & dropout_lo_mask(kb));
-              const float g1 = __uint_as_float(raw[e + f + 1] & dropout_hi_mask(kb));
-              diff = f2_fma(f2_pack(g0, g1), f2_pack(p.drop_scale, p.drop_scale),
-                            f2_pack(-d4[f], -d4[f + 1]));
-            } else {
-              diff = f2_add(f2_pack(__uint_as_float(raw[e + f]), __uint_as_float(raw[e + f + 1])),
-                            f2_pack(-d4[f], -d4[f + 1]));
+        for (int c = 0; c < C::HW; c += 32) {
+          uint32_t raw[32];
+          tmem_ld32(tmem + lane_base + C::TM_DP + bf * BM + c0 + c, raw);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) {
+            float d4[4];
+            ld_shared_v4f(dvec_addr + (c + e) * 4, d4);
+#pragma unroll
+            for (int f = 0; f < 4; f += 2) {
+              // dS = P * (dP - Dvec), two columns per packed instruction pair;
+              // with dropout dP of a kept element is scaled by 1 / (1 - p) and
+              // that of a dropped one is 0.
+              uint64_t diff;
+              if constexpr (DROP) {
+                const uint32_t kb = dropout_keep_bits(kw[(c + e) / 4], f / 2, p.drop_kadd);
+                const float g0 = __uint_as_float(raw[e + f] & dropout_lo_mask(kb));
+                const float g1 = __uint_as_float(raw[e + f + 1] & dropout_hi_mask(kb));
+                diff = f2_fma(f2_pack(g0, g1), f2_pack(p.drop_scale, p.drop_scale),
+                              f2_pack(-d4[f], -d4[f + 1]));
+              } else {
+                diff = f2_add(f2_pack(__uint_as_float(raw[e + f]), __uint_as_float(raw[e + f + 1])),
+                              f2_pack(-d4[f], -d4[f + 1]));
+              }
+              f2_unpack(f2_mul(f2_pack(pr[c + e + f], pr[c + e + f + 1]), diff), pr[c + e + f],
+                        pr[c + e + f + 1]);
             }
-            f2_unpack(f2_mul(f2_pack(pr[c + e + f], pr[c + e + f + 1]), diff), pr[c + e + f],
-                      pr[c + e + f + 1]);
           }
         }
       }
       // dS smem buffer is free once tile t - NBUF's dK and dQ MMAs have read it.
       if (use > 0 && !mbar_wait_warp(bar(C::B_DSFREE + bf), (use - 1) & 1)) { ok = false; break; }
       {
-        // dS as [key row][query] with 128-byte swizzle, 64 queries per box.
+        // dS^T packed into tensor memory after this half's P^T (the A operand
+        // of dK += dS^T Q; these score columns were read above), and dS as
+        // [key row][query] with 128-byte swizzle, 64 queries per box, in
+        // shared memory (an MN-major operand of the dQ product).
         const uint32_t row_addr = smem0 + C::OFF_DS + bf * C::DS_BYTES + r * 128;
 #pragma unroll
-        for (int c8 = 0; c8 < C::HW / 8; ++c8) {
-          const int col = c0 + c8 * 8;
-          const int bx = col / 64, chunk = ((col % 64) / 8) ^ (r & 7);
-          st_shared_v4(row_addr + bx * (BN * 128) + chunk * 16,
-                       pack2<C::FP16>(pr[8 * c8], pr[8 * c8 + 1]), pack2<C::FP16>(pr[8 * c8 + 2], pr[8 * c8 + 3]),
-                       pack2<C::FP16>(pr[8 * c8 + 4], pr[8 * c8 + 5]), pack2<C::FP16>(pr[8 * c8 + 6], pr[8 * c8 + 7]));
+        for (int c = 0; c < C::HW; c += 32) {
+          uint32_t w[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) w[e] = pack2<C::FP16>(pr[c + 2 * e], pr[c + 2 * e + 1]);
+          tmem_st16(s_tmem + C::HW / 2 + c / 2, w);
+#pragma unroll
+          for (int q8 = 0; q8 < 4; ++q8) {
+            const int col = c0 + c + q8 * 8;
+            const int bx = col / 64, chunk = ((col % 64) / 8) ^ (r & 7);
+            st_shared_v4(row_addr + bx * (BN * 128) + chunk * 16, w[4 * q8], w[4 * q8 + 1],
+                         w[4 * q8 + 2], w[4 * q8 + 3]);
+          }
         }
       }
+      tmem_st_wait();
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bar(C::B_DSREADY + bf));
@@ -729,7 +898,46 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     for (int u = nt - NBUF + 1 < 0 ? 0 : nt - NBUF + 1; ok && u < nt; ++u) ok = drain_dq(u);
     // ------------------------------------------------------------ epilogue
     if (ok && nt > 0) ok = mbar_wait_warp(bar(C::B_DONE), 0);
-    if (ok) {
+    if (ok && p.acc_f32) {
+      // float32 accumulate: this warp's 32 key rows x D/2 head-dim columns
+      // of dK (x scale), then of dV, as 32 x 32 boxes through its staging
+      // box, each added into the caller's buffer by one TMA reduce-add
+      // (rows past seqlen_k are clipped by the tensor map).  A key tile that
+      // no query sees adds nothing.
+      if (nt > 0) {
+        tc_fence_after();
+        const int krow = sq.k_row0 + k0 + quad * 32;
+#pragma unroll 1
+        for (int which = 0; which < 2; ++which) {
+          const uint32_t src = tmem + lane_base + (which == 0 ? C::TM_DK : C::TM_DV);
+          const float mul = which == 0 ? p.softmax_scale : 1.f;
+#pragma unroll 1
+          for (int c = half * (D / 2); c < (half + 1) * (D / 2); c += 32) {
+            uint32_t raw[32];
+            tmem_ld32(src + c, raw);
+            tmem_ld_wait();
+            if (staged) {
+              if (lane == 0) bulk_wait_group_read_all();
+              __syncwarp();
+            }
+#pragma unroll
+            for (int c4 = 0; c4 < 8; ++c4)
+              st_shared_v4(dqs + lane * 128 + ((c4 ^ (lane & 7)) << 4),
+                           __float_as_uint(__uint_as_float(raw[4 * c4]) * mul),
+                           __float_as_uint(__uint_as_float(raw[4 * c4 + 1]) * mul),
+                           __float_as_uint(__uint_as_float(raw[4 * c4 + 2]) * mul),
+                           __float_as_uint(__uint_as_float(raw[4 * c4 + 3]) * mul));
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0 && k0 + quad * 32 < p.seqlen_k) {
+              tma_reduce_add_4d(which == 0 ? &tm_dk : &tm_dv, dqs, c, kvh, krow, sq.tma_b);
+              bulk_commit_group();
+            }
+            staged = true;
+          }
+        }
+      }
+    } else if (ok) {
       tc_fence_after();
       // dK (x scale) staged in the Q slots, dV in the dO slots; this warp
       // writes head-dim columns [half * D/2, (half + 1) * D/2) of its rows.
@@ -772,7 +980,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     }
     tc_fence_before();
     named_bar_sync(1, 256);
-    if (ok && threadIdx.x == 0 && !row_store) {
+    if (ok && threadIdx.x == 0 && !row_store && !p.acc_f32) {
       for (int bx = 0; bx < C::NBOX; ++bx) {
         tma_store_4d(&tm_dk, smem0 + C::OFF_Q + bx * (BN * 128), bx * 64, kvh, sq.k_row0 + k0,
                      sq.tma_b);

@@ -2,25 +2,32 @@
 // value sequence (decoding with a cache), split over the keys.
 //
 // With one to a few query tokens per sequence the work is reading K and V
-// once: about G / 2 multiply-adds per byte for a group of G query heads, far
-// below the tensor-core ridge, so this path runs on the CUDA cores and is
-// bound by HBM.  One block per (key split, batch, kv head) takes all the
-// query rows that read that kv head (the G query heads of the group times
-// the Nq query tokens, at most kDecodeRows), so every K and V row is read
-// once for the whole group.  Each block writes its split's partial output
-// (16-bit) and LSE; attn_merge combines the splits (the online-softmax
-// rescale, as for split-KV calls of attn_fwd).
+// once: about R / 2 multiply-adds per byte for the R query rows that share a
+// kv head, far below the tensor-core ridge, so this path runs on the CUDA
+// cores and is bound by HBM.  One block per (key split, batch, kv head)
+// takes all the query rows that read that kv head (the G query heads of the
+// group times the Nq query tokens, R = G * Nq <= kDecodeRows), so every K and
+// V row is read once for the whole group.  Each block writes its split's
+// partial output (16-bit) and LSE; attn_merge combines the splits (the
+// online-softmax rescale, as for split-KV calls of attn_fwd).
 //
-// Within a block each warp takes 32 keys at a time:
-//   * scores: lane l owns key j0 + l, reads its K row (16-byte loads) and
-//     forms the dot product with every query row (queries in shared memory,
-//     pre-scaled by softmax_scale * log2 e, read as broadcasts);
-//   * online softmax per row across the warp (shuffle max and sum), P of
-//     the 32 keys staged in shared memory;
-//   * O += P V: lane l owns head-dim columns [l * D/32, (l + 1) * D/32) and
-//     reads each of the 32 V rows in one coalesced warp access.
-// Products go through packed f32x2 FMAs (two head-dim columns each).
-// The warps' running (max, sum, O) are combined in shared memory at the end.
+// Block: warp 8 is the producer, warps 0-7 compute.
+//   * The producer streams the split's K and V in tiles of 64 keys through a
+//     three-slot ring in shared memory (TMA, 128-byte swizzle, one mbarrier
+//     per slot for "full" and one for "empty"), so the loads of the next
+//     tiles are in flight while the current one is computed.
+//   * Warp w takes keys 8w .. 8w + 7 of each tile, in two groups of four.
+//     Scores: lane = 4 p + kk holds head-dim part p (D / 8 columns) of key
+//     kk of the group; it reads its part of the K row from the swizzled tile
+//     and of every query row from shared memory (queries pre-scaled by
+//     softmax_scale * log2 e, fp32), and three shuffles sum the parts.
+//   * Online softmax per query row over the warp's keys (running max and
+//     sum), then O += P V with lane l owning head-dim columns
+//     [l D/32, (l + 1) D/32) and P of each key taken by shuffle.
+//   * At the end the eight warps' (max, sum, O) are combined through shared
+//     memory (the ring, no longer needed) into the split's result.
+// Products go through packed f32x2 FMAs.  Grid: the host picks the number of
+// splits so that the blocks fill whole waves of the SMs.
 #pragma once
 #include <cuda_fp16.h>
 #include <stdint.h>
@@ -30,28 +37,41 @@
 
 namespace attn {
 
-constexpr int kDecodeRows = 16;  // query rows per block: group size x query tokens
-constexpr int kDecodeWarps = 8;
+constexpr int kDecodeRows = 16;    // query rows per block at most: group size x query tokens
+constexpr int kDecodeWarps = 8;    // compute warps
+constexpr int kDecodeBN = 64;      // keys per tile
+constexpr int kDecodeStages = 3;   // ring slots
+constexpr int kDecodeThreads = (kDecodeWarps + 1) * 32;
 
 struct DecodeParams {
   const uint16_t* q;  // (B, Nq, H, D)
-  const uint16_t* k;  // (B, Nk, Hkv, D)
-  const uint16_t* v;
   uint16_t* o_parts;  // (splits, B, Nq, H, D)
   float* lse_parts;   // (splits, B, H, Nq), natural log
   int batch, nheads, nheads_kv, seqlen_q, seqlen_k;
   int causal, window_left, window_right;
   float scale_log2;
-  int splits, chunk;  // keys per split (a multiple of 32)
+  int splits;
+  int key_lo;           // first key any query row can see
+  int tiles_per_split;  // key tiles (kDecodeBN keys) of one split
+  int tiles_total;      // key tiles from key_lo to the last visible key
 };
 
 template <int D>
-struct DecodeSmem {
-  static constexpr int Q = kDecodeRows * D;                    // scaled queries
-  static constexpr int P = kDecodeWarps * kDecodeRows * 32;    // P of each warp's 32 keys
-  static constexpr int O = kDecodeWarps * kDecodeRows * D;     // each warp's partial O
-  static constexpr int ML = kDecodeWarps * kDecodeRows * 2;    // each warp's max and sum
-  static constexpr int BYTES = (Q + P + O + ML) * 4;
+struct DecodeCfg {
+  static constexpr int NBOX = D / 64;                     // 64-column TMA boxes per row
+  static constexpr int BOX_BYTES = kDecodeBN * 128;       // one box: 64 rows x 128 bytes
+  static constexpr int TILE_BYTES = NBOX * BOX_BYTES;     // K or V tile
+  static constexpr int STAGE_BYTES = 2 * TILE_BYTES;      // K then V
+  static constexpr int COLS = D / 8;                      // head-dim columns of a score lane
+  static constexpr int CPL = D / 32;                      // head-dim columns of an output lane
+  static constexpr int OFF_Q = kDecodeStages * STAGE_BYTES;  // fp32 (kDecodeRows, D)
+  static constexpr int OFF_BAR = OFF_Q + kDecodeRows * D * 4;
+  static constexpr int B_FULL = 0, B_EMPTY = kDecodeStages, NBAR = 2 * kDecodeStages;
+  static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 1024;
+  // combine area (reuses the ring): per warp and row, O then (max, sum)
+  static constexpr int COMB_O = 0;
+  static constexpr int COMB_ML = kDecodeWarps * kDecodeRows * D * 4;
+  static_assert(COMB_ML + kDecodeWarps * kDecodeRows * 8 <= OFF_Q, "combine area");
 };
 
 template <bool FP16>
@@ -60,161 +80,228 @@ __device__ __forceinline__ float half_to_float(uint16_t h) {
   else return __uint_as_float((uint32_t)h << 16);
 }
 
-template <int D, bool FP16>
-__global__ void __launch_bounds__(kDecodeWarps * 32) attn_decode_kernel(const DecodeParams p) {
-  constexpr int CPL = D / 32;  // head-dim columns per lane in the P V product
-  using S = DecodeSmem<D>;
-  extern __shared__ float smem_f[];
-  float* qs = smem_f;
-  float* ps = qs + S::Q;
-  float* os = ps + S::P;
-  float* mls = os + S::O;
+// Two 16-bit values of a 32-bit word as floats (low half first).
+template <bool FP16>
+__device__ __forceinline__ void unpack2(uint32_t w, float& lo, float& hi) {
+  if constexpr (FP16) {
+    lo = __half2float(__ushort_as_half((unsigned short)(w & 0xFFFFu)));
+    hi = __half2float(__ushort_as_half((unsigned short)(w >> 16)));
+  } else {
+    lo = __uint_as_float(w << 16);
+    hi = __uint_as_float(w & 0xFFFF0000u);
+  }
+}
 
-  const int split = blockIdx.y, bk = blockIdx.x;  // x: (batch, kv head), up to 2^31 - 1
+// RMAX: rows the registers are sized for (4, 8 or 16); R <= RMAX rows are live.
+template <int D, bool FP16, int RMAX>
+__global__ void __launch_bounds__(kDecodeThreads, (RMAX <= 8) ? 2 : 1)
+    attn_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
+  using C = DecodeCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t smem0 = (smem_addr(smem_raw) + 1023u) & ~1023u;
+  uint8_t* smem_gen = smem_raw + (smem0 - smem_addr(smem_raw));
+  float* qs = reinterpret_cast<float*>(smem_gen + C::OFF_Q);
+  auto bar = [&](int i) -> uint32_t { return smem0 + C::OFF_BAR + 8u * i; };
+
+  const int split = blockIdx.y, bk = blockIdx.x;  // x: (batch, kv head)
   const int b = bk / p.nheads_kv, kvh = bk % p.nheads_kv;
   const int G = p.nheads / p.nheads_kv, Nq = p.seqlen_q, R = G * Nq;  // row r = g * Nq + i
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t warp = warp_id(), lane = lane_id();
 
-  for (int idx = threadIdx.x; idx < R * D; idx += blockDim.x) {
-    const int r = idx / D, c = idx % D, g = r / Nq, i = r % Nq;
-    const size_t src = (((size_t)b * Nq + i) * p.nheads + (size_t)kvh * G + g) * D + c;
-    qs[idx] = half_to_float<FP16>(p.q[src]) * p.scale_log2;
+  // this split's key tiles
+  const int t_begin = split * p.tiles_per_split;
+  const int t_end = min(t_begin + p.tiles_per_split, p.tiles_total);
+  const int ntiles = max(t_end - t_begin, 0);
+  const int key0 = p.key_lo + t_begin * kDecodeBN;
+
+  if (threadIdx.x == kDecodeWarps * 32) {
+    for (int i = 0; i < C::NBAR; ++i) mbar_init(bar(i), i >= C::B_EMPTY ? kDecodeWarps : 1);
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  // queries, pre-scaled, as fp32 rows (rows R .. RMAX - 1 zero)
+  for (int idx = threadIdx.x; idx < RMAX * D; idx += blockDim.x) {
+    const int r = idx / D, c = idx % D;
+    float x = 0.f;
+    if (r < R) {
+      const int g = r / Nq, i = r % Nq;
+      x = half_to_float<FP16>(
+              p.q[(((size_t)b * Nq + i) * p.nheads + (size_t)kvh * G + g) * D + c]) *
+          p.scale_log2;
+    }
+    qs[idx] = x;
   }
   __syncthreads();
 
-  const int k_begin = split * p.chunk;
-  const int k_end = min(k_begin + p.chunk, p.seqlen_k);
+  if (warp == kDecodeWarps) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && ntiles > 0) {
+      bool go = true;
+      for (int t = 0; go && t < ntiles; ++t) {
+        const int st = t % kDecodeStages, n = t / kDecodeStages;
+        if (n > 0 && !mbar_wait(bar(C::B_EMPTY + st), (n - 1) & 1)) { go = false; break; }
+        const uint32_t base = smem0 + st * C::STAGE_BYTES;
+        mbar_arrive_expect_tx(bar(C::B_FULL + st), C::STAGE_BYTES);
+        for (int bx = 0; bx < C::NBOX; ++bx) {
+          tma_load_4d(base + bx * C::BOX_BYTES, &tm_k, bar(C::B_FULL + st), bx * 64, kvh,
+                      key0 + t * kDecodeBN, b);
+          tma_load_4d(base + C::TILE_BYTES + bx * C::BOX_BYTES, &tm_v, bar(C::B_FULL + st),
+                      bx * 64, kvh, key0 + t * kDecodeBN, b);
+        }
+      }
+      // the block leaves only after its last loads have landed
+      for (int t = max(ntiles - kDecodeStages, 0); go && t < ntiles; ++t)
+        if (!mbar_wait(bar(C::B_FULL + t % kDecodeStages), (t / kDecodeStages) & 1)) break;
+    }
+  }
+
+  // ------------------------------------------------------------ compute
   const long long off = (long long)p.seqlen_k - Nq;
   const long long kInf = 1ll << 40;
   const long long rb = p.causal ? 0 : (p.window_right >= 0 ? p.window_right : kInf);
   const long long lb = p.window_left >= 0 ? p.window_left : kInf;
-  const size_t row_stride = (size_t)p.nheads_kv * D;  // elements between consecutive keys
-  const uint16_t* kbase = p.k + ((size_t)b * p.seqlen_k * p.nheads_kv + kvh) * D;
-  const uint16_t* vbase = p.v + ((size_t)b * p.seqlen_k * p.nheads_kv + kvh) * D;
-
-  float m[kDecodeRows], l[kDecodeRows];
-  uint64_t acc[kDecodeRows][CPL / 2];  // column pairs of this lane's O rows
+  const int part = (int)(lane >> 2), kk = (int)(lane & 3);
+  float m[RMAX], l[RMAX];
+  uint64_t acc[RMAX][C::CPL / 2];  // column pairs of this lane's output columns
 #pragma unroll
-  for (int r = 0; r < kDecodeRows; ++r) {
+  for (int r = 0; r < RMAX; ++r) {
     m[r] = -INFINITY;
     l[r] = 0.f;
 #pragma unroll
-    for (int c = 0; c < CPL / 2; ++c) acc[r][c] = f2_pack(0.f, 0.f);
+    for (int c = 0; c < C::CPL / 2; ++c) acc[r][c] = f2_pack(0.f, 0.f);
   }
-
-  for (int j0 = k_begin + warp * 32; j0 < k_end; j0 += kDecodeWarps * 32) {
-    const int j = j0 + lane;
-    float s[kDecodeRows];
-    {
-      uint64_t s2[kDecodeRows];  // (even, odd) column partial sums
+  if (warp < kDecodeWarps) {
+    for (int t = 0; t < ntiles; ++t) {
+      const int st = t % kDecodeStages;
+      // on expiry the status word reports the error; the warp stops reading
+      if (!mbar_wait_warp(bar(C::B_FULL + st), (t / kDecodeStages) & 1)) break;
+      const uint32_t kbase = smem0 + st * C::STAGE_BYTES;
+      const uint32_t vbase = kbase + C::TILE_BYTES;
+      const int jt = key0 + t * kDecodeBN;  // first key of the tile
+      // scores of the warp's two groups of four keys
+      float s[2][RMAX];
 #pragma unroll
-      for (int r = 0; r < kDecodeRows; ++r) s2[r] = f2_pack(0.f, 0.f);
-      if (j < k_end) {
-        const uint4* krow = reinterpret_cast<const uint4*>(kbase + (size_t)j * row_stride);
-#pragma unroll 4
-        for (int c8 = 0; c8 < D / 8; ++c8) {
-          float kf[8];
-          unpack8<FP16>(__ldg(krow + c8), kf);
-          const uint64_t k01 = f2_pack(kf[0], kf[1]), k23 = f2_pack(kf[2], kf[3]);
-          const uint64_t k45 = f2_pack(kf[4], kf[5]), k67 = f2_pack(kf[6], kf[7]);
+      for (int grp = 0; grp < 2; ++grp) {
+        const int row = (int)warp * 8 + grp * 4 + kk;  // key within the tile
+        // this lane's D/8 columns of the K row, as floats
+        float kf[C::COLS];
 #pragma unroll
-          for (int r = 0; r < kDecodeRows; ++r) {
-            if (r < R) {
-              const float4 qa = *reinterpret_cast<const float4*>(qs + r * D + c8 * 8);
-              const float4 qb = *reinterpret_cast<const float4*>(qs + r * D + c8 * 8 + 4);
-              s2[r] = f2_fma(f2_pack(qa.x, qa.y), k01, s2[r]);
-              s2[r] = f2_fma(f2_pack(qa.z, qa.w), k23, s2[r]);
-              s2[r] = f2_fma(f2_pack(qb.x, qb.y), k45, s2[r]);
-              s2[r] = f2_fma(f2_pack(qb.z, qb.w), k67, s2[r]);
+        for (int ch = 0; ch < C::COLS / 8; ++ch) {
+          const int col = part * C::COLS + ch * 8;
+          const int bx = col / 64, chunk = ((col % 64) / 8) ^ (row & 7);
+          uint32_t w0, w1, w2, w3;
+          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(w0), "=r"(w1), "=r"(w2), "=r"(w3)
+                       : "r"(kbase + bx * C::BOX_BYTES + row * 128 + chunk * 16));
+          unpack2<FP16>(w0, kf[ch * 8 + 0], kf[ch * 8 + 1]);
+          unpack2<FP16>(w1, kf[ch * 8 + 2], kf[ch * 8 + 3]);
+          unpack2<FP16>(w2, kf[ch * 8 + 4], kf[ch * 8 + 5]);
+          unpack2<FP16>(w3, kf[ch * 8 + 6], kf[ch * 8 + 7]);
+        }
+#pragma unroll
+        for (int r = 0; r < RMAX; ++r) {
+          uint64_t s2 = f2_pack(0.f, 0.f);
+          if (r < R) {
+            const uint32_t qaddr = smem0 + C::OFF_Q + (r * D + part * C::COLS) * 4;
+#pragma unroll
+            for (int c4 = 0; c4 < C::COLS / 4; ++c4) {
+              float q4[4];
+              ld_shared_v4f(qaddr + c4 * 16, q4);
+              s2 = f2_fma(f2_pack(q4[0], q4[1]), f2_pack(kf[4 * c4], kf[4 * c4 + 1]), s2);
+              s2 = f2_fma(f2_pack(q4[2], q4[3]), f2_pack(kf[4 * c4 + 2], kf[4 * c4 + 3]), s2);
             }
           }
+          float e, o;
+          f2_unpack(s2, e, o);
+          float x = e + o;
+          x += __shfl_xor_sync(0xffffffffu, x, 4);
+          x += __shfl_xor_sync(0xffffffffu, x, 8);
+          x += __shfl_xor_sync(0xffffffffu, x, 16);
+          // mask: key j of query i is visible iff i + off - lb <= j <= i + off + rb
+          const long long j = (long long)jt + row;
+          const long long i = r % Nq;
+          const bool vis = r < R && j < p.seqlen_k && j <= i + off + rb && j >= i + off - lb;
+          s[grp][r] = vis ? x : -INFINITY;
         }
       }
+      // online softmax per row over the warp's eight keys, then O += P V
+      float pr[2][RMAX];
 #pragma unroll
-      for (int r = 0; r < kDecodeRows; ++r) {
-        float e, o;
-        f2_unpack(s2[r], e, o);
-        s[r] = e + o;
-      }
-    }
-    // masks: key j of query i is visible iff i + off - lb <= j <= i + off + rb
-#pragma unroll
-    for (int r = 0; r < kDecodeRows; ++r) {
-      if (r < R) {
-        const long long i = r % Nq;
-        const bool vis = j < k_end && (long long)j <= i + off + rb && (long long)j >= i + off - lb;
-        if (!vis) s[r] = -INFINITY;
-      }
-    }
-    // online softmax of the warp's 32 keys, row by row
-    float* pw = ps + warp * kDecodeRows * 32;
-#pragma unroll
-    for (int r = 0; r < kDecodeRows; ++r) {
-      if (r < R) {
-        float mx = s[r];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      for (int r = 0; r < RMAX; ++r) {
+        float mx = fmaxf(s[0][r], s[1][r]);
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
         const float m_new = fmaxf(m[r], mx);
-        float pr = 0.f, alpha = 1.f;
+        float alpha = 1.f;
+        pr[0][r] = pr[1][r] = 0.f;
         if (m_new != -INFINITY) {
-          pr = exp2f(s[r] - m_new);
-          alpha = exp2f(m[r] - m_new);  // 0 when m[r] = -inf
+          alpha = ex2(m[r] - m_new);  // 0 when m[r] = -inf
+          pr[0][r] = ex2(s[0][r] - m_new);
+          pr[1][r] = ex2(s[1][r] - m_new);
         }
-        float sum = pr;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        float sum = pr[0][r] + pr[1][r];
+        sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+        sum += __shfl_xor_sync(0xffffffffu, sum, 2);
         l[r] = l[r] * alpha + sum;
         m[r] = m_new;
         const uint64_t a2 = f2_pack(alpha, alpha);
 #pragma unroll
-        for (int c = 0; c < CPL / 2; ++c) acc[r][c] = f2_mul(acc[r][c], a2);
-        pw[r * 32 + lane] = pr;
-      }
-    }
-    __syncwarp();
-    const int nkeys = min(32, k_end - j0);
-    for (int jj = 0; jj < nkeys; ++jj) {
-      const uint16_t* vrow = vbase + (size_t)(j0 + jj) * row_stride + lane * CPL;
-      float vf[CPL];
-      if constexpr (CPL == 4) {
-        const uint2 w = __ldg(reinterpret_cast<const uint2*>(vrow));
-        vf[0] = half_to_float<FP16>((uint16_t)(w.x & 0xFFFFu));
-        vf[1] = half_to_float<FP16>((uint16_t)(w.x >> 16));
-        vf[2] = half_to_float<FP16>((uint16_t)(w.y & 0xFFFFu));
-        vf[3] = half_to_float<FP16>((uint16_t)(w.y >> 16));
-      } else {
-        const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(vrow));
-        vf[0] = half_to_float<FP16>((uint16_t)(w & 0xFFFFu));
-        vf[1] = half_to_float<FP16>((uint16_t)(w >> 16));
+        for (int c = 0; c < C::CPL / 2; ++c) acc[r][c] = f2_mul(acc[r][c], a2);
       }
 #pragma unroll
-      for (int r = 0; r < kDecodeRows; ++r) {
-        if (r < R) {
-          const float pr = pw[r * 32 + jj];
-          const uint64_t p2 = f2_pack(pr, pr);
+      for (int key = 0; key < 8; ++key) {
+        const int row = (int)warp * 8 + key;
+        // this lane's CPL columns of the V row
+        const int col = (int)lane * C::CPL;
+        const int bx = col / 64, chunk = ((col % 64) / 8) ^ (row & 7);
+        const uint32_t vaddr = vbase + bx * C::BOX_BYTES + row * 128 + chunk * 16 + (col % 8) * 2;
+        float vf[C::CPL];
+        if constexpr (C::CPL == 4) {
+          uint32_t w0, w1;
+          asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(w0), "=r"(w1) : "r"(vaddr));
+          unpack2<FP16>(w0, vf[0], vf[1]);
+          unpack2<FP16>(w1, vf[2], vf[3]);
+        } else {
+          uint32_t w0;
+          asm volatile("ld.shared.b32 %0, [%1];" : "=r"(w0) : "r"(vaddr));
+          unpack2<FP16>(w0, vf[0], vf[1]);
+        }
 #pragma unroll
-          for (int c = 0; c < CPL / 2; ++c)
-            acc[r][c] = f2_fma(p2, f2_pack(vf[2 * c], vf[2 * c + 1]), acc[r][c]);
+        for (int r = 0; r < RMAX; ++r) {
+          if (r < R) {
+            const float pv = __shfl_sync(0xffffffffu, pr[key / 4][r], key % 4);
+            const uint64_t p2 = f2_pack(pv, pv);
+#pragma unroll
+            for (int c = 0; c < C::CPL / 2; ++c)
+              acc[r][c] = f2_fma(p2, f2_pack(vf[2 * c], vf[2 * c + 1]), acc[r][c]);
+          }
         }
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::B_EMPTY + st));
     }
-    __syncwarp();
   }
 
-  // combine the warps' running states
+  // ------------------------------------------------------------ combine
+  __syncthreads();  // every warp is done with the ring: it becomes the combine area
+  float* comb_o = reinterpret_cast<float*>(smem_gen + C::COMB_O);
+  float* comb_ml = reinterpret_cast<float*>(smem_gen + C::COMB_ML);
+  if (warp < kDecodeWarps) {
 #pragma unroll
-  for (int r = 0; r < kDecodeRows; ++r) {
-    if (r < R) {
+    for (int r = 0; r < RMAX; ++r) {
+      if (r < R) {
 #pragma unroll
-      for (int c = 0; c < CPL / 2; ++c) {
-        float lo, hi;
-        f2_unpack(acc[r][c], lo, hi);
-        os[(warp * kDecodeRows + r) * D + lane * CPL + 2 * c] = lo;
-        os[(warp * kDecodeRows + r) * D + lane * CPL + 2 * c + 1] = hi;
-      }
-      if (lane == 0) {
-        mls[(warp * kDecodeRows + r) * 2] = m[r];
-        mls[(warp * kDecodeRows + r) * 2 + 1] = l[r];
+        for (int c = 0; c < C::CPL / 2; ++c) {
+          float lo, hi;
+          f2_unpack(acc[r][c], lo, hi);
+          comb_o[(warp * kDecodeRows + r) * D + lane * C::CPL + 2 * c] = lo;
+          comb_o[(warp * kDecodeRows + r) * D + lane * C::CPL + 2 * c + 1] = hi;
+        }
+        if (lane == 0) {
+          comb_ml[(warp * kDecodeRows + r) * 2] = m[r];
+          comb_ml[(warp * kDecodeRows + r) * 2 + 1] = l[r];
+        }
       }
     }
   }
@@ -223,23 +310,22 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) attn_decode_kernel(const De
     const int r = idx / D, c = idx % D, g = r / Nq, i = r % Nq, h = kvh * G + g;
     float mx = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kDecodeWarps; ++w) mx = fmaxf(mx, mls[(w * kDecodeRows + r) * 2]);
+    for (int w = 0; w < kDecodeWarps; ++w) mx = fmaxf(mx, comb_ml[(w * kDecodeRows + r) * 2]);
     float sum = 0.f, o = 0.f;
     if (mx != -INFINITY) {
 #pragma unroll
       for (int w = 0; w < kDecodeWarps; ++w) {
-        const float sc = exp2f(mls[(w * kDecodeRows + r) * 2] - mx);
-        sum += mls[(w * kDecodeRows + r) * 2 + 1] * sc;
-        o += os[(w * kDecodeRows + r) * D + c] * sc;
+        const float sc = ex2(comb_ml[(w * kDecodeRows + r) * 2] - mx);
+        sum += comb_ml[(w * kDecodeRows + r) * 2 + 1] * sc;
+        o += comb_o[(w * kDecodeRows + r) * D + c] * sc;
       }
     }
     const float ov = sum > 0.f ? o / sum : 0.f;
-    const size_t part = ((size_t)split * p.batch + b);
-    const size_t dst = ((part * Nq + i) * p.nheads + h) * D + c;
-    if constexpr (FP16) p.o_parts[dst] = __half_as_ushort(__float2half_rn(ov));
-    else p.o_parts[dst] = (uint16_t)(pack2_rn<false>(ov, 0.f) & 0xFFFFu);
+    const size_t part_i = ((size_t)split * p.batch + b);
+    const size_t dst = ((part_i * Nq + i) * p.nheads + h) * D + c;
+    p.o_parts[dst] = (uint16_t)(pack2_rn<FP16>(ov, 0.f) & 0xFFFFu);
     if (c == 0)
-      p.lse_parts[(part * p.nheads + h) * Nq + i] =
+      p.lse_parts[(part_i * p.nheads + h) * Nq + i] =
           sum > 0.f ? (mx + __log2f(sum)) * 0.69314718055994530942f : -INFINITY;
   }
 }

@@ -189,18 +189,39 @@ int main(void) {
     assert int(out[4]) > 0 and out[5] == attn.attn_version()
 
 
+def _decode_splits(pairs, tiles, slots):
+    """The decode split rule: the split count (without empty splits) that
+    minimises waves x (tiles per block + 2), fewest splits on ties."""
+    best, best_s = None, 1
+    for s in range(1, min(tiles, 4096) + 1):
+        tps = -(-tiles // s)
+        s_eff = -(-tiles // tps)
+        cost = -(-(pairs * s_eff) // slots) * (tps + 2)
+        if best is None or cost < best:
+            best, best_s = cost, s_eff
+    return best_s
+
+
 def test_decode_host_checks(attn):
-    """attn_fwd_decode's workspace follows its split rule (about two blocks
-    per SM over the (batch, kv head) pairs, at least 256 keys per split) and
-    it refuses, before touching any pointer, more than 16 query rows per kv
+    """attn_fwd_decode's workspace follows its split rule (64-key tiles of
+    the visible key range cut so that the blocks fill whole waves of the 148
+    SMs, two blocks per SM for up to 8 query rows per kv head) and it
+    refuses, before touching any pointer, more than 16 query rows per kv
     head, head dim 256 and positional slopes."""
     fn = attn._lib.attn_fwd_decode_workspace_size
     fn.argtypes = [ctypes.POINTER(attn.AttnParams)]
     fn.restype = ctypes.c_size_t
-    p = P(attn, batch=2, seqlen_q=1, seqlen_k=5000, nheads=32, nheads_kv=4)
-    splits = min(-(-296 // 8), -(-5000 // 256))  # 20
-    rows = splits * 2 * 1 * 32
-    assert fn(ctypes.byref(p)) == -(-rows * 128 * 2 // 256) * 256 + -(-rows * 4 // 256) * 256
+    for B, Nq, Nk, H, Hkv, wl, slots in ((2, 1, 5000, 32, 4, -1, 296),
+                                         (8, 1, 32768, 32, 8, -1, 296),
+                                         (1, 2, 4000, 8, 2, 1024, 296),
+                                         (1, 3, 900, 16, 4, -1, 148)):
+        p = P(attn, batch=B, seqlen_q=Nq, seqlen_k=Nk, nheads=H, nheads_kv=Hkv, causal=True,
+              window_left=wl)
+        lo = max(0, Nk - Nq - wl) if wl >= 0 else 0
+        tiles = -(-(Nk - lo) // 64)
+        splits = _decode_splits(B * Hkv, tiles, slots)
+        rows = splits * B * Nq * H
+        assert fn(ctypes.byref(p)) == -(-rows * 128 * 2 // 256) * 256 + -(-rows * 4 // 256) * 256
     call = attn._lib.attn_fwd_decode
     vp = ctypes.c_void_p
     call.argtypes = [ctypes.POINTER(attn.AttnParams), vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]

@@ -89,8 +89,10 @@ def _identities(w, do, dk, dv):
     assert sdk.norm().item() <= 1e-2 * scale_ref, "sum dK is not ~0"
 
 
-@pytest.mark.parametrize("name", ["tiny_b1_h2_n128_d64", "causal_b2_h32_n8192_d128",
-                                  "full_b1_h16_n16384_d128", "gqa_window_b4_h32_kv8_n4096_d128"])
+# The two largest workloads are checked on many more rows, with their raw
+# errors recorded, in test_parity_configs_gpu.py (which also runs the
+# identities below on them).
+@pytest.mark.parametrize("name", ["tiny_b1_h2_n128_d64", "gqa_window_b4_h32_kv8_n4096_d128"])
 def test_bwd_full_size_sampled(attn, name):
     w = WORKLOADS[name]
     (q, k, v, do), (dq, dk, dv) = run_bwd(attn, w)

@@ -101,9 +101,10 @@ def _fake_prepare(p, out, lse, dout, workspace, stream=None):
                                         dq=torch.zeros(out.shape, dtype=torch.float64))
 
 
-def _fake_accumulate(p, q, k, v, dout, dk, dv, workspace, stream=None):
+def _fake_accumulate_f32(p, q, k, v, dout, dk_acc, dv_acc, workspace, stream=None):
     """Gradient shares of one key block, probabilities taken against the
-    given (global) LSE and D = rowsum(dO o O) from the given (global) O."""
+    given (global) LSE and D = rowsum(dO o O) from the given (global) O; the
+    key gradients are added into the float32 sums."""
     st = _STATE[workspace.data_ptr()]
     assert p.seqlen_q == q.shape[1] and p.seqlen_k == k.shape[1] and p.window_left == -1
     g = p.nheads // p.nheads_kv
@@ -123,8 +124,14 @@ def _fake_accumulate(p, q, k, v, dout, dk, dv, workspace, stream=None):
     dkh = torch.einsum("bhij,bihd->bjhd", ds, qd) * p.softmax_scale
     dvh = torch.einsum("bhij,bihd->bjhd", prob, st["do"])
     B, m, hkv, d = k.shape
-    dk.copy_(dkh.reshape(B, m, hkv, g, d).sum(3))
-    dv.copy_(dvh.reshape(B, m, hkv, g, d).sum(3))
+    assert dk_acc.dtype == torch.float32 and dv_acc.dtype == torch.float32
+    dk_acc += dkh.reshape(B, m, hkv, g, d).sum(3).float()
+    dv_acc += dvh.reshape(B, m, hkv, g, d).sum(3).float()
+
+
+def _fake_f32_to_16(src, dst, stream=None):
+    assert src.dtype == torch.float32 and src.shape == dst.shape
+    dst.copy_(src)
 
 
 def _fake_finalize(p, dq, workspace, stream=None):
@@ -137,7 +144,8 @@ def _install_fakes():
     attn.attn_merge = _fake_merge
     attn.attn_bwd_workspace_size = _fake_ws_size
     attn.attn_bwd_prepare = _fake_prepare
-    attn.attn_bwd_accumulate = _fake_accumulate
+    attn.attn_bwd_accumulate_f32 = _fake_accumulate_f32
+    attn.attn_f32_to_16 = _fake_f32_to_16
     attn.attn_bwd_finalize = _fake_finalize
 
 
@@ -147,7 +155,8 @@ def fakes(monkeypatch):
     for name, f in (("attn_fwd", _fake_fwd), ("attn_merge", _fake_merge),
                     ("attn_bwd_workspace_size", _fake_ws_size),
                     ("attn_bwd_prepare", _fake_prepare),
-                    ("attn_bwd_accumulate", _fake_accumulate),
+                    ("attn_bwd_accumulate_f32", _fake_accumulate_f32),
+                    ("attn_f32_to_16", _fake_f32_to_16),
                     ("attn_bwd_finalize", _fake_finalize)):
         monkeypatch.setattr(attn, name, f)
 
@@ -260,3 +269,38 @@ def test_ring_of_one_process_on_gpu():
     torch.cuda.synchronize()
     res = [(0, o.cpu(), lse.cpu(), dq.cpu(), dk.cpu(), dv.cpu(), True)]
     _compare_whole(res, w, "zigzag", "ring W=1 on GPU")
+
+
+@pytest.mark.gpu
+def test_accumulate_f32_adds_key_gradients():
+    """attn_bwd_accumulate_f32 adds dK (x scale) and dV in float32 into the
+    caller's sums: two calls on zeroed sums give twice the oracle's key
+    gradients, and twice the dQ share in the workspace accumulator; the
+    float32-to-16-bit conversion rounds like torch."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import io_aware_exact_33_b200 as attn
+    w = Workload("accf32", 2, 4, 2, 300, 260, 128, True, 64, -1, "bf16", 1.0, 812)
+    q, k, v, do = make_inputs(w)
+    qc, kc, vc, doc = q.cuda(), k.cuda(), v.cuda(), do.cuda()
+    args = (w.softmax_scale, w.causal, w.window_left, w.window_right)
+    o, lse = attn.attn_fwd(qc, kc, vc, *args)
+    p = attn.params_for(qc, kc, *args)
+    ws = torch.empty(attn.attn_bwd_workspace_size(p), dtype=torch.uint8, device="cuda")
+    attn.attn_bwd_prepare(p, o, lse, doc, ws)
+    dk_acc = torch.zeros(k.shape, dtype=torch.float32, device="cuda")
+    dv_acc = torch.zeros(k.shape, dtype=torch.float32, device="cuda")
+    for _ in range(2):
+        attn.attn_bwd_accumulate_f32(p, qc, kc, vc, doc, dk_acc, dv_acc, ws)
+    dq = torch.empty_like(qc)
+    attn.attn_bwd_finalize(p, dq, ws)
+    torch.cuda.synchronize()
+    assert attn.attn_get_device_status() == 0
+    dq_r, dk_r, dv_r = oracle.attention_bwd(q, k, v, do, *args)
+    check_grad(dk_acc.cpu() / 2, dk_r, "dK sum / 2")
+    check_grad(dv_acc.cpu() / 2, dv_r, "dV sum / 2")
+    check_grad(dq.cpu().double() / 2, dq_r, "dQ (two shares) / 2")
+    half = torch.empty(k.shape, dtype=torch.bfloat16, device="cuda")
+    attn.attn_f32_to_16(dk_acc, half)
+    torch.cuda.synchronize()
+    assert torch.equal(half.cpu(), dk_acc.cpu().to(torch.bfloat16))
