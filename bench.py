@@ -189,42 +189,70 @@ def max_over_ranks(value, dist, device=None):
 
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples during the timed region."""
+    """nvidia-smi clock / throttle-reason samples during the timed region.
+
+    The sampler runs every 20 ms from before the region starts (entering
+    waits for its first sample, outside the region) and each sample carries
+    its arrival time, so the summary keeps only the samples that arrived
+    while the region ran (the nearest one if the region is shorter than the
+    sampling period)."""
 
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
     NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+    PERIOD_MS = 20
 
     def __init__(self, gpu_id):
         self.gpu_id = gpu_id
         self.proc = None
+        self.samples = []  # (monotonic time, line)
+        self.t0 = self.t1 = None
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            if ln.strip():
+                self.samples.append((time.monotonic(), ln))
 
     def __enter__(self):
+        import threading
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu_id), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", str(self.PERIOD_MS)],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.reader = threading.Thread(target=self._read, daemon=True)
+            self.reader.start()
+            deadline = time.monotonic() + 5.0
+            while not self.samples and time.monotonic() < deadline:
+                time.sleep(0.005)
         except OSError:
             self.proc = None
+        self.t0 = time.monotonic()
         return self
 
     def __exit__(self, *exc):
-        self.lines = []
+        self.t1 = time.monotonic()
         if self.proc is not None:
+            time.sleep(self.PERIOD_MS / 1000.0)  # the sample that closes the region
             self.proc.terminate()
             try:
-                out, _ = self.proc.communicate(timeout=5)
+                self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+                self.proc.wait()
+            self.reader.join(timeout=5)
         return False
 
     def summary(self):
+        period = self.PERIOD_MS / 1000.0
+        inside = [ln for t, ln in self.samples
+                  if self.t0 is not None and self.t0 <= t <= self.t1 + period]
+        if not inside and self.samples and self.t0 is not None:
+            mid = 0.5 * (self.t0 + self.t1)
+            inside = [min(self.samples, key=lambda x: abs(x[0] - mid))[1]]
         sm, smax, reasons = [], [], set()
-        for ln in getattr(self, "lines", []):
+        for ln in inside:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 8:
                 continue
@@ -236,10 +264,12 @@ class ClockSampler:
             for name, val in zip(self.NAMES, parts[4:8]):
                 if val.lower().startswith("active"):
                     reasons.add(name)
+        window_ms = None if self.t0 is None else round((self.t1 - self.t0) * 1e3, 1)
         if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "window_ms": window_ms}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "window_ms": window_ms}
 
 
 # ---------------------------------------------------------------- CPU oracle

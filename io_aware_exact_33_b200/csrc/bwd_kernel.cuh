@@ -16,7 +16,7 @@
 //                   head of the GQA group that sees the key tile.
 //   bwd_convert     dQ = scale * accumulator, rounded to the input dtype.
 //
-// Main kernel roles (320 threads):
+// Main kernel roles (448 threads):
 //   warp 8      TMA producer: K_j, V_j once; Q_i (with its LSE2 statistics)
 //               and dO_i (with Dvec) per query tile through rings of their own.
 //   warp 9      TMEM allocation; issues the five MMAs per tile (one elected
@@ -30,11 +30,12 @@
 //               P^T = exp2(S^T*scale*log2e - LSE2) back into tensor memory as
 //               the 16-bit A operand of dV; dS = P o (dP - Dvec) into tensor
 //               memory beside it (the A operand of dK) and into shared
-//               memory (an MN-major operand of dQ); then the previous tile's dQ block
-//               (which reuses that tile's dP block) out of tensor memory into
-//               the fp32 accumulator with a TMA reduce-add per warp (other
-//               key tiles add to the same rows); finally dK, dV out through
-//               TMA.
+//               memory (an MN-major operand of dQ); finally dK, dV out
+//               through TMA.
+//   warps 10-13 dQ drain: each tile's dQ block (which reuses that tile's dP
+//               block) out of tensor memory into the fp32 accumulator with
+//               TMA reduce-adds (other key tiles add to the same rows), off
+//               the compute warps' path.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -359,7 +360,7 @@ struct BwdCfg {
   static constexpr int OFF_Q = OFF_V + KV_BYTES;
   static constexpr int OFF_DO = OFF_Q + QSTAGES * Q_BYTES;
   static constexpr int OFF_DS = OFF_DO + DOSTAGES * Q_BYTES;
-  // dQ staging: one 4 KB box (32 x 32 fp32, 128-byte swizzle) per compute warp
+  // dQ staging: two 4 KB boxes (32 x 32 fp32, 128-byte swizzle) per drain warp
   static constexpr int DQS_BYTES = 32 * 32 * 4;
   static constexpr int OFF_DQS = OFF_DS + NBUF * DS_BYTES;
   static constexpr int OFF_LSB = OFF_DQS + 8 * DQS_BYTES;  // -LSE2 slabs, one per Q slot
@@ -380,7 +381,7 @@ struct BwdCfg {
   static constexpr int B_DSREADY = B_PREADY + NBUF;   // 256 arrivals
   static constexpr int B_DSFREE = B_DSREADY + NBUF;
   static constexpr int B_DQFULL = B_DSFREE + NBUF;
-  static constexpr int B_DQFREE = B_DQFULL + NBUF;    // 256 arrivals
+  static constexpr int B_DQFREE = B_DQFULL + NBUF;    // 128 arrivals (the drain warps)
   static constexpr int B_DONE = B_DQFREE + NBUF;
   static constexpr int NBAR = B_DONE + 1;
   static constexpr int OFF_TMEMPTR = OFF_BAR + NBAR * 8;
@@ -388,7 +389,7 @@ struct BwdCfg {
   // tensor memory: dV, dK accumulators; per buffer an S/P block and a dP/dQ block
   static constexpr int TM_DV = 0, TM_DK = D, TM_S = 2 * D, TM_DP = 2 * D + NBUF * BM;
   static constexpr int TMEM_COLS = 512;
-  static constexpr int THREADS = 320;
+  static constexpr int THREADS = 448;  // 8 compute, producer, MMA, 4 dQ drain warps
   static_assert(TM_DP + NBUF * BM <= TMEM_COLS, "tensor memory");
   static_assert(DQT || D <= BM, "dQ block fits its dP block");
   static_assert(QSTAGES * Q_BYTES >= BN * D * 2, "dK epilogue staging");
@@ -497,9 +498,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   // latency overlaps the tensor-memory allocation and the barrier itself.
   if (warp == 8 && lane == 0) {
     for (int i = 0; i < C::NBAR; ++i) {
-      const bool many = (i >= C::B_PREADY && i < C::B_DSREADY + NBUF) ||
-                        (i >= C::B_DQFREE && i < C::B_DQFREE + NBUF);
-      mbar_init(bar(i), many ? 256 : 1);
+      uint32_t count = 1;
+      if (i >= C::B_PREADY && i < C::B_DSREADY + NBUF) count = 256;  // compute warps
+      if (i >= C::B_DQFREE && i < C::B_DQFREE + NBUF) count = 128;   // drain warps
+      mbar_init(bar(i), count);
     }
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -655,7 +657,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       if (ok) mma_commit_warp(bar(C::B_DONE));
     }
   } else if (warp < 8) {
-    // ------------------------------------------------------------ P, dS, dQ out
+    // ------------------------------------------------------------ P, dS
     // Warp w: tensor-memory lane quadrant w % 4 (key rows), query-column half
     // w / 4 (HW columns).
     const int quad = (int)(warp & 3), half = (int)(warp >> 2);
@@ -663,55 +665,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const int c0 = half * C::HW;          // first query column of this warp
     const long long j = (long long)k0 + r;
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
-    // dQ of tile u: read this warp's 32 x 32 part out of tensor memory,
-    // release the block, stage it in shared memory as a [query][head-dim]
-    // fp32 box, and add it into the accumulator with one TMA reduce-add
-    // (rows past seqlen_q are clipped by the tensor map).
-    const uint32_t dqs = smem0 + C::OFF_DQS + warp * C::DQS_BYTES;
-    bool staged = false;  // a reduce from this warp's box may still be reading it
-    auto drain_dq = [&](int u) -> bool {
-      const int bf = u % NBUF;
-      if (!mbar_wait_warp(bar(C::B_DQFULL + bf), (u / NBUF) & 1)) return false;
-      tc_fence_after();
-      const int h = kvh * group + u / nqb;
-      const int q0 = (qb_lo + u % nqb) * BM;
-      uint32_t raw[32];
-      tmem_ld32(tmem + lane_base + C::TM_DP + bf * BM + half * 32, raw);
-      tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(bar(C::B_DQFREE + bf));
-      if (staged) {
-        if (lane == 0) bulk_wait_group_read_all();
-        __syncwarp();
-      }
-      // Box element (row, col) sits at row * 128 + ((col / 4) ^ (row % 8)) * 16 + (col % 4) * 4.
-      int qrow, dcol;  // this warp's box origin in (query, head-dim)
-      if constexpr (C::DQT) {
-        // lane = head-dim column quad*32 + lane; columns = queries q0 + half*32 + c
-#pragma unroll
-        for (int c = 0; c < 32; ++c)
-          st_shared_f32(dqs + c * 128 + (((lane >> 2) ^ (c & 7)) << 4) + ((lane & 3) << 2),
-                        __uint_as_float(raw[c]));
-        qrow = q0 + half * 32;
-        dcol = quad * 32;
-      } else {
-        // lane = query q0 + quad*32 + lane; columns = head-dim half*32 + c
-#pragma unroll
-        for (int c4 = 0; c4 < 8; ++c4)
-          st_shared_v4(dqs + lane * 128 + ((c4 ^ (lane & 7)) << 4), raw[4 * c4], raw[4 * c4 + 1],
-                       raw[4 * c4 + 2], raw[4 * c4 + 3]);
-        qrow = q0 + quad * 32;
-        dcol = half * 32;
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0 && qrow < p.seqlen_q) {
-        tma_reduce_add_4d(&tm_dqacc, dqs, dcol, h, (int)prow0 + qrow, sq.tma_b);
-        bulk_commit_group();
-      }
-      staged = true;
-      return true;
-    };
     bool ok = true;
     for (int t = 0; t < nt; ++t) {
       const int qslot = t % QS, dslot = t % DS, bf = t % NBUF, use = t / NBUF;
@@ -811,10 +764,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar(C::B_PREADY + bf));
-      // Two buffers: tile t-1's dQ finished while P_t was computed; reading
-      // it out now frees its block for dP_{t+1} (issued by the MMA warp after
-      // tile t's gradient MMAs).
-      if (NBUF == 2 && t >= 1 && !drain_dq(t - 1)) { ok = false; break; }
       if (!mbar_wait_warp(bar(C::B_DPFULL + bf), use & 1)) { ok = false; break; }
       if (!FOLD && !mbar_wait_warp(bar(C::B_DOFULL + dslot), (t / DS) & 1)) { ok = false; break; }
       tc_fence_after();
@@ -891,11 +840,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bar(C::B_DSREADY + bf));
-      // One buffer: this tile's dQ (issued right after its dS) is read out
-      // before the next dP can use the block.
-      if (NBUF == 1 && !drain_dq(t)) { ok = false; break; }
     }
-    for (int u = nt - NBUF + 1 < 0 ? 0 : nt - NBUF + 1; ok && u < nt; ++u) ok = drain_dq(u);
     // ------------------------------------------------------------ epilogue
     if (ok && nt > 0) ok = mbar_wait_warp(bar(C::B_DONE), 0);
     if (ok && p.acc_f32) {
@@ -907,6 +852,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       if (nt > 0) {
         tc_fence_after();
         const int krow = sq.k_row0 + k0 + quad * 32;
+        // staging box of this warp in the (now idle) Q slots
+        const uint32_t dqs = smem0 + C::OFF_Q + warp * 4096;
+        bool staged = false;
 #pragma unroll 1
         for (int which = 0; which < 2; ++which) {
           const uint32_t src = tmem + lane_base + (which == 0 ? C::TM_DK : C::TM_DV);
@@ -989,8 +937,67 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       }
       bulk_commit_group();
     }
-    // every warp's dQ reduces (and the dK/dV stores) have read their shared
-    // memory before exit
+    // the dK/dV stores or reduces have read their shared memory before exit
+    if (lane == 0) bulk_wait_group_read_all();
+  } else if (warp >= 10) {
+    // ------------------------------------------------------------ dQ drain
+    // Warp w reads tensor-memory lane quadrant w % 4 of each tile's dQ block
+    // (64 columns: d = 128 holds dQ^T, lanes = head-dim columns and columns
+    // = queries; d = 64 holds dQ, lanes = queries and columns = head-dim),
+    // releases the block, stages it as two [query][head-dim] fp32 boxes of
+    // 32 x 32 (128-byte swizzle) and adds each into the accumulator with one
+    // TMA reduce-add (rows past seqlen_q are clipped by the tensor map).
+    const int quad = (int)(warp & 3);
+    const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+    const uint32_t dqs = smem0 + C::OFF_DQS + (warp - 10) * 2 * C::DQS_BYTES;
+    for (int u = 0; u < nt; ++u) {
+      const int bf = u % NBUF;
+      if (!mbar_wait_warp(bar(C::B_DQFULL + bf), (u / NBUF) & 1)) break;
+      tc_fence_after();
+      const int h = kvh * group + u / nqb;
+      const int q0 = (qb_lo + u % nqb) * BM;
+      uint32_t raw[2][32];
+      tmem_ld32(tmem + lane_base + C::TM_DP + bf * BM, raw[0]);
+      tmem_ld32(tmem + lane_base + C::TM_DP + bf * BM + 32, raw[1]);
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(bar(C::B_DQFREE + bf));
+      // the previous tile's reduces have read both boxes (issued a whole
+      // tile earlier)
+      if (u > 0) {
+        if (lane == 0) bulk_wait_group_read_all();
+        __syncwarp();
+      }
+#pragma unroll
+      for (int hb = 0; hb < 2; ++hb) {
+        const uint32_t box = dqs + hb * C::DQS_BYTES;
+        // Box element (row, col) sits at row * 128 + ((col / 4) ^ (row % 8)) * 16 + (col % 4) * 4.
+        int qrow, dcol;  // the box origin in (query, head-dim)
+        if constexpr (C::DQT) {
+          // lane = head-dim column quad*32 + lane; columns = queries q0 + hb*32 + c
+#pragma unroll
+          for (int c = 0; c < 32; ++c)
+            st_shared_f32(box + c * 128 + (((lane >> 2) ^ (c & 7)) << 4) + ((lane & 3) << 2),
+                          __uint_as_float(raw[hb][c]));
+          qrow = q0 + hb * 32;
+          dcol = quad * 32;
+        } else {
+          // lane = query q0 + quad*32 + lane; columns = head-dim hb*32 + c
+#pragma unroll
+          for (int c4 = 0; c4 < 8; ++c4)
+            st_shared_v4(box + lane * 128 + ((c4 ^ (lane & 7)) << 4), raw[hb][4 * c4],
+                         raw[hb][4 * c4 + 1], raw[hb][4 * c4 + 2], raw[hb][4 * c4 + 3]);
+          qrow = q0 + quad * 32;
+          dcol = hb * 32;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && qrow < p.seqlen_q) {
+          tma_reduce_add_4d(&tm_dqacc, box, dcol, h, (int)prow0 + qrow, sq.tma_b);
+          bulk_commit_group();
+        }
+      }
+    }
     if (lane == 0) bulk_wait_group_read_all();
   }
   tc_fence_before();

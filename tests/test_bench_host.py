@@ -43,15 +43,23 @@ def test_window_workload_pair_count():
 
 
 def test_clock_summary_parsing():
+    """Only samples that arrived while the timed region ran count; a region
+    shorter than the sampling period takes the sample nearest its middle."""
     c = bench.ClockSampler(0)
-    c.lines = [
-        "1965, 1965, 700.1, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
-        "1800, 1965, 990.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
-        "1320, 1965, 1001.2, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+    c.t0, c.t1 = 10.0, 10.1
+    c.samples = [
+        (9.9, "1100, 1965, 300.0, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active"),
+        (10.02, "1965, 1965, 700.1, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active"),
+        (10.05, "1800, 1965, 990.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active"),
+        (10.09, "1320, 1965, 1001.2, 0x0000000000000004, Not Active, Not Active, Not Active, Active"),
+        (10.5, "900, 1965, 100.0, 0x0000000000000000, Active, Not Active, Not Active, Not Active"),
     ]
     s = c.summary()
     assert s["sm_mhz"] == 1800 and s["sm_max_mhz"] == 1965
     assert s["reasons"] == ["sw_power_cap"] and s["samples"] == 3
+    c.t0, c.t1 = 10.2, 10.21
+    s = c.summary()
+    assert s["samples"] == 1 and s["sm_mhz"] == 1320
 
 
 def test_peaks_loaded_or_fallback():
