@@ -44,7 +44,7 @@
  * Element type of q, k, v, o, dout, dq, dk, dv: `dtype` (bf16 or fp16).
  *
  * Masks.  Key j is visible from query i iff, with off = seqlen_k - seqlen_q
- * (bottom-right alignment),
+ * + pos_offset (bottom-right alignment, moved by attn_params.pos_offset),
  *     causal:            j <= i + off
  *     window_left  >= 0: j >= i + off - window_left
  *     window_right >= 0: j <= i + off + window_right
@@ -103,7 +103,7 @@ typedef struct {
   int32_t window_right;   /* -1 = unbounded */
   /* Per-head positional slopes: NULL, or a DEVICE array of nheads floats
    * (4-byte aligned); score (i, j) of head h then gains
-   * -alibi_slopes[h] * |i + seqlen_k - seqlen_q - j| (the alibi_slopes
+   * -alibi_slopes[h] * |i + off - j|, off as in the mask rules (the alibi_slopes
    * argument of the FlashAttention-2 interface; see the mask rules below for
    * the alignment).  Read by the kernels only. */
   const float* alibi_slopes;
@@ -122,6 +122,17 @@ typedef struct {
   float dropout_p;
   uint32_t dropout_offset;
   uint64_t dropout_seed;
+  /* Position of the query rows relative to the keys beyond the bottom-right
+   * alignment (0, the value a zero-initialised struct holds, = none): the
+   * masks and the positional bias use off = seqlen_k - seqlen_q + pos_offset.
+   * For one block of a longer sequence (queries at global positions
+   * q0 .. q0 + seqlen_q - 1, keys at k0 .. k0 + seqlen_k - 1) it is
+   * q0 - k0 - (seqlen_k - seqlen_q), so that the block sees exactly the
+   * mask and bias of the whole sequence.  attn_fwd, attn_bwd and its stages
+   * and attn_fwd_e4m3 honour it; attn_fwd_decode and the packed-sequence
+   * calls require 0 (ATTN_ERR_INVALID_ARG). */
+  int32_t pos_offset;
+  int32_t reserved0;      /* must be 0 */
 } attn_params;
 
 /*

@@ -53,6 +53,8 @@ class AttnParams(ctypes.Structure):
         ("dropout_p", ctypes.c_float),
         ("dropout_offset", ctypes.c_uint32),
         ("dropout_seed", ctypes.c_uint64),
+        ("pos_offset", ctypes.c_int32),
+        ("reserved0", ctypes.c_int32),
     ]
 
 
@@ -160,15 +162,19 @@ _lib = _Lazy()
 
 def make_params(batch, seqlen_q, seqlen_k, nheads, nheads_kv, headdim, dtype=ATTN_BF16,
                 softmax_scale=None, causal=False, window_left=-1, window_right=-1,
-                alibi_slopes=None, dropout_p=0.0, dropout_seed=0, dropout_offset=0) -> AttnParams:
+                alibi_slopes=None, dropout_p=0.0, dropout_seed=0, dropout_offset=0,
+                pos_offset=0) -> AttnParams:
     """``alibi_slopes``: None, or the device address (int) of nheads float32
     slopes.  Dropout: rate ``dropout_p`` (applied as round(256 p) / 256), the
-    generator's 64-bit seed and 32-bit offset (see include/attn.h)."""
+    generator's 64-bit seed and 32-bit offset (see include/attn.h).
+    ``pos_offset`` moves the query rows relative to the keys for the masks and
+    the positional bias (0 = bottom-right alignment; include/attn.h)."""
     scale = 1.0 / math.sqrt(headdim) if softmax_scale is None else float(softmax_scale)
     return AttnParams(int(batch), int(seqlen_q), int(seqlen_k), int(nheads), int(nheads_kv),
                       int(headdim), int(dtype), scale, int(bool(causal)), int(window_left),
                       int(window_right), alibi_slopes, float(dropout_p),
-                      int(dropout_offset) & 0xFFFFFFFF, int(dropout_seed) & (2 ** 64 - 1))
+                      int(dropout_offset) & 0xFFFFFFFF, int(dropout_seed) & (2 ** 64 - 1),
+                      int(pos_offset), 0)
 
 
 def _slopes_ptr(alibi_slopes, nheads, device):
@@ -260,31 +266,33 @@ def _stream(stream):
 
 
 def params_for(q, k, softmax_scale=None, causal=False, window_left=-1, window_right=-1,
-               alibi_slopes=None, dropout_p=0.0, dropout_seed=0, dropout_offset=0):
+               alibi_slopes=None, dropout_p=0.0, dropout_seed=0, dropout_offset=0,
+               pos_offset=0):
     B, Nq, H, d = q.shape
     Bk, Nk, Hkv, dk = k.shape
     if Bk != B or dk != d:
         raise ValueError("q and k disagree on batch or head dim")
     return make_params(B, Nq, Nk, H, Hkv, d, _dtype_code(q), softmax_scale, causal, window_left,
                        window_right, _slopes_ptr(alibi_slopes, H, q.device), dropout_p,
-                       dropout_seed, dropout_offset)
+                       dropout_seed, dropout_offset, pos_offset)
 
 
 def attn_fwd(q, k, v, softmax_scale: Optional[float] = None, causal: bool = False,
              window_left: int = -1, window_right: int = -1, out=None, lse=None,
              stream=None, alibi_slopes=None, dropout_p: float = 0.0, dropout_seed: int = 0,
-             dropout_offset: int = 0) -> Tuple["torch.Tensor", "torch.Tensor"]:
+             dropout_offset: int = 0, pos_offset: int = 0) -> Tuple["torch.Tensor", "torch.Tensor"]:
     """O = softmax(q k^T * scale + bias + mask) v and the per-row natural-log LSE.
 
     q (B, Nq, H, d), k and v (B, Nk, Hkv, d), bf16 or fp16, contiguous CUDA
     tensors; ``alibi_slopes`` (optional, (H,) float32) adds
     -slope_h * |i + Nk - Nq - j|.  ``dropout_p`` > 0 drops attention
     probabilities by the generator contract of include/attn.h (seed, offset);
-    the backward needs the same three values.  Returns (out (B, Nq, H, d),
+    the backward needs the same three values.  ``pos_offset`` moves the query
+    rows relative to the keys (include/attn.h).  Returns (out (B, Nq, H, d),
     lse (B, H, Nq) float32)."""
     import torch
     p = params_for(q, k, softmax_scale, causal, window_left, window_right, alibi_slopes,
-                   dropout_p, dropout_seed, dropout_offset)
+                   dropout_p, dropout_seed, dropout_offset, pos_offset)
     B, Nq, H, d = q.shape
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _check(t, n)
@@ -414,12 +422,12 @@ def _bwd_tensors(q, k, v, out, lse, dout, dq, dk, dv):
 def attn_bwd(q, k, v, out, lse, dout, softmax_scale: Optional[float] = None, causal: bool = False,
              window_left: int = -1, window_right: int = -1, dq=None, dk=None, dv=None,
              workspace=None, stream=None, alibi_slopes=None, dropout_p: float = 0.0,
-             dropout_seed: int = 0, dropout_offset: int = 0):
+             dropout_seed: int = 0, dropout_offset: int = 0, pos_offset: int = 0):
     """Gradients (dq, dk, dv) of sum(out * dout) for attention with the same
     arguments as ``attn_fwd``; ``out`` and ``lse`` are its results."""
     import torch
     p = params_for(q, k, softmax_scale, causal, window_left, window_right, alibi_slopes,
-                   dropout_p, dropout_seed, dropout_offset)
+                   dropout_p, dropout_seed, dropout_offset, pos_offset)
     dq, dk, dv = _bwd_tensors(q, k, v, out, lse, dout, dq, dk, dv)
     ws_bytes = attn_bwd_workspace_size(p)
     if workspace is None:

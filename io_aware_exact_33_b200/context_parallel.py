@@ -13,31 +13,32 @@ as it passes, and the results are combined exactly:
   the online softmax applies tile by tile);
 - backward: the staged backward of the library.  ``attn_bwd_prepare`` runs
   once per query chunk on the merged O and LSE, every pair's
-  ``attn_bwd_accumulate`` adds its dQ share into that chunk's float32
+  ``attn_bwd_accumulate_f32`` adds its dQ share into that chunk's float32
   accumulator (exact across pairs: softmax probabilities are taken against
-  the global LSE), and ``attn_bwd_finalize`` writes dQ.  The dK / dV partial
-  of each pair is written in 16 bits by the kernel and summed into float32
-  buffers that travel round the ring behind their key/value block and arrive
-  at its owner after the last step.
+  the global LSE) and its dK / dV into a float32 buffer that travels round
+  the ring behind its key/value block and arrives at its owner after the
+  last step, and ``attn_bwd_finalize`` writes dQ.
 
 The pages name faster communication across devices as the way to longer
 contexts (FA2-Guide, "对未来Transformer架构的深远影响") without fixing a scheme;
-this is the plainest exact one.  With a causal mask, equal-size chunks make
-every pair either fully visible (key chunk before the query chunk), causal
-with Nq = Nk (the same chunk) or skipped (key chunk after).  The "zigzag"
-layout gives rank r of W the chunks r and 2W - 1 - r of 2W, so every rank
-does the same work at every step; "contiguous" gives rank r chunk r of W
-(balanced without a mask only).
+this is the plainest exact one.  Every pair is one kernel call over local
+indices with ``pos_offset`` = (query chunk - key chunk) x chunk length, so
+the kernels apply the whole sequence's causal mask, sliding window and
+positional slopes to the pair; pairs that no mask lets through are skipped.
+With a causal mask, equal-size chunks make every pair either fully visible
+(key chunk before the query chunk), causal with Nq = Nk (the same chunk) or
+skipped (key chunk after).  The "zigzag" layout gives rank r of W the chunks
+r and 2W - 1 - r of 2W, so every rank does the same causal work at every
+step; "contiguous" gives rank r chunk r of W (balanced without a mask only).
 
 Layouts: a rank's tensors are chunk-major, q (C, B, n, H, d), k and v
 (C, B, n, Hkv, d), lse (C, B, H, n), C = chunks per rank in ``chunk_ids``
 order, so each chunk is one contiguous (B, n, ...) tensor.  ``shard`` and
 ``unshard`` convert from and to whole-sequence tensors.
 
-Not supported here: sliding windows and per-head slopes (their offsets are
-relative to the global positions, which the per-pair calls do not carry),
-and packed variable-length batches.  Every rank must call these functions
-with the same shapes, in the same order (they are collective).
+Not supported here: packed variable-length batches and dropout.  Every
+rank must call these functions with the same shapes and arguments, in the
+same order (they are collective).
 """
 from __future__ import annotations
 
@@ -69,23 +70,41 @@ def num_chunks(world: int, layout: str = "zigzag") -> int:
 
 def pair_mask(q_chunk: int, k_chunk: int, causal: bool) -> int:
     """How query chunk ``q_chunk`` sees key chunk ``k_chunk`` (equal-size
-    chunks of one sequence): FULL, CAUSAL (same chunk, causal) or SKIP."""
+    chunks of one sequence) under a causal mask or none: FULL, CAUSAL (same
+    chunk, causal) or SKIP."""
     if not causal or k_chunk < q_chunk:
         return FULL
     return CAUSAL if k_chunk == q_chunk else SKIP
 
 
-def schedule(rank: int, world: int, layout: str, causal: bool) -> List[List[Tuple[int, int, bool]]]:
+def pair_visible(q_chunk: int, k_chunk: int, n: int, causal: bool, window_left: int = -1,
+                 window_right: int = -1) -> bool:
+    """Whether any key of chunk ``k_chunk`` is visible from any query of chunk
+    ``q_chunk`` (chunks of ``n`` positions): the distance j - i of global
+    positions spans (k_chunk - q_chunk) n +- (n - 1), and the masks allow
+    -window_left <= j - i <= min(0 if causal, window_right)."""
+    dmin = (k_chunk - q_chunk) * n - (n - 1)
+    dmax = (k_chunk - q_chunk) * n + (n - 1)
+    hi = None if window_right < 0 else window_right
+    if causal:
+        hi = 0 if hi is None else min(hi, 0)
+    lo = None if window_left < 0 else -window_left
+    return (hi is None or dmin <= hi) and (lo is None or dmax >= lo)
+
+
+def schedule(rank: int, world: int, layout: str, causal: bool, window_left: int = -1,
+             window_right: int = -1, n: int = 1) -> List[List[Tuple[int, int, int]]]:
     """Per ring step s (this rank then holds the key/value block of rank
-    (rank - s) mod world) the (local query chunk, block key chunk, causal)
-    triples to compute."""
+    (rank - s) mod world) the (local query chunk, block key chunk, global
+    query chunk - global key chunk) triples to compute: the pairs with any
+    visible element for chunks of ``n`` positions."""
     mine = chunk_ids(rank, world, layout)
     steps = []
     for s in range(world):
         theirs = chunk_ids((rank - s) % world, world, layout)
-        steps.append([(c, kc, pair_mask(gq, gk, causal) == CAUSAL)
+        steps.append([(c, kc, gq - gk)
                       for c, gq in enumerate(mine) for kc, gk in enumerate(theirs)
-                      if pair_mask(gq, gk, causal) != SKIP])
+                      if pair_visible(gq, gk, n, causal, window_left, window_right)])
     return steps
 
 
@@ -150,17 +169,19 @@ def _check_layout(q, k, v, ring, layout):
 
 
 def ring_attn_fwd(q, k, v, softmax_scale: Optional[float] = None, causal: bool = False,
-                  layout: str = "zigzag", group=None):
+                  layout: str = "zigzag", group=None, window_left: int = -1,
+                  window_right: int = -1, alibi_slopes=None):
     """Attention of this rank's query chunks over the whole sequence.
 
     q (C, B, n, H, d), k and v (C, B, n, Hkv, d): this rank's chunks, 16-bit
     contiguous CUDA tensors.  Returns (o (C, B, n, H, d), lse (C, B, H, n)
     float32), equal to the matching chunks of single-device attention over
-    the whole sequence."""
+    the whole sequence, with its causal mask, sliding window (positions
+    relative to the whole sequence) and per-head positional slopes."""
     ring = _Ring(group)
     C = _check_layout(q, k, v, ring, layout)
     _, B, n, H, _ = q.shape
-    steps = schedule(ring.rank, ring.world, layout, causal)
+    steps = schedule(ring.rank, ring.world, layout, causal, window_left, window_right, n)
     nparts = [sum(1 for st in steps for (c2, _, _) in st if c2 == c) for c in range(C)]
     o_parts = [torch.empty((m,) + tuple(q.shape[1:]), dtype=q.dtype, device=q.device) for m in nparts]
     lse_parts = [torch.empty((m, B, H, n), dtype=torch.float32, device=q.device) for m in nparts]
@@ -171,9 +192,10 @@ def ring_attn_fwd(q, k, v, softmax_scale: Optional[float] = None, causal: bool =
         if s + 1 < ring.world:
             nxt = torch.empty_like(kv)
             works = ring.exchange(kv, nxt)
-        for c, kc, cz in steps[s]:
-            _lib.attn_fwd(q[c], kv[0, kc], kv[1, kc], softmax_scale, cz,
-                          out=o_parts[c][slot[c]], lse=lse_parts[c][slot[c]])
+        for c, kc, dg in steps[s]:
+            _lib.attn_fwd(q[c], kv[0, kc], kv[1, kc], softmax_scale, causal, window_left,
+                          window_right, out=o_parts[c][slot[c]], lse=lse_parts[c][slot[c]],
+                          alibi_slopes=alibi_slopes, pos_offset=dg * n)
             slot[c] += 1
         _wait(works)
         if nxt is not None:
@@ -186,13 +208,15 @@ def ring_attn_fwd(q, k, v, softmax_scale: Optional[float] = None, causal: bool =
 
 
 def ring_attn_bwd(q, k, v, o, lse, do, softmax_scale: Optional[float] = None,
-                  causal: bool = False, layout: str = "zigzag", group=None):
+                  causal: bool = False, layout: str = "zigzag", group=None,
+                  window_left: int = -1, window_right: int = -1, alibi_slopes=None):
     """Gradients (dq, dk, dv) of sum(o * do) for ``ring_attn_fwd`` with the
     same arguments; ``o`` and ``lse`` are its results, ``do`` (C, B, n, H, d).
     Each rank gets the gradients of its own chunks."""
     ring = _Ring(group)
     C = _check_layout(q, k, v, ring, layout)
-    steps = schedule(ring.rank, ring.world, layout, causal)
+    n = q.shape[2]
+    steps = schedule(ring.rank, ring.world, layout, causal, window_left, window_right, n)
     # per query chunk: Dvec, LSE in base 2 and the float32 dQ accumulator
     ws, pq = [], []
     for c in range(C):
@@ -215,8 +239,9 @@ def ring_attn_bwd(q, k, v, o, lse, do, softmax_scale: Optional[float] = None,
             # the sums of the ranks the block visited before: added onto here
             _wait(dkv_works)
             dkv = dkv_in
-        for c, kc, cz in steps[s]:
-            p = _lib.params_for(q[c], kv[0, kc], softmax_scale, cz)
+        for c, kc, dg in steps[s]:
+            p = _lib.params_for(q[c], kv[0, kc], softmax_scale, causal, window_left, window_right,
+                                alibi_slopes, pos_offset=dg * n)
             _lib.attn_bwd_accumulate_f32(p, q[c], kv[0, kc], kv[1, kc], do[c], dkv[0, kc],
                                          dkv[1, kc], ws[c])
         if ring.world > 1:
@@ -239,10 +264,13 @@ def ring_attn_bwd(q, k, v, o, lse, do, softmax_scale: Optional[float] = None,
 
 class _RingAttn(torch.autograd.Function):
     @staticmethod
-    def forward(ctx, q, k, v, softmax_scale, causal, layout, group):
-        o, lse = ring_attn_fwd(q, k, v, softmax_scale, causal, layout, group)
+    def forward(ctx, q, k, v, softmax_scale, causal, layout, group, window_left, window_right,
+                alibi_slopes):
+        o, lse = ring_attn_fwd(q, k, v, softmax_scale, causal, layout, group, window_left,
+                               window_right, alibi_slopes)
         ctx.save_for_backward(q, k, v, o, lse)
-        ctx.args = (softmax_scale, causal, layout, group)
+        ctx.args = (softmax_scale, causal, layout, group, window_left, window_right,
+                    alibi_slopes)
         ctx.mark_non_differentiable(lse)
         return o, lse
 
@@ -250,12 +278,16 @@ class _RingAttn(torch.autograd.Function):
     def backward(ctx, do, _dlse):
         q, k, v, o, lse = ctx.saved_tensors
         dq, dk, dv = ring_attn_bwd(q, k, v, o, lse, do.contiguous(), *ctx.args)
-        return dq, dk, dv, None, None, None, None
+        return dq, dk, dv, None, None, None, None, None, None, None
 
 
 def ring_flash_attn_func(q, k, v, softmax_scale: Optional[float] = None, causal: bool = False,
-                         layout: str = "zigzag", group=None, return_lse: bool = False):
+                         layout: str = "zigzag", group=None, return_lse: bool = False,
+                         window_size=(-1, -1), alibi_slopes=None):
     """Differentiable ``ring_attn_fwd``: chunk-major local q, k, v in, the
-    local output chunks (and, with ``return_lse``, their LSE) out."""
-    o, lse = _RingAttn.apply(q, k, v, softmax_scale, bool(causal), layout, group)
+    local output chunks (and, with ``return_lse``, their LSE) out;
+    ``window_size`` = (left, right) in positions of the whole sequence."""
+    wl, wr = (int(x) for x in window_size)
+    o, lse = _RingAttn.apply(q, k, v, softmax_scale, bool(causal), layout, group, wl, wr,
+                             alibi_slopes)
     return (o, lse) if return_lse else o

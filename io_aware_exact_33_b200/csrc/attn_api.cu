@@ -246,6 +246,7 @@ attn_status launch_fwd(const attn_params* p, const void* q, const void* k, const
   fp.total_k = pk.total_k;
   fp.o = static_cast<uint16_t*>(o);
   fp.alibi = p->alibi_slopes;
+  fp.pos_offset = p->pos_offset;
   const uint32_t t = drop_threshold(p->dropout_p);
   fp.drop_seed = p->dropout_seed;
   fp.drop_offset = p->dropout_offset;
@@ -299,6 +300,7 @@ attn_status launch_fwd_e4m3(const attn_params* p, const void* q, const void* k, 
   fp.causal = p->causal;
   fp.window_left = p->window_left;
   fp.window_right = p->window_right;
+  fp.pos_offset = p->pos_offset;
   fp.scale_log2 = p->softmax_scale * q_scale * k_scale * 1.4426950408889634f;
   fp.num_qblocks = (p->seqlen_q + 2 * C::BM - 1) / (2 * C::BM);
   const int heads = p->batch * p->nheads;
@@ -421,6 +423,7 @@ BwdParams bwd_params(const attn_params* p, const float* lse, void* workspace, co
   bp.dk = bp.dv = nullptr;
   bp.acc_f32 = 0;
   bp.alibi = p->alibi_slopes;
+  bp.pos_offset = p->pos_offset;
   const uint32_t t = drop_threshold(p->dropout_p);
   bp.drop_seed = p->dropout_seed;
   bp.drop_offset = p->dropout_offset;
@@ -614,6 +617,7 @@ attn_status dispatch_bwd_main(const attn_params* p, const void* q, const void* k
 // max_seqlen rows (the kernels read each one's own length from the offsets).
 attn_params packed_view(const attn_varlen_params* v) {
   attn_params p;
+  std::memset(&p, 0, sizeof(p));  // pos_offset 0: each sequence is its own problem
   p.batch = v->batch;
   p.seqlen_q = v->max_seqlen_q;
   p.seqlen_k = v->max_seqlen_k;
@@ -690,6 +694,7 @@ attn_status attn_check_params(const attn_params* p, int pass) {
   if (!(p->dropout_p >= 0.f) || !(p->dropout_p < 1.f) || drop_threshold(p->dropout_p) > 255u)
     return ATTN_ERR_INVALID_ARG;
   if (d == 256 && drop_threshold(p->dropout_p) != 0) return ATTN_ERR_UNSUPPORTED_HEADDIM;
+  if (p->reserved0 != 0) return ATTN_ERR_INVALID_ARG;
   return ATTN_OK;
 }
 
@@ -732,7 +737,8 @@ attn_status attn_fwd_decode(const attn_params* p, const void* q, const void* k, 
   attn_status st = attn_check_params(p, 0);
   if (st != ATTN_OK) return st;
   if (p->headdim != 64 && p->headdim != 128) return ATTN_ERR_UNSUPPORTED_HEADDIM;
-  if (p->alibi_slopes || drop_threshold(p->dropout_p) != 0) return ATTN_ERR_INVALID_ARG;
+  if (p->alibi_slopes || drop_threshold(p->dropout_p) != 0 || p->pos_offset != 0)
+    return ATTN_ERR_INVALID_ARG;
   if ((long long)(p->nheads / p->nheads_kv) * p->seqlen_q > kDecodeRows) return ATTN_ERR_INVALID_ARG;
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   if (p->batch == 0 || p->seqlen_q == 0) return ATTN_OK;

@@ -138,8 +138,11 @@ struct BwdParams {
   // reduce-add) instead of storing them in the input dtype; dense only.
   int acc_f32;
   // Per-head positional slopes (nheads floats), or nullptr: scores gain
-  // -slope_h * |i + seqlen_k - seqlen_q - j| (kernel instantiated with ALIBI).
+  // -slope_h * |i + off - j| (kernel instantiated with ALIBI).
   const float* alibi;
+  // off = seqlen_k - seqlen_q + pos_offset places the query rows relative to
+  // the keys for the masks and the bias (0: bottom-right alignment).
+  int pos_offset;
   // Dropout (kernel instantiated with DROP; the contract in philox.cuh):
   // drop_kadd = dropout_kadd(t), drop_scale = 256 / (256 - t).
   unsigned long long drop_seed;
@@ -436,7 +439,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   const bool row_store = p.cu_q != nullptr && k0 + BN > p.seqlen_k;
 
   // Query rows that see any key of [k0, k1).
-  const long long off = (long long)p.seqlen_k - p.seqlen_q;
+  const long long off = (long long)p.seqlen_k - p.seqlen_q + p.pos_offset;
   const long long kInf = 1ll << 40;
   const long long rb = p.causal ? 0 : (p.window_right >= 0 ? p.window_right : kInf);
   const long long lb = p.window_left >= 0 ? p.window_left : kInf;

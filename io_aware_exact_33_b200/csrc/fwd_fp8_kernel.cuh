@@ -358,7 +358,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
     const uint32_t s_tmem = tmem + lane_base + C::TM_S + i * BN;
     const uint32_t o_tmem = tmem + lane_base + C::TM_O + i * D;
-    const long long off = (long long)p.seqlen_k - p.seqlen_q;
+    const long long off = (long long)p.seqlen_k - p.seqlen_q + p.pos_offset;
     const long long kInf = 1ll << 40;
     const long long rb = p.causal ? 0 : (p.window_right >= 0 ? p.window_right : kInf);
     const long long lb = p.window_left >= 0 ? p.window_left : kInf;

@@ -48,8 +48,11 @@ struct FwdParams {
   int total_q, total_k;
   uint16_t* o;
   // Per-head positional slopes (nheads floats), or nullptr: scores gain
-  // -slope_h * |i + seqlen_k - seqlen_q - j| (kernels instantiated with ALIBI).
+  // -slope_h * |i + off - j| (kernels instantiated with ALIBI).
   const float* alibi;
+  // off = seqlen_k - seqlen_q + pos_offset places the query rows relative to
+  // the keys for the masks and the bias (0: bottom-right alignment).
+  int pos_offset;
   // Dropout (kernels instantiated with DROP; the contract in philox.cuh):
   // drop_kadd = dropout_kadd(t), drop_scale = 256 / (256 - t).
   unsigned long long drop_seed;
@@ -79,7 +82,7 @@ struct KeyRange {
 };
 
 __device__ __forceinline__ KeyRange visible_keys(int q0, int q1, const FwdParams& p) {
-  const long long off = (long long)p.seqlen_k - p.seqlen_q;
+  const long long off = (long long)p.seqlen_k - p.seqlen_q + p.pos_offset;
   const long long kInf = 1ll << 40;
   const long long rb = p.causal ? 0 : (p.window_right >= 0 ? p.window_right : kInf);
   const long long lb = p.window_left >= 0 ? p.window_left : kInf;
@@ -256,7 +259,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const int r = (int)threadIdx.x;  // row within the tile == TMEM lane
     const int i = q0 + r;            // query position
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    const long long off = (long long)p.seqlen_k - p.seqlen_q;
+    const long long off = (long long)p.seqlen_k - p.seqlen_q + p.pos_offset;
     const long long kInf = 1ll << 40;
     const long long rb = p.causal ? 0 : (p.window_right >= 0 ? p.window_right : kInf);
     const long long lb = p.window_left >= 0 ? p.window_left : kInf;
@@ -827,7 +830,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
     const uint32_t s_tmem = tmem + lane_base + C::TM_S + i * BN;
     const uint32_t o_tmem = tmem + lane_base + C::TM_O + i * D;
-    const long long off = (long long)p.seqlen_k - p.seqlen_q;
+    const long long off = (long long)p.seqlen_k - p.seqlen_q + p.pos_offset;
     const long long kInf = 1ll << 40;
     const long long rb = p.causal ? 0 : (p.window_right >= 0 ? p.window_right : kInf);
     const long long lb = p.window_left >= 0 ? p.window_left : kInf;

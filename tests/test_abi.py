@@ -163,11 +163,11 @@ int main(void) {
   printf("%d %d %d %zu %zu %s\n", (int)attn_check_params(&p, 0), (int)attn_check_params(&p, 1),
          (int)attn_check_varlen_params(&v, 1), attn_bwd_workspace_size(&p),
          attn_bwd_varlen_workspace_size(&v), attn_version());
-  printf("%zu %zu %zu %zu %zu %zu %zu %zu\n", sizeof(attn_params),
+  printf("%zu %zu %zu %zu %zu %zu %zu %zu %zu\n", sizeof(attn_params),
          offsetof(attn_params, dropout_p), offsetof(attn_params, dropout_offset),
          offsetof(attn_params, dropout_seed), sizeof(attn_varlen_params),
          offsetof(attn_varlen_params, dropout_p), offsetof(attn_varlen_params, dropout_offset),
-         offsetof(attn_varlen_params, dropout_seed));
+         offsetof(attn_varlen_params, dropout_seed), offsetof(attn_params, pos_offset));
   return 0;
 }
 """)
@@ -179,11 +179,11 @@ int main(void) {
     out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()
     assert out[:3] == ["0", "0", "0"]
     # the Python mirrors of the parameter structs have the C layout
-    layout = [int(x) for x in out[6:14]]
+    layout = [int(x) for x in out[6:15]]
     A, V = attn.AttnParams, attn.AttnVarlenParams
     assert layout == [ctypes.sizeof(A), A.dropout_p.offset, A.dropout_offset.offset,
                       A.dropout_seed.offset, ctypes.sizeof(V), V.dropout_p.offset,
-                      V.dropout_offset.offset, V.dropout_seed.offset]
+                      V.dropout_offset.offset, V.dropout_seed.offset, A.pos_offset.offset]
     p = P(attn, batch=2, seqlen_q=100, seqlen_k=100, nheads=8, nheads_kv=2, headdim=128)
     assert int(out[3]) == attn.attn_bwd_workspace_size(p)
     assert int(out[4]) > 0 and out[5] == attn.attn_version()
@@ -245,3 +245,18 @@ def test_backward_wrappers_refuse_host_tensors(attn):
     for fn in (attn.attn_bwd, attn.attn_bwd_noalloc):
         with pytest.raises(ValueError, match="CUDA"):
             fn(q, k, k, q, lse, q, 0.125)
+
+
+def test_pos_offset_checks(attn):
+    """pos_offset is accepted by the dense calls; the reserved word must be 0;
+    the decode path refuses a nonzero offset before touching any pointer."""
+    p = P(attn, pos_offset=-300)
+    assert attn.attn_check_params(p, 0) == 0 and attn.attn_check_params(p, 1) == 0
+    p.reserved0 = 1
+    assert attn.attn_check_params(p, 0) == 1
+    call = attn._lib.attn_fwd_decode
+    vp = ctypes.c_void_p
+    call.argtypes = [ctypes.POINTER(attn.AttnParams), vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
+    call.restype = ctypes.c_int
+    q = P(attn, seqlen_q=1, pos_offset=5)
+    assert call(ctypes.byref(q), None, None, None, None, None, None, 0, None) == 1

@@ -18,30 +18,37 @@ import torch.multiprocessing as mp
 
 import oracle
 from attn_inputs import Workload, make_inputs
+from oracle_pins import mask_matrix
 from parity import check_grad, check_lse, check_o
 
 
 # ------------------------------------------------------------------ layouts and schedule
 @pytest.mark.parametrize("layout", ["contiguous", "zigzag"])
 @pytest.mark.parametrize("world", [1, 2, 3, 4, 5])
-@pytest.mark.parametrize("causal", [False, True])
-def test_schedule_covers_every_visible_pair_once(layout, world, causal):
+@pytest.mark.parametrize("causal,wl,wr", [(False, -1, -1), (True, -1, -1), (True, 7, -1),
+                                          (False, 5, 9), (False, -1, 0), (True, 0, -1)])
+def test_schedule_covers_every_visible_pair_once(layout, world, causal, wl, wr):
+    """Every (query chunk, key chunk) pair with a visible element (brute
+    force over the whole sequence's mask) is scheduled exactly once, with the
+    chunk distance that becomes its position offset."""
     from io_aware_exact_33_b200 import context_parallel as cp
+    n = 4
     nc = cp.num_chunks(world, layout)
     owned = sorted(g for r in range(world) for g in cp.chunk_ids(r, world, layout))
     assert owned == list(range(nc))
     seen = {}
     for r in range(world):
         mine = cp.chunk_ids(r, world, layout)
-        for s, step in enumerate(cp.schedule(r, world, layout, causal)):
+        for s, step in enumerate(cp.schedule(r, world, layout, causal, wl, wr, n)):
             theirs = cp.chunk_ids((r - s) % world, world, layout)
-            for c, kc, cz in step:
+            for c, kc, dg in step:
                 key = (mine[c], theirs[kc])
-                assert key not in seen
-                seen[key] = cz
-    want = {(a, b): (causal and a == b) for a in range(nc) for b in range(nc)
-            if not causal or b <= a}
-    assert seen == want
+                assert key not in seen and dg == key[0] - key[1]
+                seen[key] = dg
+    vis = mask_matrix(nc * n, nc * n, causal=causal, window_left=wl, window_right=wr)
+    want = {(a, b) for a in range(nc) for b in range(nc)
+            if vis[a * n:(a + 1) * n, b * n:(b + 1) * n].any()}
+    assert set(seen) == want
 
 
 @pytest.mark.parametrize("world", [1, 2, 3, 4, 8])
@@ -51,7 +58,7 @@ def test_zigzag_causal_steps_are_balanced(world):
     from io_aware_exact_33_b200 import context_parallel as cp
     for r in range(world):
         for step in cp.schedule(r, world, "zigzag", True):
-            assert sum(0.5 if cz else 1.0 for _, _, cz in step) == 2.0
+            assert sum(0.5 if dg == 0 else 1.0 for _, _, dg in step) == 2.0
 
 
 def test_shard_unshard_roundtrip():
@@ -72,14 +79,42 @@ def test_shard_unshard_roundtrip():
 _STATE = {}
 
 
+def _fake_scores(q, k, scale, causal, wl, wr, pos_offset):
+    """float64 scaled scores (B, H, nq, nk) of one pair with the masks of the
+    kernels' reading at off = nk - nq + pos_offset (-inf where hidden)."""
+    g = q.shape[2] // k.shape[2]
+    kd = k.double().repeat_interleave(g, dim=2)
+    scale = 1.0 / math.sqrt(q.shape[-1]) if scale is None else scale
+    s = torch.einsum("bihd,bjhd->bhij", q.double(), kd) * scale
+    n, m = s.shape[-2:]
+    dist = torch.arange(n)[:, None] + (m - n + pos_offset) - torch.arange(m)[None, :]  # i + off - j
+    vis = torch.ones(n, m, dtype=torch.bool)
+    if causal:
+        vis &= dist >= 0
+    if wl >= 0:
+        vis &= dist <= wl
+    if wr >= 0:
+        vis &= dist >= -wr
+    return s.masked_fill(~vis, -math.inf)
+
+
 def _fake_fwd(q, k, v, softmax_scale=None, causal=False, window_left=-1, window_right=-1,
-              out=None, lse=None, stream=None, alibi_slopes=None):
+              out=None, lse=None, stream=None, alibi_slopes=None, pos_offset=0):
+    """One pair's partial output and LSE over its keys (float64, explicit
+    masks), as attn_fwd computes them; a row that sees no key gets O = 0 and
+    LSE = -inf."""
     for t in (q, k, v, out, lse):
         assert t.is_contiguous()
     assert q.shape[1] == k.shape[1] and alibi_slopes is None
-    o, l = oracle.attention_fwd(q, k, v, softmax_scale, causal, window_left, window_right)
-    out.copy_(torch.from_numpy(o))
-    lse.copy_(torch.from_numpy(l))
+    s = _fake_scores(q, k, softmax_scale, causal, window_left, window_right, pos_offset)
+    mx = s.amax(-1, keepdim=True)
+    e = torch.exp(s - mx.clamp_min(-1e300))
+    l = e.sum(-1, keepdim=True)
+    g = q.shape[2] // k.shape[2]
+    vd = v.double().repeat_interleave(g, dim=2)
+    o = torch.einsum("bhij,bjhd->bihd", e / l.clamp_min(1e-300), vd)
+    out.copy_(o)
+    lse.copy_((mx + torch.log(l))[..., 0])
     return out, lse
 
 
@@ -106,16 +141,13 @@ def _fake_accumulate_f32(p, q, k, v, dout, dk_acc, dv_acc, workspace, stream=Non
     given (global) LSE and D = rowsum(dO o O) from the given (global) O; the
     key gradients are added into the float32 sums."""
     st = _STATE[workspace.data_ptr()]
-    assert p.seqlen_q == q.shape[1] and p.seqlen_k == k.shape[1] and p.window_left == -1
+    assert p.seqlen_q == q.shape[1] and p.seqlen_k == k.shape[1]
     g = p.nheads // p.nheads_kv
     qd = q.double()
     kd = k.double().repeat_interleave(g, dim=2)
     vd = v.double().repeat_interleave(g, dim=2)
-    s = torch.einsum("bihd,bjhd->bhij", qd, kd) * p.softmax_scale
-    if p.causal:
-        n, m = s.shape[-2:]
-        vis = torch.arange(m)[None, :] <= torch.arange(n)[:, None] + (m - n)
-        s = s.masked_fill(~vis, -math.inf)
+    s = _fake_scores(q, k, p.softmax_scale, p.causal, p.window_left, p.window_right,
+                     p.pos_offset)
     prob = torch.exp(s - st["lse"][..., None])
     dvec = (st["do"] * st["o"]).sum(-1).transpose(1, 2)  # (B, H, n)
     dp = torch.einsum("bihd,bjhd->bhij", st["do"], vd)
@@ -171,11 +203,14 @@ def _ring_rank(rank, world, store_path, w, layout, queue):
     try:
         _install_fakes()
         q, k, v, do = (cp.shard(t, rank, world, layout) for t in make_inputs(w))
-        o, lse = cp.ring_attn_fwd(q, k, v, w.softmax_scale, w.causal, layout)
-        dq, dk, dv = cp.ring_attn_bwd(q, k, v, o, lse, do, w.softmax_scale, w.causal, layout)
+        win = dict(window_left=w.window_left, window_right=w.window_right)
+        o, lse = cp.ring_attn_fwd(q, k, v, w.softmax_scale, w.causal, layout, **win)
+        dq, dk, dv = cp.ring_attn_bwd(q, k, v, o, lse, do, w.softmax_scale, w.causal, layout,
+                                      **win)
         # the autograd wrapper runs the same two passes
         ql, kl, vl = (t.clone().requires_grad_(True) for t in (q, k, v))
-        out = cp.ring_flash_attn_func(ql, kl, vl, w.softmax_scale, w.causal, layout)
+        out = cp.ring_flash_attn_func(ql, kl, vl, w.softmax_scale, w.causal, layout,
+                                      window_size=(w.window_left, w.window_right))
         out.backward(do)
         # the backward fakes use torch's CPU matrix products, whose last bits
         # may depend on memory alignment: allow one bf16 rounding step
@@ -207,11 +242,12 @@ def _run_ring(world, w, layout, tmp_path):
             for r, o, lse, dq, dk, dv, same in res]
 
 
-def _compare_whole(res, w, layout, what):
+def _compare_whole(res, w, layout, what, slopes=None):
     from io_aware_exact_33_b200 import context_parallel as cp
     q, k, v, do = make_inputs(w)
-    o_ref, lse_ref = oracle.attention_fwd(q, k, v, w.softmax_scale, w.causal)
-    g_ref = oracle.attention_bwd(q, k, v, do, w.softmax_scale, w.causal)
+    args = (w.softmax_scale, w.causal, w.window_left, w.window_right)
+    o_ref, lse_ref = oracle.attention_fwd(q, k, v, *args, alibi_slopes=slopes)
+    g_ref = oracle.attention_bwd(q, k, v, do, *args, alibi_slopes=slopes)
     o = cp.unshard([r[1] for r in res], layout)
     lse = cp.unshard([r[2] for r in res], layout, dim=2)
     check_o(o, o_ref, what + " O")
@@ -221,18 +257,19 @@ def _compare_whole(res, w, layout, what):
     assert all(r[6] for r in res), f"{what}: autograd wrapper differs from the direct calls"
 
 
-@pytest.mark.parametrize("world,layout,causal", [
-    (2, "zigzag", True), (3, "zigzag", True), (2, "contiguous", True), (3, "contiguous", False),
-    (2, "zigzag", False),
+@pytest.mark.parametrize("world,layout,causal,wl,wr", [
+    (2, "zigzag", True, -1, -1), (3, "zigzag", True, -1, -1), (2, "contiguous", True, -1, -1),
+    (3, "contiguous", False, -1, -1), (2, "zigzag", False, -1, -1),
+    (3, "zigzag", True, 7, -1), (2, "contiguous", False, 5, 9),
 ])
-def test_ring_on_gloo_ranks(world, layout, causal, tmp_path):
+def test_ring_on_gloo_ranks(world, layout, causal, wl, wr, tmp_path):
     from io_aware_exact_33_b200 import context_parallel as cp
     n = 6  # rows per chunk
     N = n * cp.num_chunks(world, layout)
-    w = Workload("cp", 2, 4, 2, N, N, 8, causal, -1, -1, "bf16", 1.0, 800 + world,
+    w = Workload("cp", 2, 4, 2, N, N, 8, causal, wl, wr, "bf16", 1.0, 800 + world,
                  softmax_scale=0.4)
     res = _run_ring(world, w, layout, tmp_path)
-    _compare_whole(res, w, layout, f"ring W={world} {layout} causal={causal}")
+    _compare_whole(res, w, layout, f"ring W={world} {layout} causal={causal} window={wl},{wr}")
 
 
 def test_ring_of_one_process(fakes):
@@ -269,6 +306,30 @@ def test_ring_of_one_process_on_gpu():
     torch.cuda.synchronize()
     res = [(0, o.cpu(), lse.cpu(), dq.cpu(), dk.cpu(), dv.cpu(), True)]
     _compare_whole(res, w, "zigzag", "ring W=1 on GPU")
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("wl,wr,with_slopes", [(150, -1, False), (-1, -1, True), (90, -1, True)])
+def test_ring_window_and_slopes_on_gpu(wl, wr, with_slopes):
+    """Sliding windows and positional slopes across chunks: every pair call
+    carries pos_offset = (query chunk - key chunk) x n, and the merged result
+    equals the oracle over the whole sequence (zigzag, two chunks of 200:
+    with a window of 150 or 90 the far pair is partly or wholly hidden)."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from io_aware_exact_33_b200 import context_parallel as cp
+    w = Workload("cpw", 2, 4, 2, 400, 400, 128, True, wl, wr, "bf16", 1.0, 813)
+    slopes = (torch.tensor([2.0 ** (-2 * (h + 1)) for h in range(4)], dtype=torch.float32)
+              if with_slopes else None)
+    sl = slopes.cuda() if with_slopes else None
+    q, k, v, do = (cp.shard(t, 0, 1).cuda() for t in make_inputs(w))
+    o, lse = cp.ring_attn_fwd(q, k, v, None, True, window_left=wl, window_right=wr,
+                              alibi_slopes=sl)
+    dq, dk, dv = cp.ring_attn_bwd(q, k, v, o, lse, do, None, True, window_left=wl,
+                                  window_right=wr, alibi_slopes=sl)
+    torch.cuda.synchronize()
+    res = [(0, o.cpu(), lse.cpu(), dq.cpu(), dk.cpu(), dv.cpu(), True)]
+    _compare_whole(res, w, "zigzag", f"ring W=1 window={wl} slopes={with_slopes}", slopes)
 
 
 @pytest.mark.gpu
