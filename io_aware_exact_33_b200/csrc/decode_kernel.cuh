@@ -179,13 +179,12 @@ __global__ void __launch_bounds__(kDecodeThreads, (RMAX <= 8) ? 2 : 1)
       const uint32_t kbase = smem0 + st * C::STAGE_BYTES;
       const uint32_t vbase = kbase + C::TILE_BYTES;
       const int jt = key0 + t * kDecodeBN;  // first key of the tile
-      // scores of the warp's two groups of four keys
-      float s[2][RMAX];
+      // scores of the warp's two groups of four keys: both groups' parts of
+      // K first, so that each query load serves both
+      float kf[2][C::COLS];  // this lane's D/8 columns of its two K rows
 #pragma unroll
       for (int grp = 0; grp < 2; ++grp) {
         const int row = (int)warp * 8 + grp * 4 + kk;  // key within the tile
-        // this lane's D/8 columns of the K row, as floats
-        float kf[C::COLS];
 #pragma unroll
         for (int ch = 0; ch < C::COLS / 8; ++ch) {
           const int col = part * C::COLS + ch * 8;
@@ -194,32 +193,40 @@ __global__ void __launch_bounds__(kDecodeThreads, (RMAX <= 8) ? 2 : 1)
           asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                        : "=r"(w0), "=r"(w1), "=r"(w2), "=r"(w3)
                        : "r"(kbase + bx * C::BOX_BYTES + row * 128 + chunk * 16));
-          unpack2<FP16>(w0, kf[ch * 8 + 0], kf[ch * 8 + 1]);
-          unpack2<FP16>(w1, kf[ch * 8 + 2], kf[ch * 8 + 3]);
-          unpack2<FP16>(w2, kf[ch * 8 + 4], kf[ch * 8 + 5]);
-          unpack2<FP16>(w3, kf[ch * 8 + 6], kf[ch * 8 + 7]);
+          unpack2<FP16>(w0, kf[grp][ch * 8 + 0], kf[grp][ch * 8 + 1]);
+          unpack2<FP16>(w1, kf[grp][ch * 8 + 2], kf[grp][ch * 8 + 3]);
+          unpack2<FP16>(w2, kf[grp][ch * 8 + 4], kf[grp][ch * 8 + 5]);
+          unpack2<FP16>(w3, kf[grp][ch * 8 + 6], kf[grp][ch * 8 + 7]);
         }
+      }
+      float s[2][RMAX];
 #pragma unroll
-        for (int r = 0; r < RMAX; ++r) {
-          uint64_t s2 = f2_pack(0.f, 0.f);
-          if (r < R) {
-            const uint32_t qaddr = smem0 + C::OFF_Q + (r * D + part * C::COLS) * 4;
+      for (int r = 0; r < RMAX; ++r) {
+        uint64_t s2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+        if (r < R) {
+          const uint32_t qaddr = smem0 + C::OFF_Q + (r * D + part * C::COLS) * 4;
 #pragma unroll
-            for (int c4 = 0; c4 < C::COLS / 4; ++c4) {
-              float q4[4];
-              ld_shared_v4f(qaddr + c4 * 16, q4);
-              s2 = f2_fma(f2_pack(q4[0], q4[1]), f2_pack(kf[4 * c4], kf[4 * c4 + 1]), s2);
-              s2 = f2_fma(f2_pack(q4[2], q4[3]), f2_pack(kf[4 * c4 + 2], kf[4 * c4 + 3]), s2);
+          for (int c4 = 0; c4 < C::COLS / 4; ++c4) {
+            float q4[4];
+            ld_shared_v4f(qaddr + c4 * 16, q4);
+            const uint64_t qa = f2_pack(q4[0], q4[1]), qb = f2_pack(q4[2], q4[3]);
+#pragma unroll
+            for (int grp = 0; grp < 2; ++grp) {
+              s2[grp] = f2_fma(qa, f2_pack(kf[grp][4 * c4], kf[grp][4 * c4 + 1]), s2[grp]);
+              s2[grp] = f2_fma(qb, f2_pack(kf[grp][4 * c4 + 2], kf[grp][4 * c4 + 3]), s2[grp]);
             }
           }
+        }
+#pragma unroll
+        for (int grp = 0; grp < 2; ++grp) {
           float e, o;
-          f2_unpack(s2, e, o);
+          f2_unpack(s2[grp], e, o);
           float x = e + o;
           x += __shfl_xor_sync(0xffffffffu, x, 4);
           x += __shfl_xor_sync(0xffffffffu, x, 8);
           x += __shfl_xor_sync(0xffffffffu, x, 16);
           // mask: key j of query i is visible iff i + off - lb <= j <= i + off + rb
-          const long long j = (long long)jt + row;
+          const long long j = (long long)jt + (int)warp * 8 + grp * 4 + kk;
           const long long i = r % Nq;
           const bool vis = r < R && j < p.seqlen_k && j <= i + off + rb && j >= i + off - lb;
           s[grp][r] = vis ? x : -INFINITY;
