@@ -17,6 +17,7 @@
 #include "decode_kernel.cuh"
 #include "fwd_fp8_kernel.cuh"
 #include "fwd_kernel.cuh"
+#include "fwd_persist_kernel.cuh"
 #include "merge_kernel.cuh"
 #include "sm100.cuh"
 
@@ -274,6 +275,85 @@ attn_status launch_fwd(const attn_params* p, const void* q, const void* k, const
                                    : FwdLaunch<C>::template kernel<false, false>());
   if (!ensure_smem(reinterpret_cast<const void*>(kern), C::SMEM_BYTES)) return ATTN_ERR_CUDA;
   kern<<<(unsigned)blocks, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mo, fp);
+  return finish(stream);
+}
+
+// Mean visible key positions per query row, from the key-tile range of
+// each 128-row query tile (the longest sequence's lengths for packed calls).
+double mean_visible_keys(const attn_params* p) {
+  const long long off = (long long)p->seqlen_k - p->seqlen_q + p->pos_offset;
+  const long long kInf = 1ll << 40;
+  const long long rb = p->causal ? 0 : (p->window_right >= 0 ? p->window_right : kInf);
+  const long long lb = p->window_left >= 0 ? p->window_left : kInf;
+  double sum = 0.0;
+  long long tiles = 0;
+  for (long long q0 = 0; q0 < p->seqlen_q; q0 += 128, ++tiles) {
+    const long long q1 = std::min(q0 + 128, (long long)p->seqlen_q) - 1;
+    const long long lo = std::max(0ll, q0 + off - lb);
+    const long long hi = std::min((long long)p->seqlen_k - 1, q1 + off + rb);
+    sum += hi >= lo ? (double)(hi - lo + 1) : 0.0;
+  }
+  return tiles ? sum / tiles : 0.0;
+}
+
+// The persistent forward (fwd_persist_kernel.cuh) for dense batches of many
+// short units: at most 12 key tiles per query tile on average and at least
+// four units per SM, no positional slopes, no dropout.  (On long units the
+// one-shot grid measured faster; packed batches keep the one-shot kernel.)
+constexpr double kPersistMaxKeys = 12 * 128;
+constexpr int kPersistMinUnitsPerSm = 4;
+bool use_persistent_fwd(const attn_params* p, const Packed& pk) {
+  if ((p->headdim != 64 && p->headdim != 128) || p->alibi_slopes ||
+      drop_threshold(p->dropout_p) != 0 || pk.on())
+    return false;
+  int sms = 148, dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long units = ((long long)p->seqlen_q + 255) / 256 * p->batch * p->nheads;
+  return units >= (long long)kPersistMinUnitsPerSm * sms &&
+         mean_visible_keys(p) <= kPersistMaxKeys;
+}
+
+template <class C>
+attn_status launch_fwd_persist(const attn_params* p, const void* q, const void* k, const void* v,
+                               void* o, float* lse, cudaStream_t stream, const Packed& pk) {
+  CUtensorMap mq, mk, mv;
+  const int mb = pk.on() ? 1 : p->batch;
+  const int nq = pk.on() ? pk.total_q : p->seqlen_q, nk = pk.on() ? pk.total_k : p->seqlen_k;
+  if (!map_bshd(&mq, q, C::FP16, mb, nq, p->nheads, C::D, C::BM) ||
+      !map_bshd(&mk, k, C::FP16, mb, nk, p->nheads_kv, C::D, C::BN) ||
+      !map_bshd(&mv, v, C::FP16, mb, nk, p->nheads_kv, C::D, C::BN))
+    return ATTN_ERR_CUDA;
+  FwdParams fp;
+  std::memset(&fp, 0, sizeof(fp));
+  fp.cu_q = pk.cu_q;
+  fp.cu_k = pk.cu_k;
+  fp.total_q = pk.total_q;
+  fp.total_k = pk.total_k;
+  fp.o = static_cast<uint16_t*>(o);
+  fp.pos_offset = p->pos_offset;
+  fp.lse = lse;
+  fp.batch = p->batch;
+  fp.nheads = p->nheads;
+  fp.nheads_kv = p->nheads_kv;
+  fp.seqlen_q = p->seqlen_q;
+  fp.seqlen_k = p->seqlen_k;
+  fp.causal = p->causal;
+  fp.window_left = p->window_left;
+  fp.window_right = p->window_right;
+  fp.scale_log2 = p->softmax_scale * 1.4426950408889634f;
+  fp.num_qblocks = (p->seqlen_q + 2 * C::BM - 1) / (2 * C::BM);
+  const int heads = p->batch * p->nheads;
+  fp.sched_group = l2_group(4.0 * p->seqlen_k * C::D / (p->nheads / p->nheads_kv), heads);
+  const long long units = (long long)fp.num_qblocks * heads;
+  if (units > INT_MAX) return ATTN_ERR_INVALID_ARG;
+  int sms = 148, dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = (int)std::min<long long>(units, sms);
+  auto kern = attn_fwd_persist_kernel<C>;
+  if (!ensure_smem(reinterpret_cast<const void*>(kern), C::SMEM_BYTES)) return ATTN_ERR_CUDA;
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, fp, (int)units);
   return finish(stream);
 }
 
@@ -578,11 +658,18 @@ void* noalloc_scratch_address() {
 attn_status dispatch_fwd(const attn_params* p, const void* q, const void* k, const void* v,
                          void* o, float* lse, cudaStream_t stream, const Packed& pk) {
   const bool fp16 = p->dtype == ATTN_FP16;
+  const bool persist = use_persistent_fwd(p, pk);
   switch (p->headdim) {
     case 64:
+      if (persist)
+        return fp16 ? launch_fwd_persist<FwdPersistCfg<64, 3, 3, true>>(p, q, k, v, o, lse, stream, pk)
+                    : launch_fwd_persist<FwdPersistCfg<64, 3, 3, false>>(p, q, k, v, o, lse, stream, pk);
       return fp16 ? launch_fwd<FwdPPCfg<64, 3, 3, true>>(p, q, k, v, o, lse, stream, pk)
                   : launch_fwd<FwdPPCfg<64, 3, 3, false>>(p, q, k, v, o, lse, stream, pk);
     case 128:
+      if (persist)
+        return fp16 ? launch_fwd_persist<FwdPersistCfg<128, 3, 2, true>>(p, q, k, v, o, lse, stream, pk)
+                    : launch_fwd_persist<FwdPersistCfg<128, 3, 2, false>>(p, q, k, v, o, lse, stream, pk);
       return fp16 ? launch_fwd<FwdPPCfg<128, 3, 2, true>>(p, q, k, v, o, lse, stream, pk)
                   : launch_fwd<FwdPPCfg<128, 3, 2, false>>(p, q, k, v, o, lse, stream, pk);
     case 256:

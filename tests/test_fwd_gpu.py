@@ -81,6 +81,24 @@ def test_fwd_wide_scores(attn, w):
     check_lse(lse, lse_ref, w.name)
 
 
+# Many short work units (at least four per SM, at most 12 key tiles per
+# query tile on average, no slopes or dropout): these run the persistent
+# forward, each CTA taking a unit after another.
+PERSIST = [
+    W("persist_causal_ragged", 6, 32, 32, 1000, 1000, 128, causal=True, seed=130),
+    W("persist_window_gqa", 4, 40, 8, 2048, 2048, 128, causal=True, wl=512, seed=131),
+    W("persist_full_short", 16, 16, 16, 640, 640, 128, seed=132),
+    W("persist_d64_fp16", 8, 48, 12, 700, 700, 64, causal=True, dtype="fp16", seed=133),
+    W("persist_nq_lt_nk", 20, 32, 16, 300, 900, 128, causal=True, seed=134),
+    W("persist_window_both", 6, 32, 32, 1500, 1500, 128, wl=200, wr=100, seed=135),
+]
+
+
+@pytest.mark.parametrize("w", PERSIST, ids=lambda w: w.name)
+def test_fwd_persistent_full(attn, w):
+    full_check(attn, w)
+
+
 @pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
 def test_fwd_small_full(attn, w):
     full_check(attn, w)
