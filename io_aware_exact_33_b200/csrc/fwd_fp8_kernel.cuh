@@ -122,6 +122,8 @@ __device__ __forceinline__ void softmax_tile_e4m3(uint32_t s_tmem, uint32_t o_tm
   };
   float mx = -INFINITY;
   {
+    // four independent running maxima (no single dependent chain)
+    float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
     uint32_t buf[2][32];
     tmem_ld32(s_tmem, buf[0]);
     tmem_ld_wait();
@@ -130,9 +132,11 @@ __device__ __forceinline__ void softmax_tile_e4m3(uint32_t s_tmem, uint32_t o_tm
       if (c + 1 < BN / 32) tmem_ld32(s_tmem + (c + 1) * 32, buf[(c + 1) & 1]);
 #pragma unroll
       for (int e = 0; e < 32; e += 2)
-        mx = max3f(mx, val(buf[c & 1][e], c * 32 + e), val(buf[c & 1][e + 1], c * 32 + e + 1));
+        mq[(e / 2) & 3] = max3f(mq[(e / 2) & 3], val(buf[c & 1][e], c * 32 + e),
+                                val(buf[c & 1][e + 1], c * 32 + e + 1));
       if (c + 1 < BN / 32) tmem_ld_wait();
     }
+    mx = max3f(mq[0], mq[1], fmaxf(mq[2], mq[3]));
   }
   const float m_tile = mx * scale_log2;  // scale > 0
   m_use = m;

@@ -302,9 +302,18 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         for (int c = 0; c < BN; ++c) s[c] = fmaf(s[c], p.scale_log2, bk * fabsf(bd - (float)c));
         sl = 1.f;
       }
-      float mx = s[0];
+      // four independent running maxima (no single dependent chain)
+      float mq[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
-      for (int c = 1; c < BN; ++c) mx = fmaxf(mx, s[c]);
+      for (int c = 4; c < BN; c += 8) {
+        mq[0] = max3f(mq[0], s[c], s[c + 1]);
+        mq[1] = max3f(mq[1], s[c + 2], s[c + 3]);
+        if (c + 4 < BN) {
+          mq[2] = max3f(mq[2], s[c + 4], s[c + 5]);
+          mq[3] = max3f(mq[3], s[c + 6], s[c + 7]);
+        }
+      }
+      const float mx = max3f(mq[0], mq[1], fmaxf(mq[2], mq[3]));
       const float m_tile = mx * sl;  // scale > 0
       // Keep the old reference max unless the row max grew by more than 8
       // (log2 units); the first tile always sets it.
@@ -314,15 +323,17 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         alpha = (m == -INFINITY) ? 0.f : ex2(m - m_tile);
       }
       const float m_sub = (m_use == -INFINITY) ? 0.f : m_use;
-      float rowsum = 0.f;
+      float rs0 = 0.f, rs1 = 0.f;  // two sums: no single dependent chain
       uint32_t packed[BN / 2];
 #pragma unroll
       for (int c = 0; c < BN; c += 2) {
         const float p0 = ex2(fmaf(s[c], sl, -m_sub));
         const float p1 = ex2(fmaf(s[c + 1], sl, -m_sub));
-        rowsum += p0 + p1;
+        rs0 += p0;
+        rs1 += p1;
         packed[c / 2] = pack2<C::FP16>(p0, p1);
       }
+      const float rowsum = rs0 + rs1;
       l = l * alpha + rowsum;
       m = m_use;
       // Rescale O (after O += P_{t-1} V_{t-1} has landed) if any row of this
@@ -513,6 +524,9 @@ __device__ __forceinline__ void softmax_tile(uint32_t s_tmem, uint32_t o_tmem, i
   const bool bounded = !ALIBI || (-bk * (float)(BN - 1) <= 64.f);  // uniform: one slope per CTA
   mx = -INFINITY;
   {
+    // four independent running maxima, so the 3-input max instructions of
+    // a chunk do not form one dependent chain
+    float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
     uint32_t buf[2][32];
     tmem_ld32(s_tmem, buf[0]);
     tmem_ld_wait();
@@ -522,7 +536,8 @@ __device__ __forceinline__ void softmax_tile(uint32_t s_tmem, uint32_t o_tmem, i
       if (bounded) {
 #pragma unroll
         for (int e = 0; e < 32; e += 2)
-          mx = max3f(mx, val(buf[c & 1][e], c * 32 + e), val(buf[c & 1][e + 1], c * 32 + e + 1));
+          mq[(e / 2) & 3] = max3f(mq[(e / 2) & 3], val(buf[c & 1][e], c * 32 + e),
+                                  val(buf[c & 1][e + 1], c * 32 + e + 1));
       } else {
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
@@ -532,6 +547,7 @@ __device__ __forceinline__ void softmax_tile(uint32_t s_tmem, uint32_t o_tmem, i
       }
       if (c + 1 < BN / 32) tmem_ld_wait();
     }
+    mx = fmaxf(mx, max3f(mq[0], mq[1], fmaxf(mq[2], mq[3])));
   }
   float m_tile = bounded ? mx * scale_log2 : mx;  // scale > 0
   if (ALIBI && bounded) m_tile += bk * fmaxf(fmaxf(-bd, bd - (float)(BN - 1)), 0.f);
