@@ -183,7 +183,11 @@ ATTN_API attn_status attn_fwd_decode(const attn_params* p, const void* q, const 
  * Backward pass: given dout = dL/dO and the forward's o and lse, writes
  * dq = dL/dQ, dk = dL/dK, dv = dL/dV (dk, dv summed over the query heads of
  * each kv group).  The score tiles are recomputed from q, k and lse.
- * Supported: headdim in {64, 128}; dtype bf16 or fp16.
+ * Supported: headdim in {64, 128, 256} (256 without dropout, as the pages
+ * give FlashAttention-2's backward: "FlashAttention 四代演进", hardware /
+ * dtype limits); dtype bf16 or fp16.  With headdim 256 the accumulate stage
+ * runs three kernels, for dV, dK and dQ, each recomputing the score tiles
+ * it needs (eight tile products instead of five, to fit tensor memory).
  * workspace: at least attn_bwd_workspace_size(p) bytes, 256-byte aligned;
  * it holds float32 rowsum(dO o O), lse in base 2 and the float32 dQ
  * accumulator.  Its contents on entry do not matter.

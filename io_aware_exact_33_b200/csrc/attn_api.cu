@@ -13,6 +13,7 @@
 #include <utility>
 
 #include "attn.h"
+#include "bwd256_kernel.cuh"
 #include "bwd_kernel.cuh"
 #include "decode_kernel.cuh"
 #include "fwd_fp8_kernel.cuh"
@@ -509,14 +510,15 @@ BwdParams bwd_params(const attn_params* p, const float* lse, void* workspace, co
   bp.drop_offset = p->dropout_offset;
   bp.drop_kadd = dropout_kadd(t);
   bp.drop_scale = 256.f / (float)(256u - t);
-  bp.num_kblocks = bp.sched_group = 0;
+  bp.num_kblocks = bp.num_qblocks = bp.sched_group = 0;
   bp.lse = lse;
   bp.dvec = reinterpret_cast<float*>(w + ws.dvec_off);
   bp.lse2 = reinterpret_cast<float*>(w + ws.lse2_off);
   bp.lse_slab = reinterpret_cast<uint16_t*>(w + ws.lsb_off);
   bp.dvec_slab = reinterpret_cast<uint16_t*>(w + ws.dvb_off);
-  // bf16 without dropout: the main kernel folds the statistics into its MMAs
-  bp.fold = (p->dtype == ATTN_BF16 && t == 0) ? 1 : 0;
+  // bf16 without dropout, d <= 128: the main kernel folds the statistics
+  // into its MMAs (the d = 256 kernels read the fp32 rows)
+  bp.fold = (p->dtype == ATTN_BF16 && t == 0 && p->headdim <= 128) ? 1 : 0;
   bp.dq_acc = reinterpret_cast<float*>(w + ws.dq_off);
   bp.batch = p->batch;
   bp.nheads = p->nheads;
@@ -595,6 +597,58 @@ attn_status launch_bwd_main(const attn_params* p, const void* q, const void* k, 
   if (!ensure_smem(reinterpret_cast<const void*>(kern), C::SMEM_BYTES)) return ATTN_ERR_CUDA;
   kern<<<(unsigned)blocks, C::THREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, ml, md, mdk,
                                                                  mdv, mdq, bpl);
+  return finish(stream);
+}
+
+// d = 256: dV, then dK (key-stationary), then dQ added to the accumulator
+// (query-stationary); see bwd256_kernel.cuh.
+template <bool FP16>
+attn_status launch_bwd256(const attn_params* p, const void* q, const void* k, const void* v,
+                          const void* dout, void* dk, void* dv, void* workspace,
+                          cudaStream_t stream, const Packed& pk, bool acc_f32) {
+  using KvV = Bwd256KvCfg<FP16, false>;
+  using KvK = Bwd256KvCfg<FP16, true>;
+  using QC = Bwd256QCfg<FP16>;
+  BwdParams bp = bwd_params(p, nullptr, workspace, pk);
+  const int mb = pk.on() ? 1 : p->batch;
+  const int nq = pk.on() ? pk.total_q : p->seqlen_q, nk = pk.on() ? pk.total_k : p->seqlen_k;
+  CUtensorMap mq64, mdo64, mk128, mv128, mq128, mdo128, mk64, mv64;
+  if (!map_bshd(&mq64, q, FP16, mb, nq, p->nheads, 256, KvV::BM) ||
+      !map_bshd(&mdo64, dout, FP16, mb, nq, p->nheads, 256, KvV::BM) ||
+      !map_bshd(&mk128, k, FP16, mb, nk, p->nheads_kv, 256, KvV::BN) ||
+      !map_bshd(&mv128, v, FP16, mb, nk, p->nheads_kv, 256, KvV::BN) ||
+      !map_bshd(&mq128, q, FP16, mb, nq, p->nheads, 256, QC::BM) ||
+      !map_bshd(&mdo128, dout, FP16, mb, nq, p->nheads, 256, QC::BM) ||
+      !map_bshd(&mk64, k, FP16, mb, nk, p->nheads_kv, 256, QC::BN) ||
+      !map_bshd(&mv64, v, FP16, mb, nk, p->nheads_kv, 256, QC::BN))
+    return ATTN_ERR_CUDA;
+  bp.acc_f32 = acc_f32 ? 1 : 0;
+  const int kv_heads = p->batch * p->nheads_kv, q_heads = p->batch * p->nheads;
+  const int group = p->nheads / p->nheads_kv;
+  bp.num_kblocks = (p->seqlen_k + KvV::BN - 1) / KvV::BN;
+  bp.num_qblocks = (p->seqlen_q + QC::BM - 1) / QC::BM;
+  const long long kv_blocks = (long long)bp.num_kblocks * kv_heads;
+  const long long q_blocks = (long long)bp.num_qblocks * q_heads;
+  if (kv_blocks > INT_MAX || q_blocks > INT_MAX) return ATTN_ERR_INVALID_ARG;
+  const bool alibi = p->alibi_slopes != nullptr;
+  // key-stationary: Q and dO of a kv head's query heads are shared by its
+  // key tiles; query-stationary: K and V of a kv head by its query tiles
+  BwdParams bkv = bp;
+  bkv.sched_group = l2_group(4.0 * p->seqlen_q * 256 * group, kv_heads);
+  BwdParams bq = bp;
+  bq.sched_group = l2_group(4.0 * p->seqlen_k * 256 / group, q_heads);
+  auto kv_v = alibi ? attn_bwd256_kv_kernel<KvV, true> : attn_bwd256_kv_kernel<KvV, false>;
+  auto kv_k = alibi ? attn_bwd256_kv_kernel<KvK, true> : attn_bwd256_kv_kernel<KvK, false>;
+  auto qk = alibi ? attn_bwd256_q_kernel<QC, true> : attn_bwd256_q_kernel<QC, false>;
+  if (!ensure_smem(reinterpret_cast<const void*>(kv_v), KvV::SMEM_BYTES) ||
+      !ensure_smem(reinterpret_cast<const void*>(kv_k), KvK::SMEM_BYTES) ||
+      !ensure_smem(reinterpret_cast<const void*>(qk), QC::SMEM_BYTES))
+    return ATTN_ERR_CUDA;
+  kv_v<<<(unsigned)kv_blocks, KvV::THREADS, KvV::SMEM_BYTES, stream>>>(mq64, mk128, mv128, mdo64,
+                                                                      bkv, dv);
+  kv_k<<<(unsigned)kv_blocks, KvK::THREADS, KvK::SMEM_BYTES, stream>>>(mq64, mk128, mv128, mdo64,
+                                                                      bkv, dk);
+  qk<<<(unsigned)q_blocks, QC::THREADS, QC::SMEM_BYTES, stream>>>(mq128, mk64, mv64, mdo128, bq);
   return finish(stream);
 }
 
@@ -695,6 +749,9 @@ attn_status dispatch_bwd_main(const attn_params* p, const void* q, const void* k
                                                        pk, acc_f32)
                   : launch_bwd_main<BwdCfg<128, false>>(p, q, k, v, dout, dk, dv, workspace, stream,
                                                         pk, acc_f32);
+    case 256:
+      return fp16 ? launch_bwd256<true>(p, q, k, v, dout, dk, dv, workspace, stream, pk, acc_f32)
+                  : launch_bwd256<false>(p, q, k, v, dout, dk, dv, workspace, stream, pk, acc_f32);
     default:
       return ATTN_ERR_UNSUPPORTED_HEADDIM;
   }
@@ -772,8 +829,7 @@ attn_status attn_check_params(const attn_params* p, int pass) {
   if (p->nheads > 65535 || p->batch > 65535) return ATTN_ERR_INVALID_ARG;
   if (p->dtype != ATTN_BF16 && p->dtype != ATTN_FP16) return ATTN_ERR_UNSUPPORTED_DTYPE;
   const int d = p->headdim;
-  if (pass == 0 && d != 64 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED_HEADDIM;
-  if (pass == 1 && d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED_HEADDIM;
+  if (d != 64 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED_HEADDIM;
   if (!(p->softmax_scale > 0.f) || !std::isfinite(p->softmax_scale)) return ATTN_ERR_INVALID_ARG;
   if (p->causal != 0 && p->causal != 1) return ATTN_ERR_INVALID_ARG;
   if (p->window_left < -1 || p->window_right < -1) return ATTN_ERR_INVALID_ARG;

@@ -122,6 +122,7 @@ struct BwdParams {
   float softmax_scale;
   long long nq_pad;
   int num_kblocks;   // key tiles per (batch, kv head): the work units
+  int num_qblocks;   // 128-row query tiles per (batch, head): the units of the d = 256 dQ kernel
   int sched_group;   // kv heads per scheduling group (grouped_lpt)
   // Packed variable-length sequences when cu_q != nullptr (see seq_span and
   // packed_row0): seqlen_q / seqlen_k then hold the longest sequence,

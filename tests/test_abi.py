@@ -81,8 +81,11 @@ def test_check_params_rejects(attn, kw, code):
     assert attn.attn_check_params(P(attn, **kw), 0) == code
 
 
-def test_bwd_headdim_256_unsupported(attn):
-    assert attn.attn_check_params(P(attn, headdim=256), 1) == 2
+def test_bwd_headdim_256_checks(attn):
+    """The backward takes head dim 256 without dropout only."""
+    assert attn.attn_check_params(P(attn, headdim=256), 1) == 0
+    assert attn.attn_check_params(P(attn, headdim=256, dropout_p=0.1), 1) == 2
+    assert attn.attn_check_params(P(attn, headdim=96), 1) == 2
 
 
 def test_causal_flag_must_be_boolean(attn):

@@ -1,6 +1,6 @@
 """Per-head positional slopes (alibi_slopes) on the GPU against the float64
-oracle with the same slopes: forward and backward for head dims 64 and 128
-(forward also 256), every mask kind, GQA, Nq != Nk, fp16, packed sequences,
+oracle with the same slopes: forward and backward for head dims 64, 128 and
+256, every mask kind, GQA, Nq != Nk, fp16, packed sequences,
 and zero slopes against no slopes."""
 import numpy as np
 import pytest
@@ -39,8 +39,9 @@ CASES = [
     (W("d128_nq_gt_nk", 1, 2, 1, 260, 130, 128, seed=506), True),
     (W("d64_fp16", 1, 4, 4, 256, 256, 64, dtype="fp16", seed=507), True),
     (W("d64_causal", 2, 2, 2, 260, 260, 64, causal=True, seed=508), True),
-    (W("d256_causal_fwd", 1, 2, 2, 300, 300, 256, causal=True, dtype="fp16", seed=509), False),
-    (W("d256_fwd", 1, 2, 1, 200, 330, 256, seed=510), False),
+    (W("d256_causal", 1, 2, 2, 300, 300, 256, causal=True, dtype="fp16", seed=509), True),
+    (W("d256", 1, 2, 1, 200, 330, 256, seed=510), True),
+    (W("d256_window", 1, 4, 2, 450, 450, 256, causal=True, wl=129, seed=512), True),
 ]
 
 

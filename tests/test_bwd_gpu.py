@@ -51,6 +51,15 @@ SMALL = [
     W("nq_gt_nk_causal_empty_rows", 1, 2, 2, 300, 130, 128, causal=True, seed=211),
     W("nq_gt_nk_d64", 1, 2, 1, 257, 65, 64, seed=212),
     W("single_row", 1, 1, 1, 1, 1, 128, seed=213),
+    # head dim 256: three kernels (dV, dK key-stationary; dQ query-stationary)
+    W("d256_n128", 1, 2, 2, 128, 128, 256, seed=220),
+    W("d256_ragged_gqa_causal", 2, 4, 2, 333, 333, 256, causal=True, seed=221),
+    W("d256_fp16_nq_lt_nk", 1, 2, 1, 200, 330, 256, dtype="fp16", seed=222),
+    W("d256_window", 1, 4, 4, 600, 600, 256, causal=True, wl=129, seed=223),
+    W("d256_window_both_sides", 1, 2, 2, 500, 500, 256, wl=100, wr=60, seed=224),
+    W("d256_nq_gt_nk_empty_rows", 1, 2, 2, 300, 130, 256, causal=True, seed=225),
+    W("d256_gqa8_causal", 1, 8, 1, 257, 257, 256, causal=True, seed=226),
+    W("d256_single_row", 1, 1, 1, 1, 1, 256, seed=227),
 ]
 
 
@@ -121,12 +130,32 @@ def test_bwd_empty_sides(attn):
     assert (dq == 0).all() and dk.numel() == 0
 
 
-def test_bwd_rejects_headdim_256(attn):
+def test_bwd_headdim_256_rejects_dropout(attn):
     q = torch.randn(1, 16, 2, 256, dtype=torch.bfloat16, device="cuda")
     o, lse = attn.attn_fwd(q, q.clone(), q.clone())
     with pytest.raises(attn.AttnError) as e:
-        attn.attn_bwd(q, q, q, o, lse, q)
+        attn.attn_bwd(q, q, q, o, lse, q, dropout_p=0.1, dropout_seed=1)
     assert e.value.status == 2
+
+
+def test_bwd_d256_accumulates(attn):
+    """attn_bwd_accumulate adds its dQ share to the accumulator (twice gives
+    twice the gradient), as for the other head dims."""
+    w = W("d256_acc", 1, 2, 2, 200, 200, 256, causal=True, seed=228)
+    q, k, v, do = (t.cuda() for t in make_inputs(w))
+    o, lse = attn.attn_fwd(q, k, v, w.scale, True)
+    p = attn.params_for(q, k, w.scale, True)
+    ws = torch.empty(attn.attn_bwd_workspace_size(p), dtype=torch.uint8, device="cuda")
+    dq1, dq2 = torch.empty_like(q), torch.empty_like(q)
+    dk, dv = torch.empty_like(k), torch.empty_like(v)
+    attn.attn_bwd_prepare(p, o, lse, do, ws)
+    attn.attn_bwd_accumulate(p, q, k, v, do, dk, dv, ws)
+    attn.attn_bwd_finalize(p, dq1, ws)
+    attn.attn_bwd_accumulate(p, q, k, v, do, dk, dv, ws)
+    attn.attn_bwd_finalize(p, dq2, ws)
+    torch.cuda.synchronize()
+    assert attn.attn_get_device_status() == 0
+    assert torch.allclose(dq2.float(), 2 * dq1.float(), rtol=1e-2, atol=1e-3)
 
 
 def test_bwd_workspace_too_small(attn):

@@ -203,3 +203,17 @@ def test_long_fp16_d256_fwd_sampled(attn):
     w = WORKLOADS[name]
     (q, k, v, _), o, lse, _, args = run(attn, w, False)
     check_fwd(name, q, k, v, o, lse, args, fwd_rows(w.seqlen_q))
+
+
+def test_long_fp16_d256_bwd_sampled(attn):
+    """The backward at the long-sequence head-dim-256 shape (N = 65536, fp16,
+    causal, the same input distribution) with one head: the oracle needs
+    every query row's statistics for the key gradients, so its cost grows
+    with N^2 d per head.  Query rows at every 64- and 128-row tile edge (the
+    two kernel tilings of the queries), key rows at every 128-key tile edge."""
+    w = WORKLOADS["long_fp16_b1_h8_n65536_d256"].replace(
+        name="long_fp16_b1_h1_n65536_d256", nheads=1, nheads_kv=1, passes="fwd+bwd")
+    (q, k, v, do), o, lse, grads, args = run(attn, w, True)
+    _identities(w, do, grads[1], grads[2])
+    check_bwd(w.name, q, k, v, do, grads, args, bwd_rows(w.seqlen_q, 64, 1024, 31),
+              bwd_rows(w.seqlen_k, 128, 256, 32))

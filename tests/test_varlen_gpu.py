@@ -45,9 +45,11 @@ CASES = [
     ("d64_causal", [260, 129], [260, 129], 2, 2, 64, "bf16", dict(causal=True), True),
     ("d128_fp16_causal", [384, 17, 255], [384, 17, 255], 2, 2, 128, "fp16", dict(causal=True),
      True),
-    ("d256_fp16_causal_fwd", [300, 129, 64], [300, 129, 64], 2, 2, 256, "fp16",
-     dict(causal=True), False),
-    ("d256_bf16_fwd", [65, 250], [200, 250], 2, 1, 256, "bf16", dict(causal=False), False),
+    ("d256_fp16_causal", [300, 129, 64], [300, 129, 64], 2, 2, 256, "fp16",
+     dict(causal=True), True),
+    ("d256_bf16", [65, 250], [200, 250], 2, 1, 256, "bf16", dict(causal=False), True),
+    ("d256_window_gqa", [400, 0, 190], [400, 0, 190], 4, 2, 256, "bf16",
+     dict(causal=True, window_left=100, window_right=0), True),
     ("many_causal", _lens(12, 1, 2000, 5), None, 8, 8, 128, "bf16", dict(causal=True), True),
 ]
 
