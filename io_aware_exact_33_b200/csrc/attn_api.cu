@@ -145,8 +145,12 @@ bool ensure_smem(const void* kernel, int bytes) {
 }
 
 // Heads per scheduling group (grouped_lpt): as many as keep the tiles they
-// share within this share of the 126 MB L2.
-constexpr double kL2GroupBudget = 64.0 * 1024 * 1024;
+// share within this share of the 126 MB L2.  16 MB leaves room for what
+// streams past them (Q, O, the dQ accumulator): on the causal N=8192
+// workload it brought the forward's DRAM reads from 593 MB to 403 MB (Q, K,
+// V read once) and the backward's traffic from 1.43 to 1.33 GB, with both
+// kernels as fast or faster than at 32 or 64 MB.
+constexpr double kL2GroupBudget = 16.0 * 1024 * 1024;
 int l2_group(double bytes_per_head, int heads) {
   double g = bytes_per_head > 0 ? kL2GroupBudget / bytes_per_head : heads;
   if (g < 1) g = 1;
