@@ -43,9 +43,12 @@ UNIT = "TFLOP/s"
 WORKLOAD = "causal_b2_h32_n8192_d128"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 NOMINAL_BF16_TFLOPS = 2250.0
+# The sources that decide the main kernels' DRAM traffic: the kernels and
+# the host code that picks their launch order (scheduling groups).
 KERNEL_SOURCES = ["io_aware_exact_33_b200/csrc/fwd_kernel.cuh",
                   "io_aware_exact_33_b200/csrc/bwd_kernel.cuh",
-                  "io_aware_exact_33_b200/csrc/sm100.cuh"]
+                  "io_aware_exact_33_b200/csrc/sm100.cuh",
+                  "io_aware_exact_33_b200/csrc/attn_api.cu"]
 
 
 # ---------------------------------------------------------------- accounting
