@@ -295,11 +295,12 @@ def test_ring_rejects_bad_layouts(fakes):
 
 # ------------------------------------------------------------------ GPU
 @pytest.mark.gpu
-def test_ring_of_one_process_on_gpu():
+@pytest.mark.parametrize("d", [128, 256])
+def test_ring_of_one_process_on_gpu(d):
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     from io_aware_exact_33_b200 import context_parallel as cp
-    w = Workload("cpg", 2, 4, 2, 400, 400, 128, True, -1, -1, "bf16", 1.0, 811)
+    w = Workload("cpg", 2, 4, 2, 400, 400, d, True, -1, -1, "bf16", 1.0, 811)
     q, k, v, do = (cp.shard(t, 0, 1).cuda() for t in make_inputs(w))
     o, lse = cp.ring_attn_fwd(q, k, v, None, True)
     dq, dk, dv = cp.ring_attn_bwd(q, k, v, o, lse, do, None, True)
@@ -333,15 +334,17 @@ def test_ring_window_and_slopes_on_gpu(wl, wr, with_slopes):
 
 
 @pytest.mark.gpu
-def test_accumulate_f32_adds_key_gradients():
+@pytest.mark.parametrize("d", [128, 256])
+def test_accumulate_f32_adds_key_gradients(d):
     """attn_bwd_accumulate_f32 adds dK (x scale) and dV in float32 into the
     caller's sums: two calls on zeroed sums give twice the oracle's key
     gradients, and twice the dQ share in the workspace accumulator; the
-    float32-to-16-bit conversion rounds like torch."""
+    float32-to-16-bit conversion rounds like torch.  Head dim 256 runs the
+    three-kernel backward."""
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     import io_aware_exact_33_b200 as attn
-    w = Workload("accf32", 2, 4, 2, 300, 260, 128, True, 64, -1, "bf16", 1.0, 812)
+    w = Workload("accf32", 2, 4, 2, 300, 260, d, True, 64, -1, "bf16", 1.0, 812)
     q, k, v, do = make_inputs(w)
     qc, kc, vc, doc = q.cuda(), k.cuda(), v.cuda(), do.cuda()
     args = (w.softmax_scale, w.causal, w.window_left, w.window_right)

@@ -117,12 +117,13 @@ def test_dropout_seed_shared_by_both_passes(fake_lib):
 
 
 @pytest.mark.gpu
-def test_functional_on_gpu():
+@pytest.mark.parametrize("d", [128, 256])
+def test_functional_on_gpu(d):
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     from io_aware_exact_33_b200.functional import flash_attn_func
     from parity import check_grad, check_o
-    w = Workload("fg", 2, 4, 2, 300, 300, 128, True, -1, -1, "bf16", 1.0, 702)
+    w = Workload("fg", 2, 4, 2, 300, 300, d, True, -1, -1, "bf16", 1.0, 702)
     q0, k0, v0, do0 = make_inputs(w)
     q, k, v = (t.cuda().requires_grad_(True) for t in (q0, k0, v0))
     out = flash_attn_func(q, k, v, causal=True)

@@ -51,6 +51,7 @@ def _ptr(t):
 CASES = [
     Workload("noalloc_d128_causal_gqa", 1, 4, 2, 300, 300, 128, True, seed=300),
     Workload("noalloc_d64_window", 2, 2, 2, 200, 260, 64, False, 40, 17, seed=301),
+    Workload("noalloc_d256_causal", 1, 2, 1, 200, 200, 256, True, seed=302),
 ]
 
 
