@@ -335,6 +335,8 @@ def run_reference(args):
     import oracle
     from attn_inputs import WORKLOADS
     w = WORKLOADS[args.workload]
+    if getattr(args, "passes", None):
+        w = w.replace(passes=args.passes)
     oracle.build()
     threads = oracle.num_threads()
     heads = max(1, min(w.nheads, threads))
@@ -396,6 +398,8 @@ def run_gpu(args):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     w = WORKLOADS[args.workload]
+    if getattr(args, "passes", None):
+        w = w.replace(passes=args.passes)
     f_fwd, f_bwd = step_flops(w)
     bwd = has_bwd(w)
 
@@ -426,7 +430,8 @@ def run_gpu(args):
         attn.attn_bwd_finalize(p, dq, ws)
         if ev: ev[4].record(stream)
 
-    launches_per_step = 4 if bwd else 1
+    # forward; prepare, main (three kernels at head dim 256: dV, dK, dQ), convert
+    launches_per_step = (1 + (5 if w.headdim == 256 else 3)) if bwd else 1
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
@@ -517,7 +522,9 @@ def run_gpu(args):
     mean = lambda xs: sum(xs) / len(xs)
     kernels = {"attn_fwd_kernel": {"ms": mean(t_fwd), "flops": f_fwd}}
     if bwd:
-        kernels["attn_bwd_kernel"] = {"ms": mean(t_main), "flops": f_bwd}
+        # head dim 256: the accumulate stage's three kernels together
+        kernels["attn_bwd_kernel" if w.headdim <= 128 else "attn_bwd256 (3 kernels)"] = {
+            "ms": mean(t_main), "flops": f_bwd}
     dominant = max(kernels, key=lambda n: kernels[n]["ms"])
     rl = {}
     for name, kk in kernels.items():
@@ -872,6 +879,9 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--workload", default=WORKLOAD,
                     help=f"attn_inputs workload to time (default {WORKLOAD}, the headline)")
+    ap.add_argument("--passes", choices=["fwd", "fwd+bwd"], default=None,
+                    help="time these passes instead of the workload's own (for example the "
+                         "backward of a forward-only workload)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:
