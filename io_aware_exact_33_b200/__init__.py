@@ -498,14 +498,15 @@ def attn_bwd_finalize(p: AttnParams, dq, workspace, stream=None) -> None:
 def attn_bwd_noalloc(q, k, v, out, lse, dout, softmax_scale: Optional[float] = None,
                      causal: bool = False, window_left: int = -1, window_right: int = -1,
                      dq=None, dk=None, dv=None, stream=None, alibi_slopes=None,
-                     dropout_p: float = 0.0, dropout_seed: int = 0, dropout_offset: int = 0):
+                     dropout_p: float = 0.0, dropout_seed: int = 0, dropout_offset: int = 0,
+                     pos_offset: int = 0):
     """Like ``attn_bwd`` but the library uses its own fixed device scratch
     (ATTN_NOALLOC_SCRATCH_BYTES) instead of a caller workspace, for callers
     that cannot allocate device memory at call time.  The output tensors are
     the caller's (allocated here only when not given).  Calls that overlap on
     the GPU share that scratch and must be serialised by the caller."""
     p = params_for(q, k, softmax_scale, causal, window_left, window_right, alibi_slopes,
-                   dropout_p, dropout_seed, dropout_offset)
+                   dropout_p, dropout_seed, dropout_offset, pos_offset)
     dq, dk, dv = _bwd_tensors(q, k, v, out, lse, dout, dq, dk, dv)
     st = _lib.attn_bwd_noalloc(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
                                _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _stream(stream))
