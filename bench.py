@@ -337,6 +337,8 @@ def run_reference(args):
     w = WORKLOADS[args.workload]
     if getattr(args, "passes", None):
         w = w.replace(passes=args.passes)
+    if getattr(args, "seqlen", None):
+        w = w.replace(seqlen_q=args.seqlen, seqlen_k=args.seqlen)
     oracle.build()
     threads = oracle.num_threads()
     heads = max(1, min(w.nheads, threads))
@@ -400,6 +402,8 @@ def run_gpu(args):
     w = WORKLOADS[args.workload]
     if getattr(args, "passes", None):
         w = w.replace(passes=args.passes)
+    if getattr(args, "seqlen", None):
+        w = w.replace(seqlen_q=args.seqlen, seqlen_k=args.seqlen)
     f_fwd, f_bwd = step_flops(w)
     bwd = has_bwd(w)
 
@@ -882,6 +886,9 @@ def main(argv=None):
     ap.add_argument("--passes", choices=["fwd", "fwd+bwd"], default=None,
                     help="time these passes instead of the workload's own (for example the "
                          "backward of a forward-only workload)")
+    ap.add_argument("--seqlen", type=int, default=None,
+                    help="query and key length instead of the workload's (a smaller case of "
+                         "the same kernels, for profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:
@@ -902,7 +909,10 @@ def main(argv=None):
     if args.workload not in WORKLOADS:
         ap.error(f"unknown workload {args.workload}; choose from "
                  f"{sorted(WORKLOADS) + sorted(VARLEN_WORKLOADS) + sorted(EXTRA_WORKLOADS)}")
-    if input_bytes(WORKLOADS[args.workload]) < 2 * 126e6:
+    wk = WORKLOADS[args.workload]
+    if args.seqlen:
+        wk = wk.replace(seqlen_q=args.seqlen, seqlen_k=args.seqlen)
+    if input_bytes(wk) < 2 * 126e6:
         ap.error(f"{args.workload} fits in L2; it is a parity case, not a bench workload")
     if args.impl == "reference":
         return run_reference(args)
