@@ -61,7 +61,8 @@ struct Bwd256KvCfg {
   static constexpr int B_DPFULL = B_SFULL + NBUF;        // per buffer (dK)
   static constexpr int B_XREADY = B_DPFULL + NBUF;       // P^T / dS^T in TMEM: 256 arrivals
   static constexpr int B_DONE = B_XREADY + NBUF;
-  static constexpr int NBAR = B_DONE + 1;
+  static constexpr int B_FLUSH = B_DONE + 1;  // every MMA of the CTA complete
+  static constexpr int NBAR = B_FLUSH + 1;
   static constexpr int OFF_TMEMPTR = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_TMEMPTR + 16 + 1024;
   // tensor memory: the accumulator (dV or dK), then per buffer an S^T block
@@ -232,6 +233,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                                    : smem0 + C::OFF_DO + (t % DS) * C::Q_BYTES;
         const uint64_t b_mn = sdesc_sw128(b_base, BM * 128, 1024);
         if (!mbar_wait_warp(bar(C::B_XREADY + bf), use & 1)) return false;
+        // dV: nothing else waits for the dO slot (the compute warps do not
+        // read it); dK: issue_s(t) waited for the Q slot
+        if (!DK && !mbar_wait_warp(bar(C::B_DOFULL + t % DS), (t / DS) & 1)) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk) {
@@ -390,6 +394,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   tc_fence_before();
   __syncthreads();
   if (warp == 9) {
+    // every MMA this warp issued has completed (also on a path that gave
+    // up early) before the tensor memory is released
+    if (nt > 0) {
+      mma_commit_warp(bar(C::B_FLUSH));
+      mbar_wait_warp(bar(C::B_FLUSH), 0);
+    }
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
@@ -424,7 +434,8 @@ struct Bwd256QCfg {
   static constexpr int B_DPFULL = B_SFULL + NBUF;      // per buffer
   static constexpr int B_DSREADY = B_DPFULL + NBUF;    // dS in TMEM: 256 arrivals
   static constexpr int B_DONE = B_DSREADY + NBUF;
-  static constexpr int NBAR = B_DONE + 1;
+  static constexpr int B_FLUSH = B_DONE + 1;  // every MMA of the CTA complete
+  static constexpr int NBAR = B_FLUSH + 1;
   static constexpr int OFF_TMEMPTR = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_TMEMPTR + 16 + 1024;
   // tensor memory: per buffer an S block and a dP block of BN fp32 columns,
@@ -701,6 +712,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   tc_fence_before();
   __syncthreads();
   if (warp == 9) {
+    // every MMA this warp issued has completed (also on a path that gave
+    // up early) before the tensor memory is released
+    if (nt > 0) {
+      mma_commit_warp(bar(C::B_FLUSH));
+      mbar_wait_warp(bar(C::B_FLUSH), 0);
+    }
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
