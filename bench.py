@@ -142,15 +142,17 @@ def kernel_source_hash():
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel):
-    """DRAM bytes per launch of `kernel` from the committed ncu summary, or
-    None if absent or taken on different kernel sources."""
+def recorded_traffic(kernel, workload):
+    """DRAM bytes per launch of `kernel` on `workload` from the committed ncu
+    summary, or None if absent, taken on another workload or on different
+    kernel sources."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             d = json.load(f)
         ent = d.get(kernel)
-        if not ent or ent.get("source_hash") != kernel_source_hash():
+        if not ent or ent.get("source_hash") != kernel_source_hash() or \
+                ent.get("workload") != workload:
             return None
         return float(ent["bytes_per_launch"])
     except (OSError, ValueError, KeyError):
@@ -530,10 +532,12 @@ def run_gpu(args):
         kernels["attn_bwd_kernel" if w.headdim <= 128 else "attn_bwd256 (3 kernels)"] = {
             "ms": mean(t_main), "flops": f_bwd}
     dominant = max(kernels, key=lambda n: kernels[n]["ms"])
+    # DRAM traffic is recorded per (kernel, workload at its own size)
+    cfg_workload = None if getattr(args, "seqlen", None) else w.name
     rl = {}
     for name, kk in kernels.items():
         achieved = kk["flops"] / (kk["ms"] / 1e3) / 1e12
-        traffic = recorded_traffic(name)
+        traffic = recorded_traffic(name, cfg_workload)
         rl[name] = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
                     "unit": UNIT, "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
                     "peak_source": f"bf16_tflops (burst) of {peak_kind}",
