@@ -301,15 +301,18 @@ double mean_visible_keys(const attn_params* p) {
   return tiles ? sum / tiles : 0.0;
 }
 
-// The persistent forward (fwd_persist_kernel.cuh) for dense batches of many
-// short units: at most 12 key tiles per query tile on average and at least
-// four units per SM, no positional slopes, no dropout.  (On long units the
-// one-shot grid measured faster; packed batches keep the one-shot kernel.)
+// The persistent forward (fwd_persist_kernel.cuh) for batches of many short
+// units, dense or packed: at most 12 key tiles per query tile on average and
+// at least four units per SM (packed batches: judged by their longest
+// sequence), no positional slopes, no dropout.  On long units the one-shot
+// grid measured faster; on the packed mix of 16 causal sequences of
+// 256-1792 tokens the persistent kernel measured 0.296 ms against 0.300.
 constexpr double kPersistMaxKeys = 12 * 128;
 constexpr int kPersistMinUnitsPerSm = 4;
 bool use_persistent_fwd(const attn_params* p, const Packed& pk) {
+  (void)pk;
   if ((p->headdim != 64 && p->headdim != 128) || p->alibi_slopes ||
-      drop_threshold(p->dropout_p) != 0 || pk.on())
+      drop_threshold(p->dropout_p) != 0)
     return false;
   int sms = 148, dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess)
