@@ -739,8 +739,8 @@ attn_status dispatch_fwd(const attn_params* p, const void* q, const void* k, con
       return fp16 ? launch_fwd<FwdPPCfg<128, 3, 2, true>>(p, q, k, v, o, lse, stream, pk)
                   : launch_fwd<FwdPPCfg<128, 3, 2, false>>(p, q, k, v, o, lse, stream, pk);
     case 256:
-      return fp16 ? launch_fwd<FwdCfg<256, 64, 2, true>>(p, q, k, v, o, lse, stream, pk)
-                  : launch_fwd<FwdCfg<256, 64, 2, false>>(p, q, k, v, o, lse, stream, pk);
+      return fp16 ? launch_fwd<FwdCfg<256, 64, 3, 2, true>>(p, q, k, v, o, lse, stream, pk)
+                  : launch_fwd<FwdCfg<256, 64, 3, 2, false>>(p, q, k, v, o, lse, stream, pk);
     default:
       return ATTN_ERR_UNSUPPORTED_HEADDIM;
   }

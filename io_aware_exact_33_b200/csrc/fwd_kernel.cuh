@@ -7,8 +7,11 @@
 // transformer optimization", items 1-2; FlashAttention-2 page, "Tile-level
 // parallelism" and "shared memory"); the mapping onto B200 is this file's:
 //
-//   warp 4      TMA producer: Q once, then K_j and V_j into a STAGES-deep
-//               ring of shared-memory slots, each guarded by mbarriers.
+//   warp 4      TMA producer: Q once, then K_j and V_j into rings of
+//               shared-memory slots of their own (KSTAGES and VSTAGES
+//               deep), each guarded by mbarriers; a K slot is free once S_j
+//               has read it, a V slot once O += P_j V_j has, so the next K
+//               tiles load while the softmax of this one runs.
 //   warp 5      allocates tensor memory; lane 0 issues every tcgen05.mma:
 //               S_j = Q K_j^T into one of two TMEM score buffers, and
 //               O += P_j V_j with P_j read straight from TMEM.
@@ -93,9 +96,9 @@ __device__ __forceinline__ KeyRange visible_keys(int q0, int q1, const FwdParams
   return {jmin, jmax};
 }
 
-template <int D_, int BN_, int STAGES_, bool FP16_>
+template <int D_, int BN_, int KSTAGES_, int VSTAGES_, bool FP16_>
 struct FwdCfg {
-  static constexpr int D = D_, BN = BN_, STAGES = STAGES_;
+  static constexpr int D = D_, BN = BN_, KSTAGES = KSTAGES_, VSTAGES = VSTAGES_;
   static constexpr bool FP16 = FP16_;
   static constexpr int BM = 128;
   static constexpr int NBOX = D / 64;              // 64-column (128-byte) boxes per row
@@ -103,14 +106,15 @@ struct FwdCfg {
   static constexpr int KV_BYTES = BN * D * 2;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
-  static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
-  static constexpr int OFF_BAR = OFF_V + STAGES * KV_BYTES;
+  static constexpr int OFF_V = OFF_K + KSTAGES * KV_BYTES;
+  static constexpr int OFF_BAR = OFF_V + VSTAGES * KV_BYTES;
   // barriers
   static constexpr int B_Q = 0;
   static constexpr int B_KFULL = 1;
-  static constexpr int B_VFULL = B_KFULL + STAGES;
-  static constexpr int B_EMPTY = B_VFULL + STAGES;
-  static constexpr int B_SFULL = B_EMPTY + STAGES;  // 2
+  static constexpr int B_VFULL = B_KFULL + KSTAGES;
+  static constexpr int B_KEMPTY = B_VFULL + VSTAGES;
+  static constexpr int B_VEMPTY = B_KEMPTY + KSTAGES;
+  static constexpr int B_SFULL = B_VEMPTY + VSTAGES;  // 2
   static constexpr int B_PREADY = B_SFULL + 2;      // 2
   static constexpr int B_OREADY = B_PREADY + 2;     // 1
   static constexpr int NBAR = B_OREADY + 1;
@@ -130,7 +134,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                     const FwdParams pin) {
-  constexpr int D = C::D, BN = C::BN, BM = C::BM, STAGES = C::STAGES;
+  constexpr int D = C::D, BN = C::BN, BM = C::BM, KS = C::KSTAGES, VS = C::VSTAGES;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t smem0 = (smem_addr(smem_raw) + 1023u) & ~1023u;
   uint8_t* smem_gen = smem_raw + (smem0 - smem_addr(smem_raw));
@@ -185,26 +189,39 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       for (int bx = 0; bx < C::NBOX; ++bx)
         tma_load_4d(smem0 + C::OFF_Q + bx * (BM * 128), &tm_q, bar(C::B_Q), bx * 64, h,
                     sq.q_row0 + q0, sq.tma_b);
-      for (int t = 0; t < nt; ++t) {
-        const int st = t % STAGES, n = t / STAGES;
-        if (n > 0 && !mbar_wait(bar(C::B_EMPTY + st), (n - 1) & 1)) break;
-        const int k0 = (t_lo + t) * BN;
+      auto load_k = [&](int t) -> bool {
+        const int st = t % KS, n = t / KS;
+        if (n > 0 && !mbar_wait(bar(C::B_KEMPTY + st), (n - 1) & 1)) return false;
         mbar_arrive_expect_tx(bar(C::B_KFULL + st), C::KV_BYTES);
         for (int bx = 0; bx < C::NBOX; ++bx)
           tma_load_4d(smem0 + C::OFF_K + st * C::KV_BYTES + bx * (BN * 128), &tm_k,
-                      bar(C::B_KFULL + st), bx * 64, kvh, sq.k_row0 + k0, sq.tma_b);
+                      bar(C::B_KFULL + st), bx * 64, kvh, sq.k_row0 + (t_lo + t) * BN,
+                      sq.tma_b);
+        return true;
+      };
+      auto load_v = [&](int t) -> bool {
+        const int st = t % VS, n = t / VS;
+        if (n > 0 && !mbar_wait(bar(C::B_VEMPTY + st), (n - 1) & 1)) return false;
         mbar_arrive_expect_tx(bar(C::B_VFULL + st), C::KV_BYTES);
         for (int bx = 0; bx < C::NBOX; ++bx)
           tma_load_4d(smem0 + C::OFF_V + st * C::KV_BYTES + bx * (BN * 128), &tm_v,
-                      bar(C::B_VFULL + st), bx * 64, kvh, sq.k_row0 + k0, sq.tma_b);
+                      bar(C::B_VFULL + st), bx * 64, kvh, sq.k_row0 + (t_lo + t) * BN,
+                      sq.tma_b);
+        return true;
+      };
+      // K runs one tile ahead of V: a V slot still in use (until O += P V
+      // of two tiles back) never holds back the next K load.
+      bool ok = load_k(0);
+      for (int t = 0; ok && t < nt; ++t) {
+        if (t + 1 < nt) ok = load_k(t + 1);
+        ok = ok && load_v(t);
       }
       // Loads still in flight must land before the CTA can exit: wait (bounded)
       // for the last fill of every slot used.
-      for (int t = nt - STAGES < 0 ? 0 : nt - STAGES; t < nt; ++t) {
-        const int st = t % STAGES, n = t / STAGES;
-        if (!mbar_wait(bar(C::B_KFULL + st), n & 1)) break;
-        if (!mbar_wait(bar(C::B_VFULL + st), n & 1)) break;
-      }
+      for (int t = nt - KS < 0 ? 0 : nt - KS; t < nt; ++t)
+        if (!mbar_wait(bar(C::B_KFULL + t % KS), (t / KS) & 1)) break;
+      for (int t = nt - VS < 0 ? 0 : nt - VS; t < nt; ++t)
+        if (!mbar_wait(bar(C::B_VFULL + t % VS), (t / VS) & 1)) break;
       mbar_wait(bar(C::B_Q), 0);
     }
   } else if (warp == 5) {
@@ -215,9 +232,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       constexpr uint32_t idesc_pv = idesc_f16(BM, D, C::FP16, false, true);
       bool ok = mbar_wait_warp(bar(C::B_Q), 0);
       auto issue_pv = [&](int u) -> bool {
-        const int st = u % STAGES, buf = u & 1;
+        const int st = u % VS, buf = u & 1;
         if (!mbar_wait_warp(bar(C::B_PREADY + buf), (u >> 1) & 1)) return false;
-        if (!mbar_wait_warp(bar(C::B_VFULL + st), (u / STAGES) & 1)) return false;
+        if (!mbar_wait_warp(bar(C::B_VFULL + st), (u / VS) & 1)) return false;
         tc_fence_after();
         const uint32_t v_base = smem0 + C::OFF_V + st * C::KV_BYTES;
         const uint32_t p_tmem = tmem + (buf ? C::TM_S1 : C::TM_S0);
@@ -230,12 +247,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           mma_ts_warp(tmem + C::TM_O, p_tmem + kk * 8, bdesc, idesc_pv, (u > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit_warp(bar(C::B_OREADY));
-        mma_commit_warp(bar(C::B_EMPTY + st));
+        mma_commit_warp(bar(C::B_VEMPTY + st));
         return true;
       };
       for (int t = 0; ok && t < nt; ++t) {
-        const int st = t % STAGES, buf = t & 1;
-        if (!mbar_wait_warp(bar(C::B_KFULL + st), (t / STAGES) & 1)) { ok = false; break; }
+        const int st = t % KS, buf = t & 1;
+        if (!mbar_wait_warp(bar(C::B_KFULL + st), (t / KS) & 1)) { ok = false; break; }
         tc_fence_after();
         const uint32_t s_tmem = tmem + (buf ? C::TM_S1 : C::TM_S0);
         const uint64_t q_desc = sdesc_sw128(smem0 + C::OFF_Q, 16, 1024);
@@ -250,6 +267,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           mma_ss_warp(s_tmem, adesc, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
         }
         mma_commit_warp(bar(C::B_SFULL + buf));
+        mma_commit_warp(bar(C::B_KEMPTY + st));
         if (t >= 1 && !issue_pv(t - 1)) { ok = false; break; }
       }
       if (ok) issue_pv(nt - 1);
