@@ -194,3 +194,32 @@ def test_extra_workloads(capsys):
         assert bench.main(["--impl", "reference", "--workload", name]) == 0
         line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
         assert line["impl"] == "reference" and "unavailable" in line
+
+
+def test_traffic_record_is_per_workload_and_sources(tmp_path, monkeypatch):
+    """The committed DRAM-traffic record applies only to the workload it was
+    captured on, at its own size, and only while the kernel sources hash the
+    same; any other case reports null."""
+    rec = {"attn_fwd_kernel": {"bytes_per_launch": 123.0, "source_hash": bench.kernel_source_hash(),
+                               "workload": "causal_b2_h32_n8192_d128"}}
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda: rec["attn_fwd_kernel"]["source_hash"])
+    assert bench.recorded_traffic("attn_fwd_kernel", "causal_b2_h32_n8192_d128") == 123.0
+    assert bench.recorded_traffic("attn_fwd_kernel", "long_fp16_b1_h8_n65536_d256") is None
+    assert bench.recorded_traffic("attn_fwd_kernel", None) is None  # --seqlen override
+    assert bench.recorded_traffic("attn_bwd_kernel", "causal_b2_h32_n8192_d128") is None
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda: "0" * 16)
+    assert bench.recorded_traffic("attn_fwd_kernel", "causal_b2_h32_n8192_d128") is None
+
+
+def test_passes_and_seqlen_overrides_refuse_l2_sized_cases(capsys):
+    """--seqlen shrinks a workload for profiling; a case whose inputs fit in
+    twice the L2 is refused (it would time L2, not HBM)."""
+    with pytest.raises(SystemExit):
+        bench.main(["--workload", "long_fp16_b1_h8_n65536_d256", "--passes", "fwd+bwd",
+                    "--seqlen", "16384"])
+    assert "fits in L2" in capsys.readouterr().err
+    with pytest.raises(SystemExit):
+        bench.main(["--passes", "bwd-only"])
